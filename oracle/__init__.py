@@ -1,0 +1,38 @@
+"""Float64 CPU oracle for exact attention (test infrastructure only).
+
+This package is the checker, not the product. Only ``tests/``,
+``__graft_entry__.smoke()`` and the ``cpu_baseline`` / ``--impl reference``
+legs of ``bench.py`` may import it. It shares no code with the CUDA path in
+``exact_attention_102_b200/`` and imports nothing from it; inputs reach it as
+plain numpy arrays.
+
+Modules
+-------
+attention
+    The plain definitions: 3-pass safe-softmax attention forward with the
+    per-row logsumexp, its analytic gradients, the paged-KV decode (gather
+    through the block table, then the forward definition), the logsumexp
+    merge of split partials, and the FP8 e4m3 block quantiser used by the
+    diagnostic FP8 oracle.
+online
+    A second, independent implementation of the forward: the tiled one-pass
+    online-softmax recurrence (running max m, running sum l, unnormalised O
+    rescaled by exp(m_old - m_new), one final diag(l)^-1). It exists only to
+    pin ``attention.attention_fwd``.
+
+Every function is pinned by ``tests/test_oracle_*.py`` against closed forms,
+invariants, finite differences, a library routine (torch's e4m3 cast) or the
+independent recurrence; see each docstring for its pin.
+"""
+
+from .attention import (  # noqa: F401
+    attention_fwd,
+    attention_bwd,
+    attention_rows,
+    paged_decode,
+    combine_partials,
+    quantize_e4m3,
+    dequantize_blocks_e4m3,
+    fp8_block_quantize,
+)
+from .online import tiled_online_fwd  # noqa: F401

@@ -1,0 +1,362 @@
+"""Pins for the float64 oracle (CPU only).
+
+Each test ties an oracle function to something other than itself: a
+hand-derived golden value, a closed form, an invariant of the definition,
+an independent implementation (the tiled online recurrence), a library
+routine (torch's float64 attention and autograd, torch's e4m3 cast) or
+central finite differences. Chosen so that a dropped scale, a wrong sign or
+index, a transposed operand, an off-by-one causal mask or a wrong log base
+fails at least one of them.
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+
+def _num(x):
+    """Golden JSON numbers: plain floats or closed-form strings."""
+    if isinstance(x, str):
+        table = {"ln3": math.log(3.0), "ln4": math.log(4.0), "ln8": math.log(8.0),
+                 "1/3": 1.0 / 3.0, "1.5ln3": 1.5 * math.log(3.0)}
+        return table[x]
+    if isinstance(x, list):
+        return [_num(y) for y in x]
+    return float(x)
+
+
+def _load(golden_dir, name):
+    with open(os.path.join(golden_dir, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- golden ---
+
+@pytest.mark.parametrize("name", ["fwd_two_keys.json", "fwd_causal_three.json"])
+def test_fwd_golden(golden_dir, name):
+    g = _load(golden_dir, name)
+    q, k, v = (np.array(_num(g[x])) for x in ("q", "k", "v"))
+    o, lse = oracle.attention_fwd(q, k, v, causal=g["causal"])
+    np.testing.assert_allclose(o, np.array(_num(g["O"])), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, np.array(_num(g["L"])), rtol=0, atol=1e-12)
+
+
+def test_bwd_golden(golden_dir):
+    g = _load(golden_dir, "bwd_two_keys.json")
+    q, k, v, do = (np.array(_num(g[x])) for x in ("q", "k", "v", "dO"))
+    dq, dk, dv, _ = oracle.attention_bwd(q, k, v, do, causal=g["causal"])
+    np.testing.assert_allclose(dq, np.array(_num(g["dQ"])), atol=1e-12)
+    np.testing.assert_allclose(dk, np.array(_num(g["dK"])), atol=1e-12)
+    np.testing.assert_allclose(dv, np.array(_num(g["dV"])), atol=1e-12)
+
+
+def test_decode_golden(golden_dir):
+    g = _load(golden_dir, "decode_table.json")
+    o, lse = oracle.paged_decode(np.array(g["q"]), np.array(g["k_cache"]),
+                                 np.array(g["v_cache"]), np.array(g["block_table"]),
+                                 np.array(g["context_lens"]), block_size=g["block_size"])
+    np.testing.assert_allclose(o, np.array(_num(g["O"])), atol=1e-12)
+    np.testing.assert_allclose(lse, np.array(_num(g["L"])), atol=1e-12)
+
+
+def test_e4m3_golden(golden_dir):
+    g = _load(golden_dir, "e4m3_rounding.json")
+    got = oracle.quantize_e4m3(np.array(g["x"]))
+    np.testing.assert_array_equal(got, np.array(g["e4m3"]))
+
+
+# ------------------------------------------------------------ invariants ---
+
+def _rand(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_rows_of_p_sum_to_one(causal):
+    q, k, v = _rand((3, 37, 16), 1)
+    rows = np.arange(37)
+    _, _, p = oracle.attention_rows(q, rows, k, v, causal)
+    np.testing.assert_allclose(p.sum(axis=1), 1.0, atol=1e-12)
+    if causal:  # nothing above the diagonal
+        assert np.all(p[np.triu_indices(37, 1)] == 0.0)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_constant_v_gives_constant(causal):
+    q, k, _ = _rand((3, 2, 2, 29, 8), 2)
+    c = np.linspace(-3, 3, 8)
+    v = np.broadcast_to(c, (2, 2, 29, 8))
+    o, _ = oracle.attention_fwd(q, k, v, causal=causal)
+    np.testing.assert_allclose(o, np.broadcast_to(c, o.shape), atol=1e-12)
+
+
+def test_key_permutation_invariance():
+    q, k, v = _rand((3, 1, 3, 41, 16), 3)
+    perm = np.random.default_rng(9).permutation(41)
+    o1, l1 = oracle.attention_fwd(q, k, v)
+    o2, l2 = oracle.attention_fwd(q, k[..., perm, :], v[..., perm, :])
+    np.testing.assert_allclose(o1, o2, atol=1e-12)
+    np.testing.assert_allclose(l1, l2, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_uniform_logits(causal):
+    """K = 0: every visible key weighs the same, L_i = log(#visible keys)."""
+    n, d = 23, 8
+    q, v = _rand((2, n, d), 4)
+    k = np.zeros((n, d))
+    o, lse = oracle.attention_fwd(q, k, v, causal=causal)
+    for i in range(n):
+        cnt = i + 1 if causal else n
+        np.testing.assert_allclose(lse[i], math.log(cnt), atol=1e-12)
+        np.testing.assert_allclose(o[i], v[:cnt].mean(axis=0), atol=1e-12)
+
+
+def test_scale_is_one_over_sqrt_d():
+    """Doubling every key equals using scale 2/sqrt(d) (pins where the scale goes)."""
+    q, k, v = _rand((3, 17, 32), 5)
+    o1, l1 = oracle.attention_fwd(q, 2 * k, v)
+    o2, l2 = oracle.attention_fwd(q, k, v, scale=2 / math.sqrt(32))
+    np.testing.assert_allclose(o1, o2, atol=1e-12)
+    np.testing.assert_allclose(l1, l2, atol=1e-12)
+
+
+def test_rotation_invariance():
+    """(QR)(KR)^T = QK^T for orthogonal R: incoherent processing leaves O, L."""
+    q, k, v = _rand((3, 2, 33, 16), 6)
+    r = synth.orthogonal_matrix(16, 2003)
+    np.testing.assert_allclose(r @ r.T, np.eye(16), atol=1e-12)
+    o1, l1 = oracle.attention_fwd(q, k, v)
+    o2, l2 = oracle.attention_fwd(q @ r, k @ r, v)
+    np.testing.assert_allclose(o1, o2, atol=1e-12)
+    np.testing.assert_allclose(l1, l2, atol=1e-12)
+
+
+def test_causal_first_row_and_last_row():
+    """Row 0 sees key 0 only; the last row equals the unmasked result."""
+    q, k, v = _rand((3, 19, 8), 7)
+    oc, lc = oracle.attention_fwd(q, k, v, causal=True)
+    on, ln = oracle.attention_fwd(q, k, v, causal=False)
+    np.testing.assert_allclose(oc[0], v[0], atol=1e-12)
+    np.testing.assert_allclose(lc[0], (q[0] @ k[0]) / math.sqrt(8), atol=1e-12)
+    np.testing.assert_allclose(oc[-1], on[-1], atol=1e-12)
+    np.testing.assert_allclose(lc[-1], ln[-1], atol=1e-12)
+    assert not np.allclose(oc[1:-1], on[1:-1])
+
+
+# ---------------------------------------- independent implementations ---
+
+def test_tiled_recurrence_matches_page_example():
+    """The pages' own tiling demo: N=16, d=8, Br=4, Bc=d, uniform [0,1) inputs
+    from seed 456, no scale. The tiled recurrence equals the direct softmax."""
+    torch.manual_seed(456)
+    n, d = 16, 8
+    q = torch.rand((n, d)).double().numpy()
+    k = torch.rand((n, d)).double().numpy()
+    v = torch.rand((n, d)).double().numpy()
+    o_t, l_t = oracle.tiled_online_fwd(q, k, v, br=4, bc=d, scale=1.0)
+    o_d, l_d = oracle.attention_fwd(q, k, v, scale=1.0)
+    np.testing.assert_allclose(o_t, o_d, atol=1e-12)
+    np.testing.assert_allclose(l_t, l_d, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("br,bc", [(1, 1), (4, 8), (16, 16), (7, 13), (64, 32), (200, 200)])
+def test_tiled_recurrence_matches_definition(causal, br, bc):
+    q, k, v = _rand((3, 131, 16), 11)
+    q = q * 3.0  # wide score range so the running max moves a lot
+    o_t, l_t = oracle.tiled_online_fwd(q, k, v, br=br, bc=bc, causal=causal)
+    o_d, l_d = oracle.attention_fwd(q, k, v, causal=causal)
+    np.testing.assert_allclose(o_t, o_d, atol=1e-12)
+    np.testing.assert_allclose(l_t, l_d, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fwd_matches_torch_float64(causal):
+    """Library routine: torch's scaled_dot_product_attention in float64."""
+    q, k, v = _rand((3, 2, 3, 57, 32), 12)
+    o, lse = oracle.attention_fwd(q, k, v, causal=causal)
+    tq, tk, tv = (torch.from_numpy(x) for x in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=causal)
+    np.testing.assert_allclose(o, ref.numpy(), atol=1e-12)
+    s = (tq @ tk.transpose(-1, -2)) / math.sqrt(32)
+    if causal:
+        s = s.masked_fill(torch.triu(torch.ones(57, 57, dtype=torch.bool), 1), -math.inf)
+    np.testing.assert_allclose(lse, torch.logsumexp(s, dim=-1).numpy(), atol=1e-12)
+
+
+# ---------------------------------------------------------------- backward ---
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_finite_differences(causal):
+    """Central differences of f = sum(O * G), float64, h = 1e-6."""
+    n, d = 6, 4
+    q, k, v, g = _rand((4, n, d), 13)
+
+    def f(q_, k_, v_):
+        o, _ = oracle.attention_fwd(q_, k_, v_, causal=causal)
+        return float((o * g).sum())
+
+    dq, dk, dv, _ = oracle.attention_bwd(q, k, v, g, causal=causal)
+    h = 1e-6
+    for x, grad, which in ((q, dq, 0), (k, dk, 1), (v, dv, 2)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(*x.shape):
+            xp = x.copy(); xp[idx] += h
+            xm = x.copy(); xm[idx] -= h
+            args_p = [q, k, v]; args_p[which] = xp
+            args_m = [q, k, v]; args_m[which] = xm
+            num[idx] = (f(*args_p) - f(*args_m)) / (2 * h)
+        np.testing.assert_allclose(grad, num, rtol=1e-6, atol=1e-8)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_matches_torch_autograd(causal):
+    """Library routine: torch autograd through float64 attention."""
+    q, k, v, g = _rand((4, 2, 2, 45, 16), 14)
+    dq, dk, dv, dd = oracle.attention_bwd(q, k, v, g, causal=causal)
+    tq, tk, tv = (torch.from_numpy(x).requires_grad_(True) for x in (q, k, v))
+    o = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=causal)
+    o.backward(torch.from_numpy(g))
+    np.testing.assert_allclose(dq, tq.grad.numpy(), atol=1e-11)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), atol=1e-11)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), atol=1e-11)
+    # D_i = sum_c dO_ic O_ic equals sum_j P_ij dP_ij
+    np.testing.assert_allclose(dd, (g * o.detach().numpy()).sum(-1), atol=1e-11)
+
+
+def test_bwd_d_identity():
+    q, k, v, g = _rand((4, 29, 8), 15)
+    o, _ = oracle.attention_fwd(q, k, v, causal=True)
+    _, _, p = oracle.attention_rows(q, np.arange(29), k, v, True)
+    dp = g @ v.T
+    _, _, _, dd = oracle.attention_bwd(q, k, v, g, causal=True)
+    np.testing.assert_allclose(dd, (p * dp).sum(axis=1), atol=1e-12)
+
+
+def test_bwd_row_chunking_is_exact(monkeypatch):
+    """Row chunks accumulate dK/dV across chunks: small chunk == one chunk."""
+    q, k, v, g = _rand((4, 1, 2, 70, 8), 16)
+    ref = oracle.attention_bwd(q, k, v, g, causal=True)
+    import oracle.attention as oa
+    monkeypatch.setattr(oa, "ROW_CHUNK", 16)
+    got = oracle.attention_bwd(q, k, v, g, causal=True)
+    for a, b in zip(ref, got):
+        np.testing.assert_allclose(a, b, atol=1e-12)
+
+
+# ----------------------------------------------------- combine / decode ---
+
+@pytest.mark.parametrize("cuts", [[0, 100], [0, 1, 100], [0, 30, 31, 77, 100], list(range(0, 101, 10))])
+def test_split_combine_equals_unsplit(cuts):
+    q, k, v = _rand((3, 4, 100, 16), 17)
+    o_ref, l_ref = oracle.attention_fwd(q[:, :1], k, v)
+    parts_o, parts_l = [], []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        o, l = oracle.attention_fwd(q[:, :1], k[:, a:b], v[:, a:b])
+        parts_o.append(o)
+        parts_l.append(l)
+    o, l = oracle.combine_partials(np.stack(parts_o), np.stack(parts_l))
+    np.testing.assert_allclose(o, o_ref, atol=1e-12)
+    np.testing.assert_allclose(l, l_ref, atol=1e-12)
+
+
+def test_combine_ignores_empty_part():
+    q, k, v = _rand((3, 2, 50, 8), 18)
+    o_ref, l_ref = oracle.attention_fwd(q[:, :1], k, v)
+    o, l = oracle.combine_partials(np.stack([o_ref, np.zeros_like(o_ref)]),
+                                   np.stack([l_ref, np.full_like(l_ref, -np.inf)]))
+    np.testing.assert_allclose(o, o_ref, atol=1e-12)
+    np.testing.assert_allclose(l, l_ref, atol=1e-12)
+
+
+def test_decode_equals_forward_on_gathered_sequence():
+    """Reduces to the forward definition: a contiguous identity table."""
+    hq, hkv, d, bs = 8, 2, 16, 4
+    rng = np.random.default_rng(19)
+    lens = np.array([1, 4, 5, 37])
+    nblk = (lens + bs - 1) // bs
+    table = np.zeros((4, nblk.max()), dtype=np.int64)
+    start = 0
+    for s in range(4):
+        table[s, :nblk[s]] = np.arange(start, start + nblk[s])
+        start += nblk[s]
+    kc = rng.standard_normal((start, hkv, bs, d))
+    vc = rng.standard_normal((start, hkv, bs, d))
+    q = rng.standard_normal((4, hq, d))
+    o, lse = oracle.paged_decode(q, kc, vc, table, lens, block_size=bs)
+    for s in range(4):
+        blocks = table[s, :nblk[s]]
+        for h in range(hq):
+            kv = h // (hq // hkv)
+            ks = kc[blocks, kv].reshape(-1, d)[:lens[s]]
+            vs = vc[blocks, kv].reshape(-1, d)[:lens[s]]
+            o_ref, l_ref = oracle.attention_fwd(q[s, h][None], ks, vs)
+            np.testing.assert_allclose(o[s, h], o_ref[0], atol=1e-12)
+            np.testing.assert_allclose(lse[s, h], l_ref[0], atol=1e-12)
+
+
+def test_decode_shared_blocks_equal_private_copies():
+    """Mapping siblings to one physical block gives the same values as copies."""
+    lay = synth.paged_decode_layout(8, 16, 40, 200, seed=5, group=4, share_frac=0.5)
+    assert lay["shared_blocks"] > 0
+    rng = np.random.default_rng(21)
+    P = lay["num_phys"]
+    kc = rng.standard_normal((P, 2, 16, 8))
+    vc = rng.standard_normal((P, 2, 16, 8))
+    q = rng.standard_normal((8, 4, 8))
+    o1, l1 = oracle.paged_decode(q, kc, vc, lay["block_table"], lay["context_lens"])
+    # private copies: give every logical block its own physical block
+    lens = lay["context_lens"]
+    nblk = (lens + 15) // 16
+    tab2 = np.zeros_like(lay["block_table"])
+    kc2, vc2 = [], []
+    for s in range(8):
+        for b in range(nblk[s]):
+            p = lay["block_table"][s, b]
+            tab2[s, b] = len(kc2)
+            kc2.append(kc[p].copy())
+            vc2.append(vc[p].copy())
+    o2, l2 = oracle.paged_decode(q, np.stack(kc2), np.stack(vc2), tab2, lens)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+
+
+# ------------------------------------------------------------------ e4m3 ---
+
+def test_e4m3_matches_torch_cast():
+    """Library routine: torch.float8_e4m3fn (RNE) on in-range values."""
+    rng = np.random.default_rng(22)
+    x = np.concatenate([rng.standard_normal(20000) * s for s in (1e-3, 0.05, 1, 30, 120)])
+    x = x[np.abs(x) <= 448]
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(oracle.quantize_e4m3(x), ref)
+    # every representable value maps to itself
+    allv = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    allv = allv[np.isfinite(allv)]
+    np.testing.assert_array_equal(oracle.quantize_e4m3(allv), allv)
+
+
+def test_fp8_block_quantize_roundtrip():
+    x = _rand((2, 3, 130, 16), 23)[0]
+    vals, sc = oracle.fp8_block_quantize(x)
+    assert sc.shape == (3, 3)
+    # per-block max maps to exactly 448
+    for h in range(3):
+        for b in range(3):
+            blk = vals[h, b * 64:(b + 1) * 64]
+            assert np.abs(blk).max() == 448.0
+    back = oracle.dequantize_blocks_e4m3(vals, sc)
+    # relative error of e4m3 is at most 2^-4 for normal numbers
+    big = np.abs(x) > np.repeat(sc, 64, axis=-1)[..., :130, None] * 2 ** -6
+    assert np.all(np.abs(back - x)[big] <= np.abs(x)[big] * 2 ** -4 + 1e-15)
+    z = np.zeros((1, 64, 4))
+    vz, sz = oracle.fp8_block_quantize(z)
+    assert sz[0, 0] == 1.0 and np.all(vz == 0)
