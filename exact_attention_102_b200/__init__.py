@@ -1,0 +1,228 @@
+"""Python binding of libfa.so, the B200 (sm_100a) exact-attention C ABI.
+
+Argument marshalling only: each function checks dtypes / shapes / devices,
+allocates outputs with torch (device memory is PyTorch's job here), and calls
+the C entry point of the same name on the current CUDA stream. Every step of
+the computation runs in the library's CUDA kernels. There is no CPU path: a
+missing or unloadable library raises.
+
+Functions (see include/fa.h for the contract of each):
+    fa_fwd, fa_bwd, fa_bwd_workspace_bytes, paged_attn_decode,
+    paged_attn_decode_workspace_bytes, fa_fp8_prepare, fa_fwd_fp8,
+    fa_last_device_error, fa_debug_wait_timeout
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfa.so")
+
+FA_OK = 0
+FA_ERR_INVALID_ARG = 1
+FA_ERR_UNSUPPORTED = 2
+FA_ERR_LAUNCH = 3
+FA_ERR_TIMEOUT = 4
+FA_ERR_WORKSPACE = 5
+
+# the symbols include/fa.h declares
+EXPORTS = (
+    "fa_status_str", "fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd",
+    "paged_attn_decode_workspace_bytes", "paged_attn_decode", "fa_fp8_prepare",
+    "fa_fwd_fp8", "fa_last_device_error", "fa_debug_wait_timeout",
+)
+
+
+class FAError(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__(f"{fn} failed: {status_str(status)} ({status})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libfa.so (built in-tree by exact_attention_102_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m exact_attention_102_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, ci, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    L.fa_status_str.restype = ctypes.c_char_p
+    L.fa_status_str.argtypes = [ci]
+    L.fa_fwd.restype = ci
+    L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, vp]
+    L.fa_bwd_workspace_bytes.restype = sz
+    L.fa_bwd_workspace_bytes.argtypes = [ci, ci, ci, ci]
+    L.fa_bwd.restype = ci
+    L.fa_bwd.argtypes = [vp] * 9 + [vp, sz, ci, ci, ci, ci, ci, vp]
+    L.paged_attn_decode_workspace_bytes.restype = sz
+    L.paged_attn_decode_workspace_bytes.argtypes = [ci, ci, ci, ci]
+    L.paged_attn_decode.restype = ci
+    L.paged_attn_decode.argtypes = [vp, vp, vp, ci, vp, ci, vp, vp, vp, ci, ci, ci, ci, ci, ci,
+                                    vp, sz, vp]
+    L.fa_fp8_prepare.restype = ci
+    L.fa_fp8_prepare.argtypes = [vp] * 10 + [ci, ci, ci, ci, vp]
+    L.fa_fwd_fp8.restype = ci
+    L.fa_fwd_fp8.argtypes = [vp] * 8 + [ci, ci, ci, ci, ci, vp]
+    L.fa_last_device_error.restype = ci
+    L.fa_last_device_error.argtypes = [vp]
+    L.fa_debug_wait_timeout.restype = ci
+    L.fa_debug_wait_timeout.argtypes = [ctypes.c_uint, vp]
+    _lib = L
+    return L
+
+
+def status_str(status: int) -> str:
+    return lib().fa_status_str(int(status)).decode()
+
+
+def _check(fn, status):
+    if status != FA_OK:
+        raise FAError(fn, status)
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _need(t, name, dtype, ndim=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims")
+
+
+def fa_fwd(q, k, v, causal=False, o=None, lse=None, stream=None):
+    """O, L = attention forward on bf16 [B, H, N, d] tensors; L is fp32 [B, H, N]."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, torch.bfloat16, 4)
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same shape [B, H, N, d]")
+    B, H, N, d = q.shape
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _need(o, "o", torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    _check("fa_fwd", lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                  B, H, N, d, int(bool(causal)), _stream(stream)))
+    return o, lse
+
+
+def fa_bwd_workspace_bytes(B, H, N, d):
+    return int(lib().fa_bwd_workspace_bytes(B, H, N, d))
+
+
+def fa_bwd(q, k, v, o, lse, do, causal=False, dq=None, dk=None, dv=None, workspace=None,
+           stream=None):
+    """dQ, dK, dV (fp32 [B, H, N, d]) of attention, recomputing P from L."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
+        _need(t, n, torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    B, H, N, d = q.shape
+    dq = torch.empty(q.shape, dtype=torch.float32, device=q.device) if dq is None else dq
+    dk = torch.empty(q.shape, dtype=torch.float32, device=q.device) if dk is None else dk
+    dv = torch.empty(q.shape, dtype=torch.float32, device=q.device) if dv is None else dv
+    for n, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _need(t, n, torch.float32, 4)
+    ws = fa_bwd_workspace_bytes(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(ws, dtype=torch.uint8, device=q.device)
+    _check("fa_bwd", lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do),
+                                  _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(),
+                                  B, H, N, d, int(bool(causal)), _stream(stream)))
+    return dq, dk, dv
+
+
+def paged_attn_decode_workspace_bytes(num_seqs, Hq, d, max_ctx):
+    return int(lib().paged_attn_decode_workspace_bytes(num_seqs, Hq, d, max_ctx))
+
+
+def paged_attn_decode(q, k_cache, v_cache, block_table, context_lens, max_ctx, o=None,
+                      lse=None, want_lse=True, workspace=None, stream=None):
+    """One-token decode over a paged cache; returns (O bf16 [S, Hq, d], L fp32 [S, Hq] or None)."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(context_lens, "context_lens", torch.int32, 1)
+    if v_cache.shape != k_cache.shape:
+        raise ValueError("k_cache and v_cache must have the same shape")
+    S, Hq, d = q.shape
+    Hkv, bs = k_cache.shape[1], k_cache.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
+    ws = paged_attn_decode_workspace_bytes(S, Hq, d, max_ctx)
+    if workspace is None:
+        workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=q.device)
+    _check("paged_attn_decode", lib().paged_attn_decode(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), k_cache.shape[0], _ptr(block_table),
+        block_table.shape[1],
+        _ptr(context_lens), _ptr(o), _ptr(lse), S, Hq, Hkv, d, bs, int(max_ctx),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+    return o, lse
+
+
+def fa_fp8_prepare(q, k, v, R, stream=None):
+    """Rotate Q, K by R and quantise Q, K, V to e4m3 with 64-row block scales."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, torch.bfloat16, 4)
+    _need(R, "R", torch.float32, 2)
+    B, H, N, d = q.shape
+    nb = (N + 63) // 64
+    q8, k8, v8 = (torch.empty(q.shape, dtype=torch.uint8, device=q.device) for _ in range(3))
+    sq, sk, sv = (torch.empty((B, H, nb), dtype=torch.float32, device=q.device) for _ in range(3))
+    _check("fa_fp8_prepare", lib().fa_fp8_prepare(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(R), _ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq), _ptr(sk),
+        _ptr(sv), B, H, N, d, _stream(stream)))
+    return q8, k8, v8, sq, sk, sv
+
+
+def fa_fwd_fp8(q8, k8, v8, sq, sk, sv, causal=False, o=None, lse=None, stream=None):
+    """Attention forward on e4m3 inputs (uint8 storage) with per-block scales."""
+    for n, t in (("q8", q8), ("k8", k8), ("v8", v8)):
+        _need(t, n, torch.uint8, 4)
+    B, H, N, d = q8.shape
+    if o is None:
+        o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q8.device)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q8.device)
+    _check("fa_fwd_fp8", lib().fa_fwd_fp8(
+        _ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq), _ptr(sk), _ptr(sv), _ptr(o), _ptr(lse),
+        B, H, N, d, int(bool(causal)), _stream(stream)))
+    return o, lse
+
+
+def fa_last_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error status."""
+    return int(lib().fa_last_device_error(_stream(stream)))
+
+
+def fa_debug_wait_timeout(timeout_us, stream=None) -> int:
+    """Launch the bounded-wait probe; returns the launch status."""
+    return int(lib().fa_debug_wait_timeout(int(timeout_us), _stream(stream)))

@@ -1,0 +1,348 @@
+// api.cu — the extern "C" boundary declared in include/fa.h: argument
+// checks, TMA tensor-map encoding, workspace carving and kernel launches.
+// No computation of the method happens here; every step runs in the kernels.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <math.h>
+#include <string.h>
+
+#include "fa.h"
+#include "kernels.h"
+#include "prim.cuh"
+
+namespace fa {
+int decode_split_blocks();
+}
+
+namespace {
+
+// Device error word: first bounded wait that gives up writes its site code.
+__device__ uint32_t g_fa_error_word;
+
+constexpr int kMaxDevices = 64;
+
+uint32_t* error_word_ptr() {
+  static uint32_t* ptrs[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (ptrs[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fa_error_word) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<uint32_t*>(p);
+  }
+  return ptrs[dev];
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 3-D view [BH][N][d] of a BHND tensor, box (box_x elements, box_y rows, 1),
+// 128-byte swizzle, zero fill outside the tensor.
+bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int elem_bytes, int d,
+              int n, int bh, uint32_t box_x, uint32_t box_y) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n),
+                        static_cast<cuuint64_t>(bh)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * elem_bytes,
+                           static_cast<cuuint64_t>(n) * d * elem_bytes};
+  cuuint32_t box[3] = {box_x, box_y, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  memset(m, 0, sizeof(*m));
+  CUresult r = fn(m, dt, 3, const_cast<void*>(ptr), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+const float kLog2e = 1.4426950408889634f;
+
+fa_status check_attn_dims(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1 || d < 1) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > (1ll << 31) - 1) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H * N > (1ll << 31) - 1) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_status_str(fa_status s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_LAUNCH: return "FA_ERR_LAUNCH";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
+  }
+  return "FA_ERR_UNKNOWN";
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int N, int d, int causal, void* stream) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return FA_ERR_INVALID_ARG;
+  fa_status st = check_attn_dims(B, H, N, d);
+  if (st != FA_OK) return st;
+  uint32_t* err = error_word_ptr();
+  if (err == nullptr) return FA_ERR_LAUNCH;
+  CUtensorMap tq, tk, tv;
+  const int bh = B * H;
+  if (!make_map(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, bh, 64, 128) ||
+      !make_map(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, bh, 64, 128) ||
+      !make_map(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, bh, 64, 128))
+    return FA_ERR_LAUNCH;
+  fa::FwdArgs a;
+  a.o = o;
+  a.lse = lse;
+  a.B = B;
+  a.H = H;
+  a.N = N;
+  a.causal = causal ? 1 : 0;
+  a.n_pairs = (N + 255) / 256;
+  a.scale_log2 = kLog2e / sqrtf(static_cast<float>(d));
+  a.err = err;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = (d == 128) ? fa::launch_fwd<128>(tq, tk, tv, a, s)
+                             : fa::launch_fwd<64>(tq, tk, tv, a, s);
+  return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1 || d < 1) return 0;
+  const size_t rows = static_cast<size_t>(B) * H * ((static_cast<size_t>(N) + 127) / 128 * 128);
+  return 2 * round256(rows * sizeof(float));
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dout, float* dq, float* dk, float* dv, void* workspace,
+                 size_t ws_bytes, int B, int H, int N, int d, int causal, void* stream) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_INVALID_ARG;
+  fa_status st = check_attn_dims(B, H, N, d);
+  if (st != FA_OK) return st;
+  if (workspace == nullptr || !aligned16(workspace) ||
+      ws_bytes < fa_bwd_workspace_bytes(B, H, N, d))
+    return FA_ERR_WORKSPACE;
+  uint32_t* err = error_word_ptr();
+  if (err == nullptr) return FA_ERR_LAUNCH;
+  const int bh = B * H;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_map(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, bh, 64, 128) ||
+      !make_map(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, bh, 64, 128) ||
+      !make_map(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, bh, 64, 128) ||
+      !make_map(&tdo, dout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, bh, 64, 128))
+    return FA_ERR_LAUNCH;
+  fa::BwdArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.dout = dout;
+  a.lse = lse;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.n_pad = (N + 127) / 128 * 128;
+  const size_t prow = static_cast<size_t>(B) * H * a.n_pad;
+  a.delta = static_cast<float*>(workspace);
+  a.lse_log2 = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                        round256(prow * sizeof(float)));
+  a.B = B;
+  a.H = H;
+  a.N = N;
+  a.causal = causal ? 1 : 0;
+  a.scale = 1.0f / sqrtf(static_cast<float>(d));
+  a.scale_log2 = a.scale * kLog2e;
+  a.err = err;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = (d == 128) ? fa::launch_bwd<128>(tq, tk, tv, tdo, a, s)
+                             : fa::launch_bwd<64>(tq, tk, tv, tdo, a, s);
+  return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+size_t paged_attn_decode_workspace_bytes(int num_seqs, int Hq, int d, int max_ctx) {
+  if (num_seqs < 1 || Hq < 1 || d < 1 || max_ctx < 1) return 0;
+  const int sb = fa::decode_split_blocks();
+  const size_t max_splits = ((static_cast<size_t>(max_ctx) + 15) / 16 + sb - 1) / sb;
+  const size_t rows = static_cast<size_t>(num_seqs) * Hq * max_splits;
+  return round256(rows * d * sizeof(float)) + round256(rows * sizeof(float));
+}
+
+fa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                            int num_phys_blocks, const int* block_table, int max_blocks_per_seq,
+                            const int* context_lens, void* o, float* lse, int num_seqs, int Hq,
+                            int Hkv, int d, int block_size, int max_ctx, void* workspace,
+                            size_t ws_bytes, void* stream) {
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || block_table == nullptr ||
+      context_lens == nullptr || !aligned16(o) || (lse != nullptr && !aligned16(lse)))
+    return FA_ERR_INVALID_ARG;
+  if (num_seqs < 1 || Hq < 1 || Hkv < 1 || d < 1 || block_size < 1 || max_ctx < 1 ||
+      max_blocks_per_seq < 1 || num_phys_blocks < 1 || Hq % Hkv != 0)
+    return FA_ERR_INVALID_ARG;
+  if (d != 128 || block_size != 16 || Hq / Hkv != 4) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(max_blocks_per_seq) * 16 < max_ctx) return FA_ERR_INVALID_ARG;
+  const size_t need = paged_attn_decode_workspace_bytes(num_seqs, Hq, d, max_ctx);
+  if (workspace == nullptr || !aligned16(workspace) || ws_bytes < need) return FA_ERR_WORKSPACE;
+  uint32_t* err = error_word_ptr();
+  if (err == nullptr) return FA_ERR_LAUNCH;
+  const int sb = fa::decode_split_blocks();
+  const int max_splits = ((max_ctx + 15) / 16 + sb - 1) / sb;
+  if (max_splits > 65535) return FA_ERR_UNSUPPORTED;
+  const size_t rows = static_cast<size_t>(num_seqs) * Hq * max_splits;
+  fa::DecodeArgs a;
+  a.q = q;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.block_table = block_table;
+  a.num_phys = num_phys_blocks;
+  a.context_lens = context_lens;
+  a.o = o;
+  a.lse = lse;
+  a.part_o = static_cast<float*>(workspace);
+  a.part_l = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                      round256(rows * d * sizeof(float)));
+  a.num_seqs = num_seqs;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.max_blocks = max_blocks_per_seq;
+  a.max_ctx = max_ctx;
+  a.max_splits = max_splits;
+  a.split_blocks = sb;
+  a.scale_log2 = kLog2e / sqrtf(static_cast<float>(d));
+  a.err = err;
+  cudaError_t e = fa::launch_decode(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+fa_status fa_fp8_prepare(const void* q, const void* k, const void* v, const float* R, void* q8,
+                         void* k8, void* v8, float* sq, float* sk, float* sv, int B, int H,
+                         int N, int d, void* stream) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(R) || !aligned16(q8) ||
+      !aligned16(k8) || !aligned16(v8) || !aligned16(sq) || !aligned16(sk) || !aligned16(sv))
+    return FA_ERR_INVALID_ARG;
+  fa_status st = check_attn_dims(B, H, N, d);
+  if (st != FA_OK) return st;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  fa::Fp8PrepArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.R = R;
+  a.q8 = static_cast<uint8_t*>(q8);
+  a.k8 = static_cast<uint8_t*>(k8);
+  a.v8 = static_cast<uint8_t*>(v8);
+  a.sq = sq;
+  a.sk = sk;
+  a.sv = sv;
+  a.B = B;
+  a.H = H;
+  a.N = N;
+  cudaError_t e = fa::launch_fp8_prepare(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* sq,
+                     const float* sk, const float* sv, void* o, float* lse, int B, int H, int N,
+                     int d, int causal, void* stream) {
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(sq) || !aligned16(sk) ||
+      !aligned16(sv) || !aligned16(o) || !aligned16(lse))
+    return FA_ERR_INVALID_ARG;
+  fa_status st = check_attn_dims(B, H, N, d);
+  if (st != FA_OK) return st;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  uint32_t* err = error_word_ptr();
+  if (err == nullptr) return FA_ERR_LAUNCH;
+  const int bh = B * H;
+  CUtensorMap tq, tk, tv;
+  // e4m3: one 128-element (128 B) row chunk per box row
+  if (!make_map(&tq, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, bh, 128, 128) ||
+      !make_map(&tk, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, bh, 128, 128) ||
+      !make_map(&tv, v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, bh, 128, 128))
+    return FA_ERR_LAUNCH;
+  fa::Fp8FwdArgs a;
+  a.sq = sq;
+  a.sk = sk;
+  a.sv = sv;
+  a.o = o;
+  a.lse = lse;
+  a.B = B;
+  a.H = H;
+  a.N = N;
+  a.causal = causal ? 1 : 0;
+  a.n_pairs = (N + 255) / 256;
+  a.scale_log2 = kLog2e / sqrtf(static_cast<float>(d));
+  a.err = err;
+  cudaError_t e = fa::launch_fwd_fp8(tq, tk, tv, a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+fa_status fa_last_device_error(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_LAUNCH;
+  uint32_t word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_fa_error_word, sizeof(word)) != cudaSuccess)
+    return FA_ERR_LAUNCH;
+  if (word == 0) return FA_OK;
+  const uint32_t zero = 0;
+  if (cudaMemcpyToSymbol(g_fa_error_word, &zero, sizeof(zero)) != cudaSuccess)
+    return FA_ERR_LAUNCH;
+  return (word & fa::kErrBadIndex) ? FA_ERR_INVALID_ARG : FA_ERR_TIMEOUT;
+}
+
+fa_status fa_debug_wait_timeout(unsigned int timeout_us, void* stream) {
+  if (timeout_us < 1 || timeout_us > 1000000u) return FA_ERR_INVALID_ARG;
+  uint32_t* err = error_word_ptr();
+  if (err == nullptr) return FA_ERR_LAUNCH;
+  cudaError_t e = fa::launch_wait_probe(err, static_cast<uint64_t>(timeout_us) * 1000ull,
+                                        static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+}  // extern "C"
+
+namespace fa {
+
+namespace {
+// One thread waits on a barrier that nothing arrives at; the bounded wait
+// gives up after `limit_ns`, records the timeout and the kernel returns.
+__global__ void wait_probe_kernel(uint32_t* err, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  const uint32_t b = smem_u32(&bar);
+  mbar_init(b, 1);
+  abort_flag = 0;
+  fence_mbar_init();
+  mbar_wait(b, 0, err, 0x7f, &abort_flag, limit_ns);
+}
+}  // namespace
+
+cudaError_t launch_wait_probe(uint32_t* err, uint64_t limit_ns, cudaStream_t stream) {
+  wait_probe_kernel<<<1, 1, 0, stream>>>(err, limit_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace fa

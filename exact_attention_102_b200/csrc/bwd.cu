@@ -1,0 +1,504 @@
+// bwd.cu — attention backward by recomputation for sm_100a.
+//
+// "Flash Attention 再学习" (jibinghu.github.io), backward: nothing N x N is
+// stored by the forward; S and P are rebuilt tile by tile from Q, K and the
+// per-row statistic. 91haoming.cn repost, "前向傳播改進": the statistic is the
+// logsumexp L = m + log l alone, so P_ij = exp(scale * q_i.k_j - L_i).
+// Same page, "并行化改進": the backward is parallel over K/V column blocks,
+// and the gradient that crosses CTAs is accumulated with atomic adds. Here
+// each CTA owns one 128-key block j (dK_j and dV_j stay on chip until the
+// end) and the cross-CTA accumulation is dQ.
+//
+// Gradients (textbook softmax backward; the pages' formula images were lost):
+//   D_i  = sum_c dO_ic O_ic                      (pre kernel; also zeroes dQ)
+//   P    = exp(scale S - L),  S = Q K^T
+//   dV_j += P^T dO_i,  dP = dO_i V_j^T,  dS = P o (dP - D_i)
+//   dK_j += scale dS^T Q_i,  dQ_i += scale dS K_j   (fp32 reductions to HBM)
+//
+// B200 mapping (one CTA per (batch*head, key block), 384 threads):
+//   warp 0       TMA producer: K_j, V_j once; Q_i and dO_i per row block
+//                through two-stage rings.
+//   warp 1       TMEM allocation; lane 0 issues all tcgen05.mma:
+//                S^T = K_j Q_i^T and dP^T = V_j dO_i^T (smem x smem),
+//                dV += P^T dO_i (P^T from TMEM), dK += dS^T Q_i and
+//                dQ_i = dS K_j (dS from shared memory, read K-major for dK
+//                and MN-major for dQ).
+//   warps 4..7   thread = key row (TMEM lane): P^T from S^T and L, packed to
+//                bf16 in TMEM; dS^T = P^T o (dP^T - D) written to shared
+//                memory in the 128-byte-swizzled layout the MMA reads; at the
+//                end, dK and dV rows to HBM.
+//   warps 8..11  thread = query row of the dQ tile: reads the fp32 dQ tile
+//                from TMEM and adds it to dQ in HBM with vector reductions.
+// TMEM (512 columns): S^T / P^T [0,128), dP^T [128,256) (reused for the dQ
+// tile once dS is out), dV [256, 256+D), dK [256+D, 256+2D).
+#include "prim.cuh"
+#include "kernels.h"
+
+namespace fa {
+
+namespace {
+
+template <int D>
+struct BwdCfg {
+  static constexpr int BK = 128;                 // keys per CTA
+  static constexpr int BQ = 128;                 // queries per iteration
+  static constexpr int TILE = 128 * D * 2;       // one 128-row bf16 tile of Q/K/V/dO
+  static constexpr int CHUNK = 128 * 128;        // one 64-column (128 B) chunk of a tile
+  static constexpr int NCHUNK = D / 64;
+  static constexpr int DS_BYTES = 128 * 128 * 2; // dS^T tile, bf16 [key][query]
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = K_OFF + TILE;
+  static constexpr int Q_OFF = V_OFF + TILE;           // 2 stages
+  static constexpr int DO_OFF = Q_OFF + 2 * TILE;      // 2 stages
+  static constexpr int DS_OFF = DO_OFF + 2 * TILE;
+  static constexpr int L_OFF = DS_OFF + DS_BYTES;       // 2 stages x 128 fp32: L * log2(e)
+  static constexpr int DL_OFF = L_OFF + 2 * 512;        // 2 stages x 128 fp32: D
+  static constexpr int BAR_OFF = DL_OFF + 2 * 512;
+  // barriers
+  static constexpr int B_KV = 0;
+  static constexpr int B_QF = 1, B_QE = 3, B_DF = 5, B_DE = 7;   // [2] each
+  static constexpr int B_ST = 9, B_DPT = 10, B_P = 11, B_DV = 12, B_DS = 13, B_DSFREE = 14;
+  static constexpr int B_DQ = 15, B_DQFREE = 16, B_END = 17, B_DRAIN = 18;
+  static constexpr int NBAR = 19;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  // d = 128 leaves no room for alignment slack: the dynamic shared memory
+  // base must already be 1024-byte aligned (checked at run time)
+  static constexpr int SMEM_BYTES = MISC_OFF + 16;
+  static constexpr uint32_t COL_ST = 0, COL_DPT = 128, COL_DV = 256, COL_DK = 256 + D;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int THREADS = 384;
+};
+
+enum : uint32_t {
+  kSiteKV = 0x31, kSiteQE = 0x32, kSiteDE = 0x33, kSiteQF = 0x34, kSiteDF = 0x35, kSiteP = 0x36,
+  kSiteDV = 0x37, kSiteDS = 0x38, kSiteDQF = 0x39, kSiteST = 0x3a, kSiteDPT = 0x3b,
+  kSiteDSF = 0x3c, kSiteDQ = 0x3d, kSiteEnd = 0x3e, kSiteDrain = 0x3f
+};
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
+}
+
+// ---------------------------------------------------------------- pre pass
+// Per padded row (bh, n), n < n_pad = ceil(N/128)*128:
+//   D[bh][n]  = sum_c dO_nc O_nc  (0 for n >= N)
+//   Ll[bh][n] = L_n * log2(e)     (+inf for n >= N, so P = 0 there)
+// and dQ rows n < N are zeroed (dQ is accumulated by the main pass).
+template <int D>
+__global__ void __launch_bounds__(256) bwd_pre_kernel(BwdArgs a) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long rows = static_cast<long long>(a.B) * a.H * a.n_pad;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  for (long long pr = warp; pr < rows; pr += nw) {
+    const long long bh = pr / a.n_pad;
+    const int n = static_cast<int>(pr - bh * a.n_pad);
+    if (n >= a.N) {
+      if (lane == 0) {
+        a.delta[pr] = 0.f;
+        a.lse_log2[pr] = INFINITY;
+      }
+      continue;
+    }
+    const long long r = bh * a.N + n;
+    const __nv_bfloat16* o = static_cast<const __nv_bfloat16*>(a.o) + r * D;
+    const __nv_bfloat16* g = static_cast<const __nv_bfloat16*>(a.dout) + r * D;
+    float acc = 0.f;
+#pragma unroll
+    for (int c = lane * 2; c < D; c += 64) {
+      const __nv_bfloat162 ov = *reinterpret_cast<const __nv_bfloat162*>(o + c);
+      const __nv_bfloat162 gv = *reinterpret_cast<const __nv_bfloat162*>(g + c);
+      acc = fmaf(__bfloat162float(ov.x), __bfloat162float(gv.x), acc);
+      acc = fmaf(__bfloat162float(ov.y), __bfloat162float(gv.y), acc);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) {
+      a.delta[pr] = acc;
+      a.lse_log2[pr] = a.lse[r] * 1.4426950408889634f;
+    }
+    float4* dq = reinterpret_cast<float4*>(a.dq + r * D);
+    for (int c = lane; c < D / 4; c += 32) dq[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+// --------------------------------------------------------------- main pass
+template <int D>
+__global__ void __launch_bounds__(384, 1)
+bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                BwdArgs a) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t base = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw;
+  if (base & 1023u) {  // 128-byte-swizzled tiles need 1024-byte aligned bases
+    if (threadIdx.x == 0) atomicCAS(a.err, 0u, kErrBadIndex + 0x30);
+    return;
+  }
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int BH = a.B * a.H;
+  const int kb = static_cast<int>(blockIdx.x) / BH;   // key block (longest work first)
+  const int bh = static_cast<int>(blockIdx.x) % BH;
+  const int nq = (a.N + C::BQ - 1) / C::BQ;
+  const int i0 = a.causal ? kb : 0;                    // first query block that sees these keys
+  const int n_it = nq - i0;
+
+  auto bar = [&](int i) -> uint32_t { return base + C::BAR_OFF + 8 * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(C::B_KV), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(C::B_QF + s), 1);
+      mbar_init(bar(C::B_QE + s), 1);
+      mbar_init(bar(C::B_DF + s), 1);
+      mbar_init(bar(C::B_DE + s), 1);
+    }
+    mbar_init(bar(C::B_ST), 1);
+    mbar_init(bar(C::B_DPT), 1);
+    mbar_init(bar(C::B_P), 128);
+    mbar_init(bar(C::B_DV), 1);
+    mbar_init(bar(C::B_DS), 128);
+    mbar_init(bar(C::B_DSFREE), 1);
+    mbar_init(bar(C::B_DQ), 1);
+    mbar_init(bar(C::B_DQFREE), 128);
+    mbar_init(bar(C::B_END), 1);
+    mbar_init(bar(C::B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmDO);
+      mbar_arrive_expect_tx(bar(C::B_KV), 2 * C::TILE);
+      for (int c = 0; c < C::NCHUNK; ++c) {
+        tma_load_3d(base + C::K_OFF + c * C::CHUNK, &tmK, bar(C::B_KV), c * 64, kb * C::BK, bh);
+        tma_load_3d(base + C::V_OFF + c * C::CHUNK, &tmV, bar(C::B_KV), c * 64, kb * C::BK, bh);
+      }
+      int issued = 0;
+      for (int it = 0; it < n_it; ++it) {
+        const int s = it & 1;
+        const uint32_t ph = ((it >> 1) & 1) ^ 1;
+        const int row = (i0 + it) * C::BQ;
+        const size_t prow = static_cast<size_t>(bh) * a.n_pad + row;   // 512 B aligned
+        if (!mbar_wait(bar(C::B_QE + s), ph, a.err, kSiteQE, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(C::B_QF + s), C::TILE + 512);
+        for (int c = 0; c < C::NCHUNK; ++c)
+          tma_load_3d(base + C::Q_OFF + s * C::TILE + c * C::CHUNK, &tmQ, bar(C::B_QF + s),
+                      c * 64, row, bh);
+        bulk_load(base + C::L_OFF + s * 512, a.lse_log2 + prow, 512, bar(C::B_QF + s));
+        if (!mbar_wait(bar(C::B_DE + s), ph, a.err, kSiteDE, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(C::B_DF + s), C::TILE + 512);
+        for (int c = 0; c < C::NCHUNK; ++c)
+          tma_load_3d(base + C::DO_OFF + s * C::TILE + c * C::CHUNK, &tmDO, bar(C::B_DF + s),
+                      c * 64, row, bh);
+        bulk_load(base + C::DL_OFF + s * 512, a.delta + prow, 512, bar(C::B_DF + s));
+        issued = it + 1;
+      }
+      for (int it = max(0, issued - 2); it < issued; ++it) {
+        mbar_wait(bar(C::B_QF + (it & 1)), (it >> 1) & 1, a.err, kSiteDrain, nullptr, 200000000ull);
+        mbar_wait(bar(C::B_DF + (it & 1)), (it >> 1) & 1, a.err, kSiteDrain, nullptr, 200000000ull);
+      }
+      mbar_wait(bar(C::B_KV), 0, a.err, kSiteDrain, nullptr, 200000000ull);
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      constexpr uint32_t idSS = idesc_f16(128, C::BQ, 1, 0, 0);   // S^T, dP^T
+      constexpr uint32_t idKM = idesc_f16(128, D, 1, 0, 1);        // dV (A tmem), dK: B MN-major
+      constexpr uint32_t idQ = idesc_f16(128, D, 1, 1, 1);         // dQ: A and B MN-major
+      const uint32_t kbase = base + C::K_OFF, vbase = base + C::V_OFF, dsb = base + C::DS_OFF;
+      bool ok = mbar_wait(bar(C::B_KV), 0, a.err, kSiteKV, abort_flag);
+      // S^T(it) = K Q_it^T ; dP^T(it) = V dO_it^T
+      auto issue_st = [&](int it) -> bool {
+        const int s = it & 1;
+        if (!mbar_wait(bar(C::B_QF + s), (it >> 1) & 1, a.err, kSiteQF, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t qb = base + C::Q_OFF + s * C::TILE;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
+          umma_f16_ss(tmem + C::COL_ST, smem_desc_sw128(kbase + off, 16, 1024),
+                      smem_desc_sw128(qb + off, 16, 1024), idSS, kk > 0);
+        }
+        umma_commit(bar(C::B_ST));
+        return true;
+      };
+      auto issue_dpt = [&](int it) -> bool {
+        const int s = it & 1;
+        if (!mbar_wait(bar(C::B_DF + s), (it >> 1) & 1, a.err, kSiteDF, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t gb = base + C::DO_OFF + s * C::TILE;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
+          umma_f16_ss(tmem + C::COL_DPT, smem_desc_sw128(vbase + off, 16, 1024),
+                      smem_desc_sw128(gb + off, 16, 1024), idSS, kk > 0);
+        }
+        umma_commit(bar(C::B_DPT));
+        return true;
+      };
+      if (ok) ok = issue_st(0) && issue_dpt(0);
+      for (int it = 0; it < n_it && ok; ++it) {
+        const int s = it & 1;
+        const uint32_t qb = base + C::Q_OFF + s * C::TILE;
+        const uint32_t gb = base + C::DO_OFF + s * C::TILE;
+        // dV += P^T dO_it  (P^T bf16 in TMEM columns [0,64))
+        ok = mbar_wait(bar(C::B_P), it & 1, a.err, kSiteP, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < C::BQ / 16; ++kk)
+          umma_f16_ts(tmem + C::COL_DV, tmem + C::COL_ST + kk * 8,
+                      smem_desc_sw128(gb + kk * 2048, C::CHUNK, 1024), idKM,
+                      (it > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(bar(C::B_DV));
+        if (it + 1 < n_it) {
+          // S^T(it+1) overwrites P^T(it): wait until dV(it) has read it
+          ok = mbar_wait(bar(C::B_DV), it & 1, a.err, kSiteDV, abort_flag);
+          if (!ok) break;
+          ok = issue_st(it + 1);
+          if (!ok) break;
+        }
+        // dK += dS^T Q_it ; dQ_it = dS K   (dS^T bf16 [key][query] in smem)
+        ok = mbar_wait(bar(C::B_DS), it & 1, a.err, kSiteDS, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < C::BQ / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
+          umma_f16_ss(tmem + C::COL_DK, smem_desc_sw128(dsb + off, 16, 1024),
+                      smem_desc_sw128(qb + kk * 2048, C::CHUNK, 1024), idKM,
+                      (it > 0 || kk > 0) ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < C::BK / 16; ++kk)
+          umma_f16_ss(tmem + C::COL_DPT, smem_desc_sw128(dsb + kk * 2048, C::CHUNK, 1024),
+                      smem_desc_sw128(kbase + kk * 2048, C::CHUNK, 1024), idQ, kk > 0 ? 1u : 0u);
+        umma_commit(bar(C::B_DQ));
+        umma_commit(bar(C::B_DSFREE));
+        umma_commit(bar(C::B_QE + s));   // Q_it and its L: S^T, P and dK done
+        umma_commit(bar(C::B_DE + s));   // dO_it and its D: dP^T, dV and dS done
+        if (it + 1 < n_it) {
+          // dP^T(it+1) overwrites the dQ tile: wait until it has been read out
+          ok = mbar_wait(bar(C::B_DQFREE), it & 1, a.err, kSiteDQF, abort_flag);
+          if (!ok) break;
+          ok = issue_dpt(it + 1);
+          if (!ok) break;
+        }
+      }
+      umma_commit(bar(C::B_END));
+      umma_commit(bar(C::B_DRAIN));
+      mbar_wait(bar(C::B_DRAIN), 0, a.err, kSiteDrain, nullptr, 200000000ull);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------- P^T and dS^T (thread = key)
+    const int r = (warp & 3) * 32 + lane;            // key within the block == TMEM lane
+    const int key = kb * C::BK + r;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t st_addr = tmem + lane_off + C::COL_ST;
+    const uint32_t dpt_addr = tmem + lane_off + C::COL_DPT;
+    const float sl2 = a.scale_log2;
+    uint8_t* ds_row = smem + C::DS_OFF + r * 128;    // row r of each 64-query chunk
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      const int s = it & 1;
+      const int q0 = (i0 + it) * C::BQ;
+      const float* Ls = reinterpret_cast<const float*>(smem + C::L_OFF + s * 512);
+      const float* Ds = reinterpret_cast<const float*>(smem + C::DL_OFF + s * 512);
+      // queries >= N have L = +inf (P = 0); the causal diagonal block and keys
+      // >= N need an explicit mask
+      const bool need_mask = (a.causal && key > q0) || key >= a.N;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_ST), it & 1, a.err, kSiteST, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t pk0[32], pk1[32];
+#define PK(i) (((i) < 32) ? pk0[(i)] : pk1[(i)-32])
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {                   // 32 queries at a time
+        uint32_t sr[32];
+        tmem_ld32(st_addr + h * 32, sr);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          const float4 lv = *reinterpret_cast<const float4*>(Ls + h * 32 + e);
+          const float L[4] = {lv.x, lv.y, lv.z, lv.w};
+          float p[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            // P = exp(scale*s - L) = exp2(s*scale*log2e - L*log2e)
+            p[u] = ex2_approx(fmaf(__uint_as_float(sr[e + u]), sl2, -L[u]));
+            if (need_mask && ((a.causal && key > q0 + h * 32 + e + u) || key >= a.N)) p[u] = 0.f;
+          }
+          PK((h * 32 + e) / 2) = pack_bf16x2(p[0], p[1]);
+          PK((h * 32 + e) / 2 + 1) = pack_bf16x2(p[2], p[3]);
+        }
+      }
+      tmem_st32(st_addr, pk0);
+      tmem_st32(st_addr + 32, pk1);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_P));
+      // dS^T = P^T o (dP^T - D)
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_DPT), it & 1, a.err, kSiteDPT, abort_flag));
+      if (!ok) break;
+      if (it > 0) {  // dS buffer reusable once dK(it-1) and dQ(it-1) have read it
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(bar(C::B_DSFREE), (it - 1) & 1, a.err, kSiteDSF, abort_flag));
+        if (!ok) break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        uint32_t dr[32];
+        tmem_ld32(dpt_addr + h * 32, dr);
+        tmem_ld_wait();
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          const float4 dv4 = *reinterpret_cast<const float4*>(Ds + h * 32 + e);
+          const float Dv[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
+          float ds[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint32_t pp = PK((h * 32 + e + u) >> 1);
+            const float pv = __uint_as_float(((e + u) & 1) ? (pp & 0xffff0000u) : (pp << 16));
+            ds[u] = pv * (__uint_as_float(dr[e + u]) - Dv[u]);
+          }
+          w[e / 2] = pack_bf16x2(ds[0], ds[1]);
+          w[e / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+        }
+        // queries h*32 .. h*32+31 = chunk (h/2), 16-byte units (h%2)*4 .. +3 of the
+        // 128-byte row, XOR-swizzled with (key row % 8) like a TMA SWIZZLE_128B tile
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int unit = (h & 1) * 4 + u;
+          uint4* dst = reinterpret_cast<uint4*>(ds_row + (h >> 1) * C::CHUNK +
+                                                ((unit ^ (r & 7)) << 4));
+          *dst = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+        }
+      }
+#undef PK
+      fence_async_smem();   // generic-proxy smem writes -> visible to the MMA
+      tc_fence_before();
+      mbar_arrive(bar(C::B_DS));
+    }
+    // ---- epilogue: dV and dK rows (thread = key) to HBM
+    if (ok) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_END), 0, a.err, kSiteEnd, abort_flag));
+      if (ok) {
+        tc_fence_after();
+        const size_t orow = (static_cast<size_t>(bh) * a.N + key) * D;
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {
+          const uint32_t src = tmem + lane_off + (which ? C::COL_DK : C::COL_DV);
+          float* dst = (which ? a.dk : a.dv) + orow;
+          const float mul = which ? a.scale : 1.f;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(src + c * 32, v);
+            tmem_ld_wait();
+            if (key < a.N) {
+              float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                d4[e] = make_float4(__uint_as_float(v[4 * e]) * mul, __uint_as_float(v[4 * e + 1]) * mul,
+                                    __uint_as_float(v[4 * e + 2]) * mul,
+                                    __uint_as_float(v[4 * e + 3]) * mul);
+            }
+          }
+        }
+      }
+    }
+    tc_fence_before();
+  } else if (warp >= 8) {
+    // ---------------------------------------- dQ tile -> HBM (thread = query)
+    const int r = (warp & 3) * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t src = tmem + lane_off + C::COL_DPT;
+    const float sc = a.scale;
+    for (int it = 0; it < n_it; ++it) {
+      const int q = (i0 + it) * C::BQ + r;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(C::B_DQ), it & 1, a.err, kSiteDQ, abort_flag)))
+        break;
+      tc_fence_after();
+      float* dst = a.dq + (static_cast<size_t>(bh) * a.N + q) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(src + c * 32, v);
+        tmem_ld_wait();
+        if (q < a.N) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            red_add_v4(dst + c * 32 + 4 * e, __uint_as_float(v[4 * e]) * sc,
+                       __uint_as_float(v[4 * e + 1]) * sc, __uint_as_float(v[4 * e + 2]) * sc,
+                       __uint_as_float(v[4 * e + 3]) * sc);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(C::B_DQFREE));
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+template <int D>
+cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tdo, const BwdArgs& a, cudaStream_t stream) {
+  using C = BwdCfg<D>;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(bwd_main_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const long long rows = static_cast<long long>(a.B) * a.H * a.n_pad;
+  const long long want = (rows + 7) / 8;
+  const int pre_blocks = static_cast<int>(want < 148 * 16 ? want : 148 * 16);
+  bwd_pre_kernel<D><<<pre_blocks, 256, 0, stream>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int nk = (a.N + C::BK - 1) / C::BK;
+  bwd_main_kernel<D><<<nk * a.B * a.H, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
+  return cudaGetLastError();
+}
+
+template cudaError_t launch_bwd<64>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                                    const CUtensorMap&, const BwdArgs&, cudaStream_t);
+template cudaError_t launch_bwd<128>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                                     const CUtensorMap&, const BwdArgs&, cudaStream_t);
+
+}  // namespace fa

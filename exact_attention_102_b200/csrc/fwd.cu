@@ -1,0 +1,386 @@
+// fwd.cu — fused one-pass attention forward for sm_100a (bf16 in, fp32
+// accumulate, bf16 O and fp32 logsumexp out).
+//
+// Algorithm ("FlashAttention系列优化", FlashAttentionV2; "Flash Attention
+// 再学习", 1-pass FlashAttention): Q row blocks form the outer loop (one CTA
+// owns two 128-row Q tiles), K/V blocks of 128 rows the inner loop. Per row
+// the kernel keeps a running max m and running sum l, keeps O unnormalised,
+// rescales it by exp(m_old - m_new) when m moves, and divides by l once at the
+// end; L = m + log l is the only statistic written (91haoming.cn repost,
+// "前向傳播改進").
+//
+// B200 mapping (the pages' A100/H100 warp layouts are prior art only):
+//   warp 0        TMA producer: Q tiles once, then K_j, V_j through an
+//                 NSTAGE-deep shared-memory ring guarded by full/empty
+//                 mbarriers (the producer/consumer circular buffer of
+//                 FlashAttention-3, with TMA).
+//   warp 1        allocates TMEM; lane 0 issues every tcgen05.mma:
+//                 S_t = Q_t K_j^T (smem x smem -> TMEM fp32) and
+//                 O_t += P_t V_j (P from TMEM x V from smem -> TMEM fp32).
+//   warps 4..7    softmax for Q tile 0, warps 8..11 for Q tile 1: each
+//                 thread owns one row (one TMEM lane), so the row max and row
+//                 sum need no shuffles. While one tile's softmax runs, the
+//                 tensor core works on the other tile (ping-pong).
+// TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+D),
+// O_1 [256+D, 256+2D). P_t (bf16, packed 2 per column) overwrites the first
+// 64 columns of S_t and feeds the P.V MMA directly from TMEM.
+// Rescale skipping: m is only moved when a new row max exceeds it by more
+// than 2^8 in exp2 units; until then exp2(x - m) <= 256, which fp32 and bf16
+// hold exactly as well as values <= 1. The final O / l and L = m + log l use
+// the same m, so the result is the same exact quantity.
+#include "prim.cuh"
+#include "kernels.h"
+
+namespace fa {
+
+namespace {
+
+template <int D>
+struct FwdCfg {
+  static constexpr int BM = 128;                 // Q rows per tile
+  static constexpr int BN = 128;                 // K/V rows per tile
+  static constexpr int TILE = 128 * D * 2;       // bytes of one 128-row bf16 tile
+  static constexpr int CHUNK = 128 * 128;        // bytes of one 64-column (128 B) chunk
+  static constexpr int NCHUNK = D / 64;
+  static constexpr int NSTAGE = (D == 128) ? 4 : 8;
+  static constexpr int Q_OFF = 0;
+  static constexpr int RING_OFF = 2 * TILE;
+  static constexpr int BAR_OFF = RING_OFF + NSTAGE * TILE;
+  // barriers: q_full | kv_full[NSTAGE] | kv_empty[NSTAGE] | s_full[2] | p_full[2] | o_full[2] | drain
+  static constexpr int B_Q = 0;
+  static constexpr int B_KVF = 1;
+  static constexpr int B_KVE = 1 + NSTAGE;
+  static constexpr int B_S = 1 + 2 * NSTAGE;
+  static constexpr int B_P = B_S + 2;
+  static constexpr int B_O = B_P + 2;
+  static constexpr int B_DRAIN = B_O + 2;
+  static constexpr int NBAR = B_DRAIN + 1;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // tmem slot (4 B), abort flag (4 B)
+  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + slack for 1024 B alignment
+  // TMEM column of S_t / P_t and of O_t
+  static __device__ __forceinline__ uint32_t s_col(int t) { return 128u * t; }
+  static __device__ __forceinline__ uint32_t o_col(int t) { return 256u + D * t; }
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int THREADS = 384;
+};
+
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+// wait-site ids (reported in the device error word)
+enum : uint32_t {
+  kSiteQ = 1, kSiteKvEmpty = 2, kSiteKvFull = 3, kSiteS = 4, kSiteP = 5, kSiteO = 6,
+  kSiteEpi = 7, kSiteDrain = 8
+};
+
+template <int D>
+__global__ void __launch_bounds__(384, 1)
+fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+           const __grid_constant__ CUtensorMap tmV, FwdArgs a) {
+  using C = FwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw_addr);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int BH = a.B * a.H;
+  const int pair = a.n_pairs - 1 - static_cast<int>(blockIdx.x) / BH;  // heaviest first
+  const int bh = static_cast<int>(blockIdx.x) % BH;
+  const int nkb = (a.N + C::BN - 1) / C::BN;
+
+  // per-tile extent: rows [q0, q0+128), key blocks [0, nkb_t)
+  int q0[2], nkb_t[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    q0[t] = (pair * 2 + t) * C::BM;
+    nkb_t[t] = (q0[t] >= a.N) ? 0 : (a.causal ? min(nkb, pair * 2 + t + 1) : nkb);
+  }
+  const int nkb_cta = max(nkb_t[0], nkb_t[1]);
+
+  auto bar = [&](int i) -> uint32_t { return base + C::BAR_OFF + 8 * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(C::B_Q), 1);
+    for (int s = 0; s < C::NSTAGE; ++s) {
+      mbar_init(bar(C::B_KVF + s), 1);
+      mbar_init(bar(C::B_KVE + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(C::B_S + t), 1);
+      mbar_init(bar(C::B_P + t), 128);
+      mbar_init(bar(C::B_O + t), 1);
+    }
+    mbar_init(bar(C::B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      int nq = (nkb_t[0] > 0) + (nkb_t[1] > 0);
+      mbar_arrive_expect_tx(bar(C::B_Q), nq * C::TILE);
+      for (int t = 0; t < 2; ++t) {
+        if (nkb_t[t] == 0) continue;
+        for (int c = 0; c < C::NCHUNK; ++c)
+          tma_load_3d(base + C::Q_OFF + t * C::TILE + c * C::CHUNK, &tmQ, bar(C::B_Q), c * 64,
+                      q0[t], bh);
+      }
+      int it = 0;
+      bool ok = true;
+      for (int j = 0; j < nkb_cta && ok; ++j) {
+        for (int w = 0; w < 2 && ok; ++w, ++it) {
+          const int s = it % C::NSTAGE;
+          const uint32_t ph = (it / C::NSTAGE) & 1;
+          ok = mbar_wait(bar(C::B_KVE + s), ph ^ 1, a.err, kSiteKvEmpty, abort_flag);
+          if (!ok) break;
+          mbar_arrive_expect_tx(bar(C::B_KVF + s), C::TILE);
+          const CUtensorMap* m = (w == 0) ? &tmK : &tmV;
+          for (int c = 0; c < C::NCHUNK; ++c)
+            tma_load_3d(base + C::RING_OFF + s * C::TILE + c * C::CHUNK, m, bar(C::B_KVF + s),
+                        c * 64, j * C::BN, bh);
+        }
+      }
+      // drain: make sure the last loads issued have landed before teardown
+      const int issued = it;
+      for (int k = max(0, issued - C::NSTAGE); k < issued; ++k)
+        mbar_wait(bar(C::B_KVF + k % C::NSTAGE), (k / C::NSTAGE) & 1, a.err, kSiteDrain,
+                  nullptr, 200000000ull);
+      if (nq) mbar_wait(bar(C::B_Q), 0, a.err, kSiteDrain, nullptr, 200000000ull);
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_f16(128, C::BN, 1, 0, 0);
+      constexpr uint32_t idPV = idesc_f16(128, D, 1, 0, 1);
+      int it = 0;
+      int npv[2] = {0, 0};
+      bool ok = mbar_wait(bar(C::B_Q), 0, a.err, kSiteQ, abort_flag);
+      for (int j = 0; j < nkb_cta && ok; ++j) {
+        // ---- S_t = Q_t K_j^T
+        {
+          const int s = it % C::NSTAGE;
+          ok = mbar_wait(bar(C::B_KVF + s), (it / C::NSTAGE) & 1, a.err, kSiteKvFull, abort_flag);
+          if (!ok) break;
+          ++it;
+          tc_fence_after();
+          const uint32_t kb = base + C::RING_OFF + s * C::TILE;
+          for (int t = 0; t < 2; ++t) {
+            if (j >= nkb_t[t]) continue;
+            if (npv[t] > 0) {  // P_t of block j-1 must be consumed before S_t is overwritten
+              ok = mbar_wait(bar(C::B_O + t), (npv[t] - 1) & 1, a.err, kSiteO, abort_flag);
+              if (!ok) break;
+              tc_fence_after();
+            }
+            const uint32_t qb = base + C::Q_OFF + t * C::TILE;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
+              umma_f16_ss(tmem + C::s_col(t), smem_desc_sw128(qb + off, 16, 1024),
+                          smem_desc_sw128(kb + off, 16, 1024), idS, kk > 0);
+            }
+            umma_commit(bar(C::B_S + t));
+          }
+          if (!ok) break;
+          umma_commit(bar(C::B_KVE + s));
+        }
+        // ---- O_t += P_t V_j
+        {
+          const int s = it % C::NSTAGE;
+          ok = mbar_wait(bar(C::B_KVF + s), (it / C::NSTAGE) & 1, a.err, kSiteKvFull, abort_flag);
+          if (!ok) break;
+          ++it;
+          const uint32_t vb = base + C::RING_OFF + s * C::TILE;
+          for (int t = 0; t < 2; ++t) {
+            if (j >= nkb_t[t]) continue;
+            ok = mbar_wait(bar(C::B_P + t), npv[t] & 1, a.err, kSiteP, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < C::BN / 16; ++kk) {
+              umma_f16_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8,
+                          smem_desc_sw128(vb + kk * 2048, C::CHUNK, 1024), idPV,
+                          (npv[t] > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(bar(C::B_O + t));
+            ++npv[t];
+          }
+          if (!ok) break;
+          umma_commit(bar(C::B_KVE + s));
+        }
+      }
+      // drain every MMA this thread issued before TMEM is released
+      umma_commit(bar(C::B_DRAIN));
+      mbar_wait(bar(C::B_DRAIN), 0, a.err, kSiteDrain, nullptr, 200000000ull);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------- softmax
+    const int t = (warp - 4) >> 2;
+    const int r = (warp & 3) * 32 + lane;           // row within the tile == TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t s_addr = tmem + lane_off + C::s_col(t);
+    const uint32_t o_addr = tmem + lane_off + C::o_col(t);
+    const int row = q0[t] + r;
+    const int limit = a.causal ? min(row, a.N - 1) : a.N - 1;  // last visible key
+    const float sl2 = a.scale_log2;
+    float m_run = -INFINITY;
+    float l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nkb_t[t]; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_S + t), j & 1, a.err, kSiteS, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, sr[c]);
+      tmem_ld_wait();
+#define SV(c) __uint_as_float(sr[(c) >> 5][(c)&31])
+      const int kbase = j * C::BN;
+      if (kbase + C::BN - 1 > limit) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (kbase + c > limit) sr[c >> 5][c & 31] = 0xff800000u;  // -inf
+      }
+      float mx0 = SV(0), mx1 = SV(1), mx2 = SV(2), mx3 = SV(3);
+#pragma unroll
+      for (int c = 4; c < 128; c += 4) {
+        mx0 = fmaxf(mx0, SV(c));
+        mx1 = fmaxf(mx1, SV(c + 1));
+        mx2 = fmaxf(mx2, SV(c + 2));
+        mx3 = fmaxf(mx3, SV(c + 3));
+      }
+      const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      float alpha = 1.f;
+      if (mx > m_run + kRescaleThreshold) {  // also true for the first block (m_run = -inf)
+        alpha = ex2_approx(m_run - mx);      // exp2(-inf) = 0 on the first block
+        m_run = mx;
+      }
+      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+      // l sums the bf16-rounded P that the P.V product uses, so numerator and
+      // denominator weigh every key identically
+      float l0 = 0.f, l1 = 0.f;
+      uint32_t pk0[32], pk1[32];
+#pragma unroll
+      for (int c = 0; c < 64; c += 2) {
+        const uint32_t u = pack_bf16x2(ex2_approx(fmaf(SV(c), sl2, -m_use)),
+                                       ex2_approx(fmaf(SV(c + 1), sl2, -m_use)));
+        l0 += __uint_as_float(u << 16);
+        l1 += __uint_as_float(u & 0xffff0000u);
+        pk0[c >> 1] = u;
+      }
+#pragma unroll
+      for (int c = 64; c < 128; c += 2) {
+        const uint32_t u = pack_bf16x2(ex2_approx(fmaf(SV(c), sl2, -m_use)),
+                                       ex2_approx(fmaf(SV(c + 1), sl2, -m_use)));
+        l0 += __uint_as_float(u << 16);
+        l1 += __uint_as_float(u & 0xffff0000u);
+        pk1[(c - 64) >> 1] = u;
+      }
+#undef SV
+      l_run = l_run * alpha + (l0 + l1);
+      tmem_st32(s_addr, pk0);
+      tmem_st32(s_addr + 32, pk1);
+      // O rescale (PV of block j-1 has completed: S_t(j) was issued after it)
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t orr[32];
+          tmem_ld32(o_addr + c * 32, orr);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+          tmem_st32(o_addr + c * 32, orr);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_P + t));
+    }
+    // ------------------------------------------------------------ epilogue
+    if (ok && nkb_t[t] > 0) {
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(bar(C::B_O + t), (nkb_t[t] - 1) & 1, a.err, kSiteEpi, abort_flag));
+      if (ok) {
+        tc_fence_after();
+        const float inv_l = 1.f / l_run;
+        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) +
+                              (static_cast<size_t>(bh) * a.N + row) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t orr[32];
+          tmem_ld32(o_addr + c * 32, orr);
+          tmem_ld_wait();
+          if (row < a.N) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int b = 8 * e;
+              dst[e] = make_uint4(
+                  pack_bf16x2(__uint_as_float(orr[b + 0]) * inv_l, __uint_as_float(orr[b + 1]) * inv_l),
+                  pack_bf16x2(__uint_as_float(orr[b + 2]) * inv_l, __uint_as_float(orr[b + 3]) * inv_l),
+                  pack_bf16x2(__uint_as_float(orr[b + 4]) * inv_l, __uint_as_float(orr[b + 5]) * inv_l),
+                  pack_bf16x2(__uint_as_float(orr[b + 6]) * inv_l, __uint_as_float(orr[b + 7]) * inv_l));
+            }
+          }
+        }
+        if (row < a.N)
+          a.lse[static_cast<size_t>(bh) * a.N + row] = (m_run + log2f(l_run)) * 0.6931471805599453f;
+      }
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+template <int D>
+int fwd_smem_bytes() {
+  return FwdCfg<D>::SMEM_BYTES;
+}
+
+template <int D>
+cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const FwdArgs& a, cudaStream_t stream) {
+  using C = FwdCfg<D>;
+  static bool attr_set[64] = {};  // per device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const int grid = a.n_pairs * a.B * a.H;
+  fwd_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, a);
+  return cudaGetLastError();
+}
+
+template cudaError_t launch_fwd<64>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                                    const FwdArgs&, cudaStream_t);
+template cudaError_t launch_fwd<128>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                                     const FwdArgs&, cudaStream_t);
+
+}  // namespace fa

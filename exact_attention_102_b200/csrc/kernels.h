@@ -1,0 +1,100 @@
+// kernels.h — launch interfaces between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fa {
+
+struct FwdArgs {
+  void* o;            // bf16 [B][H][N][D]
+  float* lse;         // fp32 [B][H][N]
+  int B, H, N;
+  int causal;
+  int n_pairs;        // ceil(N / 256): pairs of 128-row Q tiles per head
+  float scale_log2;   // softmax scale * log2(e)
+  uint32_t* err;      // device error word
+};
+
+template <int D>
+cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const FwdArgs& a, cudaStream_t stream);
+
+struct BwdArgs {
+  const void* q;      // bf16 BHND
+  const void* k;
+  const void* v;
+  const void* o;
+  const void* dout;
+  const float* lse;   // fp32 [B][H][N]
+  float* dq;          // fp32 BHND (accumulated with reductions; zeroed by the pre kernel)
+  float* dk;          // fp32 BHND
+  float* dv;          // fp32 BHND
+  float* delta;       // fp32 [B][H][n_pad]: D_i = sum_c dO_ic O_ic (0 past N)
+  float* lse_log2;    // fp32 [B][H][n_pad]: L_i * log2(e) (+inf past N)
+  int B, H, N;
+  int n_pad;          // N rounded up to a multiple of 128
+  int causal;
+  float scale;        // softmax scale
+  float scale_log2;   // scale * log2(e)
+  uint32_t* err;
+};
+
+template <int D>
+cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tdo, const BwdArgs& a, cudaStream_t stream);
+
+struct DecodeArgs {
+  const void* q;            // bf16 [S][Hq][d]
+  const void* k_cache;      // bf16 [P][Hkv][16][d]
+  const void* v_cache;
+  const int* block_table;   // int32 [S][max_blocks]
+  int num_phys;             // physical blocks per cache (valid ids are [0, num_phys))
+  const int* context_lens;  // int32 [S]
+  void* o;                  // bf16 [S][Hq][d]
+  float* lse;               // fp32 [S][Hq] or null
+  float* part_o;            // fp32 [S][Hq][max_splits][d]
+  float* part_l;            // fp32 [S][Hq][max_splits]
+  int num_seqs, Hq, Hkv, max_blocks, max_ctx, max_splits, split_blocks;
+  float scale_log2;
+  uint32_t* err;
+};
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+
+struct Fp8PrepArgs {
+  const void* q;      // bf16 BHND
+  const void* k;
+  const void* v;
+  const float* R;     // fp32 [d][d]
+  uint8_t* q8;        // e4m3 BHND
+  uint8_t* k8;
+  uint8_t* v8;
+  float* sq;          // fp32 [B][H][ceil(N/64)]
+  float* sk;
+  float* sv;
+  int B, H, N;
+};
+
+cudaError_t launch_fp8_prepare(const Fp8PrepArgs& a, cudaStream_t stream);
+
+struct Fp8FwdArgs {
+  const float* sq;
+  const float* sk;
+  const float* sv;
+  void* o;
+  float* lse;
+  int B, H, N;
+  int causal;
+  int n_pairs;
+  float scale_log2;
+  uint32_t* err;
+};
+
+cudaError_t launch_fwd_fp8(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           const Fp8FwdArgs& a, cudaStream_t stream);
+
+cudaError_t launch_wait_probe(uint32_t* err, uint64_t limit_ns, cudaStream_t stream);
+
+}  // namespace fa

@@ -1,0 +1,210 @@
+/*
+ * fa.h — C ABI of the B200 (sm_100a) exact-attention library libfa.so.
+ *
+ * What it computes (sources are web pages on FlashAttention/PagedAttention):
+ *   O = softmax(scale * Q K^T [+ causal mask]) V, one pass over K/V tiles with
+ *   a running row max m and running row sum l, the unnormalised output
+ *   rescaled by exp(m_old - m_new) and divided by l once at the end, plus the
+ *   per-row logsumexp L = m + log l
+ *     - "FlashAttention系列优化" (johneyzheng.top), sections FlashAttentionV1
+ *       (online softmax) and FlashAttentionV2 (delayed rescaling, Q-outer /
+ *       KV-inner loop order);
+ *     - FlashAttention v1/v2/v3 overview (91haoming.cn repost), "前向傳播改進"
+ *       (store only L = m + log l) and "并行化改進" (parallel over row blocks
+ *       forward, over column blocks backward);
+ *     - "Flash Attention 再学习" (jibinghu.github.io): 1-pass tiling, backward
+ *       by recomputing S and P from the stored statistics.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers, owned by the caller, at least
+ *     16-byte aligned (TMA requirement); the library keeps no reference to them
+ *     after the call returns.
+ *   - "BHND" = [B][H][N][d] contiguous row-major; bf16 = IEEE bfloat16 bits.
+ *   - Softmax scale is fixed at 1/sqrt(d). Scores, L and all accumulation are
+ *     fp32. L is the natural-log logsumexp of the scaled scores.
+ *   - Causal: query row i attends key j iff j <= i (same N for Q and K).
+ *   - d must be 64 or 128 (FA_ERR_UNSUPPORTED otherwise); N >= 1; any N is
+ *     allowed (ragged last tiles are masked / zero-filled).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream). A non-FA_OK return means nothing was launched.
+ *   - Every wait inside a kernel is bounded; a wait that gives up records an
+ *     error in a device-side word and the kernel returns early. Such failures
+ *     surface through fa_last_device_error(), not through the launch status.
+ *   - The library holds no global state apart from a per-device cache of
+ *     device attributes and the device error word.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+
+/* Symbols the shared library exports (it is built with hidden visibility). */
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,  /* null / misaligned pointer, non-positive size */
+  FA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. d not 64/128) */
+  FA_ERR_LAUNCH = 3,       /* CUDA runtime refused the launch */
+  FA_ERR_TIMEOUT = 4,      /* a bounded in-kernel wait gave up */
+  FA_ERR_WORKSPACE = 5     /* workspace missing or too small */
+} fa_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+FA_API const char* fa_status_str(fa_status s);
+
+/*
+ * fa_fwd — fused one-pass attention forward.
+ *   q, k, v : bf16 BHND inputs.
+ *   o       : bf16 BHND output, O = diag(l)^-1 * sum_j exp(S_j - m) V_j
+ *             rounded to bf16 (round to nearest even).
+ *   lse     : fp32 [B][H][N] output, L = m + log(l) (natural log), the only
+ *             softmax statistic kept for the backward.
+ * Partitioning: one CTA per (batch, head, pair of 128-row Q tiles); K/V tiles
+ * of 128 rows stream through a shared-memory ring ("并行化改進": row blocks are
+ * independent, no communication between CTAs).
+ * Errors: FA_ERR_INVALID_ARG for null/misaligned pointers or B, H, N < 1;
+ * FA_ERR_UNSUPPORTED for d not in {64, 128}; FA_ERR_LAUNCH if CUDA fails.
+ */
+FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int H, int N, int d, int causal, void* stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs: two fp32 per-row vectors over N
+ * rounded up to a multiple of 128 rows — the row statistic D and L * log2(e)
+ * (padded with 0 / +inf) — each rounded up to 256 bytes. dq itself (fp32)
+ * serves as the dQ accumulator.
+ */
+FA_API size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * fa_bwd — attention backward by recomputation.
+ *   q, k, v, o, dout : bf16 BHND (o = fa_fwd's output, dout = dL/dO).
+ *   lse              : fp32 [B][H][N] from fa_fwd.
+ *   dq, dk, dv       : fp32 BHND outputs (gradients w.r.t. q, k, v).
+ *   workspace        : device buffer of >= fa_bwd_workspace_bytes() bytes,
+ *                      owned by the caller; contents on entry are ignored.
+ * Steps: D_i = sum_c dO_ic O_ic (and dq := 0); then, per K/V column block j
+ * (one CTA),
+ * P = exp(scale*Q_i K_j^T - L_i) for every Q row block i it sees,
+ * dV_j += P^T dO_i, dP = dO_i V_j^T, dS = P o (dP - D_i),
+ * dK_j += scale dS^T Q_i, and dQ_i += scale dS K_j accumulated across CTAs
+ * with fp32 reductions; dK_j and dV_j are written once.
+ * ("Flash Attention 再学习": backward recomputes S and P from the stored
+ * statistics; 91haoming.cn repost, "并行化改進": backward is parallel over
+ * column blocks with atomic adds for the shared gradient.)
+ * Errors: as fa_fwd, plus FA_ERR_WORKSPACE when workspace is NULL or smaller
+ * than required.
+ */
+FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o,
+                 const float* lse, const void* dout, float* dq, float* dk, float* dv,
+                 void* workspace, size_t ws_bytes,
+                 int B, int H, int N, int d, int causal, void* stream);
+
+/*
+ * Bytes of device workspace paged_attn_decode needs for split partials
+ * (fp32 O and L per (sequence, query head, split)) when no sequence is
+ * longer than max_ctx tokens.
+ */
+FA_API size_t paged_attn_decode_workspace_bytes(int num_seqs, int Hq, int d, int max_ctx);
+
+/*
+ * paged_attn_decode — one query token per sequence against a paged KV cache.
+ *   q            : bf16 [num_seqs][Hq][d].
+ *   k_cache,
+ *   v_cache      : bf16 [num_phys_blocks][Hkv][block_size][d]; one
+ *                  (block, kv head) is block_size*d contiguous elements.
+ *   num_phys_blocks : number of physical blocks in each cache; a table entry
+ *                  outside [0, num_phys_blocks) is never dereferenced: the
+ *                  kernel reads block 0 in its place and records the error,
+ *                  which fa_last_device_error() reports as FA_ERR_INVALID_ARG.
+ *   block_table  : int32 [num_seqs][max_blocks_per_seq]; token t of sequence s
+ *                  is in physical block block_table[s][t / block_size] at slot
+ *                  t % block_size ("FlashAttention系列优化", PagedAttention:
+ *                  logical blocks map to physical blocks through a table;
+ *                  several sequences may map to the same physical block).
+ *                  Entries past ceil(ctx/block_size) are never read.
+ *   context_lens : int32 [num_seqs], each in [1, max_ctx].
+ *   o            : bf16 [num_seqs][Hq][d] output.
+ *   lse          : fp32 [num_seqs][Hq] output, or NULL to skip it.
+ *   Query head h reads KV head h / (Hq / Hkv). The query attends to all
+ *   context_lens[s] cached tokens (no mask).
+ *   workspace    : >= paged_attn_decode_workspace_bytes(num_seqs, Hq, d,
+ *                  max_ctx) bytes; max_ctx must bound every context length.
+ * Each (sequence, KV head, split of the context) is one CTA producing a
+ * partial (O_s, L_s); a second kernel merges them:
+ * L = log sum_s exp(L_s), O = sum_s exp(L_s - L) O_s.
+ * Errors: FA_ERR_INVALID_ARG (null/misaligned pointers, sizes < 1, Hq not a
+ * multiple of Hkv); FA_ERR_UNSUPPORTED (d != 128, block_size != 16,
+ * Hq/Hkv != 4); FA_ERR_WORKSPACE; FA_ERR_LAUNCH. Context lengths are read on
+ * the device: a length outside [1, max_ctx] is clamped into that range.
+ */
+FA_API fa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                            int num_phys_blocks, const int* block_table, int max_blocks_per_seq,
+                            const int* context_lens, void* o, float* lse,
+                            int num_seqs, int Hq, int Hkv, int d, int block_size,
+                            int max_ctx, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * fa_fp8_prepare — incoherent processing + per-block e4m3 quantisation.
+ *   q, k, v    : bf16 BHND inputs.
+ *   R          : fp32 [d][d] orthogonal matrix (row-major); Q' = Q R and
+ *                K' = K R, so Q'K'^T = Q K^T ("FlashAttention系列优化",
+ *                FlashAttentionV3: multiply Q and K by a random orthogonal
+ *                matrix to spread outliers without changing the result).
+ *   q8, k8, v8 : e4m3 BHND outputs (1 byte per element).
+ *   sq, sk, sv : fp32 [B][H][ceil(N/64)] per-block scales: a block is 64 token
+ *                rows x d of one (b, h); scale = amax / 448 (1 if the block is
+ *                all zero), x8 = round_to_nearest_even(x / scale) saturated to
+ *                +-448 ("block quantization": one scale per block).
+ * Errors: as fa_fwd (d must be 128).
+ */
+FA_API fa_status fa_fp8_prepare(const void* q, const void* k, const void* v, const float* R,
+                         void* q8, void* k8, void* v8, float* sq, float* sk, float* sv,
+                         int B, int H, int N, int d, void* stream);
+
+/*
+ * fa_fwd_fp8 — attention forward on e4m3 inputs with per-block scales.
+ *   q8, k8, v8 : e4m3 BHND (from fa_fp8_prepare); sq, sk, sv their scales.
+ *   o          : bf16 BHND output; lse: fp32 [B][H][N].
+ * S = scale * sq_i * sk_j * (q8 k8^T) per 64-row block pair; the V block
+ * scale is folded into P before P is rounded to e4m3 for the P.V product.
+ * Errors: as fa_fwd (d must be 128).
+ */
+FA_API fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8,
+                     const float* sq, const float* sk, const float* sv,
+                     void* o, float* lse, int B, int H, int N, int d, int causal,
+                     void* stream);
+
+/*
+ * fa_last_device_error — synchronises `stream`, then reads and clears the
+ * device error word of the current device. Returns FA_OK when nothing was
+ * recorded since the last call, FA_ERR_TIMEOUT when a bounded wait gave up,
+ * FA_ERR_INVALID_ARG when a kernel met an out-of-range index in its inputs
+ * (a block-table entry), or FA_ERR_LAUNCH when the synchronisation failed.
+ */
+FA_API fa_status fa_last_device_error(void* stream);
+
+/*
+ * fa_debug_wait_timeout — launches one CTA that waits on a shared-memory
+ * barrier nothing ever arrives at, using the same bounded wait as the
+ * kernels above, with a limit of `timeout_us` microseconds (1..1000000).
+ * The wait gives up, records FA_ERR_TIMEOUT in the device error word and
+ * the kernel returns. Exists so tests can check the failure path without
+ * faulting or hanging a GPU.
+ */
+FA_API fa_status fa_debug_wait_timeout(unsigned int timeout_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

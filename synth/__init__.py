@@ -80,7 +80,7 @@ def orthogonal_matrix(d, seed):
 
 
 def paged_decode_layout(num_seqs, block_size, ctx_lo, ctx_hi, seed, group=4,
-                        share_frac=0.10, extra_blocks=0):
+                        share_frac=0.10, extra_blocks=0, table_blocks=None):
     """Index structure of a paged KV cache with parallel-sampling sharing.
 
     Returns dict with numpy arrays:
@@ -93,12 +93,17 @@ def paged_decode_layout(num_seqs, block_size, ctx_lo, ctx_hi, seed, group=4,
     s_g = min(round(share_frac * mean blocks of the group), min blocks of the
     group - 1) (so the last, partially filled block is always private).
     ``extra_blocks`` unused physical blocks are added (spread by the
-    permutation) so ids are not dense.
+    permutation) so ids are not dense. The table has ``table_blocks``
+    columns (default ceil(ctx_hi / block_size), enough for any length the
+    recipe can draw).
     """
     rng = np.random.default_rng(int(seed))
     lens = rng.integers(ctx_lo, ctx_hi + 1, size=num_seqs).astype(np.int64)
     nblk = (lens + block_size - 1) // block_size
     max_blocks = int(nblk.max())
+    if table_blocks is None:
+        table_blocks = (ctx_hi + block_size - 1) // block_size
+    table_blocks = max(int(table_blocks), max_blocks)
     logical = []   # per sequence: list of "allocation ids"
     next_id = 0
     shared = 0
@@ -119,7 +124,7 @@ def paged_decode_layout(num_seqs, block_size, ctx_lo, ctx_hi, seed, group=4,
                 shared += s_g
     num_phys = next_id + int(extra_blocks)
     perm = rng.permutation(num_phys).astype(np.int64)
-    table = np.zeros((num_seqs, max_blocks), dtype=np.int32)
+    table = np.zeros((num_seqs, table_blocks), dtype=np.int32)
     for s, ids in enumerate(logical):
         table[s, :len(ids)] = perm[np.asarray(ids, dtype=np.int64)]
     return {
