@@ -1,0 +1,541 @@
+"""Benchmark of the exact-attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one forward + backward pass (fa_fwd + fa_bwd through the C ABI) of
+the long-sequence workload: B=1, H=16, N=16384, d=128, causal, bf16 inputs
+~N(0,1) (synthetic, seeded). The metric is attention fwd+bwd TFLOP/s with the
+algorithmic FLOP count 4*B*H*N^2*d (forward) + 10*B*H*N^2*d (backward: five
+N x N x d products), halved for the causal mask. Operands (5 bf16 tensors of
+67 MB plus 3 fp32 gradients of 134 MB) exceed the 126 MB L2, so no flush is
+needed between steps.
+
+Besides the headline, the JSON line carries "parts": the forward and backward
+alone, the GPT-2-small-shaped fwd+bwd (B=8, H=12, N=1024, d=64, causal), the
+paged decode (64 sequences, 32/8 heads, d=128, contexts U[512, 32768], 16-token
+blocks, shuffled table with 4-way prefix sharing) in HBM GB/s, and the FP8
+forward (B=4, H=16, N=4096, d=128) when available.
+
+Multi-GPU (torchrun): every rank runs the same per-GPU workload (independent
+heads: weak scaling, no collective on the data path); the time is the max over
+ranks. --impl reference times the float64 CPU oracle on a bounded sample of
+the same workload (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+WORKLOAD = dict(B=1, H=16, N=16384, d=128, causal=True)
+METRIC = "attention fwd+bwd TFLOP/s (bf16)"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def attn_flops(B, H, N, d, causal, bwd=False):
+    f = (10.0 if bwd else 4.0) * B * H * N * N * d
+    return f / 2 if causal else f
+
+
+# ------------------------------------------------------------------ clocks --
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []          # (arrival time, line)
+        self.window = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+            time.sleep(0.3)      # let the sampler start before the region it watches
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, t0, t1):
+        """Keep only samples that arrived inside [t0, t1] (wall clock)."""
+        self.window = (t0, t1)
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ts, line in self.lines:
+            if self.window and not (self.window[0] <= ts <= self.window[1] + 0.06):
+                continue
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# -------------------------------------------------------------- distributed --
+def _dist_init():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def _barrier(ws):
+    if ws > 1:
+        torch.distributed.barrier()
+
+
+def _max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _ev():
+    return torch.cuda.Event(enable_timing=True)
+
+
+# --------------------------------------------------------------- our arm ---
+def run_fwd_bwd(fa, B, H, N, d, causal, steps, warmup, ws, seed, sampler_gpu=None):
+    """Device-resident fwd+bwd steps. Returns timing dict (max over ranks)."""
+    x = synth.attention_inputs(B, H, N, d, seed, device="cuda")
+    o = torch.empty_like(x["q"])
+    lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    dq, dk, dv = (torch.empty((B, H, N, d), dtype=torch.float32, device="cuda") for _ in range(3))
+    wsp = torch.empty(fa.fa_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device="cuda")
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record()
+        fa.fa_fwd(x["q"], x["k"], x["v"], causal=causal, o=o, lse=lse)
+        if evs is not None:
+            evs[1].record()
+        fa.fa_bwd(x["q"], x["k"], x["v"], o, lse, x["do"], causal=causal, dq=dq, dk=dk, dv=dv,
+                  workspace=wsp)
+        if evs is not None:
+            evs[2].record()
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_error() == fa.FA_OK
+    evs = [[_ev(), _ev(), _ev()] for _ in range(steps)]
+    sampler = ClockSampler(sampler_gpu) if sampler_gpu is not None else None
+    if sampler:
+        sampler.__enter__()
+    _barrier(ws)
+    torch.cuda.synchronize()
+    start, end = _ev(), _ev()
+    t0 = time.time()
+    start.record()
+    for i in range(steps):
+        step(evs[i])
+    end.record()
+    torch.cuda.synchronize()
+    t1 = time.time()
+    _barrier(ws)
+    if sampler:
+        sampler.mark(t0, t1)
+        sampler.__exit__()
+    assert fa.fa_last_device_error() == fa.FA_OK
+    total_ms = _max_over_ranks(start.elapsed_time(end), ws)
+    fwd_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    bwd_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    return {"total_ms": total_ms, "fwd_ms": _max_over_ranks(fwd_ms, ws),
+            "bwd_ms": _max_over_ranks(bwd_ms, ws), "clocks": sampler.summary() if sampler else None,
+            "launches_per_step": 3}
+
+
+def run_e2e(fa, B, H, N, d, causal, steps, warmup, ws, seed):
+    """Same step through the public API from pinned host buffers: H2D of q, k,
+    v, dO, then fa_fwd + fa_bwd, then D2H of dQ, dK, dV, all inside the timing."""
+    xd = synth.attention_inputs(B, H, N, d, seed, device="cuda")
+    host = {n: t.cpu().pin_memory() for n, t in xd.items()}
+    dev = {n: torch.empty_like(t) for n, t in xd.items()}
+    del xd
+    o = torch.empty_like(dev["q"])
+    lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    dq, dk, dv = (torch.empty((B, H, N, d), dtype=torch.float32, device="cuda") for _ in range(3))
+    wsp = torch.empty(fa.fa_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device="cuda")
+    outs = [torch.empty((B, H, N, d), dtype=torch.float32).pin_memory() for _ in range(3)]
+
+    def step():
+        for n in ("q", "k", "v", "do"):
+            dev[n].copy_(host[n], non_blocking=True)
+        fa.fa_fwd(dev["q"], dev["k"], dev["v"], causal=causal, o=o, lse=lse)
+        fa.fa_bwd(dev["q"], dev["k"], dev["v"], o, lse, dev["do"], causal=causal, dq=dq, dk=dk,
+                  dv=dv, workspace=wsp)
+        for hbuf, t in zip(outs, (dq, dk, dv)):
+            hbuf.copy_(t, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    _barrier(ws)
+    torch.cuda.synchronize()
+    start, end = _ev(), _ev()
+    start.record()
+    for _ in range(steps):
+        step()
+    end.record()
+    torch.cuda.synchronize()
+    _barrier(ws)
+    ms = _max_over_ranks(start.elapsed_time(end), ws) / steps
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+    return ms, h2d, d2h
+
+
+def run_decode(fa, steps, warmup, seed=1004):
+    lay = synth.paged_decode_layout(64, 16, 512, 32768, seed)
+    q, kc, vc = synth.paged_decode_tensors(64, 32, 8, 128, 16, lay["num_phys"], seed,
+                                           device="cuda")
+    tab = torch.from_numpy(lay["block_table"]).cuda()
+    lens = torch.from_numpy(lay["context_lens"]).cuda()
+    o = torch.empty_like(q)
+    lse = torch.empty((64, 32), dtype=torch.float32, device="cuda")
+    wsp = torch.empty(fa.paged_attn_decode_workspace_bytes(64, 32, 128, 32768), dtype=torch.uint8,
+                      device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")   # > L2: flush between calls
+
+    def call():
+        fa.paged_attn_decode(q, kc, vc, tab, lens, 32768, o=o, lse=lse, workspace=wsp)
+
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(steps):
+        flush.zero_()
+        a, b = _ev(), _ev()
+        a.record()
+        call()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    assert fa.fa_last_device_error() == fa.FA_OK
+    ms = float(np.mean(ts))
+    lens64 = lay["context_lens"].astype(np.int64)
+    slab = 16 * 128 * 2                     # one (block, kv head) K or V slab
+    logical = int(((lens64 + 15) // 16).sum()) * 8 * slab * 2
+    unique = lay["num_phys"] * 8 * slab * 2
+    small = 64 * 32 * 128 * 2 * 2 + tab.numel() * 4
+    return {"ms": ms, "unique_bytes": unique + small, "logical_bytes": logical + small,
+            "shared_fraction": lay["shared_blocks"] / lay["total_blocks"]}
+
+
+def run_fp8(fa, steps, warmup, seed=1003):
+    B, H, N, d = 4, 16, 4096, 128
+    x = synth.fp8_inputs(B, H, N, d, seed, device="cuda")
+    R = torch.from_numpy(synth.orthogonal_matrix(d, 2003)).float().cuda()
+    try:
+        q8, k8, v8, sq, sk, sv = fa.fa_fp8_prepare(x["q"], x["k"], x["v"], R)
+        o, lse = fa.fa_fwd_fp8(q8, k8, v8, sq, sk, sv, causal=False)
+    except fa.FAError as e:
+        return {"unavailable": str(e)}
+    for _ in range(warmup):
+        fa.fa_fwd_fp8(q8, k8, v8, sq, sk, sv, causal=False, o=o, lse=lse)
+    torch.cuda.synchronize()
+    a, b = _ev(), _ev()
+    a.record()
+    for _ in range(steps):
+        fa.fa_fwd_fp8(q8, k8, v8, sq, sk, sv, causal=False, o=o, lse=lse)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    return {"ms": ms, "flops": attn_flops(B, H, N, d, False)}
+
+
+# ---------------------------------------------------------- CPU baseline ---
+def _cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else _cores()
+    except Exception:
+        return _cores()
+
+
+def oracle_sample(N, seed=1002):
+    """The float64 oracle (as it stands) on one head of the long-sequence
+    workload truncated to N positions: forward + backward. Returns (s, flops)."""
+    import oracle
+    x = synth.attention_inputs(1, 1, N, 128, seed, device="cpu")
+    q, k, v, do = (synth.to_f64(x[n])[0, 0] for n in ("q", "k", "v", "do"))
+    t0 = time.perf_counter()
+    o, lse = oracle.attention_fwd(q, k, v, causal=True)
+    oracle.attention_bwd(q, k, v, do, causal=True, o=o)
+    dt = time.perf_counter() - t0
+    return dt, attn_flops(1, 1, N, 128, True) + attn_flops(1, 1, N, 128, True, bwd=True)
+
+
+def cpu_baseline(N=16384):
+    dt, fl = oracle_sample(N)
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"float64 oracle fwd+bwd of 1 of 16 heads (B=1, N={N}, d=128, causal), "
+                      f"{dt:.1f} s on the host"}
+
+
+def run_reference(args, ws, rank):
+    """--impl reference: the oracle on the host cores, same metric and config."""
+    if rank != 0:
+        return
+    N = 4096
+    for _ in range(args.warmup):
+        oracle_sample(N)
+    t = []
+    fl = 0.0
+    for _ in range(args.steps):
+        dt, fl = oracle_sample(N)
+        t.append(dt)
+    ms = 1e3 * float(np.mean(t))
+    val = fl / (ms / 1e3) / 1e12
+    cores = _blas_threads()
+    sample = (f"each step: float64 oracle fwd+bwd of one head of the workload truncated to "
+              f"N={N} (B=1, d=128, causal)")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": _config(),
+        "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+def _config():
+    w = WORKLOAD
+    return {"workload": f"long-sequence attention fwd+bwd: B={w['B']} H={w['H']} N={w['N']} "
+                        f"d={w['d']} causal bf16",
+            "global_batch": w["B"], "seq_len": w["N"], "heads": w["H"], "head_dim": w["d"],
+            "causal": w["causal"], "parallelism": "replicas (independent heads per GPU)",
+            "l2": "operands larger than L2 (335 MB bf16 + 403 MB fp32), no flush"}
+
+
+def run_case(fa, case, shape, causal, steps, warmup):
+    """One operation at one size, for profilers: warmup + steps launches."""
+    B, H, N, d = shape
+    x = synth.attention_inputs(B, H, N, d, 1002, device="cuda", with_dout=case == "bwd")
+    if case == "fwd":
+        o, lse = fa.fa_fwd(x["q"], x["k"], x["v"], causal=causal)
+
+        def op():
+            fa.fa_fwd(x["q"], x["k"], x["v"], causal=causal, o=o, lse=lse)
+    elif case == "bwd":
+        o, lse = fa.fa_fwd(x["q"], x["k"], x["v"], causal=causal)
+        g = [torch.empty((B, H, N, d), device="cuda") for _ in range(3)]
+        wsp = torch.empty(fa.fa_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device="cuda")
+
+        def op():
+            fa.fa_bwd(x["q"], x["k"], x["v"], o, lse, x["do"], causal=causal, dq=g[0], dk=g[1],
+                      dv=g[2], workspace=wsp)
+    elif case == "fp8":
+        R = torch.from_numpy(synth.orthogonal_matrix(d, 2003)).float().cuda()
+        q8, k8, v8, sq, sk, sv = fa.fa_fp8_prepare(x["q"], x["k"], x["v"], R)
+        o, lse = fa.fa_fwd_fp8(q8, k8, v8, sq, sk, sv, causal=causal)
+
+        def op():
+            fa.fa_fwd_fp8(q8, k8, v8, sq, sk, sv, causal=causal, o=o, lse=lse)
+    elif case == "decode":
+        S = B          # sequences; contexts U[512, N]
+        lay = synth.paged_decode_layout(S, 16, 512, N, 1004)
+        q, kc, vc = synth.paged_decode_tensors(S, 32, 8, 128, 16, lay["num_phys"], 1004,
+                                               device="cuda")
+        tab = torch.from_numpy(lay["block_table"]).cuda()
+        lens = torch.from_numpy(lay["context_lens"]).cuda()
+
+        def op():
+            fa.paged_attn_decode(q, kc, vc, tab, lens, N)
+    else:
+        raise SystemExit(f"unknown case {case}")
+    for _ in range(warmup):
+        op()
+    torch.cuda.synchronize()
+    a, b = _ev(), _ev()
+    a.record()
+    for _ in range(steps):
+        op()
+    b.record()
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_error() == fa.FA_OK
+    print(json.dumps({"case": case, "shape": shape, "causal": causal,
+                      "ms": a.elapsed_time(b) / max(steps, 1)}))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-parts", action="store_true", help="headline only")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", default="headline",
+                    help="headline (default) or one op for profilers: fwd, bwd, fp8, decode")
+    ap.add_argument("--shape", default="1,16,16384,128",
+                    help="B,H,N,d for --case (decode: sequences,_,max context,_)")
+    ap.add_argument("--causal", type=int, default=1)
+    args = ap.parse_args()
+    if args.case != "headline":
+        import exact_attention_102_b200 as fa
+        torch.cuda.set_device(0)
+        run_case(fa, args.case, [int(v) for v in args.shape.split(",")], bool(args.causal),
+                 args.steps, args.warmup)
+        return
+    if args.warmup < 3:
+        args.warmup = 3
+
+    if args.impl == "reference":
+        ws = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, ws, rank)
+        return
+
+    import exact_attention_102_b200 as fa
+    ws, rank, local = _dist_init()
+    peaks = _peaks()
+    w = WORKLOAD
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
+        if "CUDA_VISIBLE_DEVICES" in os.environ else local
+    r = run_fwd_bwd(fa, w["B"], w["H"], w["N"], w["d"], w["causal"], args.steps, args.warmup, ws,
+                    seed=1002, sampler_gpu=gpu_index)
+    f_fwd = attn_flops(w["B"], w["H"], w["N"], w["d"], w["causal"])
+    f_bwd = attn_flops(w["B"], w["H"], w["N"], w["d"], w["causal"], bwd=True)
+    ms = r["total_ms"] / args.steps
+    value = ws * (f_fwd + f_bwd) / (ms / 1e3) / 1e12
+    e2e_ms, h2d, d2h = run_e2e(fa, w["B"], w["H"], w["N"], w["d"], w["causal"],
+                               max(3, args.steps // 4), 2, ws, seed=1002)
+    e2e_val = ws * (f_fwd + f_bwd) / (e2e_ms / 1e3) / 1e12
+
+    peak_t = peaks["bf16_tflops"]
+    bwd_t = f_bwd / (r["bwd_ms"] / 1e3) / 1e12
+    fwd_t = f_fwd / (r["fwd_ms"] / 1e3) / 1e12
+    dom = "bwd" if r["bwd_ms"] >= r["fwd_ms"] else "fwd"
+    ach = bwd_t if dom == "bwd" else fwd_t
+    roof = {"bound": "tensor", "kernel": "fa_bwd (pre + main)" if dom == "bwd" else "fa_fwd",
+            "achieved": ach, "peak": peak_t, "unit": "TFLOP/s", "frac": ach / peak_t,
+            "peak_source": f"{peaks['source']} bf16 burst", "traffic": None}
+
+    parts = {}
+    if not args.no_parts:
+        parts["fwd"] = {"ms": r["fwd_ms"], "TFLOP/s": fwd_t, "frac_of_bf16_peak": fwd_t / peak_t}
+        parts["bwd"] = {"ms": r["bwd_ms"], "TFLOP/s": bwd_t, "frac_of_bf16_peak": bwd_t / peak_t}
+        c1 = run_fwd_bwd(fa, 8, 12, 1024, 64, True, args.steps, args.warmup, 1, seed=1001)
+        f1 = attn_flops(8, 12, 1024, 64, True) + attn_flops(8, 12, 1024, 64, True, bwd=True)
+        parts["gpt2_small_fwd_bwd"] = {
+            "ms": c1["total_ms"] / args.steps,
+            "TFLOP/s": f1 / (c1["total_ms"] / args.steps / 1e3) / 1e12,
+            "fwd_ms": c1["fwd_ms"], "bwd_ms": c1["bwd_ms"]}
+        dec = run_decode(fa, args.steps, args.warmup)
+        gbs = dec["unique_bytes"] / (dec["ms"] / 1e3) / 1e9
+        parts["paged_decode"] = {
+            "ms": dec["ms"], "GB/s_unique": gbs,
+            "GB/s_logical": dec["logical_bytes"] / (dec["ms"] / 1e3) / 1e9,
+            "shared_block_fraction": dec["shared_fraction"],
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "traffic": None}}
+        f8 = run_fp8(fa, args.steps, args.warmup)
+        if "ms" in f8:
+            t8 = f8["flops"] / (f8["ms"] / 1e3) / 1e12
+            p8 = 2.0 * peak_t
+            parts["fp8_fwd"] = {"ms": f8["ms"], "TFLOP/s": t8, "roofline": {
+                "bound": "tensor", "achieved": t8, "peak": p8, "unit": "TFLOP/s", "frac": t8 / p8,
+                "peak_source": "measured bf16 burst x 2 (nominal fp8/bf16 ratio)"}}
+        else:
+            parts["fp8_fwd"] = f8
+
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        cpu = cpu_baseline()
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": _config(),
+            "roofline": roof, "cpu_baseline": cpu,
+            "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": r["launches_per_step"] * args.steps,
+            "clocks": r["clocks"], "parts": parts,
+        }
+        print(json.dumps(line))
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -134,7 +134,8 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   if (B < 1 || H < 1 || N < 1 || d < 1) return 0;
   const size_t rows = static_cast<size_t>(B) * H * ((static_cast<size_t>(N) + 127) / 128 * 128);
-  return 2 * round256(rows * sizeof(float));
+  const size_t elems = static_cast<size_t>(B) * H * N * d;
+  return 2 * round256(rows * sizeof(float)) + 4 * round256(elems * 2);
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -151,13 +152,26 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   uint32_t* err = error_word_ptr();
   if (err == nullptr) return FA_ERR_LAUNCH;
   const int bh = B * H;
+  const size_t n_pad = (static_cast<size_t>(N) + 127) / 128 * 128;
+  const size_t prow = static_cast<size_t>(bh) * n_pad;
+  const size_t tsz = round256(static_cast<size_t>(bh) * N * d * 2);
+  char* w = static_cast<char*>(workspace);
+  char* w16 = w + 2 * round256(prow * sizeof(float));
+  void* q16 = w16;
+  void* k16 = w16 + tsz;
+  void* v16 = w16 + 2 * tsz;
+  void* do16 = w16 + 3 * tsz;
   CUtensorMap tq, tk, tv, tdo;
-  if (!make_map(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, bh, 64, 128) ||
-      !make_map(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, bh, 64, 128) ||
-      !make_map(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, bh, 64, 128) ||
-      !make_map(&tdo, dout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, bh, 64, 128))
+  if (!make_map(&tq, q16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, 128) ||
+      !make_map(&tk, k16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, 128) ||
+      !make_map(&tv, v16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, 128) ||
+      !make_map(&tdo, do16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, 128))
     return FA_ERR_LAUNCH;
   fa::BwdArgs a;
+  a.q16 = q16;
+  a.k16 = k16;
+  a.v16 = v16;
+  a.do16 = do16;
   a.q = q;
   a.k = k;
   a.v = v;
@@ -167,8 +181,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   a.dq = dq;
   a.dk = dk;
   a.dv = dv;
-  a.n_pad = (N + 127) / 128 * 128;
-  const size_t prow = static_cast<size_t>(B) * H * a.n_pad;
+  a.n_pad = static_cast<int>(n_pad);
   a.delta = static_cast<float*>(workspace);
   a.lse_log2 = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                         round256(prow * sizeof(float)));
@@ -310,7 +323,9 @@ fa_status fa_last_device_error(void* stream) {
   const uint32_t zero = 0;
   if (cudaMemcpyToSymbol(g_fa_error_word, &zero, sizeof(zero)) != cudaSuccess)
     return FA_ERR_LAUNCH;
-  return (word & fa::kErrBadIndex) ? FA_ERR_INVALID_ARG : FA_ERR_TIMEOUT;
+  if (word & fa::kErrBadIndex) return FA_ERR_INVALID_ARG;
+  if (word & fa::kErrRange) return FA_ERR_UNSUPPORTED;
+  return FA_ERR_TIMEOUT;
 }
 
 fa_status fa_debug_wait_timeout(unsigned int timeout_us, void* stream) {

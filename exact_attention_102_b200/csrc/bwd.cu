@@ -15,6 +15,13 @@
 //   dV_j += P^T dO_i,  dP = dO_i V_j^T,  dS = P o (dP - D_i)
 //   dK_j += scale dS^T Q_i,  dQ_i += scale dS K_j   (fp32 reductions to HBM)
 //
+// Precision: the tensor-core operands of the backward are fp16. The bf16
+// inputs convert exactly (bf16 values within fp16's range are fp16 values), and
+// P and dS, which are rounded to the operand type, keep 3 more mantissa bits
+// than bf16 would give them. dS is stored scaled by 2^-8 (undone in the dQ and
+// dK epilogues) so that |dS| up to 2^24 stays finite. Inputs with |x| >= 65504
+// do not fit fp16: the conversion flags them (FA_ERR_UNSUPPORTED).
+//
 // B200 mapping (one CTA per (batch*head, key block), 384 threads):
 //   warp 0       TMA producer: K_j, V_j once; Q_i and dO_i per row block
 //                through two-stage rings.
@@ -75,10 +82,36 @@ enum : uint32_t {
   kSiteDSF = 0x3c, kSiteDQ = 0x3d, kSiteEnd = 0x3e, kSiteDrain = 0x3f
 };
 
+constexpr float kDsScale = 1.0f / 256.0f;   // dS is stored as dS * 2^-8
+
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
                "f"(c), "f"(d)
                : "memory");
+}
+
+// ------------------------------------------------------- fp16 conversion
+// q, k, v, dout (bf16) -> fp16 copies; 8 elements per thread per step.
+__global__ void __launch_bounds__(256) bwd_convert_kernel(BwdArgs a, long long n8) {
+  bool bad = false;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < 4 * n8;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int t = static_cast<int>(i / n8);
+    const long long j = i - t * n8;
+    const void* sp = t == 0 ? a.q : t == 1 ? a.k : t == 2 ? a.v : a.dout;
+    void* dp = t == 0 ? a.q16 : t == 1 ? a.k16 : t == 2 ? a.v16 : a.do16;
+    const uint4 u = static_cast<const uint4*>(sp)[j];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xffff0000u);
+      bad |= !(fabsf(lo) < 65504.f) || !(fabsf(hi) < 65504.f);
+      o[e] = pack_f16x2(lo, hi);
+    }
+    static_cast<uint4*>(dp)[j] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  if (bad) atomicCAS(a.err, 0u, kErrRange + 1);
 }
 
 // ---------------------------------------------------------------- pre pass
@@ -223,9 +256,10 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA issue
     if (lane == 0) {
-      constexpr uint32_t idSS = idesc_f16(128, C::BQ, 1, 0, 0);   // S^T, dP^T
-      constexpr uint32_t idKM = idesc_f16(128, D, 1, 0, 1);        // dV (A tmem), dK: B MN-major
-      constexpr uint32_t idQ = idesc_f16(128, D, 1, 1, 1);         // dQ: A and B MN-major
+      // fp16 x fp16 -> fp32 (format 0 = f16)
+      constexpr uint32_t idSS = idesc_f16(128, C::BQ, 0, 0, 0);   // S^T, dP^T
+      constexpr uint32_t idKM = idesc_f16(128, D, 0, 0, 1);        // dV (A tmem), dK: B MN-major
+      constexpr uint32_t idQ = idesc_f16(128, D, 0, 1, 1);         // dQ: A and B MN-major
       const uint32_t kbase = base + C::K_OFF, vbase = base + C::V_OFF, dsb = base + C::DS_OFF;
       bool ok = mbar_wait(bar(C::B_KV), 0, a.err, kSiteKV, abort_flag);
       // S^T(it) = K Q_it^T ; dP^T(it) = V dO_it^T
@@ -349,8 +383,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             p[u] = ex2_approx(fmaf(__uint_as_float(sr[e + u]), sl2, -L[u]));
             if (need_mask && ((a.causal && key > q0 + h * 32 + e + u) || key >= a.N)) p[u] = 0.f;
           }
-          PK((h * 32 + e) / 2) = pack_bf16x2(p[0], p[1]);
-          PK((h * 32 + e) / 2 + 1) = pack_bf16x2(p[2], p[3]);
+          PK((h * 32 + e) / 2) = pack_f16x2(p[0], p[1]);
+          PK((h * 32 + e) / 2 + 1) = pack_f16x2(p[2], p[3]);
         }
       }
       tmem_st32(st_addr, pk0);
@@ -381,11 +415,11 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const uint32_t pp = PK((h * 32 + e + u) >> 1);
-            const float pv = __uint_as_float(((e + u) & 1) ? (pp & 0xffff0000u) : (pp << 16));
-            ds[u] = pv * (__uint_as_float(dr[e + u]) - Dv[u]);
+            const float pv = ((e + u) & 1) ? f16_hi(pp) : f16_lo(pp);
+            ds[u] = (pv * kDsScale) * (__uint_as_float(dr[e + u]) - Dv[u]);
           }
-          w[e / 2] = pack_bf16x2(ds[0], ds[1]);
-          w[e / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+          w[e / 2] = pack_f16x2(ds[0], ds[1]);
+          w[e / 2 + 1] = pack_f16x2(ds[2], ds[3]);
         }
         // queries h*32 .. h*32+31 = chunk (h/2), 16-byte units (h%2)*4 .. +3 of the
         // 128-byte row, XOR-swizzled with (key row % 8) like a TMA SWIZZLE_128B tile
@@ -412,7 +446,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int which = 0; which < 2; ++which) {
           const uint32_t src = tmem + lane_off + (which ? C::COL_DK : C::COL_DV);
           float* dst = (which ? a.dk : a.dv) + orow;
-          const float mul = which ? a.scale : 1.f;
+          const float mul = which ? a.scale / kDsScale : 1.f;
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t v[32];
@@ -436,7 +470,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int r = (warp & 3) * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t src = tmem + lane_off + C::COL_DPT;
-    const float sc = a.scale;
+    const float sc = a.scale / kDsScale;
     for (int it = 0; it < n_it; ++it) {
       const int q = (i0 + it) * C::BQ + r;
       if (!__all_sync(0xffffffffu, mbar_wait(bar(C::B_DQ), it & 1, a.err, kSiteDQ, abort_flag)))
@@ -488,6 +522,10 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   const long long rows = static_cast<long long>(a.B) * a.H * a.n_pad;
   const long long want = (rows + 7) / 8;
   const int pre_blocks = static_cast<int>(want < 148 * 16 ? want : 148 * 16);
+  const long long n8 = static_cast<long long>(a.B) * a.H * a.N * D / 8;
+  const long long cwant = (4 * n8 + 255) / 256;
+  const int cblocks = static_cast<int>(cwant < 148 * 8 ? cwant : 148 * 8);
+  bwd_convert_kernel<<<cblocks, 256, 0, stream>>>(a, n8);
   bwd_pre_kernel<D><<<pre_blocks, 256, 0, stream>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

@@ -1,11 +1,444 @@
-// fp8.cu — FP8 prepare + forward (placeholder until the sm_100a kernels land).
+// fp8.cu — FP8 (e4m3) attention forward with per-block scales and the
+// random-orthogonal pre-rotation of Q and K, for sm_100a.
+//
+// "FlashAttention系列优化" (johneyzheng.top), FlashAttentionV3, FP8: block
+// quantisation (one scale per block of Q, K, V) and incoherent processing
+// (multiply Q and K by one random orthogonal matrix: outliers spread over all
+// coordinates while Q K^T is unchanged). 91haoming.cn repost, "FP8 低精度計算":
+// per-block rather than per-tensor scales.
+//
+// fp8_prep_kernel   one CTA per (tensor, batch*head, 64-row block): rows of Q
+//                   or K times R (fp32, CUDA cores), V as is; amax over the
+//                   64 x d block, scale = amax / 448 (1 for an all-zero block),
+//                   x8 = e4m3(x / scale) with round-to-nearest-even and
+//                   saturation.
+// fwd_fp8_kernel    the bf16 forward's pipeline (TMA producer warp, one MMA
+//                   thread, two softmax warpgroups ping-ponging two 128-row Q
+//                   tiles, S and O in TMEM) with kind::f8f6f4 MMAs:
+//                     S = q8 k8^T (fp32 accumulate); the true score is
+//                     S * sq(row block) * sk(key block) * softmax scale;
+//                     P' = P * sv(key block) / C rounded to e4m3 feeds the
+//                     P.V product from TMEM, C = max over the head's V scales
+//                     (so P' <= 256 < 448 never saturates);
+//                     O = C * (sum P' v8) / l with l the fp32 sum of P.
+//                   V stays MN-major in shared memory (tcgen05 reads e4m3
+//                   operands in either major order), so no transpose is needed.
 #include "prim.cuh"
 #include "kernels.h"
 
 namespace fa {
-cudaError_t launch_fp8_prepare(const Fp8PrepArgs&, cudaStream_t) { return cudaErrorNotSupported; }
-cudaError_t launch_fwd_fp8(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                           const Fp8FwdArgs&, cudaStream_t) {
-  return cudaErrorNotSupported;
+
+namespace {
+
+constexpr int kD = 128;
+constexpr float kE4m3Max = 448.f;
+
+// four floats -> four e4m3 bytes (byte i = element i), RNE, saturating
+__device__ __forceinline__ uint32_t pack_e4m3x4(float e0, float e1, float e2, float e3) {
+  uint32_t out;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(out)
+      : "f"(e0), "f"(e1), "f"(e2), "f"(e3));
+  return out;
 }
+
+// ------------------------------------------------------------------ prep --
+constexpr int kPrepThreads = 256;
+constexpr int kPrepSmem = 64 * kD * 4 + kD * kD * 4 + 64;   // x block, R, reduction
+
+__global__ void __launch_bounds__(kPrepThreads) fp8_prep_kernel(Fp8PrepArgs a) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  float* xs = reinterpret_cast<float*>(smem);                 // [64][128]
+  float* Rs = xs + 64 * kD;                                   // [128][128]
+  float* red = Rs + kD * kD;                                  // [8]
+  const int blk = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
+  const int nblk = (a.N + 63) / 64;
+  const int r0 = blk * 64;
+  const int rows = min(64, a.N - r0);
+  const int tid = threadIdx.x;
+  const __nv_bfloat16* src =
+      static_cast<const __nv_bfloat16*>(which == 0 ? a.q : which == 1 ? a.k : a.v) +
+      (static_cast<size_t>(bh) * a.N + r0) * kD;
+  uint8_t* dst = (which == 0 ? a.q8 : which == 1 ? a.k8 : a.v8) +
+                 (static_cast<size_t>(bh) * a.N + r0) * kD;
+  float* sc = (which == 0 ? a.sq : which == 1 ? a.sk : a.sv) + static_cast<size_t>(bh) * nblk + blk;
+
+  for (int i = tid; i < 64 * kD / 2; i += kPrepThreads) {
+    const int r = (2 * i) / kD;
+    float2 v = make_float2(0.f, 0.f);
+    if (r < rows) v = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(src)[i]);
+    xs[2 * i] = v.x;
+    xs[2 * i + 1] = v.y;
+  }
+  if (which < 2)
+    for (int i = tid; i < kD * kD; i += kPrepThreads) Rs[i] = a.R[i];
+  __syncthreads();
+
+  // y[r][c] = sum_e x[r][e] R[e][c]: thread -> column c, rows rb .. rb+31
+  const int c = tid & (kD - 1);
+  const int rb = (tid >> 7) * 32;
+  float y[32];
+  if (which < 2) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) y[i] = 0.f;
+    for (int e = 0; e < kD; ++e) {
+      const float rv = Rs[e * kD + c];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) y[i] = fmaf(xs[(rb + i) * kD + e], rv, y[i]);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) y[i] = xs[(rb + i) * kD + c];
+  }
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+    if (rb + i < rows) amax = fmaxf(amax, fabsf(y[i]));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  __syncthreads();                               // everyone is done reading xs
+  if ((tid & 31) == 0) red[tid >> 5] = amax;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) xs[(rb + i) * kD + c] = y[i];
+  __syncthreads();
+  float m = red[0];
+#pragma unroll
+  for (int w = 1; w < kPrepThreads / 32; ++w) m = fmaxf(m, red[w]);
+  const float scale = m > 0.f ? m / kE4m3Max : 1.f;
+  const float inv = 1.f / scale;
+  if (tid == 0) *sc = scale;
+  // quantise: 4 consecutive elements per thread-step, coalesced 4-byte stores
+  for (int i = tid; i < rows * kD / 4; i += kPrepThreads) {
+    const float* p = xs + 4 * i;
+    reinterpret_cast<uint32_t*>(dst)[i] =
+        pack_e4m3x4(p[0] * inv, p[1] * inv, p[2] * inv, p[3] * inv);
+  }
+}
+
+// --------------------------------------------------------------- forward --
+struct F8 {
+  static constexpr int BM = 128, BN = 128;
+  static constexpr int TILE = 128 * kD;         // bytes of a 128-row e4m3 tile (one 128 B chunk)
+  static constexpr int NSTAGE = 8;
+  static constexpr int Q_OFF = 0;
+  static constexpr int RING_OFF = 2 * TILE;
+  static constexpr int BAR_OFF = RING_OFF + NSTAGE * TILE;
+  static constexpr int B_Q = 0, B_KVF = 1, B_KVE = 1 + NSTAGE, B_S = 1 + 2 * NSTAGE;
+  static constexpr int B_P = B_S + 2, B_O = B_P + 2, B_DRAIN = B_O + 2, NBAR = B_DRAIN + 1;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;   // tmem slot, abort flag, C
+  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int THREADS = 384;
+  static __device__ __forceinline__ uint32_t s_col(int t) { return 128u * t; }
+  static __device__ __forceinline__ uint32_t o_col(int t) { return 256u + 128u * t; }
+};
+
+constexpr float kRescaleThreshold = 8.0f;
+enum : uint32_t {
+  kSQ = 0x41, kSKE = 0x42, kSKF = 0x43, kSS = 0x44, kSP = 0x45, kSO = 0x46, kSEpi = 0x47,
+  kSDrain = 0x48
+};
+
+__global__ void __launch_bounds__(384, 1)
+fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, Fp8FwdArgs a) {
+  using C = F8;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw_addr);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int BH = a.B * a.H;
+  const int pair = a.n_pairs - 1 - static_cast<int>(blockIdx.x) / BH;
+  const int bh = static_cast<int>(blockIdx.x) % BH;
+  const int nkb = (a.N + C::BN - 1) / C::BN;
+  const int nsb = (a.N + 63) / 64;                     // scale blocks per head
+  int q0[2], nkb_t[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    q0[t] = (pair * 2 + t) * C::BM;
+    nkb_t[t] = (q0[t] >= a.N) ? 0 : (a.causal ? min(nkb, pair * 2 + t + 1) : nkb);
+  }
+  const int nkb_cta = max(nkb_t[0], nkb_t[1]);
+  auto bar = [&](int i) -> uint32_t { return base + C::BAR_OFF + 8 * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
+  float* cmax = reinterpret_cast<float*>(smem + C::MISC_OFF + 8);
+  const float* svh = a.sv + static_cast<size_t>(bh) * nsb;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(C::B_Q), 1);
+    for (int s = 0; s < C::NSTAGE; ++s) {
+      mbar_init(bar(C::B_KVF + s), 1);
+      mbar_init(bar(C::B_KVE + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(C::B_S + t), 1);
+      mbar_init(bar(C::B_P + t), 128);
+      mbar_init(bar(C::B_O + t), 1);
+    }
+    mbar_init(bar(C::B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {  // C = max of the head's V block scales
+    float m = 0.f;
+    for (int i = lane; i < nsb; i += 32) m = fmaxf(m, svh[i]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if (lane == 0) *cmax = m > 0.f ? m : 1.f;
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      const int nq = (nkb_t[0] > 0) + (nkb_t[1] > 0);
+      mbar_arrive_expect_tx(bar(C::B_Q), nq * C::TILE);
+      for (int t = 0; t < 2; ++t)
+        if (nkb_t[t] > 0) tma_load_3d(base + C::Q_OFF + t * C::TILE, &tmQ, bar(C::B_Q), 0, q0[t], bh);
+      int it = 0;
+      bool ok = true;
+      for (int j = 0; j < nkb_cta && ok; ++j) {
+        for (int w = 0; w < 2 && ok; ++w, ++it) {
+          const int s = it % C::NSTAGE;
+          ok = mbar_wait(bar(C::B_KVE + s), ((it / C::NSTAGE) & 1) ^ 1, a.err, kSKE, abort_flag);
+          if (!ok) break;
+          mbar_arrive_expect_tx(bar(C::B_KVF + s), C::TILE);
+          tma_load_3d(base + C::RING_OFF + s * C::TILE, w == 0 ? &tmK : &tmV, bar(C::B_KVF + s), 0,
+                      j * C::BN, bh);
+        }
+      }
+      const int issued = it;
+      for (int k = max(0, issued - C::NSTAGE); k < issued; ++k)
+        mbar_wait(bar(C::B_KVF + k % C::NSTAGE), (k / C::NSTAGE) & 1, a.err, kSDrain, nullptr,
+                  200000000ull);
+      if (nq) mbar_wait(bar(C::B_Q), 0, a.err, kSDrain, nullptr, 200000000ull);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_e4m3(128, C::BN, 0, 0);
+      constexpr uint32_t idPV = idesc_e4m3(128, kD, 0, 1);
+      int it = 0;
+      int npv[2] = {0, 0};
+      bool ok = mbar_wait(bar(C::B_Q), 0, a.err, kSQ, abort_flag);
+      for (int j = 0; j < nkb_cta && ok; ++j) {
+        {
+          const int s = it % C::NSTAGE;
+          ok = mbar_wait(bar(C::B_KVF + s), (it / C::NSTAGE) & 1, a.err, kSKF, abort_flag);
+          if (!ok) break;
+          ++it;
+          tc_fence_after();
+          const uint32_t kb = base + C::RING_OFF + s * C::TILE;
+          for (int t = 0; t < 2; ++t) {
+            if (j >= nkb_t[t]) continue;
+            if (npv[t] > 0) {
+              ok = mbar_wait(bar(C::B_O + t), (npv[t] - 1) & 1, a.err, kSO, abort_flag);
+              if (!ok) break;
+              tc_fence_after();
+            }
+            const uint32_t qb = base + C::Q_OFF + t * C::TILE;
+#pragma unroll
+            for (int kk = 0; kk < kD / 32; ++kk)   // K = 32 e4m3 elements = 32 bytes per MMA
+              umma_f8_ss(tmem + C::s_col(t), smem_desc_sw128(qb + kk * 32, 16, 1024),
+                         smem_desc_sw128(kb + kk * 32, 16, 1024), idS, kk > 0);
+            umma_commit(bar(C::B_S + t));
+          }
+          if (!ok) break;
+          umma_commit(bar(C::B_KVE + s));
+        }
+        {
+          const int s = it % C::NSTAGE;
+          ok = mbar_wait(bar(C::B_KVF + s), (it / C::NSTAGE) & 1, a.err, kSKF, abort_flag);
+          if (!ok) break;
+          ++it;
+          const uint32_t vb = base + C::RING_OFF + s * C::TILE;
+          for (int t = 0; t < 2; ++t) {
+            if (j >= nkb_t[t]) continue;
+            ok = mbar_wait(bar(C::B_P + t), npv[t] & 1, a.err, kSP, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < C::BN / 32; ++kk)   // 32 keys = 8 TMEM columns of packed e4m3 P
+              umma_f8_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8,
+                         smem_desc_sw128(vb + kk * 4096, 16, 1024), idPV,
+                         (npv[t] > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(bar(C::B_O + t));
+            ++npv[t];
+          }
+          if (!ok) break;
+          umma_commit(bar(C::B_KVE + s));
+        }
+      }
+      umma_commit(bar(C::B_DRAIN));
+      mbar_wait(bar(C::B_DRAIN), 0, a.err, kSDrain, nullptr, 200000000ull);
+    }
+  } else if (warp >= 4) {
+    const int t = (warp - 4) >> 2;
+    const int r = (warp & 3) * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t s_addr = tmem + lane_off + C::s_col(t);
+    const uint32_t o_addr = tmem + lane_off + C::o_col(t);
+    const int row = q0[t] + r;
+    const int limit = a.causal ? min(row, a.N - 1) : a.N - 1;
+    const float* skh = a.sk + static_cast<size_t>(bh) * nsb;
+    const float inv_c = 1.f / *cmax;
+    // per-row factor: softmax scale * log2(e) * q block scale
+    const float rowf = a.scale_log2 * a.sq[static_cast<size_t>(bh) * nsb + min(row, a.N - 1) / 64];
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nkb_t[t]; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_S + t), j & 1, a.err, kSS, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, sr[c]);
+      tmem_ld_wait();
+      const int kbase = j * C::BN;
+      const int kb0 = kbase / 64;
+      const float f0 = rowf * skh[kb0];
+      const float f1 = (kb0 + 1 < nsb) ? rowf * skh[kb0 + 1] : 0.f;
+      const float pv0 = svh[kb0] * inv_c;
+      const float pv1 = (kb0 + 1 < nsb) ? svh[kb0 + 1] * inv_c : 0.f;
+#define SV(c) __uint_as_float(sr[(c) >> 5][(c)&31])
+      // scaled scores x_c = S_c * f(half) (exp2 units)
+#pragma unroll
+      for (int c = 0; c < 128; ++c)
+        sr[c >> 5][c & 31] = __float_as_uint(SV(c) * (c < 64 ? f0 : f1));
+      if (kbase + C::BN - 1 > limit) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (kbase + c > limit) sr[c >> 5][c & 31] = 0xff800000u;
+      }
+      float mx0 = SV(0), mx1 = SV(1), mx2 = SV(2), mx3 = SV(3);
+#pragma unroll
+      for (int c = 4; c < 128; c += 4) {
+        mx0 = fmaxf(mx0, SV(c));
+        mx1 = fmaxf(mx1, SV(c + 1));
+        mx2 = fmaxf(mx2, SV(c + 2));
+        mx3 = fmaxf(mx3, SV(c + 3));
+      }
+      const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+      float alpha = 1.f;
+      if (mx > m_run + kRescaleThreshold) {
+        alpha = ex2_approx(m_run - mx);
+        m_run = mx;
+      }
+      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+      float l0 = 0.f, l1 = 0.f;
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 128; c += 4) {
+        const float p0 = ex2_approx(SV(c) - m_use), p1 = ex2_approx(SV(c + 1) - m_use);
+        const float p2 = ex2_approx(SV(c + 2) - m_use), p3 = ex2_approx(SV(c + 3) - m_use);
+        l0 += p0 + p2;
+        l1 += p1 + p3;
+        const float w = c < 64 ? pv0 : pv1;
+        pk[c >> 2] = pack_e4m3x4(p0 * w, p1 * w, p2 * w, p3 * w);
+      }
+#undef SV
+      l_run = l_run * alpha + (l0 + l1);
+      tmem_st32(s_addr, pk);
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+        for (int c = 0; c < kD / 32; ++c) {
+          uint32_t orr[32];
+          tmem_ld32(o_addr + c * 32, orr);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+          tmem_st32(o_addr + c * 32, orr);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_P + t));
+    }
+    if (ok && nkb_t[t] > 0) {
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(bar(C::B_O + t), (nkb_t[t] - 1) & 1, a.err, kSEpi, abort_flag));
+      if (ok) {
+        tc_fence_after();
+        const float mul = *cmax / l_run;
+        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) + (static_cast<size_t>(bh) * a.N + row) * kD;
+#pragma unroll
+        for (int c = 0; c < kD / 32; ++c) {
+          uint32_t orr[32];
+          tmem_ld32(o_addr + c * 32, orr);
+          tmem_ld_wait();
+          if (row < a.N) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int b = 8 * e;
+              dst[e] = make_uint4(
+                  pack_bf16x2(__uint_as_float(orr[b + 0]) * mul, __uint_as_float(orr[b + 1]) * mul),
+                  pack_bf16x2(__uint_as_float(orr[b + 2]) * mul, __uint_as_float(orr[b + 3]) * mul),
+                  pack_bf16x2(__uint_as_float(orr[b + 4]) * mul, __uint_as_float(orr[b + 5]) * mul),
+                  pack_bf16x2(__uint_as_float(orr[b + 6]) * mul, __uint_as_float(orr[b + 7]) * mul));
+            }
+          }
+        }
+        if (row < a.N)
+          a.lse[static_cast<size_t>(bh) * a.N + row] = (m_run + log2f(l_run)) * 0.6931471805599453f;
+      }
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_fp8_prepare(const Fp8PrepArgs& a, cudaStream_t stream) {
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(fp8_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kPrepSmem);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  dim3 grid((a.N + 63) / 64, a.B * a.H, 3);
+  fp8_prep_kernel<<<grid, kPrepThreads, kPrepSmem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fwd_fp8(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           const Fp8FwdArgs& a, cudaStream_t stream) {
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(fwd_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         F8::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  fwd_fp8_kernel<<<a.n_pairs * a.B * a.H, F8::THREADS, F8::SMEM_BYTES, stream>>>(tq, tk, tv, a);
+  return cudaGetLastError();
+}
+
 }  // namespace fa

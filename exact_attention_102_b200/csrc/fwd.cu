@@ -238,7 +238,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     const int limit = a.causal ? min(row, a.N - 1) : a.N - 1;  // last visible key
     const float sl2 = a.scale_log2;
     float m_run = -INFINITY;
-    float l_run = 0.f;
+    float l_run = 0.f;    // sum of fp32 P
+    float lr_run = 0.f;   // sum of bf16-rounded P
     bool ok = true;
     for (int j = 0; j < nkb_t[t]; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_S + t), j & 1, a.err, kSiteS, abort_flag));
@@ -270,28 +271,36 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         m_run = mx;
       }
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      // l sums the bf16-rounded P that the P.V product uses, so numerator and
-      // denominator weigh every key identically
-      float l0 = 0.f, l1 = 0.f;
+      // Two row sums: l_run of the fp32 probabilities (for L = m + log l) and
+      // lr_run of the bf16-rounded P the P.V product consumes (for O = acc/l),
+      // so the normalisation weighs every key exactly as the numerator does.
+      float l0 = 0.f, l1 = 0.f, r0 = 0.f, r1 = 0.f;
       uint32_t pk0[32], pk1[32];
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
-        const uint32_t u = pack_bf16x2(ex2_approx(fmaf(SV(c), sl2, -m_use)),
-                                       ex2_approx(fmaf(SV(c + 1), sl2, -m_use)));
-        l0 += __uint_as_float(u << 16);
-        l1 += __uint_as_float(u & 0xffff0000u);
+        const float p0 = ex2_approx(fmaf(SV(c), sl2, -m_use));
+        const float p1 = ex2_approx(fmaf(SV(c + 1), sl2, -m_use));
+        const uint32_t u = pack_bf16x2(p0, p1);
+        l0 += p0;
+        l1 += p1;
+        r0 += __uint_as_float(u << 16);
+        r1 += __uint_as_float(u & 0xffff0000u);
         pk0[c >> 1] = u;
       }
 #pragma unroll
       for (int c = 64; c < 128; c += 2) {
-        const uint32_t u = pack_bf16x2(ex2_approx(fmaf(SV(c), sl2, -m_use)),
-                                       ex2_approx(fmaf(SV(c + 1), sl2, -m_use)));
-        l0 += __uint_as_float(u << 16);
-        l1 += __uint_as_float(u & 0xffff0000u);
+        const float p0 = ex2_approx(fmaf(SV(c), sl2, -m_use));
+        const float p1 = ex2_approx(fmaf(SV(c + 1), sl2, -m_use));
+        const uint32_t u = pack_bf16x2(p0, p1);
+        l0 += p0;
+        l1 += p1;
+        r0 += __uint_as_float(u << 16);
+        r1 += __uint_as_float(u & 0xffff0000u);
         pk1[(c - 64) >> 1] = u;
       }
 #undef SV
       l_run = l_run * alpha + (l0 + l1);
+      lr_run = lr_run * alpha + (r0 + r1);
       tmem_st32(s_addr, pk0);
       tmem_st32(s_addr + 32, pk1);
       // O rescale (PV of block j-1 has completed: S_t(j) was issued after it)
@@ -317,7 +326,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                       mbar_wait(bar(C::B_O + t), (nkb_t[t] - 1) & 1, a.err, kSiteEpi, abort_flag));
       if (ok) {
         tc_fence_after();
-        const float inv_l = 1.f / l_run;
+        const float inv_l = 1.f / lr_run;
         __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) +
                               (static_cast<size_t>(bh) * a.N + row) * D;
 #pragma unroll

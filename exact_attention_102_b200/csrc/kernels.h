@@ -33,6 +33,10 @@ struct BwdArgs {
   float* dv;          // fp32 BHND
   float* delta;       // fp32 [B][H][n_pad]: D_i = sum_c dO_ic O_ic (0 past N)
   float* lse_log2;    // fp32 [B][H][n_pad]: L_i * log2(e) (+inf past N)
+  void* q16;          // fp16 BHND copies of q, k, v, dout (the tensor-core operands)
+  void* k16;
+  void* v16;
+  void* do16;
   int B, H, N;
   int n_pad;          // N rounded up to a multiple of 128
   int causal;

@@ -14,6 +14,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace fa {
@@ -24,6 +25,7 @@ enum : uint32_t {
   kErrNone = 0,
   kErrTimeoutBase = 0x100,  // + wait site id
   kErrBadIndex = 0x10000,   // + site id: an input index was out of range
+  kErrRange = 0x20000,      // + site id: an input value outside a kernel's numeric range
 };
 
 // Default limit of one bounded wait, in nanoseconds of %globaltimer.
@@ -278,6 +280,17 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);  // .x = lo (low half), .y = hi
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ float f16_lo(uint32_t u) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(u & 0xffffu)));
+}
+__device__ __forceinline__ float f16_hi(uint32_t u) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(u >> 16)));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -80,8 +80,9 @@ FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, fl
 /*
  * Bytes of device workspace fa_bwd needs: two fp32 per-row vectors over N
  * rounded up to a multiple of 128 rows — the row statistic D and L * log2(e)
- * (padded with 0 / +inf) — each rounded up to 256 bytes. dq itself (fp32)
- * serves as the dQ accumulator.
+ * (padded with 0 / +inf) — plus fp16 copies of q, k, v and dout (the
+ * backward's tensor-core operands), each part rounded up to 256 bytes.
+ * dq itself (fp32) serves as the dQ accumulator.
  */
 FA_API size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
 
@@ -101,6 +102,10 @@ FA_API size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
  * ("Flash Attention 再学习": backward recomputes S and P from the stored
  * statistics; 91haoming.cn repost, "并行化改進": backward is parallel over
  * column blocks with atomic adds for the shared gradient.)
+ * Precision: the products run on fp16 tensor-core operands (exact copies of
+ * the bf16 inputs; P and dS rounded to fp16), accumulation is fp32. Inputs
+ * must satisfy |x| < 65504 (fp16 range); larger values are recorded and
+ * reported by fa_last_device_error() as FA_ERR_UNSUPPORTED.
  * Errors: as fa_fwd, plus FA_ERR_WORKSPACE when workspace is NULL or smaller
  * than required.
  */
@@ -189,7 +194,9 @@ FA_API fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8,
  * device error word of the current device. Returns FA_OK when nothing was
  * recorded since the last call, FA_ERR_TIMEOUT when a bounded wait gave up,
  * FA_ERR_INVALID_ARG when a kernel met an out-of-range index in its inputs
- * (a block-table entry), or FA_ERR_LAUNCH when the synchronisation failed.
+ * (a block-table entry), FA_ERR_UNSUPPORTED when an input value was outside a
+ * kernel's numeric range (fa_bwd: |x| >= 65504), or FA_ERR_LAUNCH when the
+ * synchronisation failed.
  */
 FA_API fa_status fa_last_device_error(void* stream);
 

@@ -31,6 +31,7 @@ from .attention import (  # noqa: F401
     attention_rows,
     paged_decode,
     combine_partials,
+    round_bf16,
     quantize_e4m3,
     dequantize_blocks_e4m3,
     fp8_block_quantize,

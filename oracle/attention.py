@@ -141,6 +141,25 @@ def attention_bwd(q, k, v, do, causal=False, scale=None, o=None):
             dd.reshape(lead + (n,)))
 
 
+def round_bf16(x):
+    """Round float64 values to the nearest bfloat16 value (ties to even).
+
+    bfloat16 keeps 8 significant bits (1 implicit + 7 stored) and float32's
+    exponent range. Used to model tensors that cross the library's interface
+    as bf16 (the forward's O, which the backward's D_i = sum_c dO_ic O_ic
+    reads). Pinned by torch's float32 -> bfloat16 cast.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    _, ex = np.frexp(np.where(a > 0, a, 1.0))       # a = f * 2^ex, f in [0.5, 1)
+    step = np.exp2(ex.astype(np.float64) - 8.0)     # spacing of 8-bit significands
+    r = a / step
+    rq = np.floor(r)
+    frac = r - rq
+    rq = rq + ((frac > 0.5) | ((frac == 0.5) & (np.mod(rq, 2.0) == 1.0)))
+    return np.where(a > 0, np.sign(x) * rq * step, x)
+
+
 def combine_partials(o_parts, lse_parts):
     """Merge attention partials computed over disjoint key sets.
 

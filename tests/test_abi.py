@@ -65,7 +65,7 @@ def test_bwd_rejects_bad_workspace_without_gpu():
     L = fa.lib()
     g = _p(0x10000)
     need = L.fa_bwd_workspace_bytes(2, 3, 100, 64)
-    assert need >= 2 * (2 * 3 * 128 * 4) and need % 256 == 0
+    assert need >= 2 * (2 * 3 * 128 * 4) + 4 * (2 * 3 * 100 * 64 * 2) and need % 256 == 0
     assert L.fa_bwd(*([g] * 9), _p(0), need, 2, 3, 100, 64, 1, None) == fa.FA_ERR_WORKSPACE
     assert L.fa_bwd(*([g] * 9), g, need - 1, 2, 3, 100, 64, 1, None) == fa.FA_ERR_WORKSPACE
     assert L.fa_bwd(*([g] * 8), _p(0), g, need, 2, 3, 100, 64, 1, None) == fa.FA_ERR_INVALID_ARG

@@ -360,3 +360,16 @@ def test_fp8_block_quantize_roundtrip():
     z = np.zeros((1, 64, 4))
     vz, sz = oracle.fp8_block_quantize(z)
     assert sz[0, 0] == 1.0 and np.all(vz == 0)
+
+
+def test_round_bf16_matches_torch_cast():
+    """Library routine: torch's float32 -> bfloat16 cast (RNE)."""
+    rng = np.random.default_rng(24)
+    x = np.concatenate([rng.standard_normal(50000) * s for s in (1e-30, 1e-3, 1, 7, 1e5)])
+    x = x.astype(np.float32).astype(np.float64)           # float32 inputs: one rounding only
+    ref = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(oracle.round_bf16(x), ref)
+    # worked values: 1 + 2^-8 is halfway between 1 and 1 + 2^-7 -> 1 (even);
+    # 1 + 3*2^-8 is halfway between 1 + 2^-7 and 1 + 2^-6 -> 1 + 2^-6 (even)
+    np.testing.assert_array_equal(oracle.round_bf16([1 + 2 ** -8, 1 + 3 * 2 ** -8, -3.0, 0.0]),
+                                  [1.0, 1 + 2 ** -6, -3.0, 0.0])
