@@ -18,11 +18,11 @@
 // Precision: the tensor-core operands of the backward are fp16. The bf16
 // inputs convert exactly (bf16 values within fp16's range are fp16 values), and
 // P and dS, which are rounded to the operand type, keep 3 more mantissa bits
-// than bf16 would give them. dS is stored scaled by 2^-8 (undone in the dQ and
-// dK epilogues) so that |dS| up to 2^24 stays finite. Inputs with |x| >= 65504
-// do not fit fp16: the conversion flags them (FA_ERR_UNSUPPORTED).
+// than bf16 would give them. Inputs with |x| >= 65504 do not fit fp16: the
+// conversion flags them, as does the dS pass for |dS| >= 65504
+// (FA_ERR_UNSUPPORTED through the device error word).
 //
-// B200 mapping (one CTA per (batch*head, key block), 384 threads):
+// B200 mapping (one CTA per (batch*head, key block), 512 threads):
 //   warp 0       TMA producer: K_j, V_j once; Q_i and dO_i per row block
 //                through two-stage rings.
 //   warp 1       TMEM allocation; lane 0 issues all tcgen05.mma:
@@ -31,10 +31,12 @@
 //                dQ_i = dS K_j (dS from shared memory, read K-major for dK
 //                and MN-major for dQ).
 //   warps 4..7   thread = key row (TMEM lane): P^T from S^T and L, packed to
-//                bf16 in TMEM; dS^T = P^T o (dP^T - D) written to shared
-//                memory in the 128-byte-swizzled layout the MMA reads; at the
-//                end, dK and dV rows to HBM.
-//   warps 8..11  thread = query row of the dQ tile: reads the fp32 dQ tile
+//                fp16 in TMEM (for dV and for the dS group).
+//   warps 8..11  thread = key row: copies P^T(i) out of TMEM (so S^T(i+1) can
+//                start), then dS^T = P^T o (dP^T - D) into shared memory in the
+//                128-byte-swizzled layout the MMA reads; at the end, dK and dV
+//                rows to HBM. P of block i+1 and dS of block i overlap.
+//   warps 12..15 thread = query row of the dQ tile: reads the fp32 dQ tile
 //                from TMEM and adds it to dQ in HBM with vector reductions.
 // TMEM (512 columns): S^T / P^T [0,128), dP^T [128,256) (reused for the dQ
 // tile once dS is out), dV [256, 256+D), dK [256+D, 256+2D).
@@ -65,24 +67,24 @@ struct BwdCfg {
   static constexpr int B_KV = 0;
   static constexpr int B_QF = 1, B_QE = 3, B_DF = 5, B_DE = 7;   // [2] each
   static constexpr int B_ST = 9, B_DPT = 10, B_P = 11, B_DV = 12, B_DS = 13, B_DSFREE = 14;
-  static constexpr int B_DQ = 15, B_DQFREE = 16, B_END = 17, B_DRAIN = 18;
-  static constexpr int NBAR = 19;
+  static constexpr int B_DQ = 15, B_DQFREE = 16, B_END = 17, B_DRAIN = 18, B_PR = 19;
+  static constexpr int NBAR = 20;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   // d = 128 leaves no room for alignment slack: the dynamic shared memory
   // base must already be 1024-byte aligned (checked at run time)
   static constexpr int SMEM_BYTES = MISC_OFF + 16;
   static constexpr uint32_t COL_ST = 0, COL_DPT = 128, COL_DV = 256, COL_DK = 256 + D;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr int THREADS = 384;
+  static constexpr int THREADS = 512;
 };
 
 enum : uint32_t {
   kSiteKV = 0x31, kSiteQE = 0x32, kSiteDE = 0x33, kSiteQF = 0x34, kSiteDF = 0x35, kSiteP = 0x36,
   kSiteDV = 0x37, kSiteDS = 0x38, kSiteDQF = 0x39, kSiteST = 0x3a, kSiteDPT = 0x3b,
-  kSiteDSF = 0x3c, kSiteDQ = 0x3d, kSiteEnd = 0x3e, kSiteDrain = 0x3f
+  kSiteDSF = 0x3c, kSiteDQ = 0x3d, kSiteEnd = 0x3e, kSiteDrain = 0x3f, kSitePR = 0x40
 };
 
-constexpr float kDsScale = 1.0f / 256.0f;   // dS is stored as dS * 2^-8
+constexpr float kDsScale = 1.0f;   // dS is stored unscaled (fp16: |dS| < 65504)
 
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
@@ -159,7 +161,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdArgs a) {
 
 // --------------------------------------------------------------- main pass
 template <int D>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
 bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                 BwdArgs a) {
@@ -196,6 +198,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     mbar_init(bar(C::B_ST), 1);
     mbar_init(bar(C::B_DPT), 1);
     mbar_init(bar(C::B_P), 128);
+    mbar_init(bar(C::B_PR), 128);
     mbar_init(bar(C::B_DV), 1);
     mbar_init(bar(C::B_DS), 128);
     mbar_init(bar(C::B_DSFREE), 1);
@@ -307,8 +310,10 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                       (it > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bar(C::B_DV));
         if (it + 1 < n_it) {
-          // S^T(it+1) overwrites P^T(it): wait until dV(it) has read it
-          ok = mbar_wait(bar(C::B_DV), it & 1, a.err, kSiteDV, abort_flag);
+          // S^T(it+1) overwrites P^T(it): wait until dV(it) and the dS group
+          // have both read it
+          ok = mbar_wait(bar(C::B_DV), it & 1, a.err, kSiteDV, abort_flag) &&
+               mbar_wait(bar(C::B_PR), it & 1, a.err, kSitePR, abort_flag);
           if (!ok) break;
           ok = issue_st(it + 1);
           if (!ok) break;
@@ -345,54 +350,73 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       mbar_wait(bar(C::B_DRAIN), 0, a.err, kSiteDrain, nullptr, 200000000ull);
     }
   } else if (warp >= 4 && warp < 8) {
-    // ------------------------------------------- P^T and dS^T (thread = key)
+    // ------------------------------------------------ P^T (thread = key row)
     const int r = (warp & 3) * 32 + lane;            // key within the block == TMEM lane
     const int key = kb * C::BK + r;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t st_addr = tmem + lane_off + C::COL_ST;
-    const uint32_t dpt_addr = tmem + lane_off + C::COL_DPT;
     const float sl2 = a.scale_log2;
-    uint8_t* ds_row = smem + C::DS_OFF + r * 128;    // row r of each 64-query chunk
-    bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int s = it & 1;
       const int q0 = (i0 + it) * C::BQ;
       const float* Ls = reinterpret_cast<const float*>(smem + C::L_OFF + s * 512);
-      const float* Ds = reinterpret_cast<const float*>(smem + C::DL_OFF + s * 512);
       // queries >= N have L = +inf (P = 0); the causal diagonal block and keys
       // >= N need an explicit mask
       const bool need_mask = (a.causal && key > q0) || key >= a.N;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_ST), it & 1, a.err, kSiteST, abort_flag));
-      if (!ok) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(C::B_ST), it & 1, a.err, kSiteST, abort_flag)))
+        break;
       tc_fence_after();
-      uint32_t pk0[32], pk1[32];
-#define PK(i) (((i) < 32) ? pk0[(i)] : pk1[(i)-32])
+      // queries [64*half, 64*half+64) -> fp16 pairs in TMEM columns [32*half, 32*half+32)
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {                   // 32 queries at a time
-        uint32_t sr[32];
-        tmem_ld32(st_addr + h * 32, sr);
+      for (int half = 0; half < 2; ++half) {
+        uint32_t sr0[32], sr1[32];
+        tmem_ld32(st_addr + half * 64, sr0);
+        tmem_ld32(st_addr + half * 64 + 32, sr1);
         tmem_ld_wait();
+        uint32_t pk[32];
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float4 lv = *reinterpret_cast<const float4*>(Ls + h * 32 + e);
+        for (int e = 0; e < 64; e += 4) {
+          const float4 lv = *reinterpret_cast<const float4*>(Ls + half * 64 + e);
           const float L[4] = {lv.x, lv.y, lv.z, lv.w};
           float p[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
+            const uint32_t sv = (e + u) < 32 ? sr0[e + u] : sr1[e + u - 32];
             // P = exp(scale*s - L) = exp2(s*scale*log2e - L*log2e)
-            p[u] = ex2_approx(fmaf(__uint_as_float(sr[e + u]), sl2, -L[u]));
-            if (need_mask && ((a.causal && key > q0 + h * 32 + e + u) || key >= a.N)) p[u] = 0.f;
+            p[u] = ex2_approx(fmaf(__uint_as_float(sv), sl2, -L[u]));
+            if (need_mask && ((a.causal && key > q0 + half * 64 + e + u) || key >= a.N)) p[u] = 0.f;
           }
-          PK((h * 32 + e) / 2) = pack_f16x2(p[0], p[1]);
-          PK((h * 32 + e) / 2 + 1) = pack_f16x2(p[2], p[3]);
+          pk[e / 2] = pack_f16x2(p[0], p[1]);
+          pk[e / 2 + 1] = pack_f16x2(p[2], p[3]);
         }
+        tmem_st32(st_addr + half * 32, pk);
       }
-      tmem_st32(st_addr, pk0);
-      tmem_st32(st_addr + 32, pk1);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(C::B_P));
-      // dS^T = P^T o (dP^T - D)
+    }
+    tc_fence_before();
+  } else if (warp >= 8 && warp < 12) {
+    // ---------------------------- dS^T = P^T o (dP^T - D) (thread = key row)
+    const int r = (warp & 3) * 32 + lane;
+    const int key = kb * C::BK + r;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t st_addr = tmem + lane_off + C::COL_ST;
+    const uint32_t dpt_addr = tmem + lane_off + C::COL_DPT;
+    uint8_t* ds_row = smem + C::DS_OFF + r * 128;    // row r of each 64-query chunk
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      const int s = it & 1;
+      const float* Ds = reinterpret_cast<const float*>(smem + C::DL_OFF + s * 512);
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_P), it & 1, a.err, kSiteP, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t pk0[32], pk1[32];                     // P^T(it), fp16 pairs, queries 0..127
+      tmem_ld32(st_addr, pk0);
+      tmem_ld32(st_addr + 32, pk1);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_PR));                     // S^T(it+1) may now overwrite P^T(it)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_DPT), it & 1, a.err, kSiteDPT, abort_flag));
       if (!ok) break;
       if (it > 0) {  // dS buffer reusable once dK(it-1) and dQ(it-1) have read it
@@ -401,37 +425,43 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (!ok) break;
       }
       tc_fence_after();
+      float ds_max = 0.f;
+#define PK(i) (((i) < 32) ? pk0[(i)] : pk1[(i)-32])
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        uint32_t dr[32];
-        tmem_ld32(dpt_addr + h * 32, dr);
+      for (int g = 0; g < 8; ++g) {                  // 16 queries at a time
+        uint32_t dr[16];
+        tmem_ld16(dpt_addr + g * 16, dr);
         tmem_ld_wait();
-        uint32_t w[16];
+        uint32_t w[8];
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float4 dv4 = *reinterpret_cast<const float4*>(Ds + h * 32 + e);
+        for (int e = 0; e < 16; e += 4) {
+          const float4 dv4 = *reinterpret_cast<const float4*>(Ds + g * 16 + e);
           const float Dv[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
           float ds[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const uint32_t pp = PK((h * 32 + e + u) >> 1);
-            const float pv = ((e + u) & 1) ? f16_hi(pp) : f16_lo(pp);
+            const int q = g * 16 + e + u;
+            const uint32_t pp = PK(q >> 1);
+            const float pv = (q & 1) ? f16_hi(pp) : f16_lo(pp);
             ds[u] = (pv * kDsScale) * (__uint_as_float(dr[e + u]) - Dv[u]);
           }
+          ds_max = fmaxf(ds_max, fmaxf(fmaxf(fabsf(ds[0]), fabsf(ds[1])),
+                                       fmaxf(fabsf(ds[2]), fabsf(ds[3]))));
           w[e / 2] = pack_f16x2(ds[0], ds[1]);
           w[e / 2 + 1] = pack_f16x2(ds[2], ds[3]);
         }
-        // queries h*32 .. h*32+31 = chunk (h/2), 16-byte units (h%2)*4 .. +3 of the
+        // queries g*16 .. g*16+15 = chunk g/4, 16-byte units (g%4)*2 and +1 of the
         // 128-byte row, XOR-swizzled with (key row % 8) like a TMA SWIZZLE_128B tile
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int unit = (h & 1) * 4 + u;
-          uint4* dst = reinterpret_cast<uint4*>(ds_row + (h >> 1) * C::CHUNK +
+        for (int u = 0; u < 2; ++u) {
+          const int unit = (g & 3) * 2 + u;
+          uint4* dst = reinterpret_cast<uint4*>(ds_row + (g >> 2) * C::CHUNK +
                                                 ((unit ^ (r & 7)) << 4));
           *dst = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
         }
       }
 #undef PK
+      if (!(ds_max < 65504.f)) atomicCAS(a.err, 0u, kErrRange + 2);
       fence_async_smem();   // generic-proxy smem writes -> visible to the MMA
       tc_fence_before();
       mbar_arrive(bar(C::B_DS));
@@ -465,7 +495,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
     }
     tc_fence_before();
-  } else if (warp >= 8) {
+  } else if (warp >= 12) {
     // ---------------------------------------- dQ tile -> HBM (thread = query)
     const int r = (warp & 3) * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;

@@ -17,10 +17,13 @@
 //                   tiles, S and O in TMEM) with kind::f8f6f4 MMAs:
 //                     S = q8 k8^T (fp32 accumulate); the true score is
 //                     S * sq(row block) * sk(key block) * softmax scale;
-//                     P' = P * sv(key block) / C rounded to e4m3 feeds the
-//                     P.V product from TMEM, C = max over the head's V scales
-//                     (so P' <= 256 < 448 never saturates);
-//                     O = C * (sum P' v8) / l with l the fp32 sum of P.
+//                     P' = P * sv(key block) * 256 / C rounded to e4m3 feeds
+//                     the P.V product from TMEM, C = max over the head's V
+//                     scales. P uses the exact running max (P <= 1), so
+//                     P' <= 256 < 448 never saturates, and the factor 256
+//                     keeps P' of blocks with small V scales out of e4m3's
+//                     subnormal range;
+//                     O = (C / 256) * (sum P' v8) / l, l the fp32 sum of P.
 //                   V stays MN-major in shared memory (tcgen05 reads e4m3
 //                   operands in either major order), so no transpose is needed.
 #include "prim.cuh"
@@ -136,7 +139,9 @@ struct F8 {
   static __device__ __forceinline__ uint32_t o_col(int t) { return 256u + 128u * t; }
 };
 
-constexpr float kRescaleThreshold = 8.0f;
+// exact running max (P <= 1): the e4m3 P' keeps its full range for every block
+constexpr float kRescaleThreshold = 0.0f;
+constexpr float kPScale = 256.0f;
 enum : uint32_t {
   kSQ = 0x41, kSKE = 0x42, kSKF = 0x43, kSS = 0x44, kSP = 0x45, kSO = 0x46, kSEpi = 0x47,
   kSDrain = 0x48
@@ -296,7 +301,7 @@ fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int row = q0[t] + r;
     const int limit = a.causal ? min(row, a.N - 1) : a.N - 1;
     const float* skh = a.sk + static_cast<size_t>(bh) * nsb;
-    const float inv_c = 1.f / *cmax;
+    const float inv_c = kPScale / *cmax;
     // per-row factor: softmax scale * log2(e) * q block scale
     const float rowf = a.scale_log2 * a.sq[static_cast<size_t>(bh) * nsb + min(row, a.N - 1) / 64];
     float m_run = -INFINITY, l_run = 0.f;
@@ -374,7 +379,7 @@ fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                       mbar_wait(bar(C::B_O + t), (nkb_t[t] - 1) & 1, a.err, kSEpi, abort_flag));
       if (ok) {
         tc_fence_after();
-        const float mul = *cmax / l_run;
+        const float mul = *cmax / (kPScale * l_run);
         __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) + (static_cast<size_t>(bh) * a.N + row) * kD;
 #pragma unroll
         for (int c = 0; c < kD / 32; ++c) {

@@ -104,8 +104,9 @@ FA_API size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
  * column blocks with atomic adds for the shared gradient.)
  * Precision: the products run on fp16 tensor-core operands (exact copies of
  * the bf16 inputs; P and dS rounded to fp16), accumulation is fp32. Inputs
- * must satisfy |x| < 65504 (fp16 range); larger values are recorded and
- * reported by fa_last_device_error() as FA_ERR_UNSUPPORTED.
+ * and the intermediate dS must satisfy |x| < 65504 (fp16 range); larger
+ * values are recorded and reported by fa_last_device_error() as
+ * FA_ERR_UNSUPPORTED.
  * Errors: as fa_fwd, plus FA_ERR_WORKSPACE when workspace is NULL or smaller
  * than required.
  */

@@ -159,8 +159,10 @@ def test_causal_one_hot_dv_bit_exact(N, d):
     x = {n: t.to(torch.bfloat16).cuda() for n, t in (("q", q), ("k", k), ("v", v), ("do", do))}
     dq, dk, dv = _chained(x, True)
     assert torch.equal(dv, x["do"].float())
-    # dS is zero up to rounding (dP_ii = D_i): dQ and dK vanish
-    assert float(dq.abs().max()) < 1e-2 and float(dk.abs().max()) < 1e-2
+    # dS is zero up to fp32 rounding (dP_ii = D_i, summed in different orders),
+    # so dQ = scale dS K and dK = scale dS^T Q vanish relative to |K| and |Q|
+    assert float(dq.abs().max()) < 1e-4 * float(k.abs().max())
+    assert float(dk.abs().max()) < 1e-4 * float(q.abs().max())
 
 
 def test_guard_regions_and_workspace():
