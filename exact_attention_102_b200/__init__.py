@@ -34,6 +34,7 @@ EXPORTS = (
     "fa_status_str", "fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd",
     "paged_attn_decode_workspace_bytes", "paged_attn_decode", "fa_fp8_prepare",
     "fa_fwd_fp8", "fa_last_device_error", "fa_debug_wait_timeout",
+    "paged_attn_decode_noalloc",
 )
 
 
@@ -69,6 +70,9 @@ def lib() -> ctypes.CDLL:
     L.paged_attn_decode.restype = ci
     L.paged_attn_decode.argtypes = [vp, vp, vp, ci, vp, ci, vp, vp, vp, ci, ci, ci, ci, ci, ci,
                                     vp, sz, vp]
+    L.paged_attn_decode_noalloc.restype = ci
+    L.paged_attn_decode_noalloc.argtypes = [vp, vp, vp, ci, vp, ci, vp, vp, vp, ci, ci, ci, ci,
+                                            ci, ci, vp]
     L.fa_fp8_prepare.restype = ci
     L.fa_fp8_prepare.argtypes = [vp] * 10 + [ci, ci, ci, ci, vp]
     L.fa_fwd_fp8.restype = ci
@@ -185,6 +189,27 @@ def paged_attn_decode(q, k_cache, v_cache, block_table, context_lens, max_ctx, o
         block_table.shape[1],
         _ptr(context_lens), _ptr(o), _ptr(lse), S, Hq, Hkv, d, bs, int(max_ctx),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+    return o, lse
+
+
+def paged_attn_decode_noalloc(q, k_cache, v_cache, block_table, context_lens, max_ctx, o,
+                              lse=None, stream=None):
+    """paged_attn_decode with the library's internal scratch instead of a
+    workspace. ``o`` (and ``lse`` if wanted) must be preallocated by the caller:
+    this wrapper allocates nothing."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(context_lens, "context_lens", torch.int32, 1)
+    _need(o, "o", torch.bfloat16, 3)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, 2)
+    S, Hq, d = q.shape
+    _check("paged_attn_decode_noalloc", lib().paged_attn_decode_noalloc(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), k_cache.shape[0], _ptr(block_table),
+        block_table.shape[1], _ptr(context_lens), _ptr(o), _ptr(lse), S, Hq, k_cache.shape[1], d,
+        k_cache.shape[2], int(max_ctx), _stream(stream)))
     return o, lse
 
 

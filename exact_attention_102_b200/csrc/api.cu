@@ -13,6 +13,8 @@
 
 namespace fa {
 int decode_split_blocks();
+size_t decode_scratch_bytes();
+cudaError_t decode_scratch_ptr(void** out);
 }
 
 namespace {
@@ -250,6 +252,23 @@ fa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_ca
   a.err = err;
   cudaError_t e = fa::launch_decode(a, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+fa_status paged_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                    int num_phys_blocks, const int* block_table,
+                                    int max_blocks_per_seq, const int* context_lens, void* o,
+                                    float* lse, int num_seqs, int Hq, int Hkv, int d,
+                                    int block_size, int max_ctx, void* stream) {
+  // Same checks as paged_attn_decode, then the library's own scratch array
+  // stands in for the workspace (no allocation anywhere on this path).
+  if (num_seqs < 1 || Hq < 1 || d < 1 || max_ctx < 1) return FA_ERR_INVALID_ARG;
+  const size_t need = paged_attn_decode_workspace_bytes(num_seqs, Hq, d, max_ctx);
+  if (need > fa::decode_scratch_bytes()) return FA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if (fa::decode_scratch_ptr(&scratch) != cudaSuccess) return FA_ERR_LAUNCH;
+  return paged_attn_decode(q, k_cache, v_cache, num_phys_blocks, block_table, max_blocks_per_seq,
+                           context_lens, o, lse, num_seqs, Hq, Hkv, d, block_size, max_ctx,
+                           scratch, fa::decode_scratch_bytes(), stream);
 }
 
 fa_status fa_fp8_prepare(const void* q, const void* k, const void* v, const float* R, void* q8,

@@ -333,4 +333,36 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+// --------------------------------------------------- allocation-free variant
+// Scratch for paged_attn_decode_noalloc: the split partials live in this
+// file-scope device array instead of a caller-provided workspace, for callers
+// that must not allocate device memory. Every GPU that loads the library holds
+// it (kDecodeScratchBytes) until the process exits. All calls share it: calls
+// that overlap on the GPU race on it. Nothing needs clearing between calls,
+// because the combine kernel only reads partials the split kernel of the same
+// call has just written.
+constexpr size_t kDecodeScratchBytes = size_t(16) << 20;   // 16 MiB
+static __device__ __align__(256) uint8_t g_decode_scratch[kDecodeScratchBytes];
+
+size_t decode_scratch_bytes() { return kDecodeScratchBytes; }
+
+// Device address of the scratch array on the current device. In host code the
+// array's name is only a stand-in, so the address is looked up once per device
+// (with that device current) and cached.
+cudaError_t decode_scratch_ptr(void** out) {
+  static void* ptrs[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (ptrs[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess) return e;
+    ptrs[dev] = p;
+  }
+  *out = ptrs[dev];
+  return cudaSuccess;
+}
+
 }  // namespace fa

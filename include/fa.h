@@ -160,6 +160,35 @@ FA_API fa_status paged_attn_decode(const void* q, const void* k_cache, const voi
                             int max_ctx, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * paged_attn_decode_noalloc — paged_attn_decode without a workspace argument,
+ * for callers that cannot allocate device memory on their decode path (for
+ * example an engine that fixes its whole device-memory plan at start-up and
+ * forbids allocation afterwards, or code that must not trigger the implicit
+ * synchronisation of cudaMalloc/cudaFree). The pages have no counterpart: this
+ * is an interface convenience around the same two kernels.
+ * The split partials go to a 16 MiB device array inside the library (every
+ * GPU that loads the library holds it until the process exits); the call
+ * allocates nothing. Arguments, layouts and results are those of
+ * paged_attn_decode.
+ *   - Limit: paged_attn_decode_workspace_bytes(num_seqs, Hq, d, max_ctx) must
+ *     not exceed 16 MiB (16777216 bytes); larger requests return
+ *     FA_ERR_WORKSPACE and launch nothing.
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before any
+ *     stream capture.
+ *   - All calls share the array and it keeps the last call's contents (no
+ *     clearing is needed: every partial read was written by the same call).
+ *     Calls that overlap on the GPU (different streams, or several host
+ *     threads) race on it and must be serialised by the caller.
+ */
+FA_API fa_status paged_attn_decode_noalloc(const void* q, const void* k_cache,
+                                           const void* v_cache, int num_phys_blocks,
+                                           const int* block_table, int max_blocks_per_seq,
+                                           const int* context_lens, void* o, float* lse,
+                                           int num_seqs, int Hq, int Hkv, int d, int block_size,
+                                           int max_ctx, void* stream);
+
+/*
  * fa_fp8_prepare — incoherent processing + per-block e4m3 quantisation.
  *   q, k, v    : bf16 BHND inputs.
  *   R          : fp32 [d][d] orthogonal matrix (row-major); Q' = Q R and

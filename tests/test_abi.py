@@ -107,3 +107,13 @@ def test_debug_probe_rejects_bad_limit_without_gpu():
     L = fa.lib()
     assert L.fa_debug_wait_timeout(0, None) == fa.FA_ERR_INVALID_ARG
     assert L.fa_debug_wait_timeout(2000000, None) == fa.FA_ERR_INVALID_ARG
+
+
+def test_decode_noalloc_rejects_oversize_without_gpu():
+    L = fa.lib()
+    g = _p(0x10000)
+    # 64 x 32 x 32 splits x 129 floats = 33.8 MB of partials > the 16 MiB scratch
+    assert L.paged_attn_decode_noalloc(g, g, g, 1000, g, 2048, g, g, g, 64, 32, 8, 128, 16,
+                                       32768, None) == fa.FA_ERR_WORKSPACE
+    assert L.paged_attn_decode_noalloc(g, g, g, 1000, g, 2048, g, g, g, 0, 32, 8, 128, 16,
+                                       32768, None) == fa.FA_ERR_INVALID_ARG
