@@ -164,10 +164,12 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   void* v16 = w16 + 2 * tsz;
   void* do16 = w16 + 3 * tsz;
   CUtensorMap tq, tk, tv, tdo;
-  if (!make_map(&tq, q16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, 128) ||
+  // d = 128 steps over 64 queries at a time (64-row Q / dO boxes), d = 64 over 128
+  const uint32_t qrows = d == 128 ? 64 : 128;
+  if (!make_map(&tq, q16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, qrows) ||
       !make_map(&tk, k16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, 128) ||
       !make_map(&tv, v16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, 128) ||
-      !make_map(&tdo, do16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, 128))
+      !make_map(&tdo, do16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, qrows))
     return FA_ERR_LAUNCH;
   fa::BwdArgs a;
   a.q16 = q16;
@@ -205,7 +207,7 @@ size_t paged_attn_decode_workspace_bytes(int num_seqs, int Hq, int d, int max_ct
   const int sb = fa::decode_split_blocks();
   const size_t max_splits = ((static_cast<size_t>(max_ctx) + 15) / 16 + sb - 1) / sb;
   const size_t rows = static_cast<size_t>(num_seqs) * Hq * max_splits;
-  return round256(rows * d * sizeof(float)) + round256(rows * sizeof(float));
+  return round256(rows * d * sizeof(float)) + round256(rows * sizeof(float)) + 256;
 }
 
 fa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_cache,
@@ -221,6 +223,8 @@ fa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_ca
     return FA_ERR_INVALID_ARG;
   if (d != 128 || block_size != 16 || Hq / Hkv != 4) return FA_ERR_UNSUPPORTED;
   if (static_cast<long long>(max_blocks_per_seq) * 16 < max_ctx) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(num_phys_blocks) * Hkv * block_size > (1ll << 31) - 1)
+    return FA_ERR_UNSUPPORTED;
   const size_t need = paged_attn_decode_workspace_bytes(num_seqs, Hq, d, max_ctx);
   if (workspace == nullptr || !aligned16(workspace) || ws_bytes < need) return FA_ERR_WORKSPACE;
   uint32_t* err = error_word_ptr();
@@ -241,6 +245,9 @@ fa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_ca
   a.part_o = static_cast<float*>(workspace);
   a.part_l = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                       round256(rows * d * sizeof(float)));
+  a.counter = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) +
+                                              round256(rows * d * sizeof(float)) +
+                                              round256(rows * sizeof(float)));
   a.num_seqs = num_seqs;
   a.Hq = Hq;
   a.Hkv = Hkv;
@@ -250,7 +257,15 @@ fa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_ca
   a.split_blocks = sb;
   a.scale_log2 = kLog2e / sqrtf(static_cast<float>(d));
   a.err = err;
-  cudaError_t e = fa::launch_decode(a, static_cast<cudaStream_t>(stream));
+  // K / V caches as 2-D [blocks * Hkv * 16 rows][d] for 64-column, 16-row,
+  // 128-byte-swizzled TMA boxes (one (block, kv head) slab = 2 boxes)
+  CUtensorMap tk, tv;
+  if (!make_map(&tk, k_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d,
+                num_phys_blocks * Hkv * block_size, 1, 64, block_size) ||
+      !make_map(&tv, v_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d,
+                num_phys_blocks * Hkv * block_size, 1, 64, block_size))
+    return FA_ERR_LAUNCH;
+  cudaError_t e = fa::launch_decode(tk, tv, a, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 

@@ -534,6 +534,404 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   }
 }
 
+// ------------------------------------------------- main pass, d = 128 -----
+// Same method, tiled for d = 128's TMEM budget with 64-query steps so that the
+// dQ tile gets its own double-buffered TMEM region and never blocks the next
+// step's dP^T:
+//   TMEM: S^T/P^T [0,64)  dP^T [64,128)  dQ^T x2 [128,256)  dV [256,384)
+//         dK [384,512)
+//   dQ is produced transposed, dQ^T = K^T dS^T (M = d = 128 lanes, N = 64
+//   queries), so the drain warps (thread = one head-dim column) issue
+//   reductions that are contiguous across a warp (32 consecutive floats).
+struct BwdQ64 {
+  static constexpr int D = 128;
+  static constexpr int BK = 128;                 // keys per CTA
+  static constexpr int BQ = 64;                  // queries per step
+  static constexpr int KV_TILE = 128 * D * 2;    // K or V tile (two 64-column chunks)
+  static constexpr int KV_CHUNK = 128 * 128;
+  static constexpr int Q_TILE = BQ * D * 2;      // Q or dO tile (two chunks of 64 rows)
+  static constexpr int Q_CHUNK = BQ * 128;
+  static constexpr int NS = 3;                   // Q / dO stages
+  static constexpr int DS_BYTES = BK * BQ * 2;   // dS^T fp16 [key][64 queries]: one 128 B row per key
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = K_OFF + KV_TILE;
+  static constexpr int Q_OFF = V_OFF + KV_TILE;
+  static constexpr int DO_OFF = Q_OFF + NS * Q_TILE;
+  static constexpr int DS_OFF = DO_OFF + NS * Q_TILE;
+  static constexpr int L_OFF = DS_OFF + DS_BYTES;       // NS x 64 fp32: L * log2(e)
+  static constexpr int DL_OFF = L_OFF + NS * 256;       // NS x 64 fp32: D
+  static constexpr int BAR_OFF = DL_OFF + NS * 256;
+  static constexpr int B_KV = 0, B_QF = 1, B_QE = B_QF + NS, B_DF = B_QE + NS, B_DE = B_DF + NS;
+  static constexpr int B_ST = B_DE + NS, B_DPT = B_ST + 1, B_P = B_DPT + 1, B_PR = B_P + 1;
+  static constexpr int B_DV = B_PR + 1, B_DS = B_DV + 1, B_DSFREE = B_DS + 1;
+  static constexpr int B_DQ = B_DSFREE + 1;            // [2]
+  static constexpr int B_DQFREE = B_DQ + 2;            // [2]
+  static constexpr int B_END = B_DQFREE + 2, B_DRAIN = B_END + 1, NBAR = B_DRAIN + 1;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
+  static constexpr uint32_t COL_ST = 0, COL_DPT = 64, COL_DQT = 128, COL_DV = 256, COL_DK = 384;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int THREADS = 512;
+};
+
+__global__ void __launch_bounds__(512, 1)
+bwd_q64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+               BwdArgs a) {
+  using C = BwdQ64;
+  constexpr int D = C::D;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw_addr);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int BH = a.B * a.H;
+  const int kb = static_cast<int>(blockIdx.x) / BH;   // key block (longest work first)
+  const int bh = static_cast<int>(blockIdx.x) % BH;
+  const int nq = (a.N + C::BQ - 1) / C::BQ;
+  const int i0 = a.causal ? kb * (C::BK / C::BQ) : 0;  // first query step that sees these keys
+  const int n_it = nq - i0;
+
+  auto bar = [&](int i) -> uint32_t { return base + C::BAR_OFF + 8 * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(C::B_KV), 1);
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(bar(C::B_QF + s), 1);
+      mbar_init(bar(C::B_QE + s), 1);
+      mbar_init(bar(C::B_DF + s), 1);
+      mbar_init(bar(C::B_DE + s), 1);
+    }
+    mbar_init(bar(C::B_ST), 1);
+    mbar_init(bar(C::B_DPT), 1);
+    mbar_init(bar(C::B_P), 128);
+    mbar_init(bar(C::B_PR), 128);
+    mbar_init(bar(C::B_DV), 1);
+    mbar_init(bar(C::B_DS), 128);
+    mbar_init(bar(C::B_DSFREE), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(C::B_DQ + b), 1);
+      mbar_init(bar(C::B_DQFREE + b), 128);
+    }
+    mbar_init(bar(C::B_END), 1);
+    mbar_init(bar(C::B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmDO);
+      mbar_arrive_expect_tx(bar(C::B_KV), 2 * C::KV_TILE);
+      for (int c = 0; c < 2; ++c) {
+        tma_load_3d(base + C::K_OFF + c * C::KV_CHUNK, &tmK, bar(C::B_KV), c * 64, kb * C::BK, bh);
+        tma_load_3d(base + C::V_OFF + c * C::KV_CHUNK, &tmV, bar(C::B_KV), c * 64, kb * C::BK, bh);
+      }
+      int issued = 0;
+      for (int it = 0; it < n_it; ++it) {
+        const int s = it % C::NS;
+        const uint32_t ph = ((it / C::NS) & 1) ^ 1;
+        const int row = (i0 + it) * C::BQ;
+        const size_t prow = static_cast<size_t>(bh) * a.n_pad + row;   // 256 B aligned
+        if (!mbar_wait(bar(C::B_QE + s), ph, a.err, kSiteQE, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(C::B_QF + s), C::Q_TILE + 256);
+        for (int c = 0; c < 2; ++c)
+          tma_load_3d(base + C::Q_OFF + s * C::Q_TILE + c * C::Q_CHUNK, &tmQ, bar(C::B_QF + s),
+                      c * 64, row, bh);
+        bulk_load(base + C::L_OFF + s * 256, a.lse_log2 + prow, 256, bar(C::B_QF + s));
+        if (!mbar_wait(bar(C::B_DE + s), ph, a.err, kSiteDE, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(C::B_DF + s), C::Q_TILE + 256);
+        for (int c = 0; c < 2; ++c)
+          tma_load_3d(base + C::DO_OFF + s * C::Q_TILE + c * C::Q_CHUNK, &tmDO, bar(C::B_DF + s),
+                      c * 64, row, bh);
+        bulk_load(base + C::DL_OFF + s * 256, a.delta + prow, 256, bar(C::B_DF + s));
+        issued = it + 1;
+      }
+      for (int it = max(0, issued - C::NS); it < issued; ++it) {
+        mbar_wait(bar(C::B_QF + it % C::NS), (it / C::NS) & 1, a.err, kSiteDrain, nullptr,
+                  200000000ull);
+        mbar_wait(bar(C::B_DF + it % C::NS), (it / C::NS) & 1, a.err, kSiteDrain, nullptr,
+                  200000000ull);
+      }
+      mbar_wait(bar(C::B_KV), 0, a.err, kSiteDrain, nullptr, 200000000ull);
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      constexpr uint32_t idST = idesc_f16(128, C::BQ, 0, 0, 0);  // S^T, dP^T: both K-major
+      constexpr uint32_t idKM = idesc_f16(128, D, 0, 0, 1);      // dV (A tmem), dK (A smem K-major)
+      constexpr uint32_t idQT = idesc_f16(128, C::BQ, 0, 1, 1);  // dQ^T: A = K^T, B = dS^T, MN-major
+      const uint32_t kbase = base + C::K_OFF, vbase = base + C::V_OFF, dsb = base + C::DS_OFF;
+      bool ok = mbar_wait(bar(C::B_KV), 0, a.err, kSiteKV, abort_flag);
+      auto issue_ss = [&](uint32_t d_col, uint32_t abase, uint32_t bbase) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {   // K = d: chunk kk/4, 32 B steps inside it
+          umma_f16_ss(tmem + d_col, smem_desc_sw128(abase + (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32, 16, 1024),
+                      smem_desc_sw128(bbase + (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32, 16, 1024),
+                      idST, kk > 0);
+        }
+      };
+      auto issue_st = [&](int it) -> bool {
+        const int s = it % C::NS;
+        if (!mbar_wait(bar(C::B_QF + s), (it / C::NS) & 1, a.err, kSiteQF, abort_flag)) return false;
+        tc_fence_after();
+        issue_ss(C::COL_ST, kbase, base + C::Q_OFF + s * C::Q_TILE);
+        umma_commit(bar(C::B_ST));
+        return true;
+      };
+      auto issue_dpt = [&](int it) -> bool {
+        const int s = it % C::NS;
+        if (!mbar_wait(bar(C::B_DF + s), (it / C::NS) & 1, a.err, kSiteDF, abort_flag)) return false;
+        tc_fence_after();
+        issue_ss(C::COL_DPT, vbase, base + C::DO_OFF + s * C::Q_TILE);
+        umma_commit(bar(C::B_DPT));
+        return true;
+      };
+      if (ok) ok = issue_st(0) && issue_dpt(0);
+      for (int it = 0; it < n_it && ok; ++it) {
+        const int s = it % C::NS;
+        const uint32_t qb = base + C::Q_OFF + s * C::Q_TILE;
+        const uint32_t gb = base + C::DO_OFF + s * C::Q_TILE;
+        const int buf = it & 1;
+        // dV += P^T dO_it (P^T fp16 pairs in TMEM columns [0, 32))
+        ok = mbar_wait(bar(C::B_P), it & 1, a.err, kSiteP, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < C::BQ / 16; ++kk)
+          umma_f16_ts(tmem + C::COL_DV, tmem + C::COL_ST + kk * 8,
+                      smem_desc_sw128(gb + kk * 2048, C::Q_CHUNK, 1024), idKM,
+                      (it > 0 || kk > 0) ? 1u : 0u);
+        if (it + 1 < n_it) {
+          // S^T(it+1) overwrites P^T(it): the dS group must have copied it out;
+          // dV(it), issued earlier by this thread, reads it first (tcgen05.mma
+          // from one thread executes in issue order)
+          ok = mbar_wait(bar(C::B_PR), it & 1, a.err, kSitePR, abort_flag);
+          if (!ok) break;
+          ok = issue_st(it + 1);
+          if (!ok) break;
+        }
+        ok = mbar_wait(bar(C::B_DS), it & 1, a.err, kSiteDS, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        // dK += dS^T Q_it: A = dS^T [key][query] K-major, B = Q_it MN-major
+#pragma unroll
+        for (int kk = 0; kk < C::BQ / 16; ++kk)
+          umma_f16_ss(tmem + C::COL_DK, smem_desc_sw128(dsb + kk * 32, 16, 1024),
+                      smem_desc_sw128(qb + kk * 2048, C::Q_CHUNK, 1024), idKM,
+                      (it > 0 || kk > 0) ? 1u : 0u);
+        // dQ^T_it = K^T dS^T into buffer it&1 (drained two steps ago)
+        if (it >= 2) {
+          ok = mbar_wait(bar(C::B_DQFREE + buf), ((it >> 1) - 1) & 1, a.err, kSiteDQF, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int kk = 0; kk < C::BK / 16; ++kk)
+          umma_f16_ss(tmem + C::COL_DQT + buf * 64,
+                      smem_desc_sw128(kbase + kk * 2048, C::KV_CHUNK, 1024),
+                      smem_desc_sw128(dsb + kk * 2048, 16, 1024), idQT, kk > 0 ? 1u : 0u);
+        umma_commit(bar(C::B_DQ + buf));
+        umma_commit(bar(C::B_DSFREE));
+        umma_commit(bar(C::B_QE + s));   // Q_it and its L: S^T, P, dK done
+        umma_commit(bar(C::B_DE + s));   // dO_it and its D: dP^T, dV, dS done
+        if (it + 1 < n_it) {
+          ok = issue_dpt(it + 1);        // the dS group has read dP^T(it)
+          if (!ok) break;
+        }
+      }
+      umma_commit(bar(C::B_END));
+      umma_commit(bar(C::B_DRAIN));
+      mbar_wait(bar(C::B_DRAIN), 0, a.err, kSiteDrain, nullptr, 200000000ull);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------ P^T (thread = key row)
+    const int r = (warp & 3) * 32 + lane;
+    const int key = kb * C::BK + r;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t st_addr = tmem + lane_off + C::COL_ST;
+    const float sl2 = a.scale_log2;
+    for (int it = 0; it < n_it; ++it) {
+      const int s = it % C::NS;
+      const int q0 = (i0 + it) * C::BQ;
+      const float* Ls = reinterpret_cast<const float*>(smem + C::L_OFF + s * 256);
+      const bool need_mask = (a.causal && key > q0) || key >= a.N;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(C::B_ST), it & 1, a.err, kSiteST, abort_flag)))
+        break;
+      tc_fence_after();
+      uint32_t sr0[32], sr1[32];
+      tmem_ld32(st_addr, sr0);
+      tmem_ld32(st_addr + 32, sr1);
+      tmem_ld_wait();
+      uint32_t pk[32];
+#pragma unroll
+      for (int e = 0; e < 64; e += 4) {
+        const float4 lv = *reinterpret_cast<const float4*>(Ls + e);
+        const float L[4] = {lv.x, lv.y, lv.z, lv.w};
+        float p[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t sv = (e + u) < 32 ? sr0[e + u] : sr1[e + u - 32];
+          p[u] = ex2_approx(fmaf(__uint_as_float(sv), sl2, -L[u]));
+          if (need_mask && ((a.causal && key > q0 + e + u) || key >= a.N)) p[u] = 0.f;
+        }
+        pk[e / 2] = pack_f16x2(p[0], p[1]);
+        pk[e / 2 + 1] = pack_f16x2(p[2], p[3]);
+      }
+      tmem_st32(st_addr, pk);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_P));
+    }
+    tc_fence_before();
+  } else if (warp >= 8 && warp < 12) {
+    // ---------------------------- dS^T = P^T o (dP^T - D) (thread = key row)
+    const int r = (warp & 3) * 32 + lane;
+    const int key = kb * C::BK + r;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t st_addr = tmem + lane_off + C::COL_ST;
+    const uint32_t dpt_addr = tmem + lane_off + C::COL_DPT;
+    uint8_t* ds_row = smem + C::DS_OFF + r * 128;     // one swizzled 128-byte row per key
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      const int s = it % C::NS;
+      const float* Ds = reinterpret_cast<const float*>(smem + C::DL_OFF + s * 256);
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_P), it & 1, a.err, kSiteP, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t pk[32];                                // P^T(it): fp16 pairs, 64 queries
+      tmem_ld32(st_addr, pk);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_PR));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_DPT), it & 1, a.err, kSiteDPT, abort_flag));
+      if (!ok) break;
+      if (it > 0) {
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(bar(C::B_DSFREE), (it - 1) & 1, a.err, kSiteDSF, abort_flag));
+        if (!ok) break;
+      }
+      tc_fence_after();
+      float ds_max = 0.f;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {                  // 16 queries at a time
+        uint32_t dr[16];
+        tmem_ld16(dpt_addr + g * 16, dr);
+        tmem_ld_wait();
+        uint32_t w[8];
+#pragma unroll
+        for (int e = 0; e < 16; e += 4) {
+          const float4 dv4 = *reinterpret_cast<const float4*>(Ds + g * 16 + e);
+          const float Dv[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
+          float ds[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int q = g * 16 + e + u;
+            const uint32_t pp = pk[q >> 1];
+            const float pv = (q & 1) ? f16_hi(pp) : f16_lo(pp);
+            ds[u] = pv * (__uint_as_float(dr[e + u]) - Dv[u]);
+          }
+          ds_max = fmaxf(ds_max, fmaxf(fmaxf(fabsf(ds[0]), fabsf(ds[1])),
+                                       fmaxf(fabsf(ds[2]), fabsf(ds[3]))));
+          w[e / 2] = pack_f16x2(ds[0], ds[1]);
+          w[e / 2 + 1] = pack_f16x2(ds[2], ds[3]);
+        }
+        // queries g*16 .. g*16+15 = 16-byte units 2g, 2g+1 of the key's 128-byte
+        // row, XOR-swizzled with (key row % 8) like a TMA SWIZZLE_128B tile
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          uint4* dst = reinterpret_cast<uint4*>(ds_row + (((2 * g + u) ^ (r & 7)) << 4));
+          *dst = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+        }
+      }
+      if (!(ds_max < 65504.f)) atomicCAS(a.err, 0u, kErrRange + 2);
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_DS));
+    }
+    // ---- epilogue: dV and dK rows (thread = key) to HBM
+    if (ok) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_END), 0, a.err, kSiteEnd, abort_flag));
+      if (ok) {
+        tc_fence_after();
+        const size_t orow = (static_cast<size_t>(bh) * a.N + key) * D;
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {
+          const uint32_t src = tmem + lane_off + (which ? C::COL_DK : C::COL_DV);
+          float* dst = (which ? a.dk : a.dv) + orow;
+          const float mul = which ? a.scale : 1.f;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(src + c * 32, v);
+            tmem_ld_wait();
+            if (key < a.N) {
+              float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                d4[e] = make_float4(__uint_as_float(v[4 * e]) * mul, __uint_as_float(v[4 * e + 1]) * mul,
+                                    __uint_as_float(v[4 * e + 2]) * mul,
+                                    __uint_as_float(v[4 * e + 3]) * mul);
+            }
+          }
+        }
+      }
+    }
+    tc_fence_before();
+  } else if (warp >= 12) {
+    // ------------------------ dQ^T tile -> HBM (thread = one head-dim column)
+    const int c = (warp & 3) * 32 + lane;            // TMEM lane = d index
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const float sc = a.scale;
+    for (int it = 0; it < n_it; ++it) {
+      const int buf = it & 1;
+      const int q0 = (i0 + it) * C::BQ;
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait(bar(C::B_DQ + buf), (it >> 1) & 1, a.err, kSiteDQ, abort_flag)))
+        break;
+      tc_fence_after();
+      uint32_t v0[32], v1[32];
+      tmem_ld32(tmem + lane_off + C::COL_DQT + buf * 64, v0);
+      tmem_ld32(tmem + lane_off + C::COL_DQT + buf * 64 + 32, v1);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_DQFREE + buf));          // the buffer is free again
+      float* col = a.dq + (static_cast<size_t>(bh) * a.N + q0) * D + c;
+      const int nv = min(C::BQ, a.N - q0);
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (j < nv) atomicAdd(col + static_cast<size_t>(j) * D, __uint_as_float(v0[j]) * sc);
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (32 + j < nv) atomicAdd(col + static_cast<size_t>(32 + j) * D, __uint_as_float(v1[j]) * sc);
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
 }  // namespace
 
 template <int D>
@@ -544,8 +942,12 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(bwd_main_kernel<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    cudaError_t e = D == 128 ? cudaFuncSetAttribute(bwd_q64_kernel,
+                                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                    BwdQ64::SMEM_BYTES)
+                             : cudaFuncSetAttribute(bwd_main_kernel<D>,
+                                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                    C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
@@ -560,7 +962,11 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int nk = (a.N + C::BK - 1) / C::BK;
-  bwd_main_kernel<D><<<nk * a.B * a.H, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
+  if (D == 128)
+    bwd_q64_kernel<<<nk * a.B * a.H, BwdQ64::THREADS, BwdQ64::SMEM_BYTES, stream>>>(tq, tk, tv,
+                                                                                   tdo, a);
+  else
+    bwd_main_kernel<D><<<nk * a.B * a.H, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
   return cudaGetLastError();
 }
 

@@ -5,29 +5,33 @@
 // per-sequence block table; several sequences (parallel sampling) may point
 // at the same physical block. The kernel only follows the table.
 //
-// Work split: one CTA per (sequence, KV head, split of `split_blocks`
-// 16-token blocks). A CTA serves the 4 query heads that share its KV head, so
+// Work split: one work item per (sequence, KV head, split of `split_blocks`
+// 16-token blocks); a persistent grid of two CTAs per SM takes items from a
+// global counter. An item serves the 4 query heads that share its KV head, so
 // every K/V byte is read from HBM once per query group. Each split produces a
 // partial (O_s normalised over its own keys, L_s = its logsumexp); the
 // combine kernel merges the splits with L = log sum_s exp(L_s),
 // O = sum_s exp(L_s - L) O_s, which follows from the definition of the
 // logsumexp statistic (91haoming.cn repost, "前向傳播改進").
 //
-// Inside a split CTA:
-//   warp 4 (producer)  loads the split's slice of the block table, then copies
-//                      each (block, KV head) K and V slab (16 x 128 bf16 =
-//                      4 KB each, contiguous) into an 8-stage shared-memory
-//                      ring with untiled bulk copies (no multicast), one full /
-//                      empty mbarrier pair per stage.
-//   warps 0..3         thread (t, c) = (tid / 8, tid % 8) owns token slot t of
-//                      every block and head-dim elements [8c, 8c+8) and
-//                      [64+8c, 64+8c+8): 16-byte shared loads, 64 FMAs for the
-//                      4 heads' scores, a 3-step shuffle reduction over the 8
-//                      threads of the slot, an online-softmax update per slot
-//                      (running max with rescale skipping, running sum), then
-//                      64 FMAs into the slot's unnormalised output. At the end
-//                      the 16 slot states are merged through shared memory
-//                      with the same logsumexp rule.
+// Inside a CTA:
+//   warp 4 (producer)  per item: the split's slice of the block table and the
+//                      4 query heads (1 KB bulk copy); then, per table entry,
+//                      the (block, KV head) K and V slabs (16 tokens x 128 bf16,
+//                      4 KB each) as two 64-column TMA boxes each, 128-byte
+//                      swizzled, into an 8-stage ring (full / empty mbarriers).
+//   warps 0..3         warp w takes blocks w, w+4, ... of the item and keeps its
+//                      own online-softmax state. Per block: S = Q K^T and
+//                      O += P V on the tensor cores with mma.sync m16n8k16
+//                      (bf16 in, fp32 accumulate; the 4 query heads fill 4 of
+//                      the 16 rows), K and V fragments read with ldmatrix from
+//                      the swizzled tiles; the S accumulator fragment is the P
+//                      operand fragment of the P.V product, so P never leaves
+//                      registers. The four warp states are merged at the end of
+//                      the item with the logsumexp rule.
+// Scores per block are a few thousand multiply-adds against 8 KB of HBM
+// traffic; the tensor cores only remove instruction-issue pressure so the
+// kernel can keep HBM busy.
 #include "prim.cuh"
 #include "kernels.h"
 
@@ -40,249 +44,345 @@ constexpr int kBlk = 16;          // tokens per physical block
 constexpr int kGroup = 4;         // query heads per KV head
 constexpr int kStages = 8;
 constexpr int kSlab = kBlk * kD * 2;           // bytes of one (block, kv head) K or V slab
+constexpr int kBox = kBlk * 128;               // one 64-column TMA box of a slab (2 KB)
 constexpr int kStageBytes = 2 * kSlab;         // K + V
 constexpr int kMaxSplitBlocks = 128;
-constexpr int kComputeThreads = 128;
+constexpr int kComputeWarps = 4;
+constexpr int kComputeThreads = 32 * kComputeWarps;
 constexpr int kThreads = kComputeThreads + 32;
 constexpr float kRescaleThreshold = 8.0f;
 
-// shared memory layout (bytes)
+// shared memory layout (bytes), ring 1024-byte aligned for the 128-byte swizzle
 constexpr int kRingOff = 0;
-constexpr int kTableOff = kRingOff + kStages * kStageBytes;
-constexpr int kBarOff = kTableOff + kMaxSplitBlocks * 4;
-constexpr int kMiscOff = kBarOff + 2 * kStages * 8;
-constexpr int kRedOff = kMiscOff + 16;     // cross-warp reduction scratch: [4 warps][4 heads] x 2
-constexpr int kSmemBytes = kRedOff + 2 * 16 * 4 + 128;
+constexpr int kMergeOff = kRingOff + kStages * kStageBytes;          // [4 warps][4 heads][128] fp32
+constexpr int kQOff = kMergeOff + kComputeWarps * kGroup * kD * 4;  // 2 x q group (4 x 128 bf16)
+constexpr int kQBytes = kGroup * kD * 2;
+constexpr int kTableOff = kQOff + 2 * kQBytes;
+constexpr int kDescOff = kTableOff + 2 * kMaxSplitBlocks * 4;  // 2 x {seq, kvh, split, nb, rem, -, -, -}
+constexpr int kBarOff = kDescOff + 2 * 32;        // full[S] empty[S] qfull[2] qempty[2] merge
+constexpr int kRedOff = kBarOff + (2 * kStages + 5) * 8;            // m, l: [4 warps][4 heads] x 2
+constexpr int kMiscOff = kRedOff + 2 * 16 * 4;
+constexpr int kSmemBytes = kMiscOff + 16 + 1024;
 
-enum : uint32_t { kSiteFull = 0x21, kSiteEmpty = 0x22, kSiteDrain = 0x23 };
+enum : uint32_t {
+  kSiteFull = 0x21, kSiteEmpty = 0x22, kSiteDrain = 0x23, kSiteQ = 0x24, kSiteMerge = 0x25
+};
 
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
-  f[0] = __uint_as_float(u.x << 16);
-  f[1] = __uint_as_float(u.x & 0xffff0000u);
-  f[2] = __uint_as_float(u.y << 16);
-  f[3] = __uint_as_float(u.y & 0xffff0000u);
-  f[4] = __uint_as_float(u.z << 16);
-  f[5] = __uint_as_float(u.z & 0xffff0000u);
-  f[6] = __uint_as_float(u.w << 16);
-  f[7] = __uint_as_float(u.w & 0xffff0000u);
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+// D(16x8 fp32) += A(16x16 bf16, row) * B(16x8 bf16, col)
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(DecodeArgs a) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  const int split = blockIdx.x;
-  const int kvh = blockIdx.y;
-  const int seq = blockIdx.z;
-  int ctx = a.context_lens[seq];
-  ctx = max(1, min(ctx, a.max_ctx));
-  const int nblk = (ctx + kBlk - 1) / kBlk;
-  const int first = split * a.split_blocks;
-  if (first >= nblk) return;  // this split is past the sequence's end
-  const int nb = min(nblk - first, a.split_blocks);
-
+// Persistent split kernel (see the file comment). Shared tiles: a slab's two
+// 64-column boxes are [16 rows][128 B], 16-byte units XOR-swizzled with
+// (row % 8) by the TMA.
+__global__ void __launch_bounds__(kThreads, 2)
+decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    DecodeArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (sbase - raw_addr);
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const uint32_t sbase = smem_u32(smem);
   int* table = reinterpret_cast<int*>(smem + kTableOff);
+  int* desc = reinterpret_cast<int*>(smem + kDescOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kMiscOff);
   auto full = [&](int s) -> uint32_t { return sbase + kBarOff + 8 * s; };
   auto empty = [&](int s) -> uint32_t { return sbase + kBarOff + 8 * (kStages + s); };
+  auto qfull = [&](int p) -> uint32_t { return sbase + kBarOff + 8 * (2 * kStages + p); };
+  auto qempty = [&](int p) -> uint32_t { return sbase + kBarOff + 8 * (2 * kStages + 2 + p); };
+  const uint32_t merge_bar = sbase + kBarOff + 8 * (2 * kStages + 4);
+  const long long total = static_cast<long long>(a.max_splits) * a.Hkv * a.num_seqs;
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(full(s), 1);
-      mbar_init(empty(s), kComputeThreads / 32);
+      mbar_init(empty(s), 1);                    // one consumer warp per block
     }
+    for (int p = 0; p < 2; ++p) {
+      mbar_init(qfull(p), 1);
+      mbar_init(qempty(p), kComputeWarps);
+    }
+    mbar_init(merge_bar, kComputeThreads);
     *abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
 
-  if (warp == 4) {
+  if (warp == kComputeWarps) {
     // ------------------------------------------------------------ producer
-    const int* trow = a.block_table + static_cast<size_t>(seq) * a.max_blocks + first;
-    for (int i = lane; i < nb; i += 32) {
-      int id = trow[i];
-      if (id < 0 || id >= a.num_phys) {  // never dereference a bad id
-        atomicCAS(a.err, 0u, kErrBadIndex + 1);
-        id = 0;
+    // Items are handed out dynamically: lane 0 takes the next index of the
+    // dense (sequence, KV head, split) space from a global counter and skips
+    // splits past a sequence's end. The next item is resolved while the
+    // current item's first blocks are in flight.
+    struct Item { int seq, kvh, split, nb, rem; };
+    auto resolve = [&]() -> Item {     // lane 0 only
+      Item it{0, 0, 0, 0, 0};
+      while (true) {
+        const long long idx = atomicAdd(a.counter, 1u);
+        if (idx >= total) return it;   // nb = 0: no more work
+        it.split = static_cast<int>(idx % a.max_splits);
+        const long long rest = idx / a.max_splits;
+        it.kvh = static_cast<int>(rest % a.Hkv);
+        it.seq = static_cast<int>(rest / a.Hkv);
+        const int ctx = max(1, min(a.context_lens[it.seq], a.max_ctx));
+        const int first = it.split * a.split_blocks;
+        const int nblk = (ctx + kBlk - 1) / kBlk;
+        if (first < nblk) {
+          it.nb = min(nblk - first, a.split_blocks);
+          it.rem = min(ctx - first * kBlk, it.nb * kBlk);
+          return it;
+        }
       }
-      table[i] = id;
-    }
-    __syncwarp();
+    };
+    auto bcast = [&](Item it) -> Item {
+      it.seq = __shfl_sync(0xffffffffu, it.seq, 0);
+      it.kvh = __shfl_sync(0xffffffffu, it.kvh, 0);
+      it.split = __shfl_sync(0xffffffffu, it.split, 0);
+      it.nb = __shfl_sync(0xffffffffu, it.nb, 0);
+      it.rem = __shfl_sync(0xffffffffu, it.rem, 0);
+      return it;
+    };
     if (lane == 0) {
-      const uint8_t* kc = static_cast<const uint8_t*>(a.k_cache);
-      const uint8_t* vc = static_cast<const uint8_t*>(a.v_cache);
-      int issued = 0;
-      for (int i = 0; i < nb; ++i) {
-        const int s = i % kStages;
-        if (!mbar_wait(empty(s), ((i / kStages) & 1) ^ 1, a.err, kSiteEmpty, abort_flag)) break;
-        const size_t slab = (static_cast<size_t>(table[i]) * a.Hkv + kvh) * kSlab;
-        mbar_arrive_expect_tx(full(s), kStageBytes);
-        bulk_load(sbase + kRingOff + s * kStageBytes, kc + slab, kSlab, full(s));
-        bulk_load(sbase + kRingOff + s * kStageBytes + kSlab, vc + slab, kSlab, full(s));
-        ++issued;
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+    }
+    Item cur{0, 0, 0, 0, 0};
+    if (lane == 0) cur = resolve();
+    cur = bcast(cur);
+    long long g = 0;      // blocks issued so far (ring position)
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int p = k & 1;
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(qempty(p), ((k >> 1) & 1) ^ 1, a.err, kSiteQ, abort_flag));
+      if (!ok) break;
+      if (cur.nb == 0) {               // no more work: publish the end marker
+        if (lane == 0) {
+          desc[8 * p + 3] = 0;
+          mbar_arrive(qfull(p));
+        }
+        break;
       }
-      for (int i = max(0, issued - kStages); i < issued; ++i)
-        mbar_wait(full(i % kStages), (i / kStages) & 1, a.err, kSiteDrain, nullptr, 200000000ull);
+      int* tab = table + p * kMaxSplitBlocks;
+      const int* trow =
+          a.block_table + static_cast<size_t>(cur.seq) * a.max_blocks + cur.split * a.split_blocks;
+      for (int i = lane; i < cur.nb; i += 32) {
+        int id = trow[i];
+        if (id < 0 || id >= a.num_phys) {  // never dereference a bad id
+          atomicCAS(a.err, 0u, kErrBadIndex + 1);
+          id = 0;
+        }
+        tab[i] = id;
+      }
+      __syncwarp();
+      Item nxt{0, 0, 0, 0, 0};
+      if (lane == 0) {
+        desc[8 * p + 0] = cur.seq;
+        desc[8 * p + 1] = cur.kvh;
+        desc[8 * p + 2] = cur.split;
+        desc[8 * p + 3] = cur.nb;
+        desc[8 * p + 4] = cur.rem;
+        mbar_arrive_expect_tx(qfull(p), kQBytes);
+        bulk_load(sbase + kQOff + p * kQBytes,
+                  static_cast<const __nv_bfloat16*>(a.q) +
+                      (static_cast<size_t>(cur.seq) * a.Hq + cur.kvh * kGroup) * kD,
+                  kQBytes, qfull(p));
+        const int head = min(cur.nb, kStages);
+        for (int i = 0; i < cur.nb && ok; ++i, ++g) {
+          if (i == head) nxt = resolve();   // overlaps with the blocks in flight
+          const int s = static_cast<int>(g % kStages);
+          ok = mbar_wait(empty(s), static_cast<uint32_t>((g / kStages) & 1) ^ 1, a.err, kSiteEmpty,
+                         abort_flag);
+          if (!ok) break;
+          const int row = (tab[i] * a.Hkv + cur.kvh) * kBlk;
+          const uint32_t st = sbase + kRingOff + s * kStageBytes;
+          mbar_arrive_expect_tx(full(s), kStageBytes);
+          tma_load_3d(st, &tmK, full(s), 0, row, 0);
+          tma_load_3d(st + kBox, &tmK, full(s), 64, row, 0);
+          tma_load_3d(st + kSlab, &tmV, full(s), 0, row, 0);
+          tma_load_3d(st + kSlab + kBox, &tmV, full(s), 64, row, 0);
+        }
+        if (ok && cur.nb <= head) nxt = resolve();
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      cur = bcast(nxt);
+    }
+    if (lane == 0) {
+      for (long long i = (g > kStages ? g - kStages : 0); i < g; ++i)
+        mbar_wait(full(static_cast<int>(i % kStages)), static_cast<uint32_t>((i / kStages) & 1),
+                  a.err, kSiteDrain, nullptr, 200000000ull);
     }
     return;
   }
 
   // -------------------------------------------------------------- compute
-  const int t = tid >> 3;   // token slot 0..15
-  const int c = tid & 7;    // element group
-  const int h0 = kvh * kGroup;
-  float qv[kGroup][16];
-  {
-    const __nv_bfloat16* qp =
-        static_cast<const __nv_bfloat16*>(a.q) + (static_cast<size_t>(seq) * a.Hq + h0) * kD;
-#pragma unroll
-    for (int hh = 0; hh < kGroup; ++hh) {
-      const uint4 u0 = *reinterpret_cast<const uint4*>(qp + hh * kD + 8 * c);
-      const uint4 u1 = *reinterpret_cast<const uint4*>(qp + hh * kD + 64 + 8 * c);
-      float f0[8], f1[8];
-      bf16x8_to_f32(u0, f0);
-      bf16x8_to_f32(u1, f1);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        qv[hh][e] = f0[e] * a.scale_log2;  // scores come out in exp2 units
-        qv[hh][8 + e] = f1[e] * a.scale_log2;
-      }
-    }
-  }
-  float m[kGroup], l[kGroup], acc[kGroup][16];
-#pragma unroll
-  for (int hh = 0; hh < kGroup; ++hh) {
-    m[hh] = -INFINITY;
-    l[hh] = 0.f;
-#pragma unroll
-    for (int e = 0; e < 16; ++e) acc[hh][e] = 0.f;
-  }
-
-  bool ok = true;
-  for (int i = 0; i < nb; ++i) {
-    const int s = i % kStages;
-    ok = __all_sync(0xffffffffu,
-                    mbar_wait(full(s), (i / kStages) & 1, a.err, kSiteFull, abort_flag));
-    if (!ok) break;
-    const uint8_t* kst = smem + kRingOff + s * kStageBytes + t * (kD * 2);
-    float kf[16];
+  // mma.sync fragment coordinates: group g = lane / 4 (A/C row, B column),
+  // quad index q = lane % 4 (A/B k pair 2q, 2q+1; C column pair 2q, 2q+1).
+  const int g = lane >> 2;
+  const int qd = lane & 3;
+  const bool real = g < kGroup;         // A/C rows 0..3 are the 4 heads, 4..15 padding
+  float* red = reinterpret_cast<float*>(smem + kRedOff);
+  float* mrg = reinterpret_cast<float*>(smem + kMergeOff);
+  uint32_t merge_phase = 0;
+  auto sync128 = [&]() -> bool {        // bounded, never bar.sync (see below)
+    mbar_arrive(merge_bar);
+    const bool r = mbar_wait(merge_bar, merge_phase & 1, a.err, kSiteMerge, abort_flag);
+    ++merge_phase;
+    return __all_sync(0xffffffffu, r);
+  };
+  // ldmatrix row addresses inside a stage (bytes from the stage base):
+  //  K (non-transposed, B operand of S = Q K^T): matrix mi = lane/8 covers tokens
+  //    8*(mi/2) .. +7 and 16-byte unit (mi%2) of the k-step's 32-byte slice.
+  //  V (transposed, B operand of O = P V): matrix mi covers tokens 8*(mi%2) .. +7
+  //    and the 8 columns of n-tile 2*j + mi/2.
+  const int mi = lane >> 3, rr = lane & 7;
+  const int k_tok = (mi >> 1) * 8 + rr;
+  const int v_tok = (mi & 1) * 8 + rr;
+  long long gb = 0;                      // blocks consumed by this CTA (ring position)
+  for (int k = 0;; ++k) {
+    const int p = k & 1;
+    if (!__all_sync(0xffffffffu, mbar_wait(qfull(p), (k >> 1) & 1, a.err, kSiteQ, abort_flag)))
+      break;
+    const int seq = desc[8 * p + 0], kvh = desc[8 * p + 1], split = desc[8 * p + 2];
+    const int nb = desc[8 * p + 3], rem = desc[8 * p + 4];
+    if (nb == 0) break;
+    // Q fragments (A of S = Q K^T): a0 = Q[g][16ks + 2q, +1], a2 = Q[g][16ks + 8 + 2q, +1]
+    uint32_t qa[8][2];
     {
-      const uint4 u0 = *reinterpret_cast<const uint4*>(kst + 16 * c);
-      const uint4 u1 = *reinterpret_cast<const uint4*>(kst + 128 + 16 * c);
-      float f0[8], f1[8];
-      bf16x8_to_f32(u0, f0);
-      bf16x8_to_f32(u1, f1);
+      const uint32_t* qs = reinterpret_cast<const uint32_t*>(smem + kQOff + p * kQBytes);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        kf[e] = f0[e];
-        kf[8 + e] = f1[e];
-      }
-    }
-    float x[kGroup];
-#pragma unroll
-    for (int hh = 0; hh < kGroup; ++hh) {
-      float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-      for (int e = 0; e < 16; e += 2) {
-        s0 = fmaf(qv[hh][e], kf[e], s0);
-        s1 = fmaf(qv[hh][e + 1], kf[e + 1], s1);
-      }
-      x[hh] = s0 + s1;
-    }
-#pragma unroll
-    for (int o = 1; o < 8; o <<= 1) {
-#pragma unroll
-      for (int hh = 0; hh < kGroup; ++hh) x[hh] += __shfl_xor_sync(0xffffffffu, x[hh], o);
-    }
-    const bool valid = (first + i) * kBlk + t < ctx;
-    float p[kGroup];
-#pragma unroll
-    for (int hh = 0; hh < kGroup; ++hh) {
-      if (valid && x[hh] > m[hh] + kRescaleThreshold) {
-        const float alpha = ex2_approx(m[hh] - x[hh]);  // 0 while m = -inf
-        m[hh] = x[hh];
-        l[hh] *= alpha;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) acc[hh][e] *= alpha;
-      }
-      p[hh] = valid ? ex2_approx(x[hh] - m[hh]) : 0.f;
-      l[hh] += p[hh];
-    }
-    const uint8_t* vst = kst + kSlab;
-    {
-      const uint4 u0 = *reinterpret_cast<const uint4*>(vst + 16 * c);
-      const uint4 u1 = *reinterpret_cast<const uint4*>(vst + 128 + 16 * c);
-      float f0[8], f1[8];
-      bf16x8_to_f32(u0, f0);
-      bf16x8_to_f32(u1, f1);
-#pragma unroll
-      for (int hh = 0; hh < kGroup; ++hh) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          acc[hh][e] = fmaf(p[hh], f0[e], acc[hh][e]);
-          acc[hh][8 + e] = fmaf(p[hh], f1[e], acc[hh][8 + e]);
-        }
+      for (int ks = 0; ks < 8; ++ks) {
+        qa[ks][0] = real ? qs[(g * kD + 16 * ks + 2 * qd) >> 1] : 0u;
+        qa[ks][1] = real ? qs[(g * kD + 16 * ks + 8 + 2 * qd) >> 1] : 0u;
       }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(empty(s));
-  }
-
-  // ---- merge the 16 token-slot states (same logsumexp rule as the combine)
-  float* red = reinterpret_cast<float*>(smem + kRedOff);   // [2][4 warps][4 heads]
-  float mw[kGroup];
+    if (lane == 0) mbar_arrive(qempty(p));
+    float o[16][4];                     // O rows g (head) / g+8 (padding), columns 8n + 2q, +1
 #pragma unroll
-  for (int hh = 0; hh < kGroup; ++hh) {
-    float v = m[hh];
-    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-    mw[hh] = v;
-  }
-  if (lane == 0) {
+    for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;   // per head (quad-uniform m, per-thread partial l)
+    bool ok = true;
+    for (int i = warp; i < nb; i += kComputeWarps) {
+      const long long gi = gb + i;
+      const int s = static_cast<int>(gi % kStages);
+      ok = __all_sync(0xffffffffu, mbar_wait(full(s), static_cast<uint32_t>((gi / kStages) & 1),
+                                             a.err, kSiteFull, abort_flag));
+      if (!ok) break;
+      const uint32_t st = sbase + kRingOff + s * kStageBytes;
+      // ---- S (heads x 16 tokens) = Q K^T, two n-tiles of 8 tokens
+      float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-    for (int hh = 0; hh < kGroup; ++hh) red[warp * 4 + hh] = mw[hh];
-  }
-  asm volatile("bar.sync 1, 128;" ::: "memory");
-  float M[kGroup], w[kGroup];
+      for (int ks = 0; ks < 8; ++ks) {
+        const int unit = 2 * (ks & 3) + (mi & 1);
+        const uint32_t addr = st + (ks >> 2) * kBox + k_tok * 128 + ((unit ^ (k_tok & 7)) << 4);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(addr, b0, b1, b2, b3);
+        mma_bf16(sc[0], qa[ks][0], 0u, qa[ks][1], 0u, b0, b1);
+        mma_bf16(sc[1], qa[ks][0], 0u, qa[ks][1], 0u, b2, b3);
+      }
+      // ---- online softmax over the block's tokens (exp2 units)
+      float x[4];
+      const int tok0 = i * kBlk + 2 * qd;
+      x[0] = (tok0 < rem) ? sc[0][0] * a.scale_log2 : -INFINITY;
+      x[1] = (tok0 + 1 < rem) ? sc[0][1] * a.scale_log2 : -INFINITY;
+      x[2] = (tok0 + 8 < rem) ? sc[1][0] * a.scale_log2 : -INFINITY;
+      x[3] = (tok0 + 9 < rem) ? sc[1][1] * a.scale_log2 : -INFINITY;
+      float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      if (mx > m_run + kRescaleThreshold) {   // quad-uniform
+        const float alpha = ex2_approx(m_run - mx);  // 0 while m_run = -inf
+        m_run = mx;
+        l_run *= alpha;
 #pragma unroll
-  for (int hh = 0; hh < kGroup; ++hh) {
-    M[hh] = fmaxf(fmaxf(red[hh], red[4 + hh]), fmaxf(red[8 + hh], red[12 + hh]));
-    w[hh] = (m[hh] == -INFINITY) ? 0.f : ex2_approx(m[hh] - M[hh]);
-    float lv = l[hh] * w[hh];
-    lv += __shfl_xor_sync(0xffffffffu, lv, 8);
-    lv += __shfl_xor_sync(0xffffffffu, lv, 16);
-    mw[hh] = lv;
-  }
-  if (lane == 0) {
+        for (int n = 0; n < 16; ++n) {
+          o[n][0] *= alpha;
+          o[n][1] *= alpha;
+        }
+      }
+      const float mu = (m_run == -INFINITY) ? 0.f : m_run;
+      float pv[4];
 #pragma unroll
-    for (int hh = 0; hh < kGroup; ++hh) red[16 + warp * 4 + hh] = mw[hh];
-  }
-  // every stage has been consumed: the ring can hold the [16 slots][4][128] sums
-  float* slot = reinterpret_cast<float*>(smem + kRingOff);
+      for (int e = 0; e < 4; ++e) pv[e] = real ? ex2_approx(x[e] - mu) : 0.f;
+      l_run += (pv[0] + pv[1]) + (pv[2] + pv[3]);
+      const uint32_t pa0 = pack_bf16x2(pv[0], pv[1]);   // P[g][2q, 2q+1]
+      const uint32_t pa2 = pack_bf16x2(pv[2], pv[3]);   // P[g][8 + 2q, +1]
+      // ---- O (heads x 128) += P V, 16 n-tiles of 8 columns
 #pragma unroll
-  for (int hh = 0; hh < kGroup; ++hh) {
-    float4* dst0 = reinterpret_cast<float4*>(slot + (t * kGroup + hh) * kD + 8 * c);
-    float4* dst1 = reinterpret_cast<float4*>(slot + (t * kGroup + hh) * kD + 64 + 8 * c);
-    const float ww = w[hh];
-    dst0[0] = make_float4(acc[hh][0] * ww, acc[hh][1] * ww, acc[hh][2] * ww, acc[hh][3] * ww);
-    dst0[1] = make_float4(acc[hh][4] * ww, acc[hh][5] * ww, acc[hh][6] * ww, acc[hh][7] * ww);
-    dst1[0] = make_float4(acc[hh][8] * ww, acc[hh][9] * ww, acc[hh][10] * ww, acc[hh][11] * ww);
-    dst1[1] = make_float4(acc[hh][12] * ww, acc[hh][13] * ww, acc[hh][14] * ww, acc[hh][15] * ww);
-  }
-  asm volatile("bar.sync 1, 128;" ::: "memory");
-  if (!ok) return;
-  const int dcol = tid;  // 0..127
+      for (int j = 0; j < 8; ++j) {
+        const int nt = 2 * j + (mi >> 1);          // n-tile of this lane's matrix
+        const uint32_t addr = st + kSlab + (nt >> 3) * kBox + v_tok * 128 +
+                              (((nt & 7) ^ (v_tok & 7)) << 4);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(addr, b0, b1, b2, b3);
+        mma_bf16(o[2 * j], pa0, 0u, pa2, 0u, b0, b1);
+        mma_bf16(o[2 * j + 1], pa0, 0u, pa2, 0u, b2, b3);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty(s));
+    }
+    gb += nb;
+    // The merge below synchronises the 128 compute threads through an mbarrier
+    // with bounded waits (never bar.sync): if a warp gave up above, the others
+    // give up at their next sync instead of waiting for it forever.
+    if (!__all_sync(0xffffffffu, ok)) break;
+    // ---- merge the four warps' states (logsumexp rule)
+    float lq = l_run;
+    lq += __shfl_xor_sync(0xffffffffu, lq, 1);
+    lq += __shfl_xor_sync(0xffffffffu, lq, 2);
+    if (real && qd == 0) {
+      red[warp * 4 + g] = m_run;
+      red[16 + warp * 4 + g] = lq;
+    }
+    if (real) {
 #pragma unroll
-  for (int hh = 0; hh < kGroup; ++hh) {
-    const float lt = red[16 + hh] + red[20 + hh] + red[24 + hh] + red[28 + hh];
-    float sum = 0.f;
+      for (int n = 0; n < 16; ++n)
+        *reinterpret_cast<float2*>(mrg + (warp * kGroup + g) * kD + 8 * n + 2 * qd) =
+            make_float2(o[n][0], o[n][1]);
+    }
+    if (!sync128()) break;
+    {
+      const int dcol = tid;            // 0..127
 #pragma unroll
-    for (int ts = 0; ts < kBlk; ++ts) sum += slot[(ts * kGroup + hh) * kD + dcol];
-    const size_t row = (static_cast<size_t>(seq) * a.Hq + h0 + hh) * a.max_splits + split;
-    a.part_o[row * kD + dcol] = sum / lt;
-    if (dcol == 0) a.part_l[row] = (M[hh] + log2f(lt)) * 0.6931471805599453f;
+      for (int hh = 0; hh < kGroup; ++hh) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kComputeWarps; ++w) M = fmaxf(M, red[w * 4 + hh]);
+        float lt = 0.f, sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kComputeWarps; ++w) {
+          const float mw = red[w * 4 + hh];
+          const float wgt = (mw == -INFINITY) ? 0.f : ex2_approx(mw - M);
+          lt += red[16 + w * 4 + hh] * wgt;
+          sum += mrg[(w * kGroup + hh) * kD + dcol] * wgt;
+        }
+        const size_t row = (static_cast<size_t>(seq) * a.Hq + kvh * kGroup + hh) * a.max_splits + split;
+        a.part_o[row * kD + dcol] = sum / lt;
+        if (dcol == 0) a.part_l[row] = (M + log2f(lt)) * 0.6931471805599453f;
+      }
+    }
+    if (!sync128()) break;             // red / merge buffer are reused by the next item
   }
 }
 
@@ -313,7 +413,8 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(DecodeArgs a) {
 
 int decode_split_blocks() { return 64; }
 
-cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
+cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a,
+                          cudaStream_t stream) {
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -324,8 +425,17 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     attr_set[dev] = true;
   }
   if (a.split_blocks > kMaxSplitBlocks) return cudaErrorInvalidValue;
-  dim3 g1(a.max_splits, a.Hkv, a.num_seqs);
-  decode_split_kernel<<<g1, kThreads, kSmemBytes, stream>>>(a);
+  static int sms[64] = {};
+  if (dev < 64 && sms[dev] == 0) {
+    cudaError_t e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+  }
+  const long long total = static_cast<long long>(a.max_splits) * a.Hkv * a.num_seqs;
+  const long long want = 2ll * (dev < 64 ? sms[dev] : 148);   // two resident CTAs per SM
+  const int g1 = static_cast<int>(total < want ? total : want);
+  cudaError_t ez = cudaMemsetAsync(a.counter, 0, sizeof(unsigned int), stream);
+  if (ez != cudaSuccess) return ez;
+  decode_split_kernel<<<g1, kThreads, kSmemBytes, stream>>>(tk, tv, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   dim3 g2(a.Hq, a.num_seqs);
@@ -338,9 +448,9 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
 // file-scope device array instead of a caller-provided workspace, for callers
 // that must not allocate device memory. Every GPU that loads the library holds
 // it (kDecodeScratchBytes) until the process exits. All calls share it: calls
-// that overlap on the GPU race on it. Nothing needs clearing between calls,
-// because the combine kernel only reads partials the split kernel of the same
-// call has just written.
+// that overlap on the GPU race on it. The launcher clears the work counter
+// (the only part that must start at zero) on every call, and the combine
+// kernel only reads partials the split kernel of the same call has written.
 constexpr size_t kDecodeScratchBytes = size_t(16) << 20;   // 16 MiB
 static __device__ __align__(256) uint8_t g_decode_scratch[kDecodeScratchBytes];
 

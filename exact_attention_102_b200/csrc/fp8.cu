@@ -143,7 +143,7 @@ struct F8 {
 constexpr float kRescaleThreshold = 0.0f;
 constexpr float kPScale = 256.0f;
 enum : uint32_t {
-  kSQ = 0x41, kSKE = 0x42, kSKF = 0x43, kSS = 0x44, kSP = 0x45, kSO = 0x46, kSEpi = 0x47,
+  kSQ = 0x41, kSKE = 0x42, kSKF = 0x43, kSS = 0x44, kSP = 0x45, kSEpi = 0x47,
   kSDrain = 0x48
 };
 
@@ -238,56 +238,63 @@ fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (lane == 0) {
       constexpr uint32_t idS = idesc_e4m3(128, C::BN, 0, 0);
       constexpr uint32_t idPV = idesc_e4m3(128, kD, 0, 1);
+      // Issue order per key block j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1)
+      // (tcgen05.mma from one thread executes in issue order; see fwd.cu).
       int it = 0;
       int npv[2] = {0, 0};
       bool ok = mbar_wait(bar(C::B_Q), 0, a.err, kSQ, abort_flag);
-      for (int j = 0; j < nkb_cta && ok; ++j) {
-        {
-          const int s = it % C::NSTAGE;
-          ok = mbar_wait(bar(C::B_KVF + s), (it / C::NSTAGE) & 1, a.err, kSKF, abort_flag);
-          if (!ok) break;
-          ++it;
+      auto issue_s = [&](int t, uint32_t kb) {
+        const uint32_t qb = base + C::Q_OFF + t * C::TILE;
+#pragma unroll
+        for (int kk = 0; kk < kD / 32; ++kk)   // K = 32 e4m3 elements = 32 bytes per MMA
+          umma_f8_ss(tmem + C::s_col(t), smem_desc_sw128(qb + kk * 32, 16, 1024),
+                     smem_desc_sw128(kb + kk * 32, 16, 1024), idS, kk > 0);
+        umma_commit(bar(C::B_S + t));
+      };
+      if (ok && nkb_cta > 0) {
+        const int s = it % C::NSTAGE;
+        ok = mbar_wait(bar(C::B_KVF + s), (it / C::NSTAGE) & 1, a.err, kSKF, abort_flag);
+        ++it;
+        if (ok) {
           tc_fence_after();
-          const uint32_t kb = base + C::RING_OFF + s * C::TILE;
-          for (int t = 0; t < 2; ++t) {
-            if (j >= nkb_t[t]) continue;
-            if (npv[t] > 0) {
-              ok = mbar_wait(bar(C::B_O + t), (npv[t] - 1) & 1, a.err, kSO, abort_flag);
+          for (int t = 0; t < 2; ++t)
+            if (nkb_t[t] > 0) issue_s(t, base + C::RING_OFF + s * C::TILE);
+          umma_commit(bar(C::B_KVE + s));
+        }
+      }
+      for (int j = 0; j < nkb_cta && ok; ++j) {
+        const int sv = it % C::NSTAGE;
+        ok = mbar_wait(bar(C::B_KVF + sv), (it / C::NSTAGE) & 1, a.err, kSKF, abort_flag);
+        if (!ok) break;
+        ++it;
+        const uint32_t vb = base + C::RING_OFF + sv * C::TILE;
+        int sk = -1;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (j >= nkb_t[t]) continue;
+          ok = mbar_wait(bar(C::B_P + t), npv[t] & 1, a.err, kSP, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < C::BN / 32; ++kk)   // 32 keys = 8 TMEM columns of packed e4m3 P
+            umma_f8_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8,
+                       smem_desc_sw128(vb + kk * 4096, 16, 1024), idPV,
+                       (npv[t] > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(bar(C::B_O + t));
+          ++npv[t];
+          if (j + 1 < nkb_t[t]) {
+            if (sk < 0) {
+              sk = it % C::NSTAGE;
+              ok = mbar_wait(bar(C::B_KVF + sk), (it / C::NSTAGE) & 1, a.err, kSKF, abort_flag);
+              ++it;
               if (!ok) break;
               tc_fence_after();
             }
-            const uint32_t qb = base + C::Q_OFF + t * C::TILE;
-#pragma unroll
-            for (int kk = 0; kk < kD / 32; ++kk)   // K = 32 e4m3 elements = 32 bytes per MMA
-              umma_f8_ss(tmem + C::s_col(t), smem_desc_sw128(qb + kk * 32, 16, 1024),
-                         smem_desc_sw128(kb + kk * 32, 16, 1024), idS, kk > 0);
-            umma_commit(bar(C::B_S + t));
+            issue_s(t, base + C::RING_OFF + sk * C::TILE);
           }
-          if (!ok) break;
-          umma_commit(bar(C::B_KVE + s));
         }
-        {
-          const int s = it % C::NSTAGE;
-          ok = mbar_wait(bar(C::B_KVF + s), (it / C::NSTAGE) & 1, a.err, kSKF, abort_flag);
-          if (!ok) break;
-          ++it;
-          const uint32_t vb = base + C::RING_OFF + s * C::TILE;
-          for (int t = 0; t < 2; ++t) {
-            if (j >= nkb_t[t]) continue;
-            ok = mbar_wait(bar(C::B_P + t), npv[t] & 1, a.err, kSP, abort_flag);
-            if (!ok) break;
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < C::BN / 32; ++kk)   // 32 keys = 8 TMEM columns of packed e4m3 P
-              umma_f8_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8,
-                         smem_desc_sw128(vb + kk * 4096, 16, 1024), idPV,
-                         (npv[t] > 0 || kk > 0) ? 1u : 0u);
-            umma_commit(bar(C::B_O + t));
-            ++npv[t];
-          }
-          if (!ok) break;
-          umma_commit(bar(C::B_KVE + s));
-        }
+        if (!ok) break;
+        umma_commit(bar(C::B_KVE + sv));
+        if (sk >= 0) umma_commit(bar(C::B_KVE + sk));
       }
       umma_commit(bar(C::B_DRAIN));
       mbar_wait(bar(C::B_DRAIN), 0, a.err, kSDrain, nullptr, 200000000ull);

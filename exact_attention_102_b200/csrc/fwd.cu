@@ -68,7 +68,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 // wait-site ids (reported in the device error word)
 enum : uint32_t {
-  kSiteQ = 1, kSiteKvEmpty = 2, kSiteKvFull = 3, kSiteS = 4, kSiteP = 5, kSiteO = 6,
+  kSiteQ = 1, kSiteKvEmpty = 2, kSiteKvFull = 3, kSiteS = 4, kSiteP = 5,
   kSiteEpi = 7, kSiteDrain = 8
 };
 
@@ -167,61 +167,69 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     if (lane == 0) {
       constexpr uint32_t idS = idesc_f16(128, C::BN, 1, 0, 0);
       constexpr uint32_t idPV = idesc_f16(128, D, 1, 0, 1);
+      // Issue order per key block j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1).
+      // tcgen05.mma from one thread executes in issue order, so S_t(j+1) may
+      // overwrite the P_t(j) columns PV_t(j) reads without waiting for it;
+      // the commit after S_t(j+1) also tells the softmax that PV_t(j) is done
+      // (its O rescale for block j+1 relies on that).
       int it = 0;
       int npv[2] = {0, 0};
       bool ok = mbar_wait(bar(C::B_Q), 0, a.err, kSiteQ, abort_flag);
-      for (int j = 0; j < nkb_cta && ok; ++j) {
-        // ---- S_t = Q_t K_j^T
-        {
-          const int s = it % C::NSTAGE;
-          ok = mbar_wait(bar(C::B_KVF + s), (it / C::NSTAGE) & 1, a.err, kSiteKvFull, abort_flag);
-          if (!ok) break;
-          ++it;
+      auto issue_s = [&](int t, uint32_t kb) {
+        const uint32_t qb = base + C::Q_OFF + t * C::TILE;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
+          umma_f16_ss(tmem + C::s_col(t), smem_desc_sw128(qb + off, 16, 1024),
+                      smem_desc_sw128(kb + off, 16, 1024), idS, kk > 0);
+        }
+        umma_commit(bar(C::B_S + t));
+      };
+      if (ok && nkb_cta > 0) {        // K_0
+        const int s = it % C::NSTAGE;
+        ok = mbar_wait(bar(C::B_KVF + s), (it / C::NSTAGE) & 1, a.err, kSiteKvFull, abort_flag);
+        ++it;
+        if (ok) {
           tc_fence_after();
-          const uint32_t kb = base + C::RING_OFF + s * C::TILE;
-          for (int t = 0; t < 2; ++t) {
-            if (j >= nkb_t[t]) continue;
-            if (npv[t] > 0) {  // P_t of block j-1 must be consumed before S_t is overwritten
-              ok = mbar_wait(bar(C::B_O + t), (npv[t] - 1) & 1, a.err, kSiteO, abort_flag);
+          for (int t = 0; t < 2; ++t)
+            if (nkb_t[t] > 0) issue_s(t, base + C::RING_OFF + s * C::TILE);
+          umma_commit(bar(C::B_KVE + s));
+        }
+      }
+      for (int j = 0; j < nkb_cta && ok; ++j) {
+        const int sv = it % C::NSTAGE;  // V_j
+        ok = mbar_wait(bar(C::B_KVF + sv), (it / C::NSTAGE) & 1, a.err, kSiteKvFull, abort_flag);
+        if (!ok) break;
+        ++it;
+        const uint32_t vb = base + C::RING_OFF + sv * C::TILE;
+        int sk = -1;                    // ring stage of K_{j+1}, once waited for
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (j >= nkb_t[t]) continue;
+          ok = mbar_wait(bar(C::B_P + t), npv[t] & 1, a.err, kSiteP, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < C::BN / 16; ++kk)
+            umma_f16_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8,
+                        smem_desc_sw128(vb + kk * 2048, C::CHUNK, 1024), idPV,
+                        (npv[t] > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(bar(C::B_O + t));
+          ++npv[t];
+          if (j + 1 < nkb_t[t]) {
+            if (sk < 0) {
+              sk = it % C::NSTAGE;
+              ok = mbar_wait(bar(C::B_KVF + sk), (it / C::NSTAGE) & 1, a.err, kSiteKvFull,
+                             abort_flag);
+              ++it;
               if (!ok) break;
               tc_fence_after();
             }
-            const uint32_t qb = base + C::Q_OFF + t * C::TILE;
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-              umma_f16_ss(tmem + C::s_col(t), smem_desc_sw128(qb + off, 16, 1024),
-                          smem_desc_sw128(kb + off, 16, 1024), idS, kk > 0);
-            }
-            umma_commit(bar(C::B_S + t));
+            issue_s(t, base + C::RING_OFF + sk * C::TILE);
           }
-          if (!ok) break;
-          umma_commit(bar(C::B_KVE + s));
         }
-        // ---- O_t += P_t V_j
-        {
-          const int s = it % C::NSTAGE;
-          ok = mbar_wait(bar(C::B_KVF + s), (it / C::NSTAGE) & 1, a.err, kSiteKvFull, abort_flag);
-          if (!ok) break;
-          ++it;
-          const uint32_t vb = base + C::RING_OFF + s * C::TILE;
-          for (int t = 0; t < 2; ++t) {
-            if (j >= nkb_t[t]) continue;
-            ok = mbar_wait(bar(C::B_P + t), npv[t] & 1, a.err, kSiteP, abort_flag);
-            if (!ok) break;
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < C::BN / 16; ++kk) {
-              umma_f16_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8,
-                          smem_desc_sw128(vb + kk * 2048, C::CHUNK, 1024), idPV,
-                          (npv[t] > 0 || kk > 0) ? 1u : 0u);
-            }
-            umma_commit(bar(C::B_O + t));
-            ++npv[t];
-          }
-          if (!ok) break;
-          umma_commit(bar(C::B_KVE + s));
-        }
+        if (!ok) break;
+        umma_commit(bar(C::B_KVE + sv));             // V_j: both PV_t(j) issued before
+        if (sk >= 0) umma_commit(bar(C::B_KVE + sk));  // K_{j+1}: both S_t(j+1) issued before
       }
       // drain every MMA this thread issued before TMEM is released
       umma_commit(bar(C::B_DRAIN));
@@ -303,7 +311,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       lr_run = lr_run * alpha + (r0 + r1);
       tmem_st32(s_addr, pk0);
       tmem_st32(s_addr + 32, pk1);
-      // O rescale (PV of block j-1 has completed: S_t(j) was issued after it)
+      // O rescale (PV of block j-1 has completed: S_t(j)'s commit covers it)
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {

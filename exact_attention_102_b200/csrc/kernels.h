@@ -60,12 +60,14 @@ struct DecodeArgs {
   float* lse;               // fp32 [S][Hq] or null
   float* part_o;            // fp32 [S][Hq][max_splits][d]
   float* part_l;            // fp32 [S][Hq][max_splits]
+  unsigned int* counter;    // work-item counter (zeroed by the launcher)
   int num_seqs, Hq, Hkv, max_blocks, max_ctx, max_splits, split_blocks;
   float scale_log2;
   uint32_t* err;
 };
 
-cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a,
+                          cudaStream_t stream);
 
 struct Fp8PrepArgs {
   const void* q;      // bf16 BHND

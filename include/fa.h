@@ -117,8 +117,8 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
 
 /*
  * Bytes of device workspace paged_attn_decode needs for split partials
- * (fp32 O and L per (sequence, query head, split)) when no sequence is
- * longer than max_ctx tokens.
+ * (fp32 O and L per (sequence, query head, split)) and a work counter, when
+ * no sequence is longer than max_ctx tokens.
  */
 FA_API size_t paged_attn_decode_workspace_bytes(int num_seqs, int Hq, int d, int max_ctx);
 
@@ -176,10 +176,11 @@ FA_API fa_status paged_attn_decode(const void* q, const void* k_cache, const voi
  *   - The first call on a device looks up the array's device address (once
  *     per device, with that device current); make that first call before any
  *     stream capture.
- *   - All calls share the array and it keeps the last call's contents (no
- *     clearing is needed: every partial read was written by the same call).
- *     Calls that overlap on the GPU (different streams, or several host
- *     threads) race on it and must be serialised by the caller.
+ *   - All calls share the array and it keeps the last call's contents. Each
+ *     call clears what must start at zero (its work counter) itself, and every
+ *     partial it reads was written by the same call. Calls that overlap on
+ *     the GPU (different streams, or several host threads) race on it and
+ *     must be serialised by the caller.
  */
 FA_API fa_status paged_attn_decode_noalloc(const void* q, const void* k_cache,
                                            const void* v_cache, int num_phys_blocks,

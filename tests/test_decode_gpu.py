@@ -152,3 +152,14 @@ def test_optional_lse_and_guard_regions():
     assert torch.all(wbuf[:pad] == 0x5A) and torch.all(wbuf[-pad:] == 0x5A)
     o_ref, _ = _oracle_for(list(range(S)), lay, q, kc, vc)
     assert_bf16_close(f64(o), o_ref, O_TOL, "O")
+
+
+def test_many_items_per_cta():
+    """More work items than resident CTAs (each CTA walks several items,
+    with empty splits in between): every sequence checked."""
+    lay, q, kc, vc = _inputs(40, 1, 5000, 94)
+    o, lse = _run(lay, q, kc, vc, max_ctx=5000)
+    seqs = list(range(40))
+    o_ref, l_ref = _oracle_for(seqs, lay, q, kc, vc)
+    assert_bf16_close(f64(o), o_ref, O_TOL, "O")
+    assert_lse_close(f64(lse), l_ref)
