@@ -55,9 +55,10 @@ EncodeTiledFn encode_fn() {
 }
 
 // 3-D view [BH][N][d] of a BHND tensor, box (box_x elements, box_y rows, 1),
-// 128-byte swizzle, zero fill outside the tensor.
+// 128-byte swizzle unless told otherwise, zero fill outside the tensor.
 bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int elem_bytes, int d,
-              int n, int bh, uint32_t box_x, uint32_t box_y) {
+              int n, int bh, uint32_t box_x, uint32_t box_y,
+              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n),
@@ -68,7 +69,7 @@ bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int elem_
   cuuint32_t es[3] = {1, 1, 1};
   memset(m, 0, sizeof(*m));
   CUresult r = fn(m, dt, 3, const_cast<void*>(ptr), dims, strides, box, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -163,13 +164,15 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   void* k16 = w16 + tsz;
   void* v16 = w16 + 2 * tsz;
   void* do16 = w16 + 3 * tsz;
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tdq;
   // d = 128 steps over 64 queries at a time (64-row Q / dO boxes), d = 64 over 128
   const uint32_t qrows = d == 128 ? 64 : 128;
   if (!make_map(&tq, q16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, qrows) ||
       !make_map(&tk, k16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, 128) ||
       !make_map(&tv, v16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, 128) ||
-      !make_map(&tdo, do16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, qrows))
+      !make_map(&tdo, do16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, qrows) ||
+      !make_map(&tdq, dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, N, bh, 32, 64,
+                CU_TENSOR_MAP_SWIZZLE_NONE))
     return FA_ERR_LAUNCH;
   fa::BwdArgs a;
   a.q16 = q16;
@@ -197,8 +200,8 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   a.scale_log2 = a.scale * kLog2e;
   a.err = err;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = (d == 128) ? fa::launch_bwd<128>(tq, tk, tv, tdo, a, s)
-                             : fa::launch_bwd<64>(tq, tk, tv, tdo, a, s);
+  cudaError_t e = (d == 128) ? fa::launch_bwd<128>(tq, tk, tv, tdo, tdq, a, s)
+                             : fa::launch_bwd<64>(tq, tk, tv, tdo, tdq, a, s);
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 

@@ -197,13 +197,13 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     mbar_init(bar(C::B_ST), 1);
     mbar_init(bar(C::B_DPT), 1);
-    mbar_init(bar(C::B_P), 128);
-    mbar_init(bar(C::B_PR), 128);
+    mbar_init(bar(C::B_P), 4);      // one arrival per warp
+    mbar_init(bar(C::B_PR), 4);
     mbar_init(bar(C::B_DV), 1);
-    mbar_init(bar(C::B_DS), 128);
+    mbar_init(bar(C::B_DS), 4);
     mbar_init(bar(C::B_DSFREE), 1);
     mbar_init(bar(C::B_DQ), 1);
-    mbar_init(bar(C::B_DQFREE), 128);
+    mbar_init(bar(C::B_DQFREE), 4);
     mbar_init(bar(C::B_END), 1);
     mbar_init(bar(C::B_DRAIN), 1);
     *abort_flag = 0;
@@ -393,7 +393,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(C::B_P));
+      warp_arrive(bar(C::B_P));
     }
     tc_fence_before();
   } else if (warp >= 8 && warp < 12) {
@@ -416,7 +416,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tmem_ld32(st_addr + 32, pk1);
       tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(bar(C::B_PR));                     // S^T(it+1) may now overwrite P^T(it)
+      warp_arrive(bar(C::B_PR));                     // S^T(it+1) may now overwrite P^T(it)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_DPT), it & 1, a.err, kSiteDPT, abort_flag));
       if (!ok) break;
       if (it > 0) {  // dS buffer reusable once dK(it-1) and dQ(it-1) have read it
@@ -464,7 +464,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (!(ds_max < 65504.f)) atomicCAS(a.err, 0u, kErrRange + 2);
       fence_async_smem();   // generic-proxy smem writes -> visible to the MMA
       tc_fence_before();
-      mbar_arrive(bar(C::B_DS));
+      warp_arrive(bar(C::B_DS));
     }
     // ---- epilogue: dV and dK rows (thread = key) to HBM
     if (ok) {
@@ -521,7 +521,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
       }
       tc_fence_before();
-      mbar_arrive(bar(C::B_DQFREE));
+      warp_arrive(bar(C::B_DQFREE));
     }
     tc_fence_before();
   }
@@ -535,15 +535,27 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 }
 
 // ------------------------------------------------- main pass, d = 128 -----
-// Same method, tiled for d = 128's TMEM budget with 64-query steps so that the
-// dQ tile gets its own double-buffered TMEM region and never blocks the next
-// step's dP^T:
-//   TMEM: S^T/P^T [0,64)  dP^T [64,128)  dQ^T x2 [128,256)  dV [256,384)
-//         dK [384,512)
-//   dQ is produced transposed, dQ^T = K^T dS^T (M = d = 128 lanes, N = 64
-//   queries), so the drain warps (thread = one head-dim column) issue
-//   reductions that are contiguous across a warp (32 consecutive floats).
-struct BwdQ64 {
+// Same method, tiled for d = 128 around what the tensor core does fastest: an
+// MMA whose A operand sits in TMEM runs at the full rate for N = 128, one whose
+// A operand is read from shared memory costs about twice as long for N <= 128.
+// Steps of 64 queries; every operand that can live in TMEM does:
+//   S^T  = K_j Q_i^T      A = K_j   (TMEM, loaded once per CTA), B = Q_i
+//   dP^T = V_j dO_i^T     A = V_j   (shared memory),              B = dO_i
+//   dV  += P^T dO_i       A = P^T   (TMEM, written over S^T),     B = dO_i
+//   dK  += dS^T Q_i       A = dS^T  (TMEM, written over dP^T),    B = Q_i
+//   dQ^T = K_j^T dS^T     A = K_j^T (shared memory, MN-major),    B = dS^T
+// TMEM: K [0,64)  S^T/P^T [64,128)  dP^T/dS^T [128,192)  dQ^T [192,256)
+//       dV [256,384)  dK [384,512)
+// One tcgen05 issuer executes in issue order, so S^T(i+1) may be issued right
+// after dV(i) (which reads P^T(i) from the same columns) and dP^T(i+1) right
+// after dK(i) (which reads dS^T(i)); per step the issue order is
+// dV(i), S^T(i+1) | dK(i), dP^T(i+1), dQ(i).
+// Warps 4..11 (two per TMEM lane quarter, one per 32-query half) compute P
+// and then dS for their half; dS also goes to shared memory (double-buffered)
+// for the dQ product. Warps 12..15 (thread = head-dim column) drain dQ^T to a
+// shared staging tile and add it to dQ in HBM with a TMA tensor reduce-add
+// (one 32-column x 64-row box per warp).
+struct BwdD128 {
   static constexpr int D = 128;
   static constexpr int BK = 128;                 // keys per CTA
   static constexpr int BQ = 64;                  // queries per step
@@ -553,32 +565,41 @@ struct BwdQ64 {
   static constexpr int Q_CHUNK = BQ * 128;
   static constexpr int NS = 3;                   // Q / dO stages
   static constexpr int DS_BYTES = BK * BQ * 2;   // dS^T fp16 [key][64 queries]: one 128 B row per key
+  static constexpr int DQ_STAGE = BQ * 32 * 4;   // one drain warp's fp32 box [64 queries][32 columns]
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = K_OFF + KV_TILE;
   static constexpr int Q_OFF = V_OFF + KV_TILE;
   static constexpr int DO_OFF = Q_OFF + NS * Q_TILE;
-  static constexpr int DS_OFF = DO_OFF + NS * Q_TILE;
-  static constexpr int L_OFF = DS_OFF + DS_BYTES;       // NS x 64 fp32: L * log2(e)
+  static constexpr int DS_OFF = DO_OFF + NS * Q_TILE;   // 2 buffers
+  static constexpr int DQS_OFF = DS_OFF + 2 * DS_BYTES; // 4 staging boxes
+  static constexpr int L_OFF = DQS_OFF + 4 * DQ_STAGE;  // NS x 64 fp32: L * log2(e)
   static constexpr int DL_OFF = L_OFF + NS * 256;       // NS x 64 fp32: D
   static constexpr int BAR_OFF = DL_OFF + NS * 256;
   static constexpr int B_KV = 0, B_QF = 1, B_QE = B_QF + NS, B_DF = B_QE + NS, B_DE = B_DF + NS;
-  static constexpr int B_ST = B_DE + NS, B_DPT = B_ST + 1, B_P = B_DPT + 1, B_PR = B_P + 1;
-  static constexpr int B_DV = B_PR + 1, B_DS = B_DV + 1, B_DSFREE = B_DS + 1;
-  static constexpr int B_DQ = B_DSFREE + 1;            // [2]
-  static constexpr int B_DQFREE = B_DQ + 2;            // [2]
-  static constexpr int B_END = B_DQFREE + 2, B_DRAIN = B_END + 1, NBAR = B_DRAIN + 1;
+  static constexpr int B_KT = B_DE + NS, B_ST = B_KT + 1, B_DPT = B_ST + 1, B_P = B_DPT + 1;
+  static constexpr int B_DS = B_P + 1, B_DSFREE = B_DS + 1;   // [2]
+  static constexpr int B_DQ = B_DSFREE + 2, B_DQFREE = B_DQ + 1;
+  static constexpr int B_END = B_DQFREE + 1, B_DRAIN = B_END + 1, NBAR = B_DRAIN + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
-  static constexpr uint32_t COL_ST = 0, COL_DPT = 64, COL_DQT = 128, COL_DV = 256, COL_DK = 384;
+  static constexpr uint32_t COL_K = 0, COL_S = 64, COL_DP = 128, COL_DQ = 192, COL_DV = 256,
+                            COL_DK = 384;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int THREADS = 512;
 };
+static_assert(BwdD128::SMEM_BYTES <= 232448, "d = 128 backward exceeds shared memory");
+
+// TMEM column of the 16-query group kk of a packed fp16 [key][64 queries]
+// operand whose two 32-query halves start 32 columns apart.
+__device__ __forceinline__ uint32_t half_col(int kk) {
+  return static_cast<uint32_t>((kk >> 1) * 32 + (kk & 1) * 8);
+}
 
 __global__ void __launch_bounds__(512, 1)
-bwd_q64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-               BwdArgs a) {
-  using C = BwdQ64;
+bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                const __grid_constant__ CUtensorMap tmDQ, BwdArgs a) {
+  using C = BwdD128;
   constexpr int D = C::D;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -606,17 +627,15 @@ bwd_q64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_init(bar(C::B_DF + s), 1);
       mbar_init(bar(C::B_DE + s), 1);
     }
+    mbar_init(bar(C::B_KT), 8);     // one arrival per softmax-gradient warp
     mbar_init(bar(C::B_ST), 1);
     mbar_init(bar(C::B_DPT), 1);
-    mbar_init(bar(C::B_P), 128);
-    mbar_init(bar(C::B_PR), 128);
-    mbar_init(bar(C::B_DV), 1);
-    mbar_init(bar(C::B_DS), 128);
+    mbar_init(bar(C::B_P), 8);
+    mbar_init(bar(C::B_DS), 8);
     mbar_init(bar(C::B_DSFREE), 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(C::B_DQ + b), 1);
-      mbar_init(bar(C::B_DQFREE + b), 128);
-    }
+    mbar_init(bar(C::B_DSFREE + 1), 1);
+    mbar_init(bar(C::B_DQ), 1);
+    mbar_init(bar(C::B_DQFREE), 4); // one arrival per drain warp
     mbar_init(bar(C::B_END), 1);
     mbar_init(bar(C::B_DRAIN), 1);
     *abort_flag = 0;
@@ -638,6 +657,7 @@ bwd_q64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmDO);
+      tma_prefetch_desc(&tmDQ);
       mbar_arrive_expect_tx(bar(C::B_KV), 2 * C::KV_TILE);
       for (int c = 0; c < 2; ++c) {
         tma_load_3d(base + C::K_OFF + c * C::KV_CHUNK, &tmK, bar(C::B_KV), c * 64, kb * C::BK, bh);
@@ -674,253 +694,256 @@ bwd_q64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA issue
     if (lane == 0) {
-      constexpr uint32_t idST = idesc_f16(128, C::BQ, 0, 0, 0);  // S^T, dP^T: both K-major
-      constexpr uint32_t idKM = idesc_f16(128, D, 0, 0, 1);      // dV (A tmem), dK (A smem K-major)
+      constexpr uint32_t idS = idesc_f16(128, C::BQ, 0, 0, 0);   // S^T, dP^T: K-major operands
+      constexpr uint32_t idKM = idesc_f16(128, D, 0, 0, 1);      // dV, dK: A tmem, B MN-major
       constexpr uint32_t idQT = idesc_f16(128, C::BQ, 0, 1, 1);  // dQ^T: A = K^T, B = dS^T, MN-major
-      const uint32_t kbase = base + C::K_OFF, vbase = base + C::V_OFF, dsb = base + C::DS_OFF;
-      bool ok = mbar_wait(bar(C::B_KV), 0, a.err, kSiteKV, abort_flag);
-      auto issue_ss = [&](uint32_t d_col, uint32_t abase, uint32_t bbase) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {   // K = d: chunk kk/4, 32 B steps inside it
-          umma_f16_ss(tmem + d_col, smem_desc_sw128(abase + (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32, 16, 1024),
-                      smem_desc_sw128(bbase + (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32, 16, 1024),
-                      idST, kk > 0);
-        }
-      };
-      auto issue_st = [&](int it) -> bool {
+      const uint32_t kbase = base + C::K_OFF, vbase = base + C::V_OFF;
+      bool ok = mbar_wait(bar(C::B_KV), 0, a.err, kSiteKV, abort_flag) &&
+                mbar_wait(bar(C::B_KT), 0, a.err, kSiteKV, abort_flag);
+      auto issue_s = [&](int it) -> bool {
         const int s = it % C::NS;
         if (!mbar_wait(bar(C::B_QF + s), (it / C::NS) & 1, a.err, kSiteQF, abort_flag)) return false;
         tc_fence_after();
-        issue_ss(C::COL_ST, kbase, base + C::Q_OFF + s * C::Q_TILE);
+        const uint32_t qb = base + C::Q_OFF + s * C::Q_TILE;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)   // K = d: chunk kk/4, 32 B steps inside it
+          umma_f16_ts(tmem + C::COL_S, tmem + C::COL_K + kk * 8,
+                      smem_desc_sw128(qb + (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32, 16, 1024), idS,
+                      kk > 0);
         umma_commit(bar(C::B_ST));
         return true;
       };
-      auto issue_dpt = [&](int it) -> bool {
+      auto issue_dp = [&](int it) -> bool {
         const int s = it % C::NS;
         if (!mbar_wait(bar(C::B_DF + s), (it / C::NS) & 1, a.err, kSiteDF, abort_flag)) return false;
         tc_fence_after();
-        issue_ss(C::COL_DPT, vbase, base + C::DO_OFF + s * C::Q_TILE);
+        const uint32_t gb = base + C::DO_OFF + s * C::Q_TILE;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_f16_ss(tmem + C::COL_DP,
+                      smem_desc_sw128(vbase + (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32, 16, 1024),
+                      smem_desc_sw128(gb + (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32, 16, 1024), idS,
+                      kk > 0);
         umma_commit(bar(C::B_DPT));
         return true;
       };
-      if (ok) ok = issue_st(0) && issue_dpt(0);
+      if (ok) {
+        tc_fence_after();
+        ok = issue_s(0) && issue_dp(0);
+      }
       for (int it = 0; it < n_it && ok; ++it) {
         const int s = it % C::NS;
+        const int buf = it & 1;
         const uint32_t qb = base + C::Q_OFF + s * C::Q_TILE;
         const uint32_t gb = base + C::DO_OFF + s * C::Q_TILE;
-        const int buf = it & 1;
-        // dV += P^T dO_it (P^T fp16 pairs in TMEM columns [0, 32))
+        const uint32_t dsb = base + C::DS_OFF + buf * C::DS_BYTES;
+        // dV += P^T dO_it
         ok = mbar_wait(bar(C::B_P), it & 1, a.err, kSiteP, abort_flag);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < C::BQ / 16; ++kk)
-          umma_f16_ts(tmem + C::COL_DV, tmem + C::COL_ST + kk * 8,
+          umma_f16_ts(tmem + C::COL_DV, tmem + C::COL_S + half_col(kk),
                       smem_desc_sw128(gb + kk * 2048, C::Q_CHUNK, 1024), idKM,
                       (it > 0 || kk > 0) ? 1u : 0u);
         if (it + 1 < n_it) {
-          // S^T(it+1) overwrites P^T(it): the dS group must have copied it out;
-          // dV(it), issued earlier by this thread, reads it first (tcgen05.mma
-          // from one thread executes in issue order)
-          ok = mbar_wait(bar(C::B_PR), it & 1, a.err, kSitePR, abort_flag);
-          if (!ok) break;
-          ok = issue_st(it + 1);
+          ok = issue_s(it + 1);          // after dV(it): in-order, so P^T(it) is read first
           if (!ok) break;
         }
+        // dK += dS^T Q_it
         ok = mbar_wait(bar(C::B_DS), it & 1, a.err, kSiteDS, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        // dK += dS^T Q_it: A = dS^T [key][query] K-major, B = Q_it MN-major
 #pragma unroll
         for (int kk = 0; kk < C::BQ / 16; ++kk)
-          umma_f16_ss(tmem + C::COL_DK, smem_desc_sw128(dsb + kk * 32, 16, 1024),
+          umma_f16_ts(tmem + C::COL_DK, tmem + C::COL_DP + half_col(kk),
                       smem_desc_sw128(qb + kk * 2048, C::Q_CHUNK, 1024), idKM,
                       (it > 0 || kk > 0) ? 1u : 0u);
-        // dQ^T_it = K^T dS^T into buffer it&1 (drained two steps ago)
-        if (it >= 2) {
-          ok = mbar_wait(bar(C::B_DQFREE + buf), ((it >> 1) - 1) & 1, a.err, kSiteDQF, abort_flag);
+        umma_commit(bar(C::B_QE + s));   // Q_it and its L: S^T(it), dK(it) done
+        if (it + 1 < n_it) {
+          ok = issue_dp(it + 1);         // after dK(it): dS^T(it) is read first
+          if (!ok) break;
+        }
+        // dQ^T_it = K^T dS^T (the drain warps have read dQ^T(it-1))
+        if (it >= 1) {
+          ok = mbar_wait(bar(C::B_DQFREE), (it - 1) & 1, a.err, kSiteDQF, abort_flag);
           if (!ok) break;
           tc_fence_after();
         }
 #pragma unroll
         for (int kk = 0; kk < C::BK / 16; ++kk)
-          umma_f16_ss(tmem + C::COL_DQT + buf * 64,
-                      smem_desc_sw128(kbase + kk * 2048, C::KV_CHUNK, 1024),
+          umma_f16_ss(tmem + C::COL_DQ, smem_desc_sw128(kbase + kk * 2048, C::KV_CHUNK, 1024),
                       smem_desc_sw128(dsb + kk * 2048, 16, 1024), idQT, kk > 0 ? 1u : 0u);
-        umma_commit(bar(C::B_DQ + buf));
-        umma_commit(bar(C::B_DSFREE));
-        umma_commit(bar(C::B_QE + s));   // Q_it and its L: S^T, P, dK done
-        umma_commit(bar(C::B_DE + s));   // dO_it and its D: dP^T, dV, dS done
-        if (it + 1 < n_it) {
-          ok = issue_dpt(it + 1);        // the dS group has read dP^T(it)
-          if (!ok) break;
-        }
+        umma_commit(bar(C::B_DQ));
+        umma_commit(bar(C::B_DSFREE + buf));
+        umma_commit(bar(C::B_DE + s));   // dO_it and its D: dP^T(it), dV(it) done
       }
       umma_commit(bar(C::B_END));
       umma_commit(bar(C::B_DRAIN));
       mbar_wait(bar(C::B_DRAIN), 0, a.err, kSiteDrain, nullptr, 200000000ull);
     }
-  } else if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------ P^T (thread = key row)
-    const int r = (warp & 3) * 32 + lane;
+  } else if (warp >= 4 && warp < 12) {
+    // ---------- P^T and dS^T for one 32-query half (thread = key row)
+    const int quarter = warp & 3;
+    const int h = (warp - 4) >> 2;
+    const int r = quarter * 32 + lane;
     const int key = kb * C::BK + r;
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t st_addr = tmem + lane_off + C::COL_ST;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t s_addr = tmem + lane_off + C::COL_S + 32 * h;
+    const uint32_t dp_addr = tmem + lane_off + C::COL_DP + 32 * h;
     const float sl2 = a.scale_log2;
-    for (int it = 0; it < n_it; ++it) {
-      const int s = it % C::NS;
-      const int q0 = (i0 + it) * C::BQ;
-      const float* Ls = reinterpret_cast<const float*>(smem + C::L_OFF + s * 256);
-      const bool need_mask = (a.causal && key > q0) || key >= a.N;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(C::B_ST), it & 1, a.err, kSiteST, abort_flag)))
-        break;
-      tc_fence_after();
-      uint32_t sr0[32], sr1[32];
-      tmem_ld32(st_addr, sr0);
-      tmem_ld32(st_addr + 32, sr1);
-      tmem_ld_wait();
-      uint32_t pk[32];
+    bool ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_KV), 0, a.err, kSiteKV, abort_flag));
+    if (ok) {
+      // K row r, head-dim columns [64h, 64h+64): the A operand of S^T, packed
+      // two fp16 per TMEM column like the swizzled shared-memory row it comes from
+      const uint8_t* krow = smem + C::K_OFF + h * C::KV_CHUNK + r * 128;
+      uint32_t kr[32];
 #pragma unroll
-      for (int e = 0; e < 64; e += 4) {
+      for (int u = 0; u < 8; ++u) {
+        const uint4 v = *reinterpret_cast<const uint4*>(krow + ((u ^ (r & 7)) << 4));
+        kr[4 * u] = v.x;
+        kr[4 * u + 1] = v.y;
+        kr[4 * u + 2] = v.z;
+        kr[4 * u + 3] = v.w;
+      }
+      tmem_st32(tmem + lane_off + C::COL_K + 32 * h, kr);
+      tmem_st_wait();
+      tc_fence_before();
+      warp_arrive(bar(C::B_KT));
+    }
+    for (int it = 0; it < n_it && ok; ++it) {
+      const int s = it % C::NS;
+      const int buf = it & 1;
+      const int qh = (i0 + it) * C::BQ + 32 * h;        // first query of this half
+      const float* Ls = reinterpret_cast<const float*>(smem + C::L_OFF + s * 256) + 32 * h;
+      const float* Ds = reinterpret_cast<const float*>(smem + C::DL_OFF + s * 256) + 32 * h;
+      const bool need_mask = (a.causal && key > qh) || key >= a.N;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_ST), it & 1, a.err, kSiteST, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[32];
+      tmem_ld32(s_addr, sr);
+      tmem_ld_wait();
+      uint32_t pk[16];                                 // P^T, fp16 pairs of queries
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) {
         const float4 lv = *reinterpret_cast<const float4*>(Ls + e);
         const float L[4] = {lv.x, lv.y, lv.z, lv.w};
         float p[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const uint32_t sv = (e + u) < 32 ? sr0[e + u] : sr1[e + u - 32];
-          p[u] = ex2_approx(fmaf(__uint_as_float(sv), sl2, -L[u]));
-          if (need_mask && ((a.causal && key > q0 + e + u) || key >= a.N)) p[u] = 0.f;
+          p[u] = ex2_approx(fmaf(__uint_as_float(sr[e + u]), sl2, -L[u]));
+          if (need_mask && ((a.causal && key > qh + e + u) || key >= a.N)) p[u] = 0.f;
         }
         pk[e / 2] = pack_f16x2(p[0], p[1]);
         pk[e / 2 + 1] = pack_f16x2(p[2], p[3]);
       }
-      tmem_st32(st_addr, pk);
+      tmem_st16(s_addr, pk);                           // over this half's own S^T columns
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(C::B_P));
-    }
-    tc_fence_before();
-  } else if (warp >= 8 && warp < 12) {
-    // ---------------------------- dS^T = P^T o (dP^T - D) (thread = key row)
-    const int r = (warp & 3) * 32 + lane;
-    const int key = kb * C::BK + r;
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t st_addr = tmem + lane_off + C::COL_ST;
-    const uint32_t dpt_addr = tmem + lane_off + C::COL_DPT;
-    uint8_t* ds_row = smem + C::DS_OFF + r * 128;     // one swizzled 128-byte row per key
-    bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
-      const int s = it % C::NS;
-      const float* Ds = reinterpret_cast<const float*>(smem + C::DL_OFF + s * 256);
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_P), it & 1, a.err, kSiteP, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t pk[32];                                // P^T(it): fp16 pairs, 64 queries
-      tmem_ld32(st_addr, pk);
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(bar(C::B_PR));
+      warp_arrive(bar(C::B_P));
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_DPT), it & 1, a.err, kSiteDPT, abort_flag));
       if (!ok) break;
-      if (it > 0) {
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait(bar(C::B_DSFREE), (it - 1) & 1, a.err, kSiteDSF, abort_flag));
+      if (it >= 2) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_DSFREE + buf), ((it >> 1) - 1) & 1, a.err,
+                                               kSiteDSF, abort_flag));
         if (!ok) break;
       }
       tc_fence_after();
+      uint32_t dr[32];
+      tmem_ld32(dp_addr, dr);
+      tmem_ld_wait();
+      uint32_t w[16];                                  // dS^T, fp16 pairs of queries
       float ds_max = 0.f;
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {                  // 16 queries at a time
-        uint32_t dr[16];
-        tmem_ld16(dpt_addr + g * 16, dr);
-        tmem_ld_wait();
-        uint32_t w[8];
+      for (int e = 0; e < 32; e += 4) {
+        const float4 dv4 = *reinterpret_cast<const float4*>(Ds + e);
+        const float Dv[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
+        float ds[4];
 #pragma unroll
-        for (int e = 0; e < 16; e += 4) {
-          const float4 dv4 = *reinterpret_cast<const float4*>(Ds + g * 16 + e);
-          const float Dv[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
-          float ds[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int q = g * 16 + e + u;
-            const uint32_t pp = pk[q >> 1];
-            const float pv = (q & 1) ? f16_hi(pp) : f16_lo(pp);
-            ds[u] = pv * (__uint_as_float(dr[e + u]) - Dv[u]);
-          }
-          ds_max = fmaxf(ds_max, fmaxf(fmaxf(fabsf(ds[0]), fabsf(ds[1])),
-                                       fmaxf(fabsf(ds[2]), fabsf(ds[3]))));
-          w[e / 2] = pack_f16x2(ds[0], ds[1]);
-          w[e / 2 + 1] = pack_f16x2(ds[2], ds[3]);
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t pp = pk[(e + u) >> 1];
+          const float pv = ((e + u) & 1) ? f16_hi(pp) : f16_lo(pp);
+          ds[u] = pv * (__uint_as_float(dr[e + u]) - Dv[u]);
         }
-        // queries g*16 .. g*16+15 = 16-byte units 2g, 2g+1 of the key's 128-byte
-        // row, XOR-swizzled with (key row % 8) like a TMA SWIZZLE_128B tile
+        ds_max = fmaxf(ds_max, fmaxf(fmaxf(fabsf(ds[0]), fabsf(ds[1])),
+                                     fmaxf(fabsf(ds[2]), fabsf(ds[3]))));
+        w[e / 2] = pack_f16x2(ds[0], ds[1]);
+        w[e / 2 + 1] = pack_f16x2(ds[2], ds[3]);
+      }
+      tmem_st16(dp_addr, w);                           // A operand of dK, over own dP^T columns
+      // shared memory copy for dQ: this half's 64 bytes of the key's 128-byte
+      // row, XOR-swizzled with (key row % 8) like a TMA SWIZZLE_128B tile
+      uint8_t* ds_row = smem + C::DS_OFF + buf * C::DS_BYTES + r * 128;
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          uint4* dst = reinterpret_cast<uint4*>(ds_row + (((2 * g + u) ^ (r & 7)) << 4));
-          *dst = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
-        }
+      for (int u = 0; u < 4; ++u) {
+        uint4* dst = reinterpret_cast<uint4*>(ds_row + (((4 * h + u) ^ (r & 7)) << 4));
+        *dst = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
       }
       if (!(ds_max < 65504.f)) atomicCAS(a.err, 0u, kErrRange + 2);
+      tmem_st_wait();
       fence_async_smem();
       tc_fence_before();
-      mbar_arrive(bar(C::B_DS));
+      warp_arrive(bar(C::B_DS));
     }
-    // ---- epilogue: dV and dK rows (thread = key) to HBM
+    // ---- epilogue: dV rows (half 0) or dK rows (half 1), thread = key
     if (ok) {
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_END), 0, a.err, kSiteEnd, abort_flag));
       if (ok) {
         tc_fence_after();
         const size_t orow = (static_cast<size_t>(bh) * a.N + key) * D;
+        const uint32_t src = tmem + lane_off + (h ? C::COL_DK : C::COL_DV);
+        float* dst = (h ? a.dk : a.dv) + orow;
+        const float mul = h ? a.scale : 1.f;
 #pragma unroll
-        for (int which = 0; which < 2; ++which) {
-          const uint32_t src = tmem + lane_off + (which ? C::COL_DK : C::COL_DV);
-          float* dst = (which ? a.dk : a.dv) + orow;
-          const float mul = which ? a.scale : 1.f;
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(src + c * 32, v);
+          tmem_ld_wait();
+          if (key < a.N) {
+            float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t v[32];
-            tmem_ld32(src + c * 32, v);
-            tmem_ld_wait();
-            if (key < a.N) {
-              float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
-#pragma unroll
-              for (int e = 0; e < 8; ++e)
-                d4[e] = make_float4(__uint_as_float(v[4 * e]) * mul, __uint_as_float(v[4 * e + 1]) * mul,
-                                    __uint_as_float(v[4 * e + 2]) * mul,
-                                    __uint_as_float(v[4 * e + 3]) * mul);
-            }
+            for (int e = 0; e < 8; ++e)
+              d4[e] = make_float4(__uint_as_float(v[4 * e]) * mul, __uint_as_float(v[4 * e + 1]) * mul,
+                                  __uint_as_float(v[4 * e + 2]) * mul,
+                                  __uint_as_float(v[4 * e + 3]) * mul);
           }
         }
       }
     }
     tc_fence_before();
   } else if (warp >= 12) {
-    // ------------------------ dQ^T tile -> HBM (thread = one head-dim column)
-    const int c = (warp & 3) * 32 + lane;            // TMEM lane = d index
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    // ------------- dQ^T tile -> HBM (thread = one head-dim column) via TMA
+    const int quarter = warp & 3;                    // TMEM lanes = d [32 quarter, 32 quarter + 32)
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const float sc = a.scale;
+    float* stage = reinterpret_cast<float*>(smem + C::DQS_OFF + quarter * C::DQ_STAGE);
+    const uint32_t stage_addr = base + C::DQS_OFF + quarter * C::DQ_STAGE;
     for (int it = 0; it < n_it; ++it) {
-      const int buf = it & 1;
       const int q0 = (i0 + it) * C::BQ;
-      if (!__all_sync(0xffffffffu,
-                      mbar_wait(bar(C::B_DQ + buf), (it >> 1) & 1, a.err, kSiteDQ, abort_flag)))
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(C::B_DQ), it & 1, a.err, kSiteDQ, abort_flag)))
         break;
       tc_fence_after();
       uint32_t v0[32], v1[32];
-      tmem_ld32(tmem + lane_off + C::COL_DQT + buf * 64, v0);
-      tmem_ld32(tmem + lane_off + C::COL_DQT + buf * 64 + 32, v1);
+      tmem_ld32(tmem + lane_off + C::COL_DQ, v0);
+      tmem_ld32(tmem + lane_off + C::COL_DQ + 32, v1);
       tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(bar(C::B_DQFREE + buf));          // the buffer is free again
-      float* col = a.dq + (static_cast<size_t>(bh) * a.N + q0) * D + c;
-      const int nv = min(C::BQ, a.N - q0);
+      warp_arrive(bar(C::B_DQFREE));                 // the TMEM tile is free again
+      if (lane == 0) bulk_wait_read_all();           // previous reduce has read the staging box
+      __syncwarp();
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
-        if (j < nv) atomicAdd(col + static_cast<size_t>(j) * D, __uint_as_float(v0[j]) * sc);
+      for (int j = 0; j < 32; ++j) stage[j * 32 + lane] = __uint_as_float(v0[j]) * sc;
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
-        if (32 + j < nv) atomicAdd(col + static_cast<size_t>(32 + j) * D, __uint_as_float(v1[j]) * sc);
+      for (int j = 0; j < 32; ++j) stage[(32 + j) * 32 + lane] = __uint_as_float(v1[j]) * sc;
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_reduce_add_3d(&tmDQ, stage_addr, quarter * 32, q0, bh);   // rows >= N are skipped
+        bulk_commit_group();
+      }
     }
+    if (lane == 0) bulk_wait_all();
     tc_fence_before();
   }
 
@@ -936,15 +959,16 @@ bwd_q64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
 template <int D>
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const BwdArgs& a, cudaStream_t stream) {
+                       const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a,
+                       cudaStream_t stream) {
   using C = BwdCfg<D>;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = D == 128 ? cudaFuncSetAttribute(bwd_q64_kernel,
+    cudaError_t e = D == 128 ? cudaFuncSetAttribute(bwd_d128_kernel,
                                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                    BwdQ64::SMEM_BYTES)
+                                                    BwdD128::SMEM_BYTES)
                              : cudaFuncSetAttribute(bwd_main_kernel<D>,
                                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                     C::SMEM_BYTES);
@@ -963,16 +987,18 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   if (e != cudaSuccess) return e;
   const int nk = (a.N + C::BK - 1) / C::BK;
   if (D == 128)
-    bwd_q64_kernel<<<nk * a.B * a.H, BwdQ64::THREADS, BwdQ64::SMEM_BYTES, stream>>>(tq, tk, tv,
-                                                                                   tdo, a);
+    bwd_d128_kernel<<<nk * a.B * a.H, BwdD128::THREADS, BwdD128::SMEM_BYTES, stream>>>(
+        tq, tk, tv, tdo, tdq, a);
   else
     bwd_main_kernel<D><<<nk * a.B * a.H, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
   return cudaGetLastError();
 }
 
 template cudaError_t launch_bwd<64>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                                    const CUtensorMap&, const BwdArgs&, cudaStream_t);
+                                    const CUtensorMap&, const CUtensorMap&, const BwdArgs&,
+                                    cudaStream_t);
 template cudaError_t launch_bwd<128>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                                     const CUtensorMap&, const BwdArgs&, cudaStream_t);
+                                     const CUtensorMap&, const CUtensorMap&, const BwdArgs&,
+                                     cudaStream_t);
 
 }  // namespace fa

@@ -110,7 +110,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(C::B_S + t), 1);
-      mbar_init(bar(C::B_P + t), 128);
+      mbar_init(bar(C::B_P + t), 4);   // one arrival per softmax warp
       mbar_init(bar(C::B_O + t), 1);
     }
     mbar_init(bar(C::B_DRAIN), 1);
@@ -326,7 +326,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(C::B_P + t));
+      warp_arrive(bar(C::B_P + t));
     }
     // ------------------------------------------------------------ epilogue
     if (ok && nkb_t[t] > 0) {

@@ -45,9 +45,12 @@ struct BwdArgs {
   uint32_t* err;
 };
 
+// tdq: fp32 view of dq, [BH][N][d], box 32 x 64, no swizzle (reduce-add target
+// of the d = 128 main pass; unused for d = 64)
 template <int D>
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const BwdArgs& a, cudaStream_t stream);
+                       const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a,
+                       cudaStream_t stream);
 
 struct DecodeArgs {
   const void* q;            // bf16 [S][Hq][d]
