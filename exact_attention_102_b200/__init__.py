@@ -34,7 +34,7 @@ EXPORTS = (
     "fa_status_str", "fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd",
     "paged_attn_decode_workspace_bytes", "paged_attn_decode", "fa_fp8_prepare",
     "fa_fwd_fp8", "fa_last_device_error", "fa_debug_wait_timeout",
-    "paged_attn_decode_noalloc",
+    "paged_attn_decode_noalloc", "fa_bwd_time_main_pass",
 )
 
 
@@ -79,6 +79,8 @@ def lib() -> ctypes.CDLL:
     L.fa_fwd_fp8.argtypes = [vp] * 8 + [ci, ci, ci, ci, ci, vp]
     L.fa_last_device_error.restype = ci
     L.fa_last_device_error.argtypes = [vp]
+    L.fa_bwd_time_main_pass.restype = ci
+    L.fa_bwd_time_main_pass.argtypes = [vp, vp]
     L.fa_debug_wait_timeout.restype = ci
     L.fa_debug_wait_timeout.argtypes = [ctypes.c_uint, vp]
     _lib = L
@@ -246,6 +248,17 @@ def fa_fwd_fp8(q8, k8, v8, sq, sk, sv, causal=False, o=None, lse=None, stream=No
 def fa_last_device_error(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device error status."""
     return int(lib().fa_last_device_error(_stream(stream)))
+
+
+def fa_bwd_time_main_pass(ev_begin, ev_end) -> None:
+    """The next fa_bwd call of this thread records the two torch.cuda.Event
+    objects around its main pass (profiling)."""
+    for ev in (ev_begin, ev_end):
+        if not ev.cuda_event:       # torch creates the CUDA event on first record
+            ev.record()
+    _check("fa_bwd_time_main_pass",
+           lib().fa_bwd_time_main_pass(ctypes.c_void_p(ev_begin.cuda_event),
+                                       ctypes.c_void_p(ev_end.cuda_event)))
 
 
 def fa_debug_wait_timeout(timeout_us, stream=None) -> int:

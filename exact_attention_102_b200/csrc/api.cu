@@ -74,6 +74,10 @@ bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int elem_
   return r == CUDA_SUCCESS;
 }
 
+// Events the next fa_bwd call of this thread records around its main pass.
+thread_local cudaEvent_t g_bwd_ev_begin = nullptr;
+thread_local cudaEvent_t g_bwd_ev_end = nullptr;
+
 bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -200,8 +204,10 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   a.scale_log2 = a.scale * kLog2e;
   a.err = err;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = (d == 128) ? fa::launch_bwd<128>(tq, tk, tv, tdo, tdq, a, s)
-                             : fa::launch_bwd<64>(tq, tk, tv, tdo, tdq, a, s);
+  cudaEvent_t eb = g_bwd_ev_begin, ee = g_bwd_ev_end;
+  g_bwd_ev_begin = g_bwd_ev_end = nullptr;     // one call consumes the pair
+  cudaError_t e = (d == 128) ? fa::launch_bwd<128>(tq, tk, tv, tdo, tdq, a, s, eb, ee)
+                             : fa::launch_bwd<64>(tq, tk, tv, tdo, tdq, a, s, eb, ee);
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
@@ -349,6 +355,13 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float
   a.err = err;
   cudaError_t e = fa::launch_fwd_fp8(tq, tk, tv, a, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+fa_status fa_bwd_time_main_pass(void* ev_begin, void* ev_end) {
+  if ((ev_begin == nullptr) != (ev_end == nullptr)) return FA_ERR_INVALID_ARG;
+  g_bwd_ev_begin = static_cast<cudaEvent_t>(ev_begin);
+  g_bwd_ev_end = static_cast<cudaEvent_t>(ev_end);
+  return FA_OK;
 }
 
 fa_status fa_last_device_error(void* stream) {

@@ -960,7 +960,7 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 template <int D>
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a,
-                       cudaStream_t stream) {
+                       cudaStream_t stream, cudaEvent_t ev_main_begin, cudaEvent_t ev_main_end) {
   using C = BwdCfg<D>;
   static bool attr_set[64] = {};
   int dev = 0;
@@ -986,19 +986,22 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int nk = (a.N + C::BK - 1) / C::BK;
+  if (ev_main_begin != nullptr) cudaEventRecord(ev_main_begin, stream);
   if (D == 128)
     bwd_d128_kernel<<<nk * a.B * a.H, BwdD128::THREADS, BwdD128::SMEM_BYTES, stream>>>(
         tq, tk, tv, tdo, tdq, a);
   else
     bwd_main_kernel<D><<<nk * a.B * a.H, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (ev_main_end != nullptr) cudaEventRecord(ev_main_end, stream);
+  return e;
 }
 
 template cudaError_t launch_bwd<64>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
                                     const CUtensorMap&, const CUtensorMap&, const BwdArgs&,
-                                    cudaStream_t);
+                                    cudaStream_t, cudaEvent_t, cudaEvent_t);
 template cudaError_t launch_bwd<128>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
                                      const CUtensorMap&, const CUtensorMap&, const BwdArgs&,
-                                     cudaStream_t);
+                                     cudaStream_t, cudaEvent_t, cudaEvent_t);
 
 }  // namespace fa

@@ -47,10 +47,13 @@ struct BwdArgs {
 
 // tdq: fp32 view of dq, [BH][N][d], box 32 x 64, no swizzle (reduce-add target
 // of the d = 128 main pass; unused for d = 64)
+// ev_main_begin / ev_main_end (may be null): recorded on `stream` right before
+// and right after the main pass, for timing that kernel alone.
 template <int D>
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a,
-                       cudaStream_t stream);
+                       cudaStream_t stream, cudaEvent_t ev_main_begin = nullptr,
+                       cudaEvent_t ev_main_end = nullptr);
 
 struct DecodeArgs {
   const void* q;            // bf16 [S][Hq][d]

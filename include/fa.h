@@ -221,6 +221,17 @@ FA_API fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8,
                      void* stream);
 
 /*
+ * fa_bwd_time_main_pass — for profiling. ev_begin and ev_end are cudaEvent_t
+ * handles created by the caller (both non-NULL, or both NULL to cancel). The
+ * next fa_bwd call made by this thread records ev_begin on its stream right
+ * before its main pass (the kernel that runs the five products) and ev_end
+ * right after it, so cudaEventElapsedTime gives that kernel's duration without
+ * the conversion and D/L pre pass. The pair is used by one call only.
+ * Errors: FA_ERR_INVALID_ARG when exactly one handle is NULL.
+ */
+FA_API fa_status fa_bwd_time_main_pass(void* ev_begin, void* ev_end);
+
+/*
  * fa_last_device_error — synchronises `stream`, then reads and clears the
  * device error word of the current device. Returns FA_OK when nothing was
  * recorded since the last call, FA_ERR_TIMEOUT when a bounded wait gave up,
