@@ -46,7 +46,7 @@ METRIC = "attention fwd+bwd TFLOP/s (bf16)"
 # DRAM bytes (read + write) of one d = 128 backward main-pass launch at WORKLOAD
 # (2.00 GB read + 1.16 GB written), from an ncu capture of that launch with the
 # current kernel; set to None whenever the kernel changes until captured again
-BWD_MAIN_TRAFFIC = 3.16e9
+BWD_MAIN_TRAFFIC = None
 
 
 def _peaks():

@@ -575,10 +575,12 @@ struct BwdD128 {
   static constexpr int L_OFF = DQS_OFF + 4 * DQ_STAGE;  // NS x 64 fp32: L * log2(e)
   static constexpr int DL_OFF = L_OFF + NS * 256;       // NS x 64 fp32: D
   static constexpr int BAR_OFF = DL_OFF + NS * 256;
-  static constexpr int B_KV = 0, B_QF = 1, B_QE = B_QF + NS, B_DF = B_QE + NS, B_DE = B_DF + NS;
-  static constexpr int B_KT = B_DE + NS, B_ST = B_KT + 1, B_DPT = B_ST + 1, B_P = B_DPT + 1;
-  static constexpr int B_DS = B_P + 1, B_DSFREE = B_DS + 1;   // [2]
-  static constexpr int B_DQ = B_DSFREE + 2, B_DQFREE = B_DQ + 1;
+  // B_STEP[s]: committed after dQ^T of the step held in stage s; every product
+  // of that step is then complete: the Q / dO stage and the dS buffer are free
+  // and the dQ^T tile is ready.
+  static constexpr int B_KV = 0, B_QF = 1, B_DF = B_QF + NS, B_STEP = B_DF + NS;
+  static constexpr int B_KT = B_STEP + NS, B_ST = B_KT + 1, B_DPT = B_ST + 1, B_P = B_DPT + 1;
+  static constexpr int B_DS = B_P + 1, B_DQFREE = B_DS + 1;
   static constexpr int B_END = B_DQFREE + 1, B_DRAIN = B_END + 1, NBAR = B_DRAIN + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
@@ -623,18 +625,14 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     mbar_init(bar(C::B_KV), 1);
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(bar(C::B_QF + s), 1);
-      mbar_init(bar(C::B_QE + s), 1);
       mbar_init(bar(C::B_DF + s), 1);
-      mbar_init(bar(C::B_DE + s), 1);
+      mbar_init(bar(C::B_STEP + s), 1);
     }
     mbar_init(bar(C::B_KT), 8);     // one arrival per softmax-gradient warp
     mbar_init(bar(C::B_ST), 1);
     mbar_init(bar(C::B_DPT), 1);
     mbar_init(bar(C::B_P), 8);
     mbar_init(bar(C::B_DS), 8);
-    mbar_init(bar(C::B_DSFREE), 1);
-    mbar_init(bar(C::B_DSFREE + 1), 1);
-    mbar_init(bar(C::B_DQ), 1);
     mbar_init(bar(C::B_DQFREE), 4); // one arrival per drain warp
     mbar_init(bar(C::B_END), 1);
     mbar_init(bar(C::B_DRAIN), 1);
@@ -669,13 +667,12 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const uint32_t ph = ((it / C::NS) & 1) ^ 1;
         const int row = (i0 + it) * C::BQ;
         const size_t prow = static_cast<size_t>(bh) * a.n_pad + row;   // 256 B aligned
-        if (!mbar_wait(bar(C::B_QE + s), ph, a.err, kSiteQE, abort_flag)) break;
+        if (!mbar_wait(bar(C::B_STEP + s), ph, a.err, kSiteQE, abort_flag)) break;
         mbar_arrive_expect_tx(bar(C::B_QF + s), C::Q_TILE + 256);
         for (int c = 0; c < 2; ++c)
           tma_load_3d(base + C::Q_OFF + s * C::Q_TILE + c * C::Q_CHUNK, &tmQ, bar(C::B_QF + s),
                       c * 64, row, bh);
         bulk_load(base + C::L_OFF + s * 256, a.lse_log2 + prow, 256, bar(C::B_QF + s));
-        if (!mbar_wait(bar(C::B_DE + s), ph, a.err, kSiteDE, abort_flag)) break;
         mbar_arrive_expect_tx(bar(C::B_DF + s), C::Q_TILE + 256);
         for (int c = 0; c < 2; ++c)
           tma_load_3d(base + C::DO_OFF + s * C::Q_TILE + c * C::Q_CHUNK, &tmDO, bar(C::B_DF + s),
@@ -697,19 +694,27 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       constexpr uint32_t idS = idesc_f16(128, C::BQ, 0, 0, 0);   // S^T, dP^T: K-major operands
       constexpr uint32_t idKM = idesc_f16(128, D, 0, 0, 1);      // dV, dK: A tmem, B MN-major
       constexpr uint32_t idQT = idesc_f16(128, C::BQ, 0, 1, 1);  // dQ^T: A = K^T, B = dS^T, MN-major
-      const uint32_t kbase = base + C::K_OFF, vbase = base + C::V_OFF;
+      // descriptors of the fixed tiles and of stage / buffer 0; a tile at a
+      // byte offset is the base descriptor plus offset / 16 (start-address field)
+      const uint64_t dV = smem_desc_sw128(base + C::V_OFF, 16, 1024);            // V, K-major
+      const uint64_t dKt = smem_desc_sw128(base + C::K_OFF, C::KV_CHUNK, 1024);  // K^T, MN-major
+      const uint64_t dQk = smem_desc_sw128(base + C::Q_OFF, 16, 1024);           // Q, K-major
+      const uint64_t dQm = smem_desc_sw128(base + C::Q_OFF, C::Q_CHUNK, 1024);   // Q, MN-major
+      const uint64_t dGk = smem_desc_sw128(base + C::DO_OFF, 16, 1024);          // dO, K-major
+      const uint64_t dGm = smem_desc_sw128(base + C::DO_OFF, C::Q_CHUNK, 1024);  // dO, MN-major
+      const uint64_t dDS = smem_desc_sw128(base + C::DS_OFF, 16, 1024);          // dS^T, MN-major
+      auto add = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (bytes >> 4); };
       bool ok = mbar_wait(bar(C::B_KV), 0, a.err, kSiteKV, abort_flag) &&
                 mbar_wait(bar(C::B_KT), 0, a.err, kSiteKV, abort_flag);
       auto issue_s = [&](int it) -> bool {
         const int s = it % C::NS;
         if (!mbar_wait(bar(C::B_QF + s), (it / C::NS) & 1, a.err, kSiteQF, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t qb = base + C::Q_OFF + s * C::Q_TILE;
+        const uint64_t q = add(dQk, s * C::Q_TILE);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)   // K = d: chunk kk/4, 32 B steps inside it
           umma_f16_ts(tmem + C::COL_S, tmem + C::COL_K + kk * 8,
-                      smem_desc_sw128(qb + (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32, 16, 1024), idS,
-                      kk > 0);
+                      add(q, (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32), idS, kk > 0);
         umma_commit(bar(C::B_ST));
         return true;
       };
@@ -717,13 +722,11 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const int s = it % C::NS;
         if (!mbar_wait(bar(C::B_DF + s), (it / C::NS) & 1, a.err, kSiteDF, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t gb = base + C::DO_OFF + s * C::Q_TILE;
+        const uint64_t g = add(dGk, s * C::Q_TILE);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          umma_f16_ss(tmem + C::COL_DP,
-                      smem_desc_sw128(vbase + (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32, 16, 1024),
-                      smem_desc_sw128(gb + (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32, 16, 1024), idS,
-                      kk > 0);
+          umma_f16_ss(tmem + C::COL_DP, add(dV, (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32),
+                      add(g, (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32), idS, kk > 0);
         umma_commit(bar(C::B_DPT));
         return true;
       };
@@ -733,19 +736,18 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
       for (int it = 0; it < n_it && ok; ++it) {
         const int s = it % C::NS;
-        const int buf = it & 1;
-        const uint32_t qb = base + C::Q_OFF + s * C::Q_TILE;
-        const uint32_t gb = base + C::DO_OFF + s * C::Q_TILE;
-        const uint32_t dsb = base + C::DS_OFF + buf * C::DS_BYTES;
+        const uint64_t qm = add(dQm, s * C::Q_TILE);
+        const uint64_t gm = add(dGm, s * C::Q_TILE);
+        const uint64_t ds = add(dDS, (it & 1) * C::DS_BYTES);
+        const uint32_t acc0 = it > 0 ? 1u : 0u;
         // dV += P^T dO_it
         ok = mbar_wait(bar(C::B_P), it & 1, a.err, kSiteP, abort_flag);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < C::BQ / 16; ++kk)
-          umma_f16_ts(tmem + C::COL_DV, tmem + C::COL_S + half_col(kk),
-                      smem_desc_sw128(gb + kk * 2048, C::Q_CHUNK, 1024), idKM,
-                      (it > 0 || kk > 0) ? 1u : 0u);
+          umma_f16_ts(tmem + C::COL_DV, tmem + C::COL_S + half_col(kk), add(gm, kk * 2048), idKM,
+                      kk > 0 ? 1u : acc0);
         if (it + 1 < n_it) {
           ok = issue_s(it + 1);          // after dV(it): in-order, so P^T(it) is read first
           if (!ok) break;
@@ -756,10 +758,8 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < C::BQ / 16; ++kk)
-          umma_f16_ts(tmem + C::COL_DK, tmem + C::COL_DP + half_col(kk),
-                      smem_desc_sw128(qb + kk * 2048, C::Q_CHUNK, 1024), idKM,
-                      (it > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(bar(C::B_QE + s));   // Q_it and its L: S^T(it), dK(it) done
+          umma_f16_ts(tmem + C::COL_DK, tmem + C::COL_DP + half_col(kk), add(qm, kk * 2048), idKM,
+                      kk > 0 ? 1u : acc0);
         if (it + 1 < n_it) {
           ok = issue_dp(it + 1);         // after dK(it): dS^T(it) is read first
           if (!ok) break;
@@ -772,11 +772,9 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
 #pragma unroll
         for (int kk = 0; kk < C::BK / 16; ++kk)
-          umma_f16_ss(tmem + C::COL_DQ, smem_desc_sw128(kbase + kk * 2048, C::KV_CHUNK, 1024),
-                      smem_desc_sw128(dsb + kk * 2048, 16, 1024), idQT, kk > 0 ? 1u : 0u);
-        umma_commit(bar(C::B_DQ));
-        umma_commit(bar(C::B_DSFREE + buf));
-        umma_commit(bar(C::B_DE + s));   // dO_it and its D: dP^T(it), dV(it) done
+          umma_f16_ss(tmem + C::COL_DQ, add(dKt, kk * 2048), add(ds, kk * 2048), idQT,
+                      kk > 0 ? 1u : 0u);
+        umma_commit(bar(C::B_STEP + s));  // step it complete: stage s, dS buffer, dQ^T tile
       }
       umma_commit(bar(C::B_END));
       umma_commit(bar(C::B_DRAIN));
@@ -844,9 +842,9 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       warp_arrive(bar(C::B_P));
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_DPT), it & 1, a.err, kSiteDPT, abort_flag));
       if (!ok) break;
-      if (it >= 2) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_DSFREE + buf), ((it >> 1) - 1) & 1, a.err,
-                                               kSiteDSF, abort_flag));
+      if (it >= 2) {                                   // dQ^T(it-2) has read this dS buffer
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_STEP + (it - 2) % C::NS),
+                                               ((it - 2) / C::NS) & 1, a.err, kSiteDSF, abort_flag));
         if (!ok) break;
       }
       tc_fence_after();
@@ -921,7 +919,8 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const uint32_t stage_addr = base + C::DQS_OFF + quarter * C::DQ_STAGE;
     for (int it = 0; it < n_it; ++it) {
       const int q0 = (i0 + it) * C::BQ;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(C::B_DQ), it & 1, a.err, kSiteDQ, abort_flag)))
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(C::B_STEP + it % C::NS), (it / C::NS) & 1, a.err,
+                                              kSiteDQ, abort_flag)))
         break;
       tc_fence_after();
       uint32_t v0[32], v1[32];
