@@ -546,10 +546,10 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 //   dQ^T = K_j^T dS^T     A = K_j^T (shared memory, MN-major),    B = dS^T
 // TMEM: K [0,64)  S^T/P^T [64,128)  dP^T/dS^T [128,192)  dQ^T [192,256)
 //       dV [256,384)  dK [384,512)
-// One tcgen05 issuer executes in issue order, so S^T(i+1) may be issued right
-// after dV(i) (which reads P^T(i) from the same columns) and dP^T(i+1) right
-// after dK(i) (which reads dS^T(i)); per step the issue order is
-// dV(i), S^T(i+1) | dK(i), dP^T(i+1), dQ(i).
+// One tcgen05 issuer executes in issue order, so S^T(i+2) may be issued right
+// after dV(i+1) (which reads P^T(i+1) from the same columns) and dP^T(i+1)
+// right after dK(i) (which reads dS^T(i)); per step the issue order is
+// dK(i), dP^T(i+1), dV(i+1), S^T(i+2), dQ(i).
 // Warps 4..11 (two per TMEM lane quarter, one per 32-query half) compute P
 // and then dS for their half; dS also goes to shared memory (double-buffered)
 // for the dQ product. Warps 12..15 (thread = head-dim column) drain dQ^T to a
@@ -578,10 +578,13 @@ struct BwdD128 {
   // B_STEP[s]: committed after dQ^T of the step held in stage s; every product
   // of that step is then complete: the Q / dO stage and the dS buffer are free
   // and the dQ^T tile is ready.
-  static constexpr int B_KV = 0, B_QF = 1, B_DF = B_QF + NS, B_STEP = B_DF + NS;
+  // B_FULL[s]: Q, L, dO and D of the step in stage s have landed.
+  // B_DSQ: phase i completes when the 8 softmax-gradient warps have written
+  // dS(i) and the 4 drain warps have read dQ^T(i-1) out of TMEM.
+  static constexpr int B_KV = 0, B_FULL = 1, B_STEP = B_FULL + NS;
   static constexpr int B_KT = B_STEP + NS, B_ST = B_KT + 1, B_DPT = B_ST + 1, B_P = B_DPT + 1;
-  static constexpr int B_DS = B_P + 1, B_DQFREE = B_DS + 1;
-  static constexpr int B_END = B_DQFREE + 1, B_DRAIN = B_END + 1, NBAR = B_DRAIN + 1;
+  static constexpr int B_DSQ = B_P + 1;
+  static constexpr int B_END = B_DSQ + 1, B_DRAIN = B_END + 1, NBAR = B_DRAIN + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
   static constexpr uint32_t COL_K = 0, COL_S = 64, COL_DP = 128, COL_DQ = 192, COL_DV = 256,
@@ -624,16 +627,14 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   if (threadIdx.x == 0) {
     mbar_init(bar(C::B_KV), 1);
     for (int s = 0; s < C::NS; ++s) {
-      mbar_init(bar(C::B_QF + s), 1);
-      mbar_init(bar(C::B_DF + s), 1);
+      mbar_init(bar(C::B_FULL + s), 1);
       mbar_init(bar(C::B_STEP + s), 1);
     }
     mbar_init(bar(C::B_KT), 8);     // one arrival per softmax-gradient warp
     mbar_init(bar(C::B_ST), 1);
     mbar_init(bar(C::B_DPT), 1);
     mbar_init(bar(C::B_P), 8);
-    mbar_init(bar(C::B_DS), 8);
-    mbar_init(bar(C::B_DQFREE), 4); // one arrival per drain warp
+    mbar_init(bar(C::B_DSQ), 8 + 4);  // 8 softmax-gradient warps + 4 drain warps
     mbar_init(bar(C::B_END), 1);
     mbar_init(bar(C::B_DRAIN), 1);
     *abort_flag = 0;
@@ -668,22 +669,19 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const int row = (i0 + it) * C::BQ;
         const size_t prow = static_cast<size_t>(bh) * a.n_pad + row;   // 256 B aligned
         if (!mbar_wait(bar(C::B_STEP + s), ph, a.err, kSiteQE, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(C::B_QF + s), C::Q_TILE + 256);
+        const uint32_t full = bar(C::B_FULL + s);
+        mbar_arrive_expect_tx(full, 2 * (C::Q_TILE + 256));
         for (int c = 0; c < 2; ++c)
-          tma_load_3d(base + C::Q_OFF + s * C::Q_TILE + c * C::Q_CHUNK, &tmQ, bar(C::B_QF + s),
-                      c * 64, row, bh);
-        bulk_load(base + C::L_OFF + s * 256, a.lse_log2 + prow, 256, bar(C::B_QF + s));
-        mbar_arrive_expect_tx(bar(C::B_DF + s), C::Q_TILE + 256);
+          tma_load_3d(base + C::Q_OFF + s * C::Q_TILE + c * C::Q_CHUNK, &tmQ, full, c * 64, row, bh);
+        bulk_load(base + C::L_OFF + s * 256, a.lse_log2 + prow, 256, full);
         for (int c = 0; c < 2; ++c)
-          tma_load_3d(base + C::DO_OFF + s * C::Q_TILE + c * C::Q_CHUNK, &tmDO, bar(C::B_DF + s),
-                      c * 64, row, bh);
-        bulk_load(base + C::DL_OFF + s * 256, a.delta + prow, 256, bar(C::B_DF + s));
+          tma_load_3d(base + C::DO_OFF + s * C::Q_TILE + c * C::Q_CHUNK, &tmDO, full, c * 64, row,
+                      bh);
+        bulk_load(base + C::DL_OFF + s * 256, a.delta + prow, 256, full);
         issued = it + 1;
       }
       for (int it = max(0, issued - C::NS); it < issued; ++it) {
-        mbar_wait(bar(C::B_QF + it % C::NS), (it / C::NS) & 1, a.err, kSiteDrain, nullptr,
-                  200000000ull);
-        mbar_wait(bar(C::B_DF + it % C::NS), (it / C::NS) & 1, a.err, kSiteDrain, nullptr,
+        mbar_wait(bar(C::B_FULL + it % C::NS), (it / C::NS) & 1, a.err, kSiteDrain, nullptr,
                   200000000ull);
       }
       mbar_wait(bar(C::B_KV), 0, a.err, kSiteDrain, nullptr, 200000000ull);
@@ -708,7 +706,8 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 mbar_wait(bar(C::B_KT), 0, a.err, kSiteKV, abort_flag);
       auto issue_s = [&](int it) -> bool {
         const int s = it % C::NS;
-        if (!mbar_wait(bar(C::B_QF + s), (it / C::NS) & 1, a.err, kSiteQF, abort_flag)) return false;
+        if (!mbar_wait(bar(C::B_FULL + s), (it / C::NS) & 1, a.err, kSiteQF, abort_flag))
+          return false;
         tc_fence_after();
         const uint64_t q = add(dQk, s * C::Q_TILE);
 #pragma unroll
@@ -718,10 +717,9 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         umma_commit(bar(C::B_ST));
         return true;
       };
+      // dP^T(it): stage it % NS was waited for by issue_s(it), issued before
       auto issue_dp = [&](int it) -> bool {
         const int s = it % C::NS;
-        if (!mbar_wait(bar(C::B_DF + s), (it / C::NS) & 1, a.err, kSiteDF, abort_flag)) return false;
-        tc_fence_after();
         const uint64_t g = add(dGk, s * C::Q_TILE);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
@@ -730,30 +728,37 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         umma_commit(bar(C::B_DPT));
         return true;
       };
-      if (ok) {
+      // dV(it) += P^T(it) dO_it: after P(it) is in TMEM
+      auto issue_dv = [&](int it) -> bool {
+        if (!mbar_wait(bar(C::B_P), it & 1, a.err, kSiteP, abort_flag)) return false;
         tc_fence_after();
-        ok = issue_s(0) && issue_dp(0);
-      }
-      for (int it = 0; it < n_it && ok; ++it) {
-        const int s = it % C::NS;
-        const uint64_t qm = add(dQm, s * C::Q_TILE);
-        const uint64_t gm = add(dGm, s * C::Q_TILE);
-        const uint64_t ds = add(dDS, (it & 1) * C::DS_BYTES);
+        const uint64_t gm = add(dGm, (it % C::NS) * C::Q_TILE);
         const uint32_t acc0 = it > 0 ? 1u : 0u;
-        // dV += P^T dO_it
-        ok = mbar_wait(bar(C::B_P), it & 1, a.err, kSiteP, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < C::BQ / 16; ++kk)
           umma_f16_ts(tmem + C::COL_DV, tmem + C::COL_S + half_col(kk), add(gm, kk * 2048), idKM,
                       kk > 0 ? 1u : acc0);
-        if (it + 1 < n_it) {
-          ok = issue_s(it + 1);          // after dV(it): in-order, so P^T(it) is read first
-          if (!ok) break;
-        }
-        // dK += dS^T Q_it
-        ok = mbar_wait(bar(C::B_DS), it & 1, a.err, kSiteDS, abort_flag);
+        return true;
+      };
+      // Issue order: S(0), dP(0), dV(0), S(1), then per step it
+      //   dK(it), dP(it+1), dV(it+1), S(it+2), dQ(it)
+      // Each wait (P(it+1) before dV(it+1), dS(it) before dK(it)) falls while
+      // the product issued before it is still running, so the pipe stays fed.
+      // In-order execution makes the overwrites safe: S(it+2) comes after
+      // dV(it+1) (which reads P(it+1) from the S columns), dP(it+1) after dK(it)
+      // (which reads dS(it) from the dP columns).
+      if (ok) {
+        tc_fence_after();
+        ok = issue_s(0) && issue_dp(0) && issue_dv(0);
+        if (ok && n_it > 1) ok = issue_s(1);
+      }
+      for (int it = 0; it < n_it && ok; ++it) {
+        const int s = it % C::NS;
+        const uint64_t qm = add(dQm, s * C::Q_TILE);
+        const uint64_t ds = add(dDS, (it & 1) * C::DS_BYTES);
+        const uint32_t acc0 = it > 0 ? 1u : 0u;
+        // dK += dS^T Q_it (B_DSQ phase it: dS(it) written, dQ^T(it-1) drained)
+        ok = mbar_wait(bar(C::B_DSQ), it & 1, a.err, kSiteDS, abort_flag);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -761,15 +766,11 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           umma_f16_ts(tmem + C::COL_DK, tmem + C::COL_DP + half_col(kk), add(qm, kk * 2048), idKM,
                       kk > 0 ? 1u : acc0);
         if (it + 1 < n_it) {
-          ok = issue_dp(it + 1);         // after dK(it): dS^T(it) is read first
+          ok = issue_dp(it + 1) && issue_dv(it + 1);
+          if (ok && it + 2 < n_it) ok = issue_s(it + 2);
           if (!ok) break;
         }
-        // dQ^T_it = K^T dS^T (the drain warps have read dQ^T(it-1))
-        if (it >= 1) {
-          ok = mbar_wait(bar(C::B_DQFREE), (it - 1) & 1, a.err, kSiteDQF, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-        }
+        // dQ^T_it = K^T dS^T (B_DSQ phase it covered the drain of dQ^T(it-1))
 #pragma unroll
         for (int kk = 0; kk < C::BK / 16; ++kk)
           umma_f16_ss(tmem + C::COL_DQ, add(dKt, kk * 2048), add(ds, kk * 2048), idQT,
@@ -882,7 +883,7 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tmem_st_wait();
       fence_async_smem();
       tc_fence_before();
-      warp_arrive(bar(C::B_DS));
+      warp_arrive(bar(C::B_DSQ));
     }
     // ---- epilogue: dV rows (half 0) or dK rows (half 1), thread = key
     if (ok) {
@@ -917,6 +918,7 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const float sc = a.scale;
     float* stage = reinterpret_cast<float*>(smem + C::DQS_OFF + quarter * C::DQ_STAGE);
     const uint32_t stage_addr = base + C::DQS_OFF + quarter * C::DQ_STAGE;
+    warp_arrive(bar(C::B_DSQ));                      // phase 0: no dQ^T(-1) to drain
     for (int it = 0; it < n_it; ++it) {
       const int q0 = (i0 + it) * C::BQ;
       if (!__all_sync(0xffffffffu, mbar_wait(bar(C::B_STEP + it % C::NS), (it / C::NS) & 1, a.err,
@@ -928,7 +930,7 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tmem_ld32(tmem + lane_off + C::COL_DQ + 32, v1);
       tmem_ld_wait();
       tc_fence_before();
-      warp_arrive(bar(C::B_DQFREE));                 // the TMEM tile is free again
+      warp_arrive(bar(C::B_DSQ));                    // dQ^T(it) read: counts for phase it+1
       if (lane == 0) bulk_wait_read_all();           // previous reduce has read the staging box
       __syncwarp();
 #pragma unroll

@@ -243,12 +243,16 @@ fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       int it = 0;
       int npv[2] = {0, 0};
       bool ok = mbar_wait(bar(C::B_Q), 0, a.err, kSQ, abort_flag);
-      auto issue_s = [&](int t, uint32_t kb) {
-        const uint32_t qb = base + C::Q_OFF + t * C::TILE;
+      // descriptors of Q tile 0 and ring stage 0; a tile at a byte offset is the
+      // base descriptor plus offset / 16 (start-address field)
+      const uint64_t dQ = smem_desc_sw128(base + C::Q_OFF, 16, 1024);
+      const uint64_t dR = smem_desc_sw128(base + C::RING_OFF, 16, 1024);
+      auto add = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (bytes >> 4); };
+      auto issue_s = [&](int t, int stage) {
+        const uint64_t q = add(dQ, t * C::TILE), k = add(dR, stage * C::TILE);
 #pragma unroll
         for (int kk = 0; kk < kD / 32; ++kk)   // K = 32 e4m3 elements = 32 bytes per MMA
-          umma_f8_ss(tmem + C::s_col(t), smem_desc_sw128(qb + kk * 32, 16, 1024),
-                     smem_desc_sw128(kb + kk * 32, 16, 1024), idS, kk > 0);
+          umma_f8_ss(tmem + C::s_col(t), add(q, kk * 32), add(k, kk * 32), idS, kk > 0);
         umma_commit(bar(C::B_S + t));
       };
       if (ok && nkb_cta > 0) {
@@ -258,7 +262,7 @@ fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (ok) {
           tc_fence_after();
           for (int t = 0; t < 2; ++t)
-            if (nkb_t[t] > 0) issue_s(t, base + C::RING_OFF + s * C::TILE);
+            if (nkb_t[t] > 0) issue_s(t, s);
           umma_commit(bar(C::B_KVE + s));
         }
       }
@@ -267,7 +271,7 @@ fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         ok = mbar_wait(bar(C::B_KVF + sv), (it / C::NSTAGE) & 1, a.err, kSKF, abort_flag);
         if (!ok) break;
         ++it;
-        const uint32_t vb = base + C::RING_OFF + sv * C::TILE;
+        const uint64_t vd = add(dR, sv * C::TILE);
         int sk = -1;
         for (int t = 0; t < 2 && ok; ++t) {
           if (j >= nkb_t[t]) continue;
@@ -276,10 +280,9 @@ fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < C::BN / 32; ++kk)   // 32 keys = 8 TMEM columns of packed e4m3 P
-            umma_f8_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8,
-                       smem_desc_sw128(vb + kk * 4096, 16, 1024), idPV,
+            umma_f8_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8, add(vd, kk * 4096), idPV,
                        (npv[t] > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(bar(C::B_O + t));
+          if (j + 1 == nkb_t[t]) umma_commit(bar(C::B_O + t));   // last P.V of tile t
           ++npv[t];
           if (j + 1 < nkb_t[t]) {
             if (sk < 0) {
@@ -289,7 +292,7 @@ fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
               if (!ok) break;
               tc_fence_after();
             }
-            issue_s(t, base + C::RING_OFF + sk * C::TILE);
+            issue_s(t, sk);
           }
         }
         if (!ok) break;
@@ -383,7 +386,7 @@ fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
     if (ok && nkb_t[t] > 0) {
       ok = __all_sync(0xffffffffu,
-                      mbar_wait(bar(C::B_O + t), (nkb_t[t] - 1) & 1, a.err, kSEpi, abort_flag));
+                      mbar_wait(bar(C::B_O + t), 0, a.err, kSEpi, abort_flag));
       if (ok) {
         tc_fence_after();
         const float mul = *cmax / (kPScale * l_run);

@@ -175,13 +175,18 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       int it = 0;
       int npv[2] = {0, 0};
       bool ok = mbar_wait(bar(C::B_Q), 0, a.err, kSiteQ, abort_flag);
-      auto issue_s = [&](int t, uint32_t kb) {
-        const uint32_t qb = base + C::Q_OFF + t * C::TILE;
+      // descriptors of Q tile 0 and ring stage 0; a tile at a byte offset is the
+      // base descriptor plus offset / 16 (start-address field)
+      const uint64_t dQ = smem_desc_sw128(base + C::Q_OFF, 16, 1024);        // K-major
+      const uint64_t dK = smem_desc_sw128(base + C::RING_OFF, 16, 1024);     // K-major
+      const uint64_t dVm = smem_desc_sw128(base + C::RING_OFF, C::CHUNK, 1024);  // MN-major
+      auto add = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (bytes >> 4); };
+      auto issue_s = [&](int t, int stage) {
+        const uint64_t q = add(dQ, t * C::TILE), k = add(dK, stage * C::TILE);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          umma_f16_ss(tmem + C::s_col(t), smem_desc_sw128(qb + off, 16, 1024),
-                      smem_desc_sw128(kb + off, 16, 1024), idS, kk > 0);
+          umma_f16_ss(tmem + C::s_col(t), add(q, off), add(k, off), idS, kk > 0);
         }
         umma_commit(bar(C::B_S + t));
       };
@@ -192,7 +197,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         if (ok) {
           tc_fence_after();
           for (int t = 0; t < 2; ++t)
-            if (nkb_t[t] > 0) issue_s(t, base + C::RING_OFF + s * C::TILE);
+            if (nkb_t[t] > 0) issue_s(t, s);
           umma_commit(bar(C::B_KVE + s));
         }
       }
@@ -201,7 +206,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         ok = mbar_wait(bar(C::B_KVF + sv), (it / C::NSTAGE) & 1, a.err, kSiteKvFull, abort_flag);
         if (!ok) break;
         ++it;
-        const uint32_t vb = base + C::RING_OFF + sv * C::TILE;
+        const uint64_t vm = add(dVm, sv * C::TILE);
         int sk = -1;                    // ring stage of K_{j+1}, once waited for
         for (int t = 0; t < 2 && ok; ++t) {
           if (j >= nkb_t[t]) continue;
@@ -210,10 +215,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < C::BN / 16; ++kk)
-            umma_f16_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8,
-                        smem_desc_sw128(vb + kk * 2048, C::CHUNK, 1024), idPV,
+            umma_f16_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8, add(vm, kk * 2048), idPV,
                         (npv[t] > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(bar(C::B_O + t));
+          if (j + 1 == nkb_t[t]) umma_commit(bar(C::B_O + t));   // last P.V of tile t
           ++npv[t];
           if (j + 1 < nkb_t[t]) {
             if (sk < 0) {
@@ -224,7 +228,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
               if (!ok) break;
               tc_fence_after();
             }
-            issue_s(t, base + C::RING_OFF + sk * C::TILE);
+            issue_s(t, sk);
           }
         }
         if (!ok) break;
@@ -331,7 +335,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     // ------------------------------------------------------------ epilogue
     if (ok && nkb_t[t] > 0) {
       ok = __all_sync(0xffffffffu,
-                      mbar_wait(bar(C::B_O + t), (nkb_t[t] - 1) & 1, a.err, kSiteEpi, abort_flag));
+                      mbar_wait(bar(C::B_O + t), 0, a.err, kSiteEpi, abort_flag));
       if (ok) {
         tc_fence_after();
         const float inv_l = 1.f / lr_run;
