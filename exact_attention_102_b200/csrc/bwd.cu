@@ -824,14 +824,20 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tmem_ld32(s_addr, sr);
       tmem_ld_wait();
       uint32_t pk[16];                                 // P^T, fp16 pairs of queries
+      const uint64_t nsl2 = f2_pack(-sl2, -sl2);
 #pragma unroll
       for (int e = 0; e < 32; e += 4) {
         const float4 lv = *reinterpret_cast<const float4*>(Ls + e);
-        const float L[4] = {lv.x, lv.y, lv.z, lv.w};
+        // y = L - scale log2e S on packed pairs; P = 2^-y
+        float y[4];
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), nsl2,
+                         f2_pack(lv.x, lv.y)), y[0], y[1]);
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3])), nsl2,
+                         f2_pack(lv.z, lv.w)), y[2], y[3]);
         float p[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          p[u] = ex2_approx(fmaf(__uint_as_float(sr[e + u]), sl2, -L[u]));
+          p[u] = ex2_approx(-y[u]);
           if (need_mask && ((a.causal && key > qh + e + u) || key >= a.N)) p[u] = 0.f;
         }
         pk[e / 2] = pack_f16x2(p[0], p[1]);
@@ -854,19 +860,20 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tmem_ld_wait();
       uint32_t w[16];                                  // dS^T, fp16 pairs of queries
       float ds_max = 0.f;
+      const uint64_t neg1 = f2_pack(-1.f, -1.f);
 #pragma unroll
       for (int e = 0; e < 32; e += 4) {
         const float4 dv4 = *reinterpret_cast<const float4*>(Ds + e);
-        const float Dv[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
+        // dS = P o (dP - D) on packed pairs
+        const uint64_t d01 = f2_fma(f2_pack(dv4.x, dv4.y), neg1,
+                                    f2_pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])));
+        const uint64_t d23 = f2_fma(f2_pack(dv4.z, dv4.w), neg1,
+                                    f2_pack(__uint_as_float(dr[e + 2]), __uint_as_float(dr[e + 3])));
+        const uint32_t pa = pk[e / 2], pb = pk[e / 2 + 1];
         float ds[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const uint32_t pp = pk[(e + u) >> 1];
-          const float pv = ((e + u) & 1) ? f16_hi(pp) : f16_lo(pp);
-          ds[u] = pv * (__uint_as_float(dr[e + u]) - Dv[u]);
-        }
-        ds_max = fmaxf(ds_max, fmaxf(fmaxf(fabsf(ds[0]), fabsf(ds[1])),
-                                     fmaxf(fabsf(ds[2]), fabsf(ds[3]))));
+        f2_unpack(f2_mul(f2_pack(f16_lo(pa), f16_hi(pa)), d01), ds[0], ds[1]);
+        f2_unpack(f2_mul(f2_pack(f16_lo(pb), f16_hi(pb)), d23), ds[2], ds[3]);
+        ds_max = fmax3(ds_max, fmax3(fabsf(ds[0]), fabsf(ds[1]), fabsf(ds[2])), fabsf(ds[3]));
         w[e / 2] = pack_f16x2(ds[0], ds[1]);
         w[e / 2 + 1] = pack_f16x2(ds[2], ds[3]);
       }

@@ -326,48 +326,62 @@ fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tmem_ld_wait();
       const int kbase = j * C::BN;
       const int kb0 = kbase / 64;
+      // scaled score of column c: S_c * f(half) (exp2 units); a half past the
+      // last key block is fully masked, so its factor only has to be positive
       const float f0 = rowf * skh[kb0];
-      const float f1 = (kb0 + 1 < nsb) ? rowf * skh[kb0 + 1] : 0.f;
+      const float f1 = (kb0 + 1 < nsb) ? rowf * skh[kb0 + 1] : 1.f;
       const float pv0 = svh[kb0] * inv_c;
       const float pv1 = (kb0 + 1 < nsb) ? svh[kb0 + 1] * inv_c : 0.f;
 #define SV(c) __uint_as_float(sr[(c) >> 5][(c)&31])
-      // scaled scores x_c = S_c * f(half) (exp2 units)
-#pragma unroll
-      for (int c = 0; c < 128; ++c)
-        sr[c >> 5][c & 31] = __float_as_uint(SV(c) * (c < 64 ? f0 : f1));
       if (kbase + C::BN - 1 > limit) {
 #pragma unroll
         for (int c = 0; c < 128; ++c)
           if (kbase + c > limit) sr[c >> 5][c & 31] = 0xff800000u;
       }
-      float mx0 = SV(0), mx1 = SV(1), mx2 = SV(2), mx3 = SV(3);
+      // row max of the raw scores per half, then scaled (the factors are > 0)
+      float ma0 = SV(0), ma1 = SV(1), mb0 = SV(64), mb1 = SV(65);
 #pragma unroll
-      for (int c = 4; c < 128; c += 4) {
-        mx0 = fmaxf(mx0, SV(c));
-        mx1 = fmaxf(mx1, SV(c + 1));
-        mx2 = fmaxf(mx2, SV(c + 2));
-        mx3 = fmaxf(mx3, SV(c + 3));
+      for (int c = 2; c < 62; c += 4) {
+        ma0 = fmax3(ma0, SV(c), SV(c + 1));
+        ma1 = fmax3(ma1, SV(c + 2), SV(c + 3));
+        mb0 = fmax3(mb0, SV(64 + c), SV(64 + c + 1));
+        mb1 = fmax3(mb1, SV(64 + c + 2), SV(64 + c + 3));
       }
-      const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+      ma0 = fmax3(ma0, SV(62), SV(63));
+      mb0 = fmax3(mb0, SV(126), SV(127));
+      const float mx = fmaxf(fmaxf(ma0, ma1) * f0, fmaxf(mb0, mb1) * f1);
       float alpha = 1.f;
       if (mx > m_run + kRescaleThreshold) {
         alpha = ex2_approx(m_run - mx);
         m_run = mx;
       }
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      float l0 = 0.f, l1 = 0.f;
+      const uint64_t fa = f2_pack(f0, f0), fb = f2_pack(f1, f1), negm2 = f2_pack(-m_use, -m_use);
+      const uint64_t wa = f2_pack(pv0, pv0), wb = f2_pack(pv1, pv1);
+      uint64_t la = 0, lb = 0;                       // (0.f, 0.f) pairs
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 128; c += 4) {
-        const float p0 = ex2_approx(SV(c) - m_use), p1 = ex2_approx(SV(c + 1) - m_use);
-        const float p2 = ex2_approx(SV(c + 2) - m_use), p3 = ex2_approx(SV(c + 3) - m_use);
-        l0 += p0 + p2;
-        l1 += p1 + p3;
-        const float w = c < 64 ? pv0 : pv1;
-        pk[c >> 2] = pack_e4m3x4(p0 * w, p1 * w, p2 * w, p3 * w);
+        const uint64_t f2 = c < 64 ? fa : fb, w2 = c < 64 ? wa : wb;
+        const uint64_t x01 = f2_fma(f2_pack(SV(c), SV(c + 1)), f2, negm2);
+        const uint64_t x23 = f2_fma(f2_pack(SV(c + 2), SV(c + 3)), f2, negm2);
+        float x0, x1, x2, x3;
+        f2_unpack(x01, x0, x1);
+        f2_unpack(x23, x2, x3);
+        const uint64_t p01 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+        const uint64_t p23 = f2_pack(ex2_approx(x2), ex2_approx(x3));
+        la = f2_add(la, p01);
+        lb = f2_add(lb, p23);
+        float q0, q1, q2, q3;
+        f2_unpack(f2_mul(p01, w2), q0, q1);
+        f2_unpack(f2_mul(p23, w2), q2, q3);
+        pk[c >> 2] = pack_e4m3x4(q0, q1, q2, q3);
       }
 #undef SV
-      l_run = l_run * alpha + (l0 + l1);
+      float l0, l1, l2, l3;
+      f2_unpack(la, l0, l1);
+      f2_unpack(lb, l2, l3);
+      l_run = l_run * alpha + ((l0 + l1) + (l2 + l3));
       tmem_st32(s_addr, pk);
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll

@@ -64,6 +64,11 @@ struct FwdCfg {
   static constexpr int THREADS = 384;
 };
 
+// every kPolyEvery-th pair of scores takes exp2 from exp2_poly_x2 (0: none)
+#ifndef FA_FWD_POLY_EVERY
+#define FA_FWD_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = FA_FWD_POLY_EVERY;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 // wait-site ids (reported in the device error word)
@@ -270,13 +275,15 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       }
       float mx0 = SV(0), mx1 = SV(1), mx2 = SV(2), mx3 = SV(3);
 #pragma unroll
-      for (int c = 4; c < 128; c += 4) {
-        mx0 = fmaxf(mx0, SV(c));
-        mx1 = fmaxf(mx1, SV(c + 1));
-        mx2 = fmaxf(mx2, SV(c + 2));
-        mx3 = fmaxf(mx3, SV(c + 3));
+      for (int c = 4; c < 124; c += 8) {
+        mx0 = fmax3(mx0, SV(c), SV(c + 1));
+        mx1 = fmax3(mx1, SV(c + 2), SV(c + 3));
+        mx2 = fmax3(mx2, SV(c + 4), SV(c + 5));
+        mx3 = fmax3(mx3, SV(c + 6), SV(c + 7));
       }
-      const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      mx0 = fmax3(mx0, SV(124), SV(125));
+      mx1 = fmax3(mx1, SV(126), SV(127));
+      const float mx = fmax3(fmax3(mx0, mx1, mx2), mx3, mx3) * sl2;
       float alpha = 1.f;
       if (mx > m_run + kRescaleThreshold) {  // also true for the first block (m_run = -inf)
         alpha = ex2_approx(m_run - mx);      // exp2(-inf) = 0 on the first block
@@ -286,33 +293,43 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       // Two row sums: l_run of the fp32 probabilities (for L = m + log l) and
       // lr_run of the bf16-rounded P the P.V product consumes (for O = acc/l),
       // so the normalisation weighs every key exactly as the numerator does.
-      float l0 = 0.f, l1 = 0.f, r0 = 0.f, r1 = 0.f;
+      // pairs of scores on packed fp32; every kPolyEvery-th pair takes its
+      // exp2 from the polynomial, the rest from the special-function unit
+      const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_use, -m_use);
+      uint64_t la = 0, lb = 0, ra = 0, rb = 0;     // (0.f, 0.f) pairs
       uint32_t pk0[32], pk1[32];
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
-        const float p0 = ex2_approx(fmaf(SV(c), sl2, -m_use));
-        const float p1 = ex2_approx(fmaf(SV(c + 1), sl2, -m_use));
+      for (int q = 0; q < 64; ++q) {
+        const uint64_t x2 = f2_fma(f2_pack(SV(2 * q), SV(2 * q + 1)), sl2x2, negm2);
+        uint64_t p2;
+        if (kPolyEvery > 0 && q % kPolyEvery == kPolyEvery - 1) {
+          p2 = exp2_poly_x2(x2);
+        } else {
+          float x0, x1;
+          f2_unpack(x2, x0, x1);
+          p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+        }
+        float p0, p1;
+        f2_unpack(p2, p0, p1);
         const uint32_t u = pack_bf16x2(p0, p1);
-        l0 += p0;
-        l1 += p1;
-        r0 += __uint_as_float(u << 16);
-        r1 += __uint_as_float(u & 0xffff0000u);
-        pk0[c >> 1] = u;
-      }
-#pragma unroll
-      for (int c = 64; c < 128; c += 2) {
-        const float p0 = ex2_approx(fmaf(SV(c), sl2, -m_use));
-        const float p1 = ex2_approx(fmaf(SV(c + 1), sl2, -m_use));
-        const uint32_t u = pack_bf16x2(p0, p1);
-        l0 += p0;
-        l1 += p1;
-        r0 += __uint_as_float(u << 16);
-        r1 += __uint_as_float(u & 0xffff0000u);
-        pk1[(c - 64) >> 1] = u;
+        const uint64_t rr = f2_pack(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+        if (q & 1) {
+          lb = f2_add(lb, p2);
+          rb = f2_add(rb, rr);
+        } else {
+          la = f2_add(la, p2);
+          ra = f2_add(ra, rr);
+        }
+        if (q < 32) pk0[q] = u; else pk1[q - 32] = u;
       }
 #undef SV
-      l_run = l_run * alpha + (l0 + l1);
-      lr_run = lr_run * alpha + (r0 + r1);
+      float l0, l1, l2, l3, r0, r1, r2, r3;
+      f2_unpack(la, l0, l1);
+      f2_unpack(lb, l2, l3);
+      f2_unpack(ra, r0, r1);
+      f2_unpack(rb, r2, r3);
+      l_run = l_run * alpha + ((l0 + l1) + (l2 + l3));
+      lr_run = lr_run * alpha + ((r0 + r1) + (r2 + r3));
       tmem_st32(s_addr, pk0);
       tmem_st32(s_addr + 32, pk1);
       // O rescale (PV of block j-1 has completed: S_t(j)'s commit covers it)

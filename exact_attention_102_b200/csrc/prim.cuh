@@ -324,6 +324,64 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// ------------------------------------------------- packed fp32 pairs --
+// sm_100 executes fp32 add / mul / fma on register pairs (one instruction for
+// two lanes' worth of work); a pair lives in a 64-bit register, low half first.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// max of three fp32 values in one instruction
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for a pair on the FMA / integer pipes instead of the special-function
+// unit (which does 16 exp2 per clock per SM, the softmax's bottleneck).
+// x = n + f with n = round(x) (added to 1.5 * 2^23, so n lands in the low
+// mantissa bits) and f in [-1/2, 1/2]; 2^f = 1 + f (c1 + f (c2 + f c3)),
+// coefficients fitted here by a minimax (linear program) fit of the relative
+// error on [-1/2, 1/2] with the constant term held at 1 (so 2^0 = 1 exactly):
+// max relative error 1.0e-4, below the bf16 / fp16 rounding of P. The result
+// is p * 2^n, 2^n built from its exponent bits; x <= -127 gives exactly 0.
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  const uint64_t xc = f2_pack(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
+  const uint64_t t = f2_add(xc, f2_pack(12582912.f, 12582912.f));       // 1.5 * 2^23 + n
+  const uint64_t n = f2_add(t, f2_pack(-12582912.f, -12582912.f));
+  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), xc);                // x - n
+  uint64_t p = f2_fma(f2_pack(0.055009059607982635f, 0.055009059607982635f), f,
+                      f2_pack(0.2422109693288803f, 0.2422109693288803f));
+  p = f2_fma(p, f, f2_pack(0.6932829022407532f, 0.6932829022407532f));
+  p = f2_fma(p, f, f2_pack(1.f, 1.f));
+  const uint32_t t0 = static_cast<uint32_t>(t), t1 = static_cast<uint32_t>(t >> 32);
+  const uint64_t scale = (static_cast<uint64_t>((t1 - 0x4B400000u + 127u) << 23) << 32) |
+                         ((t0 - 0x4B400000u + 127u) << 23);              // 2^n, 0 for n = -127
+  return f2_mul(p, scale);
+}
+
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);  // .x = lo (low half), .y = hi
   return *reinterpret_cast<uint32_t*>(&h);
