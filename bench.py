@@ -44,9 +44,9 @@ import synth  # noqa: E402
 WORKLOAD = dict(B=1, H=16, N=16384, d=128, causal=True)
 METRIC = "attention fwd+bwd TFLOP/s (bf16)"
 # DRAM bytes (read + write) of one d = 128 backward main-pass launch at WORKLOAD
-# (2.00 GB read + 1.16 GB written), from an ncu capture of that launch with the
+# (2.01 GB read + 1.16 GB written), from an ncu capture of that launch with the
 # current kernel; set to None whenever the kernel changes until captured again
-BWD_MAIN_TRAFFIC = None
+BWD_MAIN_TRAFFIC = 3.17e9
 
 
 def _peaks():
@@ -447,7 +447,7 @@ def run_case(fa, case, shape, causal, steps, warmup):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--steps", type=int, default=120)   # ~0.5 s timed: several clock samples
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-parts", action="store_true", help="headline only")
