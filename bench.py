@@ -317,6 +317,42 @@ def run_fp8(fa, steps, warmup, seed=1003):
     return {"ms": ms, "flops": attn_flops(B, H, N, d, False)}
 
 
+VARLEN = dict(n=16, lo=512, hi=8192, H=16, Hkv=4, d=128, causal=True, seed=1006)
+
+
+def varlen_flops(lens, H, d, causal):
+    """4 d H per visible (query, key) pair; causal with equal lengths sees
+    L (L + 1) / 2 pairs per sequence."""
+    pairs = sum(L * (L + 1) // 2 if causal else L * L for L in lens)
+    return 4.0 * d * H * pairs
+
+
+def run_fwd_varlen(fa, steps, warmup):
+    """Packed causal batch (lengths U[512, 8192], GQA 16 / 4 heads, d = 128)."""
+    w = VARLEN
+    lens = synth.packed_lengths(w["n"], w["lo"], w["hi"], w["seed"])
+    x = synth.packed_inputs(lens, lens, w["H"], w["Hkv"], w["d"], w["seed"], device="cuda")
+    cq, ck = torch.from_numpy(x["cu_q"]).cuda(), torch.from_numpy(x["cu_k"]).cuda()
+    o, lse = fa.fa_fwd_varlen(x["q"], x["k"], x["v"], cq, ck, max(lens), causal=w["causal"])
+
+    def op():
+        fa.fa_fwd_varlen(x["q"], x["k"], x["v"], cq, ck, max(lens), causal=w["causal"], o=o,
+                         lse=lse)
+    for _ in range(warmup):
+        op()
+    torch.cuda.synchronize()
+    a, b = _ev(), _ev()
+    a.record()
+    for _ in range(steps):
+        op()
+    b.record()
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_error() == fa.FA_OK
+    ms = a.elapsed_time(b) / steps
+    return {"ms": ms, "flops": varlen_flops(lens, w["H"], w["d"], w["causal"]),
+            "tokens": int(sum(lens))}
+
+
 # ---------------------------------------------------------- CPU baseline ---
 def _cores():
     try:
@@ -396,6 +432,11 @@ def _config():
 
 def run_case(fa, case, shape, causal, steps, warmup):
     """One operation at one size, for profilers: warmup + steps launches."""
+    if case == "fwd_varlen":              # the fixed packed workload (shape unused)
+        res = run_fwd_varlen(fa, steps, warmup)
+        print(json.dumps({"case": case, "ms": res["ms"],
+                          "TFLOP/s": res["flops"] / (res["ms"] / 1e3) / 1e12}))
+        return
     B, H, N, d = shape
     x = synth.attention_inputs(B, H, N, d, 1002, device="cuda", with_dout=case == "bwd")
     if case == "fwd":
@@ -524,6 +565,13 @@ def main():
             "shared_block_fraction": dec["shared_fraction"],
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm_gbs"], "traffic": None}}
+        vl = run_fwd_varlen(fa, args.steps, args.warmup)
+        parts["fwd_varlen"] = {
+            "workload": f"packed causal batch: {VARLEN['n']} sequences, lengths "
+                        f"U[{VARLEN['lo']}, {VARLEN['hi']}] (seed {VARLEN['seed']}), "
+                        f"H={VARLEN['H']} on Hkv={VARLEN['Hkv']}, d={VARLEN['d']}",
+            "ms": vl["ms"], "tokens": vl["tokens"],
+            "TFLOP/s": vl["flops"] / (vl["ms"] / 1e3) / 1e12}
         f8 = run_fp8(fa, args.steps, args.warmup)
         if "ms" in f8:
             t8 = f8["flops"] / (f8["ms"] / 1e3) / 1e12

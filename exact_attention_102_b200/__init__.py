@@ -34,7 +34,7 @@ EXPORTS = (
     "fa_status_str", "fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd",
     "paged_attn_decode_workspace_bytes", "paged_attn_decode", "fa_fp8_prepare",
     "fa_fwd_fp8", "fa_last_device_error", "fa_debug_wait_timeout",
-    "paged_attn_decode_noalloc", "fa_bwd_time_main_pass",
+    "paged_attn_decode_noalloc", "fa_bwd_time_main_pass", "fa_fwd_varlen",
 )
 
 
@@ -81,6 +81,8 @@ def lib() -> ctypes.CDLL:
     L.fa_last_device_error.argtypes = [vp]
     L.fa_bwd_time_main_pass.restype = ci
     L.fa_bwd_time_main_pass.argtypes = [vp, vp]
+    L.fa_fwd_varlen.restype = ci
+    L.fa_fwd_varlen.argtypes = [vp] * 7 + [ci] * 8 + [vp]
     L.fa_debug_wait_timeout.restype = ci
     L.fa_debug_wait_timeout.argtypes = [ctypes.c_uint, vp]
     _lib = L
@@ -134,6 +136,34 @@ def fa_fwd(q, k, v, causal=False, o=None, lse=None, stream=None):
     _need(lse, "lse", torch.float32, 3)
     _check("fa_fwd", lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
                                   B, H, N, d, int(bool(causal)), _stream(stream)))
+    return o, lse
+
+
+def fa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, causal=False, o=None,
+                  lse=None, stream=None):
+    """O, L for a packed batch: q [Tq, H, d], k / v [Tk, Hkv, d] bf16 (token-major),
+    cu_seqlens int32 [batch + 1] on the device; L is fp32 [H, Tq]. Causal is
+    aligned to the bottom right (query i of Lq sees keys j <= i + Lk - Lq)."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, torch.bfloat16, 3)
+    _need(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
+    _need(cu_seqlens_k, "cu_seqlens_k", torch.int32, 1)
+    if k.shape != v.shape or k.shape[2] != q.shape[2]:
+        raise ValueError("k and v must be [Tk, Hkv, d] with q's d")
+    if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 2:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both have batch + 1 entries")
+    Tq, H, d = q.shape
+    Tk, Hkv, _ = k.shape
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((H, Tq), dtype=torch.float32, device=q.device)
+    _need(o, "o", torch.bfloat16, 3)
+    _need(lse, "lse", torch.float32, 2)
+    _check("fa_fwd_varlen",
+           lib().fa_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens_q),
+                               _ptr(cu_seqlens_k), cu_seqlens_q.numel() - 1, int(max_seqlen_q),
+                               Tq, Tk, H, Hkv, d, int(bool(causal)), _stream(stream)))
     return o, lse
 
 

@@ -58,14 +58,14 @@ EncodeTiledFn encode_fn() {
 // 128-byte swizzle unless told otherwise, zero fill outside the tensor.
 bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int elem_bytes, int d,
               int n, int bh, uint32_t box_x, uint32_t box_y,
-              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
+              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B, uint32_t box_z = 1) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n),
                         static_cast<cuuint64_t>(bh)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * elem_bytes,
                            static_cast<cuuint64_t>(n) * d * elem_bytes};
-  cuuint32_t box[3] = {box_x, box_y, 1};
+  cuuint32_t box[3] = {box_x, box_y, box_z};
   cuuint32_t es[3] = {1, 1, 1};
   memset(m, 0, sizeof(*m));
   CUresult r = fn(m, dt, 3, const_cast<void*>(ptr), dims, strides, box, es,
@@ -132,6 +132,55 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   a.n_pairs = (N + 255) / 256;
   a.scale_log2 = kLog2e / sqrtf(static_cast<float>(d));
   a.err = err;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = (d == 128) ? fa::launch_fwd<128>(tq, tk, tv, a, s)
+                             : fa::launch_fwd<64>(tq, tk, tv, a, s);
+  return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                         const int* cu_seqlens_q, const int* cu_seqlens_k, int batch,
+                         int max_seqlen_q, int total_q, int total_k, int H, int Hkv, int d,
+                         int causal, void* stream) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || lse == nullptr ||
+      cu_seqlens_q == nullptr || cu_seqlens_k == nullptr)
+    return FA_ERR_INVALID_ARG;
+  if (batch < 1 || H < 1 || Hkv < 1 || H % Hkv != 0 || max_seqlen_q < 1 || total_q < 1 ||
+      total_k < 1 || max_seqlen_q > total_q)
+    return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const long long n_pairs = (static_cast<long long>(max_seqlen_q) + 255) / 256;
+  if (static_cast<long long>(batch) * H * n_pairs > (1ll << 31) - 1 ||
+      static_cast<long long>(total_q) * H > (1ll << 31) - 1 ||
+      static_cast<long long>(total_k) * Hkv > (1ll << 31) - 1)
+    return FA_ERR_UNSUPPORTED;
+  uint32_t* err = error_word_ptr();
+  if (err == nullptr) return FA_ERR_LAUNCH;
+  // token-major views [T][heads][d]: x = head dim, y = head, z = token; a box is
+  // 64 columns x 1 head x 128 tokens, the same 128 rows x 128 B in shared memory
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, H, total_q, 64, 1,
+                CU_TENSOR_MAP_SWIZZLE_128B, 128) ||
+      !make_map(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Hkv, total_k, 64, 1,
+                CU_TENSOR_MAP_SWIZZLE_128B, 128) ||
+      !make_map(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Hkv, total_k, 64, 1,
+                CU_TENSOR_MAP_SWIZZLE_128B, 128))
+    return FA_ERR_LAUNCH;
+  fa::FwdArgs a;
+  a.o = o;
+  a.lse = lse;
+  a.B = batch;
+  a.H = H;
+  a.N = max_seqlen_q;
+  a.causal = causal ? 1 : 0;
+  a.n_pairs = static_cast<int>(n_pairs);
+  a.scale_log2 = kLog2e / sqrtf(static_cast<float>(d));
+  a.err = err;
+  a.cu_q = cu_seqlens_q;
+  a.cu_k = cu_seqlens_k;
+  a.Hkv = Hkv;
+  a.Tq = total_q;
+  a.Tk = total_k;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = (d == 128) ? fa::launch_fwd<128>(tq, tk, tv, a, s)
                              : fa::launch_fwd<64>(tq, tk, tv, a, s);

@@ -92,16 +92,45 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   const int BH = a.B * a.H;
   const int pair = a.n_pairs - 1 - static_cast<int>(blockIdx.x) / BH;  // heaviest first
   const int bh = static_cast<int>(blockIdx.x) % BH;
-  const int nkb = (a.N + C::BN - 1) / C::BN;
 
-  // per-tile extent: rows [q0, q0+128), key blocks [0, nkb_t)
+  // The problem this CTA works on: Lq queries against Lk keys. BHND: one
+  // (batch, head) slice of length N, TMA coordinates (row, bh). Packed mode:
+  // sequence b of the batch, TMA coordinates (head, token).
+  const bool packed = a.cu_q != nullptr;
+  int Lq = a.N, Lk = a.N, tq0 = 0, tk0 = 0, hq = 0, hk = 0;
+  if (packed) {
+    const int b = bh / a.H;
+    hq = bh % a.H;
+    hk = hq / (a.H / a.Hkv);
+    tq0 = a.cu_q[b];
+    tk0 = a.cu_k[b];
+    Lq = a.cu_q[b + 1] - tq0;
+    Lk = a.cu_k[b + 1] - tk0;
+    if (tq0 < 0 || tk0 < 0 || Lq < 0 || Lk < 0 || Lq > a.N || tq0 + Lq > a.Tq || tk0 + Lk > a.Tk) {
+      if (threadIdx.x == 0 && pair == a.n_pairs - 1) atomicCAS(a.err, 0u, kErrBadIndex + 1);
+      Lq = 0;                       // nothing is read or written for this sequence
+      Lk = 0;
+    }
+  }
+  // causal: query row i sees keys j <= i + off (off = 0 when Lq == Lk)
+  const int off = a.causal ? Lk - Lq : 0;
+  const int nkb = (Lk + C::BN - 1) / C::BN;
+
+  // per-tile extent: rows [q0, q0+128), key blocks [0, nkb_t); a tile with rows
+  // but no visible key (nkb_t = 0) still writes O = 0 and L = -inf
   int q0[2], nkb_t[2];
+  bool rows_t[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     q0[t] = (pair * 2 + t) * C::BM;
-    nkb_t[t] = (q0[t] >= a.N) ? 0 : (a.causal ? min(nkb, pair * 2 + t + 1) : nkb);
+    rows_t[t] = q0[t] < Lq;
+    const int last_key = min(q0[t] + C::BM - 1, Lq - 1) + off;  // causal: last key any row sees
+    nkb_t[t] = !rows_t[t] ? 0 : !a.causal ? nkb : last_key < 0 ? 0 : min(nkb, last_key / C::BN + 1);
   }
   const int nkb_cta = max(nkb_t[0], nkb_t[1]);
+  // TMA coordinates (y, z) of Q row q and of K / V row k of this problem
+  auto q_yz = [&](int q) { return packed ? make_int2(hq, tq0 + q) : make_int2(q, bh); };
+  auto k_yz = [&](int k) { return packed ? make_int2(hk, tk0 + k) : make_int2(k, bh); };
 
   auto bar = [&](int i) -> uint32_t { return base + C::BAR_OFF + 8 * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
@@ -141,9 +170,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       mbar_arrive_expect_tx(bar(C::B_Q), nq * C::TILE);
       for (int t = 0; t < 2; ++t) {
         if (nkb_t[t] == 0) continue;
+        const int2 yz = q_yz(q0[t]);
         for (int c = 0; c < C::NCHUNK; ++c)
           tma_load_3d(base + C::Q_OFF + t * C::TILE + c * C::CHUNK, &tmQ, bar(C::B_Q), c * 64,
-                      q0[t], bh);
+                      yz.x, yz.y);
       }
       int it = 0;
       bool ok = true;
@@ -155,9 +185,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           if (!ok) break;
           mbar_arrive_expect_tx(bar(C::B_KVF + s), C::TILE);
           const CUtensorMap* m = (w == 0) ? &tmK : &tmV;
+          const int2 yz = k_yz(j * C::BN);
           for (int c = 0; c < C::NCHUNK; ++c)
             tma_load_3d(base + C::RING_OFF + s * C::TILE + c * C::CHUNK, m, bar(C::B_KVF + s),
-                        c * 64, j * C::BN, bh);
+                        c * 64, yz.x, yz.y);
         }
       }
       // drain: make sure the last loads issued have landed before teardown
@@ -252,7 +283,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     const uint32_t s_addr = tmem + lane_off + C::s_col(t);
     const uint32_t o_addr = tmem + lane_off + C::o_col(t);
     const int row = q0[t] + r;
-    const int limit = a.causal ? min(row, a.N - 1) : a.N - 1;  // last visible key
+    const int limit = a.causal ? min(row + off, Lk - 1) : Lk - 1;  // last visible key (< 0: none)
     const float sl2 = a.scale_log2;
     float m_run = -INFINITY;
     float l_run = 0.f;    // sum of fp32 P
@@ -350,20 +381,31 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       warp_arrive(bar(C::B_P + t));
     }
     // ------------------------------------------------------------ epilogue
+    // output row of query `row`: BHND [bh][row] or packed [token][head]
+    const size_t orow_idx = packed ? static_cast<size_t>(tq0 + row) * a.H + hq
+                                   : static_cast<size_t>(bh) * a.N + row;
+    const size_t lse_idx = packed ? static_cast<size_t>(hq) * a.Tq + tq0 + row
+                                  : static_cast<size_t>(bh) * a.N + row;
+    if (ok && nkb_t[t] == 0 && rows_t[t] && row < Lq) {   // sees no key: O = 0, L = -inf
+      uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) + orow_idx * D);
+#pragma unroll
+      for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
+      a.lse[lse_idx] = -INFINITY;
+    }
     if (ok && nkb_t[t] > 0) {
       ok = __all_sync(0xffffffffu,
                       mbar_wait(bar(C::B_O + t), 0, a.err, kSiteEpi, abort_flag));
       if (ok) {
         tc_fence_after();
-        const float inv_l = 1.f / lr_run;
-        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) +
-                              (static_cast<size_t>(bh) * a.N + row) * D;
+        // a row that saw no key has l = 0: O = 0, and L = m + log l = -inf
+        const float inv_l = lr_run > 0.f ? 1.f / lr_run : 0.f;
+        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + orow_idx * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t orr[32];
           tmem_ld32(o_addr + c * 32, orr);
           tmem_ld_wait();
-          if (row < a.N) {
+          if (row < Lq) {
             uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -376,8 +418,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             }
           }
         }
-        if (row < a.N)
-          a.lse[static_cast<size_t>(bh) * a.N + row] = (m_run + log2f(l_run)) * 0.6931471805599453f;
+        if (row < Lq) a.lse[lse_idx] = (m_run + log2f(l_run)) * 0.6931471805599453f;
       }
     }
     tc_fence_before();

@@ -8,13 +8,20 @@
 namespace fa {
 
 struct FwdArgs {
-  void* o;            // bf16 [B][H][N][D]
-  float* lse;         // fp32 [B][H][N]
-  int B, H, N;
+  void* o;            // bf16 [B][H][N][D]            (packed mode: [Tq][H][D])
+  float* lse;         // fp32 [B][H][N]               (packed mode: [H][Tq])
+  int B, H, N;        // packed mode: N = the longest query sequence
   int causal;
   int n_pairs;        // ceil(N / 256): pairs of 128-row Q tiles per head
   float scale_log2;   // softmax scale * log2(e)
   uint32_t* err;      // device error word
+  // packed variable-length mode when cu_q != nullptr: sequence b owns query
+  // rows [cu_q[b], cu_q[b+1]) of Q / O and key rows [cu_k[b], cu_k[b+1]) of
+  // K / V; query head h reads KV head h / (H / Hkv); causal is aligned to the
+  // bottom right (query i of Lq sees keys j <= i + Lk - Lq)
+  const int* cu_q = nullptr;
+  const int* cu_k = nullptr;
+  int Hkv = 0, Tq = 0, Tk = 0;
 };
 
 template <int D>

@@ -116,6 +116,40 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
                  int B, int H, int N, int d, int causal, void* stream);
 
 /*
+ * fa_fwd_varlen — the forward over a packed batch of variable-length
+ * sequences, with query and key lengths that may differ and grouped KV heads.
+ * Same method as fa_fwd; the layouts generalise its BHND view: every (sequence,
+ * head) is an independent problem ("Flash Attention 再学习", Flash Attention
+ * v2, thread blocks parallel over batch, heads and row blocks).
+ *   q, o          : bf16 [total_q][H][d], token-major; sequence b owns rows
+ *                   [cu_seqlens_q[b], cu_seqlens_q[b+1]).
+ *   k, v          : bf16 [total_k][Hkv][d]; sequence b owns rows
+ *                   [cu_seqlens_k[b], cu_seqlens_k[b+1]).
+ *   lse           : fp32 [H][total_q], natural log.
+ *   cu_seqlens_q/k: int32 [batch + 1] device arrays, non-decreasing,
+ *                   cu[0] = 0, cu[batch] <= total. Every query length must be
+ *                   <= max_seqlen_q (it sizes the grid); key lengths may be 0.
+ *   H, Hkv        : query head h reads KV head h / (H / Hkv); H % Hkv == 0.
+ *   causal        : aligned to the bottom right, so query i of a sequence with
+ *                   Lq queries and Lk keys sees keys j <= i + Lk - Lq (for
+ *                   Lq == Lk this is fa_fwd's mask; for Lq = 1 the query sees
+ *                   every key, as in decoding). A query that sees no key
+ *                   (Lq > Lk, or Lk = 0) gets O = 0 and L = -inf.
+ * The inputs must be finite (rows of the next sequence are read and masked).
+ * Errors: FA_ERR_INVALID_ARG for NULL / unaligned pointers, batch, H, Hkv,
+ * max_seqlen_q, totals < 1, H % Hkv != 0 or max_seqlen_q > total_q;
+ * FA_ERR_UNSUPPORTED for d not in {64, 128} or sizes beyond 32-bit indexing;
+ * FA_ERR_LAUNCH as fa_fwd. Inconsistent cu_seqlens (a length < 0, a query
+ * length > max_seqlen_q, or a range past the totals) are detected on the
+ * device: that sequence is skipped and fa_last_device_error() reports
+ * FA_ERR_INVALID_ARG.
+ */
+FA_API fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                        const int* cu_seqlens_q, const int* cu_seqlens_k, int batch,
+                        int max_seqlen_q, int total_q, int total_k, int H, int Hkv, int d,
+                        int causal, void* stream);
+
+/*
  * Bytes of device workspace paged_attn_decode needs for split partials
  * (fp32 O and L per (sequence, query head, split)) and a work counter, when
  * no sequence is longer than max_ctx tokens.

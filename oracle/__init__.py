@@ -12,8 +12,9 @@ attention
     The plain definitions: 3-pass safe-softmax attention forward with the
     per-row logsumexp, its analytic gradients, the paged-KV decode (gather
     through the block table, then the forward definition), the logsumexp
-    merge of split partials, and the FP8 e4m3 block quantiser used by the
-    diagnostic FP8 oracle.
+    merge of split partials, the packed variable-length form (sequences of
+    unequal query / key lengths, grouped KV heads, bottom-right causal), and
+    the FP8 e4m3 block quantiser used by the diagnostic FP8 oracle.
 online
     A second, independent implementation of the forward: the tiled one-pass
     online-softmax recurrence (running max m, running sum l, unnormalised O
@@ -29,6 +30,7 @@ from .attention import (  # noqa: F401
     attention_fwd,
     attention_bwd,
     attention_rows,
+    attention_varlen,
     paged_decode,
     combine_partials,
     round_bf16,

@@ -59,12 +59,20 @@ def attention_rows(q_rows, row_idx, k, v, causal, scale=None):
     if causal:
         keys = np.arange(k.shape[0])[None, :]
         s = np.where(keys <= np.asarray(row_idx)[:, None], s, -np.inf)
+    if s.shape[1] == 0:                        # no keys at all
+        s = np.full((s.shape[0], 1), -np.inf)
+        v = np.zeros((1, v.shape[-1]))
     m = s.max(axis=1)                          # pass 1: row max
-    e = np.exp(s - m[:, None])                 # masked entries give exp(-inf) = 0
+    # a row that sees no key (possible only for the packed, unequal-length
+    # form): P = 0, O = 0, L = -inf
+    empty = m == -np.inf
+    m_safe = np.where(empty, 0.0, m)
+    e = np.exp(s - m_safe[:, None])            # masked entries give exp(-inf) = 0
     l = e.sum(axis=1)                          # pass 2: row sum
-    p = e / l[:, None]                         # pass 3: normalise
+    p = e / np.where(empty, 1.0, l)[:, None]   # pass 3: normalise
     o = p @ v
-    lse = m + np.log(l)
+    with np.errstate(divide="ignore"):
+        lse = np.where(empty, -np.inf, m_safe + np.log(np.where(empty, 1.0, l)))
     return o, lse, p
 
 
@@ -93,6 +101,45 @@ def attention_fwd(q, k, v, causal=False, scale=None):
             o[bh, rows] = ob
             lse[bh, rows] = lb
     return o.reshape(lead + (n, v2.shape[-1])), lse.reshape(lead + (n,))
+
+
+def attention_varlen(q, k, v, cu_q, cu_k, causal=False, scale=None):
+    """Exact attention over a packed batch of variable-length sequences.
+
+    q: [Tq, H, d], k, v: [Tk, Hkv, d] (token-major); cu_q, cu_k: [B + 1]
+    sequence starts. Sequence b is queries cu_q[b]..cu_q[b+1]-1 against keys
+    cu_k[b]..cu_k[b+1]-1; query head h reads KV head h // (H // Hkv). Every
+    (sequence, head) is an independent instance of the forward definition
+    ([FA-relearn] "Flash Attention v2", thread blocks over batch and heads).
+    The pages define the causal mask only for equal lengths (query i sees keys
+    j <= i); for Lq queries and Lk keys it is read aligned to the bottom right,
+    query i seeing keys j <= i + Lk - Lq, which is the equal-length mask when
+    Lq = Lk and the decoding rule (the newest token sees every cached key) when
+    Lq = 1. A query seeing no key has O = 0 and L = -inf.
+    Returns (O [Tq, H, d], L [H, Tq]).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    cu_q = np.asarray(cu_q)
+    cu_k = np.asarray(cu_k)
+    tq, h, d = q.shape
+    hkv = k.shape[1]
+    group = h // hkv
+    o = np.zeros_like(q)
+    lse = np.full((h, tq), -np.inf)
+    for b in range(len(cu_q) - 1):
+        q0, q1, k0, k1 = int(cu_q[b]), int(cu_q[b + 1]), int(cu_k[b]), int(cu_k[b + 1])
+        lq, lk = q1 - q0, k1 - k0
+        if lq == 0:
+            continue
+        pos = np.arange(lq) + (lk - lq)          # causal position of each query among the keys
+        for hh in range(h):
+            ob, lb, _ = attention_rows(q[q0:q1, hh], pos, k[k0:k1, hh // group],
+                                       v[k0:k1, hh // group], causal, scale)
+            o[q0:q1, hh] = ob
+            lse[hh, q0:q1] = lb
+    return o, lse
 
 
 def attention_bwd(q, k, v, do, causal=False, scale=None, o=None):

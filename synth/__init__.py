@@ -60,6 +60,27 @@ def attention_inputs(B, H, N, d, seed, device="cpu", with_dout=True, outlier_p=0
     return out
 
 
+def packed_inputs(lens_q, lens_k, H, Hkv, d, seed, device="cpu"):
+    """A packed variable-length batch: Q [Tq, H, d], K and V [Tk, Hkv, d] bf16
+    (token-major, N(0,1) drawn as float32 in the order Q, K, V from one
+    generator) and the int32 sequence starts cu_q, cu_k (numpy, [B + 1])."""
+    cu_q = np.concatenate([[0], np.cumsum(lens_q)]).astype(np.int32)
+    cu_k = np.concatenate([[0], np.cumsum(lens_k)]).astype(np.int32)
+    g = _gen(seed, device)
+    out = {}
+    for name, shape in (("q", (int(cu_q[-1]), H, d)), ("k", (max(int(cu_k[-1]), 1), Hkv, d)),
+                        ("v", (max(int(cu_k[-1]), 1), Hkv, d))):
+        out[name] = torch.randn(shape, generator=g, device=device,
+                                dtype=torch.float32).to(torch.bfloat16)
+    out["cu_q"], out["cu_k"] = cu_q, cu_k
+    return out
+
+
+def packed_lengths(n, lo, hi, seed):
+    """n sequence lengths, integers uniform on [lo, hi], seeded."""
+    return np.random.default_rng(seed).integers(lo, hi + 1, n).astype(np.int64).tolist()
+
+
 def fp8_inputs(B, H, N, d, seed, device="cpu"):
     """The FP8 workload: N(0,1) with 0.1% of entries scaled by 50, bf16."""
     return attention_inputs(B, H, N, d, seed, device=device, with_dout=False,

@@ -117,3 +117,23 @@ def test_decode_noalloc_rejects_oversize_without_gpu():
                                        32768, None) == fa.FA_ERR_WORKSPACE
     assert L.paged_attn_decode_noalloc(g, g, g, 1000, g, 2048, g, g, g, 0, 32, 8, 128, 16,
                                        32768, None) == fa.FA_ERR_INVALID_ARG
+
+
+def test_fwd_varlen_rejects_bad_arguments_without_a_gpu():
+    """Argument checks run before any CUDA call."""
+    L = fa.lib()
+    p = ctypes.c_void_p(256)            # aligned, never dereferenced
+    null = ctypes.c_void_p(0)
+    s = ctypes.c_void_p(0)
+    call = lambda *a: L.fa_fwd_varlen(*a)
+    ok_args = [p, p, p, p, p, p, p, 2, 64, 128, 128, 8, 2, 128, 1, s]
+    args = list(ok_args); args[0] = null
+    assert call(*args) == fa.FA_ERR_INVALID_ARG            # NULL q
+    args = list(ok_args); args[12] = 3
+    assert call(*args) == fa.FA_ERR_INVALID_ARG            # H % Hkv != 0
+    args = list(ok_args); args[8] = 200
+    assert call(*args) == fa.FA_ERR_INVALID_ARG            # max_seqlen_q > total_q
+    args = list(ok_args); args[13] = 96
+    assert call(*args) == fa.FA_ERR_UNSUPPORTED            # d not in {64, 128}
+    args = list(ok_args); args[7] = 0
+    assert call(*args) == fa.FA_ERR_INVALID_ARG            # batch < 1

@@ -373,3 +373,103 @@ def test_round_bf16_matches_torch_cast():
     # 1 + 3*2^-8 is halfway between 1 + 2^-7 and 1 + 2^-6 -> 1 + 2^-6 (even)
     np.testing.assert_array_equal(oracle.round_bf16([1 + 2 ** -8, 1 + 3 * 2 ** -8, -3.0, 0.0]),
                                   [1.0, 1 + 2 ** -6, -3.0, 0.0])
+
+
+# ---------------------------------------------------------------- packed form
+def _varlen_case(lens_q, lens_k, H, Hkv, d, seed):
+    rng = np.random.default_rng(seed)
+    cu_q = np.concatenate([[0], np.cumsum(lens_q)]).astype(np.int32)
+    cu_k = np.concatenate([[0], np.cumsum(lens_k)]).astype(np.int32)
+    q = rng.standard_normal((cu_q[-1], H, d))
+    k = rng.standard_normal((cu_k[-1], Hkv, d))
+    v = rng.standard_normal((cu_k[-1], Hkv, d))
+    return q, k, v, cu_q, cu_k
+
+
+def test_varlen_equal_lengths_match_the_bhnd_forward():
+    """Equal lengths, H = Hkv: the packed form is attention_fwd on [B, H, N, d]."""
+    B, H, N, d = 3, 2, 37, 8
+    q, k, v, cu_q, cu_k = _varlen_case([N] * B, [N] * B, H, H, d, 71)
+    for causal in (False, True):
+        o, lse = oracle.attention_varlen(q, k, v, cu_q, cu_k, causal)
+        bhnd = lambda t: t.reshape(B, N, H, d).transpose(0, 2, 1, 3)
+        o2, l2 = oracle.attention_fwd(bhnd(q), bhnd(k), bhnd(v), causal)
+        np.testing.assert_allclose(bhnd(o), o2, rtol=0, atol=1e-14)
+        np.testing.assert_allclose(lse.reshape(H, B, N).transpose(1, 0, 2), l2, rtol=0, atol=1e-13)
+
+
+def test_varlen_brute_force_cross_lengths_gqa_bottom_right():
+    """Pure-Python loops over every (sequence, head, query): unequal lengths,
+    Hkv < H, bottom-right causal including queries that see no key."""
+    lens_q, lens_k = [3, 5, 1, 4], [4, 2, 6, 0]
+    H, Hkv, d = 4, 2, 3
+    q, k, v, cu_q, cu_k = _varlen_case(lens_q, lens_k, H, Hkv, d, 72)
+    for causal in (False, True):
+        o, lse = oracle.attention_varlen(q, k, v, cu_q, cu_k, causal)
+        for b in range(4):
+            lq, lk = lens_q[b], lens_k[b]
+            for h in range(H):
+                for i in range(lq):
+                    row = cu_q[b] + i
+                    keys = [j for j in range(lk) if not causal or j <= i + lk - lq]
+                    if not keys:
+                        assert np.all(o[row, h] == 0) and lse[h, row] == -np.inf
+                        continue
+                    s = [float(q[row, h] @ k[cu_k[b] + j, h // 2]) / math.sqrt(d) for j in keys]
+                    mx = max(s)
+                    w = [math.exp(x - mx) for x in s]
+                    tot = sum(w)
+                    exp_o = sum(wi / tot * v[cu_k[b] + j, h // 2] for wi, j in zip(w, keys))
+                    np.testing.assert_allclose(o[row, h], exp_o, rtol=1e-12, atol=1e-13)
+                    assert abs(lse[h, row] - (mx + math.log(tot))) < 1e-12
+
+
+def test_varlen_single_query_is_the_decode_rule():
+    """Lq = 1, causal: the query sees every key, as the paged decode's newest
+    token does (decode definition on an identity block table)."""
+    lens_k = [16, 48, 32]
+    H, Hkv, d = 8, 2, 16
+    q, k, v, cu_q, cu_k = _varlen_case([1, 1, 1], lens_k, H, Hkv, d, 73)
+    o, lse = oracle.attention_varlen(q, k, v, cu_q, cu_k, causal=True)
+    nb = [n // 16 for n in lens_k]
+    table = np.zeros((3, max(nb)), dtype=np.int32)
+    kc = np.zeros((sum(nb), Hkv, 16, d))
+    vc = np.zeros_like(kc)
+    p = 0
+    for s_ in range(3):
+        for j in range(nb[s_]):
+            table[s_, j] = p
+            rows = slice(cu_k[s_] + 16 * j, cu_k[s_] + 16 * j + 16)
+            kc[p] = k[rows].transpose(1, 0, 2)
+            vc[p] = v[rows].transpose(1, 0, 2)
+            p += 1
+    od, ld = oracle.paged_decode(q, kc, vc, table, np.array(lens_k))
+    np.testing.assert_allclose(o, od, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse, ld.T, rtol=0, atol=1e-13)
+
+
+def test_varlen_gqa_equals_repeated_kv_heads():
+    lens = [7, 20]
+    q, k, v, cu_q, cu_k = _varlen_case(lens, lens, 6, 3, 8, 74)
+    o, lse = oracle.attention_varlen(q, k, v, cu_q, cu_k, causal=True)
+    o2, l2 = oracle.attention_varlen(q, np.repeat(k, 2, axis=1), np.repeat(v, 2, axis=1),
+                                     cu_q, cu_k, causal=True)
+    np.testing.assert_array_equal(o, o2)
+    np.testing.assert_array_equal(lse, l2)
+
+
+def test_varlen_against_torch_sdpa():
+    """Library routine: torch float64 scaled_dot_product_attention per
+    sequence, with an explicit bottom-right mask."""
+    lens_q, lens_k = [5, 9], [12, 9]
+    q, k, v, cu_q, cu_k = _varlen_case(lens_q, lens_k, 2, 2, 16, 75)
+    o, _ = oracle.attention_varlen(q, k, v, cu_q, cu_k, causal=True)
+    for b in range(2):
+        qs = torch.from_numpy(q[cu_q[b]:cu_q[b + 1]].transpose(1, 0, 2).copy())
+        ks = torch.from_numpy(k[cu_k[b]:cu_k[b + 1]].transpose(1, 0, 2).copy())
+        vs = torch.from_numpy(v[cu_k[b]:cu_k[b + 1]].transpose(1, 0, 2).copy())
+        lq, lk = lens_q[b], lens_k[b]
+        mask = torch.from_numpy(np.arange(lk)[None, :] <= np.arange(lq)[:, None] + lk - lq)
+        ref = torch.nn.functional.scaled_dot_product_attention(qs, ks, vs, attn_mask=mask)
+        np.testing.assert_allclose(o[cu_q[b]:cu_q[b + 1]], ref.numpy().transpose(1, 0, 2),
+                                   rtol=0, atol=1e-12)
