@@ -335,22 +335,36 @@ def run_fwd_varlen(fa, steps, warmup):
     cq, ck = torch.from_numpy(x["cu_q"]).cuda(), torch.from_numpy(x["cu_k"]).cuda()
     o, lse = fa.fa_fwd_varlen(x["q"], x["k"], x["v"], cq, ck, max(lens), causal=w["causal"])
 
-    def op():
+    g = torch.randn(x["q"].shape, generator=torch.Generator(device="cuda").manual_seed(w["seed"]),
+                    device="cuda").to(torch.bfloat16)
+    grads = [torch.empty(t.shape, dtype=torch.float32, device="cuda")
+             for t in (x["q"], x["k"], x["k"])]
+    wsp = torch.empty(fa.fa_bwd_varlen_workspace_bytes(w["n"], max(lens), x["q"].shape[0],
+                                                       x["k"].shape[0], w["H"], w["Hkv"], w["d"]),
+                      dtype=torch.uint8, device="cuda")
+
+    def fwd():
         fa.fa_fwd_varlen(x["q"], x["k"], x["v"], cq, ck, max(lens), causal=w["causal"], o=o,
                          lse=lse)
-    for _ in range(warmup):
-        op()
-    torch.cuda.synchronize()
-    a, b = _ev(), _ev()
-    a.record()
-    for _ in range(steps):
-        op()
-    b.record()
-    torch.cuda.synchronize()
-    assert fa.fa_last_device_error() == fa.FA_OK
-    ms = a.elapsed_time(b) / steps
-    return {"ms": ms, "flops": varlen_flops(lens, w["H"], w["d"], w["causal"]),
-            "tokens": int(sum(lens))}
+
+    def bwd():
+        fa.fa_bwd_varlen(x["q"], x["k"], x["v"], o, lse, g, cq, ck, max(lens), max(lens),
+                         causal=w["causal"], dq=grads[0], dk=grads[1], dv=grads[2], workspace=wsp)
+
+    res = {"flops": varlen_flops(lens, w["H"], w["d"], w["causal"]), "tokens": int(sum(lens))}
+    for name, op in (("ms", fwd), ("bwd_ms", bwd)):
+        for _ in range(warmup):
+            op()
+        torch.cuda.synchronize()
+        a, b = _ev(), _ev()
+        a.record()
+        for _ in range(steps):
+            op()
+        b.record()
+        torch.cuda.synchronize()
+        assert fa.fa_last_device_error() == fa.FA_OK
+        res[name] = a.elapsed_time(b) / steps
+    return res
 
 
 # ---------------------------------------------------------- CPU baseline ---
@@ -435,7 +449,9 @@ def run_case(fa, case, shape, causal, steps, warmup):
     if case == "fwd_varlen":              # the fixed packed workload (shape unused)
         res = run_fwd_varlen(fa, steps, warmup)
         print(json.dumps({"case": case, "ms": res["ms"],
-                          "TFLOP/s": res["flops"] / (res["ms"] / 1e3) / 1e12}))
+                          "TFLOP/s": res["flops"] / (res["ms"] / 1e3) / 1e12,
+                          "bwd_ms": res["bwd_ms"],
+                          "bwd_TFLOP/s": 2.5 * res["flops"] / (res["bwd_ms"] / 1e3) / 1e12}))
         return
     B, H, N, d = shape
     x = synth.attention_inputs(B, H, N, d, 1002, device="cuda", with_dout=case == "bwd")
@@ -571,7 +587,8 @@ def main():
                         f"U[{VARLEN['lo']}, {VARLEN['hi']}] (seed {VARLEN['seed']}), "
                         f"H={VARLEN['H']} on Hkv={VARLEN['Hkv']}, d={VARLEN['d']}",
             "ms": vl["ms"], "tokens": vl["tokens"],
-            "TFLOP/s": vl["flops"] / (vl["ms"] / 1e3) / 1e12}
+            "TFLOP/s": vl["flops"] / (vl["ms"] / 1e3) / 1e12,
+            "bwd_ms": vl["bwd_ms"], "bwd_TFLOP/s": 2.5 * vl["flops"] / (vl["bwd_ms"] / 1e3) / 1e12}
         f8 = run_fp8(fa, args.steps, args.warmup)
         if "ms" in f8:
             t8 = f8["flops"] / (f8["ms"] / 1e3) / 1e12

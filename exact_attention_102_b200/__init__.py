@@ -35,6 +35,7 @@ EXPORTS = (
     "paged_attn_decode_workspace_bytes", "paged_attn_decode", "fa_fp8_prepare",
     "fa_fwd_fp8", "fa_last_device_error", "fa_debug_wait_timeout",
     "paged_attn_decode_noalloc", "fa_bwd_time_main_pass", "fa_fwd_varlen",
+    "fa_bwd_varlen_workspace_bytes", "fa_bwd_varlen",
 )
 
 
@@ -83,6 +84,10 @@ def lib() -> ctypes.CDLL:
     L.fa_bwd_time_main_pass.argtypes = [vp, vp]
     L.fa_fwd_varlen.restype = ci
     L.fa_fwd_varlen.argtypes = [vp] * 7 + [ci] * 8 + [vp]
+    L.fa_bwd_varlen_workspace_bytes.restype = sz
+    L.fa_bwd_varlen_workspace_bytes.argtypes = [ci] * 7
+    L.fa_bwd_varlen.restype = ci
+    L.fa_bwd_varlen.argtypes = [vp] * 10 + [sz, vp, vp] + [ci] * 9 + [vp]
     L.fa_debug_wait_timeout.restype = ci
     L.fa_debug_wait_timeout.argtypes = [ctypes.c_uint, vp]
     _lib = L
@@ -165,6 +170,39 @@ def fa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, causal=Fals
                                _ptr(cu_seqlens_k), cu_seqlens_q.numel() - 1, int(max_seqlen_q),
                                Tq, Tk, H, Hkv, d, int(bool(causal)), _stream(stream)))
     return o, lse
+
+
+def fa_bwd_varlen_workspace_bytes(batch, max_seqlen_q, total_q, total_k, H, Hkv, d):
+    return int(lib().fa_bwd_varlen_workspace_bytes(batch, max_seqlen_q, total_q, total_k, H, Hkv,
+                                                   d))
+
+
+def fa_bwd_varlen(q, k, v, o, lse, do, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                  causal=False, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """dQ [Tq, H, d], dK, dV [Tk, Hkv, d] (fp32) of fa_fwd_varlen's attention."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
+        _need(t, n, torch.bfloat16, 3)
+    _need(lse, "lse", torch.float32, 2)
+    _need(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
+    _need(cu_seqlens_k, "cu_seqlens_k", torch.int32, 1)
+    Tq, H, d = q.shape
+    Tk, Hkv, _ = k.shape
+    batch = cu_seqlens_q.numel() - 1
+    dq = torch.empty(q.shape, dtype=torch.float32, device=q.device) if dq is None else dq
+    dk = torch.empty(k.shape, dtype=torch.float32, device=q.device) if dk is None else dk
+    dv = torch.empty(k.shape, dtype=torch.float32, device=q.device) if dv is None else dv
+    for n, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _need(t, n, torch.float32, 3)
+    need = fa_bwd_varlen_workspace_bytes(batch, max_seqlen_q, Tq, Tk, H, Hkv, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _check("fa_bwd_varlen",
+           lib().fa_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq),
+                               _ptr(dk), _ptr(dv), _ptr(workspace), workspace.numel(),
+                               _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), batch, int(max_seqlen_q),
+                               int(max_seqlen_k), Tq, Tk, H, Hkv, d, int(bool(causal)),
+                               _stream(stream)))
+    return dq, dk, dv
 
 
 def fa_bwd_workspace_bytes(B, H, N, d):

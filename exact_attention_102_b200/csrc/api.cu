@@ -260,6 +260,102 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
+size_t fa_bwd_varlen_workspace_bytes(int batch, int max_seqlen_q, int total_q, int total_k, int H,
+                                     int Hkv, int d) {
+  if (batch < 1 || max_seqlen_q < 1 || total_q < 1 || total_k < 1 || H < 1 || Hkv < 1 || d < 1)
+    return 0;
+  const size_t rows = static_cast<size_t>(batch) * H *
+                      ((static_cast<size_t>(max_seqlen_q) + 127) / 128 * 128);
+  const size_t nq = static_cast<size_t>(total_q) * H * d, nk = static_cast<size_t>(total_k) * Hkv * d;
+  return 2 * round256(rows * sizeof(float)) + 2 * round256(nq * 2) + 2 * round256(nk * 2);
+}
+
+fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
+                        const float* lse, const void* dout, float* dq, float* dk, float* dv,
+                        void* workspace, size_t ws_bytes, const int* cu_seqlens_q,
+                        const int* cu_seqlens_k, int batch, int max_seqlen_q, int max_seqlen_k,
+                        int total_q, int total_k, int H, int Hkv, int d, int causal,
+                        void* stream) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || lse == nullptr ||
+      !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      cu_seqlens_q == nullptr || cu_seqlens_k == nullptr)
+    return FA_ERR_INVALID_ARG;
+  if (batch < 1 || H < 1 || Hkv < 1 || H % Hkv != 0 || max_seqlen_q < 1 || max_seqlen_k < 1 ||
+      total_q < 1 || total_k < 1 || max_seqlen_q > total_q || max_seqlen_k > total_k)
+    return FA_ERR_INVALID_ARG;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  const long long nkb = (static_cast<long long>(max_seqlen_k) + 127) / 128;
+  if (static_cast<long long>(batch) * Hkv * nkb > (1ll << 31) - 1 ||
+      static_cast<long long>(total_q) * H * d > (1ll << 40) ||
+      static_cast<long long>(batch) * H * (max_seqlen_q + 127ll) > (1ll << 31) - 1)
+    return FA_ERR_UNSUPPORTED;
+  if (workspace == nullptr || !aligned16(workspace) ||
+      ws_bytes < fa_bwd_varlen_workspace_bytes(batch, max_seqlen_q, total_q, total_k, H, Hkv, d))
+    return FA_ERR_WORKSPACE;
+  uint32_t* err = error_word_ptr();
+  if (err == nullptr) return FA_ERR_LAUNCH;
+  const size_t n_pad = (static_cast<size_t>(max_seqlen_q) + 127) / 128 * 128;
+  const size_t prow = static_cast<size_t>(batch) * H * n_pad;
+  const size_t nq = static_cast<size_t>(total_q) * H * d, nk = static_cast<size_t>(total_k) * Hkv * d;
+  char* w = static_cast<char*>(workspace);
+  char* w16 = w + 2 * round256(prow * sizeof(float));
+  void* q16 = w16;
+  void* k16 = w16 + round256(nq * 2);
+  void* v16 = w16 + round256(nq * 2) + round256(nk * 2);
+  void* do16 = w16 + round256(nq * 2) + 2 * round256(nk * 2);
+  // token-major views [T][heads][d]; Q / dO boxes of 64 tokens, K / V of 128,
+  // dQ reduce box 32 columns x 1 head x 64 tokens
+  CUtensorMap tq, tk, tv, tdo, tdq;
+  if (!make_map(&tq, q16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, H, total_q, 64, 1,
+                CU_TENSOR_MAP_SWIZZLE_128B, 64) ||
+      !make_map(&tk, k16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, Hkv, total_k, 64, 1,
+                CU_TENSOR_MAP_SWIZZLE_128B, 128) ||
+      !make_map(&tv, v16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, Hkv, total_k, 64, 1,
+                CU_TENSOR_MAP_SWIZZLE_128B, 128) ||
+      !make_map(&tdo, do16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, H, total_q, 64, 1,
+                CU_TENSOR_MAP_SWIZZLE_128B, 64) ||
+      !make_map(&tdq, dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, H, total_q, 32, 1,
+                CU_TENSOR_MAP_SWIZZLE_NONE, 64))
+    return FA_ERR_LAUNCH;
+  fa::BwdArgs a;
+  a.q16 = q16;
+  a.k16 = k16;
+  a.v16 = v16;
+  a.do16 = do16;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.dout = dout;
+  a.lse = lse;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.n_pad = static_cast<int>(n_pad);
+  a.delta = static_cast<float*>(workspace);
+  a.lse_log2 = reinterpret_cast<float*>(w + round256(prow * sizeof(float)));
+  a.B = batch;
+  a.H = H;
+  a.N = max_seqlen_q;
+  a.causal = causal ? 1 : 0;
+  a.scale = 1.0f / sqrtf(static_cast<float>(d));
+  a.scale_log2 = a.scale * kLog2e;
+  a.err = err;
+  a.cu_q = cu_seqlens_q;
+  a.cu_k = cu_seqlens_k;
+  a.Hkv = Hkv;
+  a.Tq = total_q;
+  a.Tk = total_k;
+  a.max_k = max_seqlen_k;
+  a.n_q_elems = static_cast<long long>(nq);
+  a.n_k_elems = static_cast<long long>(nk);
+  cudaEvent_t eb = g_bwd_ev_begin, ee = g_bwd_ev_end;
+  g_bwd_ev_begin = g_bwd_ev_end = nullptr;
+  cudaError_t e = fa::launch_bwd<128>(tq, tk, tv, tdo, tdq, a, static_cast<cudaStream_t>(stream),
+                                      eb, ee);
+  return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
 size_t paged_attn_decode_workspace_bytes(int num_seqs, int Hq, int d, int max_ctx) {
   if (num_seqs < 1 || Hq < 1 || d < 1 || max_ctx < 1) return 0;
   const int sb = fa::decode_split_blocks();

@@ -40,6 +40,9 @@
 //                from TMEM and adds it to dQ in HBM with vector reductions.
 // TMEM (512 columns): S^T / P^T [0,128), dP^T [128,256) (reused for the dQ
 // tile once dS is out), dV [256, 256+D), dK [256+D, 256+2D).
+#include <climits>
+#include <type_traits>
+
 #include "prim.cuh"
 #include "kernels.h"
 
@@ -94,12 +97,14 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
 
 // ------------------------------------------------------- fp16 conversion
 // q, k, v, dout (bf16) -> fp16 copies; 8 elements per thread per step.
-__global__ void __launch_bounds__(256) bwd_convert_kernel(BwdArgs a, long long n8) {
+__global__ void __launch_bounds__(256) bwd_convert_kernel(BwdArgs a, long long q8, long long k8) {
+  // q8: 8-element groups of q and of dout; k8: of k and of v
   bool bad = false;
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < 4 * n8;
+  const long long total = 2 * q8 + 2 * k8;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int t = static_cast<int>(i / n8);
-    const long long j = i - t * n8;
+    const int t = i < q8 ? 0 : i < q8 + k8 ? 1 : i < q8 + 2 * k8 ? 2 : 3;
+    const long long j = i - (t == 0 ? 0 : t == 1 ? q8 : t == 2 ? q8 + k8 : q8 + 2 * k8);
     const void* sp = t == 0 ? a.q : t == 1 ? a.k : t == 2 ? a.v : a.dout;
     void* dp = t == 0 ? a.q16 : t == 1 ? a.k16 : t == 2 ? a.v16 : a.do16;
     const uint4 u = static_cast<const uint4*>(sp)[j];
@@ -127,17 +132,29 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdArgs a) {
   const int lane = threadIdx.x & 31;
   const long long rows = static_cast<long long>(a.B) * a.H * a.n_pad;
   const int nw = (gridDim.x * blockDim.x) >> 5;
+  const bool packed = a.cu_q != nullptr;
   for (long long pr = warp; pr < rows; pr += nw) {
     const long long bh = pr / a.n_pad;
     const int n = static_cast<int>(pr - bh * a.n_pad);
-    if (n >= a.N) {
+    // query row n of this (batch, head): BHND row bh * N + n, or packed token
+    // tq0 + n of head h (row (tq0 + n) * H + h; L at [h][tq0 + n])
+    int len = a.N;
+    long long r = bh * a.N + n, lr = r;
+    if (packed) {
+      const int b = static_cast<int>(bh / a.H), h = static_cast<int>(bh % a.H);
+      const int tq0 = a.cu_q[b];
+      len = a.cu_q[b + 1] - tq0;
+      if (tq0 < 0 || len < 0 || len > a.N || tq0 + len > a.Tq) len = 0;   // reported by the main pass
+      r = static_cast<long long>(tq0 + n) * a.H + h;
+      lr = static_cast<long long>(h) * a.Tq + tq0 + n;
+    }
+    if (n >= len) {
       if (lane == 0) {
         a.delta[pr] = 0.f;
         a.lse_log2[pr] = INFINITY;
       }
       continue;
     }
-    const long long r = bh * a.N + n;
     const __nv_bfloat16* o = static_cast<const __nv_bfloat16*>(a.o) + r * D;
     const __nv_bfloat16* g = static_cast<const __nv_bfloat16*>(a.dout) + r * D;
     float acc = 0.f;
@@ -152,7 +169,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdArgs a) {
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (lane == 0) {
       a.delta[pr] = acc;
-      a.lse_log2[pr] = a.lse[r] * 1.4426950408889634f;
+      a.lse_log2[pr] = a.lse[lr] * 1.4426950408889634f;
     }
     float4* dq = reinterpret_cast<float4*>(a.dq + r * D);
     for (int c = lane; c < D / 4; c += 32) dq[c] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -600,6 +617,9 @@ __device__ __forceinline__ uint32_t half_col(int kk) {
   return static_cast<uint32_t>((kk >> 1) * 32 + (kk & 1) * 8);
 }
 
+// PACKED selects the packed variable-length form (BwdArgs.cu_q != nullptr) at
+// compile time, so the [B, H, N, d] instantiation carries none of its indexing.
+template <bool PACKED>
 __global__ void __launch_bounds__(512, 1)
 bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -613,12 +633,62 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int BH = a.B * a.H;
-  const int kb = static_cast<int>(blockIdx.x) / BH;   // key block (longest work first)
-  const int bh = static_cast<int>(blockIdx.x) % BH;
-  const int nq = (a.N + C::BQ - 1) / C::BQ;
-  const int i0 = a.causal ? kb * (C::BK / C::BQ) : 0;  // first query step that sees these keys
-  const int n_it = nq - i0;
+  // The problem of this CTA: one 128-key block of Lk keys against Lq queries.
+  // BHND: (batch, head) bh, TMA coordinates (row, bh). Packed: sequence b and
+  // KV head hk; the CTA walks every query head of the group (their dK, dV
+  // contributions add up in TMEM), TMA coordinates (head, token).
+  constexpr bool packed = PACKED;
+  int kb, bh = 0, b = 0, hk = 0, group = 1, Lq = a.N, Lk = a.N, tq0 = 0, tk0 = 0;
+  if (packed) {
+    const int BHk = a.B * a.Hkv;
+    kb = static_cast<int>(blockIdx.x) / BHk;
+    b = static_cast<int>(blockIdx.x) % BHk / a.Hkv;
+    hk = static_cast<int>(blockIdx.x) % a.Hkv;
+    group = a.H / a.Hkv;
+    tq0 = a.cu_q[b];
+    tk0 = a.cu_k[b];
+    Lq = a.cu_q[b + 1] - tq0;
+    Lk = a.cu_k[b + 1] - tk0;
+    if (tq0 < 0 || tk0 < 0 || Lq < 0 || Lk < 0 || Lq > a.N || tq0 + Lq > a.Tq || tk0 + Lk > a.Tk) {
+      if (threadIdx.x == 0 && kb == 0) atomicCAS(a.err, 0u, kErrBadIndex + 2);
+      Lq = 0;
+      Lk = 0;
+    }
+  } else {
+    kb = static_cast<int>(blockIdx.x) / (a.B * a.H);   // key block (longest work first)
+    bh = static_cast<int>(blockIdx.x) % (a.B * a.H);
+  }
+  if (kb * C::BK >= Lk) return;                        // no keys in this block
+  const int off = a.causal ? Lk - Lq : 0;              // causal: query i sees keys <= i + off
+  const int nq = (Lq + C::BQ - 1) / C::BQ;
+  const int i0 = a.causal ? max(0, kb * C::BK - off) / C::BQ : 0;  // first step seeing these keys
+  const int n_steps = max(0, nq - i0);
+  const int n_it = group * n_steps;                    // (query head, step) pairs
+  // iteration it = (query head hk * group + it / n_steps, query step i0 + it % n_steps);
+  // each role walks it in order and keeps the pair as counters (no division)
+  struct Walk {
+    int step, head;
+  };
+  auto walk_start = [&]() { return Walk{i0, hk * group}; };
+  auto walk_next = [&](Walk& w) {
+    if (++w.step == nq) {
+      w.step = i0;
+      ++w.head;
+    }
+  };
+  if (n_it == 0) {                                      // keys no query sees: dK = dV = 0
+    for (int i = threadIdx.x; i < C::BK * D / 4 * 2; i += blockDim.x) {
+      const int which = i / (C::BK * D / 4), rem = i % (C::BK * D / 4);
+      const int key = kb * C::BK + rem / (D / 4);
+      if (key < Lk) {
+        const size_t orow = packed ? (static_cast<size_t>(tk0 + key) * a.Hkv + hk) * D
+                                   : (static_cast<size_t>(bh) * a.N + key) * D;
+        reinterpret_cast<float4*>((which ? a.dk : a.dv) + orow)[rem % (D / 4)] =
+            make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    return;
+  }
 
   auto bar = [&](int i) -> uint32_t { return base + C::BAR_OFF + 8 * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
@@ -659,24 +729,29 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tma_prefetch_desc(&tmDQ);
       mbar_arrive_expect_tx(bar(C::B_KV), 2 * C::KV_TILE);
       for (int c = 0; c < 2; ++c) {
-        tma_load_3d(base + C::K_OFF + c * C::KV_CHUNK, &tmK, bar(C::B_KV), c * 64, kb * C::BK, bh);
-        tma_load_3d(base + C::V_OFF + c * C::KV_CHUNK, &tmV, bar(C::B_KV), c * 64, kb * C::BK, bh);
+        const int ky = packed ? hk : kb * C::BK, kz = packed ? tk0 + kb * C::BK : bh;
+        tma_load_3d(base + C::K_OFF + c * C::KV_CHUNK, &tmK, bar(C::B_KV), c * 64, ky, kz);
+        tma_load_3d(base + C::V_OFF + c * C::KV_CHUNK, &tmV, bar(C::B_KV), c * 64, ky, kz);
       }
       int issued = 0;
-      for (int it = 0; it < n_it; ++it) {
+      Walk w = walk_start();
+      for (int it = 0; it < n_it; ++it, walk_next(w)) {
         const int s = it % C::NS;
         const uint32_t ph = ((it / C::NS) & 1) ^ 1;
-        const int row = (i0 + it) * C::BQ;
-        const size_t prow = static_cast<size_t>(bh) * a.n_pad + row;   // 256 B aligned
+        const int row = w.step * C::BQ;
+        const int hq = w.head;
+        const size_t prow = (packed ? static_cast<size_t>(b) * a.H + hq : static_cast<size_t>(bh)) *
+                                a.n_pad + row;                           // 256 B aligned
+        const int qy = packed ? hq : row, qz = packed ? tq0 + row : bh;
         if (!mbar_wait(bar(C::B_STEP + s), ph, a.err, kSiteQE, abort_flag)) break;
         const uint32_t full = bar(C::B_FULL + s);
         mbar_arrive_expect_tx(full, 2 * (C::Q_TILE + 256));
         for (int c = 0; c < 2; ++c)
-          tma_load_3d(base + C::Q_OFF + s * C::Q_TILE + c * C::Q_CHUNK, &tmQ, full, c * 64, row, bh);
+          tma_load_3d(base + C::Q_OFF + s * C::Q_TILE + c * C::Q_CHUNK, &tmQ, full, c * 64, qy, qz);
         bulk_load(base + C::L_OFF + s * 256, a.lse_log2 + prow, 256, full);
         for (int c = 0; c < 2; ++c)
-          tma_load_3d(base + C::DO_OFF + s * C::Q_TILE + c * C::Q_CHUNK, &tmDO, full, c * 64, row,
-                      bh);
+          tma_load_3d(base + C::DO_OFF + s * C::Q_TILE + c * C::Q_CHUNK, &tmDO, full, c * 64, qy,
+                      qz);
         bulk_load(base + C::DL_OFF + s * 256, a.delta + prow, 256, full);
         issued = it + 1;
       }
@@ -810,13 +885,14 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tc_fence_before();
       warp_arrive(bar(C::B_KT));
     }
-    for (int it = 0; it < n_it && ok; ++it) {
+    Walk wk = walk_start();
+    for (int it = 0; it < n_it && ok; ++it, walk_next(wk)) {
       const int s = it % C::NS;
       const int buf = it & 1;
-      const int qh = (i0 + it) * C::BQ + 32 * h;        // first query of this half
+      const int qh = wk.step * C::BQ + 32 * h;          // first query of this half
       const float* Ls = reinterpret_cast<const float*>(smem + C::L_OFF + s * 256) + 32 * h;
       const float* Ds = reinterpret_cast<const float*>(smem + C::DL_OFF + s * 256) + 32 * h;
-      const bool need_mask = (a.causal && key > qh) || key >= a.N;
+      const bool need_mask = (a.causal && key > qh + off) || key >= Lk || qh + 31 >= Lq;
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_ST), it & 1, a.err, kSiteST, abort_flag));
       if (!ok) break;
       tc_fence_after();
@@ -825,24 +901,36 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tmem_ld_wait();
       uint32_t pk[16];                                 // P^T, fp16 pairs of queries
       const uint64_t nsl2 = f2_pack(-sl2, -sl2);
+      // queries qh + i, i in [lo, hi), see this key; the masked form runs only
+      // in the steps where some lane of the warp has a masked query
+      const int lo = a.causal ? key - off - qh : INT_MIN;
+      const int hi = key < Lk ? Lq - qh : INT_MIN;
+      auto p_loop = [&](auto masked) {
 #pragma unroll
-      for (int e = 0; e < 32; e += 4) {
-        const float4 lv = *reinterpret_cast<const float4*>(Ls + e);
-        // y = L - scale log2e S on packed pairs; P = 2^-y
-        float y[4];
-        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), nsl2,
-                         f2_pack(lv.x, lv.y)), y[0], y[1]);
-        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3])), nsl2,
-                         f2_pack(lv.z, lv.w)), y[2], y[3]);
-        float p[4];
+        for (int e = 0; e < 32; e += 4) {
+          const float4 lv = *reinterpret_cast<const float4*>(Ls + e);
+          // y = L - scale log2e S on packed pairs; P = 2^-y
+          float y[4];
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), nsl2,
+                           f2_pack(lv.x, lv.y)), y[0], y[1]);
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3])), nsl2,
+                           f2_pack(lv.z, lv.w)), y[2], y[3]);
+          float p[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          p[u] = ex2_approx(-y[u]);
-          if (need_mask && ((a.causal && key > qh + e + u) || key >= a.N)) p[u] = 0.f;
+          for (int u = 0; u < 4; ++u) {
+            p[u] = ex2_approx(-y[u]);
+            if constexpr (decltype(masked)::value) {
+              if (e + u < lo || e + u >= hi) p[u] = 0.f;
+            }
+          }
+          pk[e / 2] = pack_f16x2(p[0], p[1]);
+          pk[e / 2 + 1] = pack_f16x2(p[2], p[3]);
         }
-        pk[e / 2] = pack_f16x2(p[0], p[1]);
-        pk[e / 2 + 1] = pack_f16x2(p[2], p[3]);
-      }
+      };
+      if (__any_sync(0xffffffffu, need_mask))
+        p_loop(std::true_type{});
+      else
+        p_loop(std::false_type{});
       tmem_st16(s_addr, pk);                           // over this half's own S^T columns
       tmem_st_wait();
       tc_fence_before();
@@ -897,7 +985,8 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_END), 0, a.err, kSiteEnd, abort_flag));
       if (ok) {
         tc_fence_after();
-        const size_t orow = (static_cast<size_t>(bh) * a.N + key) * D;
+        const size_t orow = packed ? (static_cast<size_t>(tk0 + key) * a.Hkv + hk) * D
+                                   : (static_cast<size_t>(bh) * a.N + key) * D;
         const uint32_t src = tmem + lane_off + (h ? C::COL_DK : C::COL_DV);
         float* dst = (h ? a.dk : a.dv) + orow;
         const float mul = h ? a.scale : 1.f;
@@ -906,7 +995,7 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           uint32_t v[32];
           tmem_ld32(src + c * 32, v);
           tmem_ld_wait();
-          if (key < a.N) {
+          if (key < Lk) {
             float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
 #pragma unroll
             for (int e = 0; e < 8; ++e)
@@ -926,8 +1015,9 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     float* stage = reinterpret_cast<float*>(smem + C::DQS_OFF + quarter * C::DQ_STAGE);
     const uint32_t stage_addr = base + C::DQS_OFF + quarter * C::DQ_STAGE;
     warp_arrive(bar(C::B_DSQ));                      // phase 0: no dQ^T(-1) to drain
-    for (int it = 0; it < n_it; ++it) {
-      const int q0 = (i0 + it) * C::BQ;
+    Walk wq = walk_start();
+    for (int it = 0; it < n_it; ++it, walk_next(wq)) {
+      const int q0 = wq.step * C::BQ;
       if (!__all_sync(0xffffffffu, mbar_wait(bar(C::B_STEP + it % C::NS), (it / C::NS) & 1, a.err,
                                               kSiteDQ, abort_flag)))
         break;
@@ -947,7 +1037,12 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       fence_async_smem();
       __syncwarp();
       if (lane == 0) {
-        tma_reduce_add_3d(&tmDQ, stage_addr, quarter * 32, q0, bh);   // rows >= N are skipped
+        // rows past the tensor are skipped; in the packed form, rows past this
+        // sequence add exact zeros (dS = 0 there) to the next sequence's dQ
+        if (packed)
+          tma_reduce_add_3d(&tmDQ, stage_addr, quarter * 32, wq.head, tq0 + q0);
+        else
+          tma_reduce_add_3d(&tmDQ, stage_addr, quarter * 32, q0, bh);
         bulk_commit_group();
       }
     }
@@ -974,30 +1069,39 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = D == 128 ? cudaFuncSetAttribute(bwd_d128_kernel,
+    cudaError_t e = D == 128 ? cudaFuncSetAttribute(bwd_d128_kernel<false>,
                                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                     BwdD128::SMEM_BYTES)
                              : cudaFuncSetAttribute(bwd_main_kernel<D>,
                                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                     C::SMEM_BYTES);
+    if (e == cudaSuccess && D == 128)
+      e = cudaFuncSetAttribute(bwd_d128_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               BwdD128::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
   const long long rows = static_cast<long long>(a.B) * a.H * a.n_pad;
   const long long want = (rows + 7) / 8;
   const int pre_blocks = static_cast<int>(want < 148 * 16 ? want : 148 * 16);
-  const long long n8 = static_cast<long long>(a.B) * a.H * a.N * D / 8;
-  const long long cwant = (4 * n8 + 255) / 256;
+  const long long q8 = (a.cu_q ? a.n_q_elems : static_cast<long long>(a.B) * a.H * a.N * D) / 8;
+  const long long k8 = (a.cu_q ? a.n_k_elems : static_cast<long long>(a.B) * a.H * a.N * D) / 8;
+  const long long cwant = (2 * q8 + 2 * k8 + 255) / 256;
   const int cblocks = static_cast<int>(cwant < 148 * 8 ? cwant : 148 * 8);
-  bwd_convert_kernel<<<cblocks, 256, 0, stream>>>(a, n8);
+  bwd_convert_kernel<<<cblocks, 256, 0, stream>>>(a, q8, k8);
   bwd_pre_kernel<D><<<pre_blocks, 256, 0, stream>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int nk = (a.N + C::BK - 1) / C::BK;
+  const int nk = ((a.cu_q ? a.max_k : a.N) + C::BK - 1) / C::BK;
+  const int per_block = a.cu_q ? a.B * a.Hkv : a.B * a.H;   // CTAs per key block
   if (ev_main_begin != nullptr) cudaEventRecord(ev_main_begin, stream);
   if (D == 128)
-    bwd_d128_kernel<<<nk * a.B * a.H, BwdD128::THREADS, BwdD128::SMEM_BYTES, stream>>>(
-        tq, tk, tv, tdo, tdq, a);
+    if (a.cu_q)
+      bwd_d128_kernel<true><<<nk * per_block, BwdD128::THREADS, BwdD128::SMEM_BYTES, stream>>>(
+          tq, tk, tv, tdo, tdq, a);
+    else
+      bwd_d128_kernel<false><<<nk * per_block, BwdD128::THREADS, BwdD128::SMEM_BYTES, stream>>>(
+          tq, tk, tv, tdo, tdq, a);
   else
     bwd_main_kernel<D><<<nk * a.B * a.H, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
   e = cudaGetLastError();

@@ -333,7 +333,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       for (int q = 0; q < 64; ++q) {
         const uint64_t x2 = f2_fma(f2_pack(SV(2 * q), SV(2 * q + 1)), sl2x2, negm2);
         uint64_t p2;
-        if (kPolyEvery > 0 && q % kPolyEvery == kPolyEvery - 1) {
+        if (kPolyEvery > 0 && q % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
           p2 = exp2_poly_x2(x2);
         } else {
           float x0, x1;

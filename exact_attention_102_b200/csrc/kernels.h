@@ -50,6 +50,14 @@ struct BwdArgs {
   float scale;        // softmax scale
   float scale_log2;   // scale * log2(e)
   uint32_t* err;
+  // packed variable-length mode when cu_q != nullptr (d = 128): q, o, dout, dq
+  // [Tq][H][D]; k, v, dk, dv [Tk][Hkv][D]; lse [H][Tq]; N = the longest query
+  // sequence, n_pad = N rounded up to 128, delta / lse_log2 [B][H][n_pad];
+  // causal aligned to the bottom right
+  const int* cu_q = nullptr;
+  const int* cu_k = nullptr;
+  int Hkv = 0, Tq = 0, Tk = 0, max_k = 0;
+  long long n_q_elems = 0, n_k_elems = 0;   // elements of q (= dout) and of k (= v)
 };
 
 // tdq: fp32 view of dq, [BH][N][d], box 32 x 64, no swizzle (reduce-add target

@@ -150,6 +150,37 @@ FA_API fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void
                         int causal, void* stream);
 
 /*
+ * fa_bwd_varlen_workspace_bytes — device workspace fa_bwd_varlen needs: D and
+ * L log2(e) for [batch][H][max_seqlen_q rounded up to 128] rows, and fp16
+ * copies of q, k, v, dout. 0 for invalid sizes.
+ */
+FA_API size_t fa_bwd_varlen_workspace_bytes(int batch, int max_seqlen_q, int total_q,
+                                            int total_k, int H, int Hkv, int d);
+
+/*
+ * fa_bwd_varlen — gradients of fa_fwd_varlen (same method as fa_bwd: P rebuilt
+ * from L, dQ accumulated across key blocks; layouts and the bottom-right causal
+ * mask as fa_fwd_varlen).
+ *   q, o, dout    : bf16 [total_q][H][d]; lse fp32 [H][total_q] from fa_fwd_varlen.
+ *   k, v          : bf16 [total_k][Hkv][d].
+ *   dq            : fp32 [total_q][H][d]; rows of the sequences are written
+ *                   (rows past cu_seqlens_q[batch] are left as they are).
+ *   dk, dv        : fp32 [total_k][Hkv][d]; a KV head's gradient sums its
+ *                   group's query heads; rows past cu_seqlens_k[batch] untouched.
+ *   max_seqlen_q/k: bounds on every query / key length (they size the grid).
+ *   d             : 128 only for now (FA_ERR_UNSUPPORTED otherwise).
+ * Precision as fa_bwd (fp16 operands, |x| < 65504). Errors as fa_fwd_varlen,
+ * plus FA_ERR_WORKSPACE when the workspace is NULL or smaller than
+ * fa_bwd_varlen_workspace_bytes().
+ */
+FA_API fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
+                        const float* lse, const void* dout, float* dq, float* dk, float* dv,
+                        void* workspace, size_t ws_bytes, const int* cu_seqlens_q,
+                        const int* cu_seqlens_k, int batch, int max_seqlen_q, int max_seqlen_k,
+                        int total_q, int total_k, int H, int Hkv, int d, int causal,
+                        void* stream);
+
+/*
  * Bytes of device workspace paged_attn_decode needs for split partials
  * (fp32 O and L per (sequence, query head, split)) and a work counter, when
  * no sequence is longer than max_ctx tokens.

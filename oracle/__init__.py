@@ -31,6 +31,7 @@ from .attention import (  # noqa: F401
     attention_bwd,
     attention_rows,
     attention_varlen,
+    attention_varlen_bwd,
     paged_decode,
     combine_partials,
     round_bf16,

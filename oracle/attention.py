@@ -142,6 +142,43 @@ def attention_varlen(q, k, v, cu_q, cu_k, causal=False, scale=None):
     return o, lse
 
 
+def attention_varlen_bwd(q, k, v, do, cu_q, cu_k, causal=False, scale=None, o=None):
+    """Gradients of attention_varlen: per (sequence, query head) the textbook
+    backward of attention_bwd (D from ``o`` when given, as fa_bwd receives O),
+    with a KV head's dK, dV summed over the query heads that read it.
+    Returns (dQ [Tq, H, d], dK [Tk, Hkv, d], dV [Tk, Hkv, d])."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    do = np.asarray(do, dtype=np.float64)
+    tq, h, d = q.shape
+    hkv = k.shape[1]
+    group = h // hkv
+    sc = _scale(d, scale)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(len(cu_q) - 1):
+        q0, q1, k0, k1 = int(cu_q[b]), int(cu_q[b + 1]), int(cu_k[b]), int(cu_k[b + 1])
+        lq, lk = q1 - q0, k1 - k0
+        if lq == 0 or lk == 0:
+            continue
+        pos = np.arange(lq) + (lk - lq)
+        for hh in range(h):
+            kh, vh = k[k0:k1, hh // group], v[k0:k1, hh // group]
+            qh, gh = q[q0:q1, hh], do[q0:q1, hh]
+            o_h, _, p = attention_rows(qh, pos, kh, vh, causal, scale)
+            if o is not None:
+                o_h = np.asarray(o, dtype=np.float64)[q0:q1, hh]
+            dp = gh @ vh.T
+            dd = (gh * o_h).sum(axis=1)
+            ds = p * (dp - dd[:, None])
+            dq[q0:q1, hh] = sc * ds @ kh
+            dk[k0:k1, hh // group] += sc * ds.T @ qh
+            dv[k0:k1, hh // group] += p.T @ gh
+    return dq, dk, dv
+
+
 def attention_bwd(q, k, v, do, causal=False, scale=None, o=None):
     """Analytic gradients of exact attention, float64.
 

@@ -137,3 +137,17 @@ def test_fwd_varlen_rejects_bad_arguments_without_a_gpu():
     assert call(*args) == fa.FA_ERR_UNSUPPORTED            # d not in {64, 128}
     args = list(ok_args); args[7] = 0
     assert call(*args) == fa.FA_ERR_INVALID_ARG            # batch < 1
+
+
+def test_bwd_varlen_rejects_bad_arguments_without_a_gpu():
+    L = fa.lib()
+    p = ctypes.c_void_p(256)
+    s = ctypes.c_void_p(0)
+    args = [p] * 10 + [ctypes.c_size_t(1 << 30), p, p, 2, 64, 64, 128, 128, 8, 2, 128, 1, s]
+    a = list(args); a[20] = 64                # d = 64 is not supported yet
+    assert L.fa_bwd_varlen(*a) == fa.FA_ERR_UNSUPPORTED
+    a = list(args); a[19] = 3                 # H % Hkv != 0
+    assert L.fa_bwd_varlen(*a) == fa.FA_ERR_INVALID_ARG
+    a = list(args); a[9] = ctypes.c_void_p(0) # no workspace
+    assert L.fa_bwd_varlen(*a) == fa.FA_ERR_WORKSPACE
+    assert L.fa_bwd_varlen_workspace_bytes(0, 64, 128, 128, 8, 2, 128) == 0

@@ -473,3 +473,43 @@ def test_varlen_against_torch_sdpa():
         ref = torch.nn.functional.scaled_dot_product_attention(qs, ks, vs, attn_mask=mask)
         np.testing.assert_allclose(o[cu_q[b]:cu_q[b + 1]], ref.numpy().transpose(1, 0, 2),
                                    rtol=0, atol=1e-12)
+
+
+def test_varlen_bwd_equal_lengths_match_bhnd():
+    B, H, N, d = 2, 2, 19, 8
+    q, k, v, cu_q, cu_k = _varlen_case([N] * B, [N] * B, H, H, d, 76)
+    do = np.random.default_rng(77).standard_normal(q.shape)
+    bhnd = lambda t: t.reshape(B, N, H, d).transpose(0, 2, 1, 3)
+    for causal in (False, True):
+        g = oracle.attention_varlen_bwd(q, k, v, do, cu_q, cu_k, causal)
+        g2 = oracle.attention_bwd(bhnd(q), bhnd(k), bhnd(v), bhnd(do), causal)
+        for a, b_ in zip(g, g2[:3]):
+            np.testing.assert_allclose(bhnd(a), b_, rtol=0, atol=1e-13)
+
+
+def test_varlen_bwd_against_torch_autograd():
+    """Library routine: torch float64 autograd through the packed forward with
+    unequal lengths, GQA and the bottom-right mask (including rows that see
+    no key)."""
+    lens_q, lens_k = [6, 3, 9], [4, 8, 9]
+    H, Hkv, d = 4, 2, 8
+    q, k, v, cu_q, cu_k = _varlen_case(lens_q, lens_k, H, Hkv, d, 78)
+    do = np.random.default_rng(79).standard_normal(q.shape)
+    tq, tk = [torch.tensor(x, requires_grad=True) for x in (q, k)]
+    tv = torch.tensor(v, requires_grad=True)
+    outs = []
+    for b in range(3):
+        lq, lk = lens_q[b], lens_k[b]
+        qs = tq[cu_q[b]:cu_q[b + 1]].transpose(0, 1)
+        ks = tk[cu_k[b]:cu_k[b + 1]].repeat_interleave(H // Hkv, dim=1).transpose(0, 1)
+        vs = tv[cu_k[b]:cu_k[b + 1]].repeat_interleave(H // Hkv, dim=1).transpose(0, 1)
+        s = qs @ ks.transpose(1, 2) / math.sqrt(d)
+        mask = torch.from_numpy(np.arange(lk)[None, :] <= np.arange(lq)[:, None] + lk - lq)
+        s = s.masked_fill(~mask, -torch.inf)
+        p = torch.softmax(s, dim=-1).nan_to_num(0.0)       # rows without keys: P = 0
+        outs.append((p @ vs).transpose(0, 1))
+    o = torch.cat(outs)
+    (o * torch.from_numpy(do)).sum().backward()
+    g = oracle.attention_varlen_bwd(q, k, v, do, cu_q, cu_k, causal=True)
+    for got, ref in zip(g, (tq.grad, tk.grad, tv.grad)):
+        np.testing.assert_allclose(got, ref.numpy(), rtol=0, atol=1e-12)
