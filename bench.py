@@ -367,6 +367,45 @@ def run_fwd_varlen(fa, steps, warmup):
     return res
 
 
+def run_kv_pool(fa, steps):
+    """Block pool on a decoding schedule: 64 sequences = 16 prompts of 512
+    tokens forked 4 ways, then `steps` rounds of one token per sequence
+    (on-demand blocks, copy-on-write of the shared partial block on the first
+    round); host time per append. Then the device copy of 4096 blocks of
+    32 KiB per cache (K and V) in GB/s (read + write)."""
+    pool = fa.KVPool(65536, 16, 64, 1100)
+    t0 = time.perf_counter()
+    for p in range(16):
+        pool.add(4 * p)
+        pool.append(4 * p, 512)
+        for c in range(1, 4):
+            pool.fork(4 * p, 4 * p + c)
+    n_app, n_cow = 0, 0
+    for _ in range(steps):
+        for s in range(64):
+            st, copies = pool.append(s, 1)
+            n_app += 1
+            n_cow += len(copies)
+    host_s = time.perf_counter() - t0
+    kc = torch.zeros((8192, 8, 16, 128), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    src = torch.arange(0, 4096, dtype=torch.int32, device="cuda")
+    dst = torch.arange(4096, 8192, dtype=torch.int32, device="cuda")
+    for _ in range(3):
+        fa.kv_copy_blocks(kc, vc, src, dst)
+    torch.cuda.synchronize()
+    a, b = _ev(), _ev()
+    a.record()
+    for _ in range(10):
+        fa.kv_copy_blocks(kc, vc, src, dst)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / 10
+    moved = 2 * 2 * 4096 * kc[0].numel() * 2          # K and V, read + write
+    return {"appends": n_app, "copy_on_write": n_cow, "us_per_append": 1e6 * host_s / n_app,
+            "copy_ms": ms, "copy_GB/s": moved / (ms / 1e3) / 1e9}
+
+
 # ---------------------------------------------------------- CPU baseline ---
 def _cores():
     try:
@@ -446,6 +485,9 @@ def _config():
 
 def run_case(fa, case, shape, causal, steps, warmup):
     """One operation at one size, for profilers: warmup + steps launches."""
+    if case == "kv_pool":                 # the fixed pool schedule (shape unused)
+        print(json.dumps(run_kv_pool(fa, steps)))
+        return
     if case == "fwd_varlen":              # the fixed packed workload (shape unused)
         res = run_fwd_varlen(fa, steps, warmup)
         print(json.dumps({"case": case, "ms": res["ms"],
@@ -589,6 +631,10 @@ def main():
             "ms": vl["ms"], "tokens": vl["tokens"],
             "TFLOP/s": vl["flops"] / (vl["ms"] / 1e3) / 1e12,
             "bwd_ms": vl["bwd_ms"], "bwd_TFLOP/s": 2.5 * vl["flops"] / (vl["bwd_ms"] / 1e3) / 1e12}
+        kvp = run_kv_pool(fa, 64)
+        parts["kv_pool"] = dict(kvp, roofline={
+            "bound": "hbm", "achieved": kvp["copy_GB/s"], "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": kvp["copy_GB/s"] / peaks["hbm_gbs"]})
         f8 = run_fp8(fa, args.steps, args.warmup)
         if "ms" in f8:
             t8 = f8["flops"] / (f8["ms"] / 1e3) / 1e12

@@ -36,6 +36,9 @@ EXPORTS = (
     "fa_fwd_fp8", "fa_last_device_error", "fa_debug_wait_timeout",
     "paged_attn_decode_noalloc", "fa_bwd_time_main_pass", "fa_fwd_varlen",
     "fa_bwd_varlen_workspace_bytes", "fa_bwd_varlen",
+    "fa_kv_pool_create", "fa_kv_pool_destroy", "fa_kv_seq_add", "fa_kv_seq_fork", "fa_kv_seq_free",
+    "fa_kv_seq_append", "fa_kv_num_free", "fa_kv_refcount", "fa_kv_seq_len", "fa_kv_block_table",
+    "fa_kv_copy_blocks",
 )
 
 
@@ -88,6 +91,27 @@ def lib() -> ctypes.CDLL:
     L.fa_bwd_varlen_workspace_bytes.argtypes = [ci] * 7
     L.fa_bwd_varlen.restype = ci
     L.fa_bwd_varlen.argtypes = [vp] * 10 + [sz, vp, vp] + [ci] * 9 + [vp]
+    pi = ctypes.POINTER(ci)
+    L.fa_kv_pool_create.restype = ci
+    L.fa_kv_pool_create.argtypes = [ci, ci, ci, ci, ctypes.POINTER(vp)]
+    L.fa_kv_pool_destroy.restype = None
+    L.fa_kv_pool_destroy.argtypes = [vp]
+    for name in ("fa_kv_seq_add", "fa_kv_seq_free"):
+        getattr(L, name).restype = ci
+        getattr(L, name).argtypes = [vp, ci]
+    L.fa_kv_seq_fork.restype = ci
+    L.fa_kv_seq_fork.argtypes = [vp, ci, ci]
+    L.fa_kv_seq_append.restype = ci
+    L.fa_kv_seq_append.argtypes = [vp, ci, ci, pi, pi, pi]
+    L.fa_kv_num_free.restype = ci
+    L.fa_kv_num_free.argtypes = [vp]
+    for name in ("fa_kv_refcount", "fa_kv_seq_len"):
+        getattr(L, name).restype = ci
+        getattr(L, name).argtypes = [vp, ci]
+    L.fa_kv_block_table.restype = ci
+    L.fa_kv_block_table.argtypes = [vp, pi, ci, pi, ci, pi]
+    L.fa_kv_copy_blocks.restype = ci
+    L.fa_kv_copy_blocks.argtypes = [vp, vp, ci, vp, vp, ci, ctypes.c_longlong, vp]
     L.fa_debug_wait_timeout.restype = ci
     L.fa_debug_wait_timeout.argtypes = [ctypes.c_uint, vp]
     _lib = L
@@ -203,6 +227,78 @@ def fa_bwd_varlen(q, k, v, o, lse, do, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
                                int(max_seqlen_k), Tq, Tk, H, Hkv, d, int(bool(causal)),
                                _stream(stream)))
     return dq, dk, dv
+
+
+class KVPool:
+    """Paged KV-cache block pool (host side, C++ in libfa.so): on-demand
+    blocks, forks that share blocks by reference count, copy-on-write."""
+
+    def __init__(self, num_blocks, block_size, max_seqs, max_blocks_per_seq):
+        h = ctypes.c_void_p(0)
+        _check("fa_kv_pool_create",
+               lib().fa_kv_pool_create(num_blocks, block_size, max_seqs, max_blocks_per_seq,
+                                       ctypes.byref(h)))
+        self._h = h
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+        self.max_blocks = max_blocks_per_seq
+        self._src, self._dst, self._n = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            lib().fa_kv_pool_destroy(h)
+            self._h = None
+
+    def add(self, seq):
+        """Returns the fa_status (0 = ok)."""
+        return int(lib().fa_kv_seq_add(self._h, seq))
+
+    def fork(self, parent, child):
+        return int(lib().fa_kv_seq_fork(self._h, parent, child))
+
+    def free(self, seq):
+        return int(lib().fa_kv_seq_free(self._h, seq))
+
+    def append(self, seq, n_tokens):
+        """Returns (status, copies): copies lists the (src, dst) block pairs to
+        copy on the device before writing the new tokens."""
+        st = int(lib().fa_kv_seq_append(self._h, seq, n_tokens, ctypes.byref(self._src),
+                                        ctypes.byref(self._dst), ctypes.byref(self._n)))
+        copies = [(self._src.value, self._dst.value)] if st == FA_OK and self._n.value else []
+        return st, copies
+
+    def num_free(self):
+        return int(lib().fa_kv_num_free(self._h))
+
+    def refcount(self, block):
+        return int(lib().fa_kv_refcount(self._h, block))
+
+    def seq_len(self, seq):
+        return int(lib().fa_kv_seq_len(self._h, seq))
+
+    def block_tables(self, seqs, width=None):
+        """(table rows as lists of width entries, lengths) for the sequences."""
+        width = self.max_blocks if width is None else width
+        n = len(seqs)
+        ids = (ctypes.c_int * max(n, 1))(*seqs)
+        tab = (ctypes.c_int * max(n * width, 1))()
+        lens = (ctypes.c_int * max(n, 1))()
+        _check("fa_kv_block_table", lib().fa_kv_block_table(self._h, ids, n, tab, width, lens))
+        return [list(tab[i * width:(i + 1) * width]) for i in range(n)], list(lens[:n])
+
+
+def kv_copy_blocks(k_cache, v_cache, src, dst, stream=None):
+    """Copy physical block src[i] -> dst[i] in both paged caches
+    ([P][Hkv][block_size][d] bf16); src, dst int32 device tensors."""
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(src, "src", torch.int32, 1)
+    _need(dst, "dst", torch.int32, 1)
+    block_bytes = k_cache[0].numel() * 2
+    _check("fa_kv_copy_blocks",
+           lib().fa_kv_copy_blocks(_ptr(k_cache), _ptr(v_cache), k_cache.shape[0], _ptr(src),
+                                   _ptr(dst), src.numel(), block_bytes, _stream(stream)))
 
 
 def fa_bwd_workspace_bytes(B, H, N, d):

@@ -21,7 +21,7 @@ LIB = os.path.join(PKG, "libfa.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]
-SOURCES = ["api.cu", "fwd.cu", "bwd.cu", "decode.cu", "fp8.cu"]
+SOURCES = ["api.cu", "fwd.cu", "bwd.cu", "decode.cu", "fp8.cu", "kv_pool.cu"]
 
 
 def _nvcc():

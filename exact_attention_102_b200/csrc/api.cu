@@ -94,6 +94,11 @@ fa_status check_attn_dims(int B, int H, int N, int d) {
 
 }  // namespace
 
+namespace fa {
+// the device error word of the current device, for kernels launched elsewhere
+uint32_t* error_word_for_kv() { return error_word_ptr(); }
+}  // namespace fa
+
 extern "C" {
 
 const char* fa_status_str(fa_status s) {

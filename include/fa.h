@@ -297,6 +297,64 @@ FA_API fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8,
 FA_API fa_status fa_bwd_time_main_pass(void* ev_begin, void* ev_end);
 
 /*
+ * Paged KV-cache block pool ("FlashAttention系列优化", PagedAttention: blocks
+ * allocated on demand as tokens arrive; sequences of parallel sampling share
+ * physical blocks through their block tables; a reference count per block and
+ * copy-on-write keep sharing safe). Host-side, not thread-safe: the caller
+ * serialises calls on one pool. Policy: the lowest-numbered free block is
+ * handed out; an append to a sequence whose last block is partially filled and
+ * shared first copies that block (copy-on-write), then takes new blocks in
+ * order; every operation either completes or changes nothing.
+ *
+ * fa_kv_pool_create  — num_blocks physical blocks of block_size tokens, sequence
+ *                      ids [0, max_seqs), at most max_blocks_per_seq blocks per
+ *                      sequence. *out receives the pool (free with
+ *                      fa_kv_pool_destroy). FA_ERR_INVALID_ARG for sizes < 1 or
+ *                      out == NULL; FA_ERR_WORKSPACE if host memory runs out.
+ * fa_kv_seq_add      — start an empty sequence (id must be unused).
+ * fa_kv_seq_fork     — child (unused id) maps the parent's blocks and length;
+ *                      each block gains a reference.
+ * fa_kv_seq_free     — each of the sequence's blocks loses a reference (freed
+ *                      at zero); the id becomes unused.
+ * fa_kv_seq_append   — reserve slots for n_tokens after the last token. When a
+ *                      copy-on-write happens, *n_copies = 1 and copy_src[0] /
+ *                      copy_dst[0] name the blocks whose contents must be copied
+ *                      on the device (fa_kv_copy_blocks) before the new tokens
+ *                      are written; otherwise *n_copies = 0. Returns
+ *                      FA_ERR_INVALID_ARG for an unused id, n_tokens < 0 or more
+ *                      than max_blocks_per_seq blocks; FA_ERR_WORKSPACE when the
+ *                      pool has too few free blocks (the pool is the workspace).
+ * fa_kv_num_free / fa_kv_refcount / fa_kv_seq_len — queries (-1 for an invalid
+ *                      pool, block or unused sequence).
+ * fa_kv_block_table  — rows of the int32 table [n][max_blocks_per_seq] for the
+ *                      given sequences (entries past ceil(len / block_size) are
+ *                      0, which paged_attn_decode never reads) and their lengths.
+ * fa_kv_copy_blocks  — on `stream`, copy block src[i] to block dst[i] in both
+ *                      caches (device int32 arrays of n pairs; block_bytes = the
+ *                      bytes of one physical block of one cache, a multiple of
+ *                      16, e.g. Hkv * block_size * d * 2 for the
+ *                      [P][Hkv][block_size][d] bf16 caches of paged_attn_decode).
+ *                      Out-of-range block ids are skipped and reported by
+ *                      fa_last_device_error() as FA_ERR_INVALID_ARG.
+ */
+typedef struct fa_kv_pool fa_kv_pool;
+FA_API fa_status fa_kv_pool_create(int num_blocks, int block_size, int max_seqs,
+                                   int max_blocks_per_seq, fa_kv_pool** out);
+FA_API void fa_kv_pool_destroy(fa_kv_pool* pool);
+FA_API fa_status fa_kv_seq_add(fa_kv_pool* pool, int seq);
+FA_API fa_status fa_kv_seq_fork(fa_kv_pool* pool, int parent, int child);
+FA_API fa_status fa_kv_seq_free(fa_kv_pool* pool, int seq);
+FA_API fa_status fa_kv_seq_append(fa_kv_pool* pool, int seq, int n_tokens, int* copy_src,
+                                  int* copy_dst, int* n_copies);
+FA_API int fa_kv_num_free(const fa_kv_pool* pool);
+FA_API int fa_kv_refcount(const fa_kv_pool* pool, int block);
+FA_API int fa_kv_seq_len(const fa_kv_pool* pool, int seq);
+FA_API fa_status fa_kv_block_table(const fa_kv_pool* pool, const int* seqs, int n, int* table,
+                                   int max_blocks_per_seq, int* lens);
+FA_API fa_status fa_kv_copy_blocks(void* k_cache, void* v_cache, int num_blocks, const int* src,
+                                   const int* dst, int n, long long block_bytes, void* stream);
+
+/*
  * fa_last_device_error — synchronises `stream`, then reads and clears the
  * device error word of the current device. Returns FA_OK when nothing was
  * recorded since the last call, FA_ERR_TIMEOUT when a bounded wait gave up,
