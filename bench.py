@@ -368,16 +368,16 @@ def run_fwd_varlen(fa, steps, warmup):
 
 
 def run_kv_pool(fa, steps):
-    """Block pool on a decoding schedule: 64 sequences = 16 prompts of 512
+    """Block pool on a decoding schedule: 64 sequences = 16 prompts of 500
     tokens forked 4 ways, then `steps` rounds of one token per sequence
-    (on-demand blocks, copy-on-write of the shared partial block on the first
-    round); host time per append. Then the device copy of 4096 blocks of
+    (on-demand blocks; the shared partial last block of each prompt is copied
+    on write by 3 of its 4 sequences in the first round); host time per append. Then the device copy of 4096 blocks of
     32 KiB per cache (K and V) in GB/s (read + write)."""
     pool = fa.KVPool(65536, 16, 64, 1100)
     t0 = time.perf_counter()
     for p in range(16):
         pool.add(4 * p)
-        pool.append(4 * p, 512)
+        pool.append(4 * p, 500)
         for c in range(1, 4):
             pool.fork(4 * p, 4 * p + c)
     n_app, n_cow = 0, 0
