@@ -367,6 +367,48 @@ def run_fwd_varlen(fa, steps, warmup):
     return res
 
 
+PREFILL = dict(n=16, chunk=512, lo=1024, hi=16384, Hq=32, Hkv=8, d=128, seed=1007)
+
+
+def run_paged_prefill(fa, steps, warmup):
+    """Chunks of 512 new tokens for 16 sequences whose caches hold U[1024, 16384]
+    tokens (chunk included) in shuffled 16-token blocks; causal (bottom right)."""
+    w = PREFILL
+    rng = np.random.default_rng(w["seed"])
+    ctxs = rng.integers(w["lo"], w["hi"] + 1, w["n"]).astype(np.int32)
+    nb = [-(-int(c) // 16) for c in ctxs]
+    perm = rng.permutation(sum(nb)).astype(np.int32)
+    table = np.zeros((w["n"], max(nb)), dtype=np.int32)
+    p = 0
+    for s_, n in enumerate(nb):
+        table[s_, :n] = perm[p:p + n]
+        p += n
+    g = torch.Generator(device="cuda").manual_seed(w["seed"])
+    kc = torch.randn((sum(nb), w["Hkv"], 16, w["d"]), generator=g, device="cuda").to(torch.bfloat16)
+    vc = torch.randn_like(kc)
+    q = torch.randn((w["n"] * w["chunk"], w["Hq"], w["d"]), generator=g,
+                    device="cuda").to(torch.bfloat16)
+    cu_q = torch.arange(0, w["n"] * w["chunk"] + 1, w["chunk"], dtype=torch.int32, device="cuda")
+    tab = torch.from_numpy(table).cuda()
+    ctx = torch.from_numpy(ctxs).cuda()
+    o, lse = fa.fa_paged_prefill(q, kc, vc, tab, cu_q, ctx, w["chunk"])
+    for _ in range(warmup):
+        fa.fa_paged_prefill(q, kc, vc, tab, cu_q, ctx, w["chunk"], o=o, lse=lse)
+    torch.cuda.synchronize()
+    a, b = _ev(), _ev()
+    a.record()
+    for _ in range(steps):
+        fa.fa_paged_prefill(q, kc, vc, tab, cu_q, ctx, w["chunk"], o=o, lse=lse)
+    b.record()
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_error() == fa.FA_OK
+    ms = a.elapsed_time(b) / steps
+    L = w["chunk"]
+    pairs = sum(L * (int(c) - L) + L * (L + 1) // 2 for c in ctxs)
+    flops = 4.0 * w["d"] * w["Hq"] * pairs
+    return {"ms": ms, "TFLOP/s": flops / (ms / 1e3) / 1e12, "tokens": int(w["n"] * L)}
+
+
 def run_kv_pool(fa, steps):
     """Block pool on a decoding schedule: 64 sequences = 16 prompts of 500
     tokens forked 4 ways, then `steps` rounds of one token per sequence
@@ -485,6 +527,9 @@ def _config():
 
 def run_case(fa, case, shape, causal, steps, warmup):
     """One operation at one size, for profilers: warmup + steps launches."""
+    if case == "paged_prefill":           # the fixed prefill workload (shape unused)
+        print(json.dumps(run_paged_prefill(fa, steps, warmup)))
+        return
     if case == "kv_pool":                 # the fixed pool schedule (shape unused)
         print(json.dumps(run_kv_pool(fa, steps)))
         return
@@ -631,6 +676,11 @@ def main():
             "ms": vl["ms"], "tokens": vl["tokens"],
             "TFLOP/s": vl["flops"] / (vl["ms"] / 1e3) / 1e12,
             "bwd_ms": vl["bwd_ms"], "bwd_TFLOP/s": 2.5 * vl["flops"] / (vl["bwd_ms"] / 1e3) / 1e12}
+        pp = run_paged_prefill(fa, args.steps, args.warmup)
+        parts["paged_prefill"] = dict(pp, workload=(
+            f"{PREFILL['n']} chunks of {PREFILL['chunk']} tokens over paged caches of "
+            f"U[{PREFILL['lo']}, {PREFILL['hi']}] tokens, Hq={PREFILL['Hq']} on "
+            f"Hkv={PREFILL['Hkv']}, d={PREFILL['d']}, causal"))
         kvp = run_kv_pool(fa, 64)
         parts["kv_pool"] = dict(kvp, roofline={
             "bound": "hbm", "achieved": kvp["copy_GB/s"], "peak": peaks["hbm_gbs"],

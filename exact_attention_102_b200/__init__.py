@@ -38,7 +38,7 @@ EXPORTS = (
     "fa_bwd_varlen_workspace_bytes", "fa_bwd_varlen",
     "fa_kv_pool_create", "fa_kv_pool_destroy", "fa_kv_seq_add", "fa_kv_seq_fork", "fa_kv_seq_free",
     "fa_kv_seq_append", "fa_kv_num_free", "fa_kv_refcount", "fa_kv_seq_len", "fa_kv_block_table",
-    "fa_kv_copy_blocks",
+    "fa_kv_copy_blocks", "fa_paged_prefill",
 )
 
 
@@ -110,6 +110,8 @@ def lib() -> ctypes.CDLL:
         getattr(L, name).argtypes = [vp, ci]
     L.fa_kv_block_table.restype = ci
     L.fa_kv_block_table.argtypes = [vp, pi, ci, pi, ci, pi]
+    L.fa_paged_prefill.restype = ci
+    L.fa_paged_prefill.argtypes = [vp, vp, vp, ci, vp, ci, vp, vp, vp, vp] + [ci] * 8 + [vp]
     L.fa_kv_copy_blocks.restype = ci
     L.fa_kv_copy_blocks.argtypes = [vp, vp, ci, vp, vp, ci, ctypes.c_longlong, vp]
     L.fa_debug_wait_timeout.restype = ci
@@ -227,6 +229,30 @@ def fa_bwd_varlen(q, k, v, o, lse, do, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
                                int(max_seqlen_k), Tq, Tk, H, Hkv, d, int(bool(causal)),
                                _stream(stream)))
     return dq, dk, dv
+
+
+def fa_paged_prefill(q, k_cache, v_cache, block_table, cu_seqlens_q, context_lens, max_seqlen_q,
+                     causal=True, o=None, lse=None, stream=None):
+    """O [Tq, Hq, d], L [Hq, Tq] of packed chunks over a paged cache
+    ([P, Hkv, 16, d] bf16) through an int32 block table [batch, max_blocks]."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
+    _need(context_lens, "context_lens", torch.int32, 1)
+    Tq, Hq, d = q.shape
+    P, Hkv, bs, _ = k_cache.shape
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((Hq, Tq), dtype=torch.float32, device=q.device)
+    _check("fa_paged_prefill",
+           lib().fa_paged_prefill(_ptr(q), _ptr(k_cache), _ptr(v_cache), P, _ptr(block_table),
+                                  block_table.shape[1], _ptr(cu_seqlens_q), _ptr(context_lens),
+                                  _ptr(o), _ptr(lse), cu_seqlens_q.numel() - 1, int(max_seqlen_q),
+                                  Tq, Hq, Hkv, d, bs, int(bool(causal)), _stream(stream)))
+    return o, lse
 
 
 class KVPool:

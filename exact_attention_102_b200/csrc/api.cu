@@ -192,6 +192,59 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
+fa_status fa_paged_prefill(const void* q, const void* k_cache, const void* v_cache,
+                           int num_phys_blocks, const int* block_table, int max_blocks_per_seq,
+                           const int* cu_seqlens_q, const int* context_lens, void* o, float* lse,
+                           int batch, int max_seqlen_q, int total_q, int Hq, int Hkv, int d,
+                           int block_size, int causal, void* stream) {
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || block_table == nullptr ||
+      cu_seqlens_q == nullptr || context_lens == nullptr || !aligned16(o) || lse == nullptr)
+    return FA_ERR_INVALID_ARG;
+  if (batch < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || max_seqlen_q < 1 || total_q < 1 ||
+      max_seqlen_q > total_q || num_phys_blocks < 1 || max_blocks_per_seq < 1)
+    return FA_ERR_INVALID_ARG;
+  if ((d != 64 && d != 128) || block_size != 16) return FA_ERR_UNSUPPORTED;
+  const long long n_pairs = (static_cast<long long>(max_seqlen_q) + 255) / 256;
+  if (static_cast<long long>(batch) * Hq * n_pairs > (1ll << 31) - 1 ||
+      static_cast<long long>(total_q) * Hq > (1ll << 31) - 1 ||
+      static_cast<long long>(num_phys_blocks) * Hkv * 16 > (1ll << 31) - 1 ||
+      static_cast<long long>(max_blocks_per_seq) * 16 > (1ll << 31) - 1)
+    return FA_ERR_UNSUPPORTED;
+  uint32_t* err = error_word_ptr();
+  if (err == nullptr) return FA_ERR_LAUNCH;
+  // Q token-major [Tq][Hq][d]; the caches as [P * Hkv * 16][d] rows, boxes of
+  // 64 columns x 16 rows (one physical block of one KV head)
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Hq, total_q, 64, 1,
+                CU_TENSOR_MAP_SWIZZLE_128B, 128) ||
+      !make_map(&tk, k_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d,
+                num_phys_blocks * Hkv * 16, 1, 64, 16) ||
+      !make_map(&tv, v_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d,
+                num_phys_blocks * Hkv * 16, 1, 64, 16))
+    return FA_ERR_LAUNCH;
+  fa::FwdArgs a;
+  a.o = o;
+  a.lse = lse;
+  a.B = batch;
+  a.H = Hq;
+  a.N = max_seqlen_q;
+  a.causal = causal ? 1 : 0;
+  a.n_pairs = static_cast<int>(n_pairs);
+  a.scale_log2 = kLog2e / sqrtf(static_cast<float>(d));
+  a.err = err;
+  a.cu_q = cu_seqlens_q;
+  a.Hkv = Hkv;
+  a.Tq = total_q;
+  a.block_table = block_table;
+  a.ctx = context_lens;
+  a.max_blocks = max_blocks_per_seq;
+  a.num_phys = num_phys_blocks;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = (d == 128) ? fa::launch_fwd<128>(tq, tk, tv, a, s)
+                             : fa::launch_fwd<64>(tq, tk, tv, a, s);
+  return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   if (B < 1 || H < 1 || N < 1 || d < 1) return 0;
   const size_t rows = static_cast<size_t>(B) * H * ((static_cast<size_t>(N) + 127) / 128 * 128);

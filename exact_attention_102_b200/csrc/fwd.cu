@@ -77,7 +77,13 @@ enum : uint32_t {
   kSiteEpi = 7, kSiteDrain = 8
 };
 
-template <int D>
+// MODE (compile time, so each form carries only its own indexing):
+//   kBhnd  [B, H, N, d] tensors;
+//   kPacked packed variable-length Q / K / V (FwdArgs.cu_q, cu_k);
+//   kPaged  packed Q, keys gathered from a paged cache (FwdArgs.block_table).
+enum { kBhnd = 0, kPacked = 1, kPaged = 2 };
+
+template <int D, int MODE>
 __global__ void __launch_bounds__(384, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, FwdArgs a) {
@@ -96,17 +102,24 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   // The problem this CTA works on: Lq queries against Lk keys. BHND: one
   // (batch, head) slice of length N, TMA coordinates (row, bh). Packed mode:
   // sequence b of the batch, TMA coordinates (head, token).
-  const bool packed = a.cu_q != nullptr;
+  constexpr bool packed = MODE != kBhnd;
+  constexpr bool paged = MODE == kPaged;
   int Lq = a.N, Lk = a.N, tq0 = 0, tk0 = 0, hq = 0, hk = 0;
   if (packed) {
     const int b = bh / a.H;
     hq = bh % a.H;
     hk = hq / (a.H / a.Hkv);
     tq0 = a.cu_q[b];
-    tk0 = a.cu_k[b];
     Lq = a.cu_q[b + 1] - tq0;
-    Lk = a.cu_k[b + 1] - tk0;
-    if (tq0 < 0 || tk0 < 0 || Lq < 0 || Lk < 0 || Lq > a.N || tq0 + Lq > a.Tq || tk0 + Lk > a.Tk) {
+    if (paged) {                      // paged keys: the sequence's cached tokens
+      Lk = a.ctx[b];
+    } else {
+      tk0 = a.cu_k[b];
+      Lk = a.cu_k[b + 1] - tk0;
+    }
+    const long long k_end = paged ? static_cast<long long>(a.max_blocks) * 16
+                                                     : static_cast<long long>(a.Tk) - tk0;
+    if (tq0 < 0 || tk0 < 0 || Lq < 0 || Lk < 0 || Lq > a.N || tq0 + Lq > a.Tq || Lk > k_end) {
       if (threadIdx.x == 0 && pair == a.n_pairs - 1) atomicCAS(a.err, 0u, kErrBadIndex + 1);
       Lq = 0;                       // nothing is read or written for this sequence
       Lk = 0;
@@ -178,6 +191,22 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       int it = 0;
       bool ok = true;
       for (int j = 0; j < nkb_cta && ok; ++j) {
+        // paged keys: the 8 physical 16-token blocks of key block j (a block
+        // past the context reads block 0, masked like a tail; an id outside the
+        // pool is recorded and replaced by 0)
+        int phys[C::BN / 16];
+        if (paged) {
+#pragma unroll
+          for (int t = 0; t < C::BN / 16; ++t) {
+            const int lb = j * (C::BN / 16) + t;
+            int pb = lb * 16 < Lk ? a.block_table[static_cast<size_t>(bh / a.H) * a.max_blocks + lb] : 0;
+            if (pb < 0 || pb >= a.num_phys) {
+              atomicCAS(a.err, 0u, kErrBadIndex + 4);
+              pb = 0;
+            }
+            phys[t] = (pb * a.Hkv + hk) * 16;
+          }
+        }
         for (int w = 0; w < 2 && ok; ++w, ++it) {
           const int s = it % C::NSTAGE;
           const uint32_t ph = (it / C::NSTAGE) & 1;
@@ -185,10 +214,18 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           if (!ok) break;
           mbar_arrive_expect_tx(bar(C::B_KVF + s), C::TILE);
           const CUtensorMap* m = (w == 0) ? &tmK : &tmV;
-          const int2 yz = k_yz(j * C::BN);
-          for (int c = 0; c < C::NCHUNK; ++c)
-            tma_load_3d(base + C::RING_OFF + s * C::TILE + c * C::CHUNK, m, bar(C::B_KVF + s),
-                        c * 64, yz.x, yz.y);
+          if (paged) {
+            // eight 16-row boxes, each at its own row of the swizzled tile
+            for (int t = 0; t < C::BN / 16; ++t)
+              for (int c = 0; c < C::NCHUNK; ++c)
+                tma_load_3d(base + C::RING_OFF + s * C::TILE + c * C::CHUNK + t * 16 * 128, m,
+                            bar(C::B_KVF + s), c * 64, phys[t], 0);
+          } else {
+            const int2 yz = k_yz(j * C::BN);
+            for (int c = 0; c < C::NCHUNK; ++c)
+              tma_load_3d(base + C::RING_OFF + s * C::TILE + c * C::CHUNK, m, bar(C::B_KVF + s),
+                          c * 64, yz.x, yz.y);
+          }
         }
       }
       // drain: make sure the last loads issued have landed before teardown
@@ -447,13 +484,20 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
+    for (auto fn : {fwd_kernel<D, kBhnd>, fwd_kernel<D, kPacked>, fwd_kernel<D, kPaged>}) {
+      cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           C::SMEM_BYTES);
+      if (e != cudaSuccess) return e;
+    }
     attr_set[dev] = true;
   }
   const int grid = a.n_pairs * a.B * a.H;
-  fwd_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, a);
+  if (a.block_table != nullptr)
+    fwd_kernel<D, kPaged><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, a);
+  else if (a.cu_q != nullptr)
+    fwd_kernel<D, kPacked><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, a);
+  else
+    fwd_kernel<D, kBhnd><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, a);
   return cudaGetLastError();
 }
 

@@ -22,6 +22,13 @@ struct FwdArgs {
   const int* cu_q = nullptr;
   const int* cu_k = nullptr;
   int Hkv = 0, Tq = 0, Tk = 0;
+  // paged K / V (packed mode with block_table != nullptr; cu_k unused): the
+  // keys of sequence b are its ctx[b] cached tokens, token t in physical
+  // block block_table[b * max_blocks + t / 16] at slot t % 16, i.e. row
+  // (block * Hkv + kv head) * 16 + t % 16 of the [P * Hkv * 16][D] cache view
+  const int* block_table = nullptr;
+  const int* ctx = nullptr;
+  int max_blocks = 0, num_phys = 0;
 };
 
 template <int D>

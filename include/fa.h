@@ -181,6 +181,33 @@ FA_API fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, cons
                         void* stream);
 
 /*
+ * fa_paged_prefill — a chunk of new tokens per sequence attending to that
+ * sequence's paged KV cache ("FlashAttention系列优化", PagedAttention: the
+ * keys are reached through the block table, as in paged_attn_decode; the
+ * chunk is a prefill or an append of several tokens at once).
+ *   q, o          : bf16 [total_q][Hq][d]; sequence s's chunk is rows
+ *                   [cu_seqlens_q[s], cu_seqlens_q[s+1]); lse fp32 [Hq][total_q].
+ *   k_cache, v_cache, num_phys_blocks, block_table, max_blocks_per_seq:
+ *                   as paged_attn_decode ([P][Hkv][16][d] bf16; int32 table
+ *                   [batch][max_blocks_per_seq]).
+ *   context_lens  : int32 [batch], the cached tokens of each sequence,
+ *                   including the chunk's own (already written), so the chunk
+ *                   is the last Lq of its context_lens[s] tokens.
+ *   causal        : bottom-right, as fa_fwd_varlen: chunk query i sees cached
+ *                   tokens j <= context_lens[s] - Lq + i (0: every cached token).
+ *   d in {64, 128}, block_size 16, Hq % Hkv == 0.
+ * Errors as fa_fwd_varlen; a table entry outside [0, num_phys_blocks) is never
+ * dereferenced (block 0 is read instead) and is reported, like a context
+ * longer than max_blocks_per_seq * 16, by fa_last_device_error() as
+ * FA_ERR_INVALID_ARG.
+ */
+FA_API fa_status fa_paged_prefill(const void* q, const void* k_cache, const void* v_cache,
+                           int num_phys_blocks, const int* block_table, int max_blocks_per_seq,
+                           const int* cu_seqlens_q, const int* context_lens, void* o, float* lse,
+                           int batch, int max_seqlen_q, int total_q, int Hq, int Hkv, int d,
+                           int block_size, int causal, void* stream);
+
+/*
  * Bytes of device workspace paged_attn_decode needs for split partials
  * (fp32 O and L per (sequence, query head, split)) and a work counter, when
  * no sequence is longer than max_ctx tokens.

@@ -33,6 +33,7 @@ from .attention import (  # noqa: F401
     attention_varlen,
     attention_varlen_bwd,
     paged_decode,
+    paged_prefill,
     combine_partials,
     round_bf16,
     quantize_e4m3,

@@ -303,6 +303,36 @@ def paged_decode(q, k_cache, v_cache, block_table, context_lens, block_size=16, 
     return o, lse
 
 
+def paged_prefill(q, k_cache, v_cache, block_table, cu_q, context_lens, causal=True,
+                  block_size=16, scale=None):
+    """A chunk of queries per sequence over a paged KV cache, float64.
+
+    q: [Tq, Hq, d] packed chunks (sequence s owns rows cu_q[s]..cu_q[s+1]-1);
+    k_cache, v_cache: [P, Hkv, block_size, d]; block_table: [S, max_blocks];
+    context_lens: [S], the tokens in the cache for each sequence, the chunk's
+    own tokens included (they are its last Lq positions). The keys of sequence
+    s are gathered through the table exactly as in ``paged_decode``
+    ([FA-series] "PagedAttention"), then the chunk attends to them with the
+    packed form's bottom-right causal rule (``attention_varlen``): chunk query i
+    sits at position ctx - Lq + i and sees keys j <= ctx - Lq + i. For Lq = 1
+    this is the decode. Returns (O [Tq, Hq, d], L [Hq, Tq])."""
+    q = np.asarray(q, dtype=np.float64)
+    k_cache = np.asarray(k_cache)
+    v_cache = np.asarray(v_cache)
+    hkv = k_cache.shape[1]
+    n_seq = len(cu_q) - 1
+    lens = [int(context_lens[s]) for s in range(n_seq)]
+    cu_k = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    keys = np.zeros((max(int(cu_k[-1]), 1), hkv, q.shape[-1]))
+    vals = np.zeros_like(keys)
+    for s in range(n_seq):
+        t = np.arange(lens[s])
+        phys = np.asarray(block_table[s])[t // block_size]
+        keys[cu_k[s]:cu_k[s + 1]] = np.asarray(k_cache[phys, :, t % block_size], dtype=np.float64)
+        vals[cu_k[s]:cu_k[s + 1]] = np.asarray(v_cache[phys, :, t % block_size], dtype=np.float64)
+    return attention_varlen(q, keys, vals, cu_q, cu_k, causal, scale)
+
+
 # ---------------------------------------------------------------------------
 # FP8 (e4m3) block quantisation for the diagnostic FP8 oracle.
 # [FA-series] FlashAttentionV3 "block quantization": one scaling factor per

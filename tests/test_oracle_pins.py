@@ -513,3 +513,62 @@ def test_varlen_bwd_against_torch_autograd():
     g = oracle.attention_varlen_bwd(q, k, v, do, cu_q, cu_k, causal=True)
     for got, ref in zip(g, (tq.grad, tk.grad, tv.grad)):
         np.testing.assert_allclose(got, ref.numpy(), rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------- paged prefill
+def _paged_case(chunks, ctxs, hq, hkv, d, seed, bs=16, share=True):
+    rng = np.random.default_rng(seed)
+    nb = [-(-c // bs) for c in ctxs]
+    n_phys = sum(nb) + 3
+    perm = rng.permutation(n_phys)
+    table = np.zeros((len(ctxs), max(nb)), dtype=np.int32)
+    p = 0
+    for s, n in enumerate(nb):
+        for j in range(n):
+            table[s, j] = perm[p]
+            p += 1
+    if share and len(ctxs) > 1 and min(nb[:2]) > 1:
+        table[1, 0] = table[0, 0]                      # a shared first block
+    kc = rng.standard_normal((n_phys, hkv, bs, d))
+    vc = rng.standard_normal((n_phys, hkv, bs, d))
+    cu_q = np.concatenate([[0], np.cumsum(chunks)]).astype(np.int32)
+    q = rng.standard_normal((int(cu_q[-1]), hq, d))
+    return q, kc, vc, table, cu_q, np.array(ctxs)
+
+
+def test_paged_prefill_single_token_chunks_are_the_decode():
+    q, kc, vc, tab, cu_q, ctx = _paged_case([1, 1, 1], [40, 16, 77], 8, 2, 16, 90)
+    o, lse = oracle.paged_prefill(q, kc, vc, tab, cu_q, ctx)
+    od, ld = oracle.paged_decode(q, kc, vc, tab, ctx)
+    np.testing.assert_allclose(o, od, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse, ld.T, rtol=0, atol=1e-13)
+
+
+def test_paged_prefill_equals_packed_attention_on_the_gathered_sequence():
+    """Contiguous keys gathered by hand (loops over tokens) into the packed
+    form; the chunk is the last Lq positions of each context."""
+    chunks, ctxs = [5, 20, 3], [40, 20, 70]
+    q, kc, vc, tab, cu_q, ctx = _paged_case(chunks, ctxs, 4, 2, 8, 91)
+    o, lse = oracle.paged_prefill(q, kc, vc, tab, cu_q, ctx)
+    ks, vs = [], []
+    for s, n in enumerate(ctxs):
+        for t in range(n):
+            ks.append(kc[tab[s, t // 16], :, t % 16])
+            vs.append(vc[tab[s, t // 16], :, t % 16])
+    cu_k = np.concatenate([[0], np.cumsum(ctxs)]).astype(np.int32)
+    o2, l2 = oracle.attention_varlen(q, np.stack(ks), np.stack(vs), cu_q, cu_k, causal=True)
+    np.testing.assert_array_equal(o, o2)
+    np.testing.assert_array_equal(lse, l2)
+
+
+def test_paged_prefill_shared_block_equals_private_copy():
+    chunks, ctxs = [7, 9], [35, 50]
+    q, kc, vc, tab, cu_q, ctx = _paged_case(chunks, ctxs, 4, 4, 8, 92)
+    o, lse = oracle.paged_prefill(q, kc, vc, tab, cu_q, ctx)
+    tab2 = tab.copy()
+    kc2 = np.concatenate([kc, kc[tab[1, 0]][None]])
+    vc2 = np.concatenate([vc, vc[tab[1, 0]][None]])
+    tab2[1, 0] = kc.shape[0]                           # sequence 1 gets its own copy
+    o2, l2 = oracle.paged_prefill(q, kc2, vc2, tab2, cu_q, ctx)
+    np.testing.assert_array_equal(o, o2)
+    np.testing.assert_array_equal(lse, l2)
