@@ -409,6 +409,38 @@ def run_paged_prefill(fa, steps, warmup):
     return {"ms": ms, "TFLOP/s": flops / (ms / 1e3) / 1e12, "tokens": int(w["n"] * L)}
 
 
+SPARSE = dict(B=1, H=16, N=16384, d=128, density=0.25, causal=True, seed=1008)
+
+
+def run_block_sparse(fa, steps, warmup):
+    """Long-sequence causal forward with a random 128 x 128 block mask of
+    density 0.25 shared by the heads (diagonal blocks kept)."""
+    w = SPARSE
+    nb = w["N"] // 128
+    m = (np.random.default_rng(w["seed"]).random((nb, nb)) < w["density"]).astype(np.uint8)
+    np.fill_diagonal(m, 1)
+    x = synth.attention_inputs(w["B"], w["H"], w["N"], w["d"], w["seed"], device="cuda",
+                               with_dout=False)
+    mt = torch.from_numpy(m).cuda()
+    o, lse = fa.fa_fwd_block_sparse(x["q"], x["k"], x["v"], mt, causal=w["causal"])
+    for _ in range(warmup):
+        fa.fa_fwd_block_sparse(x["q"], x["k"], x["v"], mt, causal=w["causal"], o=o, lse=lse)
+    torch.cuda.synchronize()
+    a, b = _ev(), _ev()
+    a.record()
+    for _ in range(steps):
+        fa.fa_fwd_block_sparse(x["q"], x["k"], x["v"], mt, causal=w["causal"], o=o, lse=lse)
+    b.record()
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_error() == fa.FA_OK
+    ms = a.elapsed_time(b) / steps
+    # kept (query, key) pairs: full kept blocks below the diagonal, half of the diagonal ones
+    kept = sum(int(m[i, j]) for i in range(nb) for j in range(i)) * 128 * 128 + nb * 128 * 129 // 2
+    flops = 4.0 * w["B"] * w["H"] * w["d"] * kept
+    return {"ms": ms, "TFLOP/s": flops / (ms / 1e3) / 1e12,
+            "kept_fraction": kept / (w["N"] * (w["N"] + 1) / 2)}
+
+
 def run_kv_pool(fa, steps):
     """Block pool on a decoding schedule: 64 sequences = 16 prompts of 500
     tokens forked 4 ways, then `steps` rounds of one token per sequence
@@ -527,6 +559,9 @@ def _config():
 
 def run_case(fa, case, shape, causal, steps, warmup):
     """One operation at one size, for profilers: warmup + steps launches."""
+    if case == "block_sparse":            # the fixed block-sparse workload (shape unused)
+        print(json.dumps(run_block_sparse(fa, steps, warmup)))
+        return
     if case == "paged_prefill":           # the fixed prefill workload (shape unused)
         print(json.dumps(run_paged_prefill(fa, steps, warmup)))
         return
@@ -681,6 +716,10 @@ def main():
             f"{PREFILL['n']} chunks of {PREFILL['chunk']} tokens over paged caches of "
             f"U[{PREFILL['lo']}, {PREFILL['hi']}] tokens, Hq={PREFILL['Hq']} on "
             f"Hkv={PREFILL['Hkv']}, d={PREFILL['d']}, causal"))
+        bs = run_block_sparse(fa, args.steps, args.warmup)
+        parts["block_sparse_fwd"] = dict(bs, workload=(
+            f"causal B={SPARSE['B']} H={SPARSE['H']} N={SPARSE['N']} d={SPARSE['d']}, "
+            f"random 128 x 128 block mask, density {SPARSE['density']} + diagonal"))
         kvp = run_kv_pool(fa, 64)
         parts["kv_pool"] = dict(kvp, roofline={
             "bound": "hbm", "achieved": kvp["copy_GB/s"], "peak": peaks["hbm_gbs"],

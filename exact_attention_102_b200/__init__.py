@@ -38,7 +38,7 @@ EXPORTS = (
     "fa_bwd_varlen_workspace_bytes", "fa_bwd_varlen",
     "fa_kv_pool_create", "fa_kv_pool_destroy", "fa_kv_seq_add", "fa_kv_seq_fork", "fa_kv_seq_free",
     "fa_kv_seq_append", "fa_kv_num_free", "fa_kv_refcount", "fa_kv_seq_len", "fa_kv_block_table",
-    "fa_kv_copy_blocks", "fa_paged_prefill",
+    "fa_kv_copy_blocks", "fa_paged_prefill", "fa_fwd_block_sparse",
 )
 
 
@@ -110,6 +110,8 @@ def lib() -> ctypes.CDLL:
         getattr(L, name).argtypes = [vp, ci]
     L.fa_kv_block_table.restype = ci
     L.fa_kv_block_table.argtypes = [vp, pi, ci, pi, ci, pi]
+    L.fa_fwd_block_sparse.restype = ci
+    L.fa_fwd_block_sparse.argtypes = [vp] * 6 + [ctypes.c_longlong] + [ci] * 5 + [vp]
     L.fa_paged_prefill.restype = ci
     L.fa_paged_prefill.argtypes = [vp, vp, vp, ci, vp, ci, vp, vp, vp, vp] + [ci] * 8 + [vp]
     L.fa_kv_copy_blocks.restype = ci
@@ -229,6 +231,31 @@ def fa_bwd_varlen(q, k, v, o, lse, do, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
                                int(max_seqlen_k), Tq, Tk, H, Hkv, d, int(bool(causal)),
                                _stream(stream)))
     return dq, dk, dv
+
+
+def fa_fwd_block_sparse(q, k, v, block_mask, causal=False, o=None, lse=None, stream=None):
+    """fa_fwd on the (128 x 128) blocks a uint8 mask keeps: block_mask is
+    [nb, nb] (shared by all heads) or [B, H, nb, nb], nb = ceil(N / 128)."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, torch.bfloat16, 4)
+    B, H, N, d = q.shape
+    nb = (N + 127) // 128
+    _need(block_mask, "block_mask", torch.uint8)
+    if block_mask.shape == (nb, nb):
+        stride = 0
+    elif block_mask.shape == (B, H, nb, nb):
+        stride = nb * nb
+    else:
+        raise ValueError(f"block_mask must be [{nb}, {nb}] or [B, H, {nb}, {nb}]")
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _check("fa_fwd_block_sparse",
+           lib().fa_fwd_block_sparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                     _ptr(block_mask), stride, B, H, N, d, int(bool(causal)),
+                                     _stream(stream)))
+    return o, lse
 
 
 def fa_paged_prefill(q, k_cache, v_cache, block_table, cu_seqlens_q, context_lens, max_seqlen_q,

@@ -245,6 +245,43 @@ fa_status fa_paged_prefill(const void* q, const void* k_cache, const void* v_cac
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
+fa_status fa_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                              const unsigned char* block_mask, long long mask_bh_stride, int B,
+                              int H, int N, int d, int causal, void* stream) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      block_mask == nullptr || mask_bh_stride < 0)
+    return FA_ERR_INVALID_ARG;
+  fa_status st = check_attn_dims(B, H, N, d);
+  if (st != FA_OK) return st;
+  const long long nb = (static_cast<long long>(N) + 127) / 128;
+  if (mask_bh_stride != 0 && mask_bh_stride < nb * nb) return FA_ERR_INVALID_ARG;
+  if (nb > 512) return FA_ERR_UNSUPPORTED;            // N <= 65536 in this form
+  uint32_t* err = error_word_ptr();
+  if (err == nullptr) return FA_ERR_LAUNCH;
+  CUtensorMap tq, tk, tv;
+  const int bh = B * H;
+  if (!make_map(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, bh, 64, 128) ||
+      !make_map(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, bh, 64, 128) ||
+      !make_map(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, bh, 64, 128))
+    return FA_ERR_LAUNCH;
+  fa::FwdArgs a;
+  a.o = o;
+  a.lse = lse;
+  a.B = B;
+  a.H = H;
+  a.N = N;
+  a.causal = causal ? 1 : 0;
+  a.n_pairs = (N + 255) / 256;
+  a.scale_log2 = kLog2e / sqrtf(static_cast<float>(d));
+  a.err = err;
+  a.block_mask = block_mask;
+  a.mask_bh_stride = mask_bh_stride;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = (d == 128) ? fa::launch_fwd<128>(tq, tk, tv, a, s)
+                             : fa::launch_fwd<64>(tq, tk, tv, a, s);
+  return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   if (B < 1 || H < 1 || N < 1 || d < 1) return 0;
   const size_t rows = static_cast<size_t>(B) * H * ((static_cast<size_t>(N) + 127) / 128 * 128);

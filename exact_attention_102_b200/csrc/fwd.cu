@@ -56,7 +56,11 @@ struct FwdCfg {
   static constexpr int B_DRAIN = B_O + 2;
   static constexpr int NBAR = B_DRAIN + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // tmem slot (4 B), abort flag (4 B)
-  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + slack for 1024 B alignment
+  // block-sparse form: the CTA's key blocks (union of its two tiles' blocks),
+  // uint16 ids, uint8 per-tile flags, and three counts
+  static constexpr int MAX_UNION = 512;
+  static constexpr int UNION_OFF = MISC_OFF + 16;
+  static constexpr int SMEM_BYTES = UNION_OFF + 3 * MAX_UNION + 16 + 1024;  // + alignment slack
   // TMEM column of S_t / P_t and of O_t
   static __device__ __forceinline__ uint32_t s_col(int t) { return 128u * t; }
   static __device__ __forceinline__ uint32_t o_col(int t) { return 256u + D * t; }
@@ -81,7 +85,8 @@ enum : uint32_t {
 //   kBhnd  [B, H, N, d] tensors;
 //   kPacked packed variable-length Q / K / V (FwdArgs.cu_q, cu_k);
 //   kPaged  packed Q, keys gathered from a paged cache (FwdArgs.block_table).
-enum { kBhnd = 0, kPacked = 1, kPaged = 2 };
+//   kSparse [B, H, N, d] tensors with a 128 x 128 block mask (FwdArgs.block_mask).
+enum { kBhnd = 0, kPacked = 1, kPaged = 2, kSparse = 3 };
 
 template <int D, int MODE>
 __global__ void __launch_bounds__(384, 1)
@@ -102,8 +107,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   // The problem this CTA works on: Lq queries against Lk keys. BHND: one
   // (batch, head) slice of length N, TMA coordinates (row, bh). Packed mode:
   // sequence b of the batch, TMA coordinates (head, token).
-  constexpr bool packed = MODE != kBhnd;
+  constexpr bool packed = MODE == kPacked || MODE == kPaged;
   constexpr bool paged = MODE == kPaged;
+  constexpr bool sparse = MODE == kSparse;
   int Lq = a.N, Lk = a.N, tq0 = 0, tk0 = 0, hq = 0, hk = 0;
   if (packed) {
     const int b = bh / a.H;
@@ -140,7 +146,34 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     const int last_key = min(q0[t] + C::BM - 1, Lq - 1) + off;  // causal: last key any row sees
     nkb_t[t] = !rows_t[t] ? 0 : !a.causal ? nkb : last_key < 0 ? 0 : min(nkb, last_key / C::BN + 1);
   }
-  const int nkb_cta = max(nkb_t[0], nkb_t[1]);
+  int nkb_cta = max(nkb_t[0], nkb_t[1]);
+  // Block-sparse form: the CTA walks the union of its two tiles' active key
+  // blocks; a tile takes part in the first cnt_t union steps (those below its
+  // causal limit) and treats a step whose block it does not see as fully masked.
+  uint16_t* ulist = reinterpret_cast<uint16_t*>(smem + C::UNION_OFF);
+  uint8_t* uflag = smem + C::UNION_OFF + 2 * C::MAX_UNION;
+  int* ucount = reinterpret_cast<int*>(smem + C::UNION_OFF + 3 * C::MAX_UNION);
+  if constexpr (sparse) {
+    if (threadIdx.x == 0) {
+      const int nkb_all = (a.N + C::BN - 1) / C::BN;
+      const uint8_t* m0 = a.block_mask + bh * a.mask_bh_stride + static_cast<long long>(2 * pair) * nkb_all;
+      const uint8_t* m1 = m0 + nkb_all;
+      int n = 0, c0 = 0, c1 = 0;
+      for (int j = 0; j < nkb_cta && n < C::MAX_UNION; ++j) {
+        const bool a0 = j < nkb_t[0] && m0[j] != 0;
+        const bool a1 = j < nkb_t[1] && m1[j] != 0;
+        if (!(a0 || a1)) continue;
+        ulist[n] = static_cast<uint16_t>(j);
+        uflag[n] = static_cast<uint8_t>((a0 ? 1 : 0) | (a1 ? 2 : 0));
+        ++n;
+        if (j < nkb_t[0]) c0 = n;
+        if (j < nkb_t[1]) c1 = n;
+      }
+      ucount[0] = c0;
+      ucount[1] = c1;
+      ucount[2] = n;
+    }
+  }
   // TMA coordinates (y, z) of Q row q and of K / V row k of this problem
   auto q_yz = [&](int q) { return packed ? make_int2(hq, tq0 + q) : make_int2(q, bh); };
   auto k_yz = [&](int k) { return packed ? make_int2(hk, tk0 + k) : make_int2(k, bh); };
@@ -172,6 +205,11 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if constexpr (sparse) {                         // union steps replace key blocks
+    nkb_t[0] = ucount[0];
+    nkb_t[1] = ucount[1];
+    nkb_cta = ucount[2];
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -221,7 +259,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 tma_load_3d(base + C::RING_OFF + s * C::TILE + c * C::CHUNK + t * 16 * 128, m,
                             bar(C::B_KVF + s), c * 64, phys[t], 0);
           } else {
-            const int2 yz = k_yz(j * C::BN);
+            const int2 yz = k_yz((sparse ? ulist[j] : j) * C::BN);
             for (int c = 0; c < C::NCHUNK; ++c)
               tma_load_3d(base + C::RING_OFF + s * C::TILE + c * C::CHUNK, m, bar(C::B_KVF + s),
                           c * 64, yz.x, yz.y);
@@ -335,7 +373,18 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, sr[c]);
       tmem_ld_wait();
 #define SV(c) __uint_as_float(sr[(c) >> 5][(c)&31])
-      const int kbase = j * C::BN;
+      if (sparse && !((uflag[j] >> t) & 1)) {   // a block this tile does not see: P = 0
+        uint32_t zero[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) zero[c] = 0u;
+        tmem_st32(s_addr, zero);
+        tmem_st32(s_addr + 32, zero);
+        tmem_st_wait();
+        tc_fence_before();
+        warp_arrive(bar(C::B_P + t));
+        continue;
+      }
+      const int kbase = (sparse ? ulist[j] : j) * C::BN;
       if (kbase + C::BN - 1 > limit) {
 #pragma unroll
         for (int c = 0; c < 128; ++c)
@@ -484,7 +533,8 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    for (auto fn : {fwd_kernel<D, kBhnd>, fwd_kernel<D, kPacked>, fwd_kernel<D, kPaged>}) {
+    for (auto fn : {fwd_kernel<D, kBhnd>, fwd_kernel<D, kPacked>, fwd_kernel<D, kPaged>,
+                    fwd_kernel<D, kSparse>}) {
       cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            C::SMEM_BYTES);
       if (e != cudaSuccess) return e;
@@ -492,7 +542,9 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
     attr_set[dev] = true;
   }
   const int grid = a.n_pairs * a.B * a.H;
-  if (a.block_table != nullptr)
+  if (a.block_mask != nullptr)
+    fwd_kernel<D, kSparse><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, a);
+  else if (a.block_table != nullptr)
     fwd_kernel<D, kPaged><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, a);
   else if (a.cu_q != nullptr)
     fwd_kernel<D, kPacked><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, a);

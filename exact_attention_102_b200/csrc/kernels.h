@@ -29,6 +29,10 @@ struct FwdArgs {
   const int* block_table = nullptr;
   const int* ctx = nullptr;
   int max_blocks = 0, num_phys = 0;
+  // block-sparse [B, H, N, d] form (block_mask != nullptr): query block qb sees
+  // key block kb iff block_mask[bh * mask_bh_stride + qb * ceil(N / 128) + kb]
+  const uint8_t* block_mask = nullptr;
+  long long mask_bh_stride = 0;
 };
 
 template <int D>

@@ -208,6 +208,26 @@ FA_API fa_status fa_paged_prefill(const void* q, const void* k_cache, const void
                            int block_size, int causal, void* stream);
 
 /*
+ * fa_fwd_block_sparse — fa_fwd restricted to the (query block, key block)
+ * pairs a block mask keeps, blocks of 128 x 128 ("91haoming.cn" repost,
+ * FlashAttention v1, 實現效果: block-sparse FlashAttention; skipped blocks are
+ * neither loaded nor computed unless the other query tile of the CTA needs
+ * them, in which case they are masked).
+ *   block_mask     : uint8 device array; query block qb sees key block kb iff
+ *                    block_mask[bh * mask_bh_stride + qb * nb + kb] != 0, with
+ *                    nb = ceil(N / 128) and bh = b * H + h; mask_bh_stride = 0
+ *                    shares one nb x nb mask across all (b, h), otherwise it
+ *                    must be >= nb * nb.
+ *   causal         : applied on top of the block mask (key j <= query i).
+ *   A query that sees no key gets O = 0 and L = -inf. N <= 65536.
+ * Other arguments, layouts and errors as fa_fwd.
+ */
+FA_API fa_status fa_fwd_block_sparse(const void* q, const void* k, const void* v, void* o,
+                              float* lse, const unsigned char* block_mask,
+                              long long mask_bh_stride, int B, int H, int N, int d, int causal,
+                              void* stream);
+
+/*
  * Bytes of device workspace paged_attn_decode needs for split partials
  * (fp32 O and L per (sequence, query head, split)) and a work counter, when
  * no sequence is longer than max_ctx tokens.

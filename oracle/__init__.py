@@ -30,6 +30,7 @@ from .attention import (  # noqa: F401
     attention_fwd,
     attention_bwd,
     attention_rows,
+    attention_block_sparse,
     attention_varlen,
     attention_varlen_bwd,
     paged_decode,

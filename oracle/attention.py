@@ -103,6 +103,41 @@ def attention_fwd(q, k, v, causal=False, scale=None):
     return o.reshape(lead + (n, v2.shape[-1])), lse.reshape(lead + (n,))
 
 
+def attention_block_sparse(q, k, v, block_mask, causal=False, block=128, scale=None):
+    """Exact attention restricted by a block mask, float64, [..., N, d] inputs.
+
+    [FA-v1v2v3] FlashAttention v1 "實現效果" names block-sparse FlashAttention:
+    query i sees key j only if the mask keeps their (i // block, j // block)
+    pair (and j <= i when causal). block_mask: [nb, nb] or [..., nb, nb] of
+    0 / 1. A query that sees no key has O = 0 and L = -inf (as in
+    attention_varlen). Returns (O [..., N, d], L [..., N])."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    lead = q.shape[:-2]
+    n, d = q.shape[-2:]
+    bm = np.broadcast_to(np.asarray(block_mask) != 0, lead + np.asarray(block_mask).shape[-2:])
+    qf, kf, vf = q.reshape(-1, n, d), k.reshape(-1, n, d), v.reshape(-1, n, d)
+    bmf = bm.reshape(-1, *bm.shape[-2:])
+    blk = np.arange(n) // block
+    o = np.zeros_like(qf)
+    lse = np.full(qf.shape[:2], -np.inf)
+    for h in range(qf.shape[0]):
+        allowed = bmf[h][blk[:, None], blk[None, :]]
+        if causal:
+            allowed = allowed & (np.arange(n)[None, :] <= np.arange(n)[:, None])
+        s = _scale(d, scale) * (qf[h] @ kf[h].T)
+        s = np.where(allowed, s, -np.inf)
+        m = s.max(axis=1)                          # 3-pass safe softmax, empty rows kept at 0
+        empty = m == -np.inf
+        e = np.exp(s - np.where(empty, 0.0, m)[:, None])
+        l = e.sum(axis=1)
+        o[h] = (e / np.where(empty, 1.0, l)[:, None]) @ vf[h]
+        with np.errstate(divide="ignore"):
+            lse[h] = np.where(empty, -np.inf, m + np.log(np.where(empty, 1.0, l)))
+    return o.reshape(q.shape), lse.reshape(lead + (n,))
+
+
 def attention_varlen(q, k, v, cu_q, cu_k, causal=False, scale=None):
     """Exact attention over a packed batch of variable-length sequences.
 

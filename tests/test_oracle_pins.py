@@ -572,3 +572,45 @@ def test_paged_prefill_shared_block_equals_private_copy():
     o2, l2 = oracle.paged_prefill(q, kc2, vc2, tab2, cu_q, ctx)
     np.testing.assert_array_equal(o, o2)
     np.testing.assert_array_equal(lse, l2)
+
+
+# ------------------------------------------------------------- block sparse
+def test_block_sparse_all_ones_is_the_forward():
+    rng = np.random.default_rng(95)
+    q, k, v = (rng.standard_normal((2, 3, 50, 8)) for _ in range(3))
+    for causal in (False, True):
+        o, lse = oracle.attention_block_sparse(q, k, v, np.ones((4, 4)), causal, block=16)
+        o2, l2 = oracle.attention_fwd(q, k, v, causal)
+        np.testing.assert_allclose(o, o2, rtol=0, atol=1e-14)
+        np.testing.assert_allclose(lse, l2, rtol=0, atol=1e-13)
+
+
+def test_block_sparse_diagonal_mask_is_independent_segments():
+    """A block-diagonal mask splits the sequence into independent problems."""
+    rng = np.random.default_rng(96)
+    q, k, v = (rng.standard_normal((40, 8)) for _ in range(3))
+    o, lse = oracle.attention_block_sparse(q, k, v, np.eye(3), False, block=16)
+    for a, b in ((0, 16), (16, 32), (32, 40)):
+        o2, l2 = oracle.attention_fwd(q[a:b], k[a:b], v[a:b])
+        np.testing.assert_allclose(o[a:b], o2, rtol=0, atol=1e-14)
+        np.testing.assert_allclose(lse[a:b], l2, rtol=0, atol=1e-13)
+
+
+def test_block_sparse_brute_force_with_empty_rows():
+    rng = np.random.default_rng(97)
+    n, d, blk = 12, 4, 4
+    q, k, v = (rng.standard_normal((n, d)) for _ in range(3))
+    mask = np.array([[0, 1, 0], [0, 0, 0], [1, 1, 1]])
+    for causal in (False, True):
+        o, lse = oracle.attention_block_sparse(q, k, v, mask, causal, block=blk)
+        for i in range(n):
+            keys = [j for j in range(n) if mask[i // blk][j // blk] and (not causal or j <= i)]
+            if not keys:
+                assert np.all(o[i] == 0) and lse[i] == -np.inf
+                continue
+            s = [float(q[i] @ k[j]) / math.sqrt(d) for j in keys]
+            mx = max(s)
+            w = [math.exp(x - mx) for x in s]
+            np.testing.assert_allclose(o[i], sum(wi / sum(w) * v[j] for wi, j in zip(w, keys)),
+                                       rtol=1e-12, atol=1e-13)
+            assert abs(lse[i] - (mx + math.log(sum(w)))) < 1e-12
