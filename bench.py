@@ -152,11 +152,19 @@ def _barrier(ws):
 
 
 def _max_over_ranks(x, ws):
+    """The slowest rank's value (timings are reported as the max over ranks)."""
     if ws == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_value(flops_per_rank, ws, ms_max):
+    """Whole-job throughput: every rank did flops_per_rank; the job took the
+    slowest rank's time (weak scaling, replicas)."""
+    return ws * flops_per_rank / (ms_max / 1e3) / 1e12
 
 
 def _ev():
@@ -663,7 +671,7 @@ def main():
     f_fwd = attn_flops(w["B"], w["H"], w["N"], w["d"], w["causal"])
     f_bwd = attn_flops(w["B"], w["H"], w["N"], w["d"], w["causal"], bwd=True)
     ms = r["total_ms"] / args.steps
-    value = ws * (f_fwd + f_bwd) / (ms / 1e3) / 1e12
+    value = whole_job_value(f_fwd + f_bwd, ws, ms)
     e2e_ms, h2d, d2h = run_e2e(fa, w["B"], w["H"], w["N"], w["d"], w["causal"],
                                max(3, args.steps // 4), 2, ws, seed=1002)
     e2e_val = ws * (f_fwd + f_bwd) / (e2e_ms / 1e3) / 1e12
