@@ -15,6 +15,10 @@ attention
     merge of split partials, the packed variable-length form (sequences of
     unequal query / key lengths, grouped KV heads, bottom-right causal), and
     the FP8 e4m3 block quantiser used by the diagnostic FP8 oracle.
+dropout
+    Attention with dropout on the probabilities: the Philox4x32-10
+    counter-based generator written from its published definition, the keep
+    mask it defines element by element, and the dropout forward and backward.
 online
     A second, independent implementation of the forward: the tiled one-pass
     online-softmax recurrence (running max m, running sum l, unnormalised O
@@ -40,5 +44,12 @@ from .attention import (  # noqa: F401
     quantize_e4m3,
     dequantize_blocks_e4m3,
     fp8_block_quantize,
+)
+from .dropout import (  # noqa: F401
+    attention_dropout,
+    attention_dropout_bwd,
+    drop_threshold,
+    keep_mask,
+    philox4x32_10,
 )
 from .online import tiled_online_fwd  # noqa: F401
