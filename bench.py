@@ -449,6 +449,45 @@ def run_block_sparse(fa, steps, warmup):
             "kept_fraction": kept / (w["N"] * (w["N"] + 1) / 2)}
 
 
+DROPOUT = dict(B=1, H=16, N=16384, d=128, causal=True, p=0.1, seed=1009)
+
+
+def run_dropout(fa, steps, warmup):
+    """The long-sequence causal workload with dropout p = 0.1 on P: forward
+    and backward timed separately (same FLOP count as without dropout)."""
+    w = DROPOUT
+    B, H, N, d = w["B"], w["H"], w["N"], w["d"]
+    x = synth.attention_inputs(B, H, N, d, w["seed"], device="cuda")
+    o, lse = fa.fa_fwd_dropout(x["q"], x["k"], x["v"], w["p"], w["seed"], 0, causal=w["causal"])
+    g = [torch.empty((B, H, N, d), device="cuda") for _ in range(3)]
+    wsp = torch.empty(fa.fa_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device="cuda")
+
+    def fwd(off):
+        fa.fa_fwd_dropout(x["q"], x["k"], x["v"], w["p"], w["seed"], off, causal=w["causal"],
+                          o=o, lse=lse)
+
+    def bwd(off):
+        fa.fa_bwd_dropout(x["q"], x["k"], x["v"], o, lse, x["do"], w["p"], w["seed"], off,
+                          causal=w["causal"], dq=g[0], dk=g[1], dv=g[2], workspace=wsp)
+
+    out = {}
+    for name, op in (("fwd", fwd), ("bwd", bwd)):
+        for i in range(warmup):
+            op(i)
+        torch.cuda.synchronize()
+        a, b = _ev(), _ev()
+        a.record()
+        for i in range(steps):
+            op(i)
+        b.record()
+        torch.cuda.synchronize()
+        assert fa.fa_last_device_error() == fa.FA_OK
+        out[name + "_ms"] = a.elapsed_time(b) / steps
+    out["fwd_TFLOP/s"] = attn_flops(B, H, N, d, w["causal"]) / (out["fwd_ms"] / 1e3) / 1e12
+    out["bwd_TFLOP/s"] = attn_flops(B, H, N, d, w["causal"], bwd=True) / (out["bwd_ms"] / 1e3) / 1e12
+    return out
+
+
 def run_kv_pool(fa, steps):
     """Block pool on a decoding schedule: 64 sequences = 16 prompts of 500
     tokens forked 4 ways, then `steps` rounds of one token per sequence
@@ -567,6 +606,9 @@ def _config():
 
 def run_case(fa, case, shape, causal, steps, warmup):
     """One operation at one size, for profilers: warmup + steps launches."""
+    if case == "dropout":                 # the fixed dropout workload (shape unused)
+        print(json.dumps(run_dropout(fa, steps, warmup)))
+        return
     if case == "block_sparse":            # the fixed block-sparse workload (shape unused)
         print(json.dumps(run_block_sparse(fa, steps, warmup)))
         return
@@ -728,6 +770,10 @@ def main():
         parts["block_sparse_fwd"] = dict(bs, workload=(
             f"causal B={SPARSE['B']} H={SPARSE['H']} N={SPARSE['N']} d={SPARSE['d']}, "
             f"random 128 x 128 block mask, density {SPARSE['density']} + diagonal"))
+        dr = run_dropout(fa, max(3, args.steps // 4), args.warmup)
+        parts["dropout"] = dict(dr, workload=(
+            f"causal B={DROPOUT['B']} H={DROPOUT['H']} N={DROPOUT['N']} d={DROPOUT['d']}, "
+            f"dropout p={DROPOUT['p']} on P (Philox4x32-10 keep mask)"))
         kvp = run_kv_pool(fa, 64)
         parts["kv_pool"] = dict(kvp, roofline={
             "bound": "hbm", "achieved": kvp["copy_GB/s"], "peak": peaks["hbm_gbs"],

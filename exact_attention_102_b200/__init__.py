@@ -38,7 +38,8 @@ EXPORTS = (
     "fa_bwd_varlen_workspace_bytes", "fa_bwd_varlen",
     "fa_kv_pool_create", "fa_kv_pool_destroy", "fa_kv_seq_add", "fa_kv_seq_fork", "fa_kv_seq_free",
     "fa_kv_seq_append", "fa_kv_num_free", "fa_kv_refcount", "fa_kv_seq_len", "fa_kv_block_table",
-    "fa_kv_copy_blocks", "fa_paged_prefill", "fa_fwd_block_sparse",
+    "fa_kv_copy_blocks", "fa_paged_prefill", "fa_fwd_block_sparse", "fa_fwd_dropout",
+    "fa_bwd_dropout",
 )
 
 
@@ -118,6 +119,10 @@ def lib() -> ctypes.CDLL:
     L.fa_kv_copy_blocks.argtypes = [vp, vp, ci, vp, vp, ci, ctypes.c_longlong, vp]
     L.fa_debug_wait_timeout.restype = ci
     L.fa_debug_wait_timeout.argtypes = [ctypes.c_uint, vp]
+    L.fa_fwd_dropout.argtypes = [vp] * 5 + [ci] * 5 + [ctypes.c_float, ctypes.c_ulonglong,
+                                                        ctypes.c_uint, vp]
+    L.fa_bwd_dropout.argtypes = [vp] * 10 + [sz] + [ci] * 5 + [ctypes.c_float, ctypes.c_ulonglong,
+                                                               ctypes.c_uint, vp]
     _lib = L
     return L
 
@@ -170,6 +175,47 @@ def fa_fwd(q, k, v, causal=False, o=None, lse=None, stream=None):
     _check("fa_fwd", lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
                                   B, H, N, d, int(bool(causal)), _stream(stream)))
     return o, lse
+
+
+def fa_fwd_dropout(q, k, v, p_drop, seed, offset=0, causal=False, o=None, lse=None, stream=None):
+    """fa_fwd with dropout on P (keep mask from Philox4x32-10 keyed by seed,
+    counter word 3 = offset); O = (P o Z) V / keep_prob, L undropped."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, torch.bfloat16, 4)
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same shape [B, H, N, d]")
+    B, H, N, d = q.shape
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    _need(o, "o", torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    _check("fa_fwd_dropout", lib().fa_fwd_dropout(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, int(bool(causal)),
+        float(p_drop), int(seed) & (2**64 - 1), int(offset) & 0xFFFFFFFF, _stream(stream)))
+    return o, lse
+
+
+def fa_bwd_dropout(q, k, v, o, lse, do, p_drop, seed, offset=0, causal=False, dq=None, dk=None,
+                   dv=None, workspace=None, stream=None):
+    """Gradients of fa_fwd_dropout (same p_drop, seed, offset): fp32 dQ, dK, dV."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
+        _need(t, n, torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    B, H, N, d = q.shape
+    dq = torch.empty(q.shape, dtype=torch.float32, device=q.device) if dq is None else dq
+    dk = torch.empty(q.shape, dtype=torch.float32, device=q.device) if dk is None else dk
+    dv = torch.empty(q.shape, dtype=torch.float32, device=q.device) if dv is None else dv
+    for n, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _need(t, n, torch.float32, 4)
+    if workspace is None:
+        workspace = torch.empty(fa_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8,
+                                device=q.device)
+    _check("fa_bwd_dropout", lib().fa_bwd_dropout(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), B, H, N, d,
+        int(bool(causal)), float(p_drop), int(seed) & (2**64 - 1), int(offset) & 0xFFFFFFFF,
+        _stream(stream)))
+    return dq, dk, dv
 
 
 def fa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, causal=False, o=None,

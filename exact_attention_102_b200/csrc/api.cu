@@ -92,6 +92,139 @@ fa_status check_attn_dims(int B, int H, int N, int d) {
   return FA_OK;
 }
 
+// Dropout of the [B, H, N, d] forms: the byte threshold t = floor(256 p + 1/2)
+// (t <= 255), the Philox key words and counter word 3, and 256 / (256 - t).
+struct DropSpec {
+  uint32_t t, seed_lo, seed_hi, offset;
+  float scale;
+};
+
+bool drop_spec(float p, unsigned long long seed, unsigned int offset, DropSpec* out) {
+  if (!(p >= 0.f)) return false;                      // also rejects NaN
+  const double x = floor(256.0 * static_cast<double>(p) + 0.5);
+  if (x > 255.0) return false;
+  out->t = static_cast<uint32_t>(x);
+  out->seed_lo = static_cast<uint32_t>(seed & 0xffffffffull);
+  out->seed_hi = static_cast<uint32_t>(seed >> 32);
+  out->offset = offset;
+  out->scale = static_cast<float>(256.0 / (256.0 - x));
+  return true;
+}
+
+fa_status fwd_dense(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                    int N, int d, int causal, void* stream, const DropSpec* drop) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return FA_ERR_INVALID_ARG;
+  fa_status st = check_attn_dims(B, H, N, d);
+  if (st != FA_OK) return st;
+  uint32_t* err = error_word_ptr();
+  if (err == nullptr) return FA_ERR_LAUNCH;
+  CUtensorMap tq, tk, tv;
+  const int bh = B * H;
+  if (!make_map(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, bh, 64, 128) ||
+      !make_map(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, bh, 64, 128) ||
+      !make_map(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, bh, 64, 128))
+    return FA_ERR_LAUNCH;
+  fa::FwdArgs a;
+  a.o = o;
+  a.lse = lse;
+  a.B = B;
+  a.H = H;
+  a.N = N;
+  a.causal = causal ? 1 : 0;
+  a.n_pairs = (N + 255) / 256;
+  a.scale_log2 = kLog2e / sqrtf(static_cast<float>(d));
+  a.err = err;
+  if (drop != nullptr) {
+    a.dropout = 1;
+    a.drop_bias = (32768u - 128u * drop->t) * 0x00010001u;
+    a.seed_lo = drop->seed_lo;
+    a.seed_hi = drop->seed_hi;
+    a.drop_offset = drop->offset;
+    a.drop_scale = drop->scale;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = (d == 128) ? fa::launch_fwd<128>(tq, tk, tv, a, s)
+                             : fa::launch_fwd<64>(tq, tk, tv, a, s);
+  return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+fa_status bwd_dense(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                    const void* dout, float* dq, float* dk, float* dv, void* workspace,
+                    size_t ws_bytes, int B, int H, int N, int d, int causal, void* stream,
+                    const DropSpec* drop) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_INVALID_ARG;
+  fa_status st = check_attn_dims(B, H, N, d);
+  if (st != FA_OK) return st;
+  if (drop != nullptr && d != 128) return FA_ERR_UNSUPPORTED;
+  if (workspace == nullptr || !aligned16(workspace) ||
+      ws_bytes < fa_bwd_workspace_bytes(B, H, N, d))
+    return FA_ERR_WORKSPACE;
+  uint32_t* err = error_word_ptr();
+  if (err == nullptr) return FA_ERR_LAUNCH;
+  const int bh = B * H;
+  const size_t n_pad = (static_cast<size_t>(N) + 127) / 128 * 128;
+  const size_t prow = static_cast<size_t>(bh) * n_pad;
+  const size_t tsz = round256(static_cast<size_t>(bh) * N * d * 2);
+  char* w = static_cast<char*>(workspace);
+  char* w16 = w + 2 * round256(prow * sizeof(float));
+  void* q16 = w16;
+  void* k16 = w16 + tsz;
+  void* v16 = w16 + 2 * tsz;
+  void* do16 = w16 + 3 * tsz;
+  CUtensorMap tq, tk, tv, tdo, tdq;
+  // d = 128 steps over 64 queries at a time (64-row Q / dO boxes), d = 64 over 128
+  const uint32_t qrows = d == 128 ? 64 : 128;
+  if (!make_map(&tq, q16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, qrows) ||
+      !make_map(&tk, k16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, 128) ||
+      !make_map(&tv, v16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, 128) ||
+      !make_map(&tdo, do16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, qrows) ||
+      !make_map(&tdq, dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, N, bh, 32, 64,
+                CU_TENSOR_MAP_SWIZZLE_NONE))
+    return FA_ERR_LAUNCH;
+  fa::BwdArgs a;
+  a.q16 = q16;
+  a.k16 = k16;
+  a.v16 = v16;
+  a.do16 = do16;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.dout = dout;
+  a.lse = lse;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.n_pad = static_cast<int>(n_pad);
+  a.delta = static_cast<float*>(workspace);
+  a.lse_log2 = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                        round256(prow * sizeof(float)));
+  a.B = B;
+  a.H = H;
+  a.N = N;
+  a.causal = causal ? 1 : 0;
+  a.scale = 1.0f / sqrtf(static_cast<float>(d));
+  a.scale_log2 = a.scale * kLog2e;
+  a.err = err;
+  if (drop != nullptr) {
+    a.dropout = 1;
+    a.drop_t = drop->t;
+    a.seed_lo = drop->seed_lo;
+    a.seed_hi = drop->seed_hi;
+    a.drop_offset = drop->offset;
+    a.drop_scale = drop->scale;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaEvent_t eb = g_bwd_ev_begin, ee = g_bwd_ev_end;
+  g_bwd_ev_begin = g_bwd_ev_end = nullptr;     // one call consumes the pair
+  cudaError_t e = (d == 128) ? fa::launch_bwd<128>(tq, tk, tv, tdo, tdq, a, s, eb, ee)
+                             : fa::launch_bwd<64>(tq, tk, tv, tdo, tdq, a, s, eb, ee);
+  return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
 }  // namespace
 
 namespace fa {
@@ -115,32 +248,15 @@ const char* fa_status_str(fa_status s) {
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                  int N, int d, int causal, void* stream) {
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
-    return FA_ERR_INVALID_ARG;
-  fa_status st = check_attn_dims(B, H, N, d);
-  if (st != FA_OK) return st;
-  uint32_t* err = error_word_ptr();
-  if (err == nullptr) return FA_ERR_LAUNCH;
-  CUtensorMap tq, tk, tv;
-  const int bh = B * H;
-  if (!make_map(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, bh, 64, 128) ||
-      !make_map(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, bh, 64, 128) ||
-      !make_map(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, bh, 64, 128))
-    return FA_ERR_LAUNCH;
-  fa::FwdArgs a;
-  a.o = o;
-  a.lse = lse;
-  a.B = B;
-  a.H = H;
-  a.N = N;
-  a.causal = causal ? 1 : 0;
-  a.n_pairs = (N + 255) / 256;
-  a.scale_log2 = kLog2e / sqrtf(static_cast<float>(d));
-  a.err = err;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = (d == 128) ? fa::launch_fwd<128>(tq, tk, tv, a, s)
-                             : fa::launch_fwd<64>(tq, tk, tv, a, s);
-  return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+  return fwd_dense(q, k, v, o, lse, B, H, N, d, causal, stream, nullptr);
+}
+
+fa_status fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                         int H, int N, int d, int causal, float p_drop, unsigned long long seed,
+                         unsigned int offset, void* stream) {
+  DropSpec ds;
+  if (!drop_spec(p_drop, seed, offset, &ds)) return FA_ERR_INVALID_ARG;
+  return fwd_dense(q, k, v, o, lse, B, H, N, d, causal, stream, &ds);
 }
 
 fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -292,67 +408,18 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
                  const void* dout, float* dq, float* dk, float* dv, void* workspace,
                  size_t ws_bytes, int B, int H, int N, int d, int causal, void* stream) {
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
-      !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
-    return FA_ERR_INVALID_ARG;
-  fa_status st = check_attn_dims(B, H, N, d);
-  if (st != FA_OK) return st;
-  if (workspace == nullptr || !aligned16(workspace) ||
-      ws_bytes < fa_bwd_workspace_bytes(B, H, N, d))
-    return FA_ERR_WORKSPACE;
-  uint32_t* err = error_word_ptr();
-  if (err == nullptr) return FA_ERR_LAUNCH;
-  const int bh = B * H;
-  const size_t n_pad = (static_cast<size_t>(N) + 127) / 128 * 128;
-  const size_t prow = static_cast<size_t>(bh) * n_pad;
-  const size_t tsz = round256(static_cast<size_t>(bh) * N * d * 2);
-  char* w = static_cast<char*>(workspace);
-  char* w16 = w + 2 * round256(prow * sizeof(float));
-  void* q16 = w16;
-  void* k16 = w16 + tsz;
-  void* v16 = w16 + 2 * tsz;
-  void* do16 = w16 + 3 * tsz;
-  CUtensorMap tq, tk, tv, tdo, tdq;
-  // d = 128 steps over 64 queries at a time (64-row Q / dO boxes), d = 64 over 128
-  const uint32_t qrows = d == 128 ? 64 : 128;
-  if (!make_map(&tq, q16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, qrows) ||
-      !make_map(&tk, k16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, 128) ||
-      !make_map(&tv, v16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, 128) ||
-      !make_map(&tdo, do16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, qrows) ||
-      !make_map(&tdq, dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, N, bh, 32, 64,
-                CU_TENSOR_MAP_SWIZZLE_NONE))
-    return FA_ERR_LAUNCH;
-  fa::BwdArgs a;
-  a.q16 = q16;
-  a.k16 = k16;
-  a.v16 = v16;
-  a.do16 = do16;
-  a.q = q;
-  a.k = k;
-  a.v = v;
-  a.o = o;
-  a.dout = dout;
-  a.lse = lse;
-  a.dq = dq;
-  a.dk = dk;
-  a.dv = dv;
-  a.n_pad = static_cast<int>(n_pad);
-  a.delta = static_cast<float*>(workspace);
-  a.lse_log2 = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                        round256(prow * sizeof(float)));
-  a.B = B;
-  a.H = H;
-  a.N = N;
-  a.causal = causal ? 1 : 0;
-  a.scale = 1.0f / sqrtf(static_cast<float>(d));
-  a.scale_log2 = a.scale * kLog2e;
-  a.err = err;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaEvent_t eb = g_bwd_ev_begin, ee = g_bwd_ev_end;
-  g_bwd_ev_begin = g_bwd_ev_end = nullptr;     // one call consumes the pair
-  cudaError_t e = (d == 128) ? fa::launch_bwd<128>(tq, tk, tv, tdo, tdq, a, s, eb, ee)
-                             : fa::launch_bwd<64>(tq, tk, tv, tdo, tdq, a, s, eb, ee);
-  return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+  return bwd_dense(q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, B, H, N, d, causal,
+                   stream, nullptr);
+}
+
+fa_status fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o,
+                         const float* lse, const void* dout, float* dq, float* dk, float* dv,
+                         void* workspace, size_t ws_bytes, int B, int H, int N, int d, int causal,
+                         float p_drop, unsigned long long seed, unsigned int offset, void* stream) {
+  DropSpec ds;
+  if (!drop_spec(p_drop, seed, offset, &ds)) return FA_ERR_INVALID_ARG;
+  return bwd_dense(q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, B, H, N, d, causal,
+                   stream, &ds);
 }
 
 size_t fa_bwd_varlen_workspace_bytes(int batch, int max_seqlen_q, int total_q, int total_k, int H,

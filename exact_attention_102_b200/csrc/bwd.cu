@@ -619,7 +619,16 @@ __device__ __forceinline__ uint32_t half_col(int kk) {
 
 // PACKED selects the packed variable-length form (BwdArgs.cu_q != nullptr) at
 // compile time, so the [B, H, N, d] instantiation carries none of its indexing.
-template <bool PACKED>
+// DROP ([B, H, N, d] form only) applies the forward's dropout mask Z:
+// dV = (P o Z)^T dO / q and dS = P o (Z o dP / q - D), q the keep probability.
+// The keep bit of (query i, key j) is byte j % 16 of the Philox call
+// (j / 16, i, bh, offset). The 16 lanes holding keys 16g .. 16g+15 need the
+// same call per query, so each lane computes the calls of two of the 32
+// queries of its half and the words reach the lanes that need them by one
+// shuffle per element: the source lane of query 4b + c exposes, in round r,
+// word (c + r) % 4, which is what a lane needing word w reads in the round
+// with (w - r) % 4 = c.
+template <bool PACKED, bool DROP>
 __global__ void __launch_bounds__(512, 1)
 bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -931,7 +940,43 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         p_loop(std::true_type{});
       else
         p_loop(std::false_type{});
-      tmem_st16(s_addr, pk);                           // over this half's own S^T columns
+      uint32_t zm = 0xffffffffu;                       // bit e: (query qh + e, key) kept
+      if constexpr (DROP) {
+        const uint32_t g = lane & 15, jg = static_cast<uint32_t>(key) >> 4;
+        uint32_t x[2][4];                              // x[c][r] = word (lane % 4 + r) % 4
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const uint4 w = philox4x32_10(jg, static_cast<uint32_t>(qh) + g + 16u * c,
+                                        static_cast<uint32_t>(bh), a.drop_offset, a.seed_lo,
+                                        a.seed_hi);
+          const bool r1 = lane & 1, r2 = lane & 2;
+          const uint32_t a0 = r1 ? w.y : w.x, a1 = r1 ? w.z : w.y, a2 = r1 ? w.w : w.z,
+                         a3 = r1 ? w.x : w.w;
+          x[c][0] = r2 ? a2 : a0;
+          x[c][1] = r2 ? a3 : a1;
+          x[c][2] = r2 ? a0 : a2;
+          x[c][3] = r2 ? a1 : a3;
+        }
+        const int wsel = static_cast<int>(g >> 2);     // the word holding this key's byte
+        const uint32_t sh = 8u * (lane & 3);           // its byte within the word
+        const uint32_t keep_add = 256u - a.drop_t;     // byte + keep_add >= 256 iff kept
+        zm = 0u;
+#pragma unroll
+        for (int bq = 0; bq < 8; ++bq) {
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const int c = (wsel - r) & 3;              // query 4 bq + c arrives in round r
+            const uint32_t y = __shfl_sync(0xffffffffu, x[bq >> 2][r],
+                                           static_cast<int>(lane & 16) | ((4 * bq) & 15) | c);
+            zm |= ((((y >> sh) & 0xffu) + keep_add) >> 8) << (4 * bq + c);
+          }
+        }
+      }
+      uint32_t pz[16];                                 // P o Z for the dV product
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        pz[e] = DROP ? pk[e] & ((((zm >> (2 * e)) & 3u) * 0x8001u & 0x10001u) * 0xffffu) : pk[e];
+      tmem_st16(s_addr, pz);                           // over this half's own S^T columns
       tmem_st_wait();
       tc_fence_before();
       warp_arrive(bar(C::B_P));
@@ -949,14 +994,20 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       uint32_t w[16];                                  // dS^T, fp16 pairs of queries
       float ds_max = 0.f;
       const uint64_t neg1 = f2_pack(-1.f, -1.f);
+      const uint64_t dsc2 = f2_pack(a.drop_scale, a.drop_scale);
 #pragma unroll
       for (int e = 0; e < 32; e += 4) {
         const float4 dv4 = *reinterpret_cast<const float4*>(Ds + e);
+        uint64_t g01 = f2_pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1]));
+        uint64_t g23 = f2_pack(__uint_as_float(dr[e + 2]), __uint_as_float(dr[e + 3]));
+        if constexpr (DROP) {                          // dP -> Z o dP / q
+          auto z = [&](int i) { return dr[i] & (0u - ((zm >> i) & 1u)); };
+          g01 = f2_mul(f2_pack(__uint_as_float(z(e)), __uint_as_float(z(e + 1))), dsc2);
+          g23 = f2_mul(f2_pack(__uint_as_float(z(e + 2)), __uint_as_float(z(e + 3))), dsc2);
+        }
         // dS = P o (dP - D) on packed pairs
-        const uint64_t d01 = f2_fma(f2_pack(dv4.x, dv4.y), neg1,
-                                    f2_pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])));
-        const uint64_t d23 = f2_fma(f2_pack(dv4.z, dv4.w), neg1,
-                                    f2_pack(__uint_as_float(dr[e + 2]), __uint_as_float(dr[e + 3])));
+        const uint64_t d01 = f2_fma(f2_pack(dv4.x, dv4.y), neg1, g01);
+        const uint64_t d23 = f2_fma(f2_pack(dv4.z, dv4.w), neg1, g23);
         const uint32_t pa = pk[e / 2], pb = pk[e / 2 + 1];
         float ds[4];
         f2_unpack(f2_mul(f2_pack(f16_lo(pa), f16_hi(pa)), d01), ds[0], ds[1]);
@@ -989,7 +1040,7 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                                    : (static_cast<size_t>(bh) * a.N + key) * D;
         const uint32_t src = tmem + lane_off + (h ? C::COL_DK : C::COL_DV);
         float* dst = (h ? a.dk : a.dv) + orow;
-        const float mul = h ? a.scale : 1.f;
+        const float mul = h ? a.scale : (DROP ? a.drop_scale : 1.f);
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t v[32];
@@ -1069,15 +1120,18 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = D == 128 ? cudaFuncSetAttribute(bwd_d128_kernel<false>,
+    cudaError_t e = D == 128 ? cudaFuncSetAttribute(bwd_d128_kernel<false, false>,
                                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                     BwdD128::SMEM_BYTES)
                              : cudaFuncSetAttribute(bwd_main_kernel<D>,
                                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                     C::SMEM_BYTES);
     if (e == cudaSuccess && D == 128)
-      e = cudaFuncSetAttribute(bwd_d128_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               BwdD128::SMEM_BYTES);
+      e = cudaFuncSetAttribute(bwd_d128_kernel<true, false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, BwdD128::SMEM_BYTES);
+    if (e == cudaSuccess && D == 128)
+      e = cudaFuncSetAttribute(bwd_d128_kernel<false, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, BwdD128::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
@@ -1097,11 +1151,14 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   if (ev_main_begin != nullptr) cudaEventRecord(ev_main_begin, stream);
   if (D == 128)
     if (a.cu_q)
-      bwd_d128_kernel<true><<<nk * per_block, BwdD128::THREADS, BwdD128::SMEM_BYTES, stream>>>(
-          tq, tk, tv, tdo, tdq, a);
+      bwd_d128_kernel<true, false><<<nk * per_block, BwdD128::THREADS, BwdD128::SMEM_BYTES,
+                                     stream>>>(tq, tk, tv, tdo, tdq, a);
+    else if (a.dropout)
+      bwd_d128_kernel<false, true><<<nk * per_block, BwdD128::THREADS, BwdD128::SMEM_BYTES,
+                                     stream>>>(tq, tk, tv, tdo, tdq, a);
     else
-      bwd_d128_kernel<false><<<nk * per_block, BwdD128::THREADS, BwdD128::SMEM_BYTES, stream>>>(
-          tq, tk, tv, tdo, tdq, a);
+      bwd_d128_kernel<false, false><<<nk * per_block, BwdD128::THREADS, BwdD128::SMEM_BYTES,
+                                      stream>>>(tq, tk, tv, tdo, tdq, a);
   else
     bwd_main_kernel<D><<<nk * a.B * a.H, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
   e = cudaGetLastError();

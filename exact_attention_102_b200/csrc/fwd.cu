@@ -86,7 +86,10 @@ enum : uint32_t {
 //   kPacked packed variable-length Q / K / V (FwdArgs.cu_q, cu_k);
 //   kPaged  packed Q, keys gathered from a paged cache (FwdArgs.block_table).
 //   kSparse [B, H, N, d] tensors with a 128 x 128 block mask (FwdArgs.block_mask).
-enum { kBhnd = 0, kPacked = 1, kPaged = 2, kSparse = 3 };
+//   kDropout [B, H, N, d] tensors with dropout on P (FwdArgs.dropout): the
+//           P.V operand carries P o Z, the row sums keep the undropped P, and
+//           O is scaled by 1 / (keep probability) at the end.
+enum { kBhnd = 0, kPacked = 1, kPaged = 2, kSparse = 3, kDropout = 4 };
 
 template <int D, int MODE>
 __global__ void __launch_bounds__(384, 1)
@@ -110,6 +113,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   constexpr bool packed = MODE == kPacked || MODE == kPaged;
   constexpr bool paged = MODE == kPaged;
   constexpr bool sparse = MODE == kSparse;
+  constexpr bool dropout = MODE == kDropout;
   int Lq = a.N, Lk = a.N, tq0 = 0, tk0 = 0, hq = 0, hk = 0;
   if (packed) {
     const int b = bh / a.H;
@@ -415,8 +419,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_use, -m_use);
       uint64_t la = 0, lb = 0, ra = 0, rb = 0;     // (0.f, 0.f) pairs
       uint32_t pk0[32], pk1[32];
+      uint4 rnd = make_uint4(0u, 0u, 0u, 0u);     // dropout: random bytes of 16 keys
 #pragma unroll
       for (int q = 0; q < 64; ++q) {
+        if (dropout && (q & 7) == 0)
+          rnd = philox4x32_10(static_cast<uint32_t>((kbase >> 4) + (q >> 3)),
+                              static_cast<uint32_t>(row), static_cast<uint32_t>(bh),
+                              a.drop_offset, a.seed_lo, a.seed_hi);
         const uint64_t x2 = f2_fma(f2_pack(SV(2 * q), SV(2 * q + 1)), sl2x2, negm2);
         uint64_t p2;
         if (kPolyEvery > 0 && q % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
@@ -437,7 +446,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           la = f2_add(la, p2);
           ra = f2_add(ra, rr);
         }
-        if (q < 32) pk0[q] = u; else pk1[q - 32] = u;
+        uint32_t us = u;                           // P, or P o Z under dropout
+        if (dropout) {
+          const int wi = (q & 7) >> 1;             // keys 2q, 2q+1: bytes 2(q&1), +1 of word wi
+          const uint32_t w = wi == 0 ? rnd.x : wi == 1 ? rnd.y : wi == 2 ? rnd.z : rnd.w;
+          us &= (q & 1) ? keep_halves<1>(w, a.drop_bias) : keep_halves<0>(w, a.drop_bias);
+        }
+        if (q < 32) pk0[q] = us; else pk1[q - 32] = us;
       }
 #undef SV
       float l0, l1, l2, l3, r0, r1, r2, r3;
@@ -484,7 +499,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       if (ok) {
         tc_fence_after();
         // a row that saw no key has l = 0: O = 0, and L = m + log l = -inf
-        const float inv_l = lr_run > 0.f ? 1.f / lr_run : 0.f;
+        const float inv_l = lr_run > 0.f ? (dropout ? a.drop_scale : 1.f) / lr_run : 0.f;
         __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + orow_idx * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -534,7 +549,7 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
     for (auto fn : {fwd_kernel<D, kBhnd>, fwd_kernel<D, kPacked>, fwd_kernel<D, kPaged>,
-                    fwd_kernel<D, kSparse>}) {
+                    fwd_kernel<D, kSparse>, fwd_kernel<D, kDropout>}) {
       cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            C::SMEM_BYTES);
       if (e != cudaSuccess) return e;
@@ -542,7 +557,9 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
     attr_set[dev] = true;
   }
   const int grid = a.n_pairs * a.B * a.H;
-  if (a.block_mask != nullptr)
+  if (a.dropout)
+    fwd_kernel<D, kDropout><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, a);
+  else if (a.block_mask != nullptr)
     fwd_kernel<D, kSparse><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, a);
   else if (a.block_table != nullptr)
     fwd_kernel<D, kPaged><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, a);

@@ -33,6 +33,13 @@ struct FwdArgs {
   // key block kb iff block_mask[bh * mask_bh_stride + qb * ceil(N / 128) + kb]
   const uint8_t* block_mask = nullptr;
   long long mask_bh_stride = 0;
+  // dropout on P ([B, H, N, d] form): element (b, h, i, j) is kept iff byte
+  // j % 16 of Philox4x32-10((j / 16, i, b*H + h, drop_offset), (seed_lo,
+  // seed_hi)) is >= t; drop_bias = (32768 - 128 t) * 0x00010001;
+  // drop_scale = 256 / (256 - t) multiplies O
+  int dropout = 0;
+  uint32_t drop_bias = 0, seed_lo = 0, seed_hi = 0, drop_offset = 0;
+  float drop_scale = 1.f;
 };
 
 template <int D>
@@ -69,6 +76,11 @@ struct BwdArgs {
   const int* cu_k = nullptr;
   int Hkv = 0, Tq = 0, Tk = 0, max_k = 0;
   long long n_q_elems = 0, n_k_elems = 0;   // elements of q (= dout) and of k (= v)
+  // dropout on P (d = 128, [B, H, N, d] form), the forward's keep mask: drop_t
+  // is the byte threshold, drop_scale = 256 / (256 - t)
+  int dropout = 0;
+  uint32_t drop_t = 0, seed_lo = 0, seed_hi = 0, drop_offset = 0;
+  float drop_scale = 1.f;
 };
 
 // tdq: fp32 view of dq, [BH][N][d], box 32 x 64, no swizzle (reduce-add target

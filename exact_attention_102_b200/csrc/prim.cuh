@@ -398,4 +398,43 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// ------------------------------------------------------------------ dropout
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy
+// as 1, 2, 3", SC 2011): ten rounds of (c0, c1, c2, c3) ->
+// (hi(M1 c2) ^ c1 ^ k0, lo(M1 c2), hi(M0 c0) ^ c3 ^ k1, lo(M0 c0)) with
+// M0 = 0xD2511F53, M1 = 0xCD9E8D57 and 64-bit products, the key advanced by
+// (0x9E3779B9, 0xBB67AE85) between rounds.
+__device__ __forceinline__ uint4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
+                                               uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * c0;
+    const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * c2;
+    const uint32_t n0 = static_cast<uint32_t>(p1 >> 32) ^ c1 ^ k0;
+    const uint32_t n2 = static_cast<uint32_t>(p0 >> 32) ^ c3 ^ k1;
+    c1 = static_cast<uint32_t>(p1);
+    c3 = static_cast<uint32_t>(p0);
+    c0 = n0;
+    c2 = n2;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  return make_uint4(c0, c1, c2, c3);
+}
+
+// Keep mask of the two elements whose random bytes are bytes 2S and 2S+1 of
+// w: 0xffff over the 16-bit half of each element whose byte is >= t. Each byte
+// b goes to its own 16-bit lane as 128 b + 32768 - 128 t, a value in
+// [128, 65408] (no carry between lanes) whose bit 15 is set iff b >= t; the
+// second byte permute spreads that bit (the sign of the lane's high byte) over
+// the lane. bias = (32768 - 128 t) * 0x00010001.
+template <int S>
+__device__ __forceinline__ uint32_t keep_halves(uint32_t w, uint32_t bias) {
+  uint32_t x, m;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(x) : "r"(w), "n"(S ? 0x4342 : 0x4140));
+  const uint32_t y = x * 128u + bias;
+  asm("prmt.b32 %0, %1, 0, 0xBB99;" : "=r"(m) : "r"(y));
+  return m;
+}
+
 }  // namespace fa

@@ -228,6 +228,44 @@ FA_API fa_status fa_fwd_block_sparse(const void* q, const void* k, const void* v
                               void* stream);
 
 /*
+ * fa_fwd_dropout — fa_fwd with dropout on the attention probabilities
+ * ("91haoming.cn" repost, FlashAttention v1, 注意力實現改進: the matmuls, the
+ * softmax, the optional mask and dropout run in one fused kernel; the pages
+ * give no formula, so the contract is fixed here):
+ *   O = (P o Z) V / q_keep,  P = softmax(S / sqrt(d) [+ causal mask]);
+ *   lse is that of the undropped scores, exactly as fa_fwd writes it.
+ *   Z (keep mask): element (b, h, i, j) (query i, key j) is kept iff
+ *     byte (j % 16) of Philox4x32-10(counter = (j / 16, i, b * H + h, offset),
+ *     key = (seed & 0xffffffff, seed >> 32)) >= t, bytes numbered from the
+ *     low byte of output word 0 to the high byte of word 3 (Philox4x32-10:
+ *     Salmon et al., "Parallel random numbers: as easy as 1, 2, 3", SC 2011).
+ *   t = floor(256 * p_drop + 0.5) is the drop threshold; q_keep = 1 - t / 256.
+ *   p_drop: 0 <= p_drop and t <= 255, else FA_ERR_INVALID_ARG. The applied drop
+ *   probability is t / 256 (a multiple of 1/256).
+ * The same (seed, offset) in fa_bwd_dropout regenerates the same Z. Other
+ * arguments, layouts and errors as fa_fwd.
+ */
+FA_API fa_status fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse,
+                                int B, int H, int N, int d, int causal, float p_drop,
+                                unsigned long long seed, unsigned int offset, void* stream);
+
+/*
+ * fa_bwd_dropout — gradients of fa_fwd_dropout with its keep mask Z:
+ *   dV = (P o Z)^T dO / q_keep,  dP = Z o (dO V^T) / q_keep,
+ *   D_i = sum_c dO_ic O_ic (o = the dropout forward's output),
+ *   dS = P o (dP - D),  dQ = dS K / sqrt(d),  dK = dS^T Q / sqrt(d).
+ *   p_drop, seed, offset: those given to fa_fwd_dropout.
+ *   d = 128 only (FA_ERR_UNSUPPORTED otherwise).
+ * Workspace (fa_bwd_workspace_bytes), precision, other arguments and errors
+ * as fa_bwd.
+ */
+FA_API fa_status fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o,
+                                const float* lse, const void* dout, float* dq, float* dk,
+                                float* dv, void* workspace, size_t ws_bytes, int B, int H, int N,
+                                int d, int causal, float p_drop, unsigned long long seed,
+                                unsigned int offset, void* stream);
+
+/*
  * Bytes of device workspace paged_attn_decode needs for split partials
  * (fp32 O and L per (sequence, query head, split)) and a work counter, when
  * no sequence is longer than max_ctx tokens.

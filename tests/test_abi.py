@@ -151,3 +151,21 @@ def test_bwd_varlen_rejects_bad_arguments_without_a_gpu():
     a = list(args); a[9] = ctypes.c_void_p(0) # no workspace
     assert L.fa_bwd_varlen(*a) == fa.FA_ERR_WORKSPACE
     assert L.fa_bwd_varlen_workspace_bytes(0, 64, 128, 128, 8, 2, 128) == 0
+
+
+def test_dropout_rejects_bad_probability_and_head_dim_without_gpu():
+    L = fa.lib()
+    g = _p(0x10000)
+    for p in (-0.1, float("nan"), 1.0, 255.6 / 256):
+        assert L.fa_fwd_dropout(*([g] * 5), 1, 2, 128, 64, 0, p, 1, 0, None) == fa.FA_ERR_INVALID_ARG
+        assert L.fa_bwd_dropout(*([g] * 10), 1 << 30, 1, 2, 128, 128, 0, p, 1, 0,
+                                None) == fa.FA_ERR_INVALID_ARG
+    # a valid probability still meets the plain argument checks
+    assert L.fa_fwd_dropout(_p(0), *([g] * 4), 1, 2, 128, 64, 0, 0.1, 1, 0,
+                            None) == fa.FA_ERR_INVALID_ARG
+    assert L.fa_fwd_dropout(*([g] * 5), 1, 2, 128, 80, 0, 0.1, 1, 0, None) == fa.FA_ERR_UNSUPPORTED
+    need = L.fa_bwd_workspace_bytes(1, 2, 128, 64)
+    assert L.fa_bwd_dropout(*([g] * 10), need, 1, 2, 128, 64, 0, 0.1, 1, 0,
+                            None) == fa.FA_ERR_UNSUPPORTED          # backward: d = 128 only
+    assert L.fa_bwd_dropout(*([g] * 9), g, 0, 1, 2, 128, 128, 0, 0.1, 1, 0,
+                            None) == fa.FA_ERR_WORKSPACE
