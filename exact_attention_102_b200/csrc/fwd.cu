@@ -74,6 +74,7 @@ struct FwdCfg {
 #endif
 constexpr int kPolyEvery = FA_FWD_POLY_EVERY;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kOrderMax = 256;             // paged form: sequences ordered by context length
 
 // wait-site ids (reported in the device error word)
 enum : uint32_t {
@@ -115,8 +116,32 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   constexpr bool sparse = MODE == kSparse;
   constexpr bool dropout = MODE == kDropout;
   int Lq = a.N, Lk = a.N, tq0 = 0, tk0 = 0, hq = 0, hk = 0;
+  int seq = 0;                        // packed forms: the sequence of this CTA
   if (packed) {
-    const int b = bh / a.H;
+    // Paged form, longest context first: within each wave of pairs, the CTAs
+    // of the sequence with the r-th longest context (ties by index) come r-th,
+    // so long contexts do not end up in the tail of the grid (chunks of equal
+    // length over contexts of very unequal length). Up to kOrderMax sequences;
+    // beyond that, and in the plain packed form, batch order.
+    int b = bh / a.H;
+    static_assert(3 * C::MAX_UNION + 16 >= 4 * (kOrderMax + 1), "order list exceeds its area");
+    if (paged && a.B <= kOrderMax) {
+      int* klen = reinterpret_cast<int*>(smem + C::UNION_OFF);   // unused by these forms
+      int* pick = klen + kOrderMax;
+      for (int s_ = threadIdx.x; s_ < a.B; s_ += blockDim.x)
+        klen[s_] = a.ctx[s_];
+      if (threadIdx.x == 0) *pick = b;
+      __syncthreads();
+      for (int s_ = threadIdx.x; s_ < a.B; s_ += blockDim.x) {
+        const int ls = klen[s_];
+        int r = 0;
+        for (int u = 0; u < a.B; ++u) r += klen[u] > ls || (klen[u] == ls && u < s_);
+        if (r == b) *pick = s_;
+      }
+      __syncthreads();
+      b = *pick;
+    }
+    seq = b;
     hq = bh % a.H;
     hk = hq / (a.H / a.Hkv);
     tq0 = a.cu_q[b];
@@ -241,7 +266,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 #pragma unroll
           for (int t = 0; t < C::BN / 16; ++t) {
             const int lb = j * (C::BN / 16) + t;
-            int pb = lb * 16 < Lk ? a.block_table[static_cast<size_t>(bh / a.H) * a.max_blocks + lb] : 0;
+            int pb = lb * 16 < Lk ? a.block_table[static_cast<size_t>(seq) * a.max_blocks + lb] : 0;
             if (pb < 0 || pb >= a.num_phys) {
               atomicCAS(a.err, 0u, kErrBadIndex + 4);
               pb = 0;
