@@ -611,6 +611,9 @@ struct BwdD128 {
 };
 static_assert(BwdD128::SMEM_BYTES <= 232448, "d = 128 backward exceeds shared memory");
 
+constexpr int kOrderMaxB = 256;   // packed backward: sequences ordered by query length
+static_assert(BwdD128::DS_BYTES >= 4 * (kOrderMaxB + 1), "order list exceeds the dS buffer");
+
 // TMEM column of the 16-query group kk of a packed fp16 [key][64 queries]
 // operand whose two 32-query halves start 32 columns apart.
 __device__ __forceinline__ uint32_t half_col(int kk) {
@@ -649,10 +652,31 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   constexpr bool packed = PACKED;
   int kb, bh = 0, b = 0, hk = 0, group = 1, Lq = a.N, Lk = a.N, tq0 = 0, tk0 = 0;
   if (packed) {
-    const int BHk = a.B * a.Hkv;
-    kb = static_cast<int>(blockIdx.x) / BHk;
-    b = static_cast<int>(blockIdx.x) % BHk / a.Hkv;
-    hk = static_cast<int>(blockIdx.x) % a.Hkv;
+    // The key blocks of one (sequence, KV head) are adjacent in the grid, so
+    // the CTAs running at the same time stream the same Q, dO rows and add
+    // into the same dQ rows (shared in L2). Sequences come longest query range
+    // first (the work of each of their CTAs), up to kOrderMaxB of them; beyond
+    // that, batch order.
+    const int nkb_all = (a.max_k + C::BK - 1) / C::BK;
+    const int o = static_cast<int>(blockIdx.x) / nkb_all;
+    kb = static_cast<int>(blockIdx.x) % nkb_all;
+    hk = o % a.Hkv;
+    b = o / a.Hkv;
+    if (a.B <= kOrderMaxB) {
+      int* qlen = reinterpret_cast<int*>(smem + C::DS_OFF);   // free until the first dS
+      int* pick = qlen + kOrderMaxB;
+      for (int s_ = threadIdx.x; s_ < a.B; s_ += blockDim.x) qlen[s_] = a.cu_q[s_ + 1] - a.cu_q[s_];
+      if (threadIdx.x == 0) *pick = b;
+      __syncthreads();
+      for (int s_ = threadIdx.x; s_ < a.B; s_ += blockDim.x) {
+        const int ls = qlen[s_];
+        int r = 0;
+        for (int u = 0; u < a.B; ++u) r += qlen[u] > ls || (qlen[u] == ls && u < s_);
+        if (r == b) *pick = s_;
+      }
+      __syncthreads();
+      b = *pick;
+    }
     group = a.H / a.Hkv;
     tq0 = a.cu_q[b];
     tk0 = a.cu_k[b];
