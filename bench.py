@@ -44,9 +44,9 @@ import synth  # noqa: E402
 WORKLOAD = dict(B=1, H=16, N=16384, d=128, causal=True)
 METRIC = "attention fwd+bwd TFLOP/s (bf16)"
 # DRAM bytes (read + write) of one d = 128 backward main-pass launch at WORKLOAD
-# (2.01 GB read + 1.16 GB written), from an ncu capture of that launch with the
+# (0.429 GB read + 0.369 GB written), from an ncu capture of that launch with the
 # current kernel; set to None whenever the kernel changes until captured again
-BWD_MAIN_TRAFFIC = 3.17e9
+BWD_MAIN_TRAFFIC = 0.798e9
 
 
 def _peaks():
