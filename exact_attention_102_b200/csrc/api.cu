@@ -92,6 +92,16 @@ fa_status check_attn_dims(int B, int H, int N, int d) {
   return FA_OK;
 }
 
+// Grid grouping of the [B, H, N, d] forms: when the bytes the running CTAs
+// stream per head (K and V in the forward; Q, dO and the fp32 dQ in the
+// backward) exceed half of L2 over all heads, launch the heads in groups of 4
+// so that those rows are shared in L2; otherwise (everything stays in L2) one
+// group, which keeps the heaviest work first over all heads.
+int head_group_for(int BH, int N, int d, int bytes_per_elem) {
+  const double streamed = static_cast<double>(BH) * N * d * bytes_per_elem;
+  return streamed > 64.0e6 ? 4 : 0;
+}
+
 // Dropout of the [B, H, N, d] forms: the byte threshold t = floor(256 p + 1/2)
 // (t <= 255), the Philox key words and counter word 3, and 256 / (256 - t).
 struct DropSpec {
@@ -135,6 +145,7 @@ fa_status fwd_dense(const void* q, const void* k, const void* v, void* o, float*
   a.n_pairs = (N + 255) / 256;
   a.scale_log2 = kLog2e / sqrtf(static_cast<float>(d));
   a.err = err;
+  a.head_group = head_group_for(bh, N, d, 4);   // K and V, bf16
   if (drop != nullptr) {
     a.dropout = 1;
     a.drop_bias = (32768u - 128u * drop->t) * 0x00010001u;
@@ -209,6 +220,7 @@ fa_status bwd_dense(const void* q, const void* k, const void* v, const void* o, 
   a.scale = 1.0f / sqrtf(static_cast<float>(d));
   a.scale_log2 = a.scale * kLog2e;
   a.err = err;
+  a.head_group = head_group_for(bh, N, d, 8);   // Q, dO fp16 and dQ fp32
   if (drop != nullptr) {
     a.dropout = 1;
     a.drop_t = drop->t;
@@ -390,6 +402,9 @@ fa_status fa_fwd_block_sparse(const void* q, const void* k, const void* v, void*
   a.n_pairs = (N + 255) / 256;
   a.scale_log2 = kLog2e / sqrtf(static_cast<float>(d));
   a.err = err;
+  // one group: with few key blocks kept per query block, K / V reuse is low
+  // and the CTAs' work is uneven, so heaviest pair first over every head wins
+  a.head_group = 0;
   a.block_mask = block_mask;
   a.mask_bh_stride = mask_bh_stride;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
