@@ -612,10 +612,6 @@ struct BwdD128 {
 static_assert(BwdD128::SMEM_BYTES <= 232448, "d = 128 backward exceeds shared memory");
 
 constexpr int kOrderMaxB = 256;   // packed backward: sequences ordered by query length
-#ifndef FA_BWD_HEAD_GROUP
-#define FA_BWD_HEAD_GROUP 4
-#endif
-constexpr int kHeadGroup = FA_BWD_HEAD_GROUP;   // [B, H, N, d] backward: heads per grid group
 static_assert(BwdD128::DS_BYTES >= 4 * (kOrderMaxB + 1), "order list exceeds the dS buffer");
 
 // TMEM column of the 16-query group kk of a packed fp16 [key][64 queries]
@@ -692,17 +688,19 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       Lk = 0;
     }
   } else {
-    // (batch, head) slices in groups of kHeadGroup, key-block major inside a
-    // group: the heaviest key blocks still come first within each group, and
-    // the CTAs running at the same time cover few heads, so the Q, dO and dQ
-    // rows they stream are shared in L2.
+    // (batch, head) slices in groups of BwdArgs.head_group, key-block major
+    // inside a group: the heaviest key blocks still come first within each
+    // group, and the CTAs running at the same time cover few heads, so the Q,
+    // dO and dQ rows they stream are shared in L2 (the host groups only when
+    // those outgrow L2).
     const int BH = a.B * a.H;
     const int nkb_all = (a.N + C::BK - 1) / C::BK;
-    const int g = static_cast<int>(blockIdx.x) / (kHeadGroup * nkb_all);
-    const int gsize = min(kHeadGroup, BH - g * kHeadGroup);
-    const int r = static_cast<int>(blockIdx.x) - g * kHeadGroup * nkb_all;
+    const int G = a.head_group > 0 ? min(a.head_group, BH) : BH;
+    const int g = static_cast<int>(blockIdx.x) / (G * nkb_all);
+    const int gsize = min(G, BH - g * G);
+    const int r = static_cast<int>(blockIdx.x) - g * G * nkb_all;
     kb = r / gsize;
-    bh = g * kHeadGroup + r % gsize;
+    bh = g * G + r % gsize;
   }
   if (kb * C::BK >= Lk) return;                        // no keys in this block
   const int off = a.causal ? Lk - Lq : 0;              // causal: query i sees keys <= i + off

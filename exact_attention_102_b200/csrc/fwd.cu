@@ -75,10 +75,6 @@ struct FwdCfg {
 constexpr int kPolyEvery = FA_FWD_POLY_EVERY;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kOrderMax = 256;             // paged form: sequences ordered by context length
-#ifndef FA_FWD_HEAD_GROUP
-#define FA_FWD_HEAD_GROUP 4
-#endif
-constexpr int kFwdHeadGroup = FA_FWD_HEAD_GROUP;   // [B, H, N, d] forms: heads per grid group
 
 // wait-site ids (reported in the device error word)
 enum : uint32_t {
@@ -110,20 +106,22 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   const int lane = threadIdx.x & 31;
   const int BH = a.B * a.H;
   constexpr bool packed = MODE == kPacked || MODE == kPaged;
-  // [B, H, N, d] forms: (batch, head) slices in groups of kFwdHeadGroup,
+  // [B, H, N, d] forms: (batch, head) slices in groups of FwdArgs.head_group,
   // heaviest pair first inside a group, so the running CTAs cover few heads
-  // and share their K / V rows in L2. Packed forms: heaviest pair first over
-  // all (sequence, head) slots.
+  // and share their K / V rows in L2 (the host groups only when K and V
+  // outgrow L2). Packed forms: heaviest pair first over all (sequence, head)
+  // slots.
   int pair, bh;
   if (packed) {
     pair = a.n_pairs - 1 - static_cast<int>(blockIdx.x) / BH;
     bh = static_cast<int>(blockIdx.x) % BH;
   } else {
-    const int g = static_cast<int>(blockIdx.x) / (kFwdHeadGroup * a.n_pairs);
-    const int gsize = min(kFwdHeadGroup, BH - g * kFwdHeadGroup);
-    const int r = static_cast<int>(blockIdx.x) - g * kFwdHeadGroup * a.n_pairs;
+    const int G = a.head_group > 0 ? min(a.head_group, BH) : BH;
+    const int g = static_cast<int>(blockIdx.x) / (G * a.n_pairs);
+    const int gsize = min(G, BH - g * G);
+    const int r = static_cast<int>(blockIdx.x) - g * G * a.n_pairs;
     pair = a.n_pairs - 1 - r / gsize;
-    bh = g * kFwdHeadGroup + r % gsize;
+    bh = g * G + r % gsize;
   }
 
   // The problem this CTA works on: Lq queries against Lk keys. BHND: one

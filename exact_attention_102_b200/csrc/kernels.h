@@ -40,6 +40,9 @@ struct FwdArgs {
   int dropout = 0;
   uint32_t drop_bias = 0, seed_lo = 0, seed_hi = 0, drop_offset = 0;
   float drop_scale = 1.f;
+  // [B, H, N, d] forms: (batch, head) slices per grid group (<= 0: one group
+  // of all slices, i.e. heaviest pair first over every head)
+  int head_group = 0;
 };
 
 template <int D>
@@ -81,6 +84,9 @@ struct BwdArgs {
   int dropout = 0;
   uint32_t drop_t = 0, seed_lo = 0, seed_hi = 0, drop_offset = 0;
   float drop_scale = 1.f;
+  // d = 128, [B, H, N, d] form: (batch, head) slices per grid group (<= 0:
+  // one group of all slices, key-block major over every head)
+  int head_group = 0;
 };
 
 // tdq: fp32 view of dq, [BH][N][d], box 32 x 64, no swizzle (reduce-add target
