@@ -146,32 +146,54 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
 
 
-def _need(t, name, dtype, ndim=None):
+def _require_cuda(t, name):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+
+
+def _need(t, name, dtype, ndim=None, shape=None):
+    """Type, dtype, rank, exact shape (when given), contiguity, then device.
+
+    The library receives raw pointers and cannot see sizes, so every tensor it
+    reads or writes is checked here against the sizes passed with it."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor")
-    if not t.is_contiguous():
-        raise ValueError(f"{name} must be contiguous")
     if ndim is not None and t.dim() != ndim:
         raise ValueError(f"{name} must have {ndim} dims")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    _require_cuda(t, name)
+
+
+def _need_workspace(t):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("workspace must be a torch.Tensor")
+    if not t.is_contiguous():
+        raise ValueError("workspace must be contiguous")
+    _require_cuda(t, "workspace")
+
+
+def _need_lengths(t, name, n):
+    """int32 length / offset array with exactly n entries."""
+    _need(t, name, torch.int32, 1, (n,))
 
 
 def fa_fwd(q, k, v, causal=False, o=None, lse=None, stream=None):
     """O, L = attention forward on bf16 [B, H, N, d] tensors; L is fp32 [B, H, N]."""
-    for n, t in (("q", q), ("k", k), ("v", v)):
-        _need(t, n, torch.bfloat16, 4)
-    if k.shape != q.shape or v.shape != q.shape:
-        raise ValueError("q, k, v must have the same shape [B, H, N, d]")
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, shape=q.shape)
+    _need(v, "v", torch.bfloat16, shape=q.shape)
     B, H, N, d = q.shape
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    _need(o, "o", torch.bfloat16, 4)
-    _need(lse, "lse", torch.float32, 3)
+    _need(o, "o", torch.bfloat16, shape=q.shape)
+    _need(lse, "lse", torch.float32, shape=(B, H, N))
     _check("fa_fwd", lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
                                   B, H, N, d, int(bool(causal)), _stream(stream)))
     return o, lse
@@ -180,15 +202,14 @@ def fa_fwd(q, k, v, causal=False, o=None, lse=None, stream=None):
 def fa_fwd_dropout(q, k, v, p_drop, seed, offset=0, causal=False, o=None, lse=None, stream=None):
     """fa_fwd with dropout on P (keep mask from Philox4x32-10 keyed by seed,
     counter word 3 = offset); O = (P o Z) V / keep_prob, L undropped."""
-    for n, t in (("q", q), ("k", k), ("v", v)):
-        _need(t, n, torch.bfloat16, 4)
-    if k.shape != q.shape or v.shape != q.shape:
-        raise ValueError("q, k, v must have the same shape [B, H, N, d]")
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, shape=q.shape)
+    _need(v, "v", torch.bfloat16, shape=q.shape)
     B, H, N, d = q.shape
     o = torch.empty_like(q) if o is None else o
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
-    _need(o, "o", torch.bfloat16, 4)
-    _need(lse, "lse", torch.float32, 3)
+    _need(o, "o", torch.bfloat16, shape=q.shape)
+    _need(lse, "lse", torch.float32, shape=(B, H, N))
     _check("fa_fwd_dropout", lib().fa_fwd_dropout(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, int(bool(causal)),
         float(p_drop), int(seed) & (2**64 - 1), int(offset) & 0xFFFFFFFF, _stream(stream)))
@@ -198,18 +219,20 @@ def fa_fwd_dropout(q, k, v, p_drop, seed, offset=0, causal=False, o=None, lse=No
 def fa_bwd_dropout(q, k, v, o, lse, do, p_drop, seed, offset=0, causal=False, dq=None, dk=None,
                    dv=None, workspace=None, stream=None):
     """Gradients of fa_fwd_dropout (same p_drop, seed, offset): fp32 dQ, dK, dV."""
-    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
-        _need(t, n, torch.bfloat16, 4)
-    _need(lse, "lse", torch.float32, 3)
+    _need(q, "q", torch.bfloat16, 4)
+    for n, t in (("k", k), ("v", v), ("o", o), ("do", do)):
+        _need(t, n, torch.bfloat16, shape=q.shape)
     B, H, N, d = q.shape
+    _need(lse, "lse", torch.float32, shape=(B, H, N))
     dq = torch.empty(q.shape, dtype=torch.float32, device=q.device) if dq is None else dq
     dk = torch.empty(q.shape, dtype=torch.float32, device=q.device) if dk is None else dk
     dv = torch.empty(q.shape, dtype=torch.float32, device=q.device) if dv is None else dv
     for n, t in (("dq", dq), ("dk", dk), ("dv", dv)):
-        _need(t, n, torch.float32, 4)
+        _need(t, n, torch.float32, shape=q.shape)
     if workspace is None:
         workspace = torch.empty(fa_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8,
                                 device=q.device)
+    _need_workspace(workspace)
     _check("fa_bwd_dropout", lib().fa_bwd_dropout(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
         _ptr(workspace), workspace.numel() * workspace.element_size(), B, H, N, d,
@@ -223,22 +246,23 @@ def fa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, causal=Fals
     """O, L for a packed batch: q [Tq, H, d], k / v [Tk, Hkv, d] bf16 (token-major),
     cu_seqlens int32 [batch + 1] on the device; L is fp32 [H, Tq]. Causal is
     aligned to the bottom right (query i of Lq sees keys j <= i + Lk - Lq)."""
-    for n, t in (("q", q), ("k", k), ("v", v)):
-        _need(t, n, torch.bfloat16, 3)
-    _need(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
-    _need(cu_seqlens_k, "cu_seqlens_k", torch.int32, 1)
-    if k.shape != v.shape or k.shape[2] != q.shape[2]:
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k, "k", torch.bfloat16, 3)
+    _need(v, "v", torch.bfloat16, shape=k.shape)
+    if k.shape[2] != q.shape[2]:
         raise ValueError("k and v must be [Tk, Hkv, d] with q's d")
-    if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 2:
-        raise ValueError("cu_seqlens_q and cu_seqlens_k must both have batch + 1 entries")
+    _need(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
+    if cu_seqlens_q.numel() < 2:
+        raise ValueError("cu_seqlens_q must have batch + 1 >= 2 entries")
+    _need_lengths(cu_seqlens_k, "cu_seqlens_k", cu_seqlens_q.numel())
     Tq, H, d = q.shape
     Tk, Hkv, _ = k.shape
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((H, Tq), dtype=torch.float32, device=q.device)
-    _need(o, "o", torch.bfloat16, 3)
-    _need(lse, "lse", torch.float32, 2)
+    _need(o, "o", torch.bfloat16, shape=q.shape)
+    _need(lse, "lse", torch.float32, shape=(H, Tq))
     _check("fa_fwd_varlen",
            lib().fa_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens_q),
                                _ptr(cu_seqlens_k), cu_seqlens_q.numel() - 1, int(max_seqlen_q),
@@ -254,22 +278,31 @@ def fa_bwd_varlen_workspace_bytes(batch, max_seqlen_q, total_q, total_k, H, Hkv,
 def fa_bwd_varlen(q, k, v, o, lse, do, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
                   causal=False, dq=None, dk=None, dv=None, workspace=None, stream=None):
     """dQ [Tq, H, d], dK, dV [Tk, Hkv, d] (fp32) of fa_fwd_varlen's attention."""
-    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
-        _need(t, n, torch.bfloat16, 3)
-    _need(lse, "lse", torch.float32, 2)
-    _need(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
-    _need(cu_seqlens_k, "cu_seqlens_k", torch.int32, 1)
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k, "k", torch.bfloat16, 3)
+    _need(v, "v", torch.bfloat16, shape=k.shape)
+    _need(o, "o", torch.bfloat16, shape=q.shape)
+    _need(do, "do", torch.bfloat16, shape=q.shape)
+    if k.shape[2] != q.shape[2]:
+        raise ValueError("k and v must be [Tk, Hkv, d] with q's d")
     Tq, H, d = q.shape
     Tk, Hkv, _ = k.shape
+    _need(lse, "lse", torch.float32, shape=(H, Tq))
+    _need(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
+    if cu_seqlens_q.numel() < 2:
+        raise ValueError("cu_seqlens_q must have batch + 1 >= 2 entries")
+    _need_lengths(cu_seqlens_k, "cu_seqlens_k", cu_seqlens_q.numel())
     batch = cu_seqlens_q.numel() - 1
     dq = torch.empty(q.shape, dtype=torch.float32, device=q.device) if dq is None else dq
     dk = torch.empty(k.shape, dtype=torch.float32, device=q.device) if dk is None else dk
     dv = torch.empty(k.shape, dtype=torch.float32, device=q.device) if dv is None else dv
-    for n, t in (("dq", dq), ("dk", dk), ("dv", dv)):
-        _need(t, n, torch.float32, 3)
+    _need(dq, "dq", torch.float32, shape=q.shape)
+    _need(dk, "dk", torch.float32, shape=k.shape)
+    _need(dv, "dv", torch.float32, shape=k.shape)
     need = fa_bwd_varlen_workspace_bytes(batch, max_seqlen_q, Tq, Tk, H, Hkv, d)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _need_workspace(workspace)
     _check("fa_bwd_varlen",
            lib().fa_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq),
                                _ptr(dk), _ptr(dv), _ptr(workspace), workspace.numel(),
@@ -282,21 +315,26 @@ def fa_bwd_varlen(q, k, v, o, lse, do, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
 def fa_fwd_block_sparse(q, k, v, block_mask, causal=False, o=None, lse=None, stream=None):
     """fa_fwd on the (128 x 128) blocks a uint8 mask keeps: block_mask is
     [nb, nb] (shared by all heads) or [B, H, nb, nb], nb = ceil(N / 128)."""
-    for n, t in (("q", q), ("k", k), ("v", v)):
-        _need(t, n, torch.bfloat16, 4)
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, shape=q.shape)
+    _need(v, "v", torch.bfloat16, shape=q.shape)
     B, H, N, d = q.shape
     nb = (N + 127) // 128
-    _need(block_mask, "block_mask", torch.uint8)
+    if not isinstance(block_mask, torch.Tensor):
+        raise TypeError("block_mask must be a torch.Tensor")
     if block_mask.shape == (nb, nb):
         stride = 0
     elif block_mask.shape == (B, H, nb, nb):
         stride = nb * nb
     else:
         raise ValueError(f"block_mask must be [{nb}, {nb}] or [B, H, {nb}, {nb}]")
+    _need(block_mask, "block_mask", torch.uint8)
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _need(o, "o", torch.bfloat16, shape=q.shape)
+    _need(lse, "lse", torch.float32, shape=(B, H, N))
     _check("fa_fwd_block_sparse",
            lib().fa_fwd_block_sparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
                                      _ptr(block_mask), stride, B, H, N, d, int(bool(causal)),
@@ -310,16 +348,25 @@ def fa_paged_prefill(q, k_cache, v_cache, block_table, cu_seqlens_q, context_len
     ([P, Hkv, 16, d] bf16) through an int32 block table [batch, max_blocks]."""
     _need(q, "q", torch.bfloat16, 3)
     _need(k_cache, "k_cache", torch.bfloat16, 4)
-    _need(v_cache, "v_cache", torch.bfloat16, 4)
-    _need(block_table, "block_table", torch.int32, 2)
+    _need(v_cache, "v_cache", torch.bfloat16, shape=k_cache.shape)
+    if k_cache.shape[3] != q.shape[2]:
+        raise ValueError("k_cache and v_cache must be [P, Hkv, block_size, d] with q's d")
     _need(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
-    _need(context_lens, "context_lens", torch.int32, 1)
+    if cu_seqlens_q.numel() < 2:
+        raise ValueError("cu_seqlens_q must have batch + 1 >= 2 entries")
+    batch = cu_seqlens_q.numel() - 1
+    _need(block_table, "block_table", torch.int32, 2)
+    if block_table.shape[0] != batch:
+        raise ValueError(f"block_table must have one row per sequence ({batch})")
+    _need_lengths(context_lens, "context_lens", batch)
     Tq, Hq, d = q.shape
     P, Hkv, bs, _ = k_cache.shape
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((Hq, Tq), dtype=torch.float32, device=q.device)
+    _need(o, "o", torch.bfloat16, shape=q.shape)
+    _need(lse, "lse", torch.float32, shape=(Hq, Tq))
     _check("fa_paged_prefill",
            lib().fa_paged_prefill(_ptr(q), _ptr(k_cache), _ptr(v_cache), P, _ptr(block_table),
                                   block_table.shape[1], _ptr(cu_seqlens_q), _ptr(context_lens),
@@ -391,9 +438,9 @@ def kv_copy_blocks(k_cache, v_cache, src, dst, stream=None):
     """Copy physical block src[i] -> dst[i] in both paged caches
     ([P][Hkv][block_size][d] bf16); src, dst int32 device tensors."""
     _need(k_cache, "k_cache", torch.bfloat16, 4)
-    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, shape=k_cache.shape)
     _need(src, "src", torch.int32, 1)
-    _need(dst, "dst", torch.int32, 1)
+    _need(dst, "dst", torch.int32, shape=src.shape)
     block_bytes = k_cache[0].numel() * 2
     _check("fa_kv_copy_blocks",
            lib().fa_kv_copy_blocks(_ptr(k_cache), _ptr(v_cache), k_cache.shape[0], _ptr(src),
@@ -407,18 +454,20 @@ def fa_bwd_workspace_bytes(B, H, N, d):
 def fa_bwd(q, k, v, o, lse, do, causal=False, dq=None, dk=None, dv=None, workspace=None,
            stream=None):
     """dQ, dK, dV (fp32 [B, H, N, d]) of attention, recomputing P from L."""
-    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
-        _need(t, n, torch.bfloat16, 4)
-    _need(lse, "lse", torch.float32, 3)
+    _need(q, "q", torch.bfloat16, 4)
+    for n, t in (("k", k), ("v", v), ("o", o), ("do", do)):
+        _need(t, n, torch.bfloat16, shape=q.shape)
     B, H, N, d = q.shape
+    _need(lse, "lse", torch.float32, shape=(B, H, N))
     dq = torch.empty(q.shape, dtype=torch.float32, device=q.device) if dq is None else dq
     dk = torch.empty(q.shape, dtype=torch.float32, device=q.device) if dk is None else dk
     dv = torch.empty(q.shape, dtype=torch.float32, device=q.device) if dv is None else dv
     for n, t in (("dq", dq), ("dk", dk), ("dv", dv)):
-        _need(t, n, torch.float32, 4)
+        _need(t, n, torch.float32, shape=q.shape)
     ws = fa_bwd_workspace_bytes(B, H, N, d)
     if workspace is None:
         workspace = torch.empty(ws, dtype=torch.uint8, device=q.device)
+    _need_workspace(workspace)
     _check("fa_bwd", lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do),
                                   _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
                                   workspace.numel() * workspace.element_size(),
@@ -430,25 +479,37 @@ def paged_attn_decode_workspace_bytes(num_seqs, Hq, d, max_ctx):
     return int(lib().paged_attn_decode_workspace_bytes(num_seqs, Hq, d, max_ctx))
 
 
+def _need_decode(q, k_cache, v_cache, block_table, context_lens):
+    """Checks shared by the decode calls; returns (S, Hq, d)."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, shape=k_cache.shape)
+    if k_cache.shape[3] != q.shape[2]:
+        raise ValueError("k_cache and v_cache must be [P, Hkv, block_size, d] with q's d")
+    S = q.shape[0]
+    _need(block_table, "block_table", torch.int32, 2)
+    if block_table.shape[0] != S:
+        raise ValueError(f"block_table must have one row per sequence ({S})")
+    _need_lengths(context_lens, "context_lens", S)
+    return tuple(q.shape)
+
+
 def paged_attn_decode(q, k_cache, v_cache, block_table, context_lens, max_ctx, o=None,
                       lse=None, want_lse=True, workspace=None, stream=None):
     """One-token decode over a paged cache; returns (O bf16 [S, Hq, d], L fp32 [S, Hq] or None)."""
-    _need(q, "q", torch.bfloat16, 3)
-    _need(k_cache, "k_cache", torch.bfloat16, 4)
-    _need(v_cache, "v_cache", torch.bfloat16, 4)
-    _need(block_table, "block_table", torch.int32, 2)
-    _need(context_lens, "context_lens", torch.int32, 1)
-    if v_cache.shape != k_cache.shape:
-        raise ValueError("k_cache and v_cache must have the same shape")
-    S, Hq, d = q.shape
+    S, Hq, d = _need_decode(q, k_cache, v_cache, block_table, context_lens)
     Hkv, bs = k_cache.shape[1], k_cache.shape[2]
     if o is None:
         o = torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
+    _need(o, "o", torch.bfloat16, shape=q.shape)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, shape=(S, Hq))
     ws = paged_attn_decode_workspace_bytes(S, Hq, d, max_ctx)
     if workspace is None:
         workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=q.device)
+    _need_workspace(workspace)
     _check("paged_attn_decode", lib().paged_attn_decode(
         _ptr(q), _ptr(k_cache), _ptr(v_cache), k_cache.shape[0], _ptr(block_table),
         block_table.shape[1],
@@ -462,15 +523,10 @@ def paged_attn_decode_noalloc(q, k_cache, v_cache, block_table, context_lens, ma
     """paged_attn_decode with the library's internal scratch instead of a
     workspace. ``o`` (and ``lse`` if wanted) must be preallocated by the caller:
     this wrapper allocates nothing."""
-    _need(q, "q", torch.bfloat16, 3)
-    _need(k_cache, "k_cache", torch.bfloat16, 4)
-    _need(v_cache, "v_cache", torch.bfloat16, 4)
-    _need(block_table, "block_table", torch.int32, 2)
-    _need(context_lens, "context_lens", torch.int32, 1)
-    _need(o, "o", torch.bfloat16, 3)
+    S, Hq, d = _need_decode(q, k_cache, v_cache, block_table, context_lens)
+    _need(o, "o", torch.bfloat16, shape=q.shape)
     if lse is not None:
-        _need(lse, "lse", torch.float32, 2)
-    S, Hq, d = q.shape
+        _need(lse, "lse", torch.float32, shape=(S, Hq))
     _check("paged_attn_decode_noalloc", lib().paged_attn_decode_noalloc(
         _ptr(q), _ptr(k_cache), _ptr(v_cache), k_cache.shape[0], _ptr(block_table),
         block_table.shape[1], _ptr(context_lens), _ptr(o), _ptr(lse), S, Hq, k_cache.shape[1], d,
@@ -480,10 +536,11 @@ def paged_attn_decode_noalloc(q, k_cache, v_cache, block_table, context_lens, ma
 
 def fa_fp8_prepare(q, k, v, R, stream=None):
     """Rotate Q, K by R and quantise Q, K, V to e4m3 with 64-row block scales."""
-    for n, t in (("q", q), ("k", k), ("v", v)):
-        _need(t, n, torch.bfloat16, 4)
-    _need(R, "R", torch.float32, 2)
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, shape=q.shape)
+    _need(v, "v", torch.bfloat16, shape=q.shape)
     B, H, N, d = q.shape
+    _need(R, "R", torch.float32, shape=(d, d))
     nb = (N + 63) // 64
     q8, k8, v8 = (torch.empty(q.shape, dtype=torch.uint8, device=q.device) for _ in range(3))
     sq, sk, sv = (torch.empty((B, H, nb), dtype=torch.float32, device=q.device) for _ in range(3))
@@ -495,13 +552,18 @@ def fa_fp8_prepare(q, k, v, R, stream=None):
 
 def fa_fwd_fp8(q8, k8, v8, sq, sk, sv, causal=False, o=None, lse=None, stream=None):
     """Attention forward on e4m3 inputs (uint8 storage) with per-block scales."""
-    for n, t in (("q8", q8), ("k8", k8), ("v8", v8)):
-        _need(t, n, torch.uint8, 4)
+    _need(q8, "q8", torch.uint8, 4)
+    _need(k8, "k8", torch.uint8, shape=q8.shape)
+    _need(v8, "v8", torch.uint8, shape=q8.shape)
     B, H, N, d = q8.shape
+    for n, t in (("sq", sq), ("sk", sk), ("sv", sv)):
+        _need(t, n, torch.float32, shape=(B, H, (N + 63) // 64))
     if o is None:
         o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q8.device)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q8.device)
+    _need(o, "o", torch.bfloat16, shape=(B, H, N, d))
+    _need(lse, "lse", torch.float32, shape=(B, H, N))
     _check("fa_fwd_fp8", lib().fa_fwd_fp8(
         _ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq), _ptr(sk), _ptr(sv), _ptr(o), _ptr(lse),
         B, H, N, d, int(bool(causal)), _stream(stream)))
