@@ -789,7 +789,7 @@ def main():
             parts["fp8_fwd"] = f8
 
     cpu = None
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:   # the host baseline: N = 1 only
         cpu = cpu_baseline()
 
     if rank == 0:
