@@ -159,3 +159,30 @@ def test_delta_identity_with_dropout():
     z = keep_mask(1, 1, 20, p, seed, off)[0, 0]
     dp = z * (g[0, 0] @ v[0, 0].T) / keep_prob(drop_threshold(p))
     assert np.allclose(dd[0, 0], (pr * dp).sum(1), rtol=0, atol=1e-12)
+
+
+def test_forward_brute_force_loops():
+    # tiny causal case in plain loops: one Philox call per element, the
+    # softmax by its definition, kept terms summed and divided by q
+    B, H, N, d = 1, 2, 20, 4
+    q_, k, v, _ = _inputs(B, H, N, d, 12)
+    p, seed, off = 0.4, 0xABCDEF0123, 6
+    t = drop_threshold(p)
+    qk = keep_prob(t)
+    o, lse = attention_dropout(q_, k, v, p, seed, off, causal=True)
+    s = 1.0 / math.sqrt(d)
+    for h in range(H):
+        for i in range(N):
+            logits = [s * sum(q_[0, h, i, c] * k[0, h, j, c] for c in range(d)) for j in range(i + 1)]
+            m = max(logits)
+            l = sum(math.exp(x - m) for x in logits)
+            acc = [0.0] * d
+            for j in range(i + 1):
+                w = philox4x32_10(np.array([j // 16, i, h, off], dtype=np.uint64),
+                                  (seed & 0xFFFFFFFF, seed >> 32))
+                byte = (int(w[(j % 16) // 4]) >> (8 * (j % 4))) & 0xFF
+                if byte >= t:
+                    for c in range(d):
+                        acc[c] += math.exp(logits[j] - m) / l * v[0, h, j, c]
+            assert np.allclose(o[0, h, i], [a / qk for a in acc], rtol=0, atol=1e-12)
+            assert abs(lse[0, h, i] - (m + math.log(l))) < 1e-12
