@@ -15,12 +15,15 @@
 //   dV_j += P^T dO_i,  dP = dO_i V_j^T,  dS = P o (dP - D_i)
 //   dK_j += scale dS^T Q_i,  dQ_i += scale dS K_j   (fp32 reductions to HBM)
 //
-// Precision: the tensor-core operands of the backward are fp16. The bf16
-// inputs convert exactly (bf16 values within fp16's range are fp16 values), and
-// P and dS, which are rounded to the operand type, keep 3 more mantissa bits
-// than bf16 would give them. Inputs with |x| >= 65504 do not fit fp16: the
-// conversion flags them, as does the dS pass for |dS| >= 65504
-// (FA_ERR_UNSUPPORTED through the device error word).
+// Precision: the tensor-core operands of the backward are fp16 copies of the
+// bf16 inputs, each tensor multiplied by a power of two picked from its
+// largest magnitude so that its values sit inside fp16's range (an amax pass
+// and the conversion pass run before the main pass; the factors are undone in
+// fp32, see "operand scaling" below). P and dS, rounded to the operand type,
+// keep 3 more mantissa bits than bf16 would give them. The scale of dS is
+// chosen so that |dS| stays below 2^15 whenever L is the logsumexp of the
+// scores; a dS beyond fp16's range (possible only with an inconsistent L) is
+// recorded as FA_ERR_UNSUPPORTED.
 //
 // B200 mapping (one CTA per (batch*head, key block), 512 threads):
 //   warp 0       TMA producer: K_j, V_j once; Q_i and dO_i per row block
@@ -42,6 +45,8 @@
 // tile once dS is out), dV [256, 256+D), dK [256+D, 256+2D).
 #include <climits>
 #include <type_traits>
+
+#include <atomic>
 
 #include "prim.cuh"
 #include "kernels.h"
@@ -87,44 +92,154 @@ enum : uint32_t {
   kSiteDSF = 0x3c, kSiteDQ = 0x3d, kSiteEnd = 0x3e, kSiteDrain = 0x3f, kSitePR = 0x40
 };
 
-constexpr float kDsScale = 1.0f;   // dS is stored unscaled (fp16: |dS| < 65504)
-
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
                "f"(c), "f"(d)
                : "memory");
 }
 
+// ------------------------------------------------------ operand scaling
+// The tensor-core operands of the backward are fp16 (P and dS keep 3 more
+// mantissa bits than bf16 would give them, and A and B of one MMA share a
+// type). fp16 has 5 exponent bits against bf16's 8, so every input tensor X
+// is first multiplied by a power of two 2^e_X chosen from its largest
+// magnitude a_X = f 2^x (f in [0.5, 1)):
+//   e_X = 14 - x,  so |X 2^e_X| < 2^14.
+// A power-of-two factor changes no significant bit. A scaled element of
+// magnitude >= 2^-17 is an fp16 value exactly (fp16 subnormals below that keep
+// fewer than bf16's 8 bits), i.e. every element with |x| >= 2^-30 a_X converts
+// exactly; a smaller one is rounded to a multiple of 2^(-24 - e_X), an error
+// below 2^-38 a_X. The factors are undone in fp32, where they cost nothing:
+//   S    = 2^-(e_q + e_k) S',             folded into scale * log2(e)
+//   dP   = 2^-(e_do + e_v) dP'
+//   dS'  = 2^sigma dS, sigma = e_do + e_v - 14 - log2(d), so that
+//          dS' = P o (2^-(14 + log2 d) dP' - D'),  D' = 2^sigma D,
+//          and |dS| <= P (|dP| + |D|) <= 2 d a_do a_v (O within V's range)
+//          gives |dS'| < 2^15 (fp16 holds 65504)
+//   dV   = 2^-e_do (P^T dO'),  dK = scale 2^-(sigma + e_q) (dS'^T Q'),
+//   dQ   = scale 2^-(sigma + e_k) (dS' K').
+// A tensor that is all zeros or holds a non-finite value keeps e_X = 0.
+// bf16 magnitudes span 2^-133 .. 2^128, so e_X lies in [-114, 146].
+
+// x * 2^n as two exact power-of-two multiplications (each factor a normal
+// float); |n| is clamped to 252, beyond which the product of any finite
+// nonzero fp32 value is 0 or infinite anyway.
+struct Pow2 {
+  float f1, f2;
+};
+__device__ __forceinline__ Pow2 pow2_pair(int n) {
+  n = max(-252, min(252, n));
+  const int n1 = n / 2, n2 = n - n1;
+  return Pow2{__int_as_float((127 + n1) << 23), __int_as_float((127 + n2) << 23)};
+}
+__device__ __forceinline__ float mul_pow2(float x, Pow2 p) { return (x * p.f1) * p.f2; }
+__device__ __forceinline__ float mul_pow2(float x, int n) { return mul_pow2(x, pow2_pair(n)); }
+
+// e_X from the magnitude bits (0x0000 .. 0x7fff) of the largest |x|.
+__device__ __forceinline__ int scale_exp(uint32_t mag) {
+  if (mag == 0u || mag >= 0x7f80u) return 0;   // all zeros, or inf / NaN present
+  int x;
+  frexpf(__uint_as_float(mag << 16), &x);
+  return 14 - x;
+}
+
+// 14 + log2(d) for the dS scale; d is 64 or 128
+__device__ __forceinline__ int ds_shift(int D) { return D == 128 ? 21 : 20; }
+
+// The four per-tensor maxima of |q|, |k|, |v|, |dout|: one partial per block
+// (bf16 magnitude bits, compared as integers: for non-NaN values the order of
+// the bits is the order of the magnitudes, and NaN sorts above infinity).
+__global__ void __launch_bounds__(256) bwd_amax_kernel(BwdArgs a, long long q8, long long k8) {
+  __shared__ uint32_t red[8][4];
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  uint32_t m[4];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const uint4* src = static_cast<const uint4*>(t == 0 ? a.q : t == 1 ? a.k : t == 2 ? a.v : a.dout);
+    const long long n = (t == 0 || t == 3) ? q8 : k8;
+    uint32_t mm = 0u;
+    for (long long i = tid; i < n; i += stride) {
+      const uint4 u = src[i];
+      mm = __vmaxu2(mm, __vmaxu2(__vmaxu2(u.x & 0x7fff7fffu, u.y & 0x7fff7fffu),
+                                 __vmaxu2(u.z & 0x7fff7fffu, u.w & 0x7fff7fffu)));
+    }
+    mm = max(mm & 0xffffu, mm >> 16);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mm = max(mm, __shfl_xor_sync(0xffffffffu, mm, off));
+    m[t] = mm;
+  }
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0)
+    for (int t = 0; t < 4; ++t) red[w][t] = m[t];
+  __syncthreads();
+  if (threadIdx.x < 4) {
+    uint32_t r = 0u;
+    for (int i = 0; i < 8; ++i) r = max(r, red[i][threadIdx.x]);
+    a.amax_part[blockIdx.x * 4 + threadIdx.x] = r;
+  }
+}
+
+// Reduces the partial maxima into e_q, e_k, e_v, e_do (in shared memory).
+__device__ __forceinline__ void load_exps(const BwdArgs& a, int (&e)[4]) {
+  __shared__ uint32_t red[8][4];
+  uint32_t m[4] = {0u, 0u, 0u, 0u};
+  for (int i = threadIdx.x; i < kBwdAmaxBlocks; i += blockDim.x) {
+    const uint4 u = reinterpret_cast<const uint4*>(a.amax_part)[i];
+    m[0] = max(m[0], u.x);
+    m[1] = max(m[1], u.y);
+    m[2] = max(m[2], u.z);
+    m[3] = max(m[3], u.w);
+  }
+#pragma unroll
+  for (int t = 0; t < 4; ++t)
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m[t] = max(m[t], __shfl_xor_sync(0xffffffffu, m[t], off));
+  if ((threadIdx.x & 31) == 0)
+    for (int t = 0; t < 4; ++t) red[threadIdx.x >> 5][t] = m[t];
+  __syncthreads();
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    uint32_t r = 0u;
+    for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) r = max(r, red[i][t]);
+    e[t] = scale_exp(r);
+  }
+}
+
 // ------------------------------------------------------- fp16 conversion
-// q, k, v, dout (bf16) -> fp16 copies; 8 elements per thread per step.
+// q, k, v, dout (bf16) -> fp16 copies scaled by 2^e_X; 8 elements per thread
+// per step, the tensors in the reverse of the amax pass's order (the last
+// rows that pass read may still be in L2). Block 0 publishes the exponents
+// for the kernels that follow.
 __global__ void __launch_bounds__(256) bwd_convert_kernel(BwdArgs a, long long q8, long long k8) {
-  // q8: 8-element groups of q and of dout; k8: of k and of v
-  bool bad = false;
+  int e[4];
+  load_exps(a, e);
+  if (blockIdx.x == 0 && threadIdx.x < 4) a.exps[threadIdx.x] = e[threadIdx.x];
+  const Pow2 f[4] = {pow2_pair(e[0]), pow2_pair(e[1]), pow2_pair(e[2]), pow2_pair(e[3])};
   const long long total = 2 * q8 + 2 * k8;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int t = i < q8 ? 0 : i < q8 + k8 ? 1 : i < q8 + 2 * k8 ? 2 : 3;
-    const long long j = i - (t == 0 ? 0 : t == 1 ? q8 : t == 2 ? q8 + k8 : q8 + 2 * k8);
+    const int t = i < q8 ? 3 : i < q8 + k8 ? 2 : i < q8 + 2 * k8 ? 1 : 0;
+    const long long j = i - (t == 3 ? 0 : t == 2 ? q8 : t == 1 ? q8 + k8 : q8 + 2 * k8);
     const void* sp = t == 0 ? a.q : t == 1 ? a.k : t == 2 ? a.v : a.dout;
     void* dp = t == 0 ? a.q16 : t == 1 ? a.k16 : t == 2 ? a.v16 : a.do16;
+    const Pow2 et = f[t];
     const uint4 u = static_cast<const uint4*>(sp)[j];
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
     uint32_t o[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xffff0000u);
-      bad |= !(fabsf(lo) < 65504.f) || !(fabsf(hi) < 65504.f);
-      o[e] = pack_f16x2(lo, hi);
-    }
+    for (int c = 0; c < 4; ++c)
+      o[c] = pack_f16x2(mul_pow2(__uint_as_float(w[c] << 16), et),
+                        mul_pow2(__uint_as_float(w[c] & 0xffff0000u), et));
     static_cast<uint4*>(dp)[j] = make_uint4(o[0], o[1], o[2], o[3]);
   }
-  if (bad) atomicCAS(a.err, 0u, kErrRange + 1);
 }
 
 // ---------------------------------------------------------------- pre pass
 // Per padded row (bh, n), n < n_pad = ceil(N/128)*128:
-//   D[bh][n]  = sum_c dO_nc O_nc  (0 for n >= N)
-//   Ll[bh][n] = L_n * log2(e)     (+inf for n >= N, so P = 0 there)
+//   delta[bh][n] = -D'_n = -2^-(14 + log2 d) sum_c (dO_nc 2^e_do)(O_nc 2^e_v)
+//                  (0 for n >= N)
+//   Ll[bh][n]    = L_n * log2(e)     (+inf for n >= N, so P = 0 there)
 // and dQ rows n < N are zeroed (dQ is accumulated by the main pass).
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdArgs a) {
@@ -133,6 +248,8 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdArgs a) {
   const long long rows = static_cast<long long>(a.B) * a.H * a.n_pad;
   const int nw = (gridDim.x * blockDim.x) >> 5;
   const bool packed = a.cu_q != nullptr;
+  const Pow2 f_v = pow2_pair(a.exps[2]), f_do = pow2_pair(a.exps[3]);
+  const float alpha = __int_as_float((127 - ds_shift(D)) << 23);
   for (long long pr = warp; pr < rows; pr += nw) {
     const long long bh = pr / a.n_pad;
     const int n = static_cast<int>(pr - bh * a.n_pad);
@@ -162,18 +279,47 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdArgs a) {
     for (int c = lane * 2; c < D; c += 64) {
       const __nv_bfloat162 ov = *reinterpret_cast<const __nv_bfloat162*>(o + c);
       const __nv_bfloat162 gv = *reinterpret_cast<const __nv_bfloat162*>(g + c);
-      acc = fmaf(__bfloat162float(ov.x), __bfloat162float(gv.x), acc);
-      acc = fmaf(__bfloat162float(ov.y), __bfloat162float(gv.y), acc);
+      acc = fmaf(mul_pow2(__bfloat162float(ov.x), f_v), mul_pow2(__bfloat162float(gv.x), f_do), acc);
+      acc = fmaf(mul_pow2(__bfloat162float(ov.y), f_v), mul_pow2(__bfloat162float(gv.y), f_do), acc);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (lane == 0) {
-      a.delta[pr] = acc;
+      a.delta[pr] = -alpha * acc;
       a.lse_log2[pr] = a.lse[lr] * 1.4426950408889634f;
     }
     float4* dq = reinterpret_cast<float4*>(a.dq + r * D);
     for (int c = lane; c < D / 4; c += 32) dq[c] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
+}
+
+// The fp32 factors that undo the operand scales in the main passes.
+struct BwdScales {
+  float c_s;        // scale * log2(e) * 2^-(e_q + e_k): S' -> log2-domain scores
+  float alpha;      // 2^-(14 + log2 d): dP' -> the dS' units
+  float dv;         // 2^-e_do (times 1 / keep probability with dropout)
+  float dk;         // scale * 2^-(sigma + e_q)
+  float dq1, dq2;   // dq1 * dq2 = scale * 2^-(sigma + e_k) (dq2 = 1 unless out of range)
+};
+
+template <int D>
+__device__ __forceinline__ BwdScales bwd_scales(const BwdArgs& a) {
+  const int e_q = a.exps[0], e_k = a.exps[1], e_v = a.exps[2], e_do = a.exps[3];
+  const int sigma = e_do + e_v - ds_shift(D);
+  BwdScales s;
+  s.c_s = mul_pow2(a.scale_log2, -(e_q + e_k));
+  s.alpha = __int_as_float((127 - ds_shift(D)) << 23);
+  s.dv = mul_pow2(a.dropout ? a.drop_scale : 1.f, -e_do);
+  s.dk = mul_pow2(a.scale, -(sigma + e_q));
+  const int nq = -(sigma + e_k);
+  if (nq >= -100 && nq <= 100) {
+    s.dq1 = mul_pow2(a.scale, nq);
+    s.dq2 = 1.f;
+  } else {
+    s.dq1 = mul_pow2(a.scale, nq / 2);
+    s.dq2 = mul_pow2(1.f, nq - nq / 2);
+  }
+  return s;
 }
 
 // --------------------------------------------------------------- main pass
@@ -372,7 +518,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int key = kb * C::BK + r;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t st_addr = tmem + lane_off + C::COL_ST;
-    const float sl2 = a.scale_log2;
+    const float sl2 = bwd_scales<D>(a).c_s;
     for (int it = 0; it < n_it; ++it) {
       const int s = it & 1;
       const int q0 = (i0 + it) * C::BQ;
@@ -421,6 +567,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const uint32_t st_addr = tmem + lane_off + C::COL_ST;
     const uint32_t dpt_addr = tmem + lane_off + C::COL_DPT;
     uint8_t* ds_row = smem + C::DS_OFF + r * 128;    // row r of each 64-query chunk
+    const float alpha = __int_as_float((127 - ds_shift(D)) << 23);
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int s = it & 1;
@@ -460,7 +607,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             const int q = g * 16 + e + u;
             const uint32_t pp = PK(q >> 1);
             const float pv = (q & 1) ? f16_hi(pp) : f16_lo(pp);
-            ds[u] = (pv * kDsScale) * (__uint_as_float(dr[e + u]) - Dv[u]);
+            ds[u] = pv * fmaf(__uint_as_float(dr[e + u]), alpha, Dv[u]);   // Dv = -D'
           }
           ds_max = fmaxf(ds_max, fmaxf(fmaxf(fabsf(ds[0]), fabsf(ds[1])),
                                        fmaxf(fabsf(ds[2]), fabsf(ds[3]))));
@@ -493,7 +640,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int which = 0; which < 2; ++which) {
           const uint32_t src = tmem + lane_off + (which ? C::COL_DK : C::COL_DV);
           float* dst = (which ? a.dk : a.dv) + orow;
-          const float mul = which ? a.scale / kDsScale : 1.f;
+          const BwdScales sc = bwd_scales<D>(a);
+          const float mul = which ? sc.dk : sc.dv;
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t v[32];
@@ -517,7 +665,10 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int r = (warp & 3) * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t src = tmem + lane_off + C::COL_DPT;
-    const float sc = a.scale / kDsScale;
+    const BwdScales bs = bwd_scales<D>(a);
+    const float sc = bs.dq1, sc2 = bs.dq2;
+    const bool two = sc2 != 1.f;
+    auto f = [&](uint32_t v) { const float t = __uint_as_float(v) * sc; return two ? t * sc2 : t; };
     for (int it = 0; it < n_it; ++it) {
       const int q = (i0 + it) * C::BQ + r;
       if (!__all_sync(0xffffffffu, mbar_wait(bar(C::B_DQ), it & 1, a.err, kSiteDQ, abort_flag)))
@@ -532,9 +683,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (q < a.N) {
 #pragma unroll
           for (int e = 0; e < 8; ++e)
-            red_add_v4(dst + c * 32 + 4 * e, __uint_as_float(v[4 * e]) * sc,
-                       __uint_as_float(v[4 * e + 1]) * sc, __uint_as_float(v[4 * e + 2]) * sc,
-                       __uint_as_float(v[4 * e + 3]) * sc);
+            red_add_v4(dst + c * 32 + 4 * e, f(v[4 * e]), f(v[4 * e + 1]), f(v[4 * e + 2]),
+                       f(v[4 * e + 3]));
         }
       }
       tc_fence_before();
@@ -909,7 +1059,8 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t s_addr = tmem + lane_off + C::COL_S + 32 * h;
     const uint32_t dp_addr = tmem + lane_off + C::COL_DP + 32 * h;
-    const float sl2 = a.scale_log2;
+    const BwdScales sc = bwd_scales<D>(a);
+    const float sl2 = sc.c_s;
     bool ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_KV), 0, a.err, kSiteKV, abort_flag));
     if (ok) {
       // K row r, head-dim columns [64h, 64h+64): the A operand of S^T, packed
@@ -1028,21 +1179,23 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tmem_ld_wait();
       uint32_t w[16];                                  // dS^T, fp16 pairs of queries
       float ds_max = 0.f;
-      const uint64_t neg1 = f2_pack(-1.f, -1.f);
-      const uint64_t dsc2 = f2_pack(a.drop_scale, a.drop_scale);
+      // alpha (2^-(14 + log2 d)) brings dP' to the units of dS'; with dropout
+      // it also carries 1 / q
+      const float ga = DROP ? sc.alpha * a.drop_scale : sc.alpha;
+      const uint64_t ga2 = f2_pack(ga, ga);
 #pragma unroll
       for (int e = 0; e < 32; e += 4) {
-        const float4 dv4 = *reinterpret_cast<const float4*>(Ds + e);
+        const float4 dv4 = *reinterpret_cast<const float4*>(Ds + e);   // -D'
         uint64_t g01 = f2_pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1]));
         uint64_t g23 = f2_pack(__uint_as_float(dr[e + 2]), __uint_as_float(dr[e + 3]));
-        if constexpr (DROP) {                          // dP -> Z o dP / q
+        if constexpr (DROP) {                          // dP -> Z o dP
           auto z = [&](int i) { return dr[i] & (0u - ((zm >> i) & 1u)); };
-          g01 = f2_mul(f2_pack(__uint_as_float(z(e)), __uint_as_float(z(e + 1))), dsc2);
-          g23 = f2_mul(f2_pack(__uint_as_float(z(e + 2)), __uint_as_float(z(e + 3))), dsc2);
+          g01 = f2_pack(__uint_as_float(z(e)), __uint_as_float(z(e + 1)));
+          g23 = f2_pack(__uint_as_float(z(e + 2)), __uint_as_float(z(e + 3)));
         }
-        // dS = P o (dP - D) on packed pairs
-        const uint64_t d01 = f2_fma(f2_pack(dv4.x, dv4.y), neg1, g01);
-        const uint64_t d23 = f2_fma(f2_pack(dv4.z, dv4.w), neg1, g23);
+        // dS' = P o (alpha dP' - D') on packed pairs
+        const uint64_t d01 = f2_fma(g01, ga2, f2_pack(dv4.x, dv4.y));
+        const uint64_t d23 = f2_fma(g23, ga2, f2_pack(dv4.z, dv4.w));
         const uint32_t pa = pk[e / 2], pb = pk[e / 2 + 1];
         float ds[4];
         f2_unpack(f2_mul(f2_pack(f16_lo(pa), f16_hi(pa)), d01), ds[0], ds[1]);
@@ -1075,7 +1228,7 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                                    : (static_cast<size_t>(bh) * a.N + key) * D;
         const uint32_t src = tmem + lane_off + (h ? C::COL_DK : C::COL_DV);
         float* dst = (h ? a.dk : a.dv) + orow;
-        const float mul = h ? a.scale : (DROP ? a.drop_scale : 1.f);
+        const float mul = h ? sc.dk : sc.dv;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t v[32];
@@ -1097,7 +1250,9 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     // ------------- dQ^T tile -> HBM (thread = one head-dim column) via TMA
     const int quarter = warp & 3;                    // TMEM lanes = d [32 quarter, 32 quarter + 32)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const float sc = a.scale;
+    const BwdScales bs = bwd_scales<D>(a);
+    const float sc = bs.dq1, sc2 = bs.dq2;
+    const bool two = sc2 != 1.f;
     float* stage = reinterpret_cast<float*>(smem + C::DQS_OFF + quarter * C::DQ_STAGE);
     const uint32_t stage_addr = base + C::DQS_OFF + quarter * C::DQ_STAGE;
     warp_arrive(bar(C::B_DSQ));                      // phase 0: no dQ^T(-1) to drain
@@ -1116,10 +1271,22 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       warp_arrive(bar(C::B_DSQ));                    // dQ^T(it) read: counts for phase it+1
       if (lane == 0) bulk_wait_read_all();           // previous reduce has read the staging box
       __syncwarp();
+      if (two) {                                     // factor outside one float's range
 #pragma unroll
-      for (int j = 0; j < 32; ++j) stage[j * 32 + lane] = __uint_as_float(v0[j]) * sc;
+        for (int j = 0; j < 32; ++j) {
+          v0[j] = __float_as_uint(__uint_as_float(v0[j]) * sc * sc2);
+          v1[j] = __float_as_uint(__uint_as_float(v1[j]) * sc * sc2);
+        }
 #pragma unroll
-      for (int j = 0; j < 32; ++j) stage[(32 + j) * 32 + lane] = __uint_as_float(v1[j]) * sc;
+        for (int j = 0; j < 32; ++j) stage[j * 32 + lane] = __uint_as_float(v0[j]);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) stage[(32 + j) * 32 + lane] = __uint_as_float(v1[j]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) stage[j * 32 + lane] = __uint_as_float(v0[j]) * sc;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) stage[(32 + j) * 32 + lane] = __uint_as_float(v1[j]) * sc;
+      }
       fence_async_smem();
       __syncwarp();
       if (lane == 0) {
@@ -1151,7 +1318,7 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
                        const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a,
                        cudaStream_t stream, cudaEvent_t ev_main_begin, cudaEvent_t ev_main_end) {
   using C = BwdCfg<D>;
-  static bool attr_set[64] = {};
+  static std::atomic<bool> attr_set[64];   // per device; racing first calls both set it
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
@@ -1177,6 +1344,7 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   const long long k8 = (a.cu_q ? a.n_k_elems : static_cast<long long>(a.B) * a.H * a.N * D) / 8;
   const long long cwant = (2 * q8 + 2 * k8 + 255) / 256;
   const int cblocks = static_cast<int>(cwant < 148 * 8 ? cwant : 148 * 8);
+  bwd_amax_kernel<<<kBwdAmaxBlocks, 256, 0, stream>>>(a, q8, k8);
   bwd_convert_kernel<<<cblocks, 256, 0, stream>>>(a, q8, k8);
   bwd_pre_kernel<D><<<pre_blocks, 256, 0, stream>>>(a);
   cudaError_t e = cudaGetLastError();

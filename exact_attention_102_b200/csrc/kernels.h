@@ -59,12 +59,18 @@ struct BwdArgs {
   float* dq;          // fp32 BHND (accumulated with reductions; zeroed by the pre kernel)
   float* dk;          // fp32 BHND
   float* dv;          // fp32 BHND
-  float* delta;       // fp32 [B][H][n_pad]: D_i = sum_c dO_ic O_ic (0 past N)
+  // -D_i = -sum_c dO_ic O_ic in the units of the scaled dS operand (see
+  // exps): fp32 [B][H][n_pad], 0 past N
+  float* delta;
   float* lse_log2;    // fp32 [B][H][n_pad]: L_i * log2(e) (+inf past N)
-  void* q16;          // fp16 BHND copies of q, k, v, dout (the tensor-core operands)
-  void* k16;
+  void* q16;          // fp16 copies of q, k, v, dout scaled by 2^exps[t] (the
+  void* k16;          // tensor-core operands)
   void* v16;
   void* do16;
+  // kBwdAmaxBlocks x 4 partial maxima of |q|, |k|, |v|, |dout| (bf16
+  // magnitude bits), reduced into the exponents e_q, e_k, e_v, e_do
+  uint32_t* amax_part;
+  int* exps;
   int B, H, N;
   int n_pad;          // N rounded up to a multiple of 128
   int causal;
@@ -89,6 +95,9 @@ struct BwdArgs {
   int head_group = 0;
 };
 
+// Blocks of the backward's amax pass (the length of BwdArgs.amax_part / 4).
+constexpr int kBwdAmaxBlocks = 148 * 4;
+
 // tdq: fp32 view of dq, [BH][N][d], box 32 x 64, no swizzle (reduce-add target
 // of the d = 128 main pass; unused for d = 64)
 // ev_main_begin / ev_main_end (may be null): recorded on `stream` right before
@@ -112,6 +121,8 @@ struct DecodeArgs {
   float* part_l;            // fp32 [S][Hq][max_splits]
   unsigned int* counter;    // work-item counter (zeroed by the launcher)
   int num_seqs, Hq, Hkv, max_blocks, max_ctx, max_splits, split_blocks;
+  int group;                // Hq / Hkv, 1 .. decode_max_group()
+  int d;                    // head dimension, 64 or 128
   float scale_log2;
   uint32_t* err;
 };

@@ -185,17 +185,6 @@ def test_guard_regions_and_workspace():
     _check((dq, dk, dv), _expected(x, True, oracle.round_bf16(o_ex)))
 
 
-def test_out_of_range_input_is_reported():
-    """A value beyond fp16's range cannot be a tensor-core operand of the
-    backward: the conversion records it and the host sees FA_ERR_UNSUPPORTED."""
-    x = synth.attention_inputs(1, 1, 64, 64, 23, device="cuda")
-    o, lse = fa.fa_fwd(x["q"], x["k"], x["v"], causal=False)
-    x["do"][0, 0, 5, 7] = 1e6
-    fa.fa_bwd(x["q"], x["k"], x["v"], o, lse, x["do"], causal=False)
-    assert fa.fa_last_device_error() == fa.FA_ERR_UNSUPPORTED
-    assert fa.fa_last_device_error() == fa.FA_OK
-
-
 def test_repeated_calls_match():
     """dQ is accumulated with floating-point reductions whose order varies from
     run to run; two runs agree to rounding, dK and dV exactly."""

@@ -1,0 +1,90 @@
+"""CPU pins of two readings about precision that the GPU tests rely on.
+
+Both use only the oracle and the seeded generators (no GPU, no library).
+
+1. FP8 workload (B=4, H=16, N=4096, d=128, 0.1% of entries x50, R from seed
+   2003). The pages quantise Q R, K R and V to e4m3 with one scale per block
+   ("FlashAttention系列优化", FlashAttentionV3, FP低精度; 91haoming.cn repost,
+   "FP8 低精度計算"). With outliers in nearly every 64-row block, that
+   quantisation alone, every later step exact, moves O by far more than the
+   5e-2 tolerance against unquantised attention. So the FP8 parity tests
+   compare the kernel with attention on the oracle's own e4m3 codes, and
+   the plain 5e-2 applies to inputs without outliers, where the same
+   quantisation stays inside it.
+
+2. Scores beyond fp32's resolution. Scaling Q and K together by 2^8 scales
+   the scores and L by 2^16 (|S|, |L| up to ~3e5), where one fp32 ulp is
+   2^-5 .. 2^-7. A backward rebuilds P = exp(S - L) from an fp32 score and
+   the fp32 L the forward stored; their rounding alone, every other step
+   exact, moves dV by more than 1e-2. So a parity test at that scale
+   measures fp32 itself, not the kernel; the backward range tests keep S
+   fixed (Q 2^a with K 2^-a) instead.
+"""
+
+import numpy as np
+import torch
+
+import oracle
+import synth
+
+
+def _f64(t):
+    return t.to(torch.float64).numpy()
+
+
+def _deq(src):
+    vals, scales = oracle.fp8_block_quantize(src)
+    return oracle.dequantize_blocks_e4m3(vals, scales.astype(np.float32))
+
+
+def test_fp8_block_quantisation_alone_exceeds_5e2_with_outliers():
+    x = synth.fp8_inputs(4, 16, 4096, 128, 1003)
+    r32 = synth.orthogonal_matrix(128, 2003).astype(np.float32).astype(np.float64)
+    rows = np.arange(0, 4096, 16)
+    for h in (0, 1):
+        q, k, v = (_f64(x[n][0, h]) for n in ("q", "k", "v"))
+        qd, kd, vd = _deq(q @ r32), _deq(k @ r32), _deq(v)
+        o_ex, _, _ = oracle.attention_rows(q[rows], rows, k, v, False)
+        o_q, _, _ = oracle.attention_rows(qd[rows], rows, kd, vd, False)
+        gap = np.abs(o_q - o_ex)
+        # a few rows move by whole units (measured: 15.2 and 26.7), the typical
+        # row by about 2e-2
+        assert gap.max() > 5.0
+        assert np.median(gap) < 5e-2
+        # the scores carry it: quantising Q and K alone gives the same gap,
+        # quantising V alone a much smaller one
+        o_qk, _, _ = oracle.attention_rows(qd[rows], rows, kd, v, False)
+        o_v, _, _ = oracle.attention_rows((q @ r32)[rows], rows, k @ r32, vd, False)
+        assert np.abs(o_qk - o_ex).max() > 5.0
+        assert np.abs(o_v - o_ex).max() < 0.2 * gap.max()
+
+
+def test_fp8_block_quantisation_within_5e2_without_outliers():
+    x = synth.attention_inputs(1, 4, 2048, 128, 1005, with_dout=False)
+    r32 = synth.orthogonal_matrix(128, 2003).astype(np.float32).astype(np.float64)
+    for h in range(4):
+        q, k, v = (_f64(x[n][0, h]) for n in ("q", "k", "v"))
+        o_ex, _ = oracle.attention_fwd(q, k, v)
+        o_q, _ = oracle.attention_fwd(_deq(q @ r32), _deq(k @ r32), _deq(v))
+        assert np.abs(o_q - o_ex).max() < 2.5e-2      # measured 1.4e-2
+
+
+def _dv_with_fp32_scores(q, k, do, lse):
+    """dV = P^T dO with P = exp(S / sqrt(d) - L) recomputed as a backward
+    does, in float64 except that S = Q K^T and L are fp32 values (every
+    product of bf16 values is exact in fp32; only the sums and the results
+    round)."""
+    s = (q.astype(np.float32) @ k.T.astype(np.float32)).astype(np.float64)
+    s *= np.float32(1.0 / np.sqrt(q.shape[1]))
+    p = np.exp(s - lse.astype(np.float32).astype(np.float64)[:, None])
+    return p.T @ do
+
+
+def test_scores_at_2_pow_16_are_beyond_fp32_resolution():
+    x = synth.attention_inputs(1, 1, 256, 128, 1002)
+    q, k, v, do = (_f64(x[n][0, 0]) for n in ("q", "k", "v", "do"))
+    for f, lo, hi in ((1.0, 0.0, 1e-5), (2.0 ** 8, 1e-2, np.inf)):
+        _, lse = oracle.attention_fwd(q * f, k * f, v)
+        dv = oracle.attention_bwd(q * f, k * f, v, do)[2]
+        err = np.abs(_dv_with_fp32_scores(q * f, k * f, do, lse) - dv).max()
+        assert lo <= err < hi, (f, err)     # measured 3.0e-7 and 0.19
