@@ -1,5 +1,6 @@
-// api.cu — the extern "C" boundary declared in include/fa.h: argument
-// checks, TMA tensor-map encoding, workspace carving and kernel launches.
+// api.cu — the extern "C" boundary declared in include/fa.h (and the
+// profiling hook of include/fa_profiling.h): argument checks, TMA tensor-map
+// encoding, workspace carving and kernel launches.
 // No computation of the method happens here; every step runs in the kernels.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -7,12 +8,16 @@
 #include <math.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "fa.h"
+#include "fa_profiling.h"
 #include "kernels.h"
 #include "prim.cuh"
 
 namespace fa {
 int decode_split_blocks();
+int decode_max_group();
 size_t decode_scratch_bytes();
 cudaError_t decode_scratch_ptr(void** out);
 }
@@ -25,15 +30,17 @@ __device__ uint32_t g_fa_error_word;
 constexpr int kMaxDevices = 64;
 
 uint32_t* error_word_ptr() {
-  static uint32_t* ptrs[kMaxDevices] = {};
+  static std::atomic<uint32_t*> ptrs[kMaxDevices];   // racing first calls store the same value
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  if (ptrs[dev] == nullptr) {
+  uint32_t* w = ptrs[dev].load(std::memory_order_acquire);
+  if (w == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_fa_error_word) != cudaSuccess) return nullptr;
-    ptrs[dev] = static_cast<uint32_t*>(p);
+    w = static_cast<uint32_t*>(p);
+    ptrs[dev].store(w, std::memory_order_release);
   }
-  return ptrs[dev];
+  return w;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -42,14 +49,17 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
+  static std::atomic<EncodeTiledFn> cached{nullptr};
+  EncodeTiledFn fn = cached.load(std::memory_order_acquire);
   if (fn == nullptr) {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult qr;
     if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
                                          &qr) == cudaSuccess &&
-        qr == cudaDriverEntryPointSuccess)
+        qr == cudaDriverEntryPointSuccess) {
       fn = reinterpret_cast<EncodeTiledFn>(p);
+      cached.store(fn, std::memory_order_release);
+    }
   }
   return fn;
 }
@@ -83,6 +93,11 @@ bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 const float kLog2e = 1.4426950408889634f;
+
+// Backward workspace part after D and L * log2(e): the amax partials of q, k,
+// v, dout (4 words per amax block) and the four operand exponents.
+constexpr size_t kStatsBytes =
+    (4 * sizeof(uint32_t) * fa::kBwdAmaxBlocks + 4 * sizeof(int) + 255) / 256 * 256;
 
 fa_status check_attn_dims(int B, int H, int N, int d) {
   if (B < 1 || H < 1 || N < 1 || d < 1) return FA_ERR_INVALID_ARG;
@@ -180,7 +195,7 @@ fa_status bwd_dense(const void* q, const void* k, const void* v, const void* o, 
   const size_t prow = static_cast<size_t>(bh) * n_pad;
   const size_t tsz = round256(static_cast<size_t>(bh) * N * d * 2);
   char* w = static_cast<char*>(workspace);
-  char* w16 = w + 2 * round256(prow * sizeof(float));
+  char* w16 = w + 2 * round256(prow * sizeof(float)) + kStatsBytes;
   void* q16 = w16;
   void* k16 = w16 + tsz;
   void* v16 = w16 + 2 * tsz;
@@ -213,6 +228,8 @@ fa_status bwd_dense(const void* q, const void* k, const void* v, const void* o, 
   a.delta = static_cast<float*>(workspace);
   a.lse_log2 = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                         round256(prow * sizeof(float)));
+  a.amax_part = reinterpret_cast<uint32_t*>(w + 2 * round256(prow * sizeof(float)));
+  a.exps = reinterpret_cast<int*>(a.amax_part + 4 * fa::kBwdAmaxBlocks);
   a.B = B;
   a.H = H;
   a.N = N;
@@ -417,7 +434,7 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   if (B < 1 || H < 1 || N < 1 || d < 1) return 0;
   const size_t rows = static_cast<size_t>(B) * H * ((static_cast<size_t>(N) + 127) / 128 * 128);
   const size_t elems = static_cast<size_t>(B) * H * N * d;
-  return 2 * round256(rows * sizeof(float)) + 4 * round256(elems * 2);
+  return 2 * round256(rows * sizeof(float)) + kStatsBytes + 4 * round256(elems * 2);
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -444,7 +461,8 @@ size_t fa_bwd_varlen_workspace_bytes(int batch, int max_seqlen_q, int total_q, i
   const size_t rows = static_cast<size_t>(batch) * H *
                       ((static_cast<size_t>(max_seqlen_q) + 127) / 128 * 128);
   const size_t nq = static_cast<size_t>(total_q) * H * d, nk = static_cast<size_t>(total_k) * Hkv * d;
-  return 2 * round256(rows * sizeof(float)) + 2 * round256(nq * 2) + 2 * round256(nk * 2);
+  return 2 * round256(rows * sizeof(float)) + kStatsBytes + 2 * round256(nq * 2) +
+         2 * round256(nk * 2);
 }
 
 fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
@@ -475,7 +493,7 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
   const size_t prow = static_cast<size_t>(batch) * H * n_pad;
   const size_t nq = static_cast<size_t>(total_q) * H * d, nk = static_cast<size_t>(total_k) * Hkv * d;
   char* w = static_cast<char*>(workspace);
-  char* w16 = w + 2 * round256(prow * sizeof(float));
+  char* w16 = w + 2 * round256(prow * sizeof(float)) + kStatsBytes;
   void* q16 = w16;
   void* k16 = w16 + round256(nq * 2);
   void* v16 = w16 + round256(nq * 2) + round256(nk * 2);
@@ -511,6 +529,8 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
   a.n_pad = static_cast<int>(n_pad);
   a.delta = static_cast<float*>(workspace);
   a.lse_log2 = reinterpret_cast<float*>(w + round256(prow * sizeof(float)));
+  a.amax_part = reinterpret_cast<uint32_t*>(w + 2 * round256(prow * sizeof(float)));
+  a.exps = reinterpret_cast<int*>(a.amax_part + 4 * fa::kBwdAmaxBlocks);
   a.B = batch;
   a.H = H;
   a.N = max_seqlen_q;
@@ -541,21 +561,41 @@ size_t paged_attn_decode_workspace_bytes(int num_seqs, int Hq, int d, int max_ct
   return round256(rows * d * sizeof(float)) + round256(rows * sizeof(float)) + 256;
 }
 
-fa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_cache,
-                            int num_phys_blocks, const int* block_table, int max_blocks_per_seq,
-                            const int* context_lens, void* o, float* lse, int num_seqs, int Hq,
-                            int Hkv, int d, int block_size, int max_ctx, void* workspace,
-                            size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+// The argument checks of the paged decode that do not involve the workspace
+// (shared by paged_attn_decode and paged_attn_decode_noalloc).
+fa_status decode_check(const void* q, const void* k_cache, const void* v_cache,
+                       int num_phys_blocks, const int* block_table, int max_blocks_per_seq,
+                       const int* context_lens, const void* o, const float* lse, int num_seqs,
+                       int Hq, int Hkv, int d, int block_size, int max_ctx) {
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || block_table == nullptr ||
       context_lens == nullptr || !aligned16(o) || (lse != nullptr && !aligned16(lse)))
     return FA_ERR_INVALID_ARG;
   if (num_seqs < 1 || Hq < 1 || Hkv < 1 || d < 1 || block_size < 1 || max_ctx < 1 ||
       max_blocks_per_seq < 1 || num_phys_blocks < 1 || Hq % Hkv != 0)
     return FA_ERR_INVALID_ARG;
-  if (d != 128 || block_size != 16 || Hq / Hkv != 4) return FA_ERR_UNSUPPORTED;
+  if ((d != 64 && d != 128) || block_size != 16 || Hq / Hkv > fa::decode_max_group())
+    return FA_ERR_UNSUPPORTED;
   if (static_cast<long long>(max_blocks_per_seq) * 16 < max_ctx) return FA_ERR_INVALID_ARG;
   if (static_cast<long long>(num_phys_blocks) * Hkv * block_size > (1ll << 31) - 1)
     return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+fa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                            int num_phys_blocks, const int* block_table, int max_blocks_per_seq,
+                            const int* context_lens, void* o, float* lse, int num_seqs, int Hq,
+                            int Hkv, int d, int block_size, int max_ctx, void* workspace,
+                            size_t ws_bytes, void* stream) {
+  fa_status st = decode_check(q, k_cache, v_cache, num_phys_blocks, block_table,
+                              max_blocks_per_seq, context_lens, o, lse, num_seqs, Hq, Hkv, d,
+                              block_size, max_ctx);
+  if (st != FA_OK) return st;
   const size_t need = paged_attn_decode_workspace_bytes(num_seqs, Hq, d, max_ctx);
   if (workspace == nullptr || !aligned16(workspace) || ws_bytes < need) return FA_ERR_WORKSPACE;
   uint32_t* err = error_word_ptr();
@@ -586,6 +626,8 @@ fa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_ca
   a.max_ctx = max_ctx;
   a.max_splits = max_splits;
   a.split_blocks = sb;
+  a.group = Hq / Hkv;
+  a.d = d;
   a.scale_log2 = kLog2e / sqrtf(static_cast<float>(d));
   a.err = err;
   // K / V caches as 2-D [blocks * Hkv * 16 rows][d] for 64-column, 16-row,
@@ -607,7 +649,10 @@ fa_status paged_attn_decode_noalloc(const void* q, const void* k_cache, const vo
                                     int block_size, int max_ctx, void* stream) {
   // Same checks as paged_attn_decode, then the library's own scratch array
   // stands in for the workspace (no allocation anywhere on this path).
-  if (num_seqs < 1 || Hq < 1 || d < 1 || max_ctx < 1) return FA_ERR_INVALID_ARG;
+  fa_status st = decode_check(q, k_cache, v_cache, num_phys_blocks, block_table,
+                              max_blocks_per_seq, context_lens, o, lse, num_seqs, Hq, Hkv, d,
+                              block_size, max_ctx);
+  if (st != FA_OK) return st;
   const size_t need = paged_attn_decode_workspace_bytes(num_seqs, Hq, d, max_ctx);
   if (need > fa::decode_scratch_bytes()) return FA_ERR_WORKSPACE;
   void* scratch = nullptr;

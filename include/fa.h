@@ -80,9 +80,11 @@ FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, fl
 /*
  * Bytes of device workspace fa_bwd needs: two fp32 per-row vectors over N
  * rounded up to a multiple of 128 rows — the row statistic D and L * log2(e)
- * (padded with 0 / +inf) — plus fp16 copies of q, k, v and dout (the
- * backward's tensor-core operands), each part rounded up to 256 bytes.
- * dq itself (fp32) serves as the dQ accumulator.
+ * (padded with 0 / +inf) — a small block of per-tensor statistics (the
+ * largest magnitudes of q, k, v, dout and the power-of-two exponents chosen
+ * from them), plus fp16 copies of q, k, v and dout (the backward's
+ * tensor-core operands), each part rounded up to 256 bytes. dq itself (fp32)
+ * serves as the dQ accumulator.
  */
 FA_API size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
 
@@ -102,11 +104,18 @@ FA_API size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
  * ("Flash Attention 再学习": backward recomputes S and P from the stored
  * statistics; 91haoming.cn repost, "并行化改進": backward is parallel over
  * column blocks with atomic adds for the shared gradient.)
- * Precision: the products run on fp16 tensor-core operands (exact copies of
- * the bf16 inputs; P and dS rounded to fp16), accumulation is fp32. Inputs
- * and the intermediate dS must satisfy |x| < 65504 (fp16 range); larger
- * values are recorded and reported by fa_last_device_error() as
- * FA_ERR_UNSUPPORTED.
+ * Precision: the products run on fp16 tensor-core operands with fp32
+ * accumulation. Each of q, k, v, dout is first multiplied by a power of two
+ * chosen from its largest magnitude a (so that it fits fp16's range); that
+ * scaling is exact, and the fp16 copy of an element x is exact whenever
+ * |x| >= 2^-30 a (smaller ones are off by less than 2^-38 a), so every
+ * finite bf16 input is accepted and results do not depend on the inputs'
+ * binade. The factors are undone in fp32. P and dS are rounded to fp16 (3
+ * more mantissa bits than bf16), dS after a power-of-two scale that keeps it
+ * below 2^15 when L is fa_fwd's L; a dS beyond fp16's range (an inconsistent
+ * L) is reported by fa_last_device_error() as FA_ERR_UNSUPPORTED. Inputs so
+ * large that scale * |q| * |k| leaves fp32's range give non-finite results,
+ * as in the forward.
  * Errors: as fa_fwd, plus FA_ERR_WORKSPACE when workspace is NULL or smaller
  * than required.
  */
@@ -288,10 +297,16 @@ FA_API size_t paged_attn_decode_workspace_bytes(int num_seqs, int Hq, int d, int
  *                  logical blocks map to physical blocks through a table;
  *                  several sequences may map to the same physical block).
  *                  Entries past ceil(ctx/block_size) are never read.
- *   context_lens : int32 [num_seqs], each in [1, max_ctx].
+ *   context_lens : int32 [num_seqs], each in [1, max_ctx]; a length outside
+ *                  that range is reported by fa_last_device_error() as
+ *                  FA_ERR_INVALID_ARG (the kernels then use it clamped into
+ *                  the range, so nothing outside the table or the workspace is
+ *                  read or written, and that sequence's output is undefined).
  *   o            : bf16 [num_seqs][Hq][d] output.
  *   lse          : fp32 [num_seqs][Hq] output, or NULL to skip it.
- *   Query head h reads KV head h / (Hq / Hkv). The query attends to all
+ *   Query head h reads KV head h / (Hq / Hkv), with 1 <= Hq / Hkv <= 8 (one
+ *   work item serves the query heads of one KV head, so each K/V byte is read
+ *   once per group). d is 64 or 128. The query attends to all
  *   context_lens[s] cached tokens (no mask).
  *   workspace    : >= paged_attn_decode_workspace_bytes(num_seqs, Hq, d,
  *                  max_ctx) bytes; max_ctx must bound every context length.
@@ -299,9 +314,10 @@ FA_API size_t paged_attn_decode_workspace_bytes(int num_seqs, int Hq, int d, int
  * partial (O_s, L_s); a second kernel merges them:
  * L = log sum_s exp(L_s), O = sum_s exp(L_s - L) O_s.
  * Errors: FA_ERR_INVALID_ARG (null/misaligned pointers, sizes < 1, Hq not a
- * multiple of Hkv); FA_ERR_UNSUPPORTED (d != 128, block_size != 16,
- * Hq/Hkv != 4); FA_ERR_WORKSPACE; FA_ERR_LAUNCH. Context lengths are read on
- * the device: a length outside [1, max_ctx] is clamped into that range.
+ * multiple of Hkv, a table narrower than max_ctx); FA_ERR_UNSUPPORTED (d not
+ * 64 or 128, block_size != 16, Hq/Hkv > 8); FA_ERR_WORKSPACE; FA_ERR_LAUNCH.
+ * Context lengths and table entries are read on the device and checked there
+ * (see context_lens and num_phys_blocks).
  */
 FA_API fa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_cache,
                             int num_phys_blocks, const int* block_table, int max_blocks_per_seq,
@@ -371,17 +387,6 @@ FA_API fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8,
                      void* stream);
 
 /*
- * fa_bwd_time_main_pass — for profiling. ev_begin and ev_end are cudaEvent_t
- * handles created by the caller (both non-NULL, or both NULL to cancel). The
- * next fa_bwd call made by this thread records ev_begin on its stream right
- * before its main pass (the kernel that runs the five products) and ev_end
- * right after it, so cudaEventElapsedTime gives that kernel's duration without
- * the conversion and D/L pre pass. The pair is used by one call only.
- * Errors: FA_ERR_INVALID_ARG when exactly one handle is NULL.
- */
-FA_API fa_status fa_bwd_time_main_pass(void* ev_begin, void* ev_end);
-
-/*
  * Paged KV-cache block pool ("FlashAttention系列优化", PagedAttention: blocks
  * allocated on demand as tokens arrive; sequences of parallel sampling share
  * physical blocks through their block tables; a reference count per block and
@@ -444,9 +449,15 @@ FA_API fa_status fa_kv_copy_blocks(void* k_cache, void* v_cache, int num_blocks,
  * device error word of the current device. Returns FA_OK when nothing was
  * recorded since the last call, FA_ERR_TIMEOUT when a bounded wait gave up,
  * FA_ERR_INVALID_ARG when a kernel met an out-of-range index in its inputs
- * (a block-table entry), FA_ERR_UNSUPPORTED when an input value was outside a
- * kernel's numeric range (fa_bwd: |x| >= 65504), or FA_ERR_LAUNCH when the
+ * (a block-table entry, a context length), FA_ERR_UNSUPPORTED when a value
+ * left a kernel's numeric range (fa_bwd: a dS beyond fp16's range, which
+ * only an L inconsistent with the scores produces), or FA_ERR_LAUNCH when the
  * synchronisation failed.
+ * The word is one per device and process, shared by every stream and host
+ * thread: the first error recorded by any kernel of the library on that
+ * device is kept until some caller reads it here, and reading clears it for
+ * all. Callers that run the library from several streams or threads at once
+ * should read it at a point where they know which of their calls ran.
  */
 FA_API fa_status fa_last_device_error(void* stream);
 

@@ -1,4 +1,4 @@
-"""The C-ABI library loads, exports every symbol include/fa.h declares, and
+"""The C-ABI library loads, exports every symbol include/*.h declare, and
 rejects bad arguments before touching a GPU (CPU-only; no compute calls)."""
 
 import ctypes
@@ -14,9 +14,14 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def _declared():
-    src = open(os.path.join(ROOT, "include", "fa.h")).read()
-    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return set(re.findall(r"\b(fa_\w+|paged_\w+)\s*\(", src))
+    """Every function the headers under include/ declare."""
+    names = set()
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(fa_\w+|paged_\w+)\s*\(", src))
+    return names
 
 
 def test_header_declares_binding_exports():
@@ -85,9 +90,9 @@ def test_decode_rejects_bad_arguments_without_gpu():
 
     assert call(q=_p(0)) == fa.FA_ERR_INVALID_ARG
     assert call(Hq=30) == fa.FA_ERR_INVALID_ARG            # not a multiple of Hkv
-    assert call(d=64) == fa.FA_ERR_UNSUPPORTED
+    assert call(d=96) == fa.FA_ERR_UNSUPPORTED
     assert call(bs=32) == fa.FA_ERR_UNSUPPORTED
-    assert call(Hq=16) == fa.FA_ERR_UNSUPPORTED             # group of 2
+    assert call(Hq=72) == fa.FA_ERR_UNSUPPORTED             # group of 9 (at most 8)
     assert call(maxb=100) == fa.FA_ERR_INVALID_ARG          # table shorter than max_ctx
     assert call(nphys=0) == fa.FA_ERR_INVALID_ARG
     assert call(ws=_p(0)) == fa.FA_ERR_WORKSPACE
@@ -117,6 +122,10 @@ def test_decode_noalloc_rejects_oversize_without_gpu():
                                        32768, None) == fa.FA_ERR_WORKSPACE
     assert L.paged_attn_decode_noalloc(g, g, g, 1000, g, 2048, g, g, g, 0, 32, 8, 128, 16,
                                        32768, None) == fa.FA_ERR_INVALID_ARG
+    # the shared argument checks come before the scratch-size check: an
+    # oversize request with an unsupported block size reports the block size
+    assert L.paged_attn_decode_noalloc(g, g, g, 1000, g, 2048, g, g, g, 64, 32, 8, 128, 32,
+                                       32768, None) == fa.FA_ERR_UNSUPPORTED
 
 
 def test_fwd_varlen_rejects_bad_arguments_without_a_gpu():

@@ -163,3 +163,79 @@ def test_many_items_per_cta():
     o_ref, l_ref = _oracle_for(seqs, lay, q, kc, vc)
     assert_bf16_close(f64(o), o_ref, O_TOL, "O")
     assert_lse_close(f64(lse), l_ref)
+
+
+# ------------------------------------------ query groups of 1..8, d 64 / 128
+GROUPS = [(8, 8), (16, 8), (32, 8), (64, 8), (24, 3), (7, 1)]   # groups 1, 2, 4, 8, 8, 7
+
+
+def _general(num_seqs, Hq, Hkv, d, lo, hi, seed, share_frac=0.10):
+    lay = synth.paged_decode_layout(num_seqs, BS, lo, hi, seed, share_frac=share_frac)
+    q, kc, vc = synth.paged_decode_tensors(num_seqs, Hq, Hkv, d, BS, lay["num_phys"], seed,
+                                           device="cuda")
+    return lay, q, kc, vc
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("Hq,Hkv", GROUPS)
+def test_query_groups_and_head_dims(Hq, Hkv, d):
+    """Hq / Hkv from 1 to 8 query heads per KV head and d in {64, 128}: every
+    head of 12 sequences with contexts U[1, 3000] against the oracle (which
+    maps query head h to KV head h // (Hq / Hkv))."""
+    lay, q, kc, vc = _general(12, Hq, Hkv, d, 1, 3000, 500 + Hq + d)
+    o, lse = _run(lay, q, kc, vc)
+    o_ref, l_ref = _oracle_for(list(range(12)), lay, q, kc, vc)
+    assert_bf16_close(f64(o), o_ref, O_TOL, "O")
+    assert_lse_close(f64(lse), l_ref)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (16, 8), (64, 8)])
+def test_block_table_bit_exact_groups(Hq, Hkv, d):
+    """The dominant-logit check of test_block_table_bit_exact for other query
+    groups and d = 64: query head hh of a group uses coordinate hh, so the G
+    heads of one KV head pick their own target tokens independently."""
+    S = 10
+    G = Hq // Hkv
+    lay = synth.paged_decode_layout(S, BS, 40, 2000, 95 + Hq + d, share_frac=0.0, extra_blocks=5)
+    q, kc, vc = synth.paged_decode_tensors(S, Hq, Hkv, d, BS, lay["num_phys"], 96, device="cuda")
+    lens, tab = lay["context_lens"], lay["block_table"]
+    rng = np.random.default_rng(97)
+    q.zero_()
+    kc.zero_()
+    targets = np.zeros((S, Hq), dtype=np.int64)
+    for s in range(S):
+        for h in range(Hq):
+            kvh, hh = h // G, h % G
+            t = int(rng.integers(0, lens[s]))
+            while any(targets[s, kvh * G + g] == t for g in range(hh)):
+                t = int(rng.integers(0, lens[s]))
+            targets[s, h] = t
+            q[s, h, hh] = 16.0
+            kc[tab[s, t // BS], kvh, t % BS, hh] = 2000.0
+    o, lse = _run(lay, q, kc, vc)
+    for s in range(S):
+        for h in range(Hq):
+            t = targets[s, h]
+            assert torch.equal(o[s, h], vc[tab[s, t // BS], h // G, t % BS]), (s, h, t)
+
+
+@pytest.mark.parametrize("bad", [0, -3, None])
+def test_context_length_outside_range_is_reported(bad):
+    """context_lens[s] must lie in [1, max_ctx]; a length outside it (None:
+    max_ctx + 1) is reported through the device error word
+    (FA_ERR_INVALID_ARG), never silently accepted. The reads stay inside the
+    table and the workspace."""
+    lay, q, kc, vc = _inputs(4, 100, 4000, 98)
+    max_ctx = lay["block_table"].shape[1] * BS
+    lens = lay["context_lens"].copy()
+    lens[2] = max_ctx + 1 if bad is None else bad
+    tab = torch.from_numpy(lay["block_table"]).cuda()
+    o, lse = fa.paged_attn_decode(q, kc, vc, tab, torch.from_numpy(lens).cuda(), max_ctx)
+    assert fa.fa_last_device_error() == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_last_device_error() == fa.FA_OK
+    # the other sequences are unaffected
+    keep = [0, 1, 3]
+    o_ref, l_ref = _oracle_for(keep, lay, q, kc, vc)
+    assert_bf16_close(f64(o[keep]), o_ref, O_TOL, "O")
+    assert_lse_close(f64(lse[keep]), l_ref)
