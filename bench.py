@@ -43,10 +43,15 @@ import synth  # noqa: E402
 
 WORKLOAD = dict(B=1, H=16, N=16384, d=128, causal=True)
 METRIC = "attention fwd+bwd TFLOP/s (bf16)"
-# DRAM bytes (read + write) of one d = 128 backward main-pass launch at WORKLOAD
-# (0.429 GB read + 0.369 GB written), from an ncu capture of that launch with the
-# current kernel; set to None whenever the kernel changes until captured again
-BWD_MAIN_TRAFFIC = 0.798e9
+# DRAM bytes (read + write) of one d = 128 backward main-pass launch at WORKLOAD,
+# from an ncu capture of that launch with the current kernel; None whenever the
+# kernel has changed since, until captured again
+BWD_MAIN_TRAFFIC = None
+# the same for one forward launch at WORKLOAD
+FWD_TRAFFIC = None
+# a timed region shorter than this runs at burst clocks: its kernels are held to
+# the burst peak; a longer one to the sustained (power-capped) peak
+SUSTAINED_REGION_MS = 1000.0
 
 
 def _peaks():
@@ -83,7 +88,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "50"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self._t = threading.Thread(target=self._read, daemon=True)
             self._t.start()
@@ -112,7 +117,7 @@ class ClockSampler:
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ts, line in self.lines:
-            if self.window and not (self.window[0] <= ts <= self.window[1] + 0.06):
+            if self.window and not (self.window[0] <= ts <= self.window[1] + 0.03):
                 continue
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
@@ -219,10 +224,10 @@ def run_fwd_bwd(fa, B, H, N, d, causal, steps, warmup, ws, seed, sampler_gpu=Non
     fwd_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
     bwd_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
     main_ms = float(np.mean([e[3].elapsed_time(e[4]) for e in evs]))
-    # launches per step: fa_fwd 1; fa_bwd 3 (fp16 conversion, D/L pre pass, main pass)
+    # launches per step: fa_fwd 1; fa_bwd 4 (amax, fp16 conversion, D/L pre pass, main pass)
     return {"total_ms": total_ms, "fwd_ms": _max_over_ranks(fwd_ms, ws),
             "bwd_ms": _max_over_ranks(bwd_ms, ws), "bwd_main_ms": _max_over_ranks(main_ms, ws),
-            "clocks": sampler.summary() if sampler else None, "launches_per_step": 4}
+            "clocks": sampler.summary() if sampler else None, "launches_per_step": 5}
 
 
 def run_e2e(fa, B, H, N, d, causal, steps, warmup, ws, seed):
@@ -599,8 +604,9 @@ def _config():
                         f"d={w['d']} causal bf16",
             "global_batch": w["B"], "seq_len": w["N"], "heads": w["H"], "head_dim": w["d"],
             "causal": w["causal"], "parallelism": "replicas (independent heads per GPU)",
-            "operands": "fwd bf16 x bf16 -> fp32; bwd fp16 x fp16 -> fp32 (exact copies of the "
-                        "bf16 inputs; P and dS rounded to fp16)",
+            "operands": "fwd bf16 x bf16 -> fp32; bwd fp16 x fp16 -> fp32 (each input tensor "
+                        "times a power of two from its largest magnitude, then fp16: exact for "
+                        "every element within 2^30 of that magnitude; P and dS rounded to fp16)",
             "l2": "operands larger than L2 (335 MB bf16 + 403 MB fp32), no flush"}
 
 
@@ -719,8 +725,14 @@ def main():
     e2e_val = ws * (f_fwd + f_bwd) / (e2e_ms / 1e3) / 1e12
 
     peak_t = peaks["bf16_tflops"]
-    # kernels timed inside a long run of back-to-back steps: the sustained peak
     peak_s = peaks.get("bf16_tflops_sustained") or peak_t
+    # a sub-second timed region runs at burst clocks (the burst peak applies);
+    # a seconds-long one settles under the power cap (the sustained peak)
+    sustained = r["total_ms"] >= SUSTAINED_REGION_MS
+    peak = peak_s if sustained else peak_t
+    peak_src = (f"{'measured' if peaks['source'] == 'measured' else 'fallback'} bf16 "
+                + ("sustained (cuBLAS, seconds-long loop)" if sustained else "burst (cuBLAS)")
+                + f": timed region {r['total_ms']:.0f} ms")
     bwd_t = f_bwd / (r["bwd_ms"] / 1e3) / 1e12
     fwd_t = f_fwd / (r["fwd_ms"] / 1e3) / 1e12
     main_t = f_bwd / (r["bwd_main_ms"] / 1e3) / 1e12
@@ -728,11 +740,17 @@ def main():
         kern, ach = "bwd_d128_kernel (fa_bwd main pass)", main_t
         traffic = BWD_MAIN_TRAFFIC
     else:
-        kern, ach, traffic = "fwd_kernel (fa_fwd)", fwd_t, None
-    roof = {"bound": "tensor", "kernel": kern, "achieved": ach, "peak": peak_s,
-            "unit": "TFLOP/s", "frac": ach / peak_s,
-            "peak_source": f"{peaks['source']} bf16 sustained (cuBLAS, seconds-long loop)",
-            "frac_of_burst_peak": ach / peak_t, "traffic": traffic}
+        kern, ach, traffic = "fwd_kernel (fa_fwd)", fwd_t, FWD_TRAFFIC
+    roof = {"bound": "tensor", "kernel": kern, "achieved": ach, "peak": peak,
+            "unit": "TFLOP/s", "frac": ach / peak, "peak_source": peak_src,
+            "traffic": traffic,
+            "forward": {"kernel": "fwd_kernel (fa_fwd)", "achieved": fwd_t, "frac": fwd_t / peak,
+                        "traffic": FWD_TRAFFIC},
+            "backward_whole": {"achieved": bwd_t, "frac": bwd_t / peak}}
+    clk = r["clocks"]
+    if clk and clk.get("sm_mhz") and clk.get("sm_max_mhz"):
+        # step time scaled to the maximum SM clock (time x median MHz / max MHz)
+        clk["ms_per_step_at_max_clock"] = ms * clk["sm_mhz"] / clk["sm_max_mhz"]
 
     parts = {}
     if not args.no_parts:
@@ -784,7 +802,7 @@ def main():
             p8 = 2.0 * peak_t
             parts["fp8_fwd"] = {"ms": f8["ms"], "TFLOP/s": t8, "roofline": {
                 "bound": "tensor", "achieved": t8, "peak": p8, "unit": "TFLOP/s", "frac": t8 / p8,
-                "peak_source": "measured bf16 burst x 2 (nominal fp8/bf16 ratio)"}}
+                "peak_source": f"{peaks['source']} bf16 burst x 2 (nominal fp8/bf16 ratio)"}}
         else:
             parts["fp8_fwd"] = f8
 
@@ -801,7 +819,7 @@ def main():
             "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": r["launches_per_step"] * args.steps,
-            "clocks": r["clocks"], "parts": parts,
+            "clocks": clk, "parts": parts,
         }
         print(json.dumps(line))
     if ws > 1:

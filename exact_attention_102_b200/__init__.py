@@ -136,9 +136,19 @@ def _check(fn, status):
         raise FAError(fn, status)
 
 
+def _current_device():
+    return torch.cuda.current_device()
+
+
 def _stream(stream=None):
+    """The cudaStream_t to launch on: the current stream of the current device,
+    or `stream`, which must belong to the current device."""
     if stream is None:
         stream = torch.cuda.current_stream()
+    dev = getattr(stream, "device", None)
+    if isinstance(dev, torch.device) and dev.type == "cuda" and dev.index != _current_device():
+        raise ValueError(f"stream belongs to cuda:{dev.index}, but the current device is "
+                         f"cuda:{_current_device()}")
     return ctypes.c_void_p(stream.cuda_stream)
 
 
@@ -146,9 +156,20 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
 
 
-def _require_cuda(t, name):
-    if not t.is_cuda:
+def _check_device(dev, name):
+    """The library launches on the current device and encodes raw pointers, so
+    every tensor it touches must live on that device (one tensor elsewhere
+    would be read through another GPU's address space)."""
+    if dev.type != "cuda":
         raise ValueError(f"{name} must be a CUDA tensor")
+    cur = _current_device()
+    if dev.index != cur:
+        raise ValueError(f"{name} is on cuda:{dev.index}, but the current device is cuda:{cur}; "
+                         "run the call under torch.cuda.device(...) of its tensors")
+
+
+def _require_cuda(t, name):
+    _check_device(t.device, name)
 
 
 def _need(t, name, dtype, ndim=None, shape=None):

@@ -26,6 +26,8 @@
 //                     O = (C / 256) * (sum P' v8) / l, l the fp32 sum of P.
 //                   V stays MN-major in shared memory (tcgen05 reads e4m3
 //                   operands in either major order), so no transpose is needed.
+#include <atomic>
+
 #include "prim.cuh"
 #include "kernels.h"
 
@@ -441,7 +443,7 @@ fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 }  // namespace
 
 cudaError_t launch_fp8_prepare(const Fp8PrepArgs& a, cudaStream_t stream) {
-  static bool attr_set[64] = {};
+  static std::atomic<bool> attr_set[64];   // per device; racing first calls both set it
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
@@ -457,7 +459,7 @@ cudaError_t launch_fp8_prepare(const Fp8PrepArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_fwd_fp8(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                            const Fp8FwdArgs& a, cudaStream_t stream) {
-  static bool attr_set[64] = {};
+  static std::atomic<bool> attr_set[64];   // per device; racing first calls both set it
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {

@@ -28,6 +28,8 @@
 // than 2^8 in exp2 units; until then exp2(x - m) <= 256, which fp32 and bf16
 // hold exactly as well as values <= 1. The final O / l and L = m + log l use
 // the same m, so the result is the same exact quantity.
+#include <atomic>
+
 #include "prim.cuh"
 #include "kernels.h"
 
@@ -584,7 +586,7 @@ template <int D>
 cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const FwdArgs& a, cudaStream_t stream) {
   using C = FwdCfg<D>;
-  static bool attr_set[64] = {};  // per device
+  static std::atomic<bool> attr_set[64];   // per device; racing first calls both set it
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {

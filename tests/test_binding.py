@@ -57,6 +57,43 @@ def test_device_check_is_real_without_the_fake():
         fa._need(_t((2, 2)), "x", BF)
 
 
+def test_tensors_on_another_device_are_rejected(monkeypatch):
+    """Every tensor must be on the current device (the library launches there
+    with raw pointers): one tensor on cuda:1 while cuda:0 is current, or a
+    stream of cuda:1, is a ValueError before any launch. CPU tensors stand in
+    for CUDA ones through a device map."""
+    f = _FakeLib()
+    monkeypatch.setattr(fa, "lib", lambda: f)
+    monkeypatch.setattr(fa, "_current_device", lambda: 0)
+    where = {}
+    monkeypatch.setattr(fa, "_require_cuda", lambda t, name: fa._check_device(where[id(t)], name))
+
+    def on(dev, t):
+        where[id(t)] = torch.device("cuda", dev)
+        return t
+
+    q = on(0, _t((1, 2, 64, 64)))
+    k, v = on(0, _t(q.shape)), on(1, _t(q.shape))
+    with pytest.raises(ValueError, match="cuda:1"):
+        fa.fa_fwd(q, k, v, o=on(0, _t(q.shape)), lse=on(0, _t((1, 2, 64), F32)), stream=S0)
+    assert f.calls == []
+    v0 = on(0, _t(q.shape))
+    with pytest.raises(ValueError, match="cuda:1"):
+        fa.fa_fwd(q, k, v0, o=on(1, _t(q.shape)), lse=on(0, _t((1, 2, 64), F32)), stream=S0)
+    assert f.calls == []
+
+    class _Stream1:
+        cuda_stream = 0
+        device = torch.device("cuda", 1)
+
+    with pytest.raises(ValueError, match="stream"):
+        fa.fa_fwd(q, k, v0, o=on(0, _t(q.shape)), lse=on(0, _t((1, 2, 64), F32)),
+                  stream=_Stream1())
+    assert f.calls == []
+    fa.fa_fwd(q, k, v0, o=on(0, _t(q.shape)), lse=on(0, _t((1, 2, 64), F32)), stream=S0)
+    assert len(f.calls) == 1
+
+
 # ------------------------------------------------------------------ forward
 def test_fwd_shapes(lib):
     q = _t((2, 3, 50, 64))

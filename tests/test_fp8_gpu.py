@@ -14,8 +14,13 @@ when every later step is exact (float64 emulation). So:
     to e4m3 for the P.V product: per element |dO| <= 5e-2 + 2^-4 (P |V|)
     (relative e4m3 rounding of each weight) plus half a bf16 ulp of the
     output; L is checked to 1e-3 relative;
+  * the chained fa_fp8_prepare -> fa_fwd_fp8 result is held to the same bound
+    against the oracle's quantised inputs, widened only by the first-order
+    effect of the one-step code differences (computed from the oracle);
   * without outliers the whole chain meets the plain 5e-2 against unquantised
-    attention; with them the gap is recorded, not asserted.
+    attention; with them the gap to unquantised attention is recorded (the
+    CPU pin in tests/test_precision_readings.py shows the quantisation alone
+    exceeds 5e-2 there).
 """
 
 import numpy as np
@@ -100,12 +105,51 @@ def test_prepare_matches_oracle_quantiser():
         assert np.all(np.abs(got - vals)[diff] <= step[diff] * 1.01)
 
 
+def _code_flip_bound(x, r32, deq, b, h, rows):
+    """How far O_rows can move when the GPU's fp32 rotation and fp32 scale put
+    an element on the other side of an e4m3 rounding boundary than the
+    oracle's float64 ones (the one-step code differences
+    test_prepare_matches_oracle_quantiser allows), or scale it by a slightly
+    different fp32 block scale. From the oracle alone, and worst-case (so
+    loose wherever an outlier sits near an ambiguous element):
+      * an element y = x / s is ambiguous when y - e and y + e round to
+        different codes, e = the fp32 rounding bound of the rotation
+        ((d + 2) 2^-24 sum_c |x_c R_c|) over s plus 2^-18 |y| for the scale;
+        its dequantised value can then move by the difference of those codes
+        times s, and every element by 2^-18 of itself (the scale);
+      * with |dS_ij| <= scale (sum_c dq_ic |k_jc| + |q_ic| dk_jc) <= delta_i
+        for every key j, each P_ij changes by a factor within e^(+-2 delta_i),
+        so O_i moves by at most (e^(2 delta_i) - 1) max_j |V_j - O_i| +
+        e^(2 delta_i) sum_j P_ij |dV_j| (max norms over the head dimension)."""
+    d = 128
+    moves = {}
+    for name, rot in (("q", True), ("k", True), ("v", False)):
+        src = f64(x[name][b, h])
+        xe = src @ r32 if rot else src
+        err_x = (d + 2) * 2.0 ** -24 * (np.abs(src) @ np.abs(r32)) if rot else 0.0 * xe
+        vals, scales = oracle.fp8_block_quantize(xe)
+        srow = np.repeat(scales, 64)[: xe.shape[0]][:, None]
+        y = xe / srow
+        e = err_x / srow + 2.0 ** -18 * np.abs(y)
+        flip = np.abs(oracle.quantize_e4m3(y + e) - oracle.quantize_e4m3(y - e)) * srow
+        moves[name] = flip + 2.0 ** -18 * np.abs(vals) * srow
+    qd, kd, vd = (deq[n][2][b, h] for n in ("q", "k", "v"))
+    o_ref, _, p = oracle.attention_rows(qd[rows], rows, kd, vd, False)
+    sc = 1.0 / np.sqrt(d)
+    delta = sc * (moves["q"][rows] @ np.abs(kd).T + np.abs(qd[rows]) @ moves["k"].T).max(-1)
+    spread = np.abs(vd).max() + np.abs(o_ref).max(-1)                   # >= max_j |V_j - O_i|
+    grow = np.exp(2.0 * delta)
+    return ((grow - 1.0) * spread)[:, None] + grow[:, None] * (p @ moves["v"])
+
+
 def test_fp8_config_sampled_rows(record_property):
     """B=4, H=16, N=4096, d=128, no mask, seed 1003: 0.1% outliers x50, R from
     seed 2003. fa_fwd_fp8 runs on the oracle's e4m3 codes and scales (so both
     sides see identical quantised inputs); sampled rows of 8 heads. The chained
-    fa_fp8_prepare -> fa_fwd_fp8 result is recorded against unquantised
-    attention."""
+    fa_fp8_prepare -> fa_fwd_fp8 result is held to the same bound against the
+    float64 forward on the oracle's dequantised inputs, plus the first-order
+    effect of the one-step code differences the GPU's fp32 rotation may make
+    (_code_flip_bound); its gap to unquantised attention is recorded."""
     B, H, N = 4, 16, 4096
     x = synth.fp8_inputs(B, H, N, 128, 1003, device="cuda")
     r32 = synth.orthogonal_matrix(128, 2003).astype(np.float32).astype(np.float64)
@@ -116,17 +160,32 @@ def test_fp8_config_sampled_rows(record_property):
     heads = ((0, 0), (0, 7), (1, 3), (1, 15), (2, 9), (3, 0), (3, 8), (3, 15))
     for b, h in heads:
         _check_rows(o, lse, deq, b, h, rows, False)
-    # chained path (the GPU's own prepare), recorded
+    # chained path (the GPU's own prepare)
     R = torch.from_numpy(r32).float().cuda()
-    o2, _ = fa.fa_fwd_fp8(*fa.fa_fp8_prepare(x["q"], x["k"], x["v"], R), causal=False)
+    o2, lse2 = fa.fa_fwd_fp8(*fa.fa_fp8_prepare(x["q"], x["k"], x["v"], R), causal=False)
     torch.cuda.synchronize()
-    gap = 0.0
+    assert fa.fa_last_device_error() == fa.FA_OK
+    gap, over = 0.0, 0
     for b, h in heads:
+        qd, kd, vd = (deq[n][2][b, h] for n in ("q", "k", "v"))
+        o_ref, l_ref, p = oracle.attention_rows(qd[rows], rows, kd, vd, False)
+        tight = FP8_TOL + 2.0 ** -4 * (p @ np.abs(vd)) + bf16_half_ulp(o_ref)
+        bound = tight + _code_flip_bound(x, r32, deq, b, h, rows)
+        got = f64(o2[b, h, rows])
+        assert np.all(np.isfinite(got))
+        diff = np.abs(got - o_ref)
+        assert np.all(diff <= bound), f"chained b{b} h{h}: worst excess {float((diff - bound).max()):.3e}"
+        over += int((diff > tight).any(-1).sum())
+        assert_lse_close(f64(lse2[b, h, rows]), l_ref, rtol=FP8_TOL)
         o_ex, _, _ = oracle.attention_rows(f64(x["q"][b, h, rows]), rows, f64(x["k"][b, h]),
                                            f64(x["v"][b, h]), False)
-        gap = max(gap, float(np.abs(f64(o2[b, h, rows]) - o_ex).max()))
+        gap = max(gap, float(np.abs(got - o_ex).max()))
+    # code differences are rare (a few elements per head): nearly every row
+    # must meet the tight bound itself
+    assert over <= 0.01 * len(heads) * len(rows), over
+    # the pages' block quantisation alone moves O by whole units on this input
+    # (tests/test_precision_readings.py); recorded, not a kernel property
     record_property("chained_max_abs_gap_to_unquantised_attention", gap)
-    assert np.isfinite(gap)
 
 
 @pytest.mark.parametrize("causal", [False, True])

@@ -10,12 +10,10 @@ through torch. It is collected last so that a failure here cannot hide any
 other test's result.
 """
 
-import numpy as np
 import pytest
 import torch
 
 import synth
-from helpers import O_TOL, assert_close_abs, assert_lse_close, f64
 
 pytestmark = pytest.mark.gpu
 
@@ -48,9 +46,11 @@ def test_noalloc_matches_workspace_entry_point_twice():
     torch.cuda.synchronize()
     assert torch.cuda.memory_allocated() == before
     assert fa.fa_last_device_error() == fa.FA_OK
+    # the same split and combine kernels run on the same splits: only the
+    # partials' home differs, so the results are identical bit for bit
     for (o_ref, l_ref), (o, lse) in zip(refs, outs):
-        assert_close_abs(f64(o), f64(o_ref), O_TOL, "O")
-        assert_lse_close(f64(lse), f64(l_ref))
+        assert torch.equal(o, o_ref)
+        assert torch.equal(lse, l_ref)
 
 
 def test_noalloc_rejects_requests_over_the_limit():
