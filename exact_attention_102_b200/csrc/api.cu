@@ -184,7 +184,6 @@ fa_status bwd_dense(const void* q, const void* k, const void* v, const void* o, 
     return FA_ERR_INVALID_ARG;
   fa_status st = check_attn_dims(B, H, N, d);
   if (st != FA_OK) return st;
-  if (drop != nullptr && d != 128) return FA_ERR_UNSUPPORTED;
   if (workspace == nullptr || !aligned16(workspace) ||
       ws_bytes < fa_bwd_workspace_bytes(B, H, N, d))
     return FA_ERR_WORKSPACE;
@@ -201,14 +200,17 @@ fa_status bwd_dense(const void* q, const void* k, const void* v, const void* o, 
   void* v16 = w16 + 2 * tsz;
   void* do16 = w16 + 3 * tsz;
   CUtensorMap tq, tk, tv, tdo, tdq;
-  // d = 128 steps over 64 queries at a time (64-row Q / dO boxes), d = 64 over 128
+  // d = 128 steps over 64 queries at a time (64-row Q / dO boxes), d = 64 over
+  // 128. The dQ reduce-add boxes: d = 128, 32 columns x 64 rows unswizzled
+  // (the drain writes a column per thread); d = 64, 32 columns x 32 rows with
+  // the 128-byte swizzle (a row per thread).
   const uint32_t qrows = d == 128 ? 64 : 128;
   if (!make_map(&tq, q16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, qrows) ||
       !make_map(&tk, k16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, 128) ||
       !make_map(&tv, v16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, 128) ||
       !make_map(&tdo, do16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, qrows) ||
-      !make_map(&tdq, dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, N, bh, 32, 64,
-                CU_TENSOR_MAP_SWIZZLE_NONE))
+      !make_map(&tdq, dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, N, bh, 32, d == 128 ? 64 : 32,
+                d == 128 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B))
     return FA_ERR_LAUNCH;
   fa::BwdArgs a;
   a.q16 = q16;
@@ -478,7 +480,7 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
   if (batch < 1 || H < 1 || Hkv < 1 || H % Hkv != 0 || max_seqlen_q < 1 || max_seqlen_k < 1 ||
       total_q < 1 || total_k < 1 || max_seqlen_q > total_q || max_seqlen_k > total_k)
     return FA_ERR_INVALID_ARG;
-  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   const long long nkb = (static_cast<long long>(max_seqlen_k) + 127) / 128;
   if (static_cast<long long>(batch) * Hkv * nkb > (1ll << 31) - 1 ||
       static_cast<long long>(total_q) * H * d > (1ll << 40) ||
@@ -498,19 +500,21 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
   void* k16 = w16 + round256(nq * 2);
   void* v16 = w16 + round256(nq * 2) + round256(nk * 2);
   void* do16 = w16 + round256(nq * 2) + 2 * round256(nk * 2);
-  // token-major views [T][heads][d]; Q / dO boxes of 64 tokens, K / V of 128,
-  // dQ reduce box 32 columns x 1 head x 64 tokens
+  // token-major views [T][heads][d]; Q / dO boxes of one step's tokens (64 for
+  // d = 128, 128 for d = 64), K / V of 128, dQ reduce boxes as in fa_bwd
   CUtensorMap tq, tk, tv, tdo, tdq;
+  const uint32_t qrows = d == 128 ? 64 : 128;
   if (!make_map(&tq, q16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, H, total_q, 64, 1,
-                CU_TENSOR_MAP_SWIZZLE_128B, 64) ||
+                CU_TENSOR_MAP_SWIZZLE_128B, qrows) ||
       !make_map(&tk, k16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, Hkv, total_k, 64, 1,
                 CU_TENSOR_MAP_SWIZZLE_128B, 128) ||
       !make_map(&tv, v16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, Hkv, total_k, 64, 1,
                 CU_TENSOR_MAP_SWIZZLE_128B, 128) ||
       !make_map(&tdo, do16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, H, total_q, 64, 1,
-                CU_TENSOR_MAP_SWIZZLE_128B, 64) ||
+                CU_TENSOR_MAP_SWIZZLE_128B, qrows) ||
       !make_map(&tdq, dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, H, total_q, 32, 1,
-                CU_TENSOR_MAP_SWIZZLE_NONE, 64))
+                d == 128 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+                d == 128 ? 64 : 32))
     return FA_ERR_LAUNCH;
   fa::BwdArgs a;
   a.q16 = q16;
@@ -548,8 +552,9 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
   a.n_k_elems = static_cast<long long>(nk);
   cudaEvent_t eb = g_bwd_ev_begin, ee = g_bwd_ev_end;
   g_bwd_ev_begin = g_bwd_ev_end = nullptr;
-  cudaError_t e = fa::launch_bwd<128>(tq, tk, tv, tdo, tdq, a, static_cast<cudaStream_t>(stream),
-                                      eb, ee);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = (d == 128) ? fa::launch_bwd<128>(tq, tk, tv, tdo, tdq, a, s, eb, ee)
+                             : fa::launch_bwd<64>(tq, tk, tv, tdo, tdq, a, s, eb, ee);
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 

@@ -25,24 +25,19 @@
 // scores; a dS beyond fp16's range (possible only with an inconsistent L) is
 // recorded as FA_ERR_UNSUPPORTED.
 //
-// B200 mapping (one CTA per (batch*head, key block), 512 threads):
-//   warp 0       TMA producer: K_j, V_j once; Q_i and dO_i per row block
-//                through two-stage rings.
-//   warp 1       TMEM allocation; lane 0 issues all tcgen05.mma:
-//                S^T = K_j Q_i^T and dP^T = V_j dO_i^T (smem x smem),
-//                dV += P^T dO_i (P^T from TMEM), dK += dS^T Q_i and
-//                dQ_i = dS K_j (dS from shared memory, read K-major for dK
-//                and MN-major for dQ).
-//   warps 4..7   thread = key row (TMEM lane): P^T from S^T and L, packed to
-//                fp16 in TMEM (for dV and for the dS group).
-//   warps 8..11  thread = key row: copies P^T(i) out of TMEM (so S^T(i+1) can
-//                start), then dS^T = P^T o (dP^T - D) into shared memory in the
-//                128-byte-swizzled layout the MMA reads; at the end, dK and dV
-//                rows to HBM. P of block i+1 and dS of block i overlap.
-//   warps 12..15 thread = query row of the dQ tile: reads the fp32 dQ tile
-//                from TMEM and adds it to dQ in HBM with vector reductions.
-// TMEM (512 columns): S^T / P^T [0,128), dP^T [128,256) (reused for the dQ
-// tile once dS is out), dV [256, 256+D), dK [256+D, 256+2D).
+// B200 mapping (one CTA per (batch*head, 128-key block), 512 threads; the
+// kernel is bwd_ts_kernel below, templated on d = 64 / 128):
+//   warp 0       TMA producer: K_j, V_j once; Q_i, dO_i, L_i, D_i per step of
+//                64 (d = 128) or 128 (d = 64) queries through a ring.
+//   warp 1       TMEM allocation; lane 0 issues every tcgen05.mma: S^T, dP^T,
+//                dV, dK and dQ (see "main pass on TMEM operands").
+//   warps 4..11  thread = key row (TMEM lane), two warps per lane quarter,
+//                one per half of the step's queries: P^T, then dS^T, each
+//                written back into TMEM as the A operand of dV / dK, dS^T also
+//                into shared memory for the dQ product; at the end the dK and
+//                dV rows.
+//   warps 12..15 read the step's dQ tile out of TMEM and add it to dQ in HBM
+//                with TMA tensor reduce-adds.
 #include <climits>
 #include <type_traits>
 
@@ -55,48 +50,11 @@ namespace fa {
 
 namespace {
 
-template <int D>
-struct BwdCfg {
-  static constexpr int BK = 128;                 // keys per CTA
-  static constexpr int BQ = 128;                 // queries per iteration
-  static constexpr int TILE = 128 * D * 2;       // one 128-row bf16 tile of Q/K/V/dO
-  static constexpr int CHUNK = 128 * 128;        // one 64-column (128 B) chunk of a tile
-  static constexpr int NCHUNK = D / 64;
-  static constexpr int DS_BYTES = 128 * 128 * 2; // dS^T tile, bf16 [key][query]
-  static constexpr int K_OFF = 0;
-  static constexpr int V_OFF = K_OFF + TILE;
-  static constexpr int Q_OFF = V_OFF + TILE;           // 2 stages
-  static constexpr int DO_OFF = Q_OFF + 2 * TILE;      // 2 stages
-  static constexpr int DS_OFF = DO_OFF + 2 * TILE;
-  static constexpr int L_OFF = DS_OFF + DS_BYTES;       // 2 stages x 128 fp32: L * log2(e)
-  static constexpr int DL_OFF = L_OFF + 2 * 512;        // 2 stages x 128 fp32: D
-  static constexpr int BAR_OFF = DL_OFF + 2 * 512;
-  // barriers
-  static constexpr int B_KV = 0;
-  static constexpr int B_QF = 1, B_QE = 3, B_DF = 5, B_DE = 7;   // [2] each
-  static constexpr int B_ST = 9, B_DPT = 10, B_P = 11, B_DV = 12, B_DS = 13, B_DSFREE = 14;
-  static constexpr int B_DQ = 15, B_DQFREE = 16, B_END = 17, B_DRAIN = 18, B_PR = 19;
-  static constexpr int NBAR = 20;
-  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
-  // d = 128 leaves no room for alignment slack: the dynamic shared memory
-  // base must already be 1024-byte aligned (checked at run time)
-  static constexpr int SMEM_BYTES = MISC_OFF + 16;
-  static constexpr uint32_t COL_ST = 0, COL_DPT = 128, COL_DV = 256, COL_DK = 256 + D;
-  static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr int THREADS = 512;
-};
-
 enum : uint32_t {
   kSiteKV = 0x31, kSiteQE = 0x32, kSiteDE = 0x33, kSiteQF = 0x34, kSiteDF = 0x35, kSiteP = 0x36,
   kSiteDV = 0x37, kSiteDS = 0x38, kSiteDQF = 0x39, kSiteST = 0x3a, kSiteDPT = 0x3b,
   kSiteDSF = 0x3c, kSiteDQ = 0x3d, kSiteEnd = 0x3e, kSiteDrain = 0x3f, kSitePR = 0x40
 };
-
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
-}
 
 // ------------------------------------------------------ operand scaling
 // The tensor-core operands of the backward are fp16 (P and dS keep 3 more
@@ -322,450 +280,90 @@ __device__ __forceinline__ BwdScales bwd_scales(const BwdArgs& a) {
   return s;
 }
 
-// --------------------------------------------------------------- main pass
-template <int D>
-__global__ void __launch_bounds__(512, 1)
-bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                BwdArgs a) {
-  using C = BwdCfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t base = smem_u32(smem_raw);
-  uint8_t* smem = smem_raw;
-  if (base & 1023u) {  // 128-byte-swizzled tiles need 1024-byte aligned bases
-    if (threadIdx.x == 0) atomicCAS(a.err, 0u, kErrBadIndex + 0x30);
-    return;
-  }
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int BH = a.B * a.H;
-  const int kb = static_cast<int>(blockIdx.x) / BH;   // key block (longest work first)
-  const int bh = static_cast<int>(blockIdx.x) % BH;
-  const int nq = (a.N + C::BQ - 1) / C::BQ;
-  const int i0 = a.causal ? kb : 0;                    // first query block that sees these keys
-  const int n_it = nq - i0;
-
-  auto bar = [&](int i) -> uint32_t { return base + C::BAR_OFF + 8 * i; };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
-
-  if (threadIdx.x == 0) {
-    mbar_init(bar(C::B_KV), 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(C::B_QF + s), 1);
-      mbar_init(bar(C::B_QE + s), 1);
-      mbar_init(bar(C::B_DF + s), 1);
-      mbar_init(bar(C::B_DE + s), 1);
-    }
-    mbar_init(bar(C::B_ST), 1);
-    mbar_init(bar(C::B_DPT), 1);
-    mbar_init(bar(C::B_P), 4);      // one arrival per warp
-    mbar_init(bar(C::B_PR), 4);
-    mbar_init(bar(C::B_DV), 1);
-    mbar_init(bar(C::B_DS), 4);
-    mbar_init(bar(C::B_DSFREE), 1);
-    mbar_init(bar(C::B_DQ), 1);
-    mbar_init(bar(C::B_DQFREE), 4);
-    mbar_init(bar(C::B_END), 1);
-    mbar_init(bar(C::B_DRAIN), 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      tma_prefetch_desc(&tmDO);
-      mbar_arrive_expect_tx(bar(C::B_KV), 2 * C::TILE);
-      for (int c = 0; c < C::NCHUNK; ++c) {
-        tma_load_3d(base + C::K_OFF + c * C::CHUNK, &tmK, bar(C::B_KV), c * 64, kb * C::BK, bh);
-        tma_load_3d(base + C::V_OFF + c * C::CHUNK, &tmV, bar(C::B_KV), c * 64, kb * C::BK, bh);
-      }
-      int issued = 0;
-      for (int it = 0; it < n_it; ++it) {
-        const int s = it & 1;
-        const uint32_t ph = ((it >> 1) & 1) ^ 1;
-        const int row = (i0 + it) * C::BQ;
-        const size_t prow = static_cast<size_t>(bh) * a.n_pad + row;   // 512 B aligned
-        if (!mbar_wait(bar(C::B_QE + s), ph, a.err, kSiteQE, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(C::B_QF + s), C::TILE + 512);
-        for (int c = 0; c < C::NCHUNK; ++c)
-          tma_load_3d(base + C::Q_OFF + s * C::TILE + c * C::CHUNK, &tmQ, bar(C::B_QF + s),
-                      c * 64, row, bh);
-        bulk_load(base + C::L_OFF + s * 512, a.lse_log2 + prow, 512, bar(C::B_QF + s));
-        if (!mbar_wait(bar(C::B_DE + s), ph, a.err, kSiteDE, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(C::B_DF + s), C::TILE + 512);
-        for (int c = 0; c < C::NCHUNK; ++c)
-          tma_load_3d(base + C::DO_OFF + s * C::TILE + c * C::CHUNK, &tmDO, bar(C::B_DF + s),
-                      c * 64, row, bh);
-        bulk_load(base + C::DL_OFF + s * 512, a.delta + prow, 512, bar(C::B_DF + s));
-        issued = it + 1;
-      }
-      for (int it = max(0, issued - 2); it < issued; ++it) {
-        mbar_wait(bar(C::B_QF + (it & 1)), (it >> 1) & 1, a.err, kSiteDrain, nullptr, 200000000ull);
-        mbar_wait(bar(C::B_DF + (it & 1)), (it >> 1) & 1, a.err, kSiteDrain, nullptr, 200000000ull);
-      }
-      mbar_wait(bar(C::B_KV), 0, a.err, kSiteDrain, nullptr, 200000000ull);
-    }
-  } else if (warp == 1) {
-    // ----------------------------------------------------------- MMA issue
-    if (lane == 0) {
-      // fp16 x fp16 -> fp32 (format 0 = f16)
-      constexpr uint32_t idSS = idesc_f16(128, C::BQ, 0, 0, 0);   // S^T, dP^T
-      constexpr uint32_t idKM = idesc_f16(128, D, 0, 0, 1);        // dV (A tmem), dK: B MN-major
-      constexpr uint32_t idQ = idesc_f16(128, D, 0, 1, 1);         // dQ: A and B MN-major
-      const uint32_t kbase = base + C::K_OFF, vbase = base + C::V_OFF, dsb = base + C::DS_OFF;
-      bool ok = mbar_wait(bar(C::B_KV), 0, a.err, kSiteKV, abort_flag);
-      // S^T(it) = K Q_it^T ; dP^T(it) = V dO_it^T
-      auto issue_st = [&](int it) -> bool {
-        const int s = it & 1;
-        if (!mbar_wait(bar(C::B_QF + s), (it >> 1) & 1, a.err, kSiteQF, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t qb = base + C::Q_OFF + s * C::TILE;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          umma_f16_ss(tmem + C::COL_ST, smem_desc_sw128(kbase + off, 16, 1024),
-                      smem_desc_sw128(qb + off, 16, 1024), idSS, kk > 0);
-        }
-        umma_commit(bar(C::B_ST));
-        return true;
-      };
-      auto issue_dpt = [&](int it) -> bool {
-        const int s = it & 1;
-        if (!mbar_wait(bar(C::B_DF + s), (it >> 1) & 1, a.err, kSiteDF, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t gb = base + C::DO_OFF + s * C::TILE;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          umma_f16_ss(tmem + C::COL_DPT, smem_desc_sw128(vbase + off, 16, 1024),
-                      smem_desc_sw128(gb + off, 16, 1024), idSS, kk > 0);
-        }
-        umma_commit(bar(C::B_DPT));
-        return true;
-      };
-      if (ok) ok = issue_st(0) && issue_dpt(0);
-      for (int it = 0; it < n_it && ok; ++it) {
-        const int s = it & 1;
-        const uint32_t qb = base + C::Q_OFF + s * C::TILE;
-        const uint32_t gb = base + C::DO_OFF + s * C::TILE;
-        // dV += P^T dO_it  (P^T bf16 in TMEM columns [0,64))
-        ok = mbar_wait(bar(C::B_P), it & 1, a.err, kSiteP, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < C::BQ / 16; ++kk)
-          umma_f16_ts(tmem + C::COL_DV, tmem + C::COL_ST + kk * 8,
-                      smem_desc_sw128(gb + kk * 2048, C::CHUNK, 1024), idKM,
-                      (it > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(bar(C::B_DV));
-        if (it + 1 < n_it) {
-          // S^T(it+1) overwrites P^T(it): wait until dV(it) and the dS group
-          // have both read it
-          ok = mbar_wait(bar(C::B_DV), it & 1, a.err, kSiteDV, abort_flag) &&
-               mbar_wait(bar(C::B_PR), it & 1, a.err, kSitePR, abort_flag);
-          if (!ok) break;
-          ok = issue_st(it + 1);
-          if (!ok) break;
-        }
-        // dK += dS^T Q_it ; dQ_it = dS K   (dS^T bf16 [key][query] in smem)
-        ok = mbar_wait(bar(C::B_DS), it & 1, a.err, kSiteDS, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < C::BQ / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          umma_f16_ss(tmem + C::COL_DK, smem_desc_sw128(dsb + off, 16, 1024),
-                      smem_desc_sw128(qb + kk * 2048, C::CHUNK, 1024), idKM,
-                      (it > 0 || kk > 0) ? 1u : 0u);
-        }
-#pragma unroll
-        for (int kk = 0; kk < C::BK / 16; ++kk)
-          umma_f16_ss(tmem + C::COL_DPT, smem_desc_sw128(dsb + kk * 2048, C::CHUNK, 1024),
-                      smem_desc_sw128(kbase + kk * 2048, C::CHUNK, 1024), idQ, kk > 0 ? 1u : 0u);
-        umma_commit(bar(C::B_DQ));
-        umma_commit(bar(C::B_DSFREE));
-        umma_commit(bar(C::B_QE + s));   // Q_it and its L: S^T, P and dK done
-        umma_commit(bar(C::B_DE + s));   // dO_it and its D: dP^T, dV and dS done
-        if (it + 1 < n_it) {
-          // dP^T(it+1) overwrites the dQ tile: wait until it has been read out
-          ok = mbar_wait(bar(C::B_DQFREE), it & 1, a.err, kSiteDQF, abort_flag);
-          if (!ok) break;
-          ok = issue_dpt(it + 1);
-          if (!ok) break;
-        }
-      }
-      umma_commit(bar(C::B_END));
-      umma_commit(bar(C::B_DRAIN));
-      mbar_wait(bar(C::B_DRAIN), 0, a.err, kSiteDrain, nullptr, 200000000ull);
-    }
-  } else if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------ P^T (thread = key row)
-    const int r = (warp & 3) * 32 + lane;            // key within the block == TMEM lane
-    const int key = kb * C::BK + r;
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t st_addr = tmem + lane_off + C::COL_ST;
-    const float sl2 = bwd_scales<D>(a).c_s;
-    for (int it = 0; it < n_it; ++it) {
-      const int s = it & 1;
-      const int q0 = (i0 + it) * C::BQ;
-      const float* Ls = reinterpret_cast<const float*>(smem + C::L_OFF + s * 512);
-      // queries >= N have L = +inf (P = 0); the causal diagonal block and keys
-      // >= N need an explicit mask
-      const bool need_mask = (a.causal && key > q0) || key >= a.N;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(C::B_ST), it & 1, a.err, kSiteST, abort_flag)))
-        break;
-      tc_fence_after();
-      // queries [64*half, 64*half+64) -> fp16 pairs in TMEM columns [32*half, 32*half+32)
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t sr0[32], sr1[32];
-        tmem_ld32(st_addr + half * 64, sr0);
-        tmem_ld32(st_addr + half * 64 + 32, sr1);
-        tmem_ld_wait();
-        uint32_t pk[32];
-#pragma unroll
-        for (int e = 0; e < 64; e += 4) {
-          const float4 lv = *reinterpret_cast<const float4*>(Ls + half * 64 + e);
-          const float L[4] = {lv.x, lv.y, lv.z, lv.w};
-          float p[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const uint32_t sv = (e + u) < 32 ? sr0[e + u] : sr1[e + u - 32];
-            // P = exp(scale*s - L) = exp2(s*scale*log2e - L*log2e)
-            p[u] = ex2_approx(fmaf(__uint_as_float(sv), sl2, -L[u]));
-            if (need_mask && ((a.causal && key > q0 + half * 64 + e + u) || key >= a.N)) p[u] = 0.f;
-          }
-          pk[e / 2] = pack_f16x2(p[0], p[1]);
-          pk[e / 2 + 1] = pack_f16x2(p[2], p[3]);
-        }
-        tmem_st32(st_addr + half * 32, pk);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      warp_arrive(bar(C::B_P));
-    }
-    tc_fence_before();
-  } else if (warp >= 8 && warp < 12) {
-    // ---------------------------- dS^T = P^T o (dP^T - D) (thread = key row)
-    const int r = (warp & 3) * 32 + lane;
-    const int key = kb * C::BK + r;
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t st_addr = tmem + lane_off + C::COL_ST;
-    const uint32_t dpt_addr = tmem + lane_off + C::COL_DPT;
-    uint8_t* ds_row = smem + C::DS_OFF + r * 128;    // row r of each 64-query chunk
-    const float alpha = __int_as_float((127 - ds_shift(D)) << 23);
-    bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
-      const int s = it & 1;
-      const float* Ds = reinterpret_cast<const float*>(smem + C::DL_OFF + s * 512);
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_P), it & 1, a.err, kSiteP, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t pk0[32], pk1[32];                     // P^T(it), fp16 pairs, queries 0..127
-      tmem_ld32(st_addr, pk0);
-      tmem_ld32(st_addr + 32, pk1);
-      tmem_ld_wait();
-      tc_fence_before();
-      warp_arrive(bar(C::B_PR));                     // S^T(it+1) may now overwrite P^T(it)
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_DPT), it & 1, a.err, kSiteDPT, abort_flag));
-      if (!ok) break;
-      if (it > 0) {  // dS buffer reusable once dK(it-1) and dQ(it-1) have read it
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait(bar(C::B_DSFREE), (it - 1) & 1, a.err, kSiteDSF, abort_flag));
-        if (!ok) break;
-      }
-      tc_fence_after();
-      float ds_max = 0.f;
-#define PK(i) (((i) < 32) ? pk0[(i)] : pk1[(i)-32])
-#pragma unroll
-      for (int g = 0; g < 8; ++g) {                  // 16 queries at a time
-        uint32_t dr[16];
-        tmem_ld16(dpt_addr + g * 16, dr);
-        tmem_ld_wait();
-        uint32_t w[8];
-#pragma unroll
-        for (int e = 0; e < 16; e += 4) {
-          const float4 dv4 = *reinterpret_cast<const float4*>(Ds + g * 16 + e);
-          const float Dv[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
-          float ds[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int q = g * 16 + e + u;
-            const uint32_t pp = PK(q >> 1);
-            const float pv = (q & 1) ? f16_hi(pp) : f16_lo(pp);
-            ds[u] = pv * fmaf(__uint_as_float(dr[e + u]), alpha, Dv[u]);   // Dv = -D'
-          }
-          ds_max = fmaxf(ds_max, fmaxf(fmaxf(fabsf(ds[0]), fabsf(ds[1])),
-                                       fmaxf(fabsf(ds[2]), fabsf(ds[3]))));
-          w[e / 2] = pack_f16x2(ds[0], ds[1]);
-          w[e / 2 + 1] = pack_f16x2(ds[2], ds[3]);
-        }
-        // queries g*16 .. g*16+15 = chunk g/4, 16-byte units (g%4)*2 and +1 of the
-        // 128-byte row, XOR-swizzled with (key row % 8) like a TMA SWIZZLE_128B tile
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int unit = (g & 3) * 2 + u;
-          uint4* dst = reinterpret_cast<uint4*>(ds_row + (g >> 2) * C::CHUNK +
-                                                ((unit ^ (r & 7)) << 4));
-          *dst = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
-        }
-      }
-#undef PK
-      if (!(ds_max < 65504.f)) atomicCAS(a.err, 0u, kErrRange + 2);
-      fence_async_smem();   // generic-proxy smem writes -> visible to the MMA
-      tc_fence_before();
-      warp_arrive(bar(C::B_DS));
-    }
-    // ---- epilogue: dV and dK rows (thread = key) to HBM
-    if (ok) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_END), 0, a.err, kSiteEnd, abort_flag));
-      if (ok) {
-        tc_fence_after();
-        const size_t orow = (static_cast<size_t>(bh) * a.N + key) * D;
-#pragma unroll
-        for (int which = 0; which < 2; ++which) {
-          const uint32_t src = tmem + lane_off + (which ? C::COL_DK : C::COL_DV);
-          float* dst = (which ? a.dk : a.dv) + orow;
-          const BwdScales sc = bwd_scales<D>(a);
-          const float mul = which ? sc.dk : sc.dv;
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t v[32];
-            tmem_ld32(src + c * 32, v);
-            tmem_ld_wait();
-            if (key < a.N) {
-              float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
-#pragma unroll
-              for (int e = 0; e < 8; ++e)
-                d4[e] = make_float4(__uint_as_float(v[4 * e]) * mul, __uint_as_float(v[4 * e + 1]) * mul,
-                                    __uint_as_float(v[4 * e + 2]) * mul,
-                                    __uint_as_float(v[4 * e + 3]) * mul);
-            }
-          }
-        }
-      }
-    }
-    tc_fence_before();
-  } else if (warp >= 12) {
-    // ---------------------------------------- dQ tile -> HBM (thread = query)
-    const int r = (warp & 3) * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t src = tmem + lane_off + C::COL_DPT;
-    const BwdScales bs = bwd_scales<D>(a);
-    const float sc = bs.dq1, sc2 = bs.dq2;
-    const bool two = sc2 != 1.f;
-    auto f = [&](uint32_t v) { const float t = __uint_as_float(v) * sc; return two ? t * sc2 : t; };
-    for (int it = 0; it < n_it; ++it) {
-      const int q = (i0 + it) * C::BQ + r;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(C::B_DQ), it & 1, a.err, kSiteDQ, abort_flag)))
-        break;
-      tc_fence_after();
-      float* dst = a.dq + (static_cast<size_t>(bh) * a.N + q) * D;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(src + c * 32, v);
-        tmem_ld_wait();
-        if (q < a.N) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            red_add_v4(dst + c * 32 + 4 * e, f(v[4 * e]), f(v[4 * e + 1]), f(v[4 * e + 2]),
-                       f(v[4 * e + 3]));
-        }
-      }
-      tc_fence_before();
-      warp_arrive(bar(C::B_DQFREE));
-    }
-    tc_fence_before();
-  }
-
-  __syncthreads();
-  if (warp == 1) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
-  }
-}
-
-// ------------------------------------------------- main pass, d = 128 -----
-// Same method, tiled for d = 128 around what the tensor core does fastest: an
-// MMA whose A operand sits in TMEM runs at the full rate for N = 128, one whose
-// A operand is read from shared memory costs about twice as long for N <= 128.
-// Steps of 64 queries; every operand that can live in TMEM does:
+// --------------------------------- main pass on TMEM operands, d = 64 / 128
+// Same method, tiled around what the tensor core does fastest: an MMA whose A
+// operand sits in TMEM runs at the full rate for N = 128, one whose A operand
+// is read from shared memory costs about twice as long for N <= 128. Every
+// operand that can live in TMEM does. Steps of BQ queries (64 for d = 128,
+// 128 for d = 64, so that some form of the dQ product has M = 128):
 //   S^T  = K_j Q_i^T      A = K_j   (TMEM, loaded once per CTA), B = Q_i
 //   dP^T = V_j dO_i^T     A = V_j   (shared memory),              B = dO_i
 //   dV  += P^T dO_i       A = P^T   (TMEM, written over S^T),     B = dO_i
 //   dK  += dS^T Q_i       A = dS^T  (TMEM, written over dP^T),    B = Q_i
-//   dQ^T = K_j^T dS^T     A = K_j^T (shared memory, MN-major),    B = dS^T
-// TMEM: K [0,64)  S^T/P^T [64,128)  dP^T/dS^T [128,192)  dQ^T [192,256)
-//       dV [256,384)  dK [384,512)
+//   d = 128: dQ^T = K_j^T dS^T   A = K_j^T (shared, MN-major), B = dS^T (shared)
+//   d = 64:  dQ   = dS K_j       A = dS (shared, MN-major),    B = K_j (shared, MN-major)
+// TMEM, d = 128: K [0,64)  S^T/P^T [64,128)  dP^T/dS^T [128,192)  dQ^T [192,256)
+//                dV [256,384)  dK [384,512)
+//      d = 64:   K [0,32)  S^T/P^T [64,192)  dP^T/dS^T [192,320)  dQ [320,384)
+//                dV [384,448)  dK [448,512)
 // One tcgen05 issuer executes in issue order, so S^T(i+2) may be issued right
 // after dV(i+1) (which reads P^T(i+1) from the same columns) and dP^T(i+1)
 // right after dK(i) (which reads dS^T(i)); per step the issue order is
 // dK(i), dP^T(i+1), dV(i+1), S^T(i+2), dQ(i).
-// Warps 4..11 (two per TMEM lane quarter, one per 32-query half) compute P
-// and then dS for their half; dS also goes to shared memory (double-buffered)
-// for the dQ product. Warps 12..15 (thread = head-dim column) drain dQ^T to a
-// shared staging tile and add it to dQ in HBM with a TMA tensor reduce-add
-// (one 32-column x 64-row box per warp).
-struct BwdD128 {
-  static constexpr int D = 128;
+// Warps 4..11 (two per TMEM lane quarter, one per half of the step's queries)
+// compute P and then dS for their half, 32 queries at a time; dS also goes to
+// shared memory (double-buffered) for the dQ product. Warps 12..15 drain the
+// dQ tile to a shared staging box and add it to dQ in HBM with a TMA tensor
+// reduce-add: d = 128, thread = head-dim column, one 32-column x 64-row box
+// per warp; d = 64, thread = query row, two 32-column x 32-row boxes per warp,
+// one after the other through one staging box (128-byte swizzled, so the
+// row-per-thread writes meet no bank conflicts).
+template <int D_>
+struct BwdTs {
+  static constexpr int D = D_;
   static constexpr int BK = 128;                 // keys per CTA
-  static constexpr int BQ = 64;                  // queries per step
-  static constexpr int KV_TILE = 128 * D * 2;    // K or V tile (two 64-column chunks)
+  static constexpr int BQ = D == 128 ? 64 : 128; // queries per step
+  static constexpr int HQ = BQ / 2;              // queries per half (one P / dS warp)
+  static constexpr int NCH = HQ / 32;            // 32-query chunks per half
+  static constexpr int KV_TILE = 128 * D * 2;    // K or V tile (D / 64 column chunks)
   static constexpr int KV_CHUNK = 128 * 128;
-  static constexpr int Q_TILE = BQ * D * 2;      // Q or dO tile (two chunks of 64 rows)
+  static constexpr int Q_TILE = BQ * D * 2;      // Q or dO tile (D / 64 chunks of BQ rows)
   static constexpr int Q_CHUNK = BQ * 128;
-  static constexpr int NS = 3;                   // Q / dO stages
-  static constexpr int DS_BYTES = BK * BQ * 2;   // dS^T fp16 [key][64 queries]: one 128 B row per key
-  static constexpr int DQ_STAGE = BQ * 32 * 4;   // one drain warp's fp32 box [64 queries][32 columns]
+  // Q / dO stages: at least 3, because S^T(i+2) is issued (and waits for its
+  // stage) before dQ(i), whose completion frees stage i
+  static constexpr int NS = 3;
+  static constexpr int DS_CHUNK = BK * 128;      // 64 queries of dS^T: one 128 B row per key
+  static constexpr int DS_BYTES = BK * BQ * 2;   // dS^T fp16 [key][BQ queries]
+  // per drain warp: d = 128, [64 queries][32 columns]; d = 64, one [32
+  // queries][32 columns] box, used for the two column halves in turn
+  static constexpr int DQ_STAGE = D == 128 ? BQ * 32 * 4 : 32 * 32 * 4;
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = K_OFF + KV_TILE;
   static constexpr int Q_OFF = V_OFF + KV_TILE;
   static constexpr int DO_OFF = Q_OFF + NS * Q_TILE;
   static constexpr int DS_OFF = DO_OFF + NS * Q_TILE;   // 2 buffers
   static constexpr int DQS_OFF = DS_OFF + 2 * DS_BYTES; // 4 staging boxes
-  static constexpr int L_OFF = DQS_OFF + 4 * DQ_STAGE;  // NS x 64 fp32: L * log2(e)
-  static constexpr int DL_OFF = L_OFF + NS * 256;       // NS x 64 fp32: D
-  static constexpr int BAR_OFF = DL_OFF + NS * 256;
-  // B_STEP[s]: committed after dQ^T of the step held in stage s; every product
-  // of that step is then complete: the Q / dO stage and the dS buffer are free
-  // and the dQ^T tile is ready.
+  static constexpr int L_OFF = DQS_OFF + 4 * DQ_STAGE;  // NS x BQ fp32: L * log2(e)
+  static constexpr int DL_OFF = L_OFF + NS * BQ * 4;    // NS x BQ fp32: -D'
+  static constexpr int BAR_OFF = DL_OFF + NS * BQ * 4;
+  // B_STEP[s]: committed after the dQ product of the step held in stage s;
+  // every product of that step is then complete: the Q / dO stage and the dS
+  // buffer are free and the dQ tile is ready.
   // B_FULL[s]: Q, L, dO and D of the step in stage s have landed.
   // B_DSQ: phase i completes when the 8 softmax-gradient warps have written
-  // dS(i) and the 4 drain warps have read dQ^T(i-1) out of TMEM.
+  // dS(i) and the 4 drain warps have read dQ(i-1) out of TMEM.
   static constexpr int B_KV = 0, B_FULL = 1, B_STEP = B_FULL + NS;
   static constexpr int B_KT = B_STEP + NS, B_ST = B_KT + 1, B_DPT = B_ST + 1, B_P = B_DPT + 1;
   static constexpr int B_DSQ = B_P + 1;
   static constexpr int B_END = B_DSQ + 1, B_DRAIN = B_END + 1, NBAR = B_DRAIN + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
-  static constexpr uint32_t COL_K = 0, COL_S = 64, COL_DP = 128, COL_DQ = 192, COL_DV = 256,
-                            COL_DK = 384;
+  static constexpr uint32_t COL_K = 0, COL_S = 64, COL_DP = COL_S + BQ, COL_DQ = COL_DP + BQ,
+                            COL_DV = COL_DQ + 64, COL_DK = COL_DV + D;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int THREADS = 512;
 };
-static_assert(BwdD128::SMEM_BYTES <= 232448, "d = 128 backward exceeds shared memory");
+static_assert(BwdTs<128>::SMEM_BYTES <= 232448, "d = 128 backward exceeds shared memory");
+static_assert(BwdTs<64>::SMEM_BYTES <= 232448, "d = 64 backward exceeds shared memory");
+static_assert(BwdTs<128>::COL_DK + 128 == 512 && BwdTs<64>::COL_DK + 64 == 512, "TMEM plan");
+static_assert(BwdTs<64>::DQS_OFF % 1024 == 0, "swizzled staging boxes need 1024 B alignment");
 
 constexpr int kOrderMaxB = 256;   // packed backward: sequences ordered by query length
-static_assert(BwdD128::DS_BYTES >= 4 * (kOrderMaxB + 1), "order list exceeds the dS buffer");
+static_assert(BwdTs<128>::DS_BYTES >= 4 * (kOrderMaxB + 1), "order list exceeds the dS buffer");
 
-// TMEM column of the 16-query group kk of a packed fp16 [key][64 queries]
-// operand whose two 32-query halves start 32 columns apart.
+// TMEM column of the 16-query group kk of a packed fp16 [key][BQ queries]
+// operand whose 32-query chunks start 32 columns apart (each chunk's 16
+// packed columns sit over the first half of its own 32 fp32 columns).
 __device__ __forceinline__ uint32_t half_col(int kk) {
   return static_cast<uint32_t>((kk >> 1) * 32 + (kk & 1) * 8);
 }
@@ -777,17 +375,16 @@ __device__ __forceinline__ uint32_t half_col(int kk) {
 // The keep bit of (query i, key j) is byte j % 16 of the Philox call
 // (j / 16, i, bh, offset). The 16 lanes holding keys 16g .. 16g+15 need the
 // same call per query, so each lane computes the calls of two of the 32
-// queries of its half and the words reach the lanes that need them by one
+// queries of its chunk and the words reach the lanes that need them by one
 // shuffle per element: the source lane of query 4b + c exposes, in round r,
 // word (c + r) % 4, which is what a lane needing word w reads in the round
 // with (w - r) % 4 = c.
-template <bool PACKED, bool DROP>
+template <int D, bool PACKED, bool DROP>
 __global__ void __launch_bounds__(512, 1)
-bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                const __grid_constant__ CUtensorMap tmDQ, BwdArgs a) {
-  using C = BwdD128;
-  constexpr int D = C::D;
+bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+              const __grid_constant__ CUtensorMap tmDQ, BwdArgs a) {
+  using C = BwdTs<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -922,7 +519,7 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tma_prefetch_desc(&tmDO);
       tma_prefetch_desc(&tmDQ);
       mbar_arrive_expect_tx(bar(C::B_KV), 2 * C::KV_TILE);
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         const int ky = packed ? hk : kb * C::BK, kz = packed ? tk0 + kb * C::BK : bh;
         tma_load_3d(base + C::K_OFF + c * C::KV_CHUNK, &tmK, bar(C::B_KV), c * 64, ky, kz);
         tma_load_3d(base + C::V_OFF + c * C::KV_CHUNK, &tmV, bar(C::B_KV), c * 64, ky, kz);
@@ -939,14 +536,14 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const int qy = packed ? hq : row, qz = packed ? tq0 + row : bh;
         if (!mbar_wait(bar(C::B_STEP + s), ph, a.err, kSiteQE, abort_flag)) break;
         const uint32_t full = bar(C::B_FULL + s);
-        mbar_arrive_expect_tx(full, 2 * (C::Q_TILE + 256));
-        for (int c = 0; c < 2; ++c)
+        mbar_arrive_expect_tx(full, 2 * (C::Q_TILE + C::BQ * 4));
+        for (int c = 0; c < D / 64; ++c)
           tma_load_3d(base + C::Q_OFF + s * C::Q_TILE + c * C::Q_CHUNK, &tmQ, full, c * 64, qy, qz);
-        bulk_load(base + C::L_OFF + s * 256, a.lse_log2 + prow, 256, full);
-        for (int c = 0; c < 2; ++c)
+        bulk_load(base + C::L_OFF + s * C::BQ * 4, a.lse_log2 + prow, C::BQ * 4, full);
+        for (int c = 0; c < D / 64; ++c)
           tma_load_3d(base + C::DO_OFF + s * C::Q_TILE + c * C::Q_CHUNK, &tmDO, full, c * 64, qy,
                       qz);
-        bulk_load(base + C::DL_OFF + s * 256, a.delta + prow, 256, full);
+        bulk_load(base + C::DL_OFF + s * C::BQ * 4, a.delta + prow, C::BQ * 4, full);
         issued = it + 1;
       }
       for (int it = max(0, issued - C::NS); it < issued; ++it) {
@@ -960,16 +557,20 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     if (lane == 0) {
       constexpr uint32_t idS = idesc_f16(128, C::BQ, 0, 0, 0);   // S^T, dP^T: K-major operands
       constexpr uint32_t idKM = idesc_f16(128, D, 0, 0, 1);      // dV, dK: A tmem, B MN-major
-      constexpr uint32_t idQT = idesc_f16(128, C::BQ, 0, 1, 1);  // dQ^T: A = K^T, B = dS^T, MN-major
+      // dQ: d = 128, dQ^T (M = d, N = BQ), A = K^T and B = dS^T MN-major;
+      //     d = 64,  dQ   (M = BQ, N = d), A = dS and B = K MN-major
+      constexpr uint32_t idQ = D == 128 ? idesc_f16(128, C::BQ, 0, 1, 1) : idesc_f16(128, D, 0, 1, 1);
       // descriptors of the fixed tiles and of stage / buffer 0; a tile at a
       // byte offset is the base descriptor plus offset / 16 (start-address field)
       const uint64_t dV = smem_desc_sw128(base + C::V_OFF, 16, 1024);            // V, K-major
-      const uint64_t dKt = smem_desc_sw128(base + C::K_OFF, C::KV_CHUNK, 1024);  // K^T, MN-major
+      const uint64_t dKt = smem_desc_sw128(base + C::K_OFF, C::KV_CHUNK, 1024);  // K, MN-major
       const uint64_t dQk = smem_desc_sw128(base + C::Q_OFF, 16, 1024);           // Q, K-major
       const uint64_t dQm = smem_desc_sw128(base + C::Q_OFF, C::Q_CHUNK, 1024);   // Q, MN-major
       const uint64_t dGk = smem_desc_sw128(base + C::DO_OFF, 16, 1024);          // dO, K-major
       const uint64_t dGm = smem_desc_sw128(base + C::DO_OFF, C::Q_CHUNK, 1024);  // dO, MN-major
-      const uint64_t dDS = smem_desc_sw128(base + C::DS_OFF, 16, 1024);          // dS^T, MN-major
+      // dS^T, MN-major: d = 128, the B operand of dQ^T (N = 64, one block of 64
+      // queries); d = 64, the A operand of dQ (M = 128, two blocks DS_CHUNK apart)
+      const uint64_t dDS = smem_desc_sw128(base + C::DS_OFF, D == 128 ? 16 : C::DS_CHUNK, 1024);
       auto add = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (bytes >> 4); };
       bool ok = mbar_wait(bar(C::B_KV), 0, a.err, kSiteKV, abort_flag) &&
                 mbar_wait(bar(C::B_KT), 0, a.err, kSiteKV, abort_flag);
@@ -1026,7 +627,7 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const uint64_t qm = add(dQm, s * C::Q_TILE);
         const uint64_t ds = add(dDS, (it & 1) * C::DS_BYTES);
         const uint32_t acc0 = it > 0 ? 1u : 0u;
-        // dK += dS^T Q_it (B_DSQ phase it: dS(it) written, dQ^T(it-1) drained)
+        // dK += dS^T Q_it (B_DSQ phase it: dS(it) written, dQ(it-1) drained)
         ok = mbar_wait(bar(C::B_DSQ), it & 1, a.err, kSiteDS, abort_flag);
         if (!ok) break;
         tc_fence_after();
@@ -1039,43 +640,52 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           if (ok && it + 2 < n_it) ok = issue_s(it + 2);
           if (!ok) break;
         }
-        // dQ^T_it = K^T dS^T (B_DSQ phase it covered the drain of dQ^T(it-1))
+        // dQ_it (B_DSQ phase it covered the drain of dQ(it-1)); K = the 128 keys
 #pragma unroll
-        for (int kk = 0; kk < C::BK / 16; ++kk)
-          umma_f16_ss(tmem + C::COL_DQ, add(dKt, kk * 2048), add(ds, kk * 2048), idQT,
-                      kk > 0 ? 1u : 0u);
-        umma_commit(bar(C::B_STEP + s));  // step it complete: stage s, dS buffer, dQ^T tile
+        for (int kk = 0; kk < C::BK / 16; ++kk) {
+          if constexpr (D == 128)
+            umma_f16_ss(tmem + C::COL_DQ, add(dKt, kk * 2048), add(ds, kk * 2048), idQ,
+                        kk > 0 ? 1u : 0u);
+          else
+            umma_f16_ss(tmem + C::COL_DQ, add(ds, kk * 2048), add(dKt, kk * 2048), idQ,
+                        kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar(C::B_STEP + s));  // step it complete: stage s, dS buffer, dQ tile
       }
       umma_commit(bar(C::B_END));
       umma_commit(bar(C::B_DRAIN));
       mbar_wait(bar(C::B_DRAIN), 0, a.err, kSiteDrain, nullptr, 200000000ull);
     }
   } else if (warp >= 4 && warp < 12) {
-    // ---------- P^T and dS^T for one 32-query half (thread = key row)
+    // ---------- P^T and dS^T for one half of the step's queries (thread = key row)
     const int quarter = warp & 3;
     const int h = (warp - 4) >> 2;
     const int r = quarter * 32 + lane;
     const int key = kb * C::BK + r;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t s_addr = tmem + lane_off + C::COL_S + 32 * h;
-    const uint32_t dp_addr = tmem + lane_off + C::COL_DP + 32 * h;
     const BwdScales sc = bwd_scales<D>(a);
     const float sl2 = sc.c_s;
     bool ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_KV), 0, a.err, kSiteKV, abort_flag));
     if (ok) {
-      // K row r, head-dim columns [64h, 64h+64): the A operand of S^T, packed
-      // two fp16 per TMEM column like the swizzled shared-memory row it comes from
-      const uint8_t* krow = smem + C::K_OFF + h * C::KV_CHUNK + r * 128;
-      uint32_t kr[32];
+      // K row r: the A operand of S^T, packed two fp16 per TMEM column like the
+      // swizzled shared-memory row it comes from; half h copies head-dim
+      // columns [D/2 h, D/2 h + D/2)
+      constexpr int UNITS = D / 16;                   // 16-byte units per half row
+      const uint8_t* krow = smem + C::K_OFF + (D == 128 ? h * C::KV_CHUNK : 0) + r * 128;
+      uint32_t kr[UNITS * 4];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const uint4 v = *reinterpret_cast<const uint4*>(krow + ((u ^ (r & 7)) << 4));
+      for (int u = 0; u < UNITS; ++u) {
+        const int unit = (D == 128 ? 0 : UNITS * h) + u;
+        const uint4 v = *reinterpret_cast<const uint4*>(krow + ((unit ^ (r & 7)) << 4));
         kr[4 * u] = v.x;
         kr[4 * u + 1] = v.y;
         kr[4 * u + 2] = v.z;
         kr[4 * u + 3] = v.w;
       }
-      tmem_st32(tmem + lane_off + C::COL_K + 32 * h, kr);
+      if constexpr (D == 128)
+        tmem_st32(tmem + lane_off + C::COL_K + 32 * h, kr);
+      else
+        tmem_st16(tmem + lane_off + C::COL_K + 16 * h, kr);
       tmem_st_wait();
       tc_fence_before();
       warp_arrive(bar(C::B_KT));
@@ -1084,134 +694,149 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     for (int it = 0; it < n_it && ok; ++it, walk_next(wk)) {
       const int s = it % C::NS;
       const int buf = it & 1;
-      const int qh = wk.step * C::BQ + 32 * h;          // first query of this half
-      const float* Ls = reinterpret_cast<const float*>(smem + C::L_OFF + s * 256) + 32 * h;
-      const float* Ds = reinterpret_cast<const float*>(smem + C::DL_OFF + s * 256) + 32 * h;
-      const bool need_mask = (a.causal && key > qh + off) || key >= Lk || qh + 31 >= Lq;
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_ST), it & 1, a.err, kSiteST, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      uint32_t sr[32];
-      tmem_ld32(s_addr, sr);
-      tmem_ld_wait();
-      uint32_t pk[16];                                 // P^T, fp16 pairs of queries
-      const uint64_t nsl2 = f2_pack(-sl2, -sl2);
-      // queries qh + i, i in [lo, hi), see this key; the masked form runs only
-      // in the steps where some lane of the warp has a masked query
-      const int lo = a.causal ? key - off - qh : INT_MIN;
-      const int hi = key < Lk ? Lq - qh : INT_MIN;
-      auto p_loop = [&](auto masked) {
+      uint32_t pk[C::NCH][16];                         // P^T, fp16 pairs of queries
+      uint32_t zm[C::NCH];                             // bit e: (query qc + e, key) kept
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float4 lv = *reinterpret_cast<const float4*>(Ls + e);
-          // y = L - scale log2e S on packed pairs; P = 2^-y
-          float y[4];
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), nsl2,
-                           f2_pack(lv.x, lv.y)), y[0], y[1]);
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3])), nsl2,
-                           f2_pack(lv.z, lv.w)), y[2], y[3]);
-          float p[4];
+      for (int ch = 0; ch < C::NCH; ++ch) {
+        const int qoff = C::HQ * h + 32 * ch;          // first query of this chunk in the step
+        const int qh = wk.step * C::BQ + qoff;
+        const float* Ls = reinterpret_cast<const float*>(smem + C::L_OFF + s * C::BQ * 4) + qoff;
+        const uint32_t s_addr = tmem + lane_off + C::COL_S + qoff;
+        const bool need_mask = (a.causal && key > qh + off) || key >= Lk || qh + 31 >= Lq;
+        uint32_t sr[32];
+        tmem_ld32(s_addr, sr);
+        tmem_ld_wait();
+        const uint64_t nsl2 = f2_pack(-sl2, -sl2);
+        // queries qh + i, i in [lo, hi), see this key; the masked form runs only
+        // in the steps where some lane of the warp has a masked query
+        const int lo = a.causal ? key - off - qh : INT_MIN;
+        const int hi = key < Lk ? Lq - qh : INT_MIN;
+        auto p_loop = [&](auto masked) {
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            p[u] = ex2_approx(-y[u]);
-            if constexpr (decltype(masked)::value) {
-              if (e + u < lo || e + u >= hi) p[u] = 0.f;
+          for (int e = 0; e < 32; e += 4) {
+            const float4 lv = *reinterpret_cast<const float4*>(Ls + e);
+            // y = L - scale log2e S on packed pairs; P = 2^-y
+            float y[4];
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), nsl2,
+                             f2_pack(lv.x, lv.y)), y[0], y[1]);
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3])), nsl2,
+                             f2_pack(lv.z, lv.w)), y[2], y[3]);
+            float p[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              p[u] = ex2_approx(-y[u]);
+              if constexpr (decltype(masked)::value) {
+                if (e + u < lo || e + u >= hi) p[u] = 0.f;
+              }
+            }
+            pk[ch][e / 2] = pack_f16x2(p[0], p[1]);
+            pk[ch][e / 2 + 1] = pack_f16x2(p[2], p[3]);
+          }
+        };
+        if (__any_sync(0xffffffffu, need_mask))
+          p_loop(std::true_type{});
+        else
+          p_loop(std::false_type{});
+        zm[ch] = 0xffffffffu;
+        if constexpr (DROP) {
+          const uint32_t g = lane & 15, jg = static_cast<uint32_t>(key) >> 4;
+          uint32_t x[2][4];                            // x[c][r] = word (lane % 4 + r) % 4
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const uint4 w = philox4x32_10(jg, static_cast<uint32_t>(qh) + g + 16u * c,
+                                          static_cast<uint32_t>(bh), a.drop_offset, a.seed_lo,
+                                          a.seed_hi);
+            const bool r1 = lane & 1, r2 = lane & 2;
+            const uint32_t a0 = r1 ? w.y : w.x, a1 = r1 ? w.z : w.y, a2 = r1 ? w.w : w.z,
+                           a3 = r1 ? w.x : w.w;
+            x[c][0] = r2 ? a2 : a0;
+            x[c][1] = r2 ? a3 : a1;
+            x[c][2] = r2 ? a0 : a2;
+            x[c][3] = r2 ? a1 : a3;
+          }
+          const int wsel = static_cast<int>(g >> 2);   // the word holding this key's byte
+          const uint32_t sh = 8u * (lane & 3);         // its byte within the word
+          const uint32_t keep_add = 256u - a.drop_t;   // byte + keep_add >= 256 iff kept
+          uint32_t z = 0u;
+#pragma unroll
+          for (int bq = 0; bq < 8; ++bq) {
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) {
+              const int c = (wsel - rr) & 3;           // query 4 bq + c arrives in round rr
+              const uint32_t y = __shfl_sync(0xffffffffu, x[bq >> 2][rr],
+                                             static_cast<int>(lane & 16) | ((4 * bq) & 15) | c);
+              z |= ((((y >> sh) & 0xffu) + keep_add) >> 8) << (4 * bq + c);
             }
           }
-          pk[e / 2] = pack_f16x2(p[0], p[1]);
-          pk[e / 2 + 1] = pack_f16x2(p[2], p[3]);
+          zm[ch] = z;
         }
-      };
-      if (__any_sync(0xffffffffu, need_mask))
-        p_loop(std::true_type{});
-      else
-        p_loop(std::false_type{});
-      uint32_t zm = 0xffffffffu;                       // bit e: (query qh + e, key) kept
-      if constexpr (DROP) {
-        const uint32_t g = lane & 15, jg = static_cast<uint32_t>(key) >> 4;
-        uint32_t x[2][4];                              // x[c][r] = word (lane % 4 + r) % 4
+        uint32_t pz[16];                               // P o Z for the dV product
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const uint4 w = philox4x32_10(jg, static_cast<uint32_t>(qh) + g + 16u * c,
-                                        static_cast<uint32_t>(bh), a.drop_offset, a.seed_lo,
-                                        a.seed_hi);
-          const bool r1 = lane & 1, r2 = lane & 2;
-          const uint32_t a0 = r1 ? w.y : w.x, a1 = r1 ? w.z : w.y, a2 = r1 ? w.w : w.z,
-                         a3 = r1 ? w.x : w.w;
-          x[c][0] = r2 ? a2 : a0;
-          x[c][1] = r2 ? a3 : a1;
-          x[c][2] = r2 ? a0 : a2;
-          x[c][3] = r2 ? a1 : a3;
-        }
-        const int wsel = static_cast<int>(g >> 2);     // the word holding this key's byte
-        const uint32_t sh = 8u * (lane & 3);           // its byte within the word
-        const uint32_t keep_add = 256u - a.drop_t;     // byte + keep_add >= 256 iff kept
-        zm = 0u;
-#pragma unroll
-        for (int bq = 0; bq < 8; ++bq) {
-#pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            const int c = (wsel - r) & 3;              // query 4 bq + c arrives in round r
-            const uint32_t y = __shfl_sync(0xffffffffu, x[bq >> 2][r],
-                                           static_cast<int>(lane & 16) | ((4 * bq) & 15) | c);
-            zm |= ((((y >> sh) & 0xffu) + keep_add) >> 8) << (4 * bq + c);
-          }
-        }
+        for (int e = 0; e < 16; ++e)
+          pz[e] = DROP ? pk[ch][e] & ((((zm[ch] >> (2 * e)) & 3u) * 0x8001u & 0x10001u) * 0xffffu)
+                       : pk[ch][e];
+        tmem_st16(s_addr, pz);                         // over this chunk's own S^T columns
       }
-      uint32_t pz[16];                                 // P o Z for the dV product
-#pragma unroll
-      for (int e = 0; e < 16; ++e)
-        pz[e] = DROP ? pk[e] & ((((zm >> (2 * e)) & 3u) * 0x8001u & 0x10001u) * 0xffffu) : pk[e];
-      tmem_st16(s_addr, pz);                           // over this half's own S^T columns
       tmem_st_wait();
       tc_fence_before();
       warp_arrive(bar(C::B_P));
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_DPT), it & 1, a.err, kSiteDPT, abort_flag));
       if (!ok) break;
-      if (it >= 2) {                                   // dQ^T(it-2) has read this dS buffer
+      if (it >= 2) {                                   // dQ(it-2) has read this dS buffer
         ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_STEP + (it - 2) % C::NS),
                                                ((it - 2) / C::NS) & 1, a.err, kSiteDSF, abort_flag));
         if (!ok) break;
       }
       tc_fence_after();
-      uint32_t dr[32];
-      tmem_ld32(dp_addr, dr);
-      tmem_ld_wait();
-      uint32_t w[16];                                  // dS^T, fp16 pairs of queries
-      float ds_max = 0.f;
       // alpha (2^-(14 + log2 d)) brings dP' to the units of dS'; with dropout
       // it also carries 1 / q
       const float ga = DROP ? sc.alpha * a.drop_scale : sc.alpha;
       const uint64_t ga2 = f2_pack(ga, ga);
+      float ds_max = 0.f;
 #pragma unroll
-      for (int e = 0; e < 32; e += 4) {
-        const float4 dv4 = *reinterpret_cast<const float4*>(Ds + e);   // -D'
-        uint64_t g01 = f2_pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1]));
-        uint64_t g23 = f2_pack(__uint_as_float(dr[e + 2]), __uint_as_float(dr[e + 3]));
-        if constexpr (DROP) {                          // dP -> Z o dP
-          auto z = [&](int i) { return dr[i] & (0u - ((zm >> i) & 1u)); };
-          g01 = f2_pack(__uint_as_float(z(e)), __uint_as_float(z(e + 1)));
-          g23 = f2_pack(__uint_as_float(z(e + 2)), __uint_as_float(z(e + 3)));
+      for (int ch = 0; ch < C::NCH; ++ch) {
+        const int qoff = C::HQ * h + 32 * ch;
+        const float* Ds = reinterpret_cast<const float*>(smem + C::DL_OFF + s * C::BQ * 4) + qoff;
+        const uint32_t dp_addr = tmem + lane_off + C::COL_DP + qoff;
+        uint32_t dr[32];
+        tmem_ld32(dp_addr, dr);
+        tmem_ld_wait();
+        uint32_t w[16];                                // dS^T, fp16 pairs of queries
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          const float4 dv4 = *reinterpret_cast<const float4*>(Ds + e);   // -D'
+          uint64_t g01 = f2_pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1]));
+          uint64_t g23 = f2_pack(__uint_as_float(dr[e + 2]), __uint_as_float(dr[e + 3]));
+          if constexpr (DROP) {                        // dP -> Z o dP
+            auto z = [&](int i) { return dr[i] & (0u - ((zm[ch] >> i) & 1u)); };
+            g01 = f2_pack(__uint_as_float(z(e)), __uint_as_float(z(e + 1)));
+            g23 = f2_pack(__uint_as_float(z(e + 2)), __uint_as_float(z(e + 3)));
+          }
+          // dS' = P o (alpha dP' - D') on packed pairs
+          const uint64_t d01 = f2_fma(g01, ga2, f2_pack(dv4.x, dv4.y));
+          const uint64_t d23 = f2_fma(g23, ga2, f2_pack(dv4.z, dv4.w));
+          const uint32_t pa = pk[ch][e / 2], pb = pk[ch][e / 2 + 1];
+          float ds[4];
+          f2_unpack(f2_mul(f2_pack(f16_lo(pa), f16_hi(pa)), d01), ds[0], ds[1]);
+          f2_unpack(f2_mul(f2_pack(f16_lo(pb), f16_hi(pb)), d23), ds[2], ds[3]);
+          ds_max = fmax3(ds_max, fmax3(fabsf(ds[0]), fabsf(ds[1]), fabsf(ds[2])), fabsf(ds[3]));
+          w[e / 2] = pack_f16x2(ds[0], ds[1]);
+          w[e / 2 + 1] = pack_f16x2(ds[2], ds[3]);
         }
-        // dS' = P o (alpha dP' - D') on packed pairs
-        const uint64_t d01 = f2_fma(g01, ga2, f2_pack(dv4.x, dv4.y));
-        const uint64_t d23 = f2_fma(g23, ga2, f2_pack(dv4.z, dv4.w));
-        const uint32_t pa = pk[e / 2], pb = pk[e / 2 + 1];
-        float ds[4];
-        f2_unpack(f2_mul(f2_pack(f16_lo(pa), f16_hi(pa)), d01), ds[0], ds[1]);
-        f2_unpack(f2_mul(f2_pack(f16_lo(pb), f16_hi(pb)), d23), ds[2], ds[3]);
-        ds_max = fmax3(ds_max, fmax3(fabsf(ds[0]), fabsf(ds[1]), fabsf(ds[2])), fabsf(ds[3]));
-        w[e / 2] = pack_f16x2(ds[0], ds[1]);
-        w[e / 2 + 1] = pack_f16x2(ds[2], ds[3]);
-      }
-      tmem_st16(dp_addr, w);                           // A operand of dK, over own dP^T columns
-      // shared memory copy for dQ: this half's 64 bytes of the key's 128-byte
-      // row, XOR-swizzled with (key row % 8) like a TMA SWIZZLE_128B tile
-      uint8_t* ds_row = smem + C::DS_OFF + buf * C::DS_BYTES + r * 128;
+        tmem_st16(dp_addr, w);                         // A operand of dK, over own dP^T columns
+        // shared memory copy for dQ: the chunk's 64 bytes of the key's 128-byte
+        // row in its 64-query block, XOR-swizzled with (key row % 8) like a TMA
+        // SWIZZLE_128B tile
+        uint8_t* ds_row = smem + C::DS_OFF + buf * C::DS_BYTES + (qoff / 64) * C::DS_CHUNK + r * 128;
+        const int unit0 = (qoff % 64) / 8;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        uint4* dst = reinterpret_cast<uint4*>(ds_row + (((4 * h + u) ^ (r & 7)) << 4));
-        *dst = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+        for (int u = 0; u < 4; ++u) {
+          uint4* dst = reinterpret_cast<uint4*>(ds_row + (((unit0 + u) ^ (r & 7)) << 4));
+          *dst = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+        }
       }
       if (!(ds_max < 65504.f)) atomicCAS(a.err, 0u, kErrRange + 2);
       tmem_st_wait();
@@ -1247,15 +872,15 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     tc_fence_before();
   } else if (warp >= 12) {
-    // ------------- dQ^T tile -> HBM (thread = one head-dim column) via TMA
-    const int quarter = warp & 3;                    // TMEM lanes = d [32 quarter, 32 quarter + 32)
+    // ------------------------------------------ dQ tile -> HBM via TMA reduce-add
+    const int quarter = warp & 3;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const BwdScales bs = bwd_scales<D>(a);
     const float sc = bs.dq1, sc2 = bs.dq2;
     const bool two = sc2 != 1.f;
     float* stage = reinterpret_cast<float*>(smem + C::DQS_OFF + quarter * C::DQ_STAGE);
     const uint32_t stage_addr = base + C::DQS_OFF + quarter * C::DQ_STAGE;
-    warp_arrive(bar(C::B_DSQ));                      // phase 0: no dQ^T(-1) to drain
+    warp_arrive(bar(C::B_DSQ));                      // phase 0: no dQ(-1) to drain
     Walk wq = walk_start();
     for (int it = 0; it < n_it; ++it, walk_next(wq)) {
       const int q0 = wq.step * C::BQ;
@@ -1263,40 +888,75 @@ bwd_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                                               kSiteDQ, abort_flag)))
         break;
       tc_fence_after();
+      // d = 128: TMEM lanes = head-dim columns, 64 queries; d = 64: lanes =
+      // queries, 64 head-dim columns. Either way 64 values per thread.
       uint32_t v0[32], v1[32];
       tmem_ld32(tmem + lane_off + C::COL_DQ, v0);
       tmem_ld32(tmem + lane_off + C::COL_DQ + 32, v1);
       tmem_ld_wait();
       tc_fence_before();
-      warp_arrive(bar(C::B_DSQ));                    // dQ^T(it) read: counts for phase it+1
-      if (lane == 0) bulk_wait_read_all();           // previous reduce has read the staging box
-      __syncwarp();
+      warp_arrive(bar(C::B_DSQ));                    // dQ(it) read: counts for phase it+1
       if (two) {                                     // factor outside one float's range
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           v0[j] = __float_as_uint(__uint_as_float(v0[j]) * sc * sc2);
           v1[j] = __float_as_uint(__uint_as_float(v1[j]) * sc * sc2);
         }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          v0[j] = __float_as_uint(__uint_as_float(v0[j]) * sc);
+          v1[j] = __float_as_uint(__uint_as_float(v1[j]) * sc);
+        }
+      }
+      if (lane == 0) bulk_wait_read_all();           // previous reduce has read the staging box
+      __syncwarp();
+      if constexpr (D == 128) {
+        // [64 queries][32 columns], thread = column: lane-contiguous stores
 #pragma unroll
         for (int j = 0; j < 32; ++j) stage[j * 32 + lane] = __uint_as_float(v0[j]);
 #pragma unroll
         for (int j = 0; j < 32; ++j) stage[(32 + j) * 32 + lane] = __uint_as_float(v1[j]);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          // rows past the tensor are skipped; in the packed form, rows past this
+          // sequence add exact zeros (dS = 0 there) to the next sequence's dQ
+          if (packed)
+            tma_reduce_add_3d(&tmDQ, stage_addr, quarter * 32, wq.head, tq0 + q0);
+          else
+            tma_reduce_add_3d(&tmDQ, stage_addr, quarter * 32, q0, bh);
+          bulk_commit_group();
+        }
       } else {
+        // a [32 queries][32 columns] box per column half, thread = query row,
+        // 16-byte units XOR-swizzled with (row % 8) as the 128-byte-swizzled
+        // tensor map reads them; the second half waits until the first has
+        // been read out of the box
+        uint8_t* srow = reinterpret_cast<uint8_t*>(stage) + lane * 128;
+        const int qr = q0 + quarter * 32;            // this warp's 32 query rows
 #pragma unroll
-        for (int j = 0; j < 32; ++j) stage[j * 32 + lane] = __uint_as_float(v0[j]) * sc;
+        for (int c = 0; c < 2; ++c) {
+          if (c == 1) {
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+          }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) stage[(32 + j) * 32 + lane] = __uint_as_float(v1[j]) * sc;
-      }
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        // rows past the tensor are skipped; in the packed form, rows past this
-        // sequence add exact zeros (dS = 0 there) to the next sequence's dQ
-        if (packed)
-          tma_reduce_add_3d(&tmDQ, stage_addr, quarter * 32, wq.head, tq0 + q0);
-        else
-          tma_reduce_add_3d(&tmDQ, stage_addr, quarter * 32, q0, bh);
-        bulk_commit_group();
+          for (int u = 0; u < 8; ++u) {
+            const uint32_t* v = c ? v1 : v0;
+            *reinterpret_cast<uint4*>(srow + ((u ^ (lane & 7)) << 4)) =
+                make_uint4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+          }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (packed)
+              tma_reduce_add_3d(&tmDQ, stage_addr, c * 32, wq.head, tq0 + qr);
+            else
+              tma_reduce_add_3d(&tmDQ, stage_addr, c * 32, qr, bh);
+            bulk_commit_group();
+          }
+        }
       }
     }
     if (lane == 0) bulk_wait_all();
@@ -1317,23 +977,19 @@ template <int D>
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a,
                        cudaStream_t stream, cudaEvent_t ev_main_begin, cudaEvent_t ev_main_end) {
-  using C = BwdCfg<D>;
+  using C = BwdTs<D>;
   static std::atomic<bool> attr_set[64];   // per device; racing first calls both set it
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = D == 128 ? cudaFuncSetAttribute(bwd_d128_kernel<false, false>,
-                                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                    BwdD128::SMEM_BYTES)
-                             : cudaFuncSetAttribute(bwd_main_kernel<D>,
-                                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                    C::SMEM_BYTES);
-    if (e == cudaSuccess && D == 128)
-      e = cudaFuncSetAttribute(bwd_d128_kernel<true, false>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, BwdD128::SMEM_BYTES);
-    if (e == cudaSuccess && D == 128)
-      e = cudaFuncSetAttribute(bwd_d128_kernel<false, true>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, BwdD128::SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(bwd_ts_kernel<D, false, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(bwd_ts_kernel<D, true, false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(bwd_ts_kernel<D, false, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
@@ -1352,18 +1008,15 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   const int nk = ((a.cu_q ? a.max_k : a.N) + C::BK - 1) / C::BK;
   const int per_block = a.cu_q ? a.B * a.Hkv : a.B * a.H;   // CTAs per key block
   if (ev_main_begin != nullptr) cudaEventRecord(ev_main_begin, stream);
-  if (D == 128)
-    if (a.cu_q)
-      bwd_d128_kernel<true, false><<<nk * per_block, BwdD128::THREADS, BwdD128::SMEM_BYTES,
-                                     stream>>>(tq, tk, tv, tdo, tdq, a);
-    else if (a.dropout)
-      bwd_d128_kernel<false, true><<<nk * per_block, BwdD128::THREADS, BwdD128::SMEM_BYTES,
-                                     stream>>>(tq, tk, tv, tdo, tdq, a);
-    else
-      bwd_d128_kernel<false, false><<<nk * per_block, BwdD128::THREADS, BwdD128::SMEM_BYTES,
-                                      stream>>>(tq, tk, tv, tdo, tdq, a);
+  if (a.cu_q)
+    bwd_ts_kernel<D, true, false><<<nk * per_block, C::THREADS, C::SMEM_BYTES, stream>>>(
+        tq, tk, tv, tdo, tdq, a);
+  else if (a.dropout)
+    bwd_ts_kernel<D, false, true><<<nk * per_block, C::THREADS, C::SMEM_BYTES, stream>>>(
+        tq, tk, tv, tdo, tdq, a);
   else
-    bwd_main_kernel<D><<<nk * a.B * a.H, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
+    bwd_ts_kernel<D, false, false><<<nk * per_block, C::THREADS, C::SMEM_BYTES, stream>>>(
+        tq, tk, tv, tdo, tdq, a);
   e = cudaGetLastError();
   if (ev_main_end != nullptr) cudaEventRecord(ev_main_end, stream);
   return e;

@@ -153,7 +153,7 @@ def test_bwd_varlen_rejects_bad_arguments_without_a_gpu():
     p = ctypes.c_void_p(256)
     s = ctypes.c_void_p(0)
     args = [p] * 10 + [ctypes.c_size_t(1 << 30), p, p, 2, 64, 64, 128, 128, 8, 2, 128, 1, s]
-    a = list(args); a[20] = 64                # d = 64 is not supported yet
+    a = list(args); a[20] = 96                # d not in {64, 128}
     assert L.fa_bwd_varlen(*a) == fa.FA_ERR_UNSUPPORTED
     a = list(args); a[19] = 3                 # H % Hkv != 0
     assert L.fa_bwd_varlen(*a) == fa.FA_ERR_INVALID_ARG
@@ -173,8 +173,8 @@ def test_dropout_rejects_bad_probability_and_head_dim_without_gpu():
     assert L.fa_fwd_dropout(_p(0), *([g] * 4), 1, 2, 128, 64, 0, 0.1, 1, 0,
                             None) == fa.FA_ERR_INVALID_ARG
     assert L.fa_fwd_dropout(*([g] * 5), 1, 2, 128, 80, 0, 0.1, 1, 0, None) == fa.FA_ERR_UNSUPPORTED
-    need = L.fa_bwd_workspace_bytes(1, 2, 128, 64)
-    assert L.fa_bwd_dropout(*([g] * 10), need, 1, 2, 128, 64, 0, 0.1, 1, 0,
-                            None) == fa.FA_ERR_UNSUPPORTED          # backward: d = 128 only
+    need = L.fa_bwd_workspace_bytes(1, 2, 128, 96)
+    assert L.fa_bwd_dropout(*([g] * 10), need, 1, 2, 128, 96, 0, 0.1, 1, 0,
+                            None) == fa.FA_ERR_UNSUPPORTED          # d not in {64, 128}
     assert L.fa_bwd_dropout(*([g] * 9), g, 0, 1, 2, 128, 128, 0, 0.1, 1, 0,
                             None) == fa.FA_ERR_WORKSPACE

@@ -47,11 +47,12 @@ def _contract(x, cu_q, cu_k, causal, **kw):
     return grads
 
 
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
-def test_equal_lengths_match_fa_bwd(causal):
+def test_equal_lengths_match_fa_bwd(causal, d):
     """Equal lengths, H = Hkv: dK and dV agree with fa_bwd on the [B, H, N, d]
     view bit for bit; dQ (summed by reductions in varying order) to rounding."""
-    B, H, N, d = 2, 4, 300, 128
+    B, H, N = 2, 4, 300
     x, cu_q, cu_k = _case([N] * B, [N] * B, H, H, d, 700 + causal)
     o, lse = fa.fa_fwd_varlen(x["q"], x["k"], x["v"], torch.from_numpy(cu_q).cuda(),
                               torch.from_numpy(cu_k).cuda(), N, causal=causal)
@@ -67,25 +68,27 @@ def test_equal_lengths_match_fa_bwd(causal):
     assert float((bhnd(g1[0]) - g2[0]).abs().max()) < 1e-4
 
 
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
-def test_ragged_cross_lengths_gqa(causal):
+def test_ragged_cross_lengths_gqa(causal, d):
     """Unequal lengths both ways, tails off the 64 / 128 grid, a sequence with
     no queries (its dK, dV are 0) and one with no keys, 8 query heads on 2 KV
     heads; bottom-right causal includes queries that see no key."""
     lens_q = [17, 128, 200, 0, 300, 1, 64, 90]
     lens_k = [40, 128, 129, 50, 300, 500, 0, 33]
-    x, cu_q, cu_k = _case(lens_q, lens_k, 8, 2, 128, 710 + causal)
+    x, cu_q, cu_k = _case(lens_q, lens_k, 8, 2, d, 710 + causal + d)
     _, dk, dv = _contract(x, cu_q, cu_k, causal)
     k0, k1 = int(cu_k[3]), int(cu_k[4])                  # the sequence without queries
     assert torch.all(dk[k0:k1] == 0) and torch.all(dv[k0:k1] == 0)
 
 
-def test_long_mixed_batch():
+@pytest.mark.parametrize("d", [64, 128])
+def test_long_mixed_batch(d):
     """8 sequences, lengths U[1, 2048] (queries = keys), 8 heads on 4 KV heads,
     causal: every gradient element."""
     rng = np.random.default_rng(720)
     lens = rng.integers(1, 2049, 8).tolist()
-    x, cu_q, cu_k = _case(lens, lens, 8, 4, 128, 720)
+    x, cu_q, cu_k = _case(lens, lens, 8, 4, d, 720 + d)
     _contract(x, cu_q, cu_k, True)
 
 

@@ -52,12 +52,13 @@ def test_forward_keep_mask_bit_exact(p):
     assert np.array_equal(got.astype(bool), want)
 
 
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("p", [0.1, 0.5])
-def test_backward_keep_mask_bit_exact(p):
+def test_backward_keep_mask_bit_exact(p, d):
     """The backward regenerates the mask with keys on the lanes (one Philox call
     per 16 keys and query, shared across 16 lanes by shuffles). K = 0 and
-    dO_i = 2^(i div 128) e_(i mod 128) make dV_jc * N / s = sum_m Z[c + 128 m, j] 2^m."""
-    B, H, N, d = 2, 3, 384, 128
+    dO_i = 2^(i div d) e_(i mod d) make dV_jc * N / s = sum_m Z[c + d m, j] 2^m."""
+    B, H, N = 2, 3, 384
     g = torch.Generator().manual_seed(78)
     q = torch.randn((B, H, N, d), generator=g).to(torch.bfloat16).cuda()
     k = torch.zeros_like(q)
@@ -68,10 +69,10 @@ def test_backward_keep_mask_bit_exact(p):
     _, _, dv = fa.fa_bwd_dropout(q, k, v, o, lse, do, p, seed, off)
     torch.cuda.synchronize()
     assert fa.fa_last_device_error() == fa.FA_OK
-    x = f64(dv) * N / _keep_scale(p)                                    # [B, H, N keys, 128]
+    x = f64(dv) * N / _keep_scale(p)                                    # [B, H, N keys, d]
     code = np.rint(x).astype(np.int64)
-    assert np.abs(x - code).max() < 0.05 and code.min() >= 0 and code.max() <= 7
-    # bit m of code[b, h, j, c] is Z[query c + 128 m, key j]
+    assert np.abs(x - code).max() < 0.05 and code.min() >= 0 and code.max() < 2 ** (N // d)
+    # bit m of code[b, h, j, c] is Z[query c + d m, key j]
     got = np.stack([(code >> m) & 1 for m in range(N // d)], axis=-2)   # [B, H, j, m, c]
     got = got.reshape(B, H, N, N).transpose(0, 1, 3, 2)                 # [B, H, i, j]
     assert np.array_equal(got.astype(bool), keep_mask(B, H, N, p, seed, off))
@@ -85,15 +86,14 @@ def test_p_zero_is_fa_fwd_and_fa_bwd(d, causal):
     o2, l2 = fa.fa_fwd(x["q"], x["k"], x["v"], causal=causal)
     torch.cuda.synchronize()
     assert torch.equal(o, o2) and torch.equal(lse, l2)
-    if d == 128:
-        # dK and dV are summed inside one CTA: bit-equal; dQ is reduced across
-        # CTAs in an order that varies from run to run: equal to rounding
-        dq1, dk1, dv1 = fa.fa_bwd_dropout(x["q"], x["k"], x["v"], o, lse, x["do"], 0.0, 1, 0,
-                                          causal=causal)
-        dq2, dk2, dv2 = fa.fa_bwd(x["q"], x["k"], x["v"], o, lse, x["do"], causal=causal)
-        torch.cuda.synchronize()
-        assert torch.equal(dk1, dk2) and torch.equal(dv1, dv2)
-        assert float((dq1 - dq2).abs().max()) < 1e-5
+    # dK and dV are summed inside one CTA: bit-equal; dQ is reduced across
+    # CTAs in an order that varies from run to run: equal to rounding
+    dq1, dk1, dv1 = fa.fa_bwd_dropout(x["q"], x["k"], x["v"], o, lse, x["do"], 0.0, 1, 0,
+                                      causal=causal)
+    dq2, dk2, dv2 = fa.fa_bwd(x["q"], x["k"], x["v"], o, lse, x["do"], causal=causal)
+    torch.cuda.synchronize()
+    assert torch.equal(dk1, dk2) and torch.equal(dv1, dv2)
+    assert float((dq1 - dq2).abs().max()) < 1e-5
 
 
 @pytest.mark.parametrize("causal", [False, True])
@@ -114,13 +114,14 @@ def test_forward_parity(p, N, d, causal):
     assert torch.equal(lse, l_plain)                    # L is that of the undropped scores
 
 
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("N", [17, 129, 300])
 @pytest.mark.parametrize("p", [0.1, 0.5])
-def test_backward_contract(p, N, causal):
+def test_backward_contract(p, N, causal, d):
     """Gradients from the oracle's own (bf16-rounded) O and L, as fa_bwd's tests."""
-    B, H, d = 1, 2, 128
-    x = synth.attention_inputs(B, H, N, d, 4300 + N + causal, device="cuda")
+    B, H = 1, 2
+    x = synth.attention_inputs(B, H, N, d, 4300 + N + causal + d, device="cuda")
     seed, off = 2024, 1
     q, k, v, do = (f64(x[n]) for n in ("q", "k", "v", "do"))
     o_ref, l_ref = attention_dropout(q, k, v, p, seed, off, causal)

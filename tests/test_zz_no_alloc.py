@@ -57,10 +57,12 @@ def test_noalloc_rejects_requests_over_the_limit():
     q, kc, vc, tab, lens, _ = _case(4, 100, 400, 303)
     o = torch.empty_like(q)
     with pytest.raises(fa.FAError) as e:
-        # 64 sequences x 32 heads x 32 splits of partials do not fit in 16 MiB
+        # 64 sequences x 32 heads x 32 splits of partials do not fit in 16 MiB;
+        # every other argument passes the checks (the call is rejected before
+        # anything is read: a table width of 2048 entries is only declared)
         fa.lib()
         status = fa.lib().paged_attn_decode_noalloc(
-            fa._ptr(q), fa._ptr(kc), fa._ptr(vc), kc.shape[0], fa._ptr(tab), tab.shape[1],
+            fa._ptr(q), fa._ptr(kc), fa._ptr(vc), kc.shape[0], fa._ptr(tab), 2048,
             fa._ptr(lens), fa._ptr(o), None, 64, 32, 8, 128, 16, 32768, fa._stream())
         fa._check("paged_attn_decode_noalloc", status)
     assert e.value.status == fa.FA_ERR_WORKSPACE
