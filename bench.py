@@ -46,9 +46,9 @@ METRIC = "attention fwd+bwd TFLOP/s (bf16)"
 # DRAM bytes (read + write) of one d = 128 backward main-pass launch at WORKLOAD,
 # from an ncu capture of that launch with the current kernel; None whenever the
 # kernel has changed since, until captured again
-BWD_MAIN_TRAFFIC = None
+BWD_MAIN_TRAFFIC = 0.803e9
 # the same for one forward launch at WORKLOAD
-FWD_TRAFFIC = None
+FWD_TRAFFIC = 0.251e9
 # a timed region shorter than this runs at burst clocks: its kernels are held to
 # the burst peak; a longer one to the sustained (power-capped) peak
 SUSTAINED_REGION_MS = 1000.0
@@ -737,7 +737,7 @@ def main():
     fwd_t = f_fwd / (r["fwd_ms"] / 1e3) / 1e12
     main_t = f_bwd / (r["bwd_main_ms"] / 1e3) / 1e12
     if r["bwd_main_ms"] >= r["fwd_ms"]:
-        kern, ach = "bwd_d128_kernel (fa_bwd main pass)", main_t
+        kern, ach = "bwd_ts_kernel<128> (fa_bwd main pass)", main_t
         traffic = BWD_MAIN_TRAFFIC
     else:
         kern, ach, traffic = "fwd_kernel (fa_fwd)", fwd_t, FWD_TRAFFIC

@@ -145,7 +145,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   if (warp == kComputeWarps) {
     // ------------------------------------------------------------ producer
     // Items are handed out dynamically: lane 0 takes the next index of the
-    // dense (sequence, KV head, split) space from a global counter and skips
+    // dense (split, KV head, sequence) space from a global counter and skips
     // splits past a sequence's end. The next item is resolved while the
     // current item's first blocks are in flight.
     struct Item { int seq, kvh, split, nb, rem; };
@@ -154,10 +154,14 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       while (true) {
         const long long idx = atomicAdd(a.counter, 1u);
         if (idx >= total) return it;   // nb = 0: no more work
-        it.split = static_cast<int>(idx % a.max_splits);
-        const long long rest = idx / a.max_splits;
+        // split-major order: the same split of every (KV head, sequence) runs
+        // at about the same time, so blocks that several sequences share
+        // (parallel-sampling prefixes, adjacent sequences) are read from HBM
+        // once and from L2 for the others
+        it.seq = static_cast<int>(idx % a.num_seqs);
+        const long long rest = idx / a.num_seqs;
         it.kvh = static_cast<int>(rest % a.Hkv);
-        it.seq = static_cast<int>(rest / a.Hkv);
+        it.split = static_cast<int>(rest / a.Hkv);
         // a length outside [1, max_ctx] is reported by the combine kernel;
         // the clamp keeps the reads inside the table and the workspace
         const int ctx = max(1, min(a.context_lens[it.seq], a.max_ctx));
