@@ -340,12 +340,15 @@ struct BwdTs {
   // every product of that step is then complete: the Q / dO stage and the dS
   // buffer are free and the dQ tile is ready.
   // B_FULL[s]: Q, L, dO and D of the step in stage s have landed.
-  // B_DSQ: phase i completes when the 8 softmax-gradient warps have written
-  // dS(i) and the 4 drain warps have read dQ(i-1) out of TMEM.
+  // B_DS: phase i completes when the 8 softmax-gradient warps have written
+  // dS(i). B_DQF: phase i completes when the 4 drain warps have read dQ(i-1)
+  // out of TMEM, so that dQ(i) may overwrite it. dK(i) waits on the first,
+  // dQ(i) on the second: the drain of dQ(i-1) runs while dK(i), dP(i+1),
+  // dV(i+1) and S(i+2) keep the tensor pipe busy.
   static constexpr int B_KV = 0, B_FULL = 1, B_STEP = B_FULL + NS;
   static constexpr int B_KT = B_STEP + NS, B_ST = B_KT + 1, B_DPT = B_ST + 1, B_P = B_DPT + 1;
-  static constexpr int B_DSQ = B_P + 1;
-  static constexpr int B_END = B_DSQ + 1, B_DRAIN = B_END + 1, NBAR = B_DRAIN + 1;
+  static constexpr int B_DS = B_P + 1, B_DQF = B_DS + 1;
+  static constexpr int B_END = B_DQF + 1, B_DRAIN = B_END + 1, NBAR = B_DRAIN + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
   static constexpr uint32_t COL_K = 0, COL_S = 64, COL_DP = COL_S + BQ, COL_DQ = COL_DP + BQ,
@@ -495,7 +498,8 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     mbar_init(bar(C::B_ST), 1);
     mbar_init(bar(C::B_DPT), 1);
     mbar_init(bar(C::B_P), 8);
-    mbar_init(bar(C::B_DSQ), 8 + 4);  // 8 softmax-gradient warps + 4 drain warps
+    mbar_init(bar(C::B_DS), 8);       // the 8 softmax-gradient warps
+    mbar_init(bar(C::B_DQF), 4);      // the 4 drain warps
     mbar_init(bar(C::B_END), 1);
     mbar_init(bar(C::B_DRAIN), 1);
     *abort_flag = 0;
@@ -627,8 +631,8 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const uint64_t qm = add(dQm, s * C::Q_TILE);
         const uint64_t ds = add(dDS, (it & 1) * C::DS_BYTES);
         const uint32_t acc0 = it > 0 ? 1u : 0u;
-        // dK += dS^T Q_it (B_DSQ phase it: dS(it) written, dQ(it-1) drained)
-        ok = mbar_wait(bar(C::B_DSQ), it & 1, a.err, kSiteDS, abort_flag);
+        // dK += dS^T Q_it (B_DS phase it: dS(it) written)
+        ok = mbar_wait(bar(C::B_DS), it & 1, a.err, kSiteDS, abort_flag);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -640,7 +644,10 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           if (ok && it + 2 < n_it) ok = issue_s(it + 2);
           if (!ok) break;
         }
-        // dQ_it (B_DSQ phase it covered the drain of dQ(it-1)); K = the 128 keys
+        // dQ_it, once dQ(it-1) has been drained (B_DQF phase it); K = the 128 keys
+        ok = mbar_wait(bar(C::B_DQF), it & 1, a.err, kSiteDQF, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < C::BK / 16; ++kk) {
           if constexpr (D == 128)
@@ -842,7 +849,7 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       tmem_st_wait();
       fence_async_smem();
       tc_fence_before();
-      warp_arrive(bar(C::B_DSQ));
+      warp_arrive(bar(C::B_DS));
     }
     // ---- epilogue: dV rows (half 0) or dK rows (half 1), thread = key
     if (ok) {
@@ -880,7 +887,7 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const bool two = sc2 != 1.f;
     float* stage = reinterpret_cast<float*>(smem + C::DQS_OFF + quarter * C::DQ_STAGE);
     const uint32_t stage_addr = base + C::DQS_OFF + quarter * C::DQ_STAGE;
-    warp_arrive(bar(C::B_DSQ));                      // phase 0: no dQ(-1) to drain
+    warp_arrive(bar(C::B_DQF));                      // phase 0: no dQ(-1) to drain
     Walk wq = walk_start();
     for (int it = 0; it < n_it; ++it, walk_next(wq)) {
       const int q0 = wq.step * C::BQ;
@@ -895,7 +902,7 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       tmem_ld32(tmem + lane_off + C::COL_DQ + 32, v1);
       tmem_ld_wait();
       tc_fence_before();
-      warp_arrive(bar(C::B_DSQ));                    // dQ(it) read: counts for phase it+1
+      warp_arrive(bar(C::B_DQF));                    // dQ(it) read: counts for phase it+1
       if (two) {                                     // factor outside one float's range
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
