@@ -48,6 +48,22 @@
 
 namespace fa {
 
+// Pipeline trace (built only with -DFA_BWD_TRACE by exact_attention_102_b200.trace_bwd,
+// never in libfa.so): CTA 0 of the [B, H, N, d] d = 128 main pass records clock64
+// stamps of its MMA-issuing thread, of one P / dS warp and of one drain warp.
+#ifdef FA_BWD_TRACE
+__device__ unsigned long long g_bwd_trace[3][8192];
+#define FA_TRACE(row, tag)                                                             \
+  do {                                                                                 \
+    if (tr_on && tr_n[row] < 8192)                                                     \
+      g_bwd_trace[row][tr_n[row]++] = (static_cast<unsigned long long>(clock64()) << 8) | (tag); \
+  } while (0)
+#else
+#define FA_TRACE(row, tag) \
+  do {                     \
+  } while (0)
+#endif
+
 namespace {
 
 enum : uint32_t {
@@ -487,6 +503,10 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   auto bar = [&](int i) -> uint32_t { return base + C::BAR_OFF + 8 * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
+#ifdef FA_BWD_TRACE
+  const bool tr_on = blockIdx.x == 0 && D == 128 && !PACKED && !DROP;
+  int tr_n[3] = {0, 0, 0};
+#endif
 
   if (threadIdx.x == 0) {
     mbar_init(bar(C::B_KV), 1);
@@ -632,7 +652,9 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const uint64_t ds = add(dDS, (it & 1) * C::DS_BYTES);
         const uint32_t acc0 = it > 0 ? 1u : 0u;
         // dK += dS^T Q_it (B_DS phase it: dS(it) written)
+        FA_TRACE(0, 1);
         ok = mbar_wait(bar(C::B_DS), it & 1, a.err, kSiteDS, abort_flag);
+        FA_TRACE(0, 2);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -640,12 +662,18 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           umma_f16_ts(tmem + C::COL_DK, tmem + C::COL_DP + half_col(kk), add(qm, kk * 2048), idKM,
                       kk > 0 ? 1u : acc0);
         if (it + 1 < n_it) {
-          ok = issue_dp(it + 1) && issue_dv(it + 1);
+          FA_TRACE(0, 3);
+          ok = issue_dp(it + 1);
+          FA_TRACE(0, 4);
+          ok = ok && issue_dv(it + 1);
+          FA_TRACE(0, 5);
           if (ok && it + 2 < n_it) ok = issue_s(it + 2);
+          FA_TRACE(0, 6);
           if (!ok) break;
         }
         // dQ_it, once dQ(it-1) has been drained (B_DQF phase it); K = the 128 keys
         ok = mbar_wait(bar(C::B_DQF), it & 1, a.err, kSiteDQF, abort_flag);
+        FA_TRACE(0, 7);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -658,6 +686,7 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         kk > 0 ? 1u : 0u);
         }
         umma_commit(bar(C::B_STEP + s));  // step it complete: stage s, dS buffer, dQ tile
+        FA_TRACE(0, 8);
       }
       umma_commit(bar(C::B_END));
       umma_commit(bar(C::B_DRAIN));
@@ -701,7 +730,9 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     for (int it = 0; it < n_it && ok; ++it, walk_next(wk)) {
       const int s = it % C::NS;
       const int buf = it & 1;
+      if (warp == 4 && lane == 0) FA_TRACE(1, 1);
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_ST), it & 1, a.err, kSiteST, abort_flag));
+      if (warp == 4 && lane == 0) FA_TRACE(1, 2);
       if (!ok) break;
       tc_fence_after();
       uint32_t pk[C::NCH][16];                         // P^T, fp16 pairs of queries
@@ -790,7 +821,9 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       tmem_st_wait();
       tc_fence_before();
       warp_arrive(bar(C::B_P));
+      if (warp == 4 && lane == 0) FA_TRACE(1, 3);
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_DPT), it & 1, a.err, kSiteDPT, abort_flag));
+      if (warp == 4 && lane == 0) FA_TRACE(1, 4);
       if (!ok) break;
       if (it >= 2) {                                   // dQ(it-2) has read this dS buffer
         ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_STEP + (it - 2) % C::NS),
@@ -798,6 +831,7 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         if (!ok) break;
       }
       tc_fence_after();
+      if (warp == 4 && lane == 0) FA_TRACE(1, 5);
       // alpha (2^-(14 + log2 d)) brings dP' to the units of dS'; with dropout
       // it also carries 1 / q
       const float ga = DROP ? sc.alpha * a.drop_scale : sc.alpha;
@@ -850,6 +884,7 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       fence_async_smem();
       tc_fence_before();
       warp_arrive(bar(C::B_DS));
+      if (warp == 4 && lane == 0) FA_TRACE(1, 6);
     }
     // ---- epilogue: dV rows (half 0) or dK rows (half 1), thread = key
     if (ok) {
@@ -891,9 +926,11 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     Walk wq = walk_start();
     for (int it = 0; it < n_it; ++it, walk_next(wq)) {
       const int q0 = wq.step * C::BQ;
+      if (warp == 12 && lane == 0) FA_TRACE(2, 1);
       if (!__all_sync(0xffffffffu, mbar_wait(bar(C::B_STEP + it % C::NS), (it / C::NS) & 1, a.err,
                                               kSiteDQ, abort_flag)))
         break;
+      if (warp == 12 && lane == 0) FA_TRACE(2, 2);
       tc_fence_after();
       // d = 128: TMEM lanes = head-dim columns, 64 queries; d = 64: lanes =
       // queries, 64 head-dim columns. Either way 64 values per thread.
@@ -903,6 +940,7 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       tmem_ld_wait();
       tc_fence_before();
       warp_arrive(bar(C::B_DQF));                    // dQ(it) read: counts for phase it+1
+      if (warp == 12 && lane == 0) FA_TRACE(2, 3);
       if (two) {                                     // factor outside one float's range
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
@@ -1037,3 +1075,10 @@ template cudaError_t launch_bwd<128>(const CUtensorMap&, const CUtensorMap&, con
                                      cudaStream_t, cudaEvent_t, cudaEvent_t);
 
 }  // namespace fa
+
+#ifdef FA_BWD_TRACE
+// Copies the trace stamps of the last traced launch to host memory (3 x 8192 words).
+extern "C" __attribute__((visibility("default"))) int fa_bwd_trace_read(void* host) {
+  return static_cast<int>(cudaMemcpyFromSymbol(host, fa::g_bwd_trace, sizeof(fa::g_bwd_trace)));
+}
+#endif
