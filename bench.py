@@ -49,6 +49,8 @@ METRIC = "attention fwd+bwd TFLOP/s (bf16)"
 BWD_MAIN_TRAFFIC = 0.803e9
 # the same for one forward launch at WORKLOAD
 FWD_TRAFFIC = 0.251e9
+# DRAM bytes of one paged-decode launch at the c4 workload (current kernel)
+DECODE_TRAFFIC = 4.241e9
 # a timed region shorter than this runs at burst clocks: its kernels are held to
 # the burst peak; a longer one to the sustained (power-capped) peak
 SUSTAINED_REGION_MS = 1000.0
@@ -770,7 +772,7 @@ def main():
             "GB/s_logical": dec["logical_bytes"] / (dec["ms"] / 1e3) / 1e9,
             "shared_block_fraction": dec["shared_fraction"],
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / peaks["hbm_gbs"], "traffic": None}}
+                         "frac": gbs / peaks["hbm_gbs"], "traffic": DECODE_TRAFFIC}}
         vl = run_fwd_varlen(fa, args.steps, args.warmup)
         parts["fwd_varlen"] = {
             "workload": f"packed causal batch: {VARLEN['n']} sequences, lengths "
