@@ -14,7 +14,9 @@ attention
     through the block table, then the forward definition), the logsumexp
     merge of split partials, the packed variable-length form (sequences of
     unequal query / key lengths, grouped KV heads, bottom-right causal), and
-    the FP8 e4m3 block quantiser used by the diagnostic FP8 oracle.
+    the FP8 e4m3 block quantiser used by the diagnostic FP8 oracle, and the
+    gradients of the FP8 forward (straight through the quantisation, back
+    through the rotation).
 dropout
     Attention with dropout on the probabilities: the Philox4x32-10
     counter-based generator written from its published definition, the keep
@@ -44,6 +46,7 @@ from .attention import (  # noqa: F401
     quantize_e4m3,
     dequantize_blocks_e4m3,
     fp8_block_quantize,
+    attention_fp8_bwd,
 )
 from .dropout import (  # noqa: F401
     attention_dropout,

@@ -433,3 +433,32 @@ def dequantize_blocks_e4m3(vals, scales, block_rows=64):
     n = vals.shape[-2]
     rs = np.repeat(scales, block_rows, axis=-1)[..., :n]
     return vals * rs[..., None]
+
+
+def attention_fp8_bwd(q_vals, sq, k_vals, sk, v_vals, sv, R, do, o, causal=False,
+                      block_rows=64, scale=None):
+    """Gradients of the FP8 attention forward with respect to its unrotated
+    inputs Q, K and its input V, float64.
+
+    [FA-series] FlashAttentionV3 / FP低精度 and [FA-v1v2v3] "FP8 低精度計算":
+    the FP8 forward attends over Q' = Q R and K' = K R (R orthogonal, so
+    Q' K'^T = Q K^T) and V, each quantised to e4m3 with one scale per block of
+    64 rows. The pages give no FP8 backward. Reading (the plainest one that
+    makes it the backward of that forward): the quantisation is treated as the
+    identity (straight through), so the gradients are the textbook ones of
+    attention over the dequantised tensors Qh = q_vals * sq, Kh = k_vals * sk,
+    Vh = v_vals * sv (blocks of ``block_rows`` rows), with D built from the
+    forward's O, then carried back through the rotation:
+        (dQh, dKh, dVh) = attention_bwd(Qh, Kh, Vh, dO, o=O)
+        dQ = dQh R^T,  dK = dKh R^T,  dV = dVh
+    (dQ'/dQ = R: d/dQ f(Q R) = (df/dQ') R^T). Inputs: e4m3 values (float64 on
+    the e4m3 grid) [..., N, d], scales [..., ceil(N/64)], R [d, d], dO and O
+    [..., N, d]. Returns (dQ, dK, dV). Pinned by torch autograd through the
+    rotation and the block dequantisation in tests/test_oracle_pins.py.
+    """
+    qh = dequantize_blocks_e4m3(q_vals, sq, block_rows)
+    kh = dequantize_blocks_e4m3(k_vals, sk, block_rows)
+    vh = dequantize_blocks_e4m3(v_vals, sv, block_rows)
+    dqh, dkh, dvh, _ = attention_bwd(qh, kh, vh, do, causal=causal, scale=scale, o=o)
+    r = np.asarray(R, dtype=np.float64)
+    return dqh @ r.T, dkh @ r.T, dvh

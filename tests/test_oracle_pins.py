@@ -614,3 +614,36 @@ def test_block_sparse_brute_force_with_empty_rows():
             np.testing.assert_allclose(o[i], sum(wi / sum(w) * v[j] for wi, j in zip(w, keys)),
                                        rtol=1e-12, atol=1e-13)
             assert abs(lse[i] - (mx + math.log(sum(w)))) < 1e-12
+
+
+def test_fp8_backward_matches_autograd_through_rotation_and_blocks():
+    """attention_fp8_bwd against torch float64 autograd of the FP8 forward's
+    function: O = attention((Q R), (K R), V) evaluated at Q = Qh R^T, K = Kh R^T
+    (so that Q R = Qh, the dequantised block-scaled codes), with the gradient
+    taken with respect to Q, K, V. A sign or transpose slip in the rotation,
+    a wrong block scale or a dropped term fails it."""
+    import torch
+
+    rng = np.random.default_rng(2024)
+    B, H, N, d = 1, 2, 100, 16                       # two 64-row blocks, the second ragged
+    R = synth.orthogonal_matrix(d, 77)
+    x = {n: rng.standard_normal((B, H, N, d)) * rng.choice([1.0, 8.0], (B, H, N, d), p=[0.95, 0.05])
+         for n in ("q", "k", "v", "do")}
+    qv, sq = oracle.fp8_block_quantize(x["q"] @ R)
+    kv, sk = oracle.fp8_block_quantize(x["k"] @ R)
+    vv, sv = oracle.fp8_block_quantize(x["v"])
+    assert len(np.unique(sq)) > 2                    # per-block scales really differ
+    qh, kh, vh = (oracle.dequantize_blocks_e4m3(a, s) for a, s in ((qv, sq), (kv, sk), (vv, sv)))
+    for causal in (False, True):
+        o, _ = oracle.attention_fwd(qh, kh, vh, causal=causal)
+        dq, dk, dv = oracle.attention_fp8_bwd(qv, sq, kv, sk, vv, sv, R, x["do"], o, causal)
+        Rt = torch.from_numpy(R)
+        tq = torch.from_numpy(qh @ R.T).requires_grad_(True)
+        tk = torch.from_numpy(kh @ R.T).requires_grad_(True)
+        tv = torch.from_numpy(vh).requires_grad_(True)
+        out = torch.nn.functional.scaled_dot_product_attention(tq @ Rt, tk @ Rt, tv,
+                                                               is_causal=causal)
+        (out * torch.from_numpy(x["do"])).sum().backward()
+        np.testing.assert_allclose(out.detach().numpy(), o, rtol=0, atol=1e-12)
+        for got, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+            np.testing.assert_allclose(got, ref.numpy(), rtol=0, atol=1e-10)

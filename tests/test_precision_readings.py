@@ -12,7 +12,13 @@ Both use only the oracle and the seeded generators (no GPU, no library).
    the plain 5e-2 applies to inputs without outliers, where the same
    quantisation stays inside it.
 
-2. Scores beyond fp32's resolution. Scaling Q and K together by 2^8 scales
+2. FP8 backward operands. The e4m3 blocks the FP8 forward uses for Q, K, V
+   are exact fp16 values, but quantising the upstream gradient dO the same way
+   (one e4m3 scale per 64 rows) already moves dV by ~1 and dQ by ~12 on the
+   FP8 workload, far beyond 5e-2. So the FP8 backward keeps its gradient
+   products in fp16 (on the forward's e4m3 codes, exactly) rather than e4m3.
+
+3. Scores beyond fp32's resolution. Scaling Q and K together by 2^8 scales
    the scores and L by 2^16 (|S|, |L| up to ~3e5), where one fp32 ulp is
    2^-5 .. 2^-7. A backward rebuilds P = exp(S - L) from an fp32 score and
    the fp32 L the forward stored; their rounding alone, every other step
@@ -88,3 +94,22 @@ def test_scores_at_2_pow_16_are_beyond_fp32_resolution():
         dv = oracle.attention_bwd(q * f, k * f, v, do)[2]
         err = np.abs(_dv_with_fp32_scores(q * f, k * f, do, lse) - dv).max()
         assert lo <= err < hi, (f, err)     # measured 3.0e-7 and 0.19
+
+
+def test_e4m3_gradient_exceeds_5e2_on_fp8_workload():
+    x = synth.fp8_inputs(1, 1, 4096, 128, 1003)
+    g = torch.Generator().manual_seed(5)
+    do = torch.randn((1, 1, 4096, 128), generator=g).to(torch.bfloat16).double().numpy()
+    r32 = synth.orthogonal_matrix(128, 2003).astype(np.float32).astype(np.float64)
+    qv, sq = oracle.fp8_block_quantize(_f64(x["q"]) @ r32)
+    kv, sk = oracle.fp8_block_quantize(_f64(x["k"]) @ r32)
+    vv, sv = oracle.fp8_block_quantize(_f64(x["v"]))
+    qh, kh, vh = (oracle.dequantize_blocks_e4m3(a, s) for a, s in ((qv, sq), (kv, sk), (vv, sv)))
+    o, _ = oracle.attention_fwd(qh, kh, vh)
+    exact = oracle.attention_fp8_bwd(qv, sq, kv, sk, vv, sv, r32, do, o)
+    dov, sdo = oracle.fp8_block_quantize(do)
+    quant = oracle.attention_fp8_bwd(qv, sq, kv, sk, vv, sv, r32,
+                                     oracle.dequantize_blocks_e4m3(dov, sdo), o)
+    err = [np.abs(a - b).max() for a, b in zip(exact, quant)]
+    # measured: dQ 12.0, dK 5.4, dV 0.98
+    assert min(err) > 0.5, err
