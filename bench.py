@@ -329,7 +329,28 @@ def run_fp8(fa, steps, warmup, seed=1003):
     b.record()
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / steps
-    return {"ms": ms, "flops": attn_flops(B, H, N, d, False)}
+    # the FP8 backward on the same codes (dO ~ N(0, 1), drawn after the inputs)
+    g = torch.Generator(device="cuda").manual_seed(seed + 1)
+    do = torch.randn((B, H, N, d), generator=g, device="cuda").to(torch.bfloat16)
+    grads = [torch.empty((B, H, N, d), device="cuda") for _ in range(3)]
+    wsp = torch.empty(fa.fa_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device="cuda")
+
+    def bwd():
+        fa.fa_bwd_fp8(q8, k8, v8, sq, sk, sv, R, o, lse, do, causal=False, dq=grads[0],
+                      dk=grads[1], dv=grads[2], workspace=wsp)
+
+    nb = max(3, steps // 4)
+    for _ in range(warmup):
+        bwd()
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(nb):
+        bwd()
+    b.record()
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_error() == fa.FA_OK
+    return {"ms": ms, "flops": attn_flops(B, H, N, d, False), "bwd_ms": a.elapsed_time(b) / nb,
+            "bwd_flops": attn_flops(B, H, N, d, False, bwd=True)}
 
 
 VARLEN = dict(n=16, lo=512, hi=8192, H=16, Hkv=4, d=128, causal=True, seed=1006)
@@ -805,6 +826,13 @@ def main():
             parts["fp8_fwd"] = {"ms": f8["ms"], "TFLOP/s": t8, "roofline": {
                 "bound": "tensor", "achieved": t8, "peak": p8, "unit": "TFLOP/s", "frac": t8 / p8,
                 "peak_source": f"{peaks['source']} bf16 burst x 2 (nominal fp8/bf16 ratio)"}}
+            tb = f8["bwd_flops"] / (f8["bwd_ms"] / 1e3) / 1e12
+            parts["fp8_bwd"] = {
+                "ms": f8["bwd_ms"], "TFLOP/s": tb, "workload": "backward of the FP8 forward on its "
+                "codes (fp16 products, block scales in fp32, rotation back)",
+                "roofline": {"bound": "tensor", "achieved": tb, "peak": peak_t, "unit": "TFLOP/s",
+                             "frac": tb / peak_t,
+                             "peak_source": f"{peaks['source']} bf16 burst (fp16 products)"}}
         else:
             parts["fp8_fwd"] = f8
 

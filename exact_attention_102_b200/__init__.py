@@ -39,7 +39,7 @@ EXPORTS = (
     "fa_kv_pool_create", "fa_kv_pool_destroy", "fa_kv_seq_add", "fa_kv_seq_fork", "fa_kv_seq_free",
     "fa_kv_seq_append", "fa_kv_num_free", "fa_kv_refcount", "fa_kv_seq_len", "fa_kv_block_table",
     "fa_kv_copy_blocks", "fa_paged_prefill", "fa_fwd_block_sparse", "fa_fwd_dropout",
-    "fa_bwd_dropout",
+    "fa_bwd_dropout", "fa_bwd_fp8",
 )
 
 
@@ -82,6 +82,8 @@ def lib() -> ctypes.CDLL:
     L.fa_fp8_prepare.argtypes = [vp] * 10 + [ci, ci, ci, ci, vp]
     L.fa_fwd_fp8.restype = ci
     L.fa_fwd_fp8.argtypes = [vp] * 8 + [ci, ci, ci, ci, ci, vp]
+    L.fa_bwd_fp8.restype = ci
+    L.fa_bwd_fp8.argtypes = [vp] * 14 + [sz] + [ci] * 5 + [vp]
     L.fa_last_device_error.restype = ci
     L.fa_last_device_error.argtypes = [vp]
     L.fa_bwd_time_main_pass.restype = ci
@@ -569,6 +571,38 @@ def fa_fp8_prepare(q, k, v, R, stream=None):
         _ptr(q), _ptr(k), _ptr(v), _ptr(R), _ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq), _ptr(sk),
         _ptr(sv), B, H, N, d, _stream(stream)))
     return q8, k8, v8, sq, sk, sv
+
+
+def fa_bwd_fp8(q8, k8, v8, sq, sk, sv, R, o, lse, do, causal=False, dq=None, dk=None, dv=None,
+               workspace=None, stream=None):
+    """Gradients of fa_fwd_fp8 with respect to the unrotated q, k and v (fp32):
+    straight through the e4m3 quantisation, back through R (dQ = dQ' R^T)."""
+    _need(q8, "q8", torch.uint8, 4)
+    _need(k8, "k8", torch.uint8, shape=q8.shape)
+    _need(v8, "v8", torch.uint8, shape=q8.shape)
+    B, H, N, d = q8.shape
+    nb = (N + 63) // 64
+    for n, t in (("sq", sq), ("sk", sk), ("sv", sv)):
+        _need(t, n, torch.float32, shape=(B, H, nb))
+    _need(R, "R", torch.float32, shape=(d, d))
+    _need(o, "o", torch.bfloat16, shape=q8.shape)
+    _need(lse, "lse", torch.float32, shape=(B, H, N))
+    _need(do, "do", torch.bfloat16, shape=q8.shape)
+    dq = torch.empty(q8.shape, dtype=torch.float32, device=q8.device) if dq is None else dq
+    dk = torch.empty(q8.shape, dtype=torch.float32, device=q8.device) if dk is None else dk
+    dv = torch.empty(q8.shape, dtype=torch.float32, device=q8.device) if dv is None else dv
+    for n, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _need(t, n, torch.float32, shape=q8.shape)
+    if workspace is None:
+        workspace = torch.empty(fa_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8,
+                                device=q8.device)
+    _need_workspace(workspace)
+    _check("fa_bwd_fp8", lib().fa_bwd_fp8(
+        _ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq), _ptr(sk), _ptr(sv), _ptr(R), _ptr(o), _ptr(lse),
+        _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), B, H, N, d, int(bool(causal)),
+        _stream(stream)))
+    return dq, dk, dv
 
 
 def fa_fwd_fp8(q8, k8, v8, sq, sk, sv, causal=False, o=None, lse=None, stream=None):

@@ -175,15 +175,25 @@ fa_status fwd_dense(const void* q, const void* k, const void* v, void* o, float*
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
+// The FP8 backward's extra inputs: the block scales of the e4m3 codes passed
+// as q, k, v, and the rotation the codes of q and k were taken after.
+struct Fp8Spec {
+  const float* sq;
+  const float* sk;
+  const float* sv;
+  const float* R;
+};
+
 fa_status bwd_dense(const void* q, const void* k, const void* v, const void* o, const float* lse,
                     const void* dout, float* dq, float* dk, float* dv, void* workspace,
                     size_t ws_bytes, int B, int H, int N, int d, int causal, void* stream,
-                    const DropSpec* drop) {
+                    const DropSpec* drop, const Fp8Spec* f8 = nullptr) {
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
       !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return FA_ERR_INVALID_ARG;
   fa_status st = check_attn_dims(B, H, N, d);
   if (st != FA_OK) return st;
+  if (f8 != nullptr && (d != 128 || drop != nullptr)) return FA_ERR_UNSUPPORTED;
   if (workspace == nullptr || !aligned16(workspace) ||
       ws_bytes < fa_bwd_workspace_bytes(B, H, N, d))
     return FA_ERR_WORKSPACE;
@@ -248,11 +258,24 @@ fa_status bwd_dense(const void* q, const void* k, const void* v, const void* o, 
     a.drop_offset = drop->offset;
     a.drop_scale = drop->scale;
   }
+  if (f8 != nullptr) {
+    a.fp8 = 1;
+    a.sq = f8->sq;
+    a.sk = f8->sk;
+    a.sv = f8->sv;
+    a.nsb = (N + 63) / 64;
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaEvent_t eb = g_bwd_ev_begin, ee = g_bwd_ev_end;
   g_bwd_ev_begin = g_bwd_ev_end = nullptr;     // one call consumes the pair
   cudaError_t e = (d == 128) ? fa::launch_bwd<128>(tq, tk, tv, tdo, tdq, a, s, eb, ee)
                              : fa::launch_bwd<64>(tq, tk, tv, tdo, tdq, a, s, eb, ee);
+  if (e == cudaSuccess && f8 != nullptr) {
+    // gradients of the rotated inputs -> of Q and K: dQ = dQ' R^T, dK = dK' R^T
+    const long long rows = static_cast<long long>(bh) * N;
+    e = fa::launch_unrotate(dq, f8->R, rows, s);
+    if (e == cudaSuccess) e = fa::launch_unrotate(dk, f8->R, rows, s);
+  }
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
@@ -454,6 +477,18 @@ fa_status fa_bwd_dropout(const void* q, const void* k, const void* v, const void
   if (!drop_spec(p_drop, seed, offset, &ds)) return FA_ERR_INVALID_ARG;
   return bwd_dense(q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, B, H, N, d, causal,
                    stream, &ds);
+}
+
+fa_status fa_bwd_fp8(const void* q8, const void* k8, const void* v8, const float* sq,
+                     const float* sk, const float* sv, const float* R, const void* o,
+                     const float* lse, const void* dout, float* dq, float* dk, float* dv,
+                     void* workspace, size_t ws_bytes, int B, int H, int N, int d, int causal,
+                     void* stream) {
+  if (!aligned16(sq) || !aligned16(sk) || !aligned16(sv) || !aligned16(R))
+    return FA_ERR_INVALID_ARG;
+  const Fp8Spec f8{sq, sk, sv, R};
+  return bwd_dense(q8, k8, v8, o, lse, dout, dq, dk, dv, workspace, ws_bytes, B, H, N, d, causal,
+                   stream, nullptr, &f8);
 }
 
 size_t fa_bwd_varlen_workspace_bytes(int batch, int max_seqlen_q, int total_q, int total_k, int H,

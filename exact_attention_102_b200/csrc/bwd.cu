@@ -130,6 +130,18 @@ __global__ void __launch_bounds__(256) bwd_amax_kernel(BwdArgs a, long long q8, 
   uint32_t m[4];
 #pragma unroll
   for (int t = 0; t < 4; ++t) {
+    if (a.fp8 && t < 3) {
+      // FP8 backward: the largest block scale of q, k, v (positive floats
+      // compare as their bit patterns); the codes themselves need no scale
+      const float* src = t == 0 ? a.sq : t == 1 ? a.sk : a.sv;
+      const long long n = static_cast<long long>(a.B) * a.H * a.nsb;
+      uint32_t mm = 0u;
+      for (long long i = tid; i < n; i += stride) mm = max(mm, __float_as_uint(fabsf(src[i])));
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mm = max(mm, __shfl_xor_sync(0xffffffffu, mm, off));
+      m[t] = mm;
+      continue;
+    }
     const uint4* src = static_cast<const uint4*>(t == 0 ? a.q : t == 1 ? a.k : t == 2 ? a.v : a.dout);
     const long long n = (t == 0 || t == 3) ? q8 : k8;
     uint32_t mm = 0u;
@@ -180,6 +192,73 @@ __device__ __forceinline__ void load_exps(const BwdArgs& a, int (&e)[4]) {
   }
 }
 
+// FP8 backward: the operands are the forward's e4m3 codes (exact fp16 values),
+// the block scales are folded in fp32, and dO is scaled like the bf16 path.
+// dS' = dS sq_i sk_j 2^tau is bounded like R22's dS':
+//   |dS| <= 2 d max|dO| max|V|, max|V| <= 448 max(sv), so with
+//   tau = e_do + 15 - ceil(log2(2 d 2^14 448 max(sq) max(sk) max(sv)))
+//   |dS'| <= 2^15 (max|dO| 2^e_do < 2^14).
+// exps[] then holds {tau, 0, 0, e_do}.
+__device__ void fp8_convert(const BwdArgs& a, const int (&e)[4], long long q16) {
+  // e[0..2]: scale_exp of the largest block scales' bit patterns is not what is
+  // wanted here; recover the maxima from the partials directly
+  __shared__ float smax[3];
+  if (threadIdx.x < 3) {
+    uint32_t r = 0u;
+    for (int i = 0; i < kBwdAmaxBlocks; ++i) r = max(r, a.amax_part[i * 4 + threadIdx.x]);
+    smax[threadIdx.x] = __uint_as_float(r);
+  }
+  __syncthreads();
+  const int e_do = e[3];
+  const float bound = 2.f * 128.f * 16384.f * 448.f;   // 2 d 2^14 448, d = 128
+  int c = 0;
+  frexpf(bound * fmaxf(smax[0], 1e-30f) * fmaxf(smax[1], 1e-30f) * fmaxf(smax[2], 1e-30f), &c);
+  const int tau = e_do + 15 - c;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    a.exps[0] = tau;
+    a.exps[1] = 0;
+    a.exps[2] = 0;
+    a.exps[3] = e_do;
+  }
+  const Pow2 fdo = pow2_pair(e_do);
+  // units of 16 bytes: e4m3 codes of q, k, v (16 codes -> 32 bytes of fp16),
+  // then dO (8 bf16 -> 16 bytes of fp16)
+  const long long c16 = q16 / 2;                    // 16-code units per tensor
+  const long long total = 3 * c16 + q16;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    if (i < 3 * c16) {
+      const int t = static_cast<int>(i / c16);
+      const long long j = i - t * c16;
+      const uint4 u = static_cast<const uint4*>(t == 0 ? a.q : t == 1 ? a.k : a.v)[j];
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      uint32_t o[8];
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        asm("{\n\t.reg .b16 lo, hi;\n\t"
+            "mov.b32 {lo, hi}, %2;\n\t"
+            "cvt.rn.f16x2.e4m3x2 %0, lo;\n\t"
+            "cvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
+            : "=r"(o[2 * cc]), "=r"(o[2 * cc + 1])
+            : "r"(w[cc]));
+      }
+      uint4* dp = static_cast<uint4*>(t == 0 ? a.q16 : t == 1 ? a.k16 : a.v16) + 2 * j;
+      dp[0] = make_uint4(o[0], o[1], o[2], o[3]);
+      dp[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    } else {
+      const long long j = i - 3 * c16;
+      const uint4 u = static_cast<const uint4*>(a.dout)[j];
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc)
+        o[cc] = pack_f16x2(mul_pow2(__uint_as_float(w[cc] << 16), fdo),
+                           mul_pow2(__uint_as_float(w[cc] & 0xffff0000u), fdo));
+      static_cast<uint4*>(a.do16)[j] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
 // ------------------------------------------------------- fp16 conversion
 // q, k, v, dout (bf16) -> fp16 copies scaled by 2^e_X; 8 elements per thread
 // per step, the tensors in the reverse of the amax pass's order (the last
@@ -188,6 +267,10 @@ __device__ __forceinline__ void load_exps(const BwdArgs& a, int (&e)[4]) {
 __global__ void __launch_bounds__(256) bwd_convert_kernel(BwdArgs a, long long q8, long long k8) {
   int e[4];
   load_exps(a, e);
+  if (a.fp8) {
+    fp8_convert(a, e, q8);
+    return;
+  }
   if (blockIdx.x == 0 && threadIdx.x < 4) a.exps[threadIdx.x] = e[threadIdx.x];
   const Pow2 f[4] = {pow2_pair(e[0]), pow2_pair(e[1]), pow2_pair(e[2]), pow2_pair(e[3])};
   const long long total = 2 * q8 + 2 * k8;
@@ -222,8 +305,10 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdArgs a) {
   const long long rows = static_cast<long long>(a.B) * a.H * a.n_pad;
   const int nw = (gridDim.x * blockDim.x) >> 5;
   const bool packed = a.cu_q != nullptr;
-  const Pow2 f_v = pow2_pair(a.exps[2]), f_do = pow2_pair(a.exps[3]);
-  const float alpha = __int_as_float((127 - ds_shift(D)) << 23);
+  // FP8 backward: -D'' = -sum_c dO'_c O_c (O in its own units; the block
+  // scales enter in the main pass)
+  const Pow2 f_v = pow2_pair(a.fp8 ? 0 : a.exps[2]), f_do = pow2_pair(a.exps[3]);
+  const float alpha = a.fp8 ? 1.f : __int_as_float((127 - ds_shift(D)) << 23);
   for (long long pr = warp; pr < rows; pr += nw) {
     const long long bh = pr / a.n_pad;
     const int n = static_cast<int>(pr - bh * a.n_pad);
@@ -398,7 +483,13 @@ __device__ __forceinline__ uint32_t half_col(int kk) {
 // shuffle per element: the source lane of query 4b + c exposes, in round r,
 // word (c + r) % 4, which is what a lane needing word w reads in the round
 // with (w - r) % 4 = c.
-template <int D, bool PACKED, bool DROP>
+// FP8 ([B, H, N, d] form, d = 128, no dropout) runs the FP8 forward's
+// backward on its e4m3 codes (see fp8_convert): the score of (query i, key j)
+// is sq_i sk_j (codes), dP = 2^-e_do sv_j (dO' codes), and dS goes to the
+// operands as dS sq_i sk_j 2^tau, so dK_j = scale 2^-tau / sk_j (dS'^T q-codes)
+// and dQ_i = scale 2^-tau / sq_i (dS' k-codes); sq of a 64-query step and
+// sk, sv of a thread's key are one scale each.
+template <int D, bool PACKED, bool DROP, bool FP8 = false>
 __global__ void __launch_bounds__(512, 1)
 bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -700,7 +791,15 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const int key = kb * C::BK + r;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const BwdScales sc = bwd_scales<D>(a);
-    const float sl2 = sc.c_s;
+    const float sl2 = FP8 ? a.scale_log2 : sc.c_s;
+    // FP8: the block scales of this thread's key, and 2^(tau - e_do)
+    float f8_sk = 1.f, f8_sv = 1.f, f8_k0 = 1.f;
+    if constexpr (FP8) {
+      const int kblk = min(key / 64, a.nsb - 1);
+      f8_sk = a.sk[static_cast<size_t>(bh) * a.nsb + kblk];
+      f8_sv = a.sv[static_cast<size_t>(bh) * a.nsb + kblk];
+      f8_k0 = mul_pow2(1.f, a.exps[0] - a.exps[3]);
+    }
     bool ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_KV), 0, a.err, kSiteKV, abort_flag));
     if (ok) {
       // K row r: the A operand of S^T, packed two fp16 per TMEM column like the
@@ -727,6 +826,9 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       warp_arrive(bar(C::B_KT));
     }
     Walk wk = walk_start();
+    // FP8: sq of the next step, loaded one step ahead (the [B, H, N, d] walk
+    // goes through consecutive steps of one head)
+    float f8_sq_next = FP8 ? __ldg(a.sq + static_cast<size_t>(bh) * a.nsb + i0) : 1.f;
     for (int it = 0; it < n_it && ok; ++it, walk_next(wk)) {
       const int s = it % C::NS;
       const int buf = it & 1;
@@ -735,6 +837,10 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       if (warp == 4 && lane == 0) FA_TRACE(1, 2);
       if (!ok) break;
       tc_fence_after();
+      // FP8: sq of this step's 64 queries (one scale block)
+      const float f8_sq = f8_sq_next;
+      if constexpr (FP8)
+        if (wk.step + 1 < nq) f8_sq_next = __ldg(a.sq + static_cast<size_t>(bh) * a.nsb + wk.step + 1);
       uint32_t pk[C::NCH][16];                         // P^T, fp16 pairs of queries
       uint32_t zm[C::NCH];                             // bit e: (query qc + e, key) kept
 #pragma unroll
@@ -747,7 +853,8 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         uint32_t sr[32];
         tmem_ld32(s_addr, sr);
         tmem_ld_wait();
-        const uint64_t nsl2 = f2_pack(-sl2, -sl2);
+        const float sl2s = FP8 ? sl2 * f8_sq * f8_sk : sl2;
+        const uint64_t nsl2 = f2_pack(-sl2s, -sl2s);
         // queries qh + i, i in [lo, hi), see this key; the masked form runs only
         // in the steps where some lane of the warp has a masked query
         const int lo = a.causal ? key - off - qh : INT_MIN;
@@ -835,7 +942,10 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       // alpha (2^-(14 + log2 d)) brings dP' to the units of dS'; with dropout
       // it also carries 1 / q
       const float ga = DROP ? sc.alpha * a.drop_scale : sc.alpha;
-      const uint64_t ga2 = f2_pack(ga, ga);
+      // FP8: dS' = P o (2^(tau-e_do) sq sk) (sv dP' - D''); the D'' factor h
+      const float f8_h = f8_k0 * f8_sq * f8_sk;
+      const float gaf = FP8 ? f8_h * f8_sv : ga;
+      const uint64_t ga2 = f2_pack(gaf, gaf), h2 = f2_pack(f8_h, f8_h);
       float ds_max = 0.f;
 #pragma unroll
       for (int ch = 0; ch < C::NCH; ++ch) {
@@ -857,8 +967,13 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             g23 = f2_pack(__uint_as_float(z(e + 2)), __uint_as_float(z(e + 3)));
           }
           // dS' = P o (alpha dP' - D') on packed pairs
-          const uint64_t d01 = f2_fma(g01, ga2, f2_pack(dv4.x, dv4.y));
-          const uint64_t d23 = f2_fma(g23, ga2, f2_pack(dv4.z, dv4.w));
+          uint64_t nd01 = f2_pack(dv4.x, dv4.y), nd23 = f2_pack(dv4.z, dv4.w);
+          if constexpr (FP8) {
+            nd01 = f2_mul(nd01, h2);
+            nd23 = f2_mul(nd23, h2);
+          }
+          const uint64_t d01 = f2_fma(g01, ga2, nd01);
+          const uint64_t d23 = f2_fma(g23, ga2, nd23);
           const uint32_t pa = pk[ch][e / 2], pb = pk[ch][e / 2 + 1];
           float ds[4];
           f2_unpack(f2_mul(f2_pack(f16_lo(pa), f16_hi(pa)), d01), ds[0], ds[1]);
@@ -895,7 +1010,9 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                                    : (static_cast<size_t>(bh) * a.N + key) * D;
         const uint32_t src = tmem + lane_off + (h ? C::COL_DK : C::COL_DV);
         float* dst = (h ? a.dk : a.dv) + orow;
-        const float mul = h ? sc.dk : sc.dv;
+        float mul = h ? sc.dk : sc.dv;
+        if constexpr (FP8)
+          if (h) mul = mul_pow2(a.scale / f8_sk, -a.exps[0]);   // scale 2^-tau / sk
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t v[32];
@@ -918,8 +1035,10 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const int quarter = warp & 3;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const BwdScales bs = bwd_scales<D>(a);
-    const float sc = bs.dq1, sc2 = bs.dq2;
-    const bool two = sc2 != 1.f;
+    float sc = bs.dq1, sc2 = bs.dq2;
+    bool two = sc2 != 1.f;
+    const Pow2 f8_tau = pow2_pair(FP8 ? -a.exps[0] : 0);
+    float f8_sq_next = FP8 ? __ldg(a.sq + static_cast<size_t>(bh) * a.nsb + i0) : 1.f;
     float* stage = reinterpret_cast<float*>(smem + C::DQS_OFF + quarter * C::DQ_STAGE);
     const uint32_t stage_addr = base + C::DQS_OFF + quarter * C::DQ_STAGE;
     warp_arrive(bar(C::B_DQF));                      // phase 0: no dQ(-1) to drain
@@ -939,6 +1058,12 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       tmem_ld32(tmem + lane_off + C::COL_DQ + 32, v1);
       tmem_ld_wait();
       tc_fence_before();
+      if constexpr (FP8) {                           // scale 2^-tau / sq of this step
+        sc = a.scale / f8_sq_next * f8_tau.f1;
+        sc2 = f8_tau.f2;
+        two = true;
+        if (wq.step + 1 < nq) f8_sq_next = __ldg(a.sq + static_cast<size_t>(bh) * a.nsb + wq.step + 1);
+      }
       warp_arrive(bar(C::B_DQF));                    // dQ(it) read: counts for phase it+1
       if (warp == 12 && lane == 0) FA_TRACE(2, 3);
       if (two) {                                     // factor outside one float's range
@@ -1035,6 +1160,10 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(bwd_ts_kernel<D, false, true>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if constexpr (D == 128)
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(bwd_ts_kernel<D, false, false, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
@@ -1053,7 +1182,16 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   const int nk = ((a.cu_q ? a.max_k : a.N) + C::BK - 1) / C::BK;
   const int per_block = a.cu_q ? a.B * a.Hkv : a.B * a.H;   // CTAs per key block
   if (ev_main_begin != nullptr) cudaEventRecord(ev_main_begin, stream);
-  if (a.cu_q)
+  bool launched = false;
+  if constexpr (D == 128) {
+    if (a.fp8) {
+      bwd_ts_kernel<D, false, false, true><<<nk * per_block, C::THREADS, C::SMEM_BYTES, stream>>>(
+          tq, tk, tv, tdo, tdq, a);
+      launched = true;
+    }
+  }
+  if (launched) {
+  } else if (a.cu_q)
     bwd_ts_kernel<D, true, false><<<nk * per_block, C::THREADS, C::SMEM_BYTES, stream>>>(
         tq, tk, tv, tdo, tdq, a);
   else if (a.dropout)
@@ -1065,6 +1203,78 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   e = cudaGetLastError();
   if (ev_main_end != nullptr) cudaEventRecord(ev_main_end, stream);
   return e;
+}
+
+namespace {
+// In place x[r][:] <- x[r][:] R^T for 64-row tiles, d = 128. R^T sits in
+// shared memory as Rt[e][c] = R[c][e]; each of the 256 threads computes a
+// 4-row x 8-column block (rows 4 (t / 16) .., columns 8 (t % 16) ..) from float4
+// loads, 32 multiply-adds per 3 shared loads.
+constexpr int kRotThreads = 256;
+constexpr int kRotSmem = (128 * 128 + 64 * 128) * 4;
+__global__ void __launch_bounds__(kRotThreads) unrotate_kernel(float* x, const float* R,
+                                                                long long rows) {
+  extern __shared__ __align__(16) float rsm[];
+  float* Rt = rsm;                 // [e][c]
+  float* xs = rsm + 128 * 128;     // [64 rows][128]
+  for (int i = threadIdx.x; i < 128 * 128; i += kRotThreads) Rt[(i % 128) * 128 + i / 128] = R[i];
+  const int r4 = (threadIdx.x >> 4) * 4, c8 = (threadIdx.x & 15) * 8;
+  for (long long r0 = static_cast<long long>(blockIdx.x) * 64; r0 < rows;
+       r0 += static_cast<long long>(gridDim.x) * 64) {
+    const int nr = static_cast<int>(min(64ll, rows - r0));
+    __syncthreads();
+    for (int i = threadIdx.x; i < 64 * 32; i += kRotThreads)
+      reinterpret_cast<float4*>(xs)[i] =
+          i < nr * 32 ? reinterpret_cast<const float4*>(x + r0 * 128)[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    __syncthreads();
+    float y[4][8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) y[i][j] = 0.f;
+#pragma unroll 4
+    for (int e = 0; e < 128; e += 4) {
+      float4 xv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) xv[i] = *reinterpret_cast<const float4*>(xs + (r4 + i) * 128 + e);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float4 ra = *reinterpret_cast<const float4*>(Rt + (e + u) * 128 + c8);
+        const float4 rb = *reinterpret_cast<const float4*>(Rt + (e + u) * 128 + c8 + 4);
+        const float rv[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float xe = u == 0 ? xv[i].x : u == 1 ? xv[i].y : u == 2 ? xv[i].z : xv[i].w;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) y[i][j] = fmaf(xe, rv[j], y[i][j]);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (r4 + i < nr) {
+        float4* dst = reinterpret_cast<float4*>(x + (r0 + r4 + i) * 128 + c8);
+        dst[0] = make_float4(y[i][0], y[i][1], y[i][2], y[i][3]);
+        dst[1] = make_float4(y[i][4], y[i][5], y[i][6], y[i][7]);
+      }
+  }
+}
+}  // namespace
+
+cudaError_t launch_unrotate(float* x, const float* R, long long rows, cudaStream_t stream) {
+  static std::atomic<bool> attr_set[64];   // per device; racing first calls both set it
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(unrotate_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kRotSmem);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const long long tiles = (rows + 63) / 64;
+  const int grid = static_cast<int>(tiles < 148 * 2 ? tiles : 148 * 2);
+  unrotate_kernel<<<grid, kRotThreads, kRotSmem, stream>>>(x, R, rows);
+  return cudaGetLastError();
 }
 
 template cudaError_t launch_bwd<64>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,

@@ -93,6 +93,15 @@ struct BwdArgs {
   // d = 128, [B, H, N, d] form: (batch, head) slices per grid group (<= 0:
   // one group of all slices, key-block major over every head)
   int head_group = 0;
+  // FP8 backward (fp8 = 1, d = 128, [B, H, N, d] form): q, k, v are the FP8
+  // forward's e4m3 codes (q, k of the rotated inputs) with fp32 scales sq, sk,
+  // sv per 64-row block ([B][H][nsb]); the fp16 operand copies hold the codes
+  // themselves (exact), and the block scales are folded in fp32
+  int fp8 = 0;
+  const float* sq = nullptr;
+  const float* sk = nullptr;
+  const float* sv = nullptr;
+  int nsb = 0;
 };
 
 // Blocks of the backward's amax pass (the length of BwdArgs.amax_part / 4).
@@ -107,6 +116,10 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
                        const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a,
                        cudaStream_t stream, cudaEvent_t ev_main_begin = nullptr,
                        cudaEvent_t ev_main_end = nullptr);
+
+// x[r][:] <- x[r][:] R^T in place for rows r < rows of fp32 [rows][128] (the
+// FP8 backward's gradients of the rotated inputs back to the unrotated ones)
+cudaError_t launch_unrotate(float* x, const float* R, long long rows, cudaStream_t stream);
 
 struct DecodeArgs {
   const void* q;            // bf16 [S][Hq][d]

@@ -387,6 +387,34 @@ FA_API fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8,
                      void* stream);
 
 /*
+ * fa_bwd_fp8 — the backward of the FP8 forward ("FlashAttention系列优化",
+ * FlashAttentionV3 / FP低精度; 91haoming.cn repost, "FP8 低精度計算"; the
+ * pages give no FP8 backward). It returns the gradients with respect to the
+ * forward's own inputs q, k, v (before rotation and quantisation), treating
+ * the e4m3 block quantisation as the identity (straight through):
+ *   (dQ', dK', dV) = attention backward over Q' = q8 * sq, K' = k8 * sk,
+ *                    V = v8 * sv (the dequantised 64-row blocks), D from o,
+ *   dQ = dQ' R^T,  dK = dK' R^T    (R orthogonal: Q' = Q R).
+ *   q8, k8, v8, sq, sk, sv : exactly what fa_fp8_prepare returned (and
+ *                    fa_fwd_fp8 consumed); R the rotation given to it.
+ *   o, lse         : fa_fwd_fp8's outputs (bf16 BHND, fp32 [B][H][N]).
+ *   dout           : bf16 BHND; dq, dk, dv fp32 BHND outputs.
+ *   workspace      : >= fa_bwd_workspace_bytes(B, H, N, d) bytes.
+ * The products run on fp16 tensor-core operands: the e4m3 codes are fp16
+ * values exactly (so the recomputed scores are the forward's), dout is
+ * scaled by a power of two as in fa_bwd, and every block scale is applied in
+ * fp32. e4m3 gradient operands were not used: rounding dout to e4m3 alone
+ * moves dV by ~1 on the FP8 workload (tolerance 5e-2). The rotation back is a
+ * second pass over dq and dk.
+ * Errors: as fa_bwd; FA_ERR_UNSUPPORTED unless d = 128.
+ */
+FA_API fa_status fa_bwd_fp8(const void* q8, const void* k8, const void* v8, const float* sq,
+                            const float* sk, const float* sv, const float* R, const void* o,
+                            const float* lse, const void* dout, float* dq, float* dk, float* dv,
+                            void* workspace, size_t ws_bytes, int B, int H, int N, int d,
+                            int causal, void* stream);
+
+/*
  * Paged KV-cache block pool ("FlashAttention系列优化", PagedAttention: blocks
  * allocated on demand as tokens arrive; sequences of parallel sampling share
  * physical blocks through their block tables; a reference count per block and
