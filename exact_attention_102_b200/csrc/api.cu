@@ -273,8 +273,7 @@ fa_status bwd_dense(const void* q, const void* k, const void* v, const void* o, 
   if (e == cudaSuccess && f8 != nullptr) {
     // gradients of the rotated inputs -> of Q and K: dQ = dQ' R^T, dK = dK' R^T
     const long long rows = static_cast<long long>(bh) * N;
-    e = fa::launch_unrotate(dq, f8->R, rows, s);
-    if (e == cudaSuccess) e = fa::launch_unrotate(dk, f8->R, rows, s);
+    e = fa::launch_unrotate(dq, dk, f8->R, rows, a.err, s);
   }
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }

@@ -1206,62 +1206,180 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
 }
 
 namespace {
-// In place x[r][:] <- x[r][:] R^T for 64-row tiles, d = 128. R^T sits in
-// shared memory as Rt[e][c] = R[c][e]; each of the 256 threads computes a
-// 4-row x 8-column block (rows 4 (t / 16) .., columns 8 (t % 16) ..) from float4
-// loads, 32 multiply-adds per 3 shared loads.
+// In place x[r][:] <- x[r][:] R^T, d = 128, for two tensors of `rows` rows
+// each (the FP8 backward's dQ' and dK'), on the tensor core. Every fp32
+// operand v is split into bf16 terms hi = bf16(v), lo = bf16(v - hi), and the
+// product is hi_x hi_R + lo_x hi_R + hi_x lo_R with fp32 accumulation; the
+// dropped lo_x lo_R and the rounding of the lo terms leave a relative error
+// near 2^-16 of sum_e |x_e| |R_ce| per output.
+//
+// One tile = 128 rows. A (128 rows x K = 128) is the split x tile in TMEM,
+// written by the threads (two bf16 per column); B is the split R in shared
+// memory, K-major with the 128-byte swizzle (B row n = R row n, so
+// D[m][n] = sum_e x[m][e] R[n][e]); D is the fp32 accumulator in TMEM.
+// 8 warps: warp w reaches TMEM lanes 32 (w % 4) .. + 31 and takes head-dim
+// half w / 4 of the loads and of the stores, both in the 16 x 256 bit TMEM
+// shape, so that 4 neighbouring threads cover 64 (load) or 32 (store)
+// contiguous bytes of one row. Two CTAs per SM (64 KB of shared memory and
+// 256 TMEM columns each): one CTA's loads overlap the other's products, and
+// each CTA loads its next tile while its own products run.
 constexpr int kRotThreads = 256;
-constexpr int kRotSmem = (128 * 128 + 64 * 128) * 4;
-__global__ void __launch_bounds__(kRotThreads) unrotate_kernel(float* x, const float* R,
-                                                                long long rows) {
-  extern __shared__ __align__(16) float rsm[];
-  float* Rt = rsm;                 // [e][c]
-  float* xs = rsm + 128 * 128;     // [64 rows][128]
-  for (int i = threadIdx.x; i < 128 * 128; i += kRotThreads) Rt[(i % 128) * 128 + i / 128] = R[i];
-  const int r4 = (threadIdx.x >> 4) * 4, c8 = (threadIdx.x & 15) * 8;
-  for (long long r0 = static_cast<long long>(blockIdx.x) * 64; r0 < rows;
-       r0 += static_cast<long long>(gridDim.x) * 64) {
-    const int nr = static_cast<int>(min(64ll, rows - r0));
-    __syncthreads();
-    for (int i = threadIdx.x; i < 64 * 32; i += kRotThreads)
-      reinterpret_cast<float4*>(xs)[i] =
-          i < nr * 32 ? reinterpret_cast<const float4*>(x + r0 * 128)[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-    __syncthreads();
-    float y[4][8];
+// R hi, R lo, alignment and the barrier take 66.6 KB; the request is 80 KB so
+// that a third CTA (which would wait for TMEM columns) never shares an SM
+constexpr int kRotSmem = 80 * 1024;
+constexpr uint32_t kRotCols = 256;     // accumulator [0, 128), x hi [128, 192), x lo [192, 256)
+constexpr uint32_t kSiteRot = 0x41;
+
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf16x2(a, b);
+  lo = pack_bf16x2(a - __uint_as_float(hi << 16), b - __uint_as_float(hi & 0xffff0000u));
+}
+
+__global__ void __launch_bounds__(kRotThreads, 2) unrotate_kernel(float* x0, float* x1,
+                                                                   const float* __restrict__ R,
+                                                                   long long rows, uint32_t* err) {
+  extern __shared__ uint8_t rot_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(rot_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(sm);
+  const uint32_t bar = sbase + 65536;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + 65536 + 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + 65536 + 16);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // R -> bf16 hi / lo, K-major, 128-byte swizzle: K chunk e / 64 at 16 KB
+  // steps, row c at c * 128 B, 16-byte unit u of the row at unit u ^ (c % 8)
+  for (int u = threadIdx.x; u < 128 * 16; u += kRotThreads) {
+    const int c = u >> 4, e0 = (u & 15) * 8;
+    const float4 a = __ldg(reinterpret_cast<const float4*>(R + c * 128 + e0));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(R + c * 128 + e0 + 4));
+    uint4 h, l;
+    split_bf16x2(a.x, a.y, h.x, l.x);
+    split_bf16x2(a.z, a.w, h.y, l.y);
+    split_bf16x2(b.x, b.y, h.z, l.z);
+    split_bf16x2(b.z, b.w, h.w, l.w);
+    const uint32_t off = (e0 >> 6) * 16384 + c * 128 + ((((e0 & 63) >> 3) ^ (c & 7)) << 4);
+    *reinterpret_cast<uint4*>(sm + off) = h;
+    *reinterpret_cast<uint4*>(sm + 32768 + off) = l;
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), kRotCols);
+    tmem_relinquish();
+  }
+  fence_async_smem();     // R, written by the threads, seen by the tensor core
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const long long tiles_per = (rows + 127) / 128, tiles = 2 * tiles_per;
+  const int q = warp & 3, hh = warp >> 2, r_in = lane >> 2, cq = lane & 3;
+  const uint32_t id = idesc_f16(128, 128, 1, 0, 0);
+  const uint64_t dRh = smem_desc_sw128(sbase, 16, 1024);
+  const uint64_t dRl = smem_desc_sw128(sbase + 32768, 16, 1024);
+  auto add = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (bytes >> 4); };
+
+  // this thread's part of a tile: rows 32 q + 16 i + 8 s + r_in (i, s in
+  // {0, 1}); K groups j = 4 hh + g (g < 4), elements 16 j + 4 cq .. + 3
+  float4 xv[2][2][4];
+  auto load = [&](long long t) {
+    const float* X = t < tiles_per ? x0 : x1;
+    const long long r0 = (t < tiles_per ? t : t - tiles_per) * 128;
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 2; ++i)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) y[i][j] = 0.f;
-#pragma unroll 4
-    for (int e = 0; e < 128; e += 4) {
-      float4 xv[4];
+      for (int s2 = 0; s2 < 2; ++s2) {
+        const long long row = r0 + 32 * q + 16 * i + 8 * s2 + r_in;
+        const float4* src = reinterpret_cast<const float4*>(X + row * 128 + 64 * hh + 4 * cq);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) xv[i] = *reinterpret_cast<const float4*>(xs + (r4 + i) * 128 + e);
+        for (int g = 0; g < 4; ++g)
+          xv[i][s2][g] = row < rows ? __ldcs(src + 4 * g) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+  };
+
+  long long t = blockIdx.x;
+  if (t < tiles) load(t);
+  uint32_t phase = 0;
+  for (; t < tiles; t += gridDim.x) {
+    // split x into TMEM columns 128 + (K group) * 8 (hi) and 192 + .. (lo)
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float4 ra = *reinterpret_cast<const float4*>(Rt + (e + u) * 128 + c8);
-        const float4 rb = *reinterpret_cast<const float4*>(Rt + (e + u) * 128 + c8 + 4);
-        const float rv[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
+    for (int i = 0; i < 2; ++i) {
+      uint32_t hi[16], lo[16];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float xe = u == 0 ? xv[i].x : u == 1 ? xv[i].y : u == 2 ? xv[i].z : xv[i].w;
+      for (int g = 0; g < 4; ++g)
 #pragma unroll
-          for (int j = 0; j < 8; ++j) y[i][j] = fmaf(xe, rv[j], y[i][j]);
+        for (int s2 = 0; s2 < 2; ++s2) {
+          const float4 v = xv[i][s2][g];
+          split_bf16x2(v.x, v.y, hi[4 * g + 2 * s2], lo[4 * g + 2 * s2]);
+          split_bf16x2(v.z, v.w, hi[4 * g + 2 * s2 + 1], lo[4 * g + 2 * s2 + 1]);
         }
+      const uint32_t ta = tmem + (static_cast<uint32_t>(32 * q + 16 * i) << 16) + 32 * hh;
+      tmem_st_16x256b_x4(ta + 128, hi);
+      tmem_st_16x256b_x4(ta + 192, lo);
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int p = 0; p < 3; ++p) {
+        const uint32_t a_col = p == 1 ? 192 : 128;
+        const uint64_t b = p == 2 ? dRl : dRh;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_f16_ts(tmem, tmem + a_col + 8 * kk, add(b, (kk >> 2) * 16384 + (kk & 3) * 32), id,
+                      (p | kk) != 0);
+      }
+      umma_commit(bar);
+    }
+    const long long cur = t;
+    if (t + gridDim.x < tiles) load(t + gridDim.x);    // next tile, while the products run
+    const bool ok = mbar_wait(bar, phase, err, kSiteRot, abort_flag);
+    if (__syncthreads_or(!ok)) break;      // every thread leaves the loop together
+    phase ^= 1;
+    tc_fence_after();
+    float* X = cur < tiles_per ? x0 : x1;
+    const long long r0 = (cur < tiles_per ? cur : cur - tiles_per) * 128;
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) {
+      const int i = c4 >> 1, half = c4 & 1;
+      uint32_t v[16];
+      tmem_ld_16x256b_x4(
+          tmem + (static_cast<uint32_t>(32 * q + 16 * i) << 16) + 64 * hh + 32 * half, v);
+      tmem_ld_wait();
+      const long long ra = r0 + 32 * q + 16 * i + r_in, rb = ra + 8;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const int col = 64 * hh + 32 * half + 8 * g + 2 * cq;
+        if (ra < rows)
+          __stcs(reinterpret_cast<float2*>(X + ra * 128 + col),
+                 make_float2(__uint_as_float(v[4 * g]), __uint_as_float(v[4 * g + 1])));
+        if (rb < rows)
+          __stcs(reinterpret_cast<float2*>(X + rb * 128 + col),
+                 make_float2(__uint_as_float(v[4 * g + 2]), __uint_as_float(v[4 * g + 3])));
       }
     }
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (r4 + i < nr) {
-        float4* dst = reinterpret_cast<float4*>(x + (r0 + r4 + i) * 128 + c8);
-        dst[0] = make_float4(y[i][0], y[i][1], y[i][2], y[i][3]);
-        dst[1] = make_float4(y[i][4], y[i][5], y[i][6], y[i][7]);
-      }
+    tc_fence_before();
+  }
+  // a wait that gave up leaves products possibly in flight: wait for them
+  // (bounded) before the columns are freed
+  if (*abort_flag) mbar_wait(bar, phase, nullptr, kSiteRot, nullptr, 100000000ull);
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kRotCols);
   }
 }
 }  // namespace
 
-cudaError_t launch_unrotate(float* x, const float* R, long long rows, cudaStream_t stream) {
+cudaError_t launch_unrotate(float* x0, float* x1, const float* R, long long rows, uint32_t* err,
+                            cudaStream_t stream) {
   static std::atomic<bool> attr_set[64];   // per device; racing first calls both set it
   int dev = 0;
   cudaGetDevice(&dev);
@@ -1271,9 +1389,9 @@ cudaError_t launch_unrotate(float* x, const float* R, long long rows, cudaStream
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  const long long tiles = (rows + 63) / 64;
+  const long long tiles = 2 * ((rows + 127) / 128);
   const int grid = static_cast<int>(tiles < 148 * 2 ? tiles : 148 * 2);
-  unrotate_kernel<<<grid, kRotThreads, kRotSmem, stream>>>(x, R, rows);
+  unrotate_kernel<<<grid, kRotThreads, kRotSmem, stream>>>(x0, x1, R, rows, err);
   return cudaGetLastError();
 }
 

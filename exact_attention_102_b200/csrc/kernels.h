@@ -117,9 +117,11 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
                        cudaStream_t stream, cudaEvent_t ev_main_begin = nullptr,
                        cudaEvent_t ev_main_end = nullptr);
 
-// x[r][:] <- x[r][:] R^T in place for rows r < rows of fp32 [rows][128] (the
-// FP8 backward's gradients of the rotated inputs back to the unrotated ones)
-cudaError_t launch_unrotate(float* x, const float* R, long long rows, cudaStream_t stream);
+// x[r][:] <- x[r][:] R^T in place for rows r < rows of two fp32 [rows][128]
+// tensors x0, x1 (the FP8 backward's gradients of the rotated inputs back to
+// the unrotated ones); a wait that gives up records its site in *err
+cudaError_t launch_unrotate(float* x0, float* x1, const float* R, long long rows, uint32_t* err,
+                            cudaStream_t stream);
 
 struct DecodeArgs {
   const void* q;            // bf16 [S][Hq][d]
