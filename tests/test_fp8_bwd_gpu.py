@@ -10,7 +10,9 @@ derived from that arithmetic (with a factor 2 of slack on each term):
   dK'_jc: scale sum_i e_ij |Q'_ic|,  dQ'_ic: scale sum_j e_ij |K'_jc|, with
           e_ij = 2^-10 |dS_ij| + 2^-20 P_ij (|dP_ij| + |D_i|)
           (dS rounded to fp16; fp32 sums in dP and D)
-  dQ = dQ' R^T, dK = dK' R^T: the bound vector b of a row maps to b |R|^T;
+  dQ = dQ' R^T, dK = dK' R^T: the bound vector b of a row maps to b |R|^T
+          (the kernel's rotation, on split bf16 terms, adds a relative error
+          near 2^-16 of |dQ'| |R|^T, far inside the 2^-10 term);
 plus 1e-3 absolute. O and L are the oracle's (the forward's outputs are
 checked by tests/test_fp8_gpu.py).
 """
