@@ -210,17 +210,16 @@ fa_status bwd_dense(const void* q, const void* k, const void* v, const void* o, 
   void* v16 = w16 + 2 * tsz;
   void* do16 = w16 + 3 * tsz;
   CUtensorMap tq, tk, tv, tdo, tdq;
-  // d = 128 steps over 64 queries at a time (64-row Q / dO boxes), d = 64 over
-  // 128. The dQ reduce-add boxes: d = 128, 32 columns x 64 rows unswizzled
-  // (the drain writes a column per thread); d = 64, 32 columns x 32 rows with
-  // the 128-byte swizzle (a row per thread).
-  const uint32_t qrows = d == 128 ? 64 : 128;
+  // steps over 128 queries at a time (128-row Q / dO boxes). The dQ reduce-add
+  // boxes: 32 columns x 32 rows with the 128-byte swizzle (the drain writes a
+  // query row per thread).
+  const uint32_t qrows = 128;
   if (!make_map(&tq, q16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, qrows) ||
       !make_map(&tk, k16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, 128) ||
       !make_map(&tv, v16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, 128) ||
       !make_map(&tdo, do16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, qrows) ||
-      !make_map(&tdq, dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, N, bh, 32, d == 128 ? 64 : 32,
-                d == 128 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B))
+      !make_map(&tdq, dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, N, bh, 32, 32,
+                CU_TENSOR_MAP_SWIZZLE_128B))
     return FA_ERR_LAUNCH;
   fa::BwdArgs a;
   a.q16 = q16;
@@ -534,10 +533,10 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
   void* k16 = w16 + round256(nq * 2);
   void* v16 = w16 + round256(nq * 2) + round256(nk * 2);
   void* do16 = w16 + round256(nq * 2) + 2 * round256(nk * 2);
-  // token-major views [T][heads][d]; Q / dO boxes of one step's tokens (64 for
-  // d = 128, 128 for d = 64), K / V of 128, dQ reduce boxes as in fa_bwd
+  // token-major views [T][heads][d]; Q / dO boxes of one step's 128 tokens,
+  // K / V of 128, dQ reduce boxes as in fa_bwd
   CUtensorMap tq, tk, tv, tdo, tdq;
-  const uint32_t qrows = d == 128 ? 64 : 128;
+  const uint32_t qrows = 128;
   if (!make_map(&tq, q16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, H, total_q, 64, 1,
                 CU_TENSOR_MAP_SWIZZLE_128B, qrows) ||
       !make_map(&tk, k16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, Hkv, total_k, 64, 1,
@@ -547,8 +546,7 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
       !make_map(&tdo, do16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, H, total_q, 64, 1,
                 CU_TENSOR_MAP_SWIZZLE_128B, qrows) ||
       !make_map(&tdq, dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, H, total_q, 32, 1,
-                d == 128 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
-                d == 128 ? 64 : 32))
+                CU_TENSOR_MAP_SWIZZLE_128B, 32))
     return FA_ERR_LAUNCH;
   fa::BwdArgs a;
   a.q16 = q16;

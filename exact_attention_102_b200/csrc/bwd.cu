@@ -28,7 +28,7 @@
 // B200 mapping (one CTA per (batch*head, 128-key block), 512 threads; the
 // kernel is bwd_ts_kernel below, templated on d = 64 / 128):
 //   warp 0       TMA producer: K_j, V_j once; Q_i, dO_i, L_i, D_i per step of
-//                64 (d = 128) or 128 (d = 64) queries through a ring.
+//                128 queries, each refilled as soon as its last reader is done.
 //   warp 1       TMEM allocation; lane 0 issues every tcgen05.mma: S^T, dP^T,
 //                dV, dK and dQ (see "main pass on TMEM operands").
 //   warps 4..11  thread = key row (TMEM lane), two warps per lane quarter,
@@ -36,8 +36,8 @@
 //                written back into TMEM as the A operand of dV / dK, dS^T also
 //                into shared memory for the dQ product; at the end the dK and
 //                dV rows.
-//   warps 12..15 read the step's dQ tile out of TMEM and add it to dQ in HBM
-//                with TMA tensor reduce-adds.
+//   warps 12..15 thread = query row: read the step's dQ tile out of TMEM and
+//                add it to dQ in HBM with TMA tensor reduce-adds.
 #include <climits>
 #include <type_traits>
 
@@ -382,85 +382,114 @@ __device__ __forceinline__ BwdScales bwd_scales(const BwdArgs& a) {
 }
 
 // --------------------------------- main pass on TMEM operands, d = 64 / 128
-// Same method, tiled around what the tensor core does fastest: an MMA whose A
-// operand sits in TMEM runs at the full rate for N = 128, one whose A operand
-// is read from shared memory costs about twice as long for N <= 128. Every
-// operand that can live in TMEM does. Steps of BQ queries (64 for d = 128,
-// 128 for d = 64, so that some form of the dQ product has M = 128):
-//   S^T  = K_j Q_i^T      A = K_j   (TMEM, loaded once per CTA), B = Q_i
-//   dP^T = V_j dO_i^T     A = V_j   (shared memory),              B = dO_i
-//   dV  += P^T dO_i       A = P^T   (TMEM, written over S^T),     B = dO_i
-//   dK  += dS^T Q_i       A = dS^T  (TMEM, written over dP^T),    B = Q_i
-//   d = 128: dQ^T = K_j^T dS^T   A = K_j^T (shared, MN-major), B = dS^T (shared)
-//   d = 64:  dQ   = dS K_j       A = dS (shared, MN-major),    B = K_j (shared, MN-major)
-// TMEM, d = 128: K [0,64)  S^T/P^T [64,128)  dP^T/dS^T [128,192)  dQ^T [192,256)
-//                dV [256,384)  dK [384,512)
+// Same method, tiled around what the tensor core does fastest. Measured on
+// this part: a tcgen05.mma with M = 128 and N = 64 costs about as long as
+// one with N = 128, so every product here has N = 128 (d = 128) or N = d
+// (d = 64), over steps of BQ = 128 queries:
+//   S^T  = K_j Q_i^T      A = K_j  (d = 64: TMEM; d = 128: shared), B = Q_i
+//   dP^T = V_j dO_i^T     A = V_j  (shared memory),                 B = dO_i
+//   dV  += P^T dO_i       A = P^T  (TMEM, written over S^T),        B = dO_i
+//   dK  += dS^T Q_i       A = dS^T (TMEM, written over dP^T),       B = Q_i
+//   dQ   = dS K_j         A = dS   (shared, MN-major),              B = K_j (shared, MN-major)
+// TMEM, d = 128: S^T/P^T [0,128)  dP^T/dS^T, then dQ [128,256)  dV [256,384)
+//                dK [384,512): 640 columns of state in 512, because dQ(i)
+//                lands over dS^T(i) once dK(i) has read it, and dP^T(i+1)
+//                waits for the drain warps to have read dQ(i).
 //      d = 64:   K [0,32)  S^T/P^T [64,192)  dP^T/dS^T [192,320)  dQ [320,384)
 //                dV [384,448)  dK [448,512)
-// One tcgen05 issuer executes in issue order, so S^T(i+2) may be issued right
-// after dV(i+1) (which reads P^T(i+1) from the same columns) and dP^T(i+1)
-// right after dK(i) (which reads dS^T(i)); per step the issue order is
-// dK(i), dP^T(i+1), dV(i+1), S^T(i+2), dQ(i).
+// One tcgen05 issuer executes in issue order, so a product may overwrite
+// columns that the product issued just before it reads. Per step:
+//   d = 64:  dK(i), dP^T(i+1), dV(i+1), S^T(i+2), dQ(i)
+//   d = 128: dK(i) (its first half as soon as the first 32-query chunk of
+//            each half of dS(i) is in), dQ(i), [drain of dQ(i)] dP^T(i+1),
+//            dV(i+1), S^T(i+2)
+// The d = 128 chain dP^T -> dS -> dK -> dQ -> drain -> dP^T bounds the step;
+// the exp work of P(i+1) runs beside it.
 // Warps 4..11 (two per TMEM lane quarter, one per half of the step's queries)
 // compute P and then dS for their half, 32 queries at a time; dS also goes to
-// shared memory (double-buffered) for the dQ product. Warps 12..15 drain the
-// dQ tile to a shared staging box and add it to dQ in HBM with a TMA tensor
-// reduce-add: d = 128, thread = head-dim column, one 32-column x 64-row box
-// per warp; d = 64, thread = query row, two 32-column x 32-row boxes per warp,
-// one after the other through one staging box (128-byte swizzled, so the
-// row-per-thread writes meet no bank conflicts).
+// shared memory for the dQ product. Warps 12..15 drain dQ (thread = query
+// row) through 32-column x 32-row fp32 boxes with the 128-byte swizzle (so the
+// row-per-thread writes meet no bank conflicts), added to dQ in HBM by TMA
+// tensor reduce-adds: d = 128, two boxes per warp, the four column chunks in
+// two rounds; d = 64, one box, the two chunks in turn.
 template <int D_>
 struct BwdTs {
   static constexpr int D = D_;
+  // d = 128 ("wide"): S^T, dP^T and dQ are N = 128 products over 128-query
+  // steps; K stays out of TMEM (S^T reads it from shared memory) and dQ lands
+  // over the dP^T / dS^T columns once dK has read dS, so that 4 x 128
+  // columns hold S^T, dP^T (then dQ), dV and dK.
+  static constexpr bool WIDE = D == 128;
   static constexpr int BK = 128;                 // keys per CTA
-  static constexpr int BQ = D == 128 ? 64 : 128; // queries per step
+  static constexpr int BQ = 128;                 // queries per step
   static constexpr int HQ = BQ / 2;              // queries per half (one P / dS warp)
   static constexpr int NCH = HQ / 32;            // 32-query chunks per half
   static constexpr int KV_TILE = 128 * D * 2;    // K or V tile (D / 64 column chunks)
   static constexpr int KV_CHUNK = 128 * 128;
   static constexpr int Q_TILE = BQ * D * 2;      // Q or dO tile (D / 64 chunks of BQ rows)
   static constexpr int Q_CHUNK = BQ * 128;
-  // Q / dO stages: at least 3, because S^T(i+2) is issued (and waits for its
-  // stage) before dQ(i), whose completion frees stage i
-  static constexpr int NS = 3;
+  // Q / dO stages. d = 64: at least 3, because S^T(i+2) is issued (and waits
+  // for its stage) before dQ(i), whose completion frees stage i. Wide: Q
+  // takes 2 (Q_i is freed by dK(i), issued before S^T(i+2)) and dO one
+  // buffer (dO_i is last read by dV(i), dO_i+1 first by dP^T(i+1), issued
+  // after dK(i), dQ(i) and the drain of dQ(i)).
+  static constexpr int NS = WIDE ? 2 : 3;
+  static constexpr int NSG = WIDE ? 1 : NS;      // dO buffers
   static constexpr int DS_CHUNK = BK * 128;      // 64 queries of dS^T: one 128 B row per key
   static constexpr int DS_BYTES = BK * BQ * 2;   // dS^T fp16 [key][BQ queries]
-  // per drain warp: d = 128, [64 queries][32 columns]; d = 64, one [32
-  // queries][32 columns] box, used for the two column halves in turn
-  static constexpr int DQ_STAGE = D == 128 ? BQ * 32 * 4 : 32 * 32 * 4;
+  static constexpr int NDS = WIDE ? 1 : 2;       // dS buffers
+  // dQ staging: [32 queries][32 columns] fp32 boxes with the 128-byte
+  // swizzle, a query row per drain thread; wide, two per drain warp (the
+  // four column chunks in two rounds), d = 64 one (its two chunks in turn).
+  static constexpr int NBOX = WIDE ? 2 : 1;
+  static constexpr int DQ_STAGE = NBOX * 32 * 32 * 4;
+  // L log2(e) and -D' of a step: d = 64, one per stage, loaded with it;
+  // wide, one buffer each, refilled once its last reader is done (L(i+1)
+  // after P(i), D(i+1) after dS(i)), a step ahead of its next reader
+  static constexpr int LD_BYTES = (WIDE ? 1 : NS) * BQ * 4;
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = K_OFF + KV_TILE;
   static constexpr int Q_OFF = V_OFF + KV_TILE;
   static constexpr int DO_OFF = Q_OFF + NS * Q_TILE;
-  static constexpr int DS_OFF = DO_OFF + NS * Q_TILE;   // 2 buffers
-  static constexpr int DQS_OFF = DS_OFF + 2 * DS_BYTES; // 4 staging boxes
-  static constexpr int L_OFF = DQS_OFF + 4 * DQ_STAGE;  // NS x BQ fp32: L * log2(e)
-  static constexpr int DL_OFF = L_OFF + NS * BQ * 4;    // NS x BQ fp32: -D'
-  static constexpr int BAR_OFF = DL_OFF + NS * BQ * 4;
-  // B_STEP[s]: committed after the dQ product of the step held in stage s;
-  // every product of that step is then complete: the Q / dO stage and the dS
-  // buffer are free and the dQ tile is ready.
-  // B_FULL[s]: Q, L, dO and D of the step in stage s have landed.
+  static constexpr int DS_OFF = DO_OFF + NSG * Q_TILE;
+  static constexpr int DQS_OFF = DS_OFF + NDS * DS_BYTES; // the drain warps' staging boxes
+  static constexpr int L_OFF = DQS_OFF + 4 * DQ_STAGE;
+  static constexpr int DL_OFF = L_OFF + LD_BYTES;
+  static constexpr int BAR_OFF = DL_OFF + LD_BYTES;
+  // B_FULL[s]: Q (d = 64: also dO, L and D) of the step in stage s landed.
+  // B_STEP[s]: stage s is free again. d = 64: committed after the dQ product
+  // of the step (the dS buffer and the dQ tile are then ready too); wide:
+  // after its dK product.
   // B_DS: phase i completes when the 8 softmax-gradient warps have written
-  // dS(i). B_DQF: phase i completes when the 4 drain warps have read dQ(i-1)
-  // out of TMEM, so that dQ(i) may overwrite it. dK(i) waits on the first,
-  // dQ(i) on the second: the drain of dQ(i-1) runs while dK(i), dP(i+1),
-  // dV(i+1) and S(i+2) keep the tensor pipe busy.
+  // dS(i). B_DQF: phase i completes when the 4 drain warps have read dQ out of
+  // TMEM (d = 64: dQ(i-1), so that dQ(i) may overwrite it; wide: dQ(i), so
+  // that dP^T(i+1) may). Wide only: B_DQD, committed after dQ(i); B_GFULL,
+  // dO of step i landed; B_DOF, committed after dV(i) (the dO buffer is free);
+  // B_LFULL, B_DFULL: L and D of step i landed. B_DS0: the first 32-query
+  // chunk of each half of dS(i) is in TMEM (queries 0-31 and 64-95), so that
+  // dK(i) may start on them while the second chunks are computed.
   static constexpr int B_KV = 0, B_FULL = 1, B_STEP = B_FULL + NS;
   static constexpr int B_KT = B_STEP + NS, B_ST = B_KT + 1, B_DPT = B_ST + 1, B_P = B_DPT + 1;
-  static constexpr int B_DS = B_P + 1, B_DQF = B_DS + 1;
-  static constexpr int B_END = B_DQF + 1, B_DRAIN = B_END + 1, NBAR = B_DRAIN + 1;
+  static constexpr int B_DS = B_P + 1, B_DQF = B_DS + 1, B_DQD = B_DQF + 1, B_GFULL = B_DQD + 1;
+  static constexpr int B_DOF = B_GFULL + 1, B_LFULL = B_DOF + 1, B_DFULL = B_LFULL + 1;
+  static constexpr int B_DS0 = B_DFULL + 1;
+  static constexpr int B_END = B_DS0 + 1, B_DRAIN = B_END + 1, NBAR = B_DRAIN + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
-  static constexpr uint32_t COL_K = 0, COL_S = 64, COL_DP = COL_S + BQ, COL_DQ = COL_DP + BQ,
-                            COL_DV = COL_DQ + 64, COL_DK = COL_DV + D;
+  // TMEM. Wide: S^T/P^T [0,128)  dP^T/dS^T, then dQ [128,256)  dV [256,384)
+  // dK [384,512). d = 64: K [0,32)  S^T/P^T [64,192)  dP^T/dS^T [192,320)
+  // dQ [320,384)  dV [384,448)  dK [448,512).
+  static constexpr uint32_t COL_K = 0, COL_S = WIDE ? 0 : 64, COL_DP = COL_S + BQ,
+                            COL_DQ = WIDE ? COL_DP : COL_DP + BQ,
+                            COL_DV = WIDE ? COL_DP + BQ : COL_DQ + 64, COL_DK = COL_DV + D;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int THREADS = 512;
 };
 static_assert(BwdTs<128>::SMEM_BYTES <= 232448, "d = 128 backward exceeds shared memory");
 static_assert(BwdTs<64>::SMEM_BYTES <= 232448, "d = 64 backward exceeds shared memory");
 static_assert(BwdTs<128>::COL_DK + 128 == 512 && BwdTs<64>::COL_DK + 64 == 512, "TMEM plan");
-static_assert(BwdTs<64>::DQS_OFF % 1024 == 0, "swizzled staging boxes need 1024 B alignment");
+static_assert(BwdTs<64>::DQS_OFF % 1024 == 0 && BwdTs<128>::DQS_OFF % 1024 == 0,
+              "swizzled staging boxes need 1024 B alignment");
 
 constexpr int kOrderMaxB = 256;   // packed backward: sequences ordered by query length
 static_assert(BwdTs<128>::DS_BYTES >= 4 * (kOrderMaxB + 1), "order list exceeds the dS buffer");
@@ -487,7 +516,7 @@ __device__ __forceinline__ uint32_t half_col(int kk) {
 // backward on its e4m3 codes (see fp8_convert): the score of (query i, key j)
 // is sq_i sk_j (codes), dP = 2^-e_do sv_j (dO' codes), and dS goes to the
 // operands as dS sq_i sk_j 2^tau, so dK_j = scale 2^-tau / sk_j (dS'^T q-codes)
-// and dQ_i = scale 2^-tau / sq_i (dS' k-codes); sq of a 64-query step and
+// and dQ_i = scale 2^-tau / sq_i (dS' k-codes); sq of a 64-query block and
 // sk, sv of a thread's key are one scale each.
 template <int D, bool PACKED, bool DROP, bool FP8 = false>
 __global__ void __launch_bounds__(512, 1)
@@ -611,6 +640,12 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     mbar_init(bar(C::B_P), 8);
     mbar_init(bar(C::B_DS), 8);       // the 8 softmax-gradient warps
     mbar_init(bar(C::B_DQF), 4);      // the 4 drain warps
+    mbar_init(bar(C::B_DQD), 1);
+    mbar_init(bar(C::B_GFULL), 1);
+    mbar_init(bar(C::B_DOF), 1);
+    mbar_init(bar(C::B_LFULL), 1);
+    mbar_init(bar(C::B_DFULL), 1);
+    mbar_init(bar(C::B_DS0), 8);
     mbar_init(bar(C::B_END), 1);
     mbar_init(bar(C::B_DRAIN), 1);
     *abort_flag = 0;
@@ -639,7 +674,7 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         tma_load_3d(base + C::K_OFF + c * C::KV_CHUNK, &tmK, bar(C::B_KV), c * 64, ky, kz);
         tma_load_3d(base + C::V_OFF + c * C::KV_CHUNK, &tmV, bar(C::B_KV), c * 64, ky, kz);
       }
-      int issued = 0;
+      int issued = 0, g_issued = 0, l_issued = 0, d_issued = 0;
       Walk w = walk_start();
       for (int it = 0; it < n_it; ++it, walk_next(w)) {
         const int s = it % C::NS;
@@ -651,20 +686,50 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const int qy = packed ? hq : row, qz = packed ? tq0 + row : bh;
         if (!mbar_wait(bar(C::B_STEP + s), ph, a.err, kSiteQE, abort_flag)) break;
         const uint32_t full = bar(C::B_FULL + s);
-        mbar_arrive_expect_tx(full, 2 * (C::Q_TILE + C::BQ * 4));
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(base + C::Q_OFF + s * C::Q_TILE + c * C::Q_CHUNK, &tmQ, full, c * 64, qy, qz);
-        bulk_load(base + C::L_OFF + s * C::BQ * 4, a.lse_log2 + prow, C::BQ * 4, full);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(base + C::DO_OFF + s * C::Q_TILE + c * C::Q_CHUNK, &tmDO, full, c * 64, qy,
-                      qz);
-        bulk_load(base + C::DL_OFF + s * C::BQ * 4, a.delta + prow, C::BQ * 4, full);
-        issued = it + 1;
+        if constexpr (C::WIDE) {
+          mbar_arrive_expect_tx(full, C::Q_TILE);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(base + C::Q_OFF + s * C::Q_TILE + c * C::Q_CHUNK, &tmQ, full, c * 64, qy, qz);
+          issued = it + 1;
+          // dO_it into the one dO buffer once dV(it-1) has read dO_it-1
+          if (it >= 1 && !mbar_wait(bar(C::B_DOF), (it - 1) & 1, a.err, kSiteQE, abort_flag)) break;
+          mbar_arrive_expect_tx(bar(C::B_GFULL), C::Q_TILE);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(base + C::DO_OFF + c * C::Q_CHUNK, &tmDO, bar(C::B_GFULL), c * 64, qy, qz);
+          g_issued = it + 1;
+          // L_it once P(it-1) is done with the L buffer, D_it once dS(it-1)
+          // is done with the D buffer
+          if (it >= 1 && !mbar_wait(bar(C::B_P), (it - 1) & 1, a.err, kSiteQE, abort_flag)) break;
+          mbar_arrive_expect_tx(bar(C::B_LFULL), C::BQ * 4);
+          bulk_load(base + C::L_OFF, a.lse_log2 + prow, C::BQ * 4, bar(C::B_LFULL));
+          l_issued = it + 1;
+          if (it >= 1 && !mbar_wait(bar(C::B_DS), (it - 1) & 1, a.err, kSiteQE, abort_flag)) break;
+          mbar_arrive_expect_tx(bar(C::B_DFULL), C::BQ * 4);
+          bulk_load(base + C::DL_OFF, a.delta + prow, C::BQ * 4, bar(C::B_DFULL));
+          d_issued = it + 1;
+        } else {
+          mbar_arrive_expect_tx(full, 2 * (C::Q_TILE + C::BQ * 4));
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(base + C::Q_OFF + s * C::Q_TILE + c * C::Q_CHUNK, &tmQ, full, c * 64, qy, qz);
+          bulk_load(base + C::L_OFF + s * C::BQ * 4, a.lse_log2 + prow, C::BQ * 4, full);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(base + C::DO_OFF + s * C::Q_TILE + c * C::Q_CHUNK, &tmDO, full, c * 64, qy,
+                        qz);
+          bulk_load(base + C::DL_OFF + s * C::BQ * 4, a.delta + prow, C::BQ * 4, full);
+          issued = it + 1;
+        }
       }
+      // no copy may still be in flight when the CTA exits
       for (int it = max(0, issued - C::NS); it < issued; ++it) {
         mbar_wait(bar(C::B_FULL + it % C::NS), (it / C::NS) & 1, a.err, kSiteDrain, nullptr,
                   200000000ull);
       }
+      if (g_issued > 0)
+        mbar_wait(bar(C::B_GFULL), (g_issued - 1) & 1, a.err, kSiteDrain, nullptr, 200000000ull);
+      if (l_issued > 0)
+        mbar_wait(bar(C::B_LFULL), (l_issued - 1) & 1, a.err, kSiteDrain, nullptr, 200000000ull);
+      if (d_issued > 0)
+        mbar_wait(bar(C::B_DFULL), (d_issued - 1) & 1, a.err, kSiteDrain, nullptr, 200000000ull);
       mbar_wait(bar(C::B_KV), 0, a.err, kSiteDrain, nullptr, 200000000ull);
     }
   } else if (warp == 1) {
@@ -672,23 +737,23 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     if (lane == 0) {
       constexpr uint32_t idS = idesc_f16(128, C::BQ, 0, 0, 0);   // S^T, dP^T: K-major operands
       constexpr uint32_t idKM = idesc_f16(128, D, 0, 0, 1);      // dV, dK: A tmem, B MN-major
-      // dQ: d = 128, dQ^T (M = d, N = BQ), A = K^T and B = dS^T MN-major;
-      //     d = 64,  dQ   (M = BQ, N = d), A = dS and B = K MN-major
-      constexpr uint32_t idQ = D == 128 ? idesc_f16(128, C::BQ, 0, 1, 1) : idesc_f16(128, D, 0, 1, 1);
+      // dQ (M = BQ, N = d): A = dS and B = K, both MN-major
+      constexpr uint32_t idQ = idesc_f16(128, D, 0, 1, 1);
       // descriptors of the fixed tiles and of stage / buffer 0; a tile at a
       // byte offset is the base descriptor plus offset / 16 (start-address field)
       const uint64_t dV = smem_desc_sw128(base + C::V_OFF, 16, 1024);            // V, K-major
+      const uint64_t dKk = smem_desc_sw128(base + C::K_OFF, 16, 1024);           // K, K-major
       const uint64_t dKt = smem_desc_sw128(base + C::K_OFF, C::KV_CHUNK, 1024);  // K, MN-major
       const uint64_t dQk = smem_desc_sw128(base + C::Q_OFF, 16, 1024);           // Q, K-major
       const uint64_t dQm = smem_desc_sw128(base + C::Q_OFF, C::Q_CHUNK, 1024);   // Q, MN-major
       const uint64_t dGk = smem_desc_sw128(base + C::DO_OFF, 16, 1024);          // dO, K-major
       const uint64_t dGm = smem_desc_sw128(base + C::DO_OFF, C::Q_CHUNK, 1024);  // dO, MN-major
-      // dS^T, MN-major: d = 128, the B operand of dQ^T (N = 64, one block of 64
-      // queries); d = 64, the A operand of dQ (M = 128, two blocks DS_CHUNK apart)
-      const uint64_t dDS = smem_desc_sw128(base + C::DS_OFF, D == 128 ? 16 : C::DS_CHUNK, 1024);
+      // dS^T, MN-major over two 64-query blocks DS_CHUNK apart: the A operand
+      // of dQ (M = 128)
+      const uint64_t dDS = smem_desc_sw128(base + C::DS_OFF, C::DS_CHUNK, 1024);
       auto add = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (bytes >> 4); };
-      bool ok = mbar_wait(bar(C::B_KV), 0, a.err, kSiteKV, abort_flag) &&
-                mbar_wait(bar(C::B_KT), 0, a.err, kSiteKV, abort_flag);
+      bool ok = mbar_wait(bar(C::B_KV), 0, a.err, kSiteKV, abort_flag);
+      if constexpr (!C::WIDE) ok = ok && mbar_wait(bar(C::B_KT), 0, a.err, kSiteKV, abort_flag);
       auto issue_s = [&](int it) -> bool {
         const int s = it % C::NS;
         if (!mbar_wait(bar(C::B_FULL + s), (it / C::NS) & 1, a.err, kSiteQF, abort_flag))
@@ -696,16 +761,25 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         tc_fence_after();
         const uint64_t q = add(dQk, s * C::Q_TILE);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)   // K = d: chunk kk/4, 32 B steps inside it
-          umma_f16_ts(tmem + C::COL_S, tmem + C::COL_K + kk * 8,
-                      add(q, (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32), idS, kk > 0);
+        for (int kk = 0; kk < D / 16; ++kk) {  // K = d: chunk kk/4, 32 B steps inside it
+          const uint32_t kb_off = (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32;
+          if constexpr (C::WIDE)
+            umma_f16_ss(tmem + C::COL_S, add(dKk, (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32),
+                        add(q, kb_off), idS, kk > 0);
+          else
+            umma_f16_ts(tmem + C::COL_S, tmem + C::COL_K + kk * 8, add(q, kb_off), idS, kk > 0);
+        }
         umma_commit(bar(C::B_ST));
         return true;
       };
-      // dP^T(it): stage it % NS was waited for by issue_s(it), issued before
+      // dP^T(it). d = 64: stage it % NS was waited for by issue_s(it), issued
+      // before; wide: dO_it has its own barrier
       auto issue_dp = [&](int it) -> bool {
-        const int s = it % C::NS;
-        const uint64_t g = add(dGk, s * C::Q_TILE);
+        if constexpr (C::WIDE) {
+          if (!mbar_wait(bar(C::B_GFULL), it & 1, a.err, kSiteQF, abort_flag)) return false;
+          tc_fence_after();
+        }
+        const uint64_t g = add(dGk, (it % C::NSG) * C::Q_TILE);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           umma_f16_ss(tmem + C::COL_DP, add(dV, (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32),
@@ -717,21 +791,65 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       auto issue_dv = [&](int it) -> bool {
         if (!mbar_wait(bar(C::B_P), it & 1, a.err, kSiteP, abort_flag)) return false;
         tc_fence_after();
-        const uint64_t gm = add(dGm, (it % C::NS) * C::Q_TILE);
+        const uint64_t gm = add(dGm, (it % C::NSG) * C::Q_TILE);
         const uint32_t acc0 = it > 0 ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < C::BQ / 16; ++kk)
           umma_f16_ts(tmem + C::COL_DV, tmem + C::COL_S + half_col(kk), add(gm, kk * 2048), idKM,
                       kk > 0 ? 1u : acc0);
+        if constexpr (C::WIDE) umma_commit(bar(C::B_DOF));   // dO buffer free once dV(it) ran
         return true;
       };
+      // dK(it) += dS^T(it) Q_it: after dS(it) is in TMEM (B_DS phase it).
+      // Wide: the 16-query groups of the halves' first chunks (0, 1, 4, 5)
+      // go as soon as those chunks are in (B_DS0), the others after B_DS.
+      auto issue_dk = [&](int it) -> bool {
+        const uint64_t qm = add(dQm, (it % C::NS) * C::Q_TILE);
+        const uint32_t acc0 = it > 0 ? 1u : 0u;
+        if constexpr (C::WIDE) {
+          if (!mbar_wait(bar(C::B_DS0), it & 1, a.err, kSiteDS, abort_flag)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int kk = (g >> 1) * 4 + (g & 1);
+            umma_f16_ts(tmem + C::COL_DK, tmem + C::COL_DP + half_col(kk), add(qm, kk * 2048),
+                        idKM, g > 0 ? 1u : acc0);
+          }
+          if (!mbar_wait(bar(C::B_DS), it & 1, a.err, kSiteDS, abort_flag)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int kk = (g >> 1) * 4 + (g & 1) + 2;
+            umma_f16_ts(tmem + C::COL_DK, tmem + C::COL_DP + half_col(kk), add(qm, kk * 2048),
+                        idKM, 1u);
+          }
+        } else {
+          if (!mbar_wait(bar(C::B_DS), it & 1, a.err, kSiteDS, abort_flag)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < C::BQ / 16; ++kk)
+            umma_f16_ts(tmem + C::COL_DK, tmem + C::COL_DP + half_col(kk), add(qm, kk * 2048), idKM,
+                        kk > 0 ? 1u : acc0);
+        }
+        return true;
+      };
+      // dQ(it) over the 128 keys, B / A = dS(it) in buffer it % NDS
+      auto issue_dq = [&](int it) {
+        const uint64_t ds = add(dDS, (it % C::NDS) * C::DS_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < C::BK / 16; ++kk)
+          umma_f16_ss(tmem + C::COL_DQ, add(ds, kk * 2048), add(dKt, kk * 2048), idQ,
+                      kk > 0 ? 1u : 0u);
+      };
       // Issue order: S(0), dP(0), dV(0), S(1), then per step it
-      //   dK(it), dP(it+1), dV(it+1), S(it+2), dQ(it)
-      // Each wait (P(it+1) before dV(it+1), dS(it) before dK(it)) falls while
-      // the product issued before it is still running, so the pipe stays fed.
-      // In-order execution makes the overwrites safe: S(it+2) comes after
-      // dV(it+1) (which reads P(it+1) from the S columns), dP(it+1) after dK(it)
-      // (which reads dS(it) from the dP columns).
+      //   d = 64: dK(it), dP(it+1), dV(it+1), S(it+2), dQ(it)
+      //   wide:   dK(it), dQ(it), dP(it+1), dV(it+1), S(it+2)
+      // Each wait (P(it+1) before dV(it+1), dS(it) before dK(it), and, wide,
+      // the drain of dQ(it) before dP(it+1)) falls while products issued
+      // before it are still running. In-order execution makes the overwrites
+      // safe: S(it+2) comes after dV(it+1) (which reads P(it+1) from the S
+      // columns); dP(it+1) after dK(it) (which reads dS(it) from the dP
+      // columns); wide, dQ(it) lands over the dP columns after dK(it) too.
       if (ok) {
         tc_fence_after();
         ok = issue_s(0) && issue_dp(0) && issue_dv(0);
@@ -739,44 +857,47 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       }
       for (int it = 0; it < n_it && ok; ++it) {
         const int s = it % C::NS;
-        const uint64_t qm = add(dQm, s * C::Q_TILE);
-        const uint64_t ds = add(dDS, (it & 1) * C::DS_BYTES);
-        const uint32_t acc0 = it > 0 ? 1u : 0u;
-        // dK += dS^T Q_it (B_DS phase it: dS(it) written)
         FA_TRACE(0, 1);
-        ok = mbar_wait(bar(C::B_DS), it & 1, a.err, kSiteDS, abort_flag);
+        ok = issue_dk(it);
         FA_TRACE(0, 2);
         if (!ok) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < C::BQ / 16; ++kk)
-          umma_f16_ts(tmem + C::COL_DK, tmem + C::COL_DP + half_col(kk), add(qm, kk * 2048), idKM,
-                      kk > 0 ? 1u : acc0);
-        if (it + 1 < n_it) {
+        if constexpr (C::WIDE) {
+          umma_commit(bar(C::B_STEP + s));           // stage s free once dK(it) has run
+          issue_dq(it);
+          umma_commit(bar(C::B_DQD));                // dQ(it) ready, dS buffer read
           FA_TRACE(0, 3);
-          ok = issue_dp(it + 1);
-          FA_TRACE(0, 4);
-          ok = ok && issue_dv(it + 1);
-          FA_TRACE(0, 5);
-          if (ok && it + 2 < n_it) ok = issue_s(it + 2);
-          FA_TRACE(0, 6);
+          if (it + 1 < n_it) {
+            // dP(it+1) overwrites dQ(it): after the drain warps have read it
+            ok = mbar_wait(bar(C::B_DQF), it & 1, a.err, kSiteDQF, abort_flag);
+            FA_TRACE(0, 4);
+            if (!ok) break;
+            tc_fence_after();
+            ok = issue_dp(it + 1);
+            ok = ok && issue_dv(it + 1);
+            FA_TRACE(0, 5);
+            if (ok && it + 2 < n_it) ok = issue_s(it + 2);
+            FA_TRACE(0, 6);
+            if (!ok) break;
+          }
+        } else {
+          if (it + 1 < n_it) {
+            FA_TRACE(0, 3);
+            ok = issue_dp(it + 1);
+            FA_TRACE(0, 4);
+            ok = ok && issue_dv(it + 1);
+            FA_TRACE(0, 5);
+            if (ok && it + 2 < n_it) ok = issue_s(it + 2);
+            FA_TRACE(0, 6);
+            if (!ok) break;
+          }
+          // dQ_it, once dQ(it-1) has been drained (B_DQF phase it)
+          ok = mbar_wait(bar(C::B_DQF), it & 1, a.err, kSiteDQF, abort_flag);
+          FA_TRACE(0, 7);
           if (!ok) break;
+          tc_fence_after();
+          issue_dq(it);
+          umma_commit(bar(C::B_STEP + s));  // step it complete: stage s, dS buffer, dQ tile
         }
-        // dQ_it, once dQ(it-1) has been drained (B_DQF phase it); K = the 128 keys
-        ok = mbar_wait(bar(C::B_DQF), it & 1, a.err, kSiteDQF, abort_flag);
-        FA_TRACE(0, 7);
-        if (!ok) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < C::BK / 16; ++kk) {
-          if constexpr (D == 128)
-            umma_f16_ss(tmem + C::COL_DQ, add(dKt, kk * 2048), add(ds, kk * 2048), idQ,
-                        kk > 0 ? 1u : 0u);
-          else
-            umma_f16_ss(tmem + C::COL_DQ, add(ds, kk * 2048), add(dKt, kk * 2048), idQ,
-                        kk > 0 ? 1u : 0u);
-        }
-        umma_commit(bar(C::B_STEP + s));  // step it complete: stage s, dS buffer, dQ tile
         FA_TRACE(0, 8);
       }
       umma_commit(bar(C::B_END));
@@ -800,8 +921,9 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       f8_sv = a.sv[static_cast<size_t>(bh) * a.nsb + kblk];
       f8_k0 = mul_pow2(1.f, a.exps[0] - a.exps[3]);
     }
-    bool ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_KV), 0, a.err, kSiteKV, abort_flag));
-    if (ok) {
+    bool ok = true;
+    if constexpr (!C::WIDE) ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_KV), 0, a.err, kSiteKV, abort_flag));
+    if (ok && !C::WIDE) {
       // K row r: the A operand of S^T, packed two fp16 per TMEM column like the
       // swizzled shared-memory row it comes from; half h copies head-dim
       // columns [D/2 h, D/2 h + D/2)
@@ -826,28 +948,34 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       warp_arrive(bar(C::B_KT));
     }
     Walk wk = walk_start();
-    // FP8: sq of the next step, loaded one step ahead (the [B, H, N, d] walk
-    // goes through consecutive steps of one head)
-    float f8_sq_next = FP8 ? __ldg(a.sq + static_cast<size_t>(bh) * a.nsb + i0) : 1.f;
+    // FP8: sq of this half's 64 queries (one scale block) in the next step,
+    // loaded one step ahead (the [B, H, N, d] walk goes through consecutive
+    // steps of one head)
+    auto sq_of = [&](int step) {
+      return __ldg(a.sq + static_cast<size_t>(bh) * a.nsb + min(2 * step + h, a.nsb - 1));
+    };
+    float f8_sq_next = FP8 ? sq_of(i0) : 1.f;
     for (int it = 0; it < n_it && ok; ++it, walk_next(wk)) {
       const int s = it % C::NS;
-      const int buf = it & 1;
+      const int buf = it % C::NDS;
       if (warp == 4 && lane == 0) FA_TRACE(1, 1);
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_ST), it & 1, a.err, kSiteST, abort_flag));
+      if (C::WIDE && ok)
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_LFULL), it & 1, a.err, kSiteST, abort_flag));
       if (warp == 4 && lane == 0) FA_TRACE(1, 2);
       if (!ok) break;
       tc_fence_after();
-      // FP8: sq of this step's 64 queries (one scale block)
       const float f8_sq = f8_sq_next;
       if constexpr (FP8)
-        if (wk.step + 1 < nq) f8_sq_next = __ldg(a.sq + static_cast<size_t>(bh) * a.nsb + wk.step + 1);
+        if (wk.step + 1 < nq) f8_sq_next = sq_of(wk.step + 1);
       uint32_t pk[C::NCH][16];                         // P^T, fp16 pairs of queries
       uint32_t zm[C::NCH];                             // bit e: (query qc + e, key) kept
 #pragma unroll
       for (int ch = 0; ch < C::NCH; ++ch) {
         const int qoff = C::HQ * h + 32 * ch;          // first query of this chunk in the step
         const int qh = wk.step * C::BQ + qoff;
-        const float* Ls = reinterpret_cast<const float*>(smem + C::L_OFF + s * C::BQ * 4) + qoff;
+        const float* Ls =
+            reinterpret_cast<const float*>(smem + C::L_OFF + (C::WIDE ? 0 : s) * C::BQ * 4) + qoff;
         const uint32_t s_addr = tmem + lane_off + C::COL_S + qoff;
         const bool need_mask = (a.causal && key > qh + off) || key >= Lk || qh + 31 >= Lq;
         uint32_t sr[32];
@@ -930,9 +1058,13 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       warp_arrive(bar(C::B_P));
       if (warp == 4 && lane == 0) FA_TRACE(1, 3);
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_DPT), it & 1, a.err, kSiteDPT, abort_flag));
+      if (C::WIDE && ok)
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_DFULL), it & 1, a.err, kSiteDPT, abort_flag));
       if (warp == 4 && lane == 0) FA_TRACE(1, 4);
       if (!ok) break;
-      if (it >= 2) {                                   // dQ(it-2) has read this dS buffer
+      // the dS buffer: wide, dQ(it-1) has read it (it ran before dP(it), whose
+      // completion was just seen); d = 64, wait for dQ(it-2)
+      if (!C::WIDE && it >= 2) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_STEP + (it - 2) % C::NS),
                                                ((it - 2) / C::NS) & 1, a.err, kSiteDSF, abort_flag));
         if (!ok) break;
@@ -950,7 +1082,8 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 #pragma unroll
       for (int ch = 0; ch < C::NCH; ++ch) {
         const int qoff = C::HQ * h + 32 * ch;
-        const float* Ds = reinterpret_cast<const float*>(smem + C::DL_OFF + s * C::BQ * 4) + qoff;
+        const float* Ds =
+            reinterpret_cast<const float*>(smem + C::DL_OFF + (C::WIDE ? 0 : s) * C::BQ * 4) + qoff;
         const uint32_t dp_addr = tmem + lane_off + C::COL_DP + qoff;
         uint32_t dr[32];
         tmem_ld32(dp_addr, dr);
@@ -983,6 +1116,11 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           w[e / 2 + 1] = pack_f16x2(ds[2], ds[3]);
         }
         tmem_st16(dp_addr, w);                         // A operand of dK, over own dP^T columns
+        if (C::WIDE && ch == 0) {                      // first chunk in: dK may start on it
+          tmem_st_wait();
+          tc_fence_before();
+          warp_arrive(bar(C::B_DS0));
+        }
         // shared memory copy for dQ: the chunk's 64 bytes of the key's 128-byte
         // row in its 64-query block, XOR-swizzled with (key row % 8) like a TMA
         // SWIZZLE_128B tile
@@ -1038,79 +1176,129 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     float sc = bs.dq1, sc2 = bs.dq2;
     bool two = sc2 != 1.f;
     const Pow2 f8_tau = pow2_pair(FP8 ? -a.exps[0] : 0);
-    float f8_sq_next = FP8 ? __ldg(a.sq + static_cast<size_t>(bh) * a.nsb + i0) : 1.f;
-    float* stage = reinterpret_cast<float*>(smem + C::DQS_OFF + quarter * C::DQ_STAGE);
-    const uint32_t stage_addr = base + C::DQS_OFF + quarter * C::DQ_STAGE;
-    warp_arrive(bar(C::B_DQF));                      // phase 0: no dQ(-1) to drain
-    Walk wq = walk_start();
-    for (int it = 0; it < n_it; ++it, walk_next(wq)) {
-      const int q0 = wq.step * C::BQ;
-      if (warp == 12 && lane == 0) FA_TRACE(2, 1);
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(C::B_STEP + it % C::NS), (it / C::NS) & 1, a.err,
-                                              kSiteDQ, abort_flag)))
-        break;
-      if (warp == 12 && lane == 0) FA_TRACE(2, 2);
-      tc_fence_after();
-      // d = 128: TMEM lanes = head-dim columns, 64 queries; d = 64: lanes =
-      // queries, 64 head-dim columns. Either way 64 values per thread.
-      uint32_t v0[32], v1[32];
-      tmem_ld32(tmem + lane_off + C::COL_DQ, v0);
-      tmem_ld32(tmem + lane_off + C::COL_DQ + 32, v1);
-      tmem_ld_wait();
+    if constexpr (C::WIDE) {
+      // thread = query row (TMEM lane); the four 32-column chunks of its dQ
+      // row go through this warp's two swizzled [32 queries][32 columns]
+      // boxes in two rounds and are added to dQ by TMA reduce-adds. TMEM is
+      // released once the second round's chunks are in registers.
+      uint8_t* srow = smem + C::DQS_OFF + quarter * C::DQ_STAGE + lane * 128;
+      const uint32_t stage_addr = base + C::DQS_OFF + quarter * C::DQ_STAGE;
+      Walk wq = walk_start();
+      for (int it = 0; it < n_it; ++it, walk_next(wq)) {
+        const int qr = wq.step * C::BQ + quarter * 32;   // this warp's 32 query rows
+        if (warp == 12 && lane == 0) FA_TRACE(2, 1);
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(bar(C::B_DQD), it & 1, a.err, kSiteDQ, abort_flag)))
+          break;
+        if (warp == 12 && lane == 0) FA_TRACE(2, 2);
+        tc_fence_after();
+        float m1 = sc, m2 = sc2;
+        bool tw = two;
+        if constexpr (FP8) {                         // scale 2^-tau / sq of these 32 queries
+          const float sq = __ldg(a.sq + static_cast<size_t>(bh) * a.nsb + min(qr / 64, a.nsb - 1));
+          m1 = a.scale / sq * f8_tau.f1;
+          m2 = f8_tau.f2;
+          tw = true;
+        }
+        const bool inside = packed ? tq0 + qr < a.Tq : qr < a.N;   // box starts in the tensor
+        auto scale_pair = [&](uint32_t (&v0)[32], uint32_t (&v1)[32]) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float f0 = __uint_as_float(v0[j]) * m1, f1 = __uint_as_float(v1[j]) * m1;
+            v0[j] = __float_as_uint(tw ? f0 * m2 : f0);
+            v1[j] = __float_as_uint(tw ? f1 * m2 : f1);
+          }
+        };
+        auto stage_pair = [&](const uint32_t (&v0)[32], const uint32_t (&v1)[32]) {
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const uint32_t* v = c ? v1 : v0;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              *reinterpret_cast<uint4*>(srow + c * 4096 + ((u ^ (lane & 7)) << 4)) =
+                  make_uint4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+          }
+        };
+        auto reduce_pair = [&](int rd) {
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (inside) {
+              for (int c = 0; c < 2; ++c) {
+                const int x = 64 * rd + 32 * c;
+                if (packed)
+                  tma_reduce_add_3d(&tmDQ, stage_addr + c * 4096, x, wq.head, tq0 + qr);
+                else
+                  tma_reduce_add_3d(&tmDQ, stage_addr + c * 4096, x, qr, bh);
+              }
+            }
+            bulk_commit_group();
+          }
+        };
+        // columns [0, 64): out of TMEM, scaled, into the boxes (the previous
+        // step's reduces have long read them)
+        {
+          uint32_t v0[32], v1[32];
+          tmem_ld32(tmem + lane_off + C::COL_DQ, v0);
+          tmem_ld32(tmem + lane_off + C::COL_DQ + 32, v1);
+          tmem_ld_wait();
+          scale_pair(v0, v1);
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
+          stage_pair(v0, v1);
+        }
+        // columns [64, 128) out of TMEM: dP(it+1) may now overwrite dQ(it);
+        // then the first boxes go out and the second pair follows them
+        {
+          uint32_t v0[32], v1[32];
+          tmem_ld32(tmem + lane_off + C::COL_DQ + 64, v0);
+          tmem_ld32(tmem + lane_off + C::COL_DQ + 96, v1);
+          tmem_ld_wait();
+          tc_fence_before();
+          warp_arrive(bar(C::B_DQF));
+          if (warp == 12 && lane == 0) FA_TRACE(2, 3);
+          reduce_pair(0);
+          scale_pair(v0, v1);
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
+          stage_pair(v0, v1);
+          reduce_pair(1);
+        }
+      }
+      if (lane == 0) bulk_wait_all();
       tc_fence_before();
-      if constexpr (FP8) {                           // scale 2^-tau / sq of this step
-        sc = a.scale / f8_sq_next * f8_tau.f1;
-        sc2 = f8_tau.f2;
-        two = true;
-        if (wq.step + 1 < nq) f8_sq_next = __ldg(a.sq + static_cast<size_t>(bh) * a.nsb + wq.step + 1);
-      }
-      warp_arrive(bar(C::B_DQF));                    // dQ(it) read: counts for phase it+1
-      if (warp == 12 && lane == 0) FA_TRACE(2, 3);
-      if (two) {                                     // factor outside one float's range
+    } else {
+      // d = 64: thread = query row, 64 head-dim columns; a [32 queries][32
+      // columns] box per column half, 16-byte units XOR-swizzled with (row %
+      // 8) as the 128-byte-swizzled tensor map reads them; the second half
+      // waits until the first has been read out of the box
+      uint8_t* srow = smem + C::DQS_OFF + quarter * C::DQ_STAGE + lane * 128;
+      const uint32_t stage_addr = base + C::DQS_OFF + quarter * C::DQ_STAGE;
+      warp_arrive(bar(C::B_DQF));                    // phase 0: no dQ(-1) to drain
+      Walk wq = walk_start();
+      for (int it = 0; it < n_it; ++it, walk_next(wq)) {
+        const int qr = wq.step * C::BQ + quarter * 32;   // this warp's 32 query rows
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(C::B_STEP + it % C::NS), (it / C::NS) & 1,
+                                                a.err, kSiteDQ, abort_flag)))
+          break;
+        tc_fence_after();
+        uint32_t v0[32], v1[32];
+        tmem_ld32(tmem + lane_off + C::COL_DQ, v0);
+        tmem_ld32(tmem + lane_off + C::COL_DQ + 32, v1);
+        tmem_ld_wait();
+        tc_fence_before();
+        warp_arrive(bar(C::B_DQF));                  // dQ(it) read: counts for phase it+1
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          v0[j] = __float_as_uint(__uint_as_float(v0[j]) * sc * sc2);
-          v1[j] = __float_as_uint(__uint_as_float(v1[j]) * sc * sc2);
+          const float f0 = __uint_as_float(v0[j]) * sc, f1 = __uint_as_float(v1[j]) * sc;
+          v0[j] = __float_as_uint(two ? f0 * sc2 : f0);   // factor outside one float's range
+          v1[j] = __float_as_uint(two ? f1 * sc2 : f1);
         }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          v0[j] = __float_as_uint(__uint_as_float(v0[j]) * sc);
-          v1[j] = __float_as_uint(__uint_as_float(v1[j]) * sc);
-        }
-      }
-      if (lane == 0) bulk_wait_read_all();           // previous reduce has read the staging box
-      __syncwarp();
-      if constexpr (D == 128) {
-        // [64 queries][32 columns], thread = column: lane-contiguous stores
-#pragma unroll
-        for (int j = 0; j < 32; ++j) stage[j * 32 + lane] = __uint_as_float(v0[j]);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) stage[(32 + j) * 32 + lane] = __uint_as_float(v1[j]);
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          // rows past the tensor are skipped; in the packed form, rows past this
-          // sequence add exact zeros (dS = 0 there) to the next sequence's dQ
-          if (packed)
-            tma_reduce_add_3d(&tmDQ, stage_addr, quarter * 32, wq.head, tq0 + q0);
-          else
-            tma_reduce_add_3d(&tmDQ, stage_addr, quarter * 32, q0, bh);
-          bulk_commit_group();
-        }
-      } else {
-        // a [32 queries][32 columns] box per column half, thread = query row,
-        // 16-byte units XOR-swizzled with (row % 8) as the 128-byte-swizzled
-        // tensor map reads them; the second half waits until the first has
-        // been read out of the box
-        uint8_t* srow = reinterpret_cast<uint8_t*>(stage) + lane * 128;
-        const int qr = q0 + quarter * 32;            // this warp's 32 query rows
+        const bool inside = packed ? tq0 + qr < a.Tq : qr < a.N;   // box starts in the tensor
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-          if (c == 1) {
-            if (lane == 0) bulk_wait_read_all();
-            __syncwarp();
-          }
+          if (lane == 0) bulk_wait_read_all();       // the box's previous reduce has read it
+          __syncwarp();
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             const uint32_t* v = c ? v1 : v0;
@@ -1120,17 +1308,21 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           fence_async_smem();
           __syncwarp();
           if (lane == 0) {
-            if (packed)
-              tma_reduce_add_3d(&tmDQ, stage_addr, c * 32, wq.head, tq0 + qr);
-            else
-              tma_reduce_add_3d(&tmDQ, stage_addr, c * 32, qr, bh);
+            // rows past the tensor are skipped; in the packed form, rows past
+            // this sequence add exact zeros (dS = 0 there) to the next one's dQ
+            if (inside) {
+              if (packed)
+                tma_reduce_add_3d(&tmDQ, stage_addr, c * 32, wq.head, tq0 + qr);
+              else
+                tma_reduce_add_3d(&tmDQ, stage_addr, c * 32, qr, bh);
+            }
             bulk_commit_group();
           }
         }
       }
+      if (lane == 0) bulk_wait_all();
+      tc_fence_before();
     }
-    if (lane == 0) bulk_wait_all();
-    tc_fence_before();
   }
 
   __syncthreads();

@@ -3,7 +3,7 @@
 Builds a separate copy of the library with -DFA_BWD_TRACE into _build/trace/
 (libfa.so itself never carries the trace), runs fa_fwd then fa_bwd on the
 long-sequence workload (B=1, H=16, N=16384, d=128, causal) and prints, per
-64-query step of CTA 0 (the CTA with the most steps), how many SM cycles its
+128-query step of CTA 0 (the CTA with the most steps), how many SM cycles its
 single MMA-issuing thread spends on each product group and each barrier wait,
 and what one P / dS warp and one drain warp do meanwhile. A tcgen05.mma is
 accepted only as fast as the tensor core drains its queue, so the time to
@@ -93,25 +93,21 @@ def main():
 
     step = [mma[k + 1][1] - mma[k][1] for k in range(len(mma) - 1)]
     print(f"steps traced: {len(mma)} (MMA thread), {len(pds)} (P / dS warp), {len(drain)} (drain)")
-    print("SM cycles per 64-query step, median (10th-90th percentile):")
-    print(f"  step                                  {_stat(step)}")
-    print(f"  wait dS(i)                            {_stat(span(mma, 1, 2))}")
-    print(f"  issue dK(i)        4 x TS, N = 128    {_stat(span(mma, 2, 3))}")
-    print(f"  issue dP^T(i+1)    8 x SS, N = 64     {_stat(span(mma, 3, 4))}")
-    print(f"  wait P(i+1), issue dV(i+1) 4 x TS     {_stat(span(mma, 4, 5))}")
-    print(f"  wait stage, issue S^T(i+2) 8 x TS N=64 {_stat(span(mma, 5, 6))}")
-    print(f"  wait dQ drained                       {_stat(span(mma, 6, 7))}")
-    print(f"  issue dQ^T(i)      8 x SS, N = 64     {_stat(span(mma, 7, 8))}")
+    print("SM cycles per 128-query step, median (10th-90th percentile):")
+    print(f"  step                                       {_stat(step)}")
+    print(f"  wait dS(i) (two halves), issue dK(i)       {_stat(span(mma, 1, 2))}")
+    print(f"  issue dQ(i)        8 x SS, N = 128         {_stat(span(mma, 2, 3))}")
+    print(f"  wait for the drain warps to read dQ(i)     {_stat(span(mma, 3, 4))}")
+    print(f"  issue dP^T(i+1), wait P(i+1), issue dV(i+1) {_stat(span(mma, 4, 5))}")
+    print(f"  wait stage, issue S^T(i+2) 8 x SS, N = 128 {_stat(span(mma, 5, 6))}")
     print("P / dS warp (warp 4):")
-    print(f"  wait S                                {_stat(span(pds, 1, 2))}")
-    print(f"  P: load S, exp, store P, arrive       {_stat(span(pds, 2, 3))}")
-    print(f"  wait dP                               {_stat(span(pds, 3, 4))}")
-    print(f"  wait dS buffer                        {_stat(span(pds, 4, 5))}")
-    print(f"  dS: load dP, dS, stores, arrive       {_stat(span(pds, 5, 6))}")
+    print(f"  wait S and L                               {_stat(span(pds, 1, 2))}")
+    print(f"  P: load S, exp, store P, arrive            {_stat(span(pds, 2, 3))}")
+    print(f"  wait dP and D                              {_stat(span(pds, 3, 4))}")
+    print(f"  dS: load dP, dS, stores, arrive            {_stat(span(pds, 4, 6))}")
     print("drain warp (warp 12):")
-    print(f"  wait step complete                    {_stat(span(drain, 1, 2))}")
-    print(f"  read dQ tile, arrive                  {_stat(span(drain, 2, 3))}")
-
+    print(f"  wait for dQ(i)                             {_stat(span(drain, 1, 2))}")
+    print(f"  read dQ out of TMEM, arrive                {_stat(span(drain, 2, 3))}")
 
 if __name__ == "__main__":
     sys.exit(main())
