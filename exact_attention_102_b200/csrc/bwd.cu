@@ -400,9 +400,9 @@ __device__ __forceinline__ BwdScales bwd_scales(const BwdArgs& a) {
 // One tcgen05 issuer executes in issue order, so a product may overwrite
 // columns that the product issued just before it reads. Per step:
 //   d = 64:  dK(i), dP^T(i+1), dV(i+1), S^T(i+2), dQ(i)
-//   d = 128: dK(i) (its first half as soon as the first 32-query chunk of
-//            each half of dS(i) is in), dQ(i), [drain of dQ(i)] dP^T(i+1),
-//            dV(i+1), S^T(i+2)
+//   d = 128: second half of dK(i), dQ(i), [drain of dQ(i)] dP^T(i+1),
+//            dV(i+1), first half of dK(i+1) (once the first 32-query chunk of
+//            each half of dS(i+1) is in), S^T(i+2)
 // The d = 128 chain dP^T -> dS -> dK -> dQ -> drain -> dP^T bounds the step;
 // the exp work of P(i+1) runs beside it.
 // Warps 4..11 (two per TMEM lane quarter, one per half of the step's queries)
@@ -800,36 +800,30 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         if constexpr (C::WIDE) umma_commit(bar(C::B_DOF));   // dO buffer free once dV(it) ran
         return true;
       };
-      // dK(it) += dS^T(it) Q_it: after dS(it) is in TMEM (B_DS phase it).
-      // Wide: the 16-query groups of the halves' first chunks (0, 1, 4, 5)
-      // go as soon as those chunks are in (B_DS0), the others after B_DS.
+      // d = 64: dK(it) += dS^T(it) Q_it after dS(it) is in TMEM (B_DS phase it)
       auto issue_dk = [&](int it) -> bool {
+        if (!mbar_wait(bar(C::B_DS), it & 1, a.err, kSiteDS, abort_flag)) return false;
+        tc_fence_after();
         const uint64_t qm = add(dQm, (it % C::NS) * C::Q_TILE);
         const uint32_t acc0 = it > 0 ? 1u : 0u;
-        if constexpr (C::WIDE) {
-          if (!mbar_wait(bar(C::B_DS0), it & 1, a.err, kSiteDS, abort_flag)) return false;
-          tc_fence_after();
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int kk = (g >> 1) * 4 + (g & 1);
-            umma_f16_ts(tmem + C::COL_DK, tmem + C::COL_DP + half_col(kk), add(qm, kk * 2048),
-                        idKM, g > 0 ? 1u : acc0);
-          }
-          if (!mbar_wait(bar(C::B_DS), it & 1, a.err, kSiteDS, abort_flag)) return false;
-          tc_fence_after();
+        for (int kk = 0; kk < C::BQ / 16; ++kk)
+          umma_f16_ts(tmem + C::COL_DK, tmem + C::COL_DP + half_col(kk), add(qm, kk * 2048), idKM,
+                      kk > 0 ? 1u : acc0);
+        return true;
+      };
+      // wide: dK(it) in two halves, the 16-query groups of the halves' first
+      // chunks (0, 1, 4, 5) after B_DS0, the others (2, 3, 6, 7) after B_DS
+      auto issue_dk_half = [&](int it, int half) -> bool {
+        if (!mbar_wait(bar(half ? C::B_DS : C::B_DS0), it & 1, a.err, kSiteDS, abort_flag))
+          return false;
+        tc_fence_after();
+        const uint64_t qm = add(dQm, (it % C::NS) * C::Q_TILE);
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int kk = (g >> 1) * 4 + (g & 1) + 2;
-            umma_f16_ts(tmem + C::COL_DK, tmem + C::COL_DP + half_col(kk), add(qm, kk * 2048),
-                        idKM, 1u);
-          }
-        } else {
-          if (!mbar_wait(bar(C::B_DS), it & 1, a.err, kSiteDS, abort_flag)) return false;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < C::BQ / 16; ++kk)
-            umma_f16_ts(tmem + C::COL_DK, tmem + C::COL_DP + half_col(kk), add(qm, kk * 2048), idKM,
-                        kk > 0 ? 1u : acc0);
+        for (int g = 0; g < 4; ++g) {
+          const int kk = (g >> 1) * 4 + (g & 1) + 2 * half;
+          umma_f16_ts(tmem + C::COL_DK, tmem + C::COL_DP + half_col(kk), add(qm, kk * 2048), idKM,
+                      (half | g) > 0 || it > 0 ? 1u : 0u);
         }
         return true;
       };
@@ -850,18 +844,21 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       // safe: S(it+2) comes after dV(it+1) (which reads P(it+1) from the S
       // columns); dP(it+1) after dK(it) (which reads dS(it) from the dP
       // columns); wide, dQ(it) lands over the dP columns after dK(it) too.
+      // wide: the first half of dK(it+1) goes before S(it+2), so that it runs
+      // while the second chunks of dS(it+1) are computed
       if (ok) {
         tc_fence_after();
         ok = issue_s(0) && issue_dp(0) && issue_dv(0);
+        if constexpr (C::WIDE) ok = ok && issue_dk_half(0, 0);
         if (ok && n_it > 1) ok = issue_s(1);
       }
       for (int it = 0; it < n_it && ok; ++it) {
         const int s = it % C::NS;
         FA_TRACE(0, 1);
-        ok = issue_dk(it);
-        FA_TRACE(0, 2);
-        if (!ok) break;
         if constexpr (C::WIDE) {
+          ok = issue_dk_half(it, 1);
+          FA_TRACE(0, 2);
+          if (!ok) break;
           umma_commit(bar(C::B_STEP + s));           // stage s free once dK(it) has run
           issue_dq(it);
           umma_commit(bar(C::B_DQD));                // dQ(it) ready, dS buffer read
@@ -874,12 +871,16 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             tc_fence_after();
             ok = issue_dp(it + 1);
             ok = ok && issue_dv(it + 1);
+            ok = ok && issue_dk_half(it + 1, 0);
             FA_TRACE(0, 5);
             if (ok && it + 2 < n_it) ok = issue_s(it + 2);
             FA_TRACE(0, 6);
             if (!ok) break;
           }
         } else {
+          ok = issue_dk(it);
+          FA_TRACE(0, 2);
+          if (!ok) break;
           if (it + 1 < n_it) {
             FA_TRACE(0, 3);
             ok = issue_dp(it + 1);
