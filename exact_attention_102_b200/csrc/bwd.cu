@@ -145,11 +145,19 @@ __global__ void __launch_bounds__(256) bwd_amax_kernel(BwdArgs a, long long q8, 
     const uint4* src = static_cast<const uint4*>(t == 0 ? a.q : t == 1 ? a.k : t == 2 ? a.v : a.dout);
     const long long n = (t == 0 || t == 3) ? q8 : k8;
     uint32_t mm = 0u;
-    for (long long i = tid; i < n; i += stride) {
-      const uint4 u = src[i];
+    auto fold = [&](const uint4& u) {
       mm = __vmaxu2(mm, __vmaxu2(__vmaxu2(u.x & 0x7fff7fffu, u.y & 0x7fff7fffu),
                                  __vmaxu2(u.z & 0x7fff7fffu, u.w & 0x7fff7fffu)));
+    };
+    long long i = tid;
+    for (; i + 3 * stride < n; i += 4 * stride) {    // four loads in flight per thread
+      const uint4 u0 = src[i], u1 = src[i + stride], u2 = src[i + 2 * stride], u3 = src[i + 3 * stride];
+      fold(u0);
+      fold(u1);
+      fold(u2);
+      fold(u3);
     }
+    for (; i < n; i += stride) fold(src[i]);
     mm = max(mm & 0xffffu, mm >> 16);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) mm = max(mm, __shfl_xor_sync(0xffffffffu, mm, off));
@@ -274,14 +282,15 @@ __global__ void __launch_bounds__(256) bwd_convert_kernel(BwdArgs a, long long q
   if (blockIdx.x == 0 && threadIdx.x < 4) a.exps[threadIdx.x] = e[threadIdx.x];
   const Pow2 f[4] = {pow2_pair(e[0]), pow2_pair(e[1]), pow2_pair(e[2]), pow2_pair(e[3])};
   const long long total = 2 * q8 + 2 * k8;
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int t = i < q8 ? 3 : i < q8 + k8 ? 2 : i < q8 + 2 * k8 ? 1 : 0;
-    const long long j = i - (t == 3 ? 0 : t == 2 ? q8 : t == 1 ? q8 + k8 : q8 + 2 * k8);
-    const void* sp = t == 0 ? a.q : t == 1 ? a.k : t == 2 ? a.v : a.dout;
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  // unit i: tensor and offset (dout, v, k, q in this order)
+  auto locate = [&](long long i, int& t, long long& j) {
+    t = i < q8 ? 3 : i < q8 + k8 ? 2 : i < q8 + 2 * k8 ? 1 : 0;
+    j = i - (t == 3 ? 0 : t == 2 ? q8 : t == 1 ? q8 + k8 : q8 + 2 * k8);
+  };
+  auto store = [&](int t, long long j, const uint4& u) {
     void* dp = t == 0 ? a.q16 : t == 1 ? a.k16 : t == 2 ? a.v16 : a.do16;
     const Pow2 et = f[t];
-    const uint4 u = static_cast<const uint4*>(sp)[j];
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
     uint32_t o[4];
 #pragma unroll
@@ -289,6 +298,26 @@ __global__ void __launch_bounds__(256) bwd_convert_kernel(BwdArgs a, long long q
       o[c] = pack_f16x2(mul_pow2(__uint_as_float(w[c] << 16), et),
                         mul_pow2(__uint_as_float(w[c] & 0xffff0000u), et));
     static_cast<uint4*>(dp)[j] = make_uint4(o[0], o[1], o[2], o[3]);
+  };
+  auto src = [&](int t) { return static_cast<const uint4*>(t == 0 ? a.q : t == 1 ? a.k : t == 2 ? a.v : a.dout); };
+  long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+  for (; i + 3 * stride < total; i += 4 * stride) {   // four loads in flight per thread
+    int t[4];
+    long long j[4];
+    uint4 u[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      locate(i + r * stride, t[r], j[r]);
+      u[r] = src(t[r])[j[r]];
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) store(t[r], j[r], u[r]);
+  }
+  for (; i < total; i += stride) {
+    int t;
+    long long j;
+    locate(i, t, j);
+    store(t, j, src(t)[j]);
   }
 }
 
