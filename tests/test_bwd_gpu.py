@@ -85,7 +85,7 @@ def _exact_gap_bound(x, causal, o_ref_exact, sl=(slice(None), slice(None))):
 
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
-@pytest.mark.parametrize("N", [1, 17, 128, 129, 300])
+@pytest.mark.parametrize("N", [1, 17, 128, 129, 256, 300])
 def test_contract_ragged_shapes(N, d, causal):
     x = synth.attention_inputs(1, 2, N, d, 9000 + N + d, device="cuda")
     _contract(x, causal)
