@@ -707,7 +707,7 @@ fa_status fa_fp8_prepare(const void* q, const void* k, const void* v, const floa
     return FA_ERR_INVALID_ARG;
   fa_status st = check_attn_dims(B, H, N, d);
   if (st != FA_OK) return st;
-  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   fa::Fp8PrepArgs a;
   a.q = q;
   a.k = k;
@@ -722,6 +722,7 @@ fa_status fa_fp8_prepare(const void* q, const void* k, const void* v, const floa
   a.B = B;
   a.H = H;
   a.N = N;
+  a.d = d;
   cudaError_t e = fa::launch_fp8_prepare(a, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
@@ -734,15 +735,17 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float
     return FA_ERR_INVALID_ARG;
   fa_status st = check_attn_dims(B, H, N, d);
   if (st != FA_OK) return st;
-  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   uint32_t* err = error_word_ptr();
   if (err == nullptr) return FA_ERR_LAUNCH;
   const int bh = B * H;
   CUtensorMap tq, tk, tv;
-  // e4m3: one 128-element (128 B) row chunk per box row
-  if (!make_map(&tq, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, bh, 128, 128) ||
-      !make_map(&tk, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, bh, 128, 128) ||
-      !make_map(&tv, v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, bh, 128, 128))
+  // e4m3: one whole row (d bytes) per box row, swizzled over d bytes (the
+  // kernel's MMA descriptors use the same pattern)
+  const CUtensorMapSwizzle sw = d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  if (!make_map(&tq, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, bh, d, 128, sw) ||
+      !make_map(&tk, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, bh, d, 128, sw) ||
+      !make_map(&tv, v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, bh, d, 128, sw))
     return FA_ERR_LAUNCH;
   fa::Fp8FwdArgs a;
   a.sq = sq;
@@ -753,6 +756,7 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float
   a.B = B;
   a.H = H;
   a.N = N;
+  a.d = d;
   a.causal = causal ? 1 : 0;
   a.n_pairs = (N + 255) / 256;
   a.scale_log2 = kLog2e / sqrtf(static_cast<float>(d));

@@ -35,7 +35,6 @@ namespace fa {
 
 namespace {
 
-constexpr int kD = 128;
 constexpr float kE4m3Max = 448.f;
 
 // four floats -> four e4m3 bytes (byte i = element i), RNE, saturating
@@ -52,12 +51,16 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float e0, float e1, float e2, fl
 
 // ------------------------------------------------------------------ prep --
 constexpr int kPrepThreads = 256;
-constexpr int kPrepSmem = 64 * kD * 4 + kD * kD * 4 + 64;   // x block, R, reduction
+template <int D>
+constexpr int prep_smem() { return 64 * D * 4 + D * D * 4 + 64; }   // x block, R, reduction
 
+template <int D>
 __global__ void __launch_bounds__(kPrepThreads) fp8_prep_kernel(Fp8PrepArgs a) {
+  constexpr int kD = D;
+  constexpr int RPT = 64 * D / kPrepThreads;                  // rows per thread: 32 or 16
   extern __shared__ __align__(16) uint8_t smem[];
-  float* xs = reinterpret_cast<float*>(smem);                 // [64][128]
-  float* Rs = xs + 64 * kD;                                   // [128][128]
+  float* xs = reinterpret_cast<float*>(smem);                 // [64][D]
+  float* Rs = xs + 64 * kD;                                   // [D][D]
   float* red = Rs + kD * kD;                                  // [8]
   const int blk = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
   const int nblk = (a.N + 63) / 64;
@@ -82,32 +85,32 @@ __global__ void __launch_bounds__(kPrepThreads) fp8_prep_kernel(Fp8PrepArgs a) {
     for (int i = tid; i < kD * kD; i += kPrepThreads) Rs[i] = a.R[i];
   __syncthreads();
 
-  // y[r][c] = sum_e x[r][e] R[e][c]: thread -> column c, rows rb .. rb+31
+  // y[r][c] = sum_e x[r][e] R[e][c]: thread -> column c, rows rb .. rb+RPT-1
   const int c = tid & (kD - 1);
-  const int rb = (tid >> 7) * 32;
-  float y[32];
+  const int rb = (tid / kD) * RPT;
+  float y[RPT];
   if (which < 2) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) y[i] = 0.f;
+    for (int i = 0; i < RPT; ++i) y[i] = 0.f;
     for (int e = 0; e < kD; ++e) {
       const float rv = Rs[e * kD + c];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) y[i] = fmaf(xs[(rb + i) * kD + e], rv, y[i]);
+      for (int i = 0; i < RPT; ++i) y[i] = fmaf(xs[(rb + i) * kD + e], rv, y[i]);
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) y[i] = xs[(rb + i) * kD + c];
+    for (int i = 0; i < RPT; ++i) y[i] = xs[(rb + i) * kD + c];
   }
   float amax = 0.f;
 #pragma unroll
-  for (int i = 0; i < 32; ++i)
+  for (int i = 0; i < RPT; ++i)
     if (rb + i < rows) amax = fmaxf(amax, fabsf(y[i]));
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
   __syncthreads();                               // everyone is done reading xs
   if ((tid & 31) == 0) red[tid >> 5] = amax;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) xs[(rb + i) * kD + c] = y[i];
+  for (int i = 0; i < RPT; ++i) xs[(rb + i) * kD + c] = y[i];
   __syncthreads();
   float m = red[0];
 #pragma unroll
@@ -124,9 +127,13 @@ __global__ void __launch_bounds__(kPrepThreads) fp8_prep_kernel(Fp8PrepArgs a) {
 }
 
 // --------------------------------------------------------------- forward --
+// d = 128: 128-byte rows, 128-byte swizzle; d = 64: 64-byte rows, 64-byte
+// swizzle (the TMA maps and the MMA descriptors use the same pattern).
+template <int D>
 struct F8 {
   static constexpr int BM = 128, BN = 128;
-  static constexpr int TILE = 128 * kD;         // bytes of a 128-row e4m3 tile (one 128 B chunk)
+  static constexpr int TILE = 128 * D;          // bytes of a 128-row e4m3 tile (one row chunk)
+  static constexpr uint32_t SBO = 8 * D;        // bytes between 8-row groups of a tile
   static constexpr int NSTAGE = 8;
   static constexpr int Q_OFF = 0;
   static constexpr int RING_OFF = 2 * TILE;
@@ -149,10 +156,12 @@ enum : uint32_t {
   kSDrain = 0x48
 };
 
+template <int D>
 __global__ void __launch_bounds__(384, 1)
 fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, Fp8FwdArgs a) {
-  using C = F8;
+  using C = F8<D>;
+  constexpr int kD = D;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -240,6 +249,9 @@ fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (lane == 0) {
       constexpr uint32_t idS = idesc_e4m3(128, C::BN, 0, 0);
       constexpr uint32_t idPV = idesc_e4m3(128, kD, 0, 1);
+      auto desc = [](uint32_t addr) -> uint64_t {
+        return D == 128 ? smem_desc_sw128(addr, 16, C::SBO) : smem_desc_sw64(addr, 16, C::SBO);
+      };
       // Issue order per key block j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1)
       // (tcgen05.mma from one thread executes in issue order; see fwd.cu).
       int it = 0;
@@ -247,8 +259,8 @@ fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       bool ok = mbar_wait(bar(C::B_Q), 0, a.err, kSQ, abort_flag);
       // descriptors of Q tile 0 and ring stage 0; a tile at a byte offset is the
       // base descriptor plus offset / 16 (start-address field)
-      const uint64_t dQ = smem_desc_sw128(base + C::Q_OFF, 16, 1024);
-      const uint64_t dR = smem_desc_sw128(base + C::RING_OFF, 16, 1024);
+      const uint64_t dQ = desc(base + C::Q_OFF);
+      const uint64_t dR = desc(base + C::RING_OFF);
       auto add = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (bytes >> 4); };
       auto issue_s = [&](int t, int stage) {
         const uint64_t q = add(dQ, t * C::TILE), k = add(dR, stage * C::TILE);
@@ -282,8 +294,8 @@ fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < C::BN / 32; ++kk)   // 32 keys = 8 TMEM columns of packed e4m3 P
-            umma_f8_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8, add(vd, kk * 4096), idPV,
-                       (npv[t] > 0 || kk > 0) ? 1u : 0u);
+            umma_f8_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8, add(vd, kk * 32 * kD),
+                       idPV, (npv[t] > 0 || kk > 0) ? 1u : 0u);
           if (j + 1 == nkb_t[t]) umma_commit(bar(C::B_O + t));   // last P.V of tile t
           ++npv[t];
           if (j + 1 < nkb_t[t]) {
@@ -442,34 +454,47 @@ fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
 }  // namespace
 
-cudaError_t launch_fp8_prepare(const Fp8PrepArgs& a, cudaStream_t stream) {
+template <int D>
+cudaError_t launch_fp8_prepare_d(const Fp8PrepArgs& a, cudaStream_t stream) {
   static std::atomic<bool> attr_set[64];   // per device; racing first calls both set it
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(fp8_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kPrepSmem);
+    cudaError_t e = cudaFuncSetAttribute(fp8_prep_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, prep_smem<D>());
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
   dim3 grid((a.N + 63) / 64, a.B * a.H, 3);
-  fp8_prep_kernel<<<grid, kPrepThreads, kPrepSmem, stream>>>(a);
+  fp8_prep_kernel<D><<<grid, kPrepThreads, prep_smem<D>(), stream>>>(a);
   return cudaGetLastError();
 }
 
-cudaError_t launch_fwd_fp8(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                           const Fp8FwdArgs& a, cudaStream_t stream) {
+template <int D>
+cudaError_t launch_fwd_fp8_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const Fp8FwdArgs& a, cudaStream_t stream) {
+  using C = F8<D>;
   static std::atomic<bool> attr_set[64];   // per device; racing first calls both set it
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(fwd_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         F8::SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(fwd_fp8_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  fwd_fp8_kernel<<<a.n_pairs * a.B * a.H, F8::THREADS, F8::SMEM_BYTES, stream>>>(tq, tk, tv, a);
+  fwd_fp8_kernel<D><<<a.n_pairs * a.B * a.H, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, a);
   return cudaGetLastError();
+}
+
+cudaError_t launch_fp8_prepare(const Fp8PrepArgs& a, cudaStream_t stream) {
+  return a.d == 64 ? launch_fp8_prepare_d<64>(a, stream) : launch_fp8_prepare_d<128>(a, stream);
+}
+
+cudaError_t launch_fwd_fp8(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           const Fp8FwdArgs& a, cudaStream_t stream) {
+  return a.d == 64 ? launch_fwd_fp8_d<64>(tq, tk, tv, a, stream)
+                   : launch_fwd_fp8_d<128>(tq, tk, tv, a, stream);
 }
 
 }  // namespace fa

@@ -157,6 +157,7 @@ struct Fp8PrepArgs {
   float* sk;
   float* sv;
   int B, H, N;
+  int d;              // head dim, 64 or 128
 };
 
 cudaError_t launch_fp8_prepare(const Fp8PrepArgs& a, cudaStream_t stream);
@@ -168,6 +169,7 @@ struct Fp8FwdArgs {
   void* o;
   float* lse;
   int B, H, N;
+  int d;              // head dim, 64 or 128
   int causal;
   int n_pairs;
   float scale_log2;

@@ -324,6 +324,22 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// The same with the 64-byte swizzle (layout type 4): atoms of 8 rows x 64 B,
+// as TMA writes them with CU_TENSOR_MAP_SWIZZLE_64B; tile bases 512-byte
+// aligned. K-major: sbo = byte distance between consecutive 8-row groups.
+// MN-major with one 64-byte chunk along M/N: sbo = byte distance between
+// consecutive 8-row groups along K.
+__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t saddr, uint32_t lbo_bytes,
+                                                   uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;  // descriptor version for tcgen05
+  d |= static_cast<uint64_t>(4u) << 61;  // SWIZZLE_64B
+  return d;
+}
+
 // Instruction descriptor for kind::f16 with fp32 accumulate.
 // ab_fmt: 0 = f16, 1 = bf16. a_mn / b_mn: 1 when the operand is MN-major.
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, uint32_t ab_fmt, uint32_t a_mn,

@@ -264,7 +264,7 @@ FA_API fa_status fa_fwd_dropout(const void* q, const void* k, const void* v, voi
  *   D_i = sum_c dO_ic O_ic (o = the dropout forward's output),
  *   dS = P o (dP - D),  dQ = dS K / sqrt(d),  dK = dS^T Q / sqrt(d).
  *   p_drop, seed, offset: those given to fa_fwd_dropout.
- *   d = 128 only (FA_ERR_UNSUPPORTED otherwise).
+ *   d = 64 or 128 (FA_ERR_UNSUPPORTED otherwise).
  * Workspace (fa_bwd_workspace_bytes), precision, other arguments and errors
  * as fa_bwd.
  */
@@ -367,7 +367,7 @@ FA_API fa_status paged_attn_decode_noalloc(const void* q, const void* k_cache,
  *                rows x d of one (b, h); scale = amax / 448 (1 if the block is
  *                all zero), x8 = round_to_nearest_even(x / scale) saturated to
  *                +-448 ("block quantization": one scale per block).
- * Errors: as fa_fwd (d must be 128).
+ * Errors: as fa_fwd (d must be 64 or 128).
  */
 FA_API fa_status fa_fp8_prepare(const void* q, const void* k, const void* v, const float* R,
                          void* q8, void* k8, void* v8, float* sq, float* sk, float* sv,
@@ -379,7 +379,7 @@ FA_API fa_status fa_fp8_prepare(const void* q, const void* k, const void* v, con
  *   o          : bf16 BHND output; lse: fp32 [B][H][N].
  * S = scale * sq_i * sk_j * (q8 k8^T) per 64-row block pair; the V block
  * scale is folded into P before P is rounded to e4m3 for the P.V product.
- * Errors: as fa_fwd (d must be 128).
+ * Errors: as fa_fwd (d must be 64 or 128).
  */
 FA_API fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8,
                      const float* sq, const float* sk, const float* sv,

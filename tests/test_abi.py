@@ -102,9 +102,9 @@ def test_decode_rejects_bad_arguments_without_gpu():
 def test_fp8_rejects_bad_arguments_without_gpu():
     L = fa.lib()
     g = _p(0x10000)
-    assert L.fa_fp8_prepare(*([g] * 10), 1, 1, 128, 64, None) == fa.FA_ERR_UNSUPPORTED
+    assert L.fa_fp8_prepare(*([g] * 10), 1, 1, 128, 96, None) == fa.FA_ERR_UNSUPPORTED
     assert L.fa_fp8_prepare(*([g] * 9), _p(0), 1, 1, 128, 128, None) == fa.FA_ERR_INVALID_ARG
-    assert L.fa_fwd_fp8(*([g] * 8), 1, 1, 128, 64, 0, None) == fa.FA_ERR_UNSUPPORTED
+    assert L.fa_fwd_fp8(*([g] * 8), 1, 1, 128, 96, 0, None) == fa.FA_ERR_UNSUPPORTED
     assert L.fa_fwd_fp8(*([g] * 8), 1, 1, 0, 128, 0, None) == fa.FA_ERR_INVALID_ARG
 
 

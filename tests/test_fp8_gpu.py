@@ -40,9 +40,9 @@ def _e4m3_to_f64(t):
     return t.view(torch.float8_e4m3fn).to("cpu", torch.float64).numpy()
 
 
-def _prepare(B, H, N, seed):  # GPU prepare (codes checked against the oracle's)
-    x = synth.fp8_inputs(B, H, N, 128, seed, device="cuda")
-    r64 = synth.orthogonal_matrix(128, 2003)
+def _prepare(B, H, N, seed, d=128):  # GPU prepare (codes checked against the oracle's)
+    x = synth.fp8_inputs(B, H, N, d, seed, device="cuda")
+    r64 = synth.orthogonal_matrix(d, 2003)
     R = torch.from_numpy(r64).float().cuda()
     out = fa.fa_fp8_prepare(x["q"], x["k"], x["v"], R)
     torch.cuda.synchronize()
@@ -87,9 +87,10 @@ def _fwd_on_oracle_codes(deq, causal):
     return o, lse
 
 
-def test_prepare_matches_oracle_quantiser():
+@pytest.mark.parametrize("d", [64, 128])
+def test_prepare_matches_oracle_quantiser(d):
     B, H, N = 1, 3, 300
-    x, r32, (q8, k8, v8, sq, sk, sv) = _prepare(B, H, N, 31)
+    x, r32, (q8, k8, v8, sq, sk, sv) = _prepare(B, H, N, 31, d)
     for name, t8, sc, rot in (("q", q8, sq, True), ("k", k8, sk, True), ("v", v8, sv, False)):
         src = f64(x[name])
         if rot:
@@ -188,24 +189,26 @@ def test_fp8_config_sampled_rows(record_property):
     record_property("chained_max_abs_gap_to_unquantised_attention", gap)
 
 
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("N", [1, 100, 257, 640])
-def test_fp8_ragged_shapes(N, causal):
+def test_fp8_ragged_shapes(N, causal, d):
     B, H = 1, 2
-    x = synth.fp8_inputs(B, H, N, 128, 40 + N, device="cuda")
-    r32 = synth.orthogonal_matrix(128, 2003).astype(np.float32).astype(np.float64)
+    x = synth.fp8_inputs(B, H, N, d, 40 + N, device="cuda")
+    r32 = synth.orthogonal_matrix(d, 2003).astype(np.float32).astype(np.float64)
     deq = _oracle_quantised(x, r32)
     o, lse = _fwd_on_oracle_codes(deq, causal)
     for h in range(H):
         _check_rows(o, lse, deq, 0, h, np.arange(N), causal)
 
 
-def test_fp8_without_outliers_meets_plain_tolerance():
+@pytest.mark.parametrize("d", [64, 128])
+def test_fp8_without_outliers_meets_plain_tolerance(d):
     """Gaussian inputs without outliers: against unquantised attention the
     FP8 result stays within the plain 5e-2 (+ half a bf16 ulp)."""
     B, H, N = 1, 4, 2048
-    x = synth.attention_inputs(B, H, N, 128, 1005, device="cuda", with_dout=False)
-    R = torch.from_numpy(synth.orthogonal_matrix(128, 2003)).float().cuda()
+    x = synth.attention_inputs(B, H, N, d, 1005, device="cuda", with_dout=False)
+    R = torch.from_numpy(synth.orthogonal_matrix(d, 2003)).float().cuda()
     q8, k8, v8, sq, sk, sv = fa.fa_fp8_prepare(x["q"], x["k"], x["v"], R)
     o, lse = fa.fa_fwd_fp8(q8, k8, v8, sq, sk, sv, causal=False)
     torch.cuda.synchronize()
