@@ -193,7 +193,7 @@ fa_status bwd_dense(const void* q, const void* k, const void* v, const void* o, 
     return FA_ERR_INVALID_ARG;
   fa_status st = check_attn_dims(B, H, N, d);
   if (st != FA_OK) return st;
-  if (f8 != nullptr && (d != 128 || drop != nullptr)) return FA_ERR_UNSUPPORTED;
+  if (f8 != nullptr && drop != nullptr) return FA_ERR_UNSUPPORTED;
   if (workspace == nullptr || !aligned16(workspace) ||
       ws_bytes < fa_bwd_workspace_bytes(B, H, N, d))
     return FA_ERR_WORKSPACE;
@@ -272,7 +272,7 @@ fa_status bwd_dense(const void* q, const void* k, const void* v, const void* o, 
   if (e == cudaSuccess && f8 != nullptr) {
     // gradients of the rotated inputs -> of Q and K: dQ = dQ' R^T, dK = dK' R^T
     const long long rows = static_cast<long long>(bh) * N;
-    e = fa::launch_unrotate(dq, dk, f8->R, rows, a.err, s);
+    e = fa::launch_unrotate(dq, dk, f8->R, rows, d, a.err, s);
   }
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }

@@ -207,6 +207,7 @@ __device__ __forceinline__ void load_exps(const BwdArgs& a, int (&e)[4]) {
 //   tau = e_do + 15 - ceil(log2(2 d 2^14 448 max(sq) max(sk) max(sv)))
 //   |dS'| <= 2^15 (max|dO| 2^e_do < 2^14).
 // exps[] then holds {tau, 0, 0, e_do}.
+template <int D>
 __device__ void fp8_convert(const BwdArgs& a, const int (&e)[4], long long q16) {
   // e[0..2]: scale_exp of the largest block scales' bit patterns is not what is
   // wanted here; recover the maxima from the partials directly
@@ -218,7 +219,7 @@ __device__ void fp8_convert(const BwdArgs& a, const int (&e)[4], long long q16) 
   }
   __syncthreads();
   const int e_do = e[3];
-  const float bound = 2.f * 128.f * 16384.f * 448.f;   // 2 d 2^14 448, d = 128
+  const float bound = 2.f * static_cast<float>(D) * 16384.f * 448.f;   // 2 d 2^14 448
   int c = 0;
   frexpf(bound * fmaxf(smax[0], 1e-30f) * fmaxf(smax[1], 1e-30f) * fmaxf(smax[2], 1e-30f), &c);
   const int tau = e_do + 15 - c;
@@ -272,11 +273,12 @@ __device__ void fp8_convert(const BwdArgs& a, const int (&e)[4], long long q16) 
 // per step, the tensors in the reverse of the amax pass's order (the last
 // rows that pass read may still be in L2). Block 0 publishes the exponents
 // for the kernels that follow.
+template <int D>
 __global__ void __launch_bounds__(256) bwd_convert_kernel(BwdArgs a, long long q8, long long k8) {
   int e[4];
   load_exps(a, e);
   if (a.fp8) {
-    fp8_convert(a, e, q8);
+    fp8_convert<D>(a, e, q8);
     return;
   }
   if (blockIdx.x == 0 && threadIdx.x < 4) a.exps[threadIdx.x] = e[threadIdx.x];
@@ -1318,11 +1320,20 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         tmem_ld_wait();
         tc_fence_before();
         warp_arrive(bar(C::B_DQF));                  // dQ(it) read: counts for phase it+1
+        float m1 = sc, m2 = sc2;
+        bool tw = two;
+        if constexpr (FP8) {                         // scale 2^-tau / sq of this thread's row
+          const float sq = __ldg(a.sq + static_cast<size_t>(bh) * a.nsb +
+                                 min((qr + lane) / 64, a.nsb - 1));
+          m1 = a.scale / sq * f8_tau.f1;
+          m2 = f8_tau.f2;
+          tw = true;
+        }
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const float f0 = __uint_as_float(v0[j]) * sc, f1 = __uint_as_float(v1[j]) * sc;
-          v0[j] = __float_as_uint(two ? f0 * sc2 : f0);   // factor outside one float's range
-          v1[j] = __float_as_uint(two ? f1 * sc2 : f1);
+          const float f0 = __uint_as_float(v0[j]) * m1, f1 = __uint_as_float(v1[j]) * m1;
+          v0[j] = __float_as_uint(tw ? f0 * m2 : f0);   // factor outside one float's range
+          v1[j] = __float_as_uint(tw ? f1 * m2 : f1);
         }
         const bool inside = packed ? tq0 + qr < a.Tq : qr < a.N;   // box starts in the tensor
 #pragma unroll
@@ -1382,10 +1393,9 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(bwd_ts_kernel<D, false, true>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-    if constexpr (D == 128)
-      if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(bwd_ts_kernel<D, false, false, true>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(bwd_ts_kernel<D, false, false, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
@@ -1397,23 +1407,17 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   const long long cwant = (2 * q8 + 2 * k8 + 255) / 256;
   const int cblocks = static_cast<int>(cwant < 148 * 8 ? cwant : 148 * 8);
   bwd_amax_kernel<<<kBwdAmaxBlocks, 256, 0, stream>>>(a, q8, k8);
-  bwd_convert_kernel<<<cblocks, 256, 0, stream>>>(a, q8, k8);
+  bwd_convert_kernel<D><<<cblocks, 256, 0, stream>>>(a, q8, k8);
   bwd_pre_kernel<D><<<pre_blocks, 256, 0, stream>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int nk = ((a.cu_q ? a.max_k : a.N) + C::BK - 1) / C::BK;
   const int per_block = a.cu_q ? a.B * a.Hkv : a.B * a.H;   // CTAs per key block
   if (ev_main_begin != nullptr) cudaEventRecord(ev_main_begin, stream);
-  bool launched = false;
-  if constexpr (D == 128) {
-    if (a.fp8) {
-      bwd_ts_kernel<D, false, false, true><<<nk * per_block, C::THREADS, C::SMEM_BYTES, stream>>>(
-          tq, tk, tv, tdo, tdq, a);
-      launched = true;
-    }
-  }
-  if (launched) {
-  } else if (a.cu_q)
+  if (a.fp8)
+    bwd_ts_kernel<D, false, false, true><<<nk * per_block, C::THREADS, C::SMEM_BYTES, stream>>>(
+        tq, tk, tv, tdo, tdq, a);
+  else if (a.cu_q)
     bwd_ts_kernel<D, true, false><<<nk * per_block, C::THREADS, C::SMEM_BYTES, stream>>>(
         tq, tk, tv, tdo, tdq, a);
   else if (a.dropout)
@@ -1600,8 +1604,68 @@ __global__ void __launch_bounds__(kRotThreads, 2) unrotate_kernel(float* x0, flo
 }
 }  // namespace
 
-cudaError_t launch_unrotate(float* x0, float* x1, const float* R, long long rows, uint32_t* err,
-                            cudaStream_t stream) {
+namespace {
+// d = 64: x[r][:] <- x[r][:] R^T in fp32 on the CUDA cores (64 x 64 multiply-
+// adds per row), in place, 64-row tiles of both tensors. Rt[e][c] = R[c][e]
+// in shared memory; thread t computes rows 4 (t / 16) .. + 3, columns
+// 4 (t % 16) .. + 3.
+constexpr int kRot64Smem = 2 * 64 * 64 * 4;
+__global__ void __launch_bounds__(256) unrotate64_kernel(float* x0, float* x1,
+                                                        const float* __restrict__ R, long long rows) {
+  extern __shared__ __align__(16) float rs[];
+  float* Rt = rs;
+  float* xs = rs + 64 * 64;
+  for (int i = threadIdx.x; i < 64 * 64; i += 256) Rt[(i % 64) * 64 + i / 64] = R[i];
+  const int r4 = (threadIdx.x >> 4) * 4, c4 = (threadIdx.x & 15) * 4;
+  const long long tiles_per = (rows + 63) / 64;
+  for (long long t = blockIdx.x; t < 2 * tiles_per; t += gridDim.x) {
+    float* X = t < tiles_per ? x0 : x1;
+    const long long r0 = (t < tiles_per ? t : t - tiles_per) * 64;
+    const int nr = static_cast<int>(min(64ll, rows - r0));
+    __syncthreads();                               // Rt written / previous tile read
+    for (int i = threadIdx.x; i < 64 * 16; i += 256)
+      reinterpret_cast<float4*>(xs)[i] = i < nr * 16 ? reinterpret_cast<const float4*>(X + r0 * 64)[i]
+                                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+    __syncthreads();
+    float y[4][4] = {};
+#pragma unroll 8
+    for (int e = 0; e < 64; ++e) {
+      const float4 rv = *reinterpret_cast<const float4*>(Rt + e * 64 + c4);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float xe = xs[(r4 + i) * 64 + e];
+        y[i][0] = fmaf(xe, rv.x, y[i][0]);
+        y[i][1] = fmaf(xe, rv.y, y[i][1]);
+        y[i][2] = fmaf(xe, rv.z, y[i][2]);
+        y[i][3] = fmaf(xe, rv.w, y[i][3]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (r4 + i < nr)
+        *reinterpret_cast<float4*>(X + (r0 + r4 + i) * 64 + c4) =
+            make_float4(y[i][0], y[i][1], y[i][2], y[i][3]);
+  }
+}
+}  // namespace
+
+cudaError_t launch_unrotate(float* x0, float* x1, const float* R, long long rows, int d,
+                            uint32_t* err, cudaStream_t stream) {
+  if (d == 64) {
+    static std::atomic<bool> attr64[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr64[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(unrotate64_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kRot64Smem);
+      if (e != cudaSuccess) return e;
+      attr64[dev] = true;
+    }
+    const long long tiles = 2 * ((rows + 63) / 64);
+    const int grid = static_cast<int>(tiles < 148 * 4 ? tiles : 148 * 4);
+    unrotate64_kernel<<<grid, 256, kRot64Smem, stream>>>(x0, x1, R, rows);
+    return cudaGetLastError();
+  }
   static std::atomic<bool> attr_set[64];   // per device; racing first calls both set it
   int dev = 0;
   cudaGetDevice(&dev);

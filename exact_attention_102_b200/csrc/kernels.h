@@ -93,7 +93,7 @@ struct BwdArgs {
   // d = 128, [B, H, N, d] form: (batch, head) slices per grid group (<= 0:
   // one group of all slices, key-block major over every head)
   int head_group = 0;
-  // FP8 backward (fp8 = 1, d = 128, [B, H, N, d] form): q, k, v are the FP8
+  // FP8 backward (fp8 = 1, [B, H, N, d] form): q, k, v are the FP8
   // forward's e4m3 codes (q, k of the rotated inputs) with fp32 scales sq, sk,
   // sv per 64-row block ([B][H][nsb]); the fp16 operand copies hold the codes
   // themselves (exact), and the block scales are folded in fp32
@@ -120,8 +120,8 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
 // x[r][:] <- x[r][:] R^T in place for rows r < rows of two fp32 [rows][128]
 // tensors x0, x1 (the FP8 backward's gradients of the rotated inputs back to
 // the unrotated ones); a wait that gives up records its site in *err
-cudaError_t launch_unrotate(float* x0, float* x1, const float* R, long long rows, uint32_t* err,
-                            cudaStream_t stream);
+cudaError_t launch_unrotate(float* x0, float* x1, const float* R, long long rows, int d,
+                            uint32_t* err, cudaStream_t stream);
 
 struct DecodeArgs {
   const void* q;            // bf16 [S][Hq][d]

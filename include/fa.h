@@ -406,7 +406,7 @@ FA_API fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8,
  * fp32. e4m3 gradient operands were not used: rounding dout to e4m3 alone
  * moves dV by ~1 on the FP8 workload (tolerance 5e-2). The rotation back is a
  * second pass over dq and dk.
- * Errors: as fa_bwd; FA_ERR_UNSUPPORTED unless d = 128.
+ * Errors: as fa_bwd; FA_ERR_UNSUPPORTED unless d = 64 or 128.
  */
 FA_API fa_status fa_bwd_fp8(const void* q8, const void* k8, const void* v8, const float* sq,
                             const float* sk, const float* sv, const float* R, const void* o,

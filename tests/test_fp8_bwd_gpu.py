@@ -32,11 +32,11 @@ pytestmark = pytest.mark.gpu
 fa = pytest.importorskip("exact_attention_102_b200")
 
 
-def _inputs(B, H, N, seed):
-    x = synth.fp8_inputs(B, H, N, 128, seed, device="cuda")
+def _inputs(B, H, N, seed, d=128):
+    x = synth.fp8_inputs(B, H, N, d, seed, device="cuda")
     g = torch.Generator(device="cuda").manual_seed(seed + 1)
-    x["do"] = torch.randn((B, H, N, 128), generator=g, device="cuda").to(torch.bfloat16)
-    r32 = synth.orthogonal_matrix(128, 2003).astype(np.float32).astype(np.float64)
+    x["do"] = torch.randn((B, H, N, d), generator=g, device="cuda").to(torch.bfloat16)
+    r32 = synth.orthogonal_matrix(d, 2003).astype(np.float32).astype(np.float64)
     codes = {}
     for name, rot in (("q", True), ("k", True), ("v", False)):
         src = f64(x[name])
@@ -78,7 +78,7 @@ def _run(x, r32, codes, causal, heads):
 
 
 def _check_head(got, deq, o_in, do, r32, codes, b, h, causal):
-    d = 128
+    d = r32.shape[0]
     sc = 1.0 / math.sqrt(d)
     q, k, v = (deq[n][b, h] for n in ("q", "k", "v"))
     g = do[b, h]
@@ -105,10 +105,11 @@ def _check_head(got, deq, o_in, do, r32, codes, b, h, causal):
                                      f"{float((diff - lim).max()):.3e}, max err {float(diff.max()):.3e}")
 
 
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("N", [64, 100, 300, 513])
-def test_ragged_shapes(N, causal):
-    x, r32, codes = _inputs(1, 2, N, 60 + N + causal)
+def test_ragged_shapes(N, causal, d):
+    x, r32, codes = _inputs(1, 2, N, 60 + N + causal, d)
     heads = [(0, 0), (0, 1)]
     got, deq, o_in = _run(x, r32, codes, causal, heads)
     for b, h in heads:
@@ -126,11 +127,12 @@ def test_fp8_config_two_heads():
         _check_head(got, deq, o_in, f64(x["do"]), r32, codes, b, h, False)
 
 
-def test_identity_rotation_and_unit_scales_match_fa_bwd():
+@pytest.mark.parametrize("d", [64, 128])
+def test_identity_rotation_and_unit_scales_match_fa_bwd(d):
     """Codes on the e4m3 grid with every scale 1 and R = I: the FP8 backward
     is fa_bwd on the same values (dK, dV to fp32 rounding of differently
     scaled operands, dQ likewise)."""
-    B, H, N, d = 1, 2, 200, 128
+    B, H, N = 1, 2, 200
     g = torch.Generator().manual_seed(91)
     vals = {n: oracle.quantize_e4m3(torch.randn((B, H, N, d), generator=g).double().numpy() * 0.5)
             for n in ("q", "k", "v")}
