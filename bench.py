@@ -233,37 +233,65 @@ def run_fwd_bwd(fa, B, H, N, d, causal, steps, warmup, ws, seed, sampler_gpu=Non
 
 
 def run_e2e(fa, B, H, N, d, causal, steps, warmup, ws, seed):
-    """Same step through the public API from pinned host buffers: H2D of q, k,
-    v, dO, then fa_fwd + fa_bwd, then D2H of dQ, dK, dV, all inside the timing."""
+    """Same step through the public API from pinned host buffers, as a
+    pipeline would run it: every step copies its inputs q, k, v, dO in (H2D),
+    runs fa_fwd + fa_bwd, and copies dQ, dK, dV out (D2H), all inside the
+    timing; the copies run on streams of their own, so that step i's compute
+    overlaps step i+1's H2D and step i-1's D2H (device buffers doubled)."""
     xd = synth.attention_inputs(B, H, N, d, seed, device="cuda")
     host = {n: t.cpu().pin_memory() for n, t in xd.items()}
-    dev = {n: torch.empty_like(t) for n, t in xd.items()}
+    dev = [{n: torch.empty_like(t) for n, t in xd.items()} for _ in range(2)]
     del xd
-    o = torch.empty_like(dev["q"])
+    o = torch.empty_like(dev[0]["q"])
     lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
-    dq, dk, dv = (torch.empty((B, H, N, d), dtype=torch.float32, device="cuda") for _ in range(3))
+    grads = [[torch.empty((B, H, N, d), dtype=torch.float32, device="cuda") for _ in range(3)]
+             for _ in range(2)]
     wsp = torch.empty(fa.fa_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device="cuda")
     outs = [torch.empty((B, H, N, d), dtype=torch.float32).pin_memory() for _ in range(3)]
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    computed = [None, None]     # compute of the step that last used buffer b is done
+    drained = [None, None]      # D2H of the step that last used buffer b is done
 
-    def step():
-        for n in ("q", "k", "v", "do"):
-            dev[n].copy_(host[n], non_blocking=True)
-        fa.fa_fwd(dev["q"], dev["k"], dev["v"], causal=causal, o=o, lse=lse)
-        fa.fa_bwd(dev["q"], dev["k"], dev["v"], o, lse, dev["do"], causal=causal, dq=dq, dk=dk,
-                  dv=dv, workspace=wsp)
-        for hbuf, t in zip(outs, (dq, dk, dv)):
-            hbuf.copy_(t, non_blocking=True)
+    def step(i):
+        b = i % 2
+        with torch.cuda.stream(s_in):              # H2D of step i into buffer b
+            if computed[b] is not None:
+                s_in.wait_event(computed[b])
+            for n in ("q", "k", "v", "do"):
+                dev[b][n].copy_(host[n], non_blocking=True)
+            landed = torch.cuda.Event()
+            landed.record(s_in)
+        with torch.cuda.stream(s_cmp):             # fa_fwd + fa_bwd of step i
+            s_cmp.wait_event(landed)
+            if drained[b] is not None:
+                s_cmp.wait_event(drained[b])
+            x, g = dev[b], grads[b]
+            fa.fa_fwd(x["q"], x["k"], x["v"], causal=causal, o=o, lse=lse)
+            fa.fa_bwd(x["q"], x["k"], x["v"], o, lse, x["do"], causal=causal, dq=g[0], dk=g[1],
+                      dv=g[2], workspace=wsp)
+            computed[b] = torch.cuda.Event()
+            computed[b].record(s_cmp)
+        with torch.cuda.stream(s_out):             # D2H of step i's gradients
+            s_out.wait_event(computed[b])
+            for hbuf, t in zip(outs, grads[b]):
+                hbuf.copy_(t, non_blocking=True)
+            drained[b] = torch.cuda.Event()
+            drained[b].record(s_out)
 
-    for _ in range(warmup):
-        step()
+    for i in range(warmup):
+        step(i)
     torch.cuda.synchronize()
     _barrier(ws)
     torch.cuda.synchronize()
     start, end = _ev(), _ev()
-    start.record()
-    for _ in range(steps):
-        step()
-    end.record()
+    start.record(s_in)                             # before the first H2D
+    for st in (s_cmp, s_out):
+        st.wait_event(start)
+    for i in range(steps):
+        step(warmup + i)
+    for st in (s_in, s_cmp):                       # end after the last D2H
+        s_out.wait_stream(st)
+    end.record(s_out)
     torch.cuda.synchronize()
     _barrier(ws)
     ms = _max_over_ranks(start.elapsed_time(end), ws) / steps
@@ -847,7 +875,8 @@ def main():
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": _config(),
             "roofline": roof, "cpu_baseline": cpu,
             "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
+                    "d2h_bytes_per_step": d2h,
+                    "copies": "own streams: step i's H2D and D2H overlap steps i-1 and i+1"},
             "gpu_launches": r["launches_per_step"] * args.steps,
             "clocks": clk, "parts": parts,
         }
