@@ -340,46 +340,80 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdArgs a) {
   // scales enter in the main pass)
   const Pow2 f_v = pow2_pair(a.fp8 ? 0 : a.exps[2]), f_do = pow2_pair(a.exps[3]);
   const float alpha = a.fp8 ? 1.f : __int_as_float((127 - ds_shift(D)) << 23);
-  for (long long pr = warp; pr < rows; pr += nw) {
-    const long long bh = pr / a.n_pad;
-    const int n = static_cast<int>(pr - bh * a.n_pad);
-    // query row n of this (batch, head): BHND row bh * N + n, or packed token
-    // tq0 + n of head h (row (tq0 + n) * H + h; L at [h][tq0 + n])
-    int len = a.N;
-    long long r = bh * a.N + n, lr = r;
-    if (packed) {
-      const int b = static_cast<int>(bh / a.H), h = static_cast<int>(bh % a.H);
-      const int tq0 = a.cu_q[b];
-      len = a.cu_q[b + 1] - tq0;
-      if (tq0 < 0 || len < 0 || len > a.N || tq0 + len > a.Tq) len = 0;   // reported by the main pass
-      r = static_cast<long long>(tq0 + n) * a.H + h;
-      lr = static_cast<long long>(h) * a.Tq + tq0 + n;
-    }
-    if (n >= len) {
-      if (lane == 0) {
-        a.delta[pr] = 0.f;
-        a.lse_log2[pr] = INFINITY;
+  // four rows per warp per iteration, every load issued before the first
+  // reduction (one row alone keeps too little in flight at d = 64)
+  constexpr int R = 4;
+  constexpr int PER = D / 64;                      // bf16 pairs per lane per row
+  for (long long base = static_cast<long long>(warp) * R; base < rows;
+       base += static_cast<long long>(nw) * R) {
+    long long rr[R], lrr[R];
+    int state[R];                                  // 0: past the rows, 1: padding row, 2: live
+    __nv_bfloat162 ov[R][PER], gv[R][PER];
+#pragma unroll
+    for (int u = 0; u < R; ++u) {
+      const long long pr = base + u;
+      state[u] = 0;
+      rr[u] = lrr[u] = 0;
+      if (pr < rows) {
+        const long long bh = pr / a.n_pad;
+        const int n = static_cast<int>(pr - bh * a.n_pad);
+        // query row n of this (batch, head): BHND row bh * N + n, or packed
+        // token tq0 + n of head h (row (tq0 + n) * H + h; L at [h][tq0 + n])
+        int len = a.N;
+        long long r = bh * a.N + n, lr = r;
+        if (packed) {
+          const int b = static_cast<int>(bh / a.H), h = static_cast<int>(bh % a.H);
+          const int tq0 = a.cu_q[b];
+          len = a.cu_q[b + 1] - tq0;
+          if (tq0 < 0 || len < 0 || len > a.N || tq0 + len > a.Tq) len = 0;   // reported by the main pass
+          r = static_cast<long long>(tq0 + n) * a.H + h;
+          lr = static_cast<long long>(h) * a.Tq + tq0 + n;
+        }
+        state[u] = n < len ? 2 : 1;
+        rr[u] = r;
+        lrr[u] = lr;
       }
-      continue;
-    }
-    const __nv_bfloat16* o = static_cast<const __nv_bfloat16*>(a.o) + r * D;
-    const __nv_bfloat16* g = static_cast<const __nv_bfloat16*>(a.dout) + r * D;
-    float acc = 0.f;
 #pragma unroll
-    for (int c = lane * 2; c < D; c += 64) {
-      const __nv_bfloat162 ov = *reinterpret_cast<const __nv_bfloat162*>(o + c);
-      const __nv_bfloat162 gv = *reinterpret_cast<const __nv_bfloat162*>(g + c);
-      acc = fmaf(mul_pow2(__bfloat162float(ov.x), f_v), mul_pow2(__bfloat162float(gv.x), f_do), acc);
-      acc = fmaf(mul_pow2(__bfloat162float(ov.y), f_v), mul_pow2(__bfloat162float(gv.y), f_do), acc);
+      for (int k = 0; k < PER; ++k) {
+        if (state[u] == 2) {
+          const int c = lane * 2 + 64 * k;
+          ov[u][k] = reinterpret_cast<const __nv_bfloat162*>(static_cast<const __nv_bfloat16*>(a.o) +
+                                                             rr[u] * D + c)[0];
+          gv[u][k] = reinterpret_cast<const __nv_bfloat162*>(
+              static_cast<const __nv_bfloat16*>(a.dout) + rr[u] * D + c)[0];
+        } else {
+          ov[u][k] = gv[u][k] = __floats2bfloat162_rn(0.f, 0.f);
+        }
+      }
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) {
-      a.delta[pr] = -alpha * acc;
-      a.lse_log2[pr] = a.lse[lr] * 1.4426950408889634f;
+    for (int u = 0; u < R; ++u) {
+      if (state[u] == 0) continue;
+      const long long pr = base + u;
+      if (state[u] == 1) {
+        if (lane == 0) {
+          a.delta[pr] = 0.f;
+          a.lse_log2[pr] = INFINITY;
+        }
+        continue;
+      }
+      float acc = 0.f;
+#pragma unroll
+      for (int k = 0; k < PER; ++k) {
+        acc = fmaf(mul_pow2(__bfloat162float(ov[u][k].x), f_v),
+                   mul_pow2(__bfloat162float(gv[u][k].x), f_do), acc);
+        acc = fmaf(mul_pow2(__bfloat162float(ov[u][k].y), f_v),
+                   mul_pow2(__bfloat162float(gv[u][k].y), f_do), acc);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (lane == 0) {
+        a.delta[pr] = -alpha * acc;
+        a.lse_log2[pr] = a.lse[lrr[u]] * 1.4426950408889634f;
+      }
+      float4* dq = reinterpret_cast<float4*>(a.dq + rr[u] * D);
+      for (int c = lane; c < D / 4; c += 32) dq[c] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    float4* dq = reinterpret_cast<float4*>(a.dq + r * D);
-    for (int c = lane; c < D / 4; c += 32) dq[c] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 }
 
