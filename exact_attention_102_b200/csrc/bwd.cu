@@ -42,6 +42,7 @@
 #include <type_traits>
 
 #include <atomic>
+#include <utility>
 
 #include "prim.cuh"
 #include "kernels.h"
@@ -124,6 +125,7 @@ __device__ __forceinline__ int ds_shift(int D) { return D == 128 ? 21 : 20; }
 // (bf16 magnitude bits, compared as integers: for non-NaN values the order of
 // the bits is the order of the magnitudes, and NaN sorts above infinity).
 __global__ void __launch_bounds__(256) bwd_amax_kernel(BwdArgs a, long long q8, long long k8) {
+  pdl_wait();                 // the inputs may come from the kernel before this one
   __shared__ uint32_t red[8][4];
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -172,6 +174,7 @@ __global__ void __launch_bounds__(256) bwd_amax_kernel(BwdArgs a, long long q8, 
     for (int i = 0; i < 8; ++i) r = max(r, red[i][threadIdx.x]);
     a.amax_part[blockIdx.x * 4 + threadIdx.x] = r;
   }
+  pdl_trigger();              // this block's work is done: the next kernel may start
 }
 
 // Reduces the partial maxima into e_q, e_k, e_v, e_do (in shared memory).
@@ -275,6 +278,7 @@ __device__ void fp8_convert(const BwdArgs& a, const int (&e)[4], long long q16) 
 // for the kernels that follow.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_convert_kernel(BwdArgs a, long long q8, long long k8) {
+  pdl_wait();                 // the amax partials
   int e[4];
   load_exps(a, e);
   if (a.fp8) {
@@ -331,6 +335,7 @@ __global__ void __launch_bounds__(256) bwd_convert_kernel(BwdArgs a, long long q
 // and dQ rows n < N are zeroed (dQ is accumulated by the main pass).
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdArgs a) {
+  pdl_wait();                 // the exponents of the conversion pass
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const long long rows = static_cast<long long>(a.B) * a.H * a.n_pad;
@@ -724,6 +729,8 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the operand copies, D, L and the zeroed dQ of the passes before this one
+  pdl_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -1440,27 +1447,23 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   const long long k8 = (a.cu_q ? a.n_k_elems : static_cast<long long>(a.B) * a.H * a.N * D) / 8;
   const long long cwant = (2 * q8 + 2 * k8 + 255) / 256;
   const int cblocks = static_cast<int>(cwant < 148 * 8 ? cwant : 148 * 8);
-  bwd_amax_kernel<<<kBwdAmaxBlocks, 256, 0, stream>>>(a, q8, k8);
-  bwd_convert_kernel<D><<<cblocks, 256, 0, stream>>>(a, q8, k8);
-  bwd_pre_kernel<D><<<pre_blocks, 256, 0, stream>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(bwd_amax_kernel, dim3(kBwdAmaxBlocks), dim3(256), 0, stream, a, q8, k8);
+  if (e == cudaSuccess)
+    e = launch_pdl(bwd_convert_kernel<D>, dim3(cblocks), dim3(256), 0, stream, a, q8, k8);
+  if (e == cudaSuccess) e = launch_pdl(bwd_pre_kernel<D>, dim3(pre_blocks), dim3(256), 0, stream, a);
   if (e != cudaSuccess) return e;
   const int nk = ((a.cu_q ? a.max_k : a.N) + C::BK - 1) / C::BK;
   const int per_block = a.cu_q ? a.B * a.Hkv : a.B * a.H;   // CTAs per key block
   if (ev_main_begin != nullptr) cudaEventRecord(ev_main_begin, stream);
-  if (a.fp8)
-    bwd_ts_kernel<D, false, false, true><<<nk * per_block, C::THREADS, C::SMEM_BYTES, stream>>>(
-        tq, tk, tv, tdo, tdq, a);
-  else if (a.cu_q)
-    bwd_ts_kernel<D, true, false><<<nk * per_block, C::THREADS, C::SMEM_BYTES, stream>>>(
-        tq, tk, tv, tdo, tdq, a);
-  else if (a.dropout)
-    bwd_ts_kernel<D, false, true><<<nk * per_block, C::THREADS, C::SMEM_BYTES, stream>>>(
-        tq, tk, tv, tdo, tdq, a);
-  else
-    bwd_ts_kernel<D, false, false><<<nk * per_block, C::THREADS, C::SMEM_BYTES, stream>>>(
-        tq, tk, tv, tdo, tdq, a);
-  e = cudaGetLastError();
+  {
+    void (*k)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, BwdArgs) =
+        a.fp8 ? bwd_ts_kernel<D, false, false, true>
+              : a.cu_q ? bwd_ts_kernel<D, true, false>
+                       : a.dropout ? bwd_ts_kernel<D, false, true> : bwd_ts_kernel<D, false, false>;
+    e = launch_pdl(k, dim3(nk * per_block), dim3(C::THREADS), C::SMEM_BYTES, stream, tq, tk, tv, tdo,
+                   tdq, a);
+  }
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (ev_main_end != nullptr) cudaEventRecord(ev_main_end, stream);
   return e;
 }

@@ -99,6 +99,9 @@ __global__ void __launch_bounds__(384, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, FwdArgs a) {
   using C = FwdCfg<D>;
+  // launched with programmatic serialization: the kernel before this one may
+  // still be finishing, and anything read below may be its output
+  pdl_wait();
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -599,17 +602,13 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
     attr_set[dev] = true;
   }
   const int grid = a.n_pairs * a.B * a.H;
-  if (a.dropout)
-    fwd_kernel<D, kDropout><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, a);
-  else if (a.block_mask != nullptr)
-    fwd_kernel<D, kSparse><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, a);
-  else if (a.block_table != nullptr)
-    fwd_kernel<D, kPaged><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, a);
-  else if (a.cu_q != nullptr)
-    fwd_kernel<D, kPacked><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, a);
-  else
-    fwd_kernel<D, kBhnd><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, a);
-  return cudaGetLastError();
+  void (*k)(CUtensorMap, CUtensorMap, CUtensorMap, FwdArgs) =
+      a.dropout ? fwd_kernel<D, kDropout>
+      : a.block_mask != nullptr ? fwd_kernel<D, kSparse>
+      : a.block_table != nullptr ? fwd_kernel<D, kPaged>
+      : a.cu_q != nullptr ? fwd_kernel<D, kPacked> : fwd_kernel<D, kBhnd>;
+  cudaError_t e = launch_pdl(k, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, stream, tq, tk, tv, a);
+  return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
 template cudaError_t launch_fwd<64>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,

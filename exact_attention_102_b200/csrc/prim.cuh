@@ -13,6 +13,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <utility>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
@@ -110,6 +111,36 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_
       return false;
     }
   }
+}
+
+// ------------------------------------------- programmatic dependent launch --
+// A kernel launched with programmatic stream serialization may start while
+// the kernel before it in the stream is still running: it waits here, before
+// its first read of anything that kernel writes, for that kernel to complete
+// and its writes to be visible (a no-op without such a predecessor).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the dependent kernel of this grid start launching its CTAs now.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Host side: launch with programmatic stream serialization, so that the
+// kernel may start while the one before it in the stream finishes (it calls
+// pdl_wait before reading anything that kernel or any earlier one writes).
+template <typename... P, typename... A>
+inline cudaError_t launch_pdl(void (*k)(P...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, A&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, std::forward<A>(args)...);
 }
 
 // ------------------------------------------------------------------ TMA --
