@@ -1441,7 +1441,7 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
     attr_set[dev] = true;
   }
   const long long rows = static_cast<long long>(a.B) * a.H * a.n_pad;
-  const long long want = (rows + 7) / 8;
+  const long long want = (rows + 31) / 32;                  // 8 warps x 4 rows per block
   const int pre_blocks = static_cast<int>(want < 148 * 16 ? want : 148 * 16);
   const long long q8 = (a.cu_q ? a.n_q_elems : static_cast<long long>(a.B) * a.H * a.N * D) / 8;
   const long long k8 = (a.cu_q ? a.n_k_elems : static_cast<long long>(a.B) * a.H * a.N * D) / 8;
