@@ -712,6 +712,19 @@ def run_case(fa, case, shape, causal, steps, warmup):
 
         def op():
             fa.fa_fwd_fp8(q8, k8, v8, sq, sk, sv, causal=causal, o=o, lse=lse)
+    elif case == "fp8_bwd":
+        x = synth.fp8_inputs(B, H, N, d, 1003, device="cuda")
+        R = torch.from_numpy(synth.orthogonal_matrix(d, 2003)).float().cuda()
+        q8, k8, v8, sq, sk, sv = fa.fa_fp8_prepare(x["q"], x["k"], x["v"], R)
+        o, lse = fa.fa_fwd_fp8(q8, k8, v8, sq, sk, sv, causal=causal)
+        g = torch.Generator(device="cuda").manual_seed(1004)
+        do = torch.randn((B, H, N, d), generator=g, device="cuda").to(torch.bfloat16)
+        grads = [torch.empty((B, H, N, d), device="cuda") for _ in range(3)]
+        wsp = torch.empty(fa.fa_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device="cuda")
+
+        def op():
+            fa.fa_bwd_fp8(q8, k8, v8, sq, sk, sv, R, o, lse, do, causal=causal, dq=grads[0],
+                          dk=grads[1], dv=grads[2], workspace=wsp)
     elif case == "decode":
         S = B          # sequences; contexts U[512, N]
         lay = synth.paged_decode_layout(S, 16, 512, N, 1004)
@@ -747,7 +760,8 @@ def main():
     ap.add_argument("--no-parts", action="store_true", help="headline only")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--case", default="headline",
-                    help="headline (default) or one op for profilers: fwd, bwd, fp8, decode")
+                    help="headline (default) or one op for profilers: fwd, bwd, fp8, fp8_bwd, "
+                         "decode")
     ap.add_argument("--shape", default="1,16,16384,128",
                     help="B,H,N,d for --case (decode: sequences,_,max context,_)")
     ap.add_argument("--causal", type=int, default=1)

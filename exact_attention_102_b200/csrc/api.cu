@@ -723,6 +723,8 @@ fa_status fa_fp8_prepare(const void* q, const void* k, const void* v, const floa
   a.H = H;
   a.N = N;
   a.d = d;
+  a.err = error_word_ptr();
+  if (a.err == nullptr) return FA_ERR_LAUNCH;
   cudaError_t e = fa::launch_fp8_prepare(a, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }

@@ -55,14 +55,14 @@ template <int D>
 constexpr int prep_smem() { return 64 * D * 4 + D * D * 4 + 64; }   // x block, R, reduction
 
 template <int D>
-__global__ void __launch_bounds__(kPrepThreads) fp8_prep_kernel(Fp8PrepArgs a) {
+__global__ void __launch_bounds__(kPrepThreads) fp8_prep_kernel(Fp8PrepArgs a, int which0) {
   constexpr int kD = D;
   constexpr int RPT = 64 * D / kPrepThreads;                  // rows per thread: 32 or 16
   extern __shared__ __align__(16) uint8_t smem[];
   float* xs = reinterpret_cast<float*>(smem);                 // [64][D]
   float* Rs = xs + 64 * kD;                                   // [D][D]
   float* red = Rs + kD * kD;                                  // [8]
-  const int blk = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
+  const int blk = blockIdx.x, bh = blockIdx.y, which = which0 + static_cast<int>(blockIdx.z);
   const int nblk = (a.N + 63) / 64;
   const int r0 = blk * 64;
   const int rows = min(64, a.N - r0);
@@ -123,6 +123,258 @@ __global__ void __launch_bounds__(kPrepThreads) fp8_prep_kernel(Fp8PrepArgs a) {
     const float* p = xs + 4 * i;
     reinterpret_cast<uint32_t*>(dst)[i] =
         pack_e4m3x4(p[0] * inv, p[1] * inv, p[2] * inv, p[3] * inv);
+  }
+}
+
+// ------------------------------------------------------ prep of V (d = 128) --
+// V is not rotated: one CTA per (batch*head, 64-row block) reads the block
+// (8 bf16 per thread and step, coalesced), reduces its amax and writes the
+// e4m3 codes with the same scale and rounding as fp8_prep_kernel.
+__global__ void __launch_bounds__(256) fp8_quant_v_kernel(Fp8PrepArgs a) {
+  constexpr int D = 128;
+  __shared__ float red[8];
+  const int blk = blockIdx.x, bh = blockIdx.y;
+  const int nsb = (a.N + 63) / 64;
+  const int r0 = blk * 64;
+  const int rows = min(64, a.N - r0);
+  const int n16 = rows * D / 8;                        // 16-byte units of the block
+  const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.v) +
+                                                    (static_cast<size_t>(bh) * a.N + r0) * D);
+  uint4 u[4];
+  float m = 0.f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int i = threadIdx.x + 256 * k;
+    u[k] = i < n16 ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t w[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      m = fmax3(m, fabsf(__uint_as_float(w[c] << 16)), fabsf(__uint_as_float(w[c] & 0xffff0000u)));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  m = red[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w]);
+  const float scale = m > 0.f ? m / kE4m3Max : 1.f;
+  const float inv = 1.f / scale;
+  if (threadIdx.x == 0) a.sv[static_cast<size_t>(bh) * nsb + blk] = scale;
+  uint2* dst = reinterpret_cast<uint2*>(a.v8 + (static_cast<size_t>(bh) * a.N + r0) * D);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int i = threadIdx.x + 256 * k;
+    if (i < n16) {
+      const uint32_t w[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
+      float f[8];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        f[2 * c] = __uint_as_float(w[c] << 16) * inv;
+        f[2 * c + 1] = __uint_as_float(w[c] & 0xffff0000u) * inv;
+      }
+      dst[i] = make_uint2(pack_e4m3x4(f[0], f[1], f[2], f[3]), pack_e4m3x4(f[4], f[5], f[6], f[7]));
+    }
+  }
+}
+
+// ------------------------------------------------ prep of Q, K (d = 128) --
+// Q R and K R on the tensor core, then the same per-64-row-block amax / 448
+// scale and e4m3 codes as fp8_prep_kernel. The inputs are bf16, so x is an
+// exact tcgen05 operand; R (fp32) is split into bf16 terms hi = bf16(R),
+// lo = bf16(R - hi), and y = x hi + x lo with fp32 accumulation (the dropped
+// rounding of lo is near 2^-18 of sum_e |x_e| |R_ec|).
+// One tile = 128 rows of one (tensor, batch*head): two scale blocks. A = the
+// x tile in TMEM (two bf16 per column), written by the threads from the 16 x
+// 256 bit shape; B = R^T (B row n = column n of R) split in shared memory,
+// K-major, 128-byte swizzle; D = fp32 in TMEM. 8 warps: warp w reaches TMEM
+// lanes 32 (w % 4) .. + 31 and takes head-dim half w / 4. Persistent CTAs,
+// two per SM; each loads its next tile while its products run.
+constexpr int kRotThreads = 256;
+constexpr int kRotSmem = 80 * 1024;    // R^T hi, lo (64 KB) + barrier; 80 KB keeps 2 CTAs per SM
+constexpr uint32_t kRotCols = 256;     // D [0, 128), x [128, 192)
+constexpr uint32_t kSiteRot = 0x49;
+
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf16x2(a, b);
+  lo = pack_bf16x2(a - __uint_as_float(hi << 16), b - __uint_as_float(hi & 0xffff0000u));
+}
+
+__global__ void __launch_bounds__(kRotThreads, 2) fp8_rot_kernel(Fp8PrepArgs a) {
+  constexpr int D = 128;
+  extern __shared__ uint8_t rot_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(rot_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(sm);
+  const uint32_t bar = sbase + 65536;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + 65536 + 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + 65536 + 16);
+  float* red = reinterpret_cast<float*>(sm + 65536 + 32);      // [8 warps] block maxima
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // R^T -> bf16 hi / lo, K-major, 128-byte swizzle: B[n][k] = R[k][n]; K chunk
+  // k / 64 at 16 KB steps, row n at n * 128 B, 16-byte unit u at u ^ (n % 8)
+  for (int u = threadIdx.x; u < 128 * 16; u += kRotThreads) {
+    const int n = u >> 4, k0 = (u & 15) * 8;
+    float r[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) r[i] = __ldg(a.R + (k0 + i) * D + n);
+    uint4 h, l;
+    split_bf16x2(r[0], r[1], h.x, l.x);
+    split_bf16x2(r[2], r[3], h.y, l.y);
+    split_bf16x2(r[4], r[5], h.z, l.z);
+    split_bf16x2(r[6], r[7], h.w, l.w);
+    const uint32_t off = (k0 >> 6) * 16384 + n * 128 + ((((k0 & 63) >> 3) ^ (n & 7)) << 4);
+    *reinterpret_cast<uint4*>(sm + off) = h;
+    *reinterpret_cast<uint4*>(sm + 32768 + off) = l;
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), kRotCols);
+    tmem_relinquish();
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int nsb = (a.N + 63) / 64;
+  const int tiles_per_head = (a.N + 127) / 128;
+  const long long tiles_per = static_cast<long long>(a.B) * a.H * tiles_per_head;
+  const long long tiles = 2 * tiles_per;            // Q, then K
+  const int q = warp & 3, hh = warp >> 2, r_in = lane >> 2, cq = lane & 3;
+  const uint32_t id = idesc_f16(128, 128, 1, 0, 0);
+  const uint64_t dRh = smem_desc_sw128(sbase, 16, 1024);
+  const uint64_t dRl = smem_desc_sw128(sbase + 32768, 16, 1024);
+  auto add = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (bytes >> 4); };
+  struct Tile { int which, bh, p; };
+  auto tile_of = [&](long long t) {
+    Tile x;
+    x.which = t < tiles_per ? 0 : 1;
+    const long long r = t - x.which * tiles_per;
+    x.bh = static_cast<int>(r / tiles_per_head);
+    x.p = static_cast<int>(r - static_cast<long long>(x.bh) * tiles_per_head);
+    return x;
+  };
+  // this thread's part of a tile: rows 32 q + 16 i + 8 s + r_in (i, s in {0, 1});
+  // K groups j = 4 hh + g (g < 4), elements 16 j + 4 cq .. + 3 (8 bytes)
+  uint2 xv[2][2][4];
+  auto load = [&](long long t) {
+    const Tile tl = tile_of(t);
+    const __nv_bfloat16* X = static_cast<const __nv_bfloat16*>(tl.which ? a.k : a.q) +
+                             static_cast<size_t>(tl.bh) * a.N * D;
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int s2 = 0; s2 < 2; ++s2) {
+        const int row = tl.p * 128 + 32 * q + 16 * i + 8 * s2 + r_in;
+        const uint2* src = reinterpret_cast<const uint2*>(X + static_cast<size_t>(row) * D + 64 * hh + 4 * cq);
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+          xv[i][s2][g] = row < a.N ? __ldg(src + 4 * g) : make_uint2(0u, 0u);
+      }
+  };
+
+  long long t = blockIdx.x;
+  if (t < tiles) load(t);
+  uint32_t phase = 0;
+  for (; t < tiles; t += gridDim.x) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      uint32_t w[16];
+#pragma unroll
+      for (int g = 0; g < 4; ++g)
+#pragma unroll
+        for (int s2 = 0; s2 < 2; ++s2) {
+          w[4 * g + 2 * s2] = xv[i][s2][g].x;
+          w[4 * g + 2 * s2 + 1] = xv[i][s2][g].y;
+        }
+      tmem_st_16x256b_x4(tmem + (static_cast<uint32_t>(32 * q + 16 * i) << 16) + 128 + 32 * hh, w);
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int pr = 0; pr < 2; ++pr) {
+        const uint64_t b = pr ? dRl : dRh;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_f16_ts(tmem, tmem + 128 + 8 * kk, add(b, (kk >> 2) * 16384 + (kk & 3) * 32), id,
+                      (pr | kk) != 0);
+      }
+      umma_commit(bar);
+    }
+    const Tile cur = tile_of(t);
+    if (t + gridDim.x < tiles) load(t + gridDim.x);    // next tile, while the products run
+    const bool ok = mbar_wait(bar, phase, a.err, kSiteRot, abort_flag);
+    if (__syncthreads_or(!ok)) break;
+    phase ^= 1;
+    tc_fence_after();
+    // y of this thread: rows 32 q + 16 i + r_in (+ 8), 64 columns of half hh
+    uint32_t v[4][16];
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4)
+      tmem_ld_16x256b_x4(tmem + (static_cast<uint32_t>(32 * q + 16 * (c4 >> 1)) << 16) + 64 * hh +
+                             32 * (c4 & 1), v[c4]);
+    tmem_ld_wait();
+    // amax of this thread's rows (all in scale block q / 2 of the tile; rows
+    // past N hold zeros)
+    float m = 0.f;
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4)
+#pragma unroll
+      for (int e = 0; e < 16; ++e) m = fmaxf(m, fabsf(__uint_as_float(v[c4][e])));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if (lane == 0) red[warp] = m;
+    tc_fence_before();
+    __syncthreads();
+    // block q / 2: warps {0, 1, 4, 5} or {2, 3, 6, 7}
+    const int b0 = (q >> 1) * 2;
+    const float bm = fmaxf(fmaxf(red[b0], red[b0 + 1]), fmaxf(red[b0 + 4], red[b0 + 5]));
+    const float scale = bm > 0.f ? bm / kE4m3Max : 1.f;
+    const float inv = 1.f / scale;
+    const int blk = cur.p * 2 + (q >> 1);
+    float* sc = (cur.which ? a.sk : a.sq) + static_cast<size_t>(cur.bh) * nsb;
+    if ((warp == 0 || warp == 2) && lane == 0 && blk < nsb) sc[blk] = scale;
+    uint8_t* dst = (cur.which ? a.k8 : a.q8) + static_cast<size_t>(cur.bh) * a.N * D;
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) {
+      const int i = c4 >> 1;
+      const int ra = cur.p * 128 + 32 * q + 16 * i + r_in, rb = ra + 8;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        // this lane's two columns, and its neighbour's (lane ^ 1) two: four
+        // consecutive codes, stored by the even lane of the pair
+        const uint32_t ca = pack_e4m3x4(__uint_as_float(v[c4][4 * g]) * inv,
+                                        __uint_as_float(v[c4][4 * g + 1]) * inv, 0.f, 0.f) & 0xffffu;
+        const uint32_t cb = pack_e4m3x4(__uint_as_float(v[c4][4 * g + 2]) * inv,
+                                        __uint_as_float(v[c4][4 * g + 3]) * inv, 0.f, 0.f) & 0xffffu;
+        const uint32_t na = __shfl_xor_sync(0xffffffffu, ca, 1);
+        const uint32_t nb = __shfl_xor_sync(0xffffffffu, cb, 1);
+        if ((cq & 1) == 0) {
+          const int col = 64 * hh + 32 * (c4 & 1) + 8 * g + 2 * cq;
+          if (ra < a.N) *reinterpret_cast<uint32_t*>(dst + static_cast<size_t>(ra) * D + col) = ca | (na << 16);
+          if (rb < a.N) *reinterpret_cast<uint32_t*>(dst + static_cast<size_t>(rb) * D + col) = cb | (nb << 16);
+        }
+      }
+    }
+    __syncthreads();                                   // red is rewritten by the next tile
+  }
+  // a wait that gave up: let the products in flight finish (bounded) before
+  // the columns are freed
+  if (*abort_flag) mbar_wait(bar, phase, nullptr, kSiteRot, nullptr, 100000000ull);
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kRotCols);
   }
 }
 
@@ -465,8 +717,23 @@ cudaError_t launch_fp8_prepare_d(const Fp8PrepArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  dim3 grid((a.N + 63) / 64, a.B * a.H, 3);
-  fp8_prep_kernel<D><<<grid, kPrepThreads, prep_smem<D>(), stream>>>(a);
+  if constexpr (D == 128) {
+    // Q, K on the tensor core; V (no rotation) by a plain quantising kernel
+    static std::atomic<bool> rot_set[64];
+    if (dev < 64 && !rot_set[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(fp8_rot_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kRotSmem);
+      if (e != cudaSuccess) return e;
+      rot_set[dev] = true;
+    }
+    const long long tiles = 2ll * a.B * a.H * ((a.N + 127) / 128);
+    const int grid = static_cast<int>(tiles < 148 * 2 ? tiles : 148 * 2);
+    fp8_rot_kernel<<<grid, kRotThreads, kRotSmem, stream>>>(a);
+    fp8_quant_v_kernel<<<dim3((a.N + 63) / 64, a.B * a.H), 256, 0, stream>>>(a);
+  } else {
+    dim3 grid((a.N + 63) / 64, a.B * a.H, 3);
+    fp8_prep_kernel<D><<<grid, kPrepThreads, prep_smem<D>(), stream>>>(a, 0);
+  }
   return cudaGetLastError();
 }
 

@@ -158,6 +158,7 @@ struct Fp8PrepArgs {
   float* sv;
   int B, H, N;
   int d;              // head dim, 64 or 128
+  uint32_t* err = nullptr;   // device error word (a bounded wait that gives up records its site)
 };
 
 cudaError_t launch_fp8_prepare(const Fp8PrepArgs& a, cudaStream_t stream);
