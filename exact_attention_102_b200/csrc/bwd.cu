@@ -333,11 +333,21 @@ __global__ void __launch_bounds__(256) bwd_convert_kernel(BwdArgs a, long long q
 //                  (0 for n >= N)
 //   Ll[bh][n]    = L_n * log2(e)     (+inf for n >= N, so P = 0 there)
 // and dQ rows n < N are zeroed (dQ is accumulated by the main pass).
+// A row is read by D / 8 lanes, 16 bytes of O and of dO each; a warp takes
+// kPreGroups groups of 32 / (D / 8) rows at a time, with every load of the
+// groups (L included) issued before the first reduction.
+constexpr int kPreGroups = 4;
+template <int D>
+constexpr int pre_rows_per_warp() { return kPreGroups * 32 / (D / 8); }
+
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdArgs a) {
   pdl_wait();                 // the exponents of the conversion pass
+  constexpr int LPR = D / 8;                       // lanes per row
+  constexpr int RPG = 32 / LPR;                    // rows per group
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
+  const int sub = lane % LPR;                      // 8-element slice of the row
   const long long rows = static_cast<long long>(a.B) * a.H * a.n_pad;
   const int nw = (gridDim.x * blockDim.x) >> 5;
   const bool packed = a.cu_q != nullptr;
@@ -345,20 +355,19 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdArgs a) {
   // scales enter in the main pass)
   const Pow2 f_v = pow2_pair(a.fp8 ? 0 : a.exps[2]), f_do = pow2_pair(a.exps[3]);
   const float alpha = a.fp8 ? 1.f : __int_as_float((127 - ds_shift(D)) << 23);
-  // four rows per warp per iteration, every load issued before the first
-  // reduction (one row alone keeps too little in flight at d = 64)
-  constexpr int R = 4;
-  constexpr int PER = D / 64;                      // bf16 pairs per lane per row
-  for (long long base = static_cast<long long>(warp) * R; base < rows;
-       base += static_cast<long long>(nw) * R) {
-    long long rr[R], lrr[R];
-    int state[R];                                  // 0: past the rows, 1: padding row, 2: live
-    __nv_bfloat162 ov[R][PER], gv[R][PER];
+  for (long long base = static_cast<long long>(warp) * (RPG * kPreGroups); base < rows;
+       base += static_cast<long long>(nw) * (RPG * kPreGroups)) {
+    long long rr[kPreGroups];
+    int state[kPreGroups];                         // 0: past the rows, 1: padding row, 2: live
+    uint4 ov[kPreGroups], gv[kPreGroups];
+    float lv[kPreGroups];
 #pragma unroll
-    for (int u = 0; u < R; ++u) {
-      const long long pr = base + u;
+    for (int u = 0; u < kPreGroups; ++u) {
+      const long long pr = base + u * RPG + lane / LPR;
       state[u] = 0;
-      rr[u] = lrr[u] = 0;
+      rr[u] = 0;
+      ov[u] = gv[u] = make_uint4(0u, 0u, 0u, 0u);
+      lv[u] = 0.f;
       if (pr < rows) {
         const long long bh = pr / a.n_pad;
         const int n = static_cast<int>(pr - bh * a.n_pad);
@@ -376,48 +385,39 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdArgs a) {
         }
         state[u] = n < len ? 2 : 1;
         rr[u] = r;
-        lrr[u] = lr;
-      }
-#pragma unroll
-      for (int k = 0; k < PER; ++k) {
         if (state[u] == 2) {
-          const int c = lane * 2 + 64 * k;
-          ov[u][k] = reinterpret_cast<const __nv_bfloat162*>(static_cast<const __nv_bfloat16*>(a.o) +
-                                                             rr[u] * D + c)[0];
-          gv[u][k] = reinterpret_cast<const __nv_bfloat162*>(
-              static_cast<const __nv_bfloat16*>(a.dout) + rr[u] * D + c)[0];
-        } else {
-          ov[u][k] = gv[u][k] = __floats2bfloat162_rn(0.f, 0.f);
+          ov[u] = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.o) + r * D)[sub];
+          gv[u] = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.dout) + r * D)[sub];
+          if (sub == 0) lv[u] = a.lse[lr];
         }
       }
     }
 #pragma unroll
-    for (int u = 0; u < R; ++u) {
-      if (state[u] == 0) continue;
-      const long long pr = base + u;
-      if (state[u] == 1) {
-        if (lane == 0) {
-          a.delta[pr] = 0.f;
-          a.lse_log2[pr] = INFINITY;
-        }
-        continue;
-      }
+    for (int u = 0; u < kPreGroups; ++u) {
+      const uint32_t o4[4] = {ov[u].x, ov[u].y, ov[u].z, ov[u].w};
+      const uint32_t g4[4] = {gv[u].x, gv[u].y, gv[u].z, gv[u].w};
       float acc = 0.f;
 #pragma unroll
-      for (int k = 0; k < PER; ++k) {
-        acc = fmaf(mul_pow2(__bfloat162float(ov[u][k].x), f_v),
-                   mul_pow2(__bfloat162float(gv[u][k].x), f_do), acc);
-        acc = fmaf(mul_pow2(__bfloat162float(ov[u][k].y), f_v),
-                   mul_pow2(__bfloat162float(gv[u][k].y), f_do), acc);
+      for (int c = 0; c < 4; ++c) {
+        acc = fmaf(mul_pow2(__uint_as_float(o4[c] << 16), f_v),
+                   mul_pow2(__uint_as_float(g4[c] << 16), f_do), acc);
+        acc = fmaf(mul_pow2(__uint_as_float(o4[c] & 0xffff0000u), f_v),
+                   mul_pow2(__uint_as_float(g4[c] & 0xffff0000u), f_do), acc);
       }
+      // the row's lanes are LPR consecutive lanes: a butterfly inside them
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-      if (lane == 0) {
-        a.delta[pr] = -alpha * acc;
-        a.lse_log2[pr] = a.lse[lrr[u]] * 1.4426950408889634f;
+      for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (state[u] == 0) continue;
+      const long long pr = base + u * RPG + lane / LPR;
+      if (sub == 0) {
+        a.delta[pr] = state[u] == 2 ? -alpha * acc : 0.f;
+        a.lse_log2[pr] = state[u] == 2 ? lv[u] * 1.4426950408889634f : INFINITY;
       }
-      float4* dq = reinterpret_cast<float4*>(a.dq + rr[u] * D);
-      for (int c = lane; c < D / 4; c += 32) dq[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (state[u] == 2) {
+        float4* dq = reinterpret_cast<float4*>(a.dq + rr[u] * D);
+        dq[sub] = make_float4(0.f, 0.f, 0.f, 0.f);
+        dq[sub + LPR] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
   }
 }
@@ -1441,8 +1441,9 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
     attr_set[dev] = true;
   }
   const long long rows = static_cast<long long>(a.B) * a.H * a.n_pad;
-  const long long want = (rows + 31) / 32;                  // 8 warps x 4 rows per block
-  const int pre_blocks = static_cast<int>(want < 148 * 16 ? want : 148 * 16);
+  const long long per_blk = 8LL * pre_rows_per_warp<D>();   // 8 warps per block
+  const long long want = (rows + per_blk - 1) / per_blk;
+  const int pre_blocks = static_cast<int>(want < 148 * 8 ? want : 148 * 8);
   const long long q8 = (a.cu_q ? a.n_q_elems : static_cast<long long>(a.B) * a.H * a.N * D) / 8;
   const long long k8 = (a.cu_q ? a.n_k_elems : static_cast<long long>(a.B) * a.H * a.N * D) / 8;
   const long long cwant = (2 * q8 + 2 * k8 + 255) / 256;
