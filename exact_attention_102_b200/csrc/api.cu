@@ -214,9 +214,13 @@ fa_status bwd_dense(const void* q, const void* k, const void* v, const void* o, 
   // boxes: 32 columns x 32 rows with the 128-byte swizzle (the drain writes a
   // query row per thread).
   const uint32_t qrows = 128;
+  // K and V: the bf16 inputs themselves (the main pass converts them in shared
+  // memory), or the fp16 copies of the FP8 backward's codes
+  const bool kv16 = f8 != nullptr;
+  const CUtensorMapDataType kv_dt = kv16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   if (!make_map(&tq, q16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, qrows) ||
-      !make_map(&tk, k16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, 128) ||
-      !make_map(&tv, v16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, 128) ||
+      !make_map(&tk, kv16 ? k16 : k, kv_dt, 2, d, N, bh, 64, 128) ||
+      !make_map(&tv, kv16 ? v16 : v, kv_dt, 2, d, N, bh, 64, 128) ||
       !make_map(&tdo, do16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, bh, 64, qrows) ||
       !make_map(&tdq, dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, N, bh, 32, 32,
                 CU_TENSOR_MAP_SWIZZLE_128B))
@@ -539,9 +543,10 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
   const uint32_t qrows = 128;
   if (!make_map(&tq, q16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, H, total_q, 64, 1,
                 CU_TENSOR_MAP_SWIZZLE_128B, qrows) ||
-      !make_map(&tk, k16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, Hkv, total_k, 64, 1,
+      // K, V: the bf16 inputs (converted in shared memory by the main pass)
+      !make_map(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Hkv, total_k, 64, 1,
                 CU_TENSOR_MAP_SWIZZLE_128B, 128) ||
-      !make_map(&tv, v16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, Hkv, total_k, 64, 1,
+      !make_map(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Hkv, total_k, 64, 1,
                 CU_TENSOR_MAP_SWIZZLE_128B, 128) ||
       !make_map(&tdo, do16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, H, total_q, 64, 1,
                 CU_TENSOR_MAP_SWIZZLE_128B, qrows) ||

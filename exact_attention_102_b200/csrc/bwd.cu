@@ -50,7 +50,7 @@
 namespace fa {
 
 // Pipeline trace (built only with -DFA_BWD_TRACE by exact_attention_102_b200.trace_bwd,
-// never in libfa.so): CTA 0 of the [B, H, N, d] d = 128 main pass records clock64
+// never in libfa.so): CTA 0 of the [B, H, N, d] main pass records clock64
 // stamps of its MMA-issuing thread, of one P / dS warp and of one drain warp.
 #ifdef FA_BWD_TRACE
 __device__ unsigned long long g_bwd_trace[3][8192];
@@ -271,11 +271,22 @@ __device__ void fp8_convert(const BwdArgs& a, const int (&e)[4], long long q16) 
   }
 }
 
+// Eight bf16 values (one 16-byte unit) -> eight fp16 values times 2^e.
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4& u, Pow2 f) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    o[c] = pack_f16x2(mul_pow2(__uint_as_float(w[c] << 16), f),
+                      mul_pow2(__uint_as_float(w[c] & 0xffff0000u), f));
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 // ------------------------------------------------------- fp16 conversion
-// q, k, v, dout (bf16) -> fp16 copies scaled by 2^e_X; 8 elements per thread
-// per step, the tensors in the reverse of the amax pass's order (the last
-// rows that pass read may still be in L2). Block 0 publishes the exponents
-// for the kernels that follow.
+// q, dout (bf16) -> fp16 copies scaled by 2^e_X; 8 elements per thread per
+// step, dout first (the amax pass reads it last, so its last rows may still
+// be in L2). K and V are converted by the main pass itself, once per CTA, in
+// shared memory. Block 0 publishes the exponents for the kernels that follow.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_convert_kernel(BwdArgs a, long long q8, long long k8) {
   pdl_wait();                 // the amax partials
@@ -287,25 +298,18 @@ __global__ void __launch_bounds__(256) bwd_convert_kernel(BwdArgs a, long long q
   }
   if (blockIdx.x == 0 && threadIdx.x < 4) a.exps[threadIdx.x] = e[threadIdx.x];
   const Pow2 f[4] = {pow2_pair(e[0]), pow2_pair(e[1]), pow2_pair(e[2]), pow2_pair(e[3])};
-  const long long total = 2 * q8 + 2 * k8;
+  (void)k8;
+  const long long total = 2 * q8;
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  // unit i: tensor and offset (dout, v, k, q in this order)
+  // unit i: tensor (dout, then q) and offset
   auto locate = [&](long long i, int& t, long long& j) {
-    t = i < q8 ? 3 : i < q8 + k8 ? 2 : i < q8 + 2 * k8 ? 1 : 0;
-    j = i - (t == 3 ? 0 : t == 2 ? q8 : t == 1 ? q8 + k8 : q8 + 2 * k8);
+    t = i < q8 ? 3 : 0;
+    j = i < q8 ? i : i - q8;
   };
   auto store = [&](int t, long long j, const uint4& u) {
-    void* dp = t == 0 ? a.q16 : t == 1 ? a.k16 : t == 2 ? a.v16 : a.do16;
-    const Pow2 et = f[t];
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-    uint32_t o[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-      o[c] = pack_f16x2(mul_pow2(__uint_as_float(w[c] << 16), et),
-                        mul_pow2(__uint_as_float(w[c] & 0xffff0000u), et));
-    static_cast<uint4*>(dp)[j] = make_uint4(o[0], o[1], o[2], o[3]);
+    static_cast<uint4*>(t == 0 ? a.q16 : a.do16)[j] = bf16x8_to_f16x8(u, f[t]);
   };
-  auto src = [&](int t) { return static_cast<const uint4*>(t == 0 ? a.q : t == 1 ? a.k : t == 2 ? a.v : a.dout); };
+  auto src = [&](int t) { return static_cast<const uint4*>(t == 0 ? a.q : a.dout); };
   long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
   for (; i + 3 * stride < total; i += 4 * stride) {   // four loads in flight per thread
     int t[4];
@@ -543,7 +547,8 @@ struct BwdTs {
   static constexpr int B_DS = B_P + 1, B_DQF = B_DS + 1, B_DQD = B_DQF + 1, B_GFULL = B_DQD + 1;
   static constexpr int B_DOF = B_GFULL + 1, B_LFULL = B_DOF + 1, B_DFULL = B_LFULL + 1;
   static constexpr int B_DS0 = B_DFULL + 1;
-  static constexpr int B_END = B_DS0 + 1, B_DRAIN = B_END + 1, NBAR = B_DRAIN + 1;
+  static constexpr int B_KVC = B_DS0 + 1;       // K, V converted to fp16 in place (bf16 inputs)
+  static constexpr int B_END = B_KVC + 1, B_DRAIN = B_END + 1, NBAR = B_DRAIN + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
   // TMEM. Wide: S^T/P^T [0,128)  dP^T/dS^T, then dQ [128,256)  dV [256,384)
@@ -694,7 +699,7 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
 #ifdef FA_BWD_TRACE
-  const bool tr_on = blockIdx.x == 0 && D == 128 && !PACKED && !DROP;
+  const bool tr_on = blockIdx.x == 0 && !PACKED && !DROP;
   int tr_n[3] = {0, 0, 0};
 #endif
 
@@ -716,6 +721,7 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     mbar_init(bar(C::B_LFULL), 1);
     mbar_init(bar(C::B_DFULL), 1);
     mbar_init(bar(C::B_DS0), 8);
+    mbar_init(bar(C::B_KVC), 8);      // the 8 softmax-gradient warps
     mbar_init(bar(C::B_END), 1);
     mbar_init(bar(C::B_DRAIN), 1);
     *abort_flag = 0;
@@ -824,7 +830,9 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       // of dQ (M = 128)
       const uint64_t dDS = smem_desc_sw128(base + C::DS_OFF, C::DS_CHUNK, 1024);
       auto add = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (bytes >> 4); };
-      bool ok = mbar_wait(bar(C::B_KV), 0, a.err, kSiteKV, abort_flag);
+      // K and V as fp16 operands: the FP8 backward's copies of the codes come
+      // in by TMA as they are; bf16 inputs are converted in shared memory first
+      bool ok = mbar_wait(bar(FP8 ? C::B_KV : C::B_KVC), 0, a.err, kSiteKV, abort_flag);
       if constexpr (!C::WIDE) ok = ok && mbar_wait(bar(C::B_KT), 0, a.err, kSiteKV, abort_flag);
       auto issue_s = [&](int it) -> bool {
         const int s = it % C::NS;
@@ -995,18 +1003,39 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       f8_k0 = mul_pow2(1.f, a.exps[0] - a.exps[3]);
     }
     bool ok = true;
-    if constexpr (!C::WIDE) ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_KV), 0, a.err, kSiteKV, abort_flag));
+    // bf16 K and V (TMA copies of the inputs) -> fp16 scaled by 2^e_K, 2^e_V,
+    // in place: thread (r, h) converts the 16-byte units of K row r and V row
+    // r that it reads below for the TMEM copy of K (d = 64: half h of the
+    // row; d = 128: chunk h), which together cover both tiles
+    constexpr int UNITS = D / 16;                     // 16-byte units per half row
+    auto unit_addr = [&](int off, int u) -> uint8_t* {
+      const int unit = (D == 128 ? 0 : UNITS * h) + u;
+      return smem + off + (D == 128 ? h * C::KV_CHUNK : 0) + r * 128 + ((unit ^ (r & 7)) << 4);
+    };
+    if constexpr (!FP8 || !C::WIDE)
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_KV), 0, a.err, kSiteKV, abort_flag));
+    if constexpr (!FP8) {
+      if (ok) {
+        const Pow2 fk = pow2_pair(a.exps[1]), fv = pow2_pair(a.exps[2]);
+#pragma unroll
+        for (int u = 0; u < UNITS; ++u) {
+          uint4* pk = reinterpret_cast<uint4*>(unit_addr(C::K_OFF, u));
+          uint4* pv = reinterpret_cast<uint4*>(unit_addr(C::V_OFF, u));
+          *pk = bf16x8_to_f16x8(*pk, fk);
+          *pv = bf16x8_to_f16x8(*pv, fv);
+        }
+        fence_async_smem();                           // for the tensor core's reads
+        warp_arrive(bar(C::B_KVC));
+      }
+    }
     if (ok && !C::WIDE) {
       // K row r: the A operand of S^T, packed two fp16 per TMEM column like the
       // swizzled shared-memory row it comes from; half h copies head-dim
       // columns [D/2 h, D/2 h + D/2)
-      constexpr int UNITS = D / 16;                   // 16-byte units per half row
-      const uint8_t* krow = smem + C::K_OFF + (D == 128 ? h * C::KV_CHUNK : 0) + r * 128;
       uint32_t kr[UNITS * 4];
 #pragma unroll
       for (int u = 0; u < UNITS; ++u) {
-        const int unit = (D == 128 ? 0 : UNITS * h) + u;
-        const uint4 v = *reinterpret_cast<const uint4*>(krow + ((unit ^ (r & 7)) << 4));
+        const uint4 v = *reinterpret_cast<const uint4*>(unit_addr(C::K_OFF, u));
         kr[4 * u] = v.x;
         kr[4 * u + 1] = v.y;
         kr[4 * u + 2] = v.z;

@@ -1,16 +1,18 @@
 """Pipeline trace of the backward main pass (a profiling tool, not the library).
 
 Builds a separate copy of the library with -DFA_BWD_TRACE into _build/trace/
-(libfa.so itself never carries the trace), runs fa_fwd then fa_bwd on the
-long-sequence workload (B=1, H=16, N=16384, d=128, causal) and prints, per
-128-query step of CTA 0 (the CTA with the most steps), how many SM cycles its
+(libfa.so itself never carries the trace), runs fa_fwd then fa_bwd on a causal
+[B, H, N, d] workload (by default the long-sequence one, B=1, H=16, N=16384,
+d=128) and prints, per 128-query step of CTA 0 (a CTA with the most steps,
+key block 0), how many SM cycles its
 single MMA-issuing thread spends on each product group and each barrier wait,
 and what one P / dS warp and one drain warp do meanwhile. A tcgen05.mma is
 accepted only as fast as the tensor core drains its queue, so the time to
 issue a group of products is, in steady state, the time the tensor core
 spends on them.
 
-Usage: python -m exact_attention_102_b200.trace_bwd   (needs a B200)
+Usage: python -m exact_attention_102_b200.trace_bwd [--shape B,H,N,d]   (needs a B200;
+d = 64 or 128)
 """
 
 from __future__ import annotations
@@ -65,17 +67,23 @@ def _stat(x):
     return f"{int(np.median(x)):5d} ({int(np.percentile(x, 10))}-{int(np.percentile(x, 90))})"
 
 
-def main():
+def main(argv=None):
+    import argparse
+
     import torch
 
     import exact_attention_102_b200 as fa
     import synth
 
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--shape", default="1,16,16384,128", help="B,H,N,d (d = 64 or 128)")
+    B, H, N, d = (int(v) for v in ap.parse_args(argv).shape.split(","))
+    if d not in (64, 128):
+        raise SystemExit("d must be 64 or 128")
     lib = build_traced()
     fa.LIB_PATH = lib
     fa._lib = None
     torch.cuda.set_device(0)
-    B, H, N, d = 1, 16, 16384, 128
     x = synth.attention_inputs(B, H, N, d, 1002, device="cuda")
     o, lse = fa.fa_fwd(x["q"], x["k"], x["v"], causal=True)
     for _ in range(3):
@@ -92,9 +100,22 @@ def main():
         return [r[b] - r[a] for r in recs if a in r and b in r]
 
     step = [mma[k + 1][1] - mma[k][1] for k in range(len(mma) - 1)]
+    print(f"B={B} H={H} N={N} d={d}, causal")
     print(f"steps traced: {len(mma)} (MMA thread), {len(pds)} (P / dS warp), {len(drain)} (drain)")
     print("SM cycles per 128-query step, median (10th-90th percentile):")
     print(f"  step                                       {_stat(step)}")
+    if d == 64:
+        print(f"  wait dS(i), issue dK(i)                    {_stat(span(mma, 1, 2))}")
+        print(f"  issue dP^T(i+1)                            {_stat(span(mma, 3, 4))}")
+        print(f"  wait P(i+1), issue dV(i+1)                 {_stat(span(mma, 4, 5))}")
+        print(f"  wait stage, issue S^T(i+2)                 {_stat(span(mma, 5, 6))}")
+        print(f"  wait for the drain warps to read dQ(i-1)   {_stat(span(mma, 6, 7))}")
+        print(f"  issue dQ(i)                                {_stat(span(mma, 7, 8))}")
+        print("P / dS warp (warp 4):")
+        print(f"  first step: from the loop's start to S(0)  {span(pds, 1, 2)[0] if pds else 0}")
+        print(f"  P: load S, exp, store P, arrive            {_stat(span(pds, 2, 3))}")
+        print(f"  dS: load dP, dS, stores, arrive            {_stat(span(pds, 4, 6))}")
+        return 0
     print(f"  wait dS(i) (two halves), issue dK(i)       {_stat(span(mma, 1, 2))}")
     print(f"  issue dQ(i)        8 x SS, N = 128         {_stat(span(mma, 2, 3))}")
     print(f"  wait for the drain warps to read dQ(i)     {_stat(span(mma, 3, 4))}")
