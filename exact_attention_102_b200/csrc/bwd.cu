@@ -463,25 +463,26 @@ __device__ __forceinline__ BwdScales bwd_scales(const BwdArgs& a) {
 //   S^T  = K_j Q_i^T      A = K_j  (d = 64: TMEM; d = 128: shared), B = Q_i
 //   dP^T = V_j dO_i^T     A = V_j  (shared memory),                 B = dO_i
 //   dV  += P^T dO_i       A = P^T  (TMEM, written over S^T),        B = dO_i
-//   dK  += dS^T Q_i       A = dS^T (TMEM, written over dP^T),       B = Q_i
+//   dK  += dS^T Q_i       A = dS^T (d = 64: TMEM, written over dP^T;
+//                                   d = 128: shared, K-major),     B = Q_i
 //   dQ   = dS K_j         A = dS   (shared, MN-major),              B = K_j (shared, MN-major)
-// TMEM, d = 128: S^T/P^T [0,128)  dP^T/dS^T, then dQ [128,256)  dV [256,384)
+// TMEM, d = 128: S^T/P^T [0,128)  dP^T, then dQ [128,256)  dV [256,384)
 //                dK [384,512): 640 columns of state in 512, because dQ(i)
-//                lands over dS^T(i) once dK(i) has read it, and dP^T(i+1)
-//                waits for the drain warps to have read dQ(i).
+//                lands over dP^T(i) once the softmax-gradient warps have read
+//                it, and dP^T(i+1) waits for the drain warps to have read dQ(i).
 //      d = 64:   K [0,32)  S^T/P^T [64,192)  dP^T/dS^T [192,320)  dQ [320,384)
 //                dV [384,448)  dK [448,512)
 // One tcgen05 issuer executes in issue order, so a product may overwrite
 // columns that the product issued just before it reads. Per step:
 //   d = 64:  dK(i), dP^T(i+1), dV(i+1), S^T(i+2), dQ(i)
-//   d = 128: second half of dK(i), dQ(i), [drain of dQ(i)] dP^T(i+1),
-//            dV(i+1), first half of dK(i+1) (once the first 32-query chunk of
-//            each half of dS(i+1) is in), S^T(i+2)
-// The d = 128 chain dP^T -> dS -> dK -> dQ -> drain -> dP^T bounds the step;
-// the exp work of P(i+1) runs beside it.
+//   d = 128: dQ(i), second half of dK(i) [while the drain reads dQ(i)],
+//            dP^T(i+1), dV(i+1), S^T(i+2), first half of dK(i+1) (once the
+//            first 32-query chunk of each half of dS(i+1) is in)
+// The d = 128 chain dP^T -> dS -> dQ -> drain -> dP^T bounds the step; the
+// exp work of P(i+1) and the dK halves run beside it.
 // Warps 4..11 (two per TMEM lane quarter, one per half of the step's queries)
 // compute P and then dS for their half, 32 queries at a time; dS also goes to
-// shared memory for the dQ product. Warps 12..15 drain dQ (thread = query
+// shared memory for the dQ product (d = 128: for dK too). Warps 12..15 drain dQ (thread = query
 // row) through 32-column x 32-row fp32 boxes with the 128-byte swizzle (so the
 // row-per-thread writes meet no bank conflicts), added to dQ in HBM by TMA
 // tensor reduce-adds: d = 128, two boxes per warp, the four column chunks in
@@ -540,8 +541,8 @@ struct BwdTs {
   // that dP^T(i+1) may). Wide only: B_DQD, committed after dQ(i); B_GFULL,
   // dO of step i landed; B_DOF, committed after dV(i) (the dO buffer is free);
   // B_LFULL, B_DFULL: L and D of step i landed. B_DS0: the first 32-query
-  // chunk of each half of dS(i) is in TMEM (queries 0-31 and 64-95), so that
-  // dK(i) may start on them while the second chunks are computed.
+  // chunk of each half of dS(i) is in shared memory (queries 0-31 and 64-95),
+  // so that dK(i) may start on them while the second chunks are computed.
   static constexpr int B_KV = 0, B_FULL = 1, B_STEP = B_FULL + NS;
   static constexpr int B_KT = B_STEP + NS, B_ST = B_KT + 1, B_DPT = B_ST + 1, B_P = B_DPT + 1;
   static constexpr int B_DS = B_P + 1, B_DQF = B_DS + 1, B_DQD = B_DQF + 1, B_GFULL = B_DQD + 1;
@@ -551,7 +552,7 @@ struct BwdTs {
   static constexpr int B_END = B_KVC + 1, B_DRAIN = B_END + 1, NBAR = B_DRAIN + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
-  // TMEM. Wide: S^T/P^T [0,128)  dP^T/dS^T, then dQ [128,256)  dV [256,384)
+  // TMEM. Wide: S^T/P^T [0,128)  dP^T, then dQ [128,256)  dV [256,384)
   // dK [384,512). d = 64: K [0,32)  S^T/P^T [64,192)  dP^T/dS^T [192,320)
   // dQ [320,384)  dV [384,448)  dK [448,512).
   static constexpr uint32_t COL_K = 0, COL_S = WIDE ? 0 : 64, COL_DP = COL_S + BQ,
@@ -829,6 +830,9 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       // dS^T, MN-major over two 64-query blocks DS_CHUNK apart: the A operand
       // of dQ (M = 128)
       const uint64_t dDS = smem_desc_sw128(base + C::DS_OFF, C::DS_CHUNK, 1024);
+      // the same dS buffer as the K-major A operand of dK (wide): a key row of
+      // 128 bytes per 64-query block, the blocks DS_CHUNK apart
+      const uint64_t dDSk = smem_desc_sw128(base + C::DS_OFF, 16, 1024);
       auto add = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (bytes >> 4); };
       // K and V as fp16 operands: the FP8 backward's copies of the codes come
       // in by TMA as they are; bf16 inputs are converted in shared memory first
@@ -892,18 +896,20 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                       kk > 0 ? 1u : acc0);
         return true;
       };
-      // wide: dK(it) in two halves, the 16-query groups of the halves' first
-      // chunks (0, 1, 4, 5) after B_DS0, the others (2, 3, 6, 7) after B_DS
+      // wide: dK(it) += dS^T(it) Q_it with dS^T from shared memory, in two
+      // halves: the 16-query groups of the halves' first chunks (0, 1, 4, 5)
+      // after B_DS0, the others (2, 3, 6, 7) after B_DS
       auto issue_dk_half = [&](int it, int half) -> bool {
         if (!mbar_wait(bar(half ? C::B_DS : C::B_DS0), it & 1, a.err, kSiteDS, abort_flag))
           return false;
         tc_fence_after();
         const uint64_t qm = add(dQm, (it % C::NS) * C::Q_TILE);
+        const uint64_t dsk = add(dDSk, (it % C::NDS) * C::DS_BYTES);
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
           const int kk = (g >> 1) * 4 + (g & 1) + 2 * half;
-          umma_f16_ts(tmem + C::COL_DK, tmem + C::COL_DP + half_col(kk), add(qm, kk * 2048), idKM,
-                      (half | g) > 0 || it > 0 ? 1u : 0u);
+          umma_f16_ss(tmem + C::COL_DK, add(dsk, (kk >> 2) * C::DS_CHUNK + (kk & 3) * 32),
+                      add(qm, kk * 2048), idKM, (half | g) > 0 || it > 0 ? 1u : 0u);
         }
         return true;
       };
@@ -917,15 +923,20 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       };
       // Issue order: S(0), dP(0), dV(0), S(1), then per step it
       //   d = 64: dK(it), dP(it+1), dV(it+1), S(it+2), dQ(it)
-      //   wide:   dK(it), dQ(it), dP(it+1), dV(it+1), S(it+2)
-      // Each wait (P(it+1) before dV(it+1), dS(it) before dK(it), and, wide,
-      // the drain of dQ(it) before dP(it+1)) falls while products issued
-      // before it are still running. In-order execution makes the overwrites
-      // safe: S(it+2) comes after dV(it+1) (which reads P(it+1) from the S
-      // columns); dP(it+1) after dK(it) (which reads dS(it) from the dP
-      // columns); wide, dQ(it) lands over the dP columns after dK(it) too.
-      // wide: the first half of dK(it+1) goes before S(it+2), so that it runs
-      // while the second chunks of dS(it+1) are computed
+      //   wide:   dQ(it), dK(it) second half, dP(it+1), dV(it+1), S(it+2),
+      //           dK(it+1) first half
+      // Each wait (P(it+1) before dV(it+1), dS(it) before dK(it) and dQ(it),
+      // and, wide, the drain of dQ(it) before dP(it+1)) falls while products
+      // issued before it are still running. In-order execution makes the
+      // overwrites safe: S(it+2) comes after dV(it+1) (which reads P(it+1)
+      // from the S columns); d = 64, dP(it+1) after dK(it) (which reads dS(it)
+      // from the dP columns). Wide, dK reads dS from shared memory, so dQ(it)
+      // may land over the dP columns as soon as the softmax-gradient warps
+      // have read dP(it) (B_DS), and dK(it)'s second half runs while the
+      // drain warps read dQ(it) out of TMEM. S(it+2) goes before the first
+      // half of dK(it+1) (which waits for the first chunks of dS(it+1)), so
+      // that the next scores are ready when the softmax-gradient warps are
+      // done with dS(it+1)
       if (ok) {
         tc_fence_after();
         ok = issue_s(0) && issue_dp(0) && issue_dv(0);
@@ -936,12 +947,16 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const int s = it % C::NS;
         FA_TRACE(0, 1);
         if constexpr (C::WIDE) {
-          ok = issue_dk_half(it, 1);
+          // all of dS(it) in shared memory, dP(it) read out of TMEM
+          ok = mbar_wait(bar(C::B_DS), it & 1, a.err, kSiteDS, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          issue_dq(it);
+          umma_commit(bar(C::B_DQD));                // dQ(it) ready in TMEM
           FA_TRACE(0, 2);
+          ok = issue_dk_half(it, 1);
           if (!ok) break;
           umma_commit(bar(C::B_STEP + s));           // stage s free once dK(it) has run
-          issue_dq(it);
-          umma_commit(bar(C::B_DQD));                // dQ(it) ready, dS buffer read
           FA_TRACE(0, 3);
           if (it + 1 < n_it) {
             // dP(it+1) overwrites dQ(it): after the drain warps have read it
@@ -951,9 +966,9 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             tc_fence_after();
             ok = issue_dp(it + 1);
             ok = ok && issue_dv(it + 1);
-            ok = ok && issue_dk_half(it + 1, 0);
             FA_TRACE(0, 5);
             if (ok && it + 2 < n_it) ok = issue_s(it + 2);
+            ok = ok && issue_dk_half(it + 1, 0);
             FA_TRACE(0, 6);
             if (!ok) break;
           }
@@ -1217,21 +1232,23 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           w[e / 2] = pack_f16x2(ds[0], ds[1]);
           w[e / 2 + 1] = pack_f16x2(ds[2], ds[3]);
         }
-        tmem_st16(dp_addr, w);                         // A operand of dK, over own dP^T columns
-        if (C::WIDE && ch == 0) {                      // first chunk in: dK may start on it
-          tmem_st_wait();
-          tc_fence_before();
-          warp_arrive(bar(C::B_DS0));
-        }
-        // shared memory copy for dQ: the chunk's 64 bytes of the key's 128-byte
-        // row in its 64-query block, XOR-swizzled with (key row % 8) like a TMA
-        // SWIZZLE_128B tile
+        // d = 64: the A operand of dK, over own dP^T columns (wide: dK reads
+        // the shared-memory copy)
+        if constexpr (!C::WIDE) tmem_st16(dp_addr, w);
+        // shared memory copy for dQ (and, wide, dK): the chunk's 64 bytes of the
+        // key's 128-byte row in its 64-query block, XOR-swizzled with (key row
+        // % 8) like a TMA SWIZZLE_128B tile
         uint8_t* ds_row = smem + C::DS_OFF + buf * C::DS_BYTES + (qoff / 64) * C::DS_CHUNK + r * 128;
         const int unit0 = (qoff % 64) / 8;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           uint4* dst = reinterpret_cast<uint4*>(ds_row + (((unit0 + u) ^ (r & 7)) << 4));
           *dst = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+        }
+        if (C::WIDE && ch == 0) {                      // first chunk in: dK may start on it
+          fence_async_smem();
+          tc_fence_before();
+          warp_arrive(bar(C::B_DS0));
         }
       }
       if (!(ds_max < 65504.f)) atomicCAS(a.err, 0u, kErrRange + 2);

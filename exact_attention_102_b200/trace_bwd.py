@@ -116,11 +116,11 @@ def main(argv=None):
         print(f"  P: load S, exp, store P, arrive            {_stat(span(pds, 2, 3))}")
         print(f"  dS: load dP, dS, stores, arrive            {_stat(span(pds, 4, 6))}")
         return 0
-    print(f"  wait dS(i) (two halves), issue dK(i)       {_stat(span(mma, 1, 2))}")
-    print(f"  issue dQ(i)        8 x SS, N = 128         {_stat(span(mma, 2, 3))}")
+    print(f"  wait dS(i), issue dQ(i)  8 x SS, N = 128   {_stat(span(mma, 1, 2))}")
+    print(f"  issue dK(i) second half  4 x SS, N = 128   {_stat(span(mma, 2, 3))}")
     print(f"  wait for the drain warps to read dQ(i)     {_stat(span(mma, 3, 4))}")
-    print(f"  issue dP^T(i+1), wait P(i+1), issue dV(i+1) {_stat(span(mma, 4, 5))}")
-    print(f"  wait stage, issue S^T(i+2) 8 x SS, N = 128 {_stat(span(mma, 5, 6))}")
+    print(f"  dP^T(i+1), wait P(i+1), dV(i+1)            {_stat(span(mma, 4, 5))}")
+    print(f"  S^T(i+2), wait dS(i+1) chunks, dK half 1   {_stat(span(mma, 5, 6))}")
     print("P / dS warp (warp 4):")
     print(f"  wait S and L                               {_stat(span(pds, 1, 2))}")
     print(f"  P: load S, exp, store P, arrive            {_stat(span(pds, 2, 3))}")
