@@ -82,9 +82,11 @@ FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, fl
  * rounded up to a multiple of 128 rows — the row statistic D and L * log2(e)
  * (padded with 0 / +inf) — a small block of per-tensor statistics (the
  * largest magnitudes of q, k, v, dout and the power-of-two exponents chosen
- * from them), plus fp16 copies of q, k, v and dout (the backward's
- * tensor-core operands), each part rounded up to 256 bytes. dq itself (fp32)
- * serves as the dQ accumulator.
+ * from them), plus room for fp16 copies of q, k, v and dout (the backward's
+ * tensor-core operands: fa_bwd and fa_bwd_dropout write the copies of q and
+ * dout and convert k and v inside the main pass; fa_bwd_fp8 writes all
+ * four), each part rounded up to 256 bytes. dq itself (fp32) serves as the dQ
+ * accumulator.
  */
 FA_API size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
 
@@ -160,8 +162,9 @@ FA_API fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void
 
 /*
  * fa_bwd_varlen_workspace_bytes — device workspace fa_bwd_varlen needs: D and
- * L log2(e) for [batch][H][max_seqlen_q rounded up to 128] rows, and fp16
- * copies of q, k, v, dout. 0 for invalid sizes.
+ * L log2(e) for [batch][H][max_seqlen_q rounded up to 128] rows, and room for
+ * fp16 copies of q, k, v, dout (those of q and dout are written; k and v are
+ * converted inside the main pass). 0 for invalid sizes.
  */
 FA_API size_t fa_bwd_varlen_workspace_bytes(int batch, int max_seqlen_q, int total_q,
                                             int total_k, int H, int Hkv, int d);
