@@ -18,8 +18,9 @@
 // Precision: the tensor-core operands of the backward are fp16 copies of the
 // bf16 inputs, each tensor multiplied by a power of two picked from its
 // largest magnitude so that its values sit inside fp16's range (an amax pass
-// and the conversion pass run before the main pass; the factors are undone in
-// fp32, see "operand scaling" below). P and dS, rounded to the operand type,
+// and the conversion pass, which copies Q and dO, run before the main pass;
+// the main pass converts K and V itself; the factors are undone in fp32, see
+// "operand scaling" below). P and dS, rounded to the operand type,
 // keep 3 more mantissa bits than bf16 would give them. The scale of dS is
 // chosen so that |dS| stays below 2^15 whenever L is the logsumexp of the
 // scores; a dS beyond fp16's range (possible only with an inconsistent L) is
@@ -32,10 +33,11 @@
 //   warp 1       TMEM allocation; lane 0 issues every tcgen05.mma: S^T, dP^T,
 //                dV, dK and dQ (see "main pass on TMEM operands").
 //   warps 4..11  thread = key row (TMEM lane), two warps per lane quarter,
-//                one per half of the step's queries: P^T, then dS^T, each
-//                written back into TMEM as the A operand of dV / dK, dS^T also
-//                into shared memory for the dQ product; at the end the dK and
-//                dV rows.
+//                one per half of the step's queries: first the in-place fp16
+//                conversion of K and V, then per step P^T, written back into
+//                TMEM as the A operand of dV, and dS, written into shared
+//                memory for the dQ and dK products (d = 64: dS^T into TMEM
+//                for dK); at the end the dK and dV rows.
 //   warps 12..15 thread = query row: read the step's dQ tile out of TMEM and
 //                add it to dQ in HBM with TMA tensor reduce-adds.
 #include <climits>
@@ -491,9 +493,10 @@ template <int D_>
 struct BwdTs {
   static constexpr int D = D_;
   // d = 128 ("wide"): S^T, dP^T and dQ are N = 128 products over 128-query
-  // steps; K stays out of TMEM (S^T reads it from shared memory) and dQ lands
-  // over the dP^T / dS^T columns once dK has read dS, so that 4 x 128
-  // columns hold S^T, dP^T (then dQ), dV and dK.
+  // steps; K and dS stay out of TMEM (S^T, dQ and dK read them from shared
+  // memory) and dQ lands over the dP^T columns once the softmax-gradient
+  // warps have read dP, so that 4 x 128 columns hold S^T, dP^T (then dQ), dV
+  // and dK.
   static constexpr bool WIDE = D == 128;
   static constexpr int BK = 128;                 // keys per CTA
   static constexpr int BQ = 128;                 // queries per step
