@@ -582,7 +582,20 @@ fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const float rowf = a.scale_log2 * a.sq[static_cast<size_t>(bh) * nsb + min(row, a.N - 1) / 64];
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
+    // the key and value block scales of key block j: loaded one block ahead,
+    // so that their latency falls under the previous block's softmax
+    auto scales_of = [&](int jj, float& k0, float& k1, float& v0, float& v1) {
+      const int kb = jj * (C::BN / 64);
+      k0 = skh[kb];
+      k1 = kb + 1 < nsb ? skh[kb + 1] : 1.f;
+      v0 = svh[kb];
+      v1 = kb + 1 < nsb ? svh[kb + 1] : 0.f;
+    };
+    float nk0 = 1.f, nk1 = 1.f, nv0 = 0.f, nv1 = 0.f;
+    if (nkb_t[t] > 0) scales_of(0, nk0, nk1, nv0, nv1);
     for (int j = 0; j < nkb_t[t]; ++j) {
+      const float sk0 = nk0, sk1 = nk1, sv0 = nv0, sv1 = nv1;
+      if (j + 1 < nkb_t[t]) scales_of(j + 1, nk0, nk1, nv0, nv1);
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_S + t), j & 1, a.err, kSS, abort_flag));
       if (!ok) break;
       tc_fence_after();
@@ -594,10 +607,10 @@ fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const int kb0 = kbase / 64;
       // scaled score of column c: S_c * f(half) (exp2 units); a half past the
       // last key block is fully masked, so its factor only has to be positive
-      const float f0 = rowf * skh[kb0];
-      const float f1 = (kb0 + 1 < nsb) ? rowf * skh[kb0 + 1] : 1.f;
-      const float pv0 = svh[kb0] * inv_c;
-      const float pv1 = (kb0 + 1 < nsb) ? svh[kb0 + 1] * inv_c : 0.f;
+      const float f0 = rowf * sk0;
+      const float f1 = (kb0 + 1 < nsb) ? rowf * sk1 : 1.f;
+      const float pv0 = sv0 * inv_c;
+      const float pv1 = (kb0 + 1 < nsb) ? sv1 * inv_c : 0.f;
 #define SV(c) __uint_as_float(sr[(c) >> 5][(c)&31])
       if (kbase + C::BN - 1 > limit) {
 #pragma unroll
