@@ -370,6 +370,12 @@ FA_API fa_status paged_attn_decode_noalloc(const void* q, const void* k_cache,
  *                rows x d of one (b, h); scale = amax / 448 (1 if the block is
  *                all zero), x8 = round_to_nearest_even(x / scale) saturated to
  *                +-448 ("block quantization": one scale per block).
+ * Precision of the rotation: d = 128 runs Q R and K R on the tensor core
+ * with the bf16 inputs exact and R split into two bf16 terms (R = hi + lo,
+ * |R - hi - lo| <= 2^-18 |R|), accumulating in fp32, so each rotated value is
+ * within (2^-18 + 2 d 2^-23) sum_c |x_c R_c| of the exact product; d = 64
+ * rotates in fp32 on the CUDA cores. A value that lands that close to an e4m3
+ * rounding boundary may take the neighbouring code.
  * Errors: as fa_fwd (d must be 64 or 128).
  */
 FA_API fa_status fa_fp8_prepare(const void* q, const void* k, const void* v, const float* R,
