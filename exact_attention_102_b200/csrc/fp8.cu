@@ -33,6 +33,22 @@
 
 namespace fa {
 
+// Softmax trace (built only with -DFA_FP8_TRACE by exact_attention_102_b200.trace_fp8,
+// never in libfa.so): in CTA 0 of the forward, lane 0 of the first softmax warp
+// of each tile records clock64 stamps around the steps of every key block.
+#ifdef FA_FP8_TRACE
+__device__ unsigned long long g_fp8_trace[2][4096];
+#define FA_F8_TRACE(tag)                                                                  \
+  do {                                                                                    \
+    if (tr_on && tr_n < 4096)                                                             \
+      g_fp8_trace[t][tr_n++] = (static_cast<unsigned long long>(clock64()) << 8) | (tag); \
+  } while (0)
+#else
+#define FA_F8_TRACE(tag) \
+  do {                   \
+  } while (0)
+#endif
+
 namespace {
 
 constexpr float kE4m3Max = 448.f;
@@ -593,16 +609,23 @@ fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     };
     float nk0 = 1.f, nk1 = 1.f, nv0 = 0.f, nv1 = 0.f;
     if (nkb_t[t] > 0) scales_of(0, nk0, nk1, nv0, nv1);
+#ifdef FA_FP8_TRACE
+    const bool tr_on = blockIdx.x == 0 && lane == 0 && (warp & 3) == 0;
+    int tr_n = 0;
+#endif
     for (int j = 0; j < nkb_t[t]; ++j) {
+      FA_F8_TRACE(1);
       const float sk0 = nk0, sk1 = nk1, sv0 = nv0, sv1 = nv1;
       if (j + 1 < nkb_t[t]) scales_of(j + 1, nk0, nk1, nv0, nv1);
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_S + t), j & 1, a.err, kSS, abort_flag));
       if (!ok) break;
+      FA_F8_TRACE(2);
       tc_fence_after();
       uint32_t sr[4][32];
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, sr[c]);
       tmem_ld_wait();
+      FA_F8_TRACE(3);
       const int kbase = j * C::BN;
       const int kb0 = kbase / 64;
       // scaled score of column c: S_c * f(half) (exp2 units); a half past the
@@ -661,8 +684,11 @@ fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       f2_unpack(la, l0, l1);
       f2_unpack(lb, l2, l3);
       l_run = l_run * alpha + ((l0 + l1) + (l2 + l3));
+      FA_F8_TRACE(4);
       tmem_st32(s_addr, pk);
+      FA_F8_TRACE(5);
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        FA_F8_TRACE(9);
 #pragma unroll
         for (int c = 0; c < kD / 32; ++c) {
           uint32_t orr[32];
@@ -674,8 +700,10 @@ fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
       }
       tmem_st_wait();
+      FA_F8_TRACE(6);
       tc_fence_before();
       warp_arrive(bar(C::B_P + t));
+      FA_F8_TRACE(7);
     }
     if (ok && nkb_t[t] > 0) {
       ok = __all_sync(0xffffffffu,
@@ -778,3 +806,10 @@ cudaError_t launch_fwd_fp8(const CUtensorMap& tq, const CUtensorMap& tk, const C
 }
 
 }  // namespace fa
+
+#ifdef FA_FP8_TRACE
+// Copies the trace stamps of the last traced launch to host memory (2 x 4096 words).
+extern "C" __attribute__((visibility("default"))) int fa_fp8_trace_read(void* host) {
+  return static_cast<int>(cudaMemcpyFromSymbol(host, fa::g_fp8_trace, sizeof(fa::g_fp8_trace)));
+}
+#endif
