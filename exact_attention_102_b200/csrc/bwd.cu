@@ -1306,6 +1306,16 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       uint8_t* srow = smem + C::DQS_OFF + quarter * C::DQ_STAGE + lane * 128;
       const uint32_t stage_addr = base + C::DQS_OFF + quarter * C::DQ_STAGE;
       Walk wq = walk_start();
+      // FP8: s_q of this warp's 32 query rows, loaded one step ahead (the
+      // scale of the first column pair comes before the second pair's TMEM
+      // read and the arrival that lets dP(it+1) start)
+      auto sq_of_rows = [&](const Walk& w) {
+        const int q = w.step * C::BQ + quarter * 32;
+        return __ldg(a.sq + static_cast<size_t>(bh) * a.nsb + min(q / 64, a.nsb - 1));
+      };
+      float sq_next = 1.f;
+      if constexpr (FP8)
+        if (n_it > 0) sq_next = sq_of_rows(wq);
       for (int it = 0; it < n_it; ++it, walk_next(wq)) {
         const int qr = wq.step * C::BQ + quarter * 32;   // this warp's 32 query rows
         if (warp == 12 && lane == 0) FA_TRACE(2, 1);
@@ -1317,7 +1327,12 @@ bwd_ts_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         float m1 = sc, m2 = sc2;
         bool tw = two;
         if constexpr (FP8) {                         // scale 2^-tau / sq of these 32 queries
-          const float sq = __ldg(a.sq + static_cast<size_t>(bh) * a.nsb + min(qr / 64, a.nsb - 1));
+          const float sq = sq_next;
+          if (it + 1 < n_it) {
+            Walk wn = wq;
+            walk_next(wn);
+            sq_next = sq_of_rows(wn);
+          }
           m1 = a.scale / sq * f8_tau.f1;
           m2 = f8_tau.f2;
           tw = true;
