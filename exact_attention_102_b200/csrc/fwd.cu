@@ -35,6 +35,22 @@
 
 namespace fa {
 
+// Softmax trace (built only with -DFA_FWD_TRACE by exact_attention_102_b200.trace_fwd,
+// never in libfa.so): in CTA 0 of the forward, lane 0 of the first softmax warp
+// of each tile records clock64 stamps around the steps of every key block.
+#ifdef FA_FWD_TRACE
+__device__ unsigned long long g_fwd_trace[2][4096];
+#define FA_FWD_STAMP(tag)                                                                 \
+  do {                                                                                    \
+    if (tr_on && tr_n < 4096)                                                             \
+      g_fwd_trace[t][tr_n++] = (static_cast<unsigned long long>(clock64()) << 8) | (tag); \
+  } while (0)
+#else
+#define FA_FWD_STAMP(tag) \
+  do {                    \
+  } while (0)
+#endif
+
 namespace {
 
 template <int D>
@@ -413,14 +429,21 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     float l_run = 0.f;    // sum of fp32 P
     float lr_run = 0.f;   // sum of bf16-rounded P
     bool ok = true;
+#ifdef FA_FWD_TRACE
+    const bool tr_on = blockIdx.x == 0 && lane == 0 && (warp & 3) == 0;
+    int tr_n = 0;
+#endif
     for (int j = 0; j < nkb_t[t]; ++j) {
+      FA_FWD_STAMP(1);
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_S + t), j & 1, a.err, kSiteS, abort_flag));
       if (!ok) break;
+      FA_FWD_STAMP(2);
       tc_fence_after();
       uint32_t sr[4][32];
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, sr[c]);
       tmem_ld_wait();
+      FA_FWD_STAMP(3);
 #define SV(c) __uint_as_float(sr[(c) >> 5][(c)&31])
       if (sparse && !((uflag[j] >> t) & 1)) {   // a block this tile does not see: P = 0
         uint32_t zero[32];
@@ -507,10 +530,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       f2_unpack(rb, r2, r3);
       l_run = l_run * alpha + ((l0 + l1) + (l2 + l3));
       lr_run = lr_run * alpha + ((r0 + r1) + (r2 + r3));
+      FA_FWD_STAMP(4);
       tmem_st32(s_addr, pk0);
       tmem_st32(s_addr + 32, pk1);
+      FA_FWD_STAMP(5);
       // O rescale (PV of block j-1 has completed: S_t(j)'s commit covers it)
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        FA_FWD_STAMP(9);
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t orr[32];
@@ -523,8 +549,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         }
       }
       tmem_st_wait();
+      FA_FWD_STAMP(6);
       tc_fence_before();
       warp_arrive(bar(C::B_P + t));
+      FA_FWD_STAMP(7);
     }
     // ------------------------------------------------------------ epilogue
     // output row of query `row`: BHND [bh][row] or packed [token][head]
@@ -617,3 +645,10 @@ template cudaError_t launch_fwd<128>(const CUtensorMap&, const CUtensorMap&, con
                                      const FwdArgs&, cudaStream_t);
 
 }  // namespace fa
+
+#ifdef FA_FWD_TRACE
+// Copies the trace stamps of the last traced launch to host memory (2 x 4096 words).
+extern "C" __attribute__((visibility("default"))) int fa_fwd_trace_read(void* host) {
+  return static_cast<int>(cudaMemcpyFromSymbol(host, fa::g_fwd_trace, sizeof(fa::g_fwd_trace)));
+}
+#endif
