@@ -20,7 +20,9 @@
 //   warps 4..7    softmax for Q tile 0, warps 8..11 for Q tile 1: each
 //                 thread owns one row (one TMEM lane), so the row max and row
 //                 sum need no shuffles. While one tile's softmax runs, the
-//                 tensor core works on the other tile (ping-pong).
+//                 tensor core works on the other tile (ping-pong). P goes
+//                 out in two halves of 64 keys: P.V starts on the first while
+//                 the exps of the second run.
 // TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+D),
 // O_1 [256+D, 256+2D). P_t (bf16, packed 2 per column) overwrites the first
 // 64 columns of S_t and feeds the P.V MMA directly from TMEM.
@@ -71,7 +73,8 @@ struct FwdCfg {
   static constexpr int B_S = 1 + 2 * NSTAGE;
   static constexpr int B_P = B_S + 2;
   static constexpr int B_O = B_P + 2;
-  static constexpr int B_DRAIN = B_O + 2;
+  static constexpr int B_P0 = B_O + 2;          // first 64 keys of P_t in TMEM
+  static constexpr int B_DRAIN = B_P0 + 2;
   static constexpr int NBAR = B_DRAIN + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // tmem slot (4 B), abort flag (4 B)
   // block-sparse form: the CTA's key blocks (union of its two tiles' blocks),
@@ -257,6 +260,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       mbar_init(bar(C::B_S + t), 1);
       mbar_init(bar(C::B_P + t), 4);   // one arrival per softmax warp
       mbar_init(bar(C::B_O + t), 1);
+      mbar_init(bar(C::B_P0 + t), 4);
     }
     mbar_init(bar(C::B_DRAIN), 1);
     *abort_flag = 0;
@@ -386,13 +390,21 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         int sk = -1;                    // ring stage of K_{j+1}, once waited for
         for (int t = 0; t < 2 && ok; ++t) {
           if (j >= nkb_t[t]) continue;
+          // P.V(j) in two halves of 64 keys, each as soon as its half of P is in
+          ok = mbar_wait(bar(C::B_P0 + t), npv[t] & 1, a.err, kSiteP, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < C::BN / 32; ++kk)
+            umma_f16_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8, add(vm, kk * 2048), idPV,
+                        (npv[t] > 0 || kk > 0) ? 1u : 0u);
           ok = mbar_wait(bar(C::B_P + t), npv[t] & 1, a.err, kSiteP, abort_flag);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < C::BN / 16; ++kk)
+          for (int kk = C::BN / 32; kk < C::BN / 16; ++kk)
             umma_f16_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8, add(vm, kk * 2048), idPV,
-                        (npv[t] > 0 || kk > 0) ? 1u : 0u);
+                        1u);
           if (j + 1 == nkb_t[t]) umma_commit(bar(C::B_O + t));   // last P.V of tile t
           ++npv[t];
           if (j + 1 < nkb_t[t]) {
@@ -453,6 +465,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         tmem_st32(s_addr + 32, zero);
         tmem_st_wait();
         tc_fence_before();
+        warp_arrive(bar(C::B_P0 + t));
         warp_arrive(bar(C::B_P + t));
         continue;
       }
@@ -486,42 +499,69 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       // exp2 from the polynomial, the rest from the special-function unit
       const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_use, -m_use);
       uint64_t la = 0, lb = 0, ra = 0, rb = 0;     // (0.f, 0.f) pairs
-      uint32_t pk0[32], pk1[32];
       uint4 rnd = make_uint4(0u, 0u, 0u, 0u);     // dropout: random bytes of 16 keys
 #pragma unroll
-      for (int q = 0; q < 64; ++q) {
-        if (dropout && (q & 7) == 0)
-          rnd = philox4x32_10(static_cast<uint32_t>((kbase >> 4) + (q >> 3)),
-                              static_cast<uint32_t>(row), static_cast<uint32_t>(bh),
-                              a.drop_offset, a.seed_lo, a.seed_hi);
-        const uint64_t x2 = f2_fma(f2_pack(SV(2 * q), SV(2 * q + 1)), sl2x2, negm2);
-        uint64_t p2;
-        if (kPolyEvery > 0 && q % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
-          p2 = exp2_poly_x2(x2);
-        } else {
-          float x0, x1;
-          f2_unpack(x2, x0, x1);
-          p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+      for (int hq = 0; hq < 2; ++hq) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int qq = 0; qq < 32; ++qq) {
+          const int q = 32 * hq + qq;
+          if (dropout && (q & 7) == 0)
+            rnd = philox4x32_10(static_cast<uint32_t>((kbase >> 4) + (q >> 3)),
+                                static_cast<uint32_t>(row), static_cast<uint32_t>(bh),
+                                a.drop_offset, a.seed_lo, a.seed_hi);
+          const uint64_t x2 = f2_fma(f2_pack(SV(2 * q), SV(2 * q + 1)), sl2x2, negm2);
+          uint64_t p2;
+          if (kPolyEvery > 0 && q % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
+            p2 = exp2_poly_x2(x2);
+          } else {
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+          }
+          float p0, p1;
+          f2_unpack(p2, p0, p1);
+          const uint32_t u = pack_bf16x2(p0, p1);
+          const uint64_t rr = f2_pack(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+          if (q & 1) {
+            lb = f2_add(lb, p2);
+            rb = f2_add(rb, rr);
+          } else {
+            la = f2_add(la, p2);
+            ra = f2_add(ra, rr);
+          }
+          uint32_t us = u;                           // P, or P o Z under dropout
+          if (dropout) {
+            const int wi = (q & 7) >> 1;             // keys 2q, 2q+1: bytes 2(q&1), +1 of word wi
+            const uint32_t w = wi == 0 ? rnd.x : wi == 1 ? rnd.y : wi == 2 ? rnd.z : rnd.w;
+            us &= (q & 1) ? keep_halves<1>(w, a.drop_bias) : keep_halves<0>(w, a.drop_bias);
+          }
+          pk[qq] = us;
         }
-        float p0, p1;
-        f2_unpack(p2, p0, p1);
-        const uint32_t u = pack_bf16x2(p0, p1);
-        const uint64_t rr = f2_pack(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
-        if (q & 1) {
-          lb = f2_add(lb, p2);
-          rb = f2_add(rb, rr);
-        } else {
-          la = f2_add(la, p2);
-          ra = f2_add(ra, rr);
+        tmem_st32(s_addr + 32 * hq, pk);
+        if (hq == 0) {
+          // O rescale before P.V(j) starts on the first 64 keys (PV of block
+          // j-1 has completed: S_t(j)'s commit covers it)
+          if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+            FA_FWD_STAMP(9);
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t orr[32];
+              tmem_ld32(o_addr + c * 32, orr);
+              tmem_ld_wait();
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+              tmem_st32(o_addr + c * 32, orr);
+            }
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          warp_arrive(bar(C::B_P0 + t));                 // the first 64 keys: P.V may start
+          FA_FWD_STAMP(4);
         }
-        uint32_t us = u;                           // P, or P o Z under dropout
-        if (dropout) {
-          const int wi = (q & 7) >> 1;             // keys 2q, 2q+1: bytes 2(q&1), +1 of word wi
-          const uint32_t w = wi == 0 ? rnd.x : wi == 1 ? rnd.y : wi == 2 ? rnd.z : rnd.w;
-          us &= (q & 1) ? keep_halves<1>(w, a.drop_bias) : keep_halves<0>(w, a.drop_bias);
-        }
-        if (q < 32) pk0[q] = us; else pk1[q - 32] = us;
       }
+      FA_FWD_STAMP(5);
 #undef SV
       float l0, l1, l2, l3, r0, r1, r2, r3;
       f2_unpack(la, l0, l1);
@@ -530,24 +570,6 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       f2_unpack(rb, r2, r3);
       l_run = l_run * alpha + ((l0 + l1) + (l2 + l3));
       lr_run = lr_run * alpha + ((r0 + r1) + (r2 + r3));
-      FA_FWD_STAMP(4);
-      tmem_st32(s_addr, pk0);
-      tmem_st32(s_addr + 32, pk1);
-      FA_FWD_STAMP(5);
-      // O rescale (PV of block j-1 has completed: S_t(j)'s commit covers it)
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        FA_FWD_STAMP(9);
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t orr[32];
-          tmem_ld32(o_addr + c * 32, orr);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-          tmem_st32(o_addr + c * 32, orr);
-        }
-      }
       tmem_st_wait();
       FA_FWD_STAMP(6);
       tc_fence_before();

@@ -5,8 +5,9 @@ Builds a separate copy of the library with -DFA_FWD_TRACE into _build/trace_fwd/
 workload (B=1, H=16, N=16384, d=128, causal, seed 1002) and prints, per key
 block of CTA 0 (the heaviest pair of query tiles, 127 and 128 key blocks),
 how many SM cycles the first softmax warp of each of its two query tiles
-spends waiting for S, loading it out of TMEM, on the max / exp2 / bf16
-packing and the row sums, storing P, rescaling O and arriving; and how far
+spends waiting for S, loading it out of TMEM, on the max and the first 64
+keys' exp2 and P (with the O rescale, after which P.V may start on them), on
+the other 64 keys, on the row sums and the stores, and arriving; and how far
 apart the two tiles run.
 
 Usage: python -m exact_attention_102_b200.trace_fwd   (needs a B200)
@@ -103,9 +104,9 @@ def main():
         print(f"  whole block                            {_stat(block)}")
         print(f"  wait for S                             {_stat(span(1, 2))}")
         print(f"  load S out of TMEM                     {_stat(span(2, 3))}")
-        print(f"  max, exp2, bf16 packing, row sums      {_stat(span(3, 4))}")
-        print(f"  store P into TMEM                      {_stat(span(4, 5))}")
-        print(f"  rescale O (when needed), wait          {_stat(span(5, 6))}")
+        print(f"  max; keys 0-63: exp2, P, O rescale     {_stat(span(3, 4))}")
+        print(f"  keys 64-127: exp2, P into TMEM         {_stat(span(4, 5))}")
+        print(f"  row sums, wait for the TMEM stores      {_stat(span(5, 6))}")
         print(f"  arrive                                 {_stat(span(6, 7))}")
     n = min(len(firsts[0]), len(firsts[1]))
     off = [firsts[1][k] - firsts[0][k] for k in range(n)]
