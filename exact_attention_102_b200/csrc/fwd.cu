@@ -154,6 +154,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   constexpr bool paged = MODE == kPaged;
   constexpr bool sparse = MODE == kSparse;
   constexpr bool dropout = MODE == kDropout;
+  // P published in two halves (P.V starts on the first 64 keys while the
+  // exps of the rest run); the block-sparse form publishes it whole (its
+  // skipped blocks and union bookkeeping leave no registers for the split)
+  constexpr bool split_p = !sparse;
   int Lq = a.N, Lk = a.N, tq0 = 0, tk0 = 0, hq = 0, hk = 0;
   int seq = 0;                        // packed forms: the sequence of this CTA
   if (packed) {
@@ -391,20 +395,23 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         for (int t = 0; t < 2 && ok; ++t) {
           if (j >= nkb_t[t]) continue;
           // P.V(j) in two halves of 64 keys, each as soon as its half of P is in
-          ok = mbar_wait(bar(C::B_P0 + t), npv[t] & 1, a.err, kSiteP, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
+          // (the block-sparse form: all of P at once)
+          if constexpr (split_p) {
+            ok = mbar_wait(bar(C::B_P0 + t), npv[t] & 1, a.err, kSiteP, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < C::BN / 32; ++kk)
-            umma_f16_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8, add(vm, kk * 2048), idPV,
-                        (npv[t] > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < C::BN / 32; ++kk)
+              umma_f16_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8, add(vm, kk * 2048),
+                          idPV, (npv[t] > 0 || kk > 0) ? 1u : 0u);
+          }
           ok = mbar_wait(bar(C::B_P + t), npv[t] & 1, a.err, kSiteP, abort_flag);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
-          for (int kk = C::BN / 32; kk < C::BN / 16; ++kk)
+          for (int kk = split_p ? C::BN / 32 : 0; kk < C::BN / 16; ++kk)
             umma_f16_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8, add(vm, kk * 2048), idPV,
-                        1u);
+                        (npv[t] > 0 || kk > 0) ? 1u : 0u);
           if (j + 1 == nkb_t[t]) umma_commit(bar(C::B_O + t));   // last P.V of tile t
           ++npv[t];
           if (j + 1 < nkb_t[t]) {
@@ -465,7 +472,6 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         tmem_st32(s_addr + 32, zero);
         tmem_st_wait();
         tc_fence_before();
-        warp_arrive(bar(C::B_P0 + t));
         warp_arrive(bar(C::B_P + t));
         continue;
       }
@@ -539,7 +545,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           pk[qq] = us;
         }
         tmem_st32(s_addr + 32 * hq, pk);
-        if (hq == 0) {
+        if (split_p && hq == 0) {
           // O rescale before P.V(j) starts on the first 64 keys (PV of block
           // j-1 has completed: S_t(j)'s commit covers it)
           if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
@@ -562,6 +568,22 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         }
       }
       FA_FWD_STAMP(5);
+      if constexpr (!split_p) {
+        // O rescale (PV of block j-1 has completed: S_t(j)'s commit covers it)
+        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          FA_FWD_STAMP(9);
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t orr[32];
+            tmem_ld32(o_addr + c * 32, orr);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+            tmem_st32(o_addr + c * 32, orr);
+          }
+        }
+      }
 #undef SV
       float l0, l1, l2, l3, r0, r1, r2, r3;
       f2_unpack(la, l0, l1);
